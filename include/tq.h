@@ -1,0 +1,200 @@
+/*
+ * tq.h — C ABI of libtq, a B200 (sm_100a) implementation of the TurboQuant hot path:
+ * encode (random rotation, stored norm, Lloyd-Max codes, bit-packing, QJL sign sketch of the
+ * residual), scoring of full-precision queries against packed keys, decode attention over a
+ * compressed KV cache, and inner-product top-k search over a compressed database.
+ *
+ * Sources (web pages, by title and section):
+ *   [LP] "TurboQuant 学习路径：论文 → 技术 → 数学" (zzszmyf.github.io)
+ *   [JJ] "谷歌 TurboQuant 深度拆解：LLM 内存压缩 6 倍、推理加速 8 倍、零精度损失" (juejin.cn)
+ *   [VC] vocus.cc article on TurboQuant (PolarQuant stage, QJL 1-bit stage)
+ *   [ZC] "TurboQuant+ 深度解析" (zhichai.net)
+ * The pages print no API ([JJ] 第四部分 "没有官方代码"); the calls below follow the problem the
+ * pages state: compress key/value or database vectors with no per-block constants, then score a
+ * full-precision query against the compressed keys ([JJ] 第一部分, 第二部分).
+ *
+ * Conventions for every call:
+ *   - Plain C; no allocation on the data calls (encode, scores, attend, search); the caller owns
+ *     every data buffer (inputs, packed arrays, outputs, workspace) and passes raw pointers.
+ *   - "device" pointers are CUDA global-memory addresses on the context's device; "host"
+ *     pointers are ordinary CPU memory.  Device buffers must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  Data calls
+ *     only enqueue work and return; results are ready when the stream reaches that point.
+ *   - Arguments are validated on the host before any launch: a bad shape, pointer or alignment
+ *     returns TQ_EINVAL, an unsupported size TQ_EUNSUPPORTED, and nothing is launched.  A launch
+ *     failure returns TQ_ECUDA.  tq_last_error() then holds a one-line, thread-local message.
+ *   - Input values are not checked: NaN or Inf inputs give undefined outputs.
+ *   - Kernels never trap or assert; out-of-range slots or block-table entries are skipped.
+ *   - Outputs are undefined after an error.
+ *
+ * Supported sizes: d (vector length) a power of two in [8, 1024]; mse_bits in [1, 4];
+ * qjl_m = 0 (MSE stage only) or a multiple of 32 in [32, 1024]; attention group size
+ * n_q_heads / n_kv_heads in {1, 2, 4, 8}; search k in [1, 32].
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TQ_OK = 0,
+  TQ_EINVAL = 1,        /* bad argument: null pointer, bad shape, misaligned buffer, ws too small */
+  TQ_EUNSUPPORTED = 2,  /* well-formed but outside the supported sizes listed above */
+  TQ_ENOMEM = 3,        /* context creation could not allocate its constants */
+  TQ_ECUDA = 4,         /* a CUDA call or kernel launch failed */
+  TQ_ETIMEOUT = 5       /* reserved for bounded device waits (no call waits on the device today) */
+} tq_status;
+
+typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
+
+/* Quantizer shape for one tensor role (keys, values, or a search database).
+ *   d        vector length
+ *   mse_bits b: bits per coordinate of the Lloyd-Max stage (2^b levels)
+ *   qjl_m    m: rows of the Gaussian JL matrix S (1 sign bit each); 0 = no QJL stage
+ * "b bits per coordinate" for keys in the pages' sense = (b-1) MSE bits + 1 QJL bit with m = d
+ * ([JJ] 第二部分 "两步结合的效果": 2 + 1 = 3 bits). */
+typedef struct {
+  int32_t d;
+  int32_t mse_bits;
+  int32_t qjl_m;
+} tq_spec;
+
+/* Packed, caller-owned device arrays indexed by slot (one slot = one encoded vector).
+ *   codes  [capacity][code_bytes]  b bit-planes of d bits, plane t holding bit t of every code:
+ *                                  bit t of code_j is bit (t*d + j) of the vector's
+ *                                  little-endian bit stream; padded to a multiple of 16 bytes.
+ *   signs  [capacity][sign_bytes]  QJL bits, bit i = [ (S r)_i >= 0 ]; NULL when qjl_m == 0.
+ *   norm   [capacity]  fp32 ||x||
+ *   rnorm  [capacity]  fp32 ||r||, r the rotated-domain residual; NULL when qjl_m == 0.
+ * code_bytes = roundup(b*d/8, 16), sign_bytes = roundup(m/8, 16) (tq_ctx_layout). */
+typedef struct {
+  void *codes;
+  void *signs;
+  float *norm;
+  float *rnorm;
+  int64_t capacity;
+} tq_packed;
+
+typedef struct tq_ctx tq_ctx; /* opaque; owns read-only device constants, usable from any stream */
+
+/* Decode-attention descriptor.  Query head hq of sequence b reads KV head hq / (n_q_heads /
+ * n_kv_heads) over tokens [0, seq_lens[b]).  The slot of token t is
+ *   contiguous (block_table == NULL): (b * n_kv_heads + h) * ctx_stride + t
+ *   paged:      (block_table[b * max_blocks + t / block_size] * n_kv_heads + h) * block_size
+ *               + t % block_size
+ * in both the K and the V packed arrays. */
+typedef struct {
+  int32_t batch;
+  int32_t n_q_heads;
+  int32_t n_kv_heads;
+  float scale;                 /* softmax scale on the estimated scores; 0 = 1/sqrt(d) */
+  const int32_t *seq_lens;     /* device [batch]; values above max_seq_len are clamped to it */
+  const int32_t *block_table;  /* device [batch][max_blocks] or NULL (contiguous) */
+  int32_t max_blocks;          /* row stride of block_table */
+  int32_t block_size;          /* tokens per block (paged); ignored when contiguous */
+  int64_t ctx_stride;          /* slots per (batch, kv head) row (contiguous); ignored when paged */
+  int32_t max_seq_len;         /* host-known upper bound of seq_lens; sizes the split grid */
+  tq_packed k;                 /* keys, encoded with the K context */
+  tq_packed v;                 /* values, encoded with the V context (MSE stage only) */
+} tq_attn_desc;
+
+/* Lloyd-Max codebook for one coordinate of a randomly rotated unit vector in R^d.
+ * [JJ] 第六部分 "为什么随机旋转这么关键" gives the coordinate density
+ *   f_X(x) = Gamma(d/2)/(sqrt(pi) Gamma((d-1)/2)) (1-x^2)^((d-3)/2) on [-1, 1];
+ * [JJ] 第二部分 第一步 and [LP] 三.4 name the Lloyd-Max quantizer for it.  Host-only, fp64.
+ *   centroids     host out [2^bits], ascending
+ *   thresholds    host out [2^bits - 1], midpoints of neighbouring centroids
+ *   mse_per_coord host out, nullable: E[(X - Q(X))^2]
+ * Errors: TQ_EINVAL on null outputs; TQ_EUNSUPPORTED outside the supported d and bits. */
+tq_status tq_make_codebook(int32_t d, int32_t bits, double *centroids, double *thresholds,
+                           double *mse_per_coord);
+
+/* Create a quantizer context on `device`: builds the codebook and uploads the rotation signs D,
+ * the JL matrix S and the codebook (fp32) once.  D and S are drawn by the caller
+ * ([LP] 二.2: FJLT D = random signs; standard JL R_ij ~ N(0,1)); the same D and S must be used
+ * to encode and to score.
+ *   spec        host, read during the call
+ *   rot_signs   host int8 [d], entries +1 or -1
+ *   qjl_matrix  host fp32 [qjl_m][d] row-major; may be NULL when qjl_m == 0
+ *   out         host out: the new context
+ * Errors: TQ_EINVAL (nulls, a sign not +-1), TQ_EUNSUPPORTED (sizes), TQ_ENOMEM, TQ_ECUDA. */
+tq_status tq_ctx_create(const tq_spec *spec, const int8_t *rot_signs, const float *qjl_matrix,
+                        int32_t device, tq_ctx **out);
+
+/* Free a context (NULL is accepted).  The caller must ensure no queued work still uses it. */
+tq_status tq_ctx_destroy(tq_ctx *ctx);
+
+/* Bytes per slot of the packed code and sign arrays for this context (host out pointers). */
+tq_status tq_ctx_layout(const tq_ctx *ctx, int64_t *code_bytes, int64_t *sign_bytes);
+
+/* Encode n vectors into packed slots ([JJ] 第二部分 第一步 + 第二步; [VC] 第一/二階段):
+ *   nu = ||x||, u = x/nu (0 if nu = 0), y = (1/sqrt(d)) H (D u),
+ *   code_j = #{thresholds <= y_j}, r = y - c[code], gamma = ||r||, bit_i = [(S r)_i >= 0].
+ *   x      device [n][ld] of dtype (row i at x + i*ld elements), ld >= d
+ *   slots  device int64 [n] or NULL: row i goes to slot slots[i] (or i); rows whose slot is
+ *          outside [0, out.capacity) are skipped
+ *   out    packed arrays written at those slots
+ *   ws     device workspace of tq_encode_workspace_size() bytes (NULL allowed when that is 0)
+ * Errors: TQ_EINVAL (nulls, ld < d, n < 0, alignment, ws too small), TQ_ECUDA. */
+tq_status tq_encode_workspace_size(const tq_ctx *ctx, int64_t n, size_t *bytes);
+tq_status tq_encode_kv(const tq_ctx *ctx, const void *x, tq_dtype dtype, int64_t n, int64_t ld,
+                       const int64_t *slots, tq_packed out, void *ws, size_t ws_bytes,
+                       void *stream);
+
+/* Estimated inner products of nq full-precision queries with n packed keys (slots 0..n-1)
+ * ([JJ] 第二部分 第二步 and 第六部分 "无偏估计的数学保证"):
+ *   q' = (1/sqrt(d)) H (D q), p = S q',
+ *   out[i][k] = nu_k ( <q', c[code_k]> + sqrt(pi/2)/m * gamma_k * sum_j (2 bit_kj - 1) p_j ).
+ *   q    device [nq][d] of dtype
+ *   out  device fp32 [nq][n]
+ *   ws   device workspace of tq_scores_workspace_size() bytes
+ * Errors: TQ_EINVAL (nulls, n > keys.capacity, alignment, ws too small), TQ_ECUDA. */
+tq_status tq_scores_workspace_size(const tq_ctx *ctx, int32_t nq, size_t *bytes);
+tq_status tq_scores(const tq_ctx *ctx, const void *q, tq_dtype dtype, int32_t nq, tq_packed keys,
+                    int64_t n, float *out, void *ws, size_t ws_bytes, void *stream);
+
+/* One decode step of attention over the compressed cache ([JJ] 第一部分 "KV 缓存是什么",
+ * 第三部分 "推理速度"): logits = scale * estimated scores against the K cache, softmax over the
+ * sequence, output = sum_t w_t * nu_t * D_V (1/sqrt(d)) H c_V[code_t] (V's MSE stage).
+ *   kctx, vctx  contexts used to encode K and V (same d; vctx must have qjl_m == 0)
+ *   q           device [batch][n_q_heads][d] of dtype
+ *   out         device fp32 [batch][n_q_heads][d]; an empty sequence gives zeros
+ *   ws          device workspace of tq_attend_workspace_size() bytes
+ * Errors: TQ_EINVAL (nulls, shapes, alignment, ws too small), TQ_EUNSUPPORTED (group size,
+ * vctx with a QJL stage, d mismatch), TQ_ECUDA. */
+tq_status tq_attend_workspace_size(const tq_ctx *kctx, const tq_ctx *vctx,
+                                   const tq_attn_desc *desc, size_t *bytes);
+tq_status tq_attend_decode(const tq_ctx *kctx, const tq_ctx *vctx, const tq_attn_desc *desc,
+                           const void *q, tq_dtype dtype, float *out, void *ws, size_t ws_bytes,
+                           void *stream);
+
+/* Inner-product top-k over n packed database vectors (slots 0..n-1) ([JJ] 第三部分 "向量搜索"):
+ * order by (estimated score descending, index ascending).
+ *   q           device [nq][d] of dtype
+ *   out_scores  device fp32 [nq][k]
+ *   out_idx     device int64 [nq][k]
+ *   ws          device workspace of tq_search_workspace_size() bytes
+ * Errors: TQ_EINVAL (nulls, k > n, alignment, ws too small), TQ_EUNSUPPORTED (k > 32),
+ * TQ_ECUDA. */
+tq_status tq_search_workspace_size(const tq_ctx *ctx, int32_t nq, int64_t n, int32_t k,
+                                   size_t *bytes);
+tq_status tq_search_topk(const tq_ctx *ctx, const void *q, tq_dtype dtype, int32_t nq,
+                         tq_packed db, int64_t n, int32_t k, float *out_scores, int64_t *out_idx,
+                         void *ws, size_t ws_bytes, void *stream);
+
+/* Thread-local description of the last error on this thread ("" if none). */
+const char *tq_last_error(void);
+
+/* Library version string. */
+const char *tq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H */

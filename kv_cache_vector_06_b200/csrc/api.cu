@@ -1,0 +1,419 @@
+// C-ABI entry points of libtq: argument validation, context management and orchestration of the
+// kernels.  Every data call validates on the host first and only then enqueues work on the
+// caller's stream; nothing here allocates on a data call.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+
+#include "tq_internal.h"
+
+namespace {
+thread_local char g_err[512] = "";
+
+bool is_pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+tq_status check_spec(const tq_spec *s) {
+  if (!s) return tq_fail(TQ_EINVAL, "spec is NULL");
+  if (!is_pow2(s->d) || s->d < 8 || s->d > 1024)
+    return tq_fail(TQ_EUNSUPPORTED, "d=%d: must be a power of two in [8, 1024]", s->d);
+  if (s->mse_bits < 1 || s->mse_bits > 4)
+    return tq_fail(TQ_EUNSUPPORTED, "mse_bits=%d: must be in [1, 4]", s->mse_bits);
+  if (s->qjl_m < 0 || s->qjl_m > 1024 || (s->qjl_m % 32) != 0)
+    return tq_fail(TQ_EUNSUPPORTED, "qjl_m=%d: must be 0 or a multiple of 32 in [32, 1024]",
+                   s->qjl_m);
+  return TQ_OK;
+}
+
+tq_status check_ctx(const tq_ctx *c, const char *name) {
+  if (!c) return tq_fail(TQ_EINVAL, "%s is NULL", name);
+  return TQ_OK;
+}
+
+tq_status set_device(const tq_ctx *c) {
+  int cur = -1;
+  cudaError_t e = cudaGetDevice(&cur);
+  if (e != cudaSuccess) return tq_cuda_check(e, "cudaGetDevice");
+  if (cur != c->device) return tq_cuda_check(cudaSetDevice(c->device), "cudaSetDevice");
+  return TQ_OK;
+}
+
+tq_status check_packed(const tq_ctx *c, const tq_packed &p, int64_t need, const char *name,
+                       bool need_signs) {
+  if (!p.codes || !p.norm) return tq_fail(TQ_EINVAL, "%s: codes/norm is NULL", name);
+  if (!aligned16(p.codes)) return tq_fail(TQ_EINVAL, "%s: codes not 16-byte aligned", name);
+  if ((reinterpret_cast<uintptr_t>(p.norm) & 3u) != 0)
+    return tq_fail(TQ_EINVAL, "%s: norm not 4-byte aligned", name);
+  if (need_signs && c->spec.qjl_m > 0) {
+    if (!p.signs || !p.rnorm) return tq_fail(TQ_EINVAL, "%s: signs/rnorm is NULL", name);
+    if (!aligned16(p.signs)) return tq_fail(TQ_EINVAL, "%s: signs not 16-byte aligned", name);
+    if ((reinterpret_cast<uintptr_t>(p.rnorm) & 3u) != 0)
+      return tq_fail(TQ_EINVAL, "%s: rnorm not 4-byte aligned", name);
+  }
+  if (p.capacity < 0) return tq_fail(TQ_EINVAL, "%s: negative capacity", name);
+  if (need > p.capacity)
+    return tq_fail(TQ_EINVAL, "%s: %lld slots needed, capacity %lld", name, (long long)need,
+                   (long long)p.capacity);
+  return TQ_OK;
+}
+
+size_t query_prep_bytes(const tq_ctx *c, int64_t nq) {
+  return (size_t)tq_align_up(nq * c->spec.d * 4, 256) + (size_t)tq_align_up(nq * c->spec.qjl_m * 4, 256);
+}
+
+// q (any dtype) -> q' [nq][d] and p [nq][m] in the workspace
+tq_status prep_queries(const tq_ctx *c, const void *q, tq_dtype dt, int64_t nq, float *qr, float *p,
+                       cudaStream_t st) {
+  cudaError_t e = launch_rotate(c->k, ROT_QUERY, q, dt, nq, c->spec.d, nullptr, 0, nullptr,
+                                nullptr, nullptr, qr, st);
+  if (e != cudaSuccess) return tq_cuda_check(e, "query rotation launch");
+  if (c->spec.qjl_m > 0) {
+    e = launch_project(c->k, PROJ_DENSE, qr, nq, nullptr, 0, nullptr, p, st);
+    if (e != cudaSuccess) return tq_cuda_check(e, "query projection launch");
+  }
+  return TQ_OK;
+}
+
+constexpr int64_t kEncodeChunk = 1 << 16;  // rows per residual-workspace pass
+}  // namespace
+
+tq_status tq_fail(tq_status st, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+tq_status tq_cuda_check(cudaError_t e, const char *what) {
+  if (e == cudaSuccess) return TQ_OK;
+  return tq_fail(TQ_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+extern "C" {
+
+const char *tq_last_error(void) { return g_err; }
+const char *tq_version(void) { return "libtq 0.1 (sm_100a)"; }
+
+tq_status tq_make_codebook(int32_t d, int32_t bits, double *centroids, double *thresholds,
+                           double *mse_per_coord) {
+  g_err[0] = 0;
+  if (!centroids || !thresholds) return tq_fail(TQ_EINVAL, "centroids/thresholds is NULL");
+  tq_spec s{d, bits, 0};
+  tq_status st = check_spec(&s);
+  if (st != TQ_OK) return st;
+  return tq_codebook_fp64(d, bits, centroids, thresholds, mse_per_coord);
+}
+
+tq_status tq_ctx_create(const tq_spec *spec, const int8_t *rot_signs, const float *qjl_matrix,
+                        int32_t device, tq_ctx **out) {
+  g_err[0] = 0;
+  if (!out) return tq_fail(TQ_EINVAL, "out is NULL");
+  *out = nullptr;
+  tq_status st = check_spec(spec);
+  if (st != TQ_OK) return st;
+  if (!rot_signs) return tq_fail(TQ_EINVAL, "rot_signs is NULL");
+  if (spec->qjl_m > 0 && !qjl_matrix) return tq_fail(TQ_EINVAL, "qjl_matrix is NULL with qjl_m > 0");
+  const int d = spec->d, m = spec->qjl_m, L = 1 << spec->mse_bits;
+  for (int j = 0; j < d; ++j)
+    if (rot_signs[j] != 1 && rot_signs[j] != -1)
+      return tq_fail(TQ_EINVAL, "rot_signs[%d] = %d: must be +1 or -1", j, (int)rot_signs[j]);
+
+  tq_ctx *c = new (std::nothrow) tq_ctx();
+  if (!c) return tq_fail(TQ_ENOMEM, "host allocation failed");
+  c->device = device;
+  c->spec = *spec;
+  c->code_bytes = tq_align_up(((int64_t)spec->mse_bits * d + 7) / 8, 16);
+  c->sign_bytes = m > 0 ? tq_align_up((m + 7) / 8, 16) : 0;
+  tq_codebook_fp64(d, spec->mse_bits, c->centroids, c->thresholds, &c->mse_per_coord);
+
+  cudaError_t e = cudaSetDevice(device);
+  if (e != cudaSuccess) {
+    delete c;
+    return tq_cuda_check(e, "cudaSetDevice");
+  }
+  float hs[1024];
+  for (int j = 0; j < d; ++j) hs[j] = (float)rot_signs[j];
+  e = cudaMalloc(&c->dev_signs, sizeof(float) * d);
+  if (e == cudaSuccess && m > 0) e = cudaMalloc(&c->dev_S, sizeof(float) * (size_t)m * d);
+  if (e != cudaSuccess) {
+    cudaFree(c->dev_signs);
+    delete c;
+    cudaGetLastError();
+    return tq_fail(TQ_ENOMEM, "cudaMalloc of context constants failed");
+  }
+  e = cudaMemcpy(c->dev_signs, hs, sizeof(float) * d, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && m > 0)
+    e = cudaMemcpy(c->dev_S, qjl_matrix, sizeof(float) * (size_t)m * d, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    cudaFree(c->dev_signs);
+    cudaFree(c->dev_S);
+    delete c;
+    return tq_cuda_check(e, "upload of context constants");
+  }
+  TqConsts &k = c->k;
+  k.d = d;
+  k.bits = spec->mse_bits;
+  k.levels = L;
+  k.m = m;
+  k.code_words = (int)(c->code_bytes / 4);
+  k.sign_words = (int)(c->sign_bytes / 4);
+  k.inv_sqrt_d = (float)(1.0 / std::sqrt((double)d));
+  k.qjl_scale = m > 0 ? (float)(std::sqrt(M_PI / 2.0) / m) : 0.0f;
+  for (int i = 0; i < TQ_MAX_LEVELS; ++i) {
+    k.centroids[i] = i < L ? (float)c->centroids[i] : 0.0f;
+    k.thresholds[i] = i < L - 1 ? (float)c->thresholds[i] : INFINITY;
+  }
+  k.signs = c->dev_signs;
+  k.S = c->dev_S;
+  *out = c;
+  return TQ_OK;
+}
+
+tq_status tq_ctx_destroy(tq_ctx *ctx) {
+  if (!ctx) return TQ_OK;
+  int cur = -1;
+  cudaGetDevice(&cur);
+  cudaSetDevice(ctx->device);
+  cudaFree(ctx->dev_signs);
+  cudaFree(ctx->dev_S);
+  if (cur >= 0) cudaSetDevice(cur);
+  delete ctx;
+  return TQ_OK;
+}
+
+tq_status tq_ctx_layout(const tq_ctx *ctx, int64_t *code_bytes, int64_t *sign_bytes) {
+  g_err[0] = 0;
+  tq_status st = check_ctx(ctx, "ctx");
+  if (st != TQ_OK) return st;
+  if (code_bytes) *code_bytes = ctx->code_bytes;
+  if (sign_bytes) *sign_bytes = ctx->sign_bytes;
+  return TQ_OK;
+}
+
+tq_status tq_encode_workspace_size(const tq_ctx *ctx, int64_t n, size_t *bytes) {
+  g_err[0] = 0;
+  tq_status st = check_ctx(ctx, "ctx");
+  if (st != TQ_OK) return st;
+  if (!bytes) return tq_fail(TQ_EINVAL, "bytes is NULL");
+  if (n < 0) return tq_fail(TQ_EINVAL, "n < 0");
+  const int64_t rows = n < kEncodeChunk ? n : kEncodeChunk;
+  *bytes = ctx->spec.qjl_m > 0 ? (size_t)(rows * ctx->spec.d * 4) : 0;
+  return TQ_OK;
+}
+
+tq_status tq_encode_kv(const tq_ctx *ctx, const void *x, tq_dtype dtype, int64_t n, int64_t ld,
+                       const int64_t *slots, tq_packed out, void *ws, size_t ws_bytes,
+                       void *stream) {
+  g_err[0] = 0;
+  tq_status st = check_ctx(ctx, "ctx");
+  if (st != TQ_OK) return st;
+  if (n < 0) return tq_fail(TQ_EINVAL, "n < 0");
+  if (n == 0) return TQ_OK;
+  if (!x) return tq_fail(TQ_EINVAL, "x is NULL");
+  if (dtype != TQ_F32 && dtype != TQ_BF16) return tq_fail(TQ_EINVAL, "unknown dtype %d", (int)dtype);
+  if (ld < ctx->spec.d) return tq_fail(TQ_EINVAL, "ld=%lld < d=%d", (long long)ld, ctx->spec.d);
+  const int esz = dtype == TQ_F32 ? 4 : 2;
+  if (!aligned16(x) || (ld * esz) % 16 != 0)
+    return tq_fail(TQ_EINVAL, "x must be 16-byte aligned with a row stride that is a multiple of 16 bytes");
+  if (slots && (reinterpret_cast<uintptr_t>(slots) & 7u))
+    return tq_fail(TQ_EINVAL, "slots not 8-byte aligned");
+  st = check_packed(ctx, out, slots ? 0 : n, "out", true);
+  if (st != TQ_OK) return st;
+  size_t need = 0;
+  tq_encode_workspace_size(ctx, n, &need);
+  if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws)))
+    return tq_fail(TQ_EINVAL, "workspace: %zu bytes (16-byte aligned) needed, %zu given", need, ws_bytes);
+  st = set_device(ctx);
+  if (st != TQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool qjl = ctx->spec.qjl_m > 0;
+  for (int64_t r0 = 0; r0 < n; r0 += kEncodeChunk) {
+    const int64_t rows = (n - r0) < kEncodeChunk ? (n - r0) : kEncodeChunk;
+    const char *xr = static_cast<const char *>(x) + r0 * ld * esz;
+    const int64_t *sl = slots ? slots + r0 : nullptr;
+    // without a slot map, chunk rows land at slots r0 + i: shift the packed base pointers
+    tq_packed o = out;
+    if (!slots) {
+      o.codes = static_cast<char *>(out.codes) + r0 * ctx->code_bytes;
+      o.norm = out.norm + r0;
+      if (qjl) {
+        o.signs = static_cast<char *>(out.signs) + r0 * ctx->sign_bytes;
+        o.rnorm = out.rnorm + r0;
+      }
+      o.capacity = out.capacity - r0;
+    }
+    cudaError_t e = launch_rotate(ctx->k, ROT_ENCODE, xr, dtype, rows, ld, sl, o.capacity,
+                                  static_cast<uint32_t *>(o.codes), o.norm, qjl ? o.rnorm : nullptr,
+                                  qjl ? static_cast<float *>(ws) : nullptr, s);
+    if (e != cudaSuccess) return tq_cuda_check(e, "encode rotation launch");
+    if (qjl) {
+      e = launch_project(ctx->k, PROJ_SIGNS, static_cast<const float *>(ws), rows, sl, o.capacity,
+                         static_cast<uint32_t *>(o.signs), nullptr, s);
+      if (e != cudaSuccess) return tq_cuda_check(e, "QJL projection launch");
+    }
+  }
+  return TQ_OK;
+}
+
+tq_status tq_scores_workspace_size(const tq_ctx *ctx, int32_t nq, size_t *bytes) {
+  g_err[0] = 0;
+  tq_status st = check_ctx(ctx, "ctx");
+  if (st != TQ_OK) return st;
+  if (!bytes) return tq_fail(TQ_EINVAL, "bytes is NULL");
+  if (nq < 0) return tq_fail(TQ_EINVAL, "nq < 0");
+  *bytes = query_prep_bytes(ctx, nq);
+  return TQ_OK;
+}
+
+tq_status tq_scores(const tq_ctx *ctx, const void *q, tq_dtype dtype, int32_t nq, tq_packed keys,
+                    int64_t n, float *out, void *ws, size_t ws_bytes, void *stream) {
+  g_err[0] = 0;
+  tq_status st = check_ctx(ctx, "ctx");
+  if (st != TQ_OK) return st;
+  if (nq < 0 || n < 0) return tq_fail(TQ_EINVAL, "nq < 0 or n < 0");
+  if (nq == 0 || n == 0) return TQ_OK;
+  if (!q || !out) return tq_fail(TQ_EINVAL, "q/out is NULL");
+  if (dtype != TQ_F32 && dtype != TQ_BF16) return tq_fail(TQ_EINVAL, "unknown dtype %d", (int)dtype);
+  if (!aligned16(q) || !aligned16(out)) return tq_fail(TQ_EINVAL, "q/out not 16-byte aligned");
+  st = check_packed(ctx, keys, n, "keys", true);
+  if (st != TQ_OK) return st;
+  const size_t need = query_prep_bytes(ctx, nq);
+  if (!ws || ws_bytes < need || !aligned16(ws))
+    return tq_fail(TQ_EINVAL, "workspace: %zu bytes (16-byte aligned) needed, %zu given", need, ws_bytes);
+  st = set_device(ctx);
+  if (st != TQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float *qr = static_cast<float *>(ws);
+  float *p = reinterpret_cast<float *>(static_cast<char *>(ws) + tq_align_up((int64_t)nq * ctx->spec.d * 4, 256));
+  st = prep_queries(ctx, q, dtype, nq, qr, p, s);
+  if (st != TQ_OK) return st;
+  return tq_cuda_check(launch_scores(ctx->k, qr, p, nq, keys, n, out, s), "scores launch");
+}
+
+static tq_status check_attn(const tq_ctx *kctx, const tq_ctx *vctx, const tq_attn_desc *desc) {
+  tq_status st = check_ctx(kctx, "kctx");
+  if (st != TQ_OK) return st;
+  st = check_ctx(vctx, "vctx");
+  if (st != TQ_OK) return st;
+  if (!desc) return tq_fail(TQ_EINVAL, "desc is NULL");
+  if (kctx->spec.d != vctx->spec.d)
+    return tq_fail(TQ_EUNSUPPORTED, "K and V contexts differ in d (%d vs %d)", kctx->spec.d, vctx->spec.d);
+  if (vctx->spec.qjl_m != 0)
+    return tq_fail(TQ_EUNSUPPORTED, "the V context must be MSE-only (qjl_m == 0)");
+  if (desc->batch < 0 || desc->n_q_heads <= 0 || desc->n_kv_heads <= 0)
+    return tq_fail(TQ_EINVAL, "batch/n_q_heads/n_kv_heads");
+  if (desc->n_q_heads % desc->n_kv_heads != 0)
+    return tq_fail(TQ_EINVAL, "n_q_heads %% n_kv_heads != 0");
+  const int g = desc->n_q_heads / desc->n_kv_heads;
+  if (g != 1 && g != 2 && g != 4 && g != 8)
+    return tq_fail(TQ_EUNSUPPORTED, "group size %d: must be 1, 2, 4 or 8", g);
+  if (desc->max_seq_len < 0) return tq_fail(TQ_EINVAL, "max_seq_len < 0");
+  if (!desc->seq_lens && desc->batch > 0) return tq_fail(TQ_EINVAL, "seq_lens is NULL");
+  if (desc->block_table) {
+    if (desc->block_size <= 0 || desc->max_blocks <= 0)
+      return tq_fail(TQ_EINVAL, "paged: block_size and max_blocks must be > 0");
+    if ((int64_t)desc->max_blocks * desc->block_size < desc->max_seq_len)
+      return tq_fail(TQ_EINVAL, "paged: max_blocks * block_size < max_seq_len");
+  } else {
+    if (desc->ctx_stride < desc->max_seq_len)
+      return tq_fail(TQ_EINVAL, "contiguous: ctx_stride < max_seq_len");
+  }
+  st = check_packed(kctx, desc->k, 0, "desc->k", true);
+  if (st != TQ_OK) return st;
+  return check_packed(vctx, desc->v, 0, "desc->v", false);
+}
+
+tq_status tq_attend_workspace_size(const tq_ctx *kctx, const tq_ctx *vctx, const tq_attn_desc *desc,
+                                   size_t *bytes) {
+  g_err[0] = 0;
+  tq_status st = check_attn(kctx, vctx, desc);
+  if (st != TQ_OK) return st;
+  if (!bytes) return tq_fail(TQ_EINVAL, "bytes is NULL");
+  const AttnPlan plan = attn_plan(*desc);
+  const int64_t nq = (int64_t)desc->batch * desc->n_q_heads;
+  *bytes = query_prep_bytes(kctx, nq) + attn_partials_bytes(*desc, plan, kctx->spec.d);
+  return TQ_OK;
+}
+
+tq_status tq_attend_decode(const tq_ctx *kctx, const tq_ctx *vctx, const tq_attn_desc *desc,
+                           const void *q, tq_dtype dtype, float *out, void *ws, size_t ws_bytes,
+                           void *stream) {
+  g_err[0] = 0;
+  tq_status st = check_attn(kctx, vctx, desc);
+  if (st != TQ_OK) return st;
+  if (desc->batch == 0) return TQ_OK;
+  if (!q || !out) return tq_fail(TQ_EINVAL, "q/out is NULL");
+  if (dtype != TQ_F32 && dtype != TQ_BF16) return tq_fail(TQ_EINVAL, "unknown dtype %d", (int)dtype);
+  if (!aligned16(q) || !aligned16(out)) return tq_fail(TQ_EINVAL, "q/out not 16-byte aligned");
+  size_t need = 0;
+  tq_attend_workspace_size(kctx, vctx, desc, &need);
+  if (!ws || ws_bytes < need || !aligned16(ws))
+    return tq_fail(TQ_EINVAL, "workspace: %zu bytes (16-byte aligned) needed, %zu given", need, ws_bytes);
+  st = set_device(kctx);
+  if (st != TQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t nq = (int64_t)desc->batch * desc->n_q_heads;
+  float *qr = static_cast<float *>(ws);
+  float *p = reinterpret_cast<float *>(static_cast<char *>(ws) + tq_align_up(nq * kctx->spec.d * 4, 256));
+  float *part = reinterpret_cast<float *>(static_cast<char *>(ws) + query_prep_bytes(kctx, nq));
+  st = prep_queries(kctx, q, dtype, nq, qr, p, s);
+  if (st != TQ_OK) return st;
+  const AttnPlan plan = attn_plan(*desc);
+  return tq_cuda_check(launch_attend(kctx->k, vctx->k, *desc, plan, qr, p, part, out, s),
+                       "attention launch");
+}
+
+tq_status tq_search_workspace_size(const tq_ctx *ctx, int32_t nq, int64_t n, int32_t k, size_t *bytes) {
+  g_err[0] = 0;
+  tq_status st = check_ctx(ctx, "ctx");
+  if (st != TQ_OK) return st;
+  if (!bytes) return tq_fail(TQ_EINVAL, "bytes is NULL");
+  if (nq < 0 || n < 0 || k < 1) return tq_fail(TQ_EINVAL, "nq/n/k");
+  if (k > 32) return tq_fail(TQ_EUNSUPPORTED, "k=%d: at most 32", k);
+  const SearchPlan plan = search_plan(nq, n, k);
+  const int64_t cands = (int64_t)nq * plan.shards * k;
+  *bytes = query_prep_bytes(ctx, nq) + (size_t)tq_align_up(cands * 4, 256) + (size_t)tq_align_up(cands * 8, 256);
+  return TQ_OK;
+}
+
+tq_status tq_search_topk(const tq_ctx *ctx, const void *q, tq_dtype dtype, int32_t nq, tq_packed db,
+                         int64_t n, int32_t k, float *out_scores, int64_t *out_idx, void *ws,
+                         size_t ws_bytes, void *stream) {
+  g_err[0] = 0;
+  tq_status st = check_ctx(ctx, "ctx");
+  if (st != TQ_OK) return st;
+  if (nq < 0 || n < 0) return tq_fail(TQ_EINVAL, "nq < 0 or n < 0");
+  if (k < 1 || k > n) return tq_fail(TQ_EINVAL, "k=%d must be in [1, n=%lld]", k, (long long)n);
+  if (k > 32) return tq_fail(TQ_EUNSUPPORTED, "k=%d: at most 32", k);
+  if (nq == 0) return TQ_OK;
+  if (!q || !out_scores || !out_idx) return tq_fail(TQ_EINVAL, "q/out is NULL");
+  if (dtype != TQ_F32 && dtype != TQ_BF16) return tq_fail(TQ_EINVAL, "unknown dtype %d", (int)dtype);
+  if (!aligned16(q) || !aligned16(out_scores) || !aligned16(out_idx))
+    return tq_fail(TQ_EINVAL, "q/out not 16-byte aligned");
+  st = check_packed(ctx, db, n, "db", true);
+  if (st != TQ_OK) return st;
+  size_t need = 0;
+  tq_search_workspace_size(ctx, nq, n, k, &need);
+  if (!ws || ws_bytes < need || !aligned16(ws))
+    return tq_fail(TQ_EINVAL, "workspace: %zu bytes (16-byte aligned) needed, %zu given", need, ws_bytes);
+  st = set_device(ctx);
+  if (st != TQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const SearchPlan plan = search_plan(nq, n, k);
+  const int64_t cands = (int64_t)nq * plan.shards * k;
+  char *w = static_cast<char *>(ws);
+  float *qr = reinterpret_cast<float *>(w);
+  float *p = reinterpret_cast<float *>(w + tq_align_up((int64_t)nq * ctx->spec.d * 4, 256));
+  w += query_prep_bytes(ctx, nq);
+  float *cs = reinterpret_cast<float *>(w);
+  int64_t *ci = reinterpret_cast<int64_t *>(w + tq_align_up(cands * 4, 256));
+  st = prep_queries(ctx, q, dtype, nq, qr, p, s);
+  if (st != TQ_OK) return st;
+  return tq_cuda_check(launch_search(ctx->k, plan, qr, p, nq, db, n, k, cs, ci, out_scores, out_idx, s),
+                       "search launch");
+}
+
+}  // extern "C"

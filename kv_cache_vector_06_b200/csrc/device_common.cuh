@@ -1,0 +1,115 @@
+// Device helpers shared by the libtq kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "tq_internal.h"
+
+#define TQ_FULL_MASK 0xffffffffu
+
+// Bit (t*d + j) of a packed code row read as 32-bit little-endian words: bit t of code_j.
+__device__ __forceinline__ int code_bit(const uint32_t *row, int t, int j, int d) {
+  const int pos = t * d + j;
+  return (int)((row[pos >> 5] >> (pos & 31)) & 1u);
+}
+
+// 32 consecutive coordinates [32w, 32w+32) of bit-plane t as one word (d >= 32), or the whole
+// d-bit plane t in the low d bits (d < 32; then w must be 0).
+__device__ __forceinline__ uint32_t plane_word(const uint32_t *row, int t, int w, int d) {
+  if (d >= 32) return row[t * (d >> 5) + w];
+  const uint64_t v = (uint64_t)row[0] | ((uint64_t)row[1] << 32);
+  return (uint32_t)((v >> (t * d)) & ((1ull << d) - 1ull));
+}
+
+// Estimated inner products of NQ prepared queries with one packed key:
+//   nu * ( sum_j q'_j c[code_j] + qjl_scale * gamma * sum_i (2 bit_i - 1) p_i )
+// qs: [d][NQ] (shared), ps: [m][NQ] (shared), cent: [levels] (shared).
+template <int NQ>
+__device__ __forceinline__ void estimate_scores(const TqConsts &c, const uint32_t *code_row,
+                                                const uint32_t *sign_row, float nu, float gamma,
+                                                const float *qs, const float *ps,
+                                                const float *cent, float out[NQ]) {
+  float a[NQ], s2[NQ];
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) {
+    a[q] = 0.f;
+    s2[q] = 0.f;
+  }
+  const int d = c.d;
+  const int nw = d >= 32 ? (d >> 5) : 1;
+  const int nb = d >= 32 ? 32 : d;
+  for (int w = 0; w < nw; ++w) {
+    uint32_t pw[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+      if (t < c.bits) pw[t] = plane_word(code_row, t, w, d);
+    for (int jj = 0; jj < nb; ++jj) {
+      int code = 0;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) code |= (int)((pw[t] >> jj) & 1u) << t;
+      const float cv = cent[code];
+      const float *qj = qs + (size_t)(w * 32 + jj) * NQ;
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) a[q] = fmaf(qj[q], cv, a[q]);
+    }
+  }
+  if (c.m > 0) {
+    const int mw = c.m >> 5;
+    for (int w = 0; w < mw; ++w) {
+      const uint32_t sw = sign_row[w];
+#pragma unroll 8
+      for (int jj = 0; jj < 32; ++jj) {
+        const float sg = ((sw >> jj) & 1u) ? 1.f : -1.f;
+        const float *pj = ps + (size_t)(w * 32 + jj) * NQ;
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) s2[q] = fmaf(pj[q], sg, s2[q]);
+      }
+    }
+  }
+  const float cg = c.qjl_scale * gamma;
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) out[q] = nu * fmaf(cg, s2[q], a[q]);
+}
+
+// (score desc, index asc) ordering used by top-k.
+__device__ __forceinline__ bool tq_better(float s1, int64_t i1, float s2, int64_t i2) {
+  return s1 > s2 || (s1 == s2 && i1 < i2);
+}
+
+// Warp-cooperative sorted top-k list (k <= 32): lane i < k holds the i-th best (score, index).
+// Insert the candidates held one per lane (valid flags); keeps the list sorted.
+__device__ __forceinline__ void warp_topk_insert(float &bs, int64_t &bi, int k, float cs,
+                                                 int64_t ci, bool valid) {
+  const int lane = threadIdx.x & 31;
+  float ts = __shfl_sync(TQ_FULL_MASK, bs, k - 1);
+  int64_t ti = __shfl_sync(TQ_FULL_MASK, bi, k - 1);
+  unsigned mask = __ballot_sync(TQ_FULL_MASK, valid && tq_better(cs, ci, ts, ti));
+  while (mask) {
+    const int src = __ffs(mask) - 1;
+    mask &= mask - 1;
+    const float s = __shfl_sync(TQ_FULL_MASK, cs, src);
+    const int64_t i = __shfl_sync(TQ_FULL_MASK, ci, src);
+    if (!tq_better(s, i, ts, ti)) continue;  // uniform: every lane holds the same ts/ti
+    const bool mine_better = lane < k && tq_better(bs, bi, s, i);
+    const int pos = __popc(__ballot_sync(TQ_FULL_MASK, mine_better));
+    const float us = __shfl_up_sync(TQ_FULL_MASK, bs, 1);
+    const int64_t ui = __shfl_up_sync(TQ_FULL_MASK, bi, 1);
+    if (lane > pos && lane < k) {
+      bs = us;
+      bi = ui;
+    }
+    if (lane == pos) {
+      bs = s;
+      bi = i;
+    }
+    ts = __shfl_sync(TQ_FULL_MASK, bs, k - 1);
+    ti = __shfl_sync(TQ_FULL_MASK, bi, k - 1);
+  }
+}
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t h) {
+  return __uint_as_float(((uint32_t)h) << 16);
+}

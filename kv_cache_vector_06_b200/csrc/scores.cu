@@ -1,0 +1,54 @@
+// tq_scores: estimated inner products of prepared queries with every packed key.
+//   out[i][k] = nu_k ( <q'_i, c[code_k]> + sqrt(pi/2)/m gamma_k sum_j (2 bit_kj - 1) p_ij )
+// ("谷歌 TurboQuant 深度拆解" 第二部分 第二步 and 第六部分 "无偏估计的数学保证").
+// One thread per key and 8 queries per CTA; the prepared queries sit in shared memory as
+// [coordinate][query] so that all lanes read the same coordinate (broadcast) at once.
+#include "device_common.cuh"
+
+namespace {
+
+constexpr int kScThreads = 128;
+constexpr int kScQ = 8;
+
+__global__ void __launch_bounds__(kScThreads)
+scores_kernel(TqConsts c, const float *__restrict__ qr, const float *__restrict__ p, int nq,
+              tq_packed keys, int64_t n, float *__restrict__ out) {
+  extern __shared__ float sm[];
+  float *qs = sm;                       // [d][kScQ]
+  float *ps = qs + c.d * kScQ;          // [m][kScQ]
+  float *cent = ps + c.m * kScQ;        // [16]
+  const int q0 = blockIdx.y * kScQ;
+  for (int i = threadIdx.x; i < c.d * kScQ; i += blockDim.x) {
+    const int j = i / kScQ, q = i % kScQ;
+    qs[i] = (q0 + q < nq) ? qr[(int64_t)(q0 + q) * c.d + j] : 0.f;
+  }
+  for (int i = threadIdx.x; i < c.m * kScQ; i += blockDim.x) {
+    const int j = i / kScQ, q = i % kScQ;
+    ps[i] = (q0 + q < nq) ? p[(int64_t)(q0 + q) * c.m + j] : 0.f;
+  }
+  if (threadIdx.x < TQ_MAX_LEVELS) cent[threadIdx.x] = c.centroids[threadIdx.x];
+  __syncthreads();
+  const int64_t key = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (key >= n) return;
+  const uint32_t *crow = static_cast<const uint32_t *>(keys.codes) + key * c.code_words;
+  const uint32_t *srow = c.m > 0 ? static_cast<const uint32_t *>(keys.signs) + key * c.sign_words : nullptr;
+  const float gamma = c.m > 0 ? keys.rnorm[key] : 0.f;
+  float sc[kScQ];
+  estimate_scores<kScQ>(c, crow, srow, keys.norm[key], gamma, qs, ps, cent, sc);
+#pragma unroll
+  for (int q = 0; q < kScQ; ++q)
+    if (q0 + q < nq) out[(int64_t)(q0 + q) * n + key] = sc[q];
+}
+
+}  // namespace
+
+cudaError_t launch_scores(const TqConsts &c, const float *qr, const float *p, int nq,
+                          const tq_packed &keys, int64_t n, float *out, cudaStream_t st) {
+  if (n <= 0 || nq <= 0) return cudaSuccess;
+  const size_t smem = sizeof(float) * ((size_t)(c.d + c.m) * kScQ + TQ_MAX_LEVELS);
+  cudaError_t e = cudaFuncSetAttribute(scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)((n + kScThreads - 1) / kScThreads), (unsigned)((nq + kScQ - 1) / kScQ));
+  scores_kernel<<<grid, kScThreads, smem, st>>>(c, qr, p, nq, keys, n, out);
+  return cudaGetLastError();
+}

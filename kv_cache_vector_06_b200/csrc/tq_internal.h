@@ -1,0 +1,93 @@
+// Internal declarations shared by the libtq translation units (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "tq.h"
+
+#define TQ_MAX_LEVELS 16
+
+// Read-only constants of one quantizer, passed to kernels by value (kernel parameter space).
+struct TqConsts {
+  int d;          // vector length (power of two, 8..1024)
+  int bits;       // MSE bits per coordinate (1..4)
+  int levels;     // 2^bits
+  int m;          // QJL rows (0 or multiple of 32)
+  int code_words; // 32-bit words per packed code row
+  int sign_words; // 32-bit words per packed sign row
+  float inv_sqrt_d;
+  float qjl_scale;  // sqrt(pi/2)/m, 0 when m == 0
+  float centroids[TQ_MAX_LEVELS];
+  float thresholds[TQ_MAX_LEVELS];  // [levels-1] used
+  const float *signs;  // device [d], +-1.0f (rotation D)
+  const float *S;      // device [m][d] row-major (JL matrix)
+};
+
+struct tq_ctx {
+  int device;
+  tq_spec spec;
+  int64_t code_bytes;
+  int64_t sign_bytes;
+  double centroids[TQ_MAX_LEVELS];
+  double thresholds[TQ_MAX_LEVELS];
+  double mse_per_coord;
+  float *dev_signs;  // [d]
+  float *dev_S;      // [m][d]
+  TqConsts k;        // kernel view
+};
+
+// ---------------------------------------------------------------- host helpers (api.cu)
+tq_status tq_fail(tq_status st, const char *fmt, ...);
+tq_status tq_cuda_check(cudaError_t e, const char *what);
+
+// ---------------------------------------------------------------- codebook.cpp
+tq_status tq_codebook_fp64(int d, int bits, double *centroids, double *thresholds, double *mse);
+
+// ---------------------------------------------------------------- kernels (launchers)
+// Rotate rows of x: ENCODE mode normalises, quantizes, packs codes, writes norm (and, when the
+// context has a QJL stage, the residual rows to `resid` and rnorm).  QUERY mode writes
+// q' = (1/sqrt d) H D q (no normalisation) to `resid` as fp32 [n][d].
+enum RotateMode { ROT_ENCODE = 0, ROT_QUERY = 1 };
+cudaError_t launch_rotate(const TqConsts &c, RotateMode mode, const void *x, tq_dtype dtype,
+                          int64_t n, int64_t ld, const int64_t *slots, int64_t capacity,
+                          uint32_t *codes, float *norm, float *rnorm, float *resid,
+                          cudaStream_t st);
+
+// Z = R S^T for rows of R ([n][d] fp32).  SIGNS: pack bit = [z >= 0] into `signs` at the rows'
+// slots.  DENSE: write Z as fp32 [n][m] to `zout`.
+enum ProjEpilogue { PROJ_SIGNS = 0, PROJ_DENSE = 1 };
+cudaError_t launch_project(const TqConsts &c, ProjEpilogue ep, const float *R, int64_t n,
+                           const int64_t *slots, int64_t capacity, uint32_t *signs, float *zout,
+                           cudaStream_t st);
+
+// out[i][k] = estimated score of prepared query i against slot k.
+cudaError_t launch_scores(const TqConsts &c, const float *qr, const float *p, int nq,
+                          const tq_packed &keys, int64_t n, float *out, cudaStream_t st);
+
+// Attention over the compressed cache, split over the context, then combined.
+struct AttnPlan {
+  int group;        // n_q_heads / n_kv_heads
+  int chunk;        // tokens per split
+  int splits;       // splits per (batch, kv head)
+};
+AttnPlan attn_plan(const tq_attn_desc &desc);
+size_t attn_partials_bytes(const tq_attn_desc &desc, const AttnPlan &plan, int d);
+cudaError_t launch_attend(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc,
+                          const AttnPlan &plan, const float *qr, const float *p, float *partials,
+                          float *out, cudaStream_t st);
+
+// Search: per-(query tile, shard) top-k candidates, then a per-query merge.
+struct SearchPlan {
+  int qtile;   // queries per CTA
+  int shards;  // row shards
+};
+SearchPlan search_plan(int nq, int64_t n, int k);
+cudaError_t launch_search(const TqConsts &c, const SearchPlan &plan, const float *qr,
+                          const float *p, int nq, const tq_packed &db, int64_t n, int k,
+                          float *cand_s, int64_t *cand_i, float *out_s, int64_t *out_i,
+                          cudaStream_t st);
+
+static inline int64_t tq_align_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }

@@ -1,0 +1,235 @@
+"""GPU parity of every C-ABI data call against the fp64 oracle, at sizes the oracle finishes in
+seconds that still span several tiles / splits and a ragged tail.
+
+Stage isolation: scores, attention and search are checked against the oracle evaluated on the
+library's OWN packed bytes (decoded by the oracle's unpacker), so that an allowed near-threshold
+code flip in encode cannot mask or fake an error downstream; encode itself is checked against
+the oracle's encoding with the threshold band.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import attention as oattn
+from oracle import search as osearch
+from parity import (Quantizer, assert_attention_close, assert_scores_close, assert_topk_equivalent,
+                    compare_encode, oracle_cache, oracle_scores_from_packed, unpack)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def tq():
+    from kv_cache_vector_06_b200 import tq as _tq
+    return _tq
+
+
+def _enc(tq, q, x, slots=None, capacity=None):
+    cap = capacity if capacity is not None else x.shape[0]
+    packed = tq.Packed.allocate(q.ctx, cap)
+    tq.encode_kv(q.ctx, x.cuda(), packed, slots=None if slots is None else slots.cuda())
+    torch.cuda.synchronize()
+    return packed
+
+
+@pytest.mark.parametrize("d", [8, 16, 32, 64, 128, 256, 512, 1024])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_encode_all_dims_and_bits(tq, d, bits):
+    m = min(d, 128) if d >= 32 else 32
+    n = 1000 + 37
+    q = Quantizer(d, bits, m, seed=d * 10 + bits)
+    g = torch.Generator().manual_seed(d + bits)
+    x = torch.randn(n, d, generator=g) * torch.exp(torch.randn(d, generator=g))
+    packed = _enc(tq, q, x)
+    codes, sbits, norm, rnorm = unpack(q, packed)
+    compare_encode(q, q.oracle_encode(x.double().numpy()), codes, sbits, norm, rnorm)
+
+
+@pytest.mark.parametrize("m", [0, 32, 96])
+def test_encode_mse_only_and_odd_m(tq, m):
+    d, bits, n = 128, 3, 777
+    q = Quantizer(d, bits, m, seed=5)
+    x = torch.randn(n, d, generator=torch.Generator().manual_seed(1))
+    packed = _enc(tq, q, x)
+    codes, sbits, norm, rnorm = unpack(q, packed)
+    compare_encode(q, q.oracle_encode(x.double().numpy()), codes, sbits, norm, rnorm)
+
+
+def test_encode_bf16_strided_and_slots(tq):
+    d, bits, m, n = 128, 2, 128, 333
+    q = Quantizer(d, bits, m, seed=9)
+    base = synth.channel_scaled(1, 1, n, d + 64, seed=3)[0, 0]       # bf16 [n, d+64]
+    x = base[:, :d]                                                  # row stride d + 64
+    cap = 1000
+    slots = torch.randperm(cap, generator=torch.Generator().manual_seed(2))[:n].to(torch.int64)
+    packed = tq.Packed.allocate(q.ctx, cap)
+    tq.encode_kv(q.ctx, base.cuda()[:, :d], packed, slots=slots.cuda())
+    torch.cuda.synchronize()
+    codes, sbits, norm, rnorm = unpack(q, packed, rows=slots)
+    compare_encode(q, q.oracle_encode(x.double().numpy()), codes, sbits, norm, rnorm)
+    # untouched slots stay zero
+    mask = torch.ones(cap, dtype=torch.bool)
+    mask[slots] = False
+    assert packed.codes.cpu()[mask].abs().sum() == 0
+
+
+def test_encode_zero_vector_and_out_of_range_slots(tq):
+    d, bits, m = 64, 2, 64
+    q = Quantizer(d, bits, m, seed=1)
+    x = torch.randn(4, d)
+    x[1] = 0
+    slots = torch.tensor([0, 1, 5, -1], dtype=torch.int64)   # 5 and -1 are outside capacity 4
+    packed = tq.Packed.allocate(q.ctx, 4)
+    packed.norm.fill_(-7.0)
+    tq.encode_kv(q.ctx, x.cuda(), packed, slots=slots.cuda())
+    torch.cuda.synchronize()
+    nrm = packed.norm.cpu()
+    assert nrm[1].item() == 0.0 and nrm[2].item() == -7.0 and nrm[3].item() == -7.0
+    codes, sbits, norm, rnorm = unpack(q, packed, rows=[0, 1])
+    compare_encode(q, q.oracle_encode(x[:2].double().numpy()), codes, sbits, norm, rnorm)
+
+
+def test_tiny_config_scores(tq):
+    """Tiny: one head, d=128, 4096 fp32 keys with outlier channels, 8 queries, 2 MSE bits +
+    QJL m=128; exact and estimated logits."""
+    keys, queries = synth.tiny(seed=0)
+    q = Quantizer(128, 2, 128, seed=0)
+    packed = _enc(tq, q, keys)
+    codes, sbits, norm, rnorm = unpack(q, packed)
+    stats = compare_encode(q, q.oracle_encode(keys.double().numpy()), codes, sbits, norm, rnorm)
+    got = tq.scores(q.ctx, queries.cuda(), packed).cpu().numpy()
+    ref = oracle_scores_from_packed(q, queries.double().numpy(), codes, sbits, norm, rnorm)
+    assert_scores_close(got, ref)
+    # the estimate tracks the exact logits <q, k>
+    exact = queries.double().numpy() @ keys.double().numpy().T
+    rel = np.linalg.norm(got - exact) / np.linalg.norm(exact)
+    assert rel < 0.2, rel
+    assert stats["code_flips"] <= 0.0001 * codes.size
+
+
+def test_scores_bf16_queries_and_small_d(tq):
+    for d, bits, m in [(8, 1, 32), (16, 4, 64), (256, 3, 256)]:
+        q = Quantizer(d, bits, m, seed=d)
+        x = torch.randn(501, d, generator=torch.Generator().manual_seed(d))
+        qq = torch.randn(13, d, generator=torch.Generator().manual_seed(d + 1)).to(torch.bfloat16)
+        packed = _enc(tq, q, x)
+        codes, sbits, norm, rnorm = unpack(q, packed)
+        got = tq.scores(q.ctx, qq.cuda(), packed).cpu().numpy()
+        ref = oracle_scores_from_packed(q, qq.double().numpy(), codes, sbits, norm, rnorm)
+        assert_scores_close(got, ref)
+
+
+def _attention_case(tq, d, kbits, km, vbits, batch, hkv, group, lens, paged, qdtype, seed):
+    kq = Quantizer(d, kbits, km, seed=seed)
+    vq = Quantizer(d, vbits, 0, seed=seed + 50)
+    hq = hkv * group
+    maxlen = int(max(lens))
+    blk = synth.BLOCK_TOKENS
+    lens_t = torch.tensor(lens, dtype=torch.int32)
+    if paged:
+        table, nblocks = synth.shuffled_block_table(lens_t, seed=seed + 7)
+        cap = nblocks * hkv * blk
+    else:
+        table = None
+        cap = batch * hkv * maxlen
+    K = synth.channel_scaled(batch, hkv, maxlen, d, seed=seed + 1)
+    V = synth.channel_scaled(batch, hkv, maxlen, d, seed=seed + 2)
+    # slots of every (b, h, t < len)
+    rows, slots = [], []
+    for b in range(batch):
+        for h in range(hkv):
+            sl = oattn.token_slots(b, h, lens[b], hkv, ctx_stride=maxlen,
+                                   block_table=None if table is None else table.numpy())
+            rows.append((b, h, lens[b]))
+            slots.append(sl)
+    kx = torch.cat([K[b, h, :L] for b, h, L in rows])
+    vx = torch.cat([V[b, h, :L] for b, h, L in rows])
+    sl = torch.as_tensor(np.concatenate(slots), dtype=torch.int64)
+    kp = tq.Packed.allocate(kq.ctx, cap)
+    vp = tq.Packed.allocate(vq.ctx, cap)
+    tq.encode_kv(kq.ctx, kx.cuda(), kp, slots=sl.cuda())
+    tq.encode_kv(vq.ctx, vx.cuda(), vp, slots=sl.cuda())
+    qx = synth.decode_queries(batch, hq, d, seed=seed + 3, dtype=qdtype)
+    out = tq.attend_decode(kq.ctx, vq.ctx, qx.cuda(), kp, vp, lens_t.cuda(), maxlen, n_kv_heads=hkv,
+                           ctx_stride=maxlen, block_table=None if table is None else table.cuda(),
+                           block_size=blk)
+    torch.cuda.synchronize()
+    kc = oracle_cache(kq, *unpack(kq, kp))
+    vc = oracle_cache(vq, *unpack(vq, vp))
+    ref = oattn.attend_decode(qx.double().numpy(), kc, vc, lens, hkv, kq.D64, kq.S64, kq.c, vq.D64, vq.c,
+                              ctx_stride=maxlen, block_table=None if table is None else table.numpy())
+    assert_attention_close(out.cpu().numpy(), ref)
+    # encode parity on these rows too
+    compare_encode(kq, kq.oracle_encode(kx.double().numpy()), *unpack(kq, kp, rows=sl))
+    return out
+
+
+@pytest.mark.parametrize("kbits,vbits", [(2, 3), (3, 2)])
+def test_attention_contiguous_gqa4(tq, kbits, vbits):
+    _attention_case(tq, 128, kbits, 128, vbits, batch=2, hkv=2, group=4, lens=[1500, 333], paged=False,
+                    qdtype=torch.bfloat16, seed=11 + kbits)
+
+
+def test_attention_paged_ragged(tq):
+    _attention_case(tq, 128, 2, 128, 3, batch=3, hkv=2, group=4, lens=[700, 16, 1031], paged=True,
+                    qdtype=torch.bfloat16, seed=21)
+
+
+@pytest.mark.parametrize("group", [1, 2, 8])
+def test_attention_group_sizes_and_dims(tq, group):
+    _attention_case(tq, 64, 2, 64, 2, batch=1, hkv=2, group=group, lens=[300], paged=False,
+                    qdtype=torch.float32, seed=31 + group)
+
+
+def test_attention_d256_and_multi_split(tq):
+    _attention_case(tq, 256, 3, 256, 3, batch=1, hkv=1, group=4, lens=[5000], paged=False,
+                    qdtype=torch.float32, seed=41)
+
+
+def test_attention_empty_and_single_token(tq):
+    out = _attention_case(tq, 128, 2, 128, 3, batch=3, hkv=1, group=4, lens=[0, 1, 17], paged=True,
+                          qdtype=torch.float32, seed=51)
+    assert torch.all(out[0] == 0)
+
+
+@pytest.mark.parametrize("d,bits,m", [(128, 2, 128), (256, 1, 256), (1024, 3, 1024)])
+def test_search_topk_small(tq, d, bits, m):
+    n, nq, k = 5003, 17, 10
+    q = Quantizer(d, bits, m, seed=61 + bits)
+    X = synth.unit_rows(n, d, seed=0)
+    Q = synth.unit_rows(nq, d, seed=1)
+    packed = _enc(tq, q, X)
+    codes, sbits, norm, rnorm = unpack(q, packed)
+    s, i = tq.search_topk(q.ctx, Q.cuda(), packed, k)
+    torch.cuda.synchronize()
+    ref_full = oracle_scores_from_packed(q, Q.double().numpy(), codes, sbits, norm, rnorm)
+    ref_s, ref_i = osearch.topk(ref_full, k)
+    assert_topk_equivalent(s.cpu().numpy(), i.cpu().numpy(), lambda r, idx: ref_full[r, idx], ref_s)
+
+
+def test_search_k_edge_cases(tq):
+    d, bits, m = 64, 2, 64
+    q = Quantizer(d, bits, m, seed=3)
+    X = synth.unit_rows(40, d, seed=4)
+    Q = synth.unit_rows(3, d, seed=5)
+    packed = _enc(tq, q, X)
+    codes, sbits, norm, rnorm = unpack(q, packed)
+    ref_full = oracle_scores_from_packed(q, Q.double().numpy(), codes, sbits, norm, rnorm)
+    for k in (1, 32):
+        s, i = tq.search_topk(q.ctx, Q.cuda(), packed, k)
+        ref_s, _ = osearch.topk(ref_full, k)
+        assert_topk_equivalent(s.cpu().numpy(), i.cpu().numpy(), lambda r, idx: ref_full[r, idx], ref_s)
+    # duplicate rows: equal scores must come back in index order
+    Xd = torch.cat([X[:5], X[:5]])
+    pd = _enc(tq, q, Xd)
+    s, i = tq.search_topk(q.ctx, Q.cuda(), pd, 10)
+    ii, ss = i.cpu().numpy(), s.cpu().numpy()
+    for r in range(3):
+        assert sorted(ii[r].tolist()) == list(range(10))
+        for a in range(9):
+            assert ss[r, a] >= ss[r, a + 1]
+            if ss[r, a] == ss[r, a + 1]:
+                assert ii[r, a] < ii[r, a + 1]
