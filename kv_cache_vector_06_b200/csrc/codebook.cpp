@@ -66,6 +66,13 @@ tq_status tq_codebook_fp64(int d, int bits, double *centroids, double *threshold
     c.swap(cn);
     if (move < 1e-13) break;
   }
+  // the density is even, so the exact codebook is antisymmetric: impose c_i = -c_(L-1-i), which
+  // makes the middle threshold exactly 0
+  for (int i = 0; i < L / 2; ++i) {
+    const double a = 0.5 * (c[L - 1 - i] - c[i]);
+    c[i] = -a;
+    c[L - 1 - i] = a;
+  }
   for (int i = 0; i < L; ++i) centroids[i] = c[i];
   for (int i = 1; i < L; ++i) thresholds[i - 1] = 0.5 * (c[i - 1] + c[i]);
   if (mse) {

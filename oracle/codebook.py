@@ -97,6 +97,9 @@ def lloyd_max(d: int, bits: int, tol: float = 1e-13, max_iter: int = 1_000_000):
         c = c_new
         if move < tol:
             break
+    # f_X is even, so the Lloyd-Max fixed point is antisymmetric (c_i = -c_{L-1-i}); impose it
+    # exactly so that the middle threshold is exactly 0 (ties at y = 0 go to the upper cell).
+    c = 0.5 * (c - c[::-1])
     t = 0.5 * (c[:-1] + c[1:])
     return c, t, it
 

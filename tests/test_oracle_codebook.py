@@ -65,7 +65,8 @@ def test_lloyd_max_fixed_point_conditions(d, bits):
 @pytest.mark.parametrize("bits", BITS)
 def test_codebook_is_symmetric(d, bits):
     c, t = codebook.codebook(d, bits)
-    np.testing.assert_allclose(c, -c[::-1], atol=1e-14)
+    np.testing.assert_array_equal(c, -c[::-1])
+    assert t[len(t) // 2] == 0.0
 
 
 @pytest.mark.parametrize("d", DIMS)
