@@ -187,6 +187,18 @@ tq_status tq_search_topk(const tq_ctx *ctx, const void *q, tq_dtype dtype, int32
                          tq_packed db, int64_t n, int32_t k, float *out_scores, int64_t *out_idx,
                          void *ws, size_t ws_bytes, void *stream);
 
+/* Instrumentation, off by default.  While enabled, every kernel that a data call launches is
+ * bracketed by two CUDA events recorded on the caller's stream (so the pair times exactly that
+ * kernel on the stream it runs on).  tq_profile_read waits for the recorded events and reports,
+ * for kernel kind `index` (0, 1, ... until it returns TQ_EINVAL), its name, the number of
+ * launches and their summed device time in milliseconds since the last reset.  Do not enable
+ * while capturing a CUDA graph.
+ *   name  host out buffer of name_len bytes (nullable); launches, total_ms host outs (nullable) */
+tq_status tq_profile_enable(int32_t on);
+tq_status tq_profile_reset(void);
+tq_status tq_profile_read(int32_t index, char *name, int32_t name_len, int64_t *launches,
+                          double *total_ms);
+
 /* Thread-local description of the last error on this thread ("" if none). */
 const char *tq_last_error(void);
 

@@ -226,7 +226,9 @@ cudaError_t launch_split(const TqConsts &kc, const TqConsts &vc, const AttnArgs 
   cudaError_t e = cudaFuncSetAttribute(attend_split_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
+  tq_prof_begin(TQK_ATTEND_SPLIT, st);
   attend_split_kernel<G><<<grid, kAtThreads, smem, st>>>(kc, vc, a, qr, p, part);
+  tq_prof_end(TQK_ATTEND_SPLIT, st);
   return cudaGetLastError();
 }
 
@@ -283,7 +285,9 @@ cudaError_t launch_attend(const TqConsts &kc, const TqConsts &vc, const tq_attn_
   cudaError_t e2 = cudaFuncSetAttribute(attend_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)smem);
   if (e2 != cudaSuccess) return e2;
+  tq_prof_begin(TQK_ATTEND_COMBINE, st);
   attend_combine_kernel<<<(unsigned)((int64_t)desc.batch * desc.n_q_heads), kAtThreads, smem, st>>>(
       vc, plan.splits, partials, out);
+  tq_prof_end(TQK_ATTEND_COMBINE, st);
   return cudaGetLastError();
 }

@@ -112,9 +112,12 @@ cudaError_t launch_project(const TqConsts &c, ProjEpilogue ep, const float *R, i
                            cudaStream_t st) {
   if (n <= 0 || c.m <= 0) return cudaSuccess;
   dim3 grid((unsigned)((n + kPT - 1) / kPT), (unsigned)((c.m + kPT - 1) / kPT));
+  const int kind = ep == PROJ_SIGNS ? TQK_QJL_PROJECT : TQK_QUERY_PROJECT;
+  tq_prof_begin(kind, st);
   if (ep == PROJ_SIGNS)
     project_kernel<PROJ_SIGNS><<<grid, 256, 0, st>>>(c, R, n, slots, capacity, signs, zout);
   else
     project_kernel<PROJ_DENSE><<<grid, 256, 0, st>>>(c, R, n, slots, capacity, signs, zout);
+  tq_prof_end(kind, st);
   return cudaGetLastError();
 }

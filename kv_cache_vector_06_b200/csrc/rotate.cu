@@ -192,8 +192,11 @@ cudaError_t launch_rotate_d(const TqConsts &c, RotateMode mode, const void *x, t
                             cudaStream_t st) {
   constexpr int VPB = (kRotThreads / 32) * RotLayout<D>::VPW;  // vectors per block
   const int64_t blocks = (n + VPB - 1) / VPB;
+  const int kind = mode == ROT_ENCODE ? TQK_ROTATE_ENCODE : TQK_ROTATE_QUERY;
+  tq_prof_begin(kind, st);
   rotate_kernel<D><<<(unsigned)blocks, kRotThreads, 0, st>>>(c, (int)mode, x, (int)dtype, n, ld, slots,
                                                              capacity, codes, norm, rnorm, resid);
+  tq_prof_end(kind, st);
   return cudaGetLastError();
 }
 

@@ -49,6 +49,8 @@ cudaError_t launch_scores(const TqConsts &c, const float *qr, const float *p, in
   cudaError_t e = cudaFuncSetAttribute(scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((n + kScThreads - 1) / kScThreads), (unsigned)((nq + kScQ - 1) / kScQ));
+  tq_prof_begin(TQK_SCORES, st);
   scores_kernel<<<grid, kScThreads, smem, st>>>(c, qr, p, nq, keys, n, out);
+  tq_prof_end(TQK_SCORES, st);
   return cudaGetLastError();
 }

@@ -122,12 +122,16 @@ cudaError_t launch_search(const TqConsts &c, const SearchPlan &plan, const float
   cudaError_t e = cudaFuncSetAttribute(search_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)plan.shards, (unsigned)((nq + kSrQ - 1) / kSrQ));
+  tq_prof_begin(TQK_SEARCH_SCAN, st);
   search_scan_kernel<<<grid, kSrThreads, smem, st>>>(c, qr, p, nq, db, n, k, rows_per_shard, plan.shards,
                                                      cand_s, cand_i);
+  tq_prof_end(TQK_SEARCH_SCAN, st);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int wpb = 4;
+  tq_prof_begin(TQK_SEARCH_MERGE, st);
   search_merge_kernel<<<(unsigned)((nq + wpb - 1) / wpb), 32 * wpb, 0, st>>>(nq, plan.shards, k, cand_s,
                                                                              cand_i, out_s, out_i);
+  tq_prof_end(TQK_SEARCH_MERGE, st);
   return cudaGetLastError();
 }

@@ -43,6 +43,14 @@ struct tq_ctx {
 tq_status tq_fail(tq_status st, const char *fmt, ...);
 tq_status tq_cuda_check(cudaError_t e, const char *what);
 
+// ---------------------------------------------------------------- profile.cu
+enum TqKernelKind {
+  TQK_ROTATE_ENCODE = 0, TQK_QJL_PROJECT, TQK_ROTATE_QUERY, TQK_QUERY_PROJECT, TQK_SCORES,
+  TQK_ATTEND_SPLIT, TQK_ATTEND_COMBINE, TQK_SEARCH_SCAN, TQK_SEARCH_MERGE, TQK_COUNT
+};
+void tq_prof_begin(int kind, cudaStream_t st);
+void tq_prof_end(int kind, cudaStream_t st);
+
 // ---------------------------------------------------------------- codebook.cpp
 tq_status tq_codebook_fp64(int d, int bits, double *centroids, double *thresholds, double *mse);
 

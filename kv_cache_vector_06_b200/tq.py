@@ -64,6 +64,9 @@ def _load():
         "tq_search_workspace_size": (st, [c_void_p, c_int32, c_int64, c_int32, POINTER(c_size_t)]),
         "tq_search_topk": (st, [c_void_p, c_void_p, c_int, c_int32, PackedC, c_int64, c_int32, c_void_p,
                                 c_void_p, c_void_p, c_size_t, c_void_p]),
+        "tq_profile_enable": (st, [c_int32]),
+        "tq_profile_reset": (st, []),
+        "tq_profile_read": (st, [c_int32, ctypes.c_char_p, c_int32, POINTER(c_int64), POINTER(c_double)]),
         "tq_last_error": (c_char_p, []),
         "tq_version": (c_char_p, []),
     }
@@ -329,3 +332,25 @@ def search_topk(ctx: Context, q: torch.Tensor, db: Packed, k: int, n: int = None
                               _dev(out_scores, ctx.device, "out_scores", torch.float32),
                               _dev(out_idx, ctx.device, "out_idx", torch.int64), w, wb, _stream_ptr(stream)))
     return out_scores, out_idx
+
+
+def profile_enable(on: bool = True):
+    _check(LIB.tq_profile_enable(1 if on else 0))
+
+
+def profile_reset():
+    _check(LIB.tq_profile_reset())
+
+
+def profile_read() -> dict:
+    """{kernel name: (launches, total device ms)} since the last reset."""
+    out = {}
+    i = 0
+    buf = ctypes.create_string_buffer(64)
+    while True:
+        n, ms = c_int64(), c_double()
+        if LIB.tq_profile_read(i, buf, 64, ctypes.byref(n), ctypes.byref(ms)) != 0:
+            break
+        out[buf.value.decode()] = (n.value, ms.value)
+        i += 1
+    return out
