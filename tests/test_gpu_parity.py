@@ -103,10 +103,14 @@ def test_tiny_config_scores(tq):
     got = tq.scores(q.ctx, queries.cuda(), packed).cpu().numpy()
     ref = oracle_scores_from_packed(q, queries.double().numpy(), codes, sbits, norm, rnorm)
     assert_scores_close(got, ref)
-    # the estimate tracks the exact logits <q, k>
+    # end to end the library estimate is as close to the exact logits <q, k> as the oracle's own
+    # encode + estimate (the estimator's noise, not the implementation, sets that distance)
     exact = queries.double().numpy() @ keys.double().numpy().T
-    rel = np.linalg.norm(got - exact) / np.linalg.norm(exact)
-    assert rel < 0.2, rel
+    enc = q.oracle_encode(keys.double().numpy())
+    own = oracle_scores_from_packed(q, queries.double().numpy(), enc.codes, enc.bits, enc.norm, enc.rnorm)
+    rel_gpu = np.linalg.norm(got - exact) / np.linalg.norm(exact)
+    rel_oracle = np.linalg.norm(own - exact) / np.linalg.norm(exact)
+    assert abs(rel_gpu - rel_oracle) < 0.02 * rel_oracle, (rel_gpu, rel_oracle)
     assert stats["code_flips"] <= 0.0001 * codes.size
 
 
