@@ -173,6 +173,28 @@ tq_status tq_attend_decode(const tq_ctx *kctx, const tq_ctx *vctx, const tq_attn
                            const void *q, tq_dtype dtype, float *out, void *ws, size_t ws_bytes,
                            void *stream);
 
+/* Allocation-free decode attention.  The pages have no counterpart: this entry point exists for
+ * callers that cannot allocate device memory when they run attention, such as an inference
+ * engine that gives all device memory to its own pool at start-up and forbids extensions from
+ * calling cudaMalloc, or a latency-critical decode loop in which an allocator call could
+ * synchronize the device.
+ * Same arguments, layouts and results as tq_attend_decode, without the workspace: the scratch
+ * space is one fixed TQ_NOALLOC_SCRATCH_BYTES (8 MiB) array of device memory that the library
+ * defines statically; every GPU that loads the library keeps it until the process exits.
+ *   - The first call on a device looks up that array's device address (cudaGetSymbolAddress,
+ *     with the context's device made current) and caches it; make this first call before any
+ *     CUDA graph capture on that device.
+ *   - A request whose tq_attend_workspace_size exceeds TQ_NOALLOC_SCRATCH_BYTES returns
+ *     TQ_EINVAL with a message naming both sizes; nothing is launched.
+ *   - All calls on a device share the array and leave their contents in it.  No element needs to
+ *     start at zero (each call writes what it reads), but calls that overlap on the GPU (other
+ *     streams, other host threads) race on it: order them on one stream or with events.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine (with the tq_profile_*
+ *     instrumentation switched on, the library creates CUDA event objects as for any call). */
+#define TQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+tq_status tq_attend_decode_noalloc(const tq_ctx *kctx, const tq_ctx *vctx, const tq_attn_desc *desc,
+                                   const void *q, tq_dtype dtype, float *out, void *stream);
+
 /* Inner-product top-k over n packed database vectors (slots 0..n-1) ([JJ] 第三部分 "向量搜索"):
  * order by (estimated score descending, index ascending).
  *   q           device [nq][d] of dtype

@@ -61,6 +61,8 @@ def _load():
         "tq_attend_workspace_size": (st, [c_void_p, c_void_p, POINTER(AttnDesc), POINTER(c_size_t)]),
         "tq_attend_decode": (st, [c_void_p, c_void_p, POINTER(AttnDesc), c_void_p, c_int, c_void_p,
                                   c_void_p, c_size_t, c_void_p]),
+        "tq_attend_decode_noalloc": (st, [c_void_p, c_void_p, POINTER(AttnDesc), c_void_p, c_int, c_void_p,
+                                          c_void_p]),
         "tq_search_workspace_size": (st, [c_void_p, c_int32, c_int64, c_int32, POINTER(c_size_t)]),
         "tq_search_topk": (st, [c_void_p, c_void_p, c_int, c_int32, PackedC, c_int64, c_int32, c_void_p,
                                 c_void_p, c_void_p, c_size_t, c_void_p]),
@@ -307,6 +309,23 @@ def attend_decode(kctx: Context, vctx: Context, q: torch.Tensor, kcache: Packed,
     _check(LIB.tq_attend_decode(kctx.handle, vctx.handle, ctypes.byref(desc), _dev(q, kctx.device, "q"),
                                 _dtype_code(q), _dev(out, kctx.device, "out", torch.float32), w, wb,
                                 _stream_ptr(stream)))
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def attend_decode_noalloc(kctx: Context, vctx: Context, q: torch.Tensor, out: torch.Tensor, desc: AttnDesc,
+                          stream=None):
+    """tq_attend_decode_noalloc: decode attention whose scratch is the library's fixed 8 MiB
+    device array, for callers that cannot allocate device memory.  `out` must be preallocated
+    (fp32 [batch, n_q_heads, d]); `desc` comes from make_attn_desc.  Calls that overlap on the GPU
+    share that array and race; order them on one stream."""
+    if q.dim() != 3 or q.shape[2] != kctx.d:
+        raise ValueError(f"q must be [batch, heads, {kctx.d}]")
+    _check(LIB.tq_attend_decode_noalloc(kctx.handle, vctx.handle, ctypes.byref(desc), _dev(q, kctx.device, "q"),
+                                        _dtype_code(q), _dev(out, kctx.device, "out", torch.float32),
+                                        _stream_ptr(stream)))
     return out
 
 
