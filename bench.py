@@ -177,7 +177,8 @@ class DecodeLayerBench:
         seed = 1000 * rank
         self.kctx = tq.Context(self.d, self.kmse, self.m, synth.rotation_signs(self.d, seed + 1),
                                synth.qjl_matrix(self.m, self.d, seed + 2), device=dev.index)
-        self.vctx = tq.Context(self.d, w["v_bits"], 0, synth.rotation_signs(self.d, seed + 3), device=dev.index)
+        self.vctx = tq.Context(self.d, w["v_bits"], 0, synth.rotation_signs(self.d, seed + 3), device=dev.index,
+                               layout=tq.LAYOUT_BLOCK16)
         cap = self.batch * self.hkv * self.ctx
         g = torch.Generator(device=dev)
         g.manual_seed(seed + 7)
@@ -476,13 +477,13 @@ def ours_arm(args, world, rank):
 
     prof = profile_kernels(bench, min(args.steps, 10 * N_LAYERS))
     launches_per_step = sum(n for n, _ in prof.values()) / min(args.steps, 10 * N_LAYERS)
-    split_n, split_ms = prof.get("attend_split", (0, 0.0))
+    split_n, split_ms = prof.get("attend_split", (0, 0.0))  # the split kernel (tensor-core path here)
     peaks, src = measured_peaks()
     roof = None
     if split_n:
         per_launch_s = split_ms / split_n / 1e3
         achieved = bench.bytes_per_step / per_launch_s / 1e9
-        roof = {"kernel": "attend_split", "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+        roof = {"kernel": "attend_mma_kernel (split-context, tensor cores)", "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
                 "peak_source": src + " (burst copy)", "us_per_launch": per_launch_s * 1e6,
                 "algorithmic_bytes_per_launch": bench.bytes_per_step}

@@ -62,7 +62,20 @@ typedef struct {
   int32_t d;
   int32_t mse_bits;
   int32_t qjl_m;
+  int32_t layout;   /* tq_layout of the packed codes (TQ_LAYOUT_ROWS unless stated) */
 } tq_spec;
+
+/* Packed-code layouts.
+ *   TQ_LAYOUT_ROWS     every slot owns one code row (see tq_packed).
+ *   TQ_LAYOUT_BLOCK16  token-transposed blocks for attention values: MSE-only contexts
+ *                      (qjl_m == 0), capacities a multiple of 16.  Slots 16k .. 16k+15 share the
+ *                      16 * code_bytes bytes of block k, read as little-endian 32-bit words W:
+ *                        W[q*d + j], q < b/2:  bit t      = bit 2q   of code_j of slot 16k+t,
+ *                                              bit 16 + t = bit 2q+1 of code_j of slot 16k+t;
+ *                        W[(b/2)*d + j/2] (b odd): bit 16*(j%2) + t = bit b-1 of code_j of slot 16k+t,
+ *                      for t in [0,16), j in [0,d).  One word then holds one coordinate of 16
+ *                      tokens in two planes, the operand shape of the tensor-core value sum. */
+typedef enum { TQ_LAYOUT_ROWS = 0, TQ_LAYOUT_BLOCK16 = 1 } tq_layout;
 
 /* Packed, caller-owned device arrays indexed by slot (one slot = one encoded vector).
  *   codes  [capacity][code_bytes]  b bit-planes of d bits, plane t holding bit t of every code:
@@ -146,7 +159,8 @@ tq_status tq_encode_kv(const tq_ctx *ctx, const void *x, tq_dtype dtype, int64_t
                        const int64_t *slots, tq_packed out, void *ws, size_t ws_bytes,
                        void *stream);
 
-/* Estimated inner products of nq full-precision queries with n packed keys (slots 0..n-1)
+/* Estimated inner products of nq full-precision queries with n packed keys (slots 0..n-1);
+ * the context must use TQ_LAYOUT_ROWS
  * ([JJ] 第二部分 第二步 and 第六部分 "无偏估计的数学保证"):
  *   q' = (1/sqrt(d)) H (D q), p = S q',
  *   out[i][k] = nu_k ( <q', c[code_k]> + sqrt(pi/2)/m * gamma_k * sum_j (2 bit_kj - 1) p_j ).
@@ -161,7 +175,8 @@ tq_status tq_scores(const tq_ctx *ctx, const void *q, tq_dtype dtype, int32_t nq
 /* One decode step of attention over the compressed cache ([JJ] 第一部分 "KV 缓存是什么",
  * 第三部分 "推理速度"): logits = scale * estimated scores against the K cache, softmax over the
  * sequence, output = sum_t w_t * nu_t * D_V (1/sqrt(d)) H c_V[code_t] (V's MSE stage).
- *   kctx, vctx  contexts used to encode K and V (same d; vctx must have qjl_m == 0)
+ *   kctx, vctx  contexts used to encode K and V (same d; kctx in TQ_LAYOUT_ROWS; vctx with
+ *               qjl_m == 0, either layout; TQ_LAYOUT_BLOCK16 values enable the tensor-core path)
  *   q           device [batch][n_q_heads][d] of dtype
  *   out         device fp32 [batch][n_q_heads][d]; an empty sequence gives zeros
  *   ws          device workspace of tq_attend_workspace_size() bytes
@@ -195,7 +210,8 @@ tq_status tq_attend_decode(const tq_ctx *kctx, const tq_ctx *vctx, const tq_attn
 tq_status tq_attend_decode_noalloc(const tq_ctx *kctx, const tq_ctx *vctx, const tq_attn_desc *desc,
                                    const void *q, tq_dtype dtype, float *out, void *stream);
 
-/* Inner-product top-k over n packed database vectors (slots 0..n-1) ([JJ] 第三部分 "向量搜索"):
+/* Inner-product top-k over n packed database vectors (slots 0..n-1) ([JJ] 第三部分 "向量搜索");
+ * the context must use TQ_LAYOUT_ROWS:
  * order by (estimated score descending, index ascending).
  *   q           device [nq][d] of dtype
  *   out_scores  device fp32 [nq][k]

@@ -24,6 +24,10 @@ tq_status check_spec(const tq_spec *s) {
   if (s->qjl_m < 0 || s->qjl_m > 1024 || (s->qjl_m % 32) != 0)
     return tq_fail(TQ_EUNSUPPORTED, "qjl_m=%d: must be 0 or a multiple of 32 in [32, 1024]",
                    s->qjl_m);
+  if (s->layout != TQ_LAYOUT_ROWS && s->layout != TQ_LAYOUT_BLOCK16)
+    return tq_fail(TQ_EINVAL, "layout=%d: unknown", s->layout);
+  if (s->layout == TQ_LAYOUT_BLOCK16 && s->qjl_m != 0)
+    return tq_fail(TQ_EUNSUPPORTED, "TQ_LAYOUT_BLOCK16 holds MSE-only codes (qjl_m must be 0)");
   return TQ_OK;
 }
 
@@ -53,6 +57,8 @@ tq_status check_packed(const tq_ctx *c, const tq_packed &p, int64_t need, const 
       return tq_fail(TQ_EINVAL, "%s: rnorm not 4-byte aligned", name);
   }
   if (p.capacity < 0) return tq_fail(TQ_EINVAL, "%s: negative capacity", name);
+  if (c->spec.layout == TQ_LAYOUT_BLOCK16 && (p.capacity % 16) != 0)
+    return tq_fail(TQ_EINVAL, "%s: TQ_LAYOUT_BLOCK16 needs a capacity that is a multiple of 16", name);
   if (need > p.capacity)
     return tq_fail(TQ_EINVAL, "%s: %lld slots needed, capacity %lld", name, (long long)need,
                    (long long)p.capacity);
@@ -101,7 +107,7 @@ tq_status tq_make_codebook(int32_t d, int32_t bits, double *centroids, double *t
                            double *mse_per_coord) {
   g_err[0] = 0;
   if (!centroids || !thresholds) return tq_fail(TQ_EINVAL, "centroids/thresholds is NULL");
-  tq_spec s{d, bits, 0};
+  tq_spec s{d, bits, 0, TQ_LAYOUT_ROWS};
   tq_status st = check_spec(&s);
   if (st != TQ_OK) return st;
   return tq_codebook_fp64(d, bits, centroids, thresholds, mse_per_coord);
@@ -160,6 +166,7 @@ tq_status tq_ctx_create(const tq_spec *spec, const int8_t *rot_signs, const floa
   k.m = m;
   k.code_words = (int)(c->code_bytes / 4);
   k.sign_words = (int)(c->sign_bytes / 4);
+  k.layout = spec->layout;
   k.inv_sqrt_d = (float)(1.0 / std::sqrt((double)d));
   k.qjl_scale = m > 0 ? (float)(std::sqrt(M_PI / 2.0) / m) : 0.0f;
   for (int i = 0; i < TQ_MAX_LEVELS; ++i) {
@@ -168,6 +175,38 @@ tq_status tq_ctx_create(const tq_spec *spec, const int8_t *rot_signs, const floa
   }
   k.signs = c->dev_signs;
   k.S = c->dev_S;
+  // odd bit-plane expansion of the codebook for the tensor-core attention path:
+  // e_S = 2^-b sum_code c[code] prod_{P in S} s_P(code), S in {0}, {1}, {2}, {0,1,2}
+  k.fast_ok = 0;
+  for (int i = 0; i < 4; ++i) k.plane_coef[i] = 0.f;
+  k.plane_coef_sum = 0.f;
+  if (spec->mse_bits <= 3) {
+    const int b = spec->mse_bits;
+    const int nsets = b == 3 ? 4 : b;
+    double coef[4] = {0, 0, 0, 0};
+    for (int code = 0; code < L; ++code) {
+      double sg[3];
+      for (int P = 0; P < 3; ++P) sg[P] = ((code >> P) & 1) ? 1.0 : -1.0;
+      for (int S = 0; S < nsets; ++S) {
+        const double prod = S < 3 ? sg[S] : sg[0] * sg[1] * sg[2];
+        coef[S] += c->centroids[code] * prod / L;
+      }
+    }
+    double worst = 0.0;
+    for (int code = 0; code < L; ++code) {
+      double sg[3], rec = 0.0;
+      for (int P = 0; P < 3; ++P) sg[P] = ((code >> P) & 1) ? 1.0 : -1.0;
+      for (int S = 0; S < nsets; ++S) rec += coef[S] * (S < 3 ? sg[S] : sg[0] * sg[1] * sg[2]);
+      worst = std::fmax(worst, std::fabs(rec - c->centroids[code]));
+    }
+    double sum = 0.0;
+    for (int S = 0; S < nsets; ++S) {
+      k.plane_coef[S] = (float)coef[S];
+      sum += coef[S];
+    }
+    k.plane_coef_sum = (float)sum;
+    k.fast_ok = worst <= 1e-9 * std::fabs(c->centroids[L - 1]) ? 1 : 0;
+  }
   *out = c;
   return TQ_OK;
 }
@@ -278,6 +317,7 @@ tq_status tq_scores(const tq_ctx *ctx, const void *q, tq_dtype dtype, int32_t nq
   if (!q || !out) return tq_fail(TQ_EINVAL, "q/out is NULL");
   if (dtype != TQ_F32 && dtype != TQ_BF16) return tq_fail(TQ_EINVAL, "unknown dtype %d", (int)dtype);
   if (!aligned16(q) || !aligned16(out)) return tq_fail(TQ_EINVAL, "q/out not 16-byte aligned");
+  if (ctx->spec.layout != TQ_LAYOUT_ROWS) return tq_fail(TQ_EUNSUPPORTED, "tq_scores needs TQ_LAYOUT_ROWS");
   st = check_packed(ctx, keys, n, "keys", true);
   if (st != TQ_OK) return st;
   const size_t need = query_prep_bytes(ctx, nq);
@@ -303,6 +343,12 @@ static tq_status check_attn(const tq_ctx *kctx, const tq_ctx *vctx, const tq_att
     return tq_fail(TQ_EUNSUPPORTED, "K and V contexts differ in d (%d vs %d)", kctx->spec.d, vctx->spec.d);
   if (vctx->spec.qjl_m != 0)
     return tq_fail(TQ_EUNSUPPORTED, "the V context must be MSE-only (qjl_m == 0)");
+  if (kctx->spec.layout != TQ_LAYOUT_ROWS)
+    return tq_fail(TQ_EUNSUPPORTED, "the K context must use TQ_LAYOUT_ROWS");
+  if (vctx->spec.layout == TQ_LAYOUT_BLOCK16 && !desc->block_table && (desc->ctx_stride % 16) != 0)
+    return tq_fail(TQ_EINVAL, "TQ_LAYOUT_BLOCK16 values need ctx_stride to be a multiple of 16");
+  if (vctx->spec.layout == TQ_LAYOUT_BLOCK16 && desc->block_table && (desc->block_size % 16) != 0)
+    return tq_fail(TQ_EINVAL, "TQ_LAYOUT_BLOCK16 values need block_size to be a multiple of 16");
   if (desc->batch < 0 || desc->n_q_heads <= 0 || desc->n_kv_heads <= 0)
     return tq_fail(TQ_EINVAL, "batch/n_q_heads/n_kv_heads");
   if (desc->n_q_heads % desc->n_kv_heads != 0)
@@ -332,7 +378,7 @@ tq_status tq_attend_workspace_size(const tq_ctx *kctx, const tq_ctx *vctx, const
   tq_status st = check_attn(kctx, vctx, desc);
   if (st != TQ_OK) return st;
   if (!bytes) return tq_fail(TQ_EINVAL, "bytes is NULL");
-  const AttnPlan plan = attn_plan(*desc);
+  const AttnPlan plan = attn_plan(*desc, kctx->k, vctx->k);
   const int64_t nq = (int64_t)desc->batch * desc->n_q_heads;
   *bytes = query_prep_bytes(kctx, nq) + attn_partials_bytes(*desc, plan, kctx->spec.d);
   return TQ_OK;
@@ -361,7 +407,7 @@ tq_status tq_attend_decode(const tq_ctx *kctx, const tq_ctx *vctx, const tq_attn
   float *part = reinterpret_cast<float *>(static_cast<char *>(ws) + query_prep_bytes(kctx, nq));
   st = prep_queries(kctx, q, dtype, nq, qr, p, s);
   if (st != TQ_OK) return st;
-  const AttnPlan plan = attn_plan(*desc);
+  const AttnPlan plan = attn_plan(*desc, kctx->k, vctx->k);
   return tq_cuda_check(launch_attend(kctx->k, vctx->k, *desc, plan, qr, p, part, out, s),
                        "attention launch");
 }
@@ -393,6 +439,7 @@ tq_status tq_search_topk(const tq_ctx *ctx, const void *q, tq_dtype dtype, int32
   if (dtype != TQ_F32 && dtype != TQ_BF16) return tq_fail(TQ_EINVAL, "unknown dtype %d", (int)dtype);
   if (!aligned16(q) || !aligned16(out_scores) || !aligned16(out_idx))
     return tq_fail(TQ_EINVAL, "q/out not 16-byte aligned");
+  if (ctx->spec.layout != TQ_LAYOUT_ROWS) return tq_fail(TQ_EUNSUPPORTED, "tq_search_topk needs TQ_LAYOUT_ROWS");
   st = check_packed(ctx, db, n, "db", true);
   if (st != TQ_OK) return st;
   size_t need = 0;

@@ -147,7 +147,6 @@ attend_split_kernel(TqConsts kc, TqConsts vc, AttnArgs a, const float *__restric
     for (int i = 0; i < nt; ++i) {
       const int64_t si = sl[i];
       if (si < 0) continue;
-      const uint32_t *vrow = vcodes + si * vc.code_words;
       float wv[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) wv[g] = lg[g * kAtTile + i];
@@ -155,9 +154,7 @@ attend_split_kernel(TqConsts kc, TqConsts vc, AttnArgs a, const float *__restric
       for (int dd = 0; dd < kMaxDpt; ++dd) {
         const int j = tid + dd * kAtThreads;
         if (j < d) {
-          int code = 0;
-          for (int tb = 0; tb < vc.bits; ++tb) code |= code_bit(vrow, tb, j, d) << tb;
-          const float cv = centV[code];
+          const float cv = centV[slot_code(vcodes, si, j, vc)];
 #pragma unroll
           for (int g = 0; g < G; ++g) acc[g][dd] = fmaf(wv[g], cv, acc[g][dd]);
         }
@@ -234,9 +231,18 @@ cudaError_t launch_split(const TqConsts &kc, const TqConsts &vc, const AttnArgs 
 
 }  // namespace
 
-AttnPlan attn_plan(const tq_attn_desc &desc) {
+AttnPlan attn_plan(const tq_attn_desc &desc, const TqConsts &kc, const TqConsts &vc) {
   AttnPlan p;
   p.group = desc.n_q_heads / desc.n_kv_heads;
+  p.fast = attn_fast_eligible(kc, vc, desc);
+  p.extra = 0;
+  if (p.fast) {
+    const int maxlen = desc.max_seq_len > 0 ? desc.max_seq_len : 1;
+    p.chunk = attn_fast_chunk(desc);
+    p.splits = (maxlen + p.chunk - 1) / p.chunk;
+    p.extra = attn_fast_extra_bytes(kc, desc);
+    return p;
+  }
   const int64_t rows = (int64_t)desc.batch * desc.n_kv_heads;
   const int maxlen = desc.max_seq_len > 0 ? desc.max_seq_len : 1;
   const int64_t want = rows > 0 ? (4 * 148 + rows - 1) / rows : 1;
@@ -249,7 +255,8 @@ AttnPlan attn_plan(const tq_attn_desc &desc) {
 }
 
 size_t attn_partials_bytes(const tq_attn_desc &desc, const AttnPlan &plan, int d) {
-  return sizeof(float) * (size_t)desc.batch * desc.n_q_heads * plan.splits * (d + 2);
+  return (size_t)tq_align_up((int64_t)sizeof(float) * desc.batch * desc.n_q_heads * plan.splits * (d + 2), 256) +
+         plan.extra;
 }
 
 cudaError_t launch_attend(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc,
@@ -273,7 +280,12 @@ cudaError_t launch_attend(const TqConsts &kc, const TqConsts &vc, const tq_attn_
   a.v = desc.v;
   dim3 grid((unsigned)plan.splits, (unsigned)desc.n_kv_heads, (unsigned)desc.batch);
   cudaError_t e;
-  switch (plan.group) {
+  if (plan.fast) {
+    void *extra = reinterpret_cast<char *>(partials) +
+                  tq_align_up((int64_t)sizeof(float) * desc.batch * desc.n_q_heads * plan.splits * (kc.d + 2), 256);
+    e = launch_attend_fast(kc, vc, desc, plan, qr, p, extra, partials, st);
+    if (e != cudaSuccess) return e;
+  } else switch (plan.group) {
     case 1: e = launch_split<1>(kc, vc, a, grid, qr, p, partials, st); break;
     case 2: e = launch_split<2>(kc, vc, a, grid, qr, p, partials, st); break;
     case 4: e = launch_split<4>(kc, vc, a, grid, qr, p, partials, st); break;

@@ -1,0 +1,488 @@
+// Tensor-core decode attention for head_dim 128 and 4 query heads per KV head.
+//
+// Same mathematics as attend_split_kernel (estimated logits "谷歌 TurboQuant 深度拆解" 第二部分
+// 第二步, softmax, value sum in the rotated domain), reorganised so that the per-bit work runs on
+// the tensor cores as exact integer matrix products:
+//
+//  * A symmetric Lloyd-Max codebook is an odd function of the bit-plane signs s_P = 2 b_P - 1:
+//      c(code) = sum_P e_P s_P  (+ e_3 s_0 s_1 s_2 for 3 bits),
+//    so <q', c[code]> = sum_P 2 e_P <q', b_P> - (sum_P e_P) sum_j q'_j, with b_P the 0/1 plane
+//    (the 3-bit cubic term uses the parity plane b_0 ^ b_1 ^ b_2).  The QJL term is likewise
+//    2 <p, b_sign> - sum_i p_i.
+//  * Logits: one m16n8k32 u8 x s8 MMA per (16 keys, plane, 32 coordinates).  A = the keys' bit
+//    words masked in place (w & (0x01010101 << shift): bytes 0 or 2^shift, one LOP3 per 4
+//    elements); B = the query term 2 e_P q' (or 2 p) in 32-bit fixed point split into four signed
+//    byte limbs and pre-scaled by 2^-shift, built once per (sequence, KV head) by kfrag_kernel.
+//    Columns: 4 heads x 4 limbs (two n-tiles), so each thread ends with all limbs of one head.
+//  * Values are stored token-transposed (TQ_LAYOUT_BLOCK16): one 32-bit word = one coordinate of
+//    16 tokens in two planes, so (w >> t) & 0x01010101 gives four tokens of one coordinate, the
+//    A operand of an MMA that contracts over tokens.  B = the softmax weights times the value
+//    norms in 16-bit fixed point (two byte limbs), columns = 4 heads x 2 planes x 2 limbs.
+//  * Softmax is two-pass per chunk (all logits of the chunk, then one max per head), so every
+//    value product of the chunk shares one fixed-point scale and the int32 accumulators need no
+//    rescaling; splits are merged by attend_combine_kernel as for the general kernel.
+// Each CTA: 8 warps, one chunk of CH tokens of one (sequence, KV head).
+#include <cmath>
+
+#include "device_common.cuh"
+
+namespace {
+
+constexpr int kD = 128;
+constexpr int kG = 4;
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+struct MmaArgs {
+  int hq, hkv, max_len, chunk, splits, block_size, max_blocks;
+  int64_t ctx_stride;
+  float scale;
+  const int32_t *seq_lens;
+  const int32_t *block_table;
+  tq_packed k, v;
+};
+
+__device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ int64_t token_slot(const MmaArgs &a, int b, int h, int t) {
+  if (a.block_table) {
+    const int blk = a.block_table[(int64_t)b * a.max_blocks + t / a.block_size];
+    return blk < 0 ? -1 : ((int64_t)blk * a.hkv + h) * a.block_size + t % a.block_size;
+  }
+  return ((int64_t)b * a.hkv + h) * a.ctx_stride + t;
+}
+
+// Signed byte limbs of v = l0 + 2^8 l1 + 2^16 l2 + 2^24 l3, each l in [-128, 127].
+__device__ __forceinline__ int next_limb(int &v) {
+  const int l = ((v + 128) & 255) - 128;
+  v = (v - l) >> 8;
+  return l;
+}
+
+__device__ __forceinline__ float warp_max_f(float x) {
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) x = fmaxf(x, __shfl_xor_sync(TQ_FULL_MASK, x, s));
+  return x;
+}
+__device__ __forceinline__ float warp_sum_f(float x) {
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) x += __shfl_xor_sync(TQ_FULL_MASK, x, s);
+  return x;
+}
+
+template <int BK, bool QJL>
+struct KPlanes {
+  static constexpr int code = BK + (BK == 3 ? 1 : 0);  // code planes (+ parity plane for 3 bits)
+  static constexpr int all = code + (QJL ? 1 : 0);     // + the QJL sign plane
+  static constexpr int regs = all * 4 * 2 * 2;          // planes x k-steps x n-tiles x regs
+};
+
+// Query-side B fragments of the logit MMAs for one (sequence, KV head): for plane P, k-step s,
+// n-tile nt, register r and lane (gid, t): bytes i = 0..3 hold limb (gid & 1) + 2 nt of
+//   round(X_P[head gid/2][32 t + s + 4 r + 8 i] * 2^(F - s - 4 r)),
+// X_P = 2 e_P q' (code planes, parity), 2 p (sign plane); F per head and part so that
+// |X| 2^F <= 2^30.  kconst: 2^-F_code, 2^-F_sign, (sum e_P) sum q', sum p per head.
+template <int BK, bool QJL>
+__global__ void __launch_bounds__(kThreads)
+kfrag_kernel(TqConsts kc, const float *__restrict__ qr, const float *__restrict__ p,
+             uint32_t *__restrict__ kfrag, float *__restrict__ kconst) {
+  using KP = KPlanes<BK, QJL>;
+  __shared__ float X[KP::all][kG][kD];
+  __shared__ float red[kG][4];
+  __shared__ int fexp[kG][2];
+  const int grp = blockIdx.x;  // b * hkv + h; its query heads are rows grp * 4 + g
+  const int tid = threadIdx.x;
+  for (int i = tid; i < kG * kD; i += kThreads) {
+    const int g = i / kD, j = i % kD;
+    const float q = qr[((int64_t)grp * kG + g) * kD + j];
+#pragma unroll
+    for (int P = 0; P < BK; ++P) X[P][g][j] = 2.f * kc.plane_coef[P] * q;
+    if constexpr (BK == 3) X[3][g][j] = 2.f * kc.plane_coef[3] * q;
+    if constexpr (QJL) X[KP::code][g][j] = 2.f * p[((int64_t)grp * kG + g) * kD + j];
+  }
+  __syncthreads();
+  const int warp = tid >> 5, lane = tid & 31;
+  if (warp < kG) {
+    const int g = warp;
+    float mc = 0.f, ms = 0.f, sq = 0.f, sp = 0.f;
+    for (int j = lane; j < kD; j += 32) {
+#pragma unroll
+      for (int P = 0; P < KP::code; ++P) mc = fmaxf(mc, fabsf(X[P][g][j]));
+      if constexpr (QJL) {
+        ms = fmaxf(ms, fabsf(X[KP::code][g][j]));
+        sp += 0.5f * X[KP::code][g][j];
+      }
+      sq += qr[((int64_t)grp * kG + g) * kD + j];
+    }
+    mc = warp_max_f(mc);
+    ms = warp_max_f(ms);
+    sq = warp_sum_f(sq);
+    sp = warp_sum_f(sp);
+    if (lane == 0) {
+      int ec = 0, es = 0;
+      frexpf(mc, &ec);  // mc < 2^ec
+      frexpf(ms, &es);
+      fexp[g][0] = mc > 0.f ? 30 - ec : 0;
+      fexp[g][1] = ms > 0.f ? 30 - es : 0;
+      red[g][0] = ldexpf(1.f, -fexp[g][0]);
+      red[g][1] = ldexpf(1.f, -fexp[g][1]);
+      red[g][2] = kc.plane_coef_sum * sq;
+      red[g][3] = sp;
+    }
+  }
+  __syncthreads();
+  if (tid < 16) kconst[(int64_t)grp * 16 + tid] = red[tid % 4][tid / 4];
+  uint32_t *out = kfrag + (int64_t)grp * KP::regs * 32;
+  for (int idx = tid; idx < KP::regs * 32; idx += kThreads) {
+    const int ln = idx & 31;
+    int rest = idx >> 5;
+    const int r = rest & 1;
+    rest >>= 1;
+    const int nt = rest & 1;
+    rest >>= 1;
+    const int s = rest & 3;
+    const int P = rest >> 2;
+    const int gid = ln >> 2, t = ln & 3;
+    const int g = gid >> 1, limb = (gid & 1) + 2 * nt;
+    const int shift = s + 4 * r;
+    const int F = fexp[g][(QJL && P == KP::code) ? 1 : 0];
+    uint32_t word = 0u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int j = 32 * t + s + 4 * r + 8 * i;
+      int v = __float2int_rn(ldexpf(X[P][g][j], F - shift));
+      int l = 0;
+#pragma unroll
+      for (int k = 0; k <= 3; ++k) {
+        const int li = next_limb(v);
+        if (k == limb) l = li;
+      }
+      word |= (uint32_t)(l & 255) << (8 * i);
+    }
+    out[idx] = word;
+  }
+}
+
+template <int BK, int BV, bool QJL, int CH>
+__global__ void __launch_bounds__(kThreads, 1)
+attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restrict__ kfrag,
+                  const float *__restrict__ kconst, float *__restrict__ part) {
+  using KP = KPlanes<BK, QJL>;
+  constexpr int NBLK = CH / 16;
+  constexpr int KB_PER_WARP = NBLK / kWarps;
+  constexpr int VT = BV == 3 ? 2 : 1;  // value word types: (p0,p1) and (p2, parity)
+  __shared__ float lg[kG][CH];         // logits, then weights * value norms
+  __shared__ int64_t sslot[CH];        // slot of each chunk token, -1 if masked
+  __shared__ uint4 vfrag[NBLK][32];    // value-side B fragments per 16-token block
+  __shared__ float red[kWarps][3 * kG];
+  __shared__ float hstat[5][kG];       // max logit, sum w, sum w*nu, fixed-point multiplier, its inverse
+
+  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gid = lane >> 2, t = lane & 3;
+  int L = a.seq_lens[b];
+  L = L < 0 ? 0 : (L > a.max_len ? a.max_len : L);
+  const int t0 = s * CH;
+  const int t1 = min(L, t0 + CH);
+  const int64_t grp = (int64_t)b * a.hkv + h;
+  const int64_t cap = min(a.k.capacity, a.v.capacity);
+  const uint32_t *kcodes = static_cast<const uint32_t *>(a.k.codes);
+  const uint32_t *ksigns = static_cast<const uint32_t *>(a.k.signs);
+  const uint32_t *vcodes = static_cast<const uint32_t *>(a.v.codes);
+
+  // ---------------------------------------------------------------- phase 1: logits (keys x heads)
+  {
+    uint32_t kb[KP::all][4][2][2];
+    const uint32_t *fr = kfrag + grp * KP::regs * 32 + lane;
+#pragma unroll
+    for (int P = 0; P < KP::all; ++P)
+#pragma unroll
+      for (int st = 0; st < 4; ++st)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int r = 0; r < 2; ++r) kb[P][st][nt][r] = fr[((((P * 4 + st) * 2 + nt) * 2) + r) * 32];
+    const float cfc = kconst[grp * 16 + t], cfs = kconst[grp * 16 + 4 + t];
+    const float cq = kconst[grp * 16 + 8 + t], cp = kconst[grp * 16 + 12 + t];
+#pragma unroll 1
+    for (int mb = 0; mb < KB_PER_WARP; ++mb) {
+      const int blk = warp * KB_PER_WARP + mb;
+      const int tb = t0 + blk * 16;
+      uint32_t w[2][KP::all];
+      float nu[2], gam[2];
+      bool ok[2];
+      int64_t slot[2];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int tok = tb + gid + 8 * r;
+        ok[r] = tok < t1;
+        slot[r] = ok[r] ? token_slot(a, b, h, tok) : -1;
+        ok[r] = ok[r] && slot[r] >= 0 && slot[r] < cap;
+#pragma unroll
+        for (int P = 0; P < BK; ++P) w[r][P] = ok[r] ? kcodes[slot[r] * kc.code_words + P * 4 + t] : 0u;
+        if constexpr (BK == 3) w[r][3] = w[r][0] ^ w[r][1] ^ w[r][2];
+        if constexpr (QJL) w[r][KP::code] = ok[r] ? ksigns[slot[r] * kc.sign_words + t] : 0u;
+        nu[r] = ok[r] ? a.k.norm[slot[r]] : 0.f;
+        gam[r] = (QJL && ok[r]) ? a.k.rnorm[slot[r]] : 0.f;
+      }
+      int acc[2][2][4];
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+#pragma unroll
+        for (int y = 0; y < 2; ++y)
+#pragma unroll
+          for (int z = 0; z < 4; ++z) acc[x][y][z] = 0;
+#pragma unroll
+      for (int P = 0; P < KP::all; ++P) {
+        const int pt = (QJL && P == KP::code) ? 1 : 0;
+#pragma unroll
+        for (int st = 0; st < 4; ++st) {
+          const uint32_t mlo = 0x01010101u << st, mhi = 0x01010101u << (st + 4);
+          const uint32_t a0 = w[0][P] & mlo, a1 = w[1][P] & mlo, a2 = w[0][P] & mhi, a3 = w[1][P] & mhi;
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) mma_u8s8(acc[pt][nt], a0, a1, a2, a3, kb[P][st][nt][0], kb[P][st][nt][1]);
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const float dc = (float)acc[0][0][2 * r] + 256.f * (float)acc[0][0][2 * r + 1] +
+                         65536.f * (float)acc[0][1][2 * r] + 16777216.f * (float)acc[0][1][2 * r + 1];
+        float sc = fmaf(dc, cfc, -cq);
+        if constexpr (QJL) {
+          const float ds = (float)acc[1][0][2 * r] + 256.f * (float)acc[1][0][2 * r + 1] +
+                           65536.f * (float)acc[1][1][2 * r] + 16777216.f * (float)acc[1][1][2 * r + 1];
+          sc = fmaf(kc.qjl_scale * gam[r], fmaf(ds, cfs, -cp), sc);
+        }
+        const int i = blk * 16 + gid + 8 * r;
+        lg[t][i] = ok[r] ? a.scale * nu[r] * sc : -INFINITY;
+        if (t == 0) sslot[i] = ok[r] ? slot[r] : -1;
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---------------------------------------------------------------- phase 2: softmax weights
+  if (warp < kG) {
+    float mx = -INFINITY;
+    for (int i = lane; i < CH; i += 32) mx = fmaxf(mx, lg[warp][i]);
+    mx = warp_max_f(mx);
+    if (lane == 0) hstat[0][warp] = mx;
+  }
+  __syncthreads();
+  {
+    float sw[kG], sW[kG], mW[kG];
+#pragma unroll
+    for (int g = 0; g < kG; ++g) sw[g] = sW[g] = mW[g] = 0.f;
+    for (int i = threadIdx.x; i < CH; i += kThreads) {
+      const int64_t sl = sslot[i];
+      const float nv = sl >= 0 ? a.v.norm[sl] : 0.f;
+#pragma unroll
+      for (int g = 0; g < kG; ++g) {
+        const float wgt = sl >= 0 ? __expf(lg[g][i] - hstat[0][g]) : 0.f;
+        const float W = wgt * nv;
+        lg[g][i] = W;
+        sw[g] += wgt;
+        sW[g] += W;
+        mW[g] = fmaxf(mW[g], fabsf(W));
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < kG; ++g) {
+      sw[g] = warp_sum_f(sw[g]);
+      sW[g] = warp_sum_f(sW[g]);
+      mW[g] = warp_max_f(mW[g]);
+    }
+    if (lane == 0)
+#pragma unroll
+      for (int g = 0; g < kG; ++g) {
+        red[warp][g] = sw[g];
+        red[warp][kG + g] = sW[g];
+        red[warp][2 * kG + g] = mW[g];
+      }
+  }
+  __syncthreads();
+  if (threadIdx.x < kG) {
+    const int g = threadIdx.x;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f;
+    for (int w = 0; w < kWarps; ++w) {
+      a0 += red[w][g];
+      a1 += red[w][kG + g];
+      a2 = fmaxf(a2, red[w][2 * kG + g]);
+    }
+    int e = 0;
+    frexpf(a2, &e);  // a2 < 2^e
+    const int F = a2 > 0.f ? 14 - e : 0;
+    hstat[1][g] = a0;
+    hstat[2][g] = a1;
+    hstat[3][g] = ldexpf(1.f, F);
+    hstat[4][g] = ldexpf(1.f, -F);
+  }
+  __syncthreads();
+  {
+    // B fragments of the value MMAs: lane (gid, t) = column (head gid/2, plane gid&1) and
+    // tokens t, t+8 (register 0) and t+4, t+12 (register 1); n-tile = limb.
+    const int g = gid >> 1, ps = gid & 1;
+    const float mul = hstat[3][g];
+    for (int kb = warp; kb < NBLK; kb += kWarps) {
+      const float *wr = &lg[g][kb * 16];
+      int v[4] = {__float2int_rn(wr[t] * mul), __float2int_rn(wr[t + 8] * mul),
+                  __float2int_rn(wr[t + 4] * mul), __float2int_rn(wr[t + 12] * mul)};
+      uint32_t lo[4], hi[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        lo[i] = (uint32_t)(next_limb(v[i]) & 255);
+        hi[i] = (uint32_t)(next_limb(v[i]) & 255);
+      }
+      const int sh = 16 * ps;
+      vfrag[kb][lane] = make_uint4((lo[0] | (lo[1] << 8)) << sh, (lo[2] | (lo[3] << 8)) << sh,
+                                   (hi[0] | (hi[1] << 8)) << sh, (hi[2] | (hi[3] << 8)) << sh);
+    }
+  }
+  __syncthreads();
+
+  // ---------------------------------------------------------------- phase 3: value sum
+  // warp w owns coordinates 16 w .. 16 w + 15; row gid <-> coordinate 16 w + 2 gid, row gid + 8
+  // <-> 16 w + 2 gid + 1, so a thread's two rows are adjacent words.
+  const int j0 = warp * 16 + 2 * gid;
+  int accv[VT][2][4];
+#pragma unroll
+  for (int x = 0; x < VT; ++x)
+#pragma unroll
+    for (int y = 0; y < 2; ++y)
+#pragma unroll
+      for (int z = 0; z < 4; ++z) accv[x][y][z] = 0;
+#pragma unroll 2
+  for (int kb = 0; kb < NBLK; ++kb) {
+    const int tb = t0 + kb * 16;
+    if (tb >= t1) break;
+    const int64_t base = token_slot(a, b, h, tb);  // first slot of a 16-slot block
+    if (base < 0 || base >= a.v.capacity) continue;
+    const uint32_t *vb = vcodes + (base >> 4) * (int64_t)(16 * vc.code_words);
+    const uint2 A = *reinterpret_cast<const uint2 *>(vb + j0);
+    uint32_t X[VT][2];
+    X[0][0] = A.x;
+    X[0][1] = A.y;
+    if constexpr (BV == 3) {
+      const uint32_t hw = vb[kD + (j0 >> 1)];
+      const uint32_t p0 = (A.x ^ (A.x >> 16) ^ hw) & 0xffffu;
+      const uint32_t p1 = (A.y ^ (A.y >> 16) ^ (hw >> 16)) & 0xffffu;
+      X[VT - 1][0] = (hw & 0xffffu) | (p0 << 16);
+      X[VT - 1][1] = (hw >> 16) | (p1 << 16);
+    }
+    const uint4 fb = vfrag[kb][lane];
+#pragma unroll
+    for (int x = 0; x < VT; ++x) {
+      const uint32_t a0 = (X[x][0] >> t) & 0x01010101u, a1 = (X[x][1] >> t) & 0x01010101u;
+      const uint32_t a2 = (X[x][0] >> (t + 4)) & 0x01010101u, a3 = (X[x][1] >> (t + 4)) & 0x01010101u;
+      mma_u8s8(accv[x][0], a0, a1, a2, a3, fb.x, fb.y);
+      mma_u8s8(accv[x][1], a0, a1, a2, a3, fb.z, fb.w);
+    }
+  }
+  // accv[x][limb][c]: c0/c1 = (coordinate j0, head t, plane lo/hi), c2/c3 = (j0 + 1, ...)
+  const float inv = hstat[4][t];
+  const float csum = vc.plane_coef_sum * hstat[2][t];
+  const int64_t pbase = (((int64_t)b * a.hq + (int64_t)h * kG + t) * a.splits + s) * (kD + 2);
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    float v = 0.f;
+#pragma unroll
+    for (int x = 0; x < VT; ++x)
+#pragma unroll
+      for (int ps = 0; ps < 2; ++ps) {
+        const float D = (float)accv[x][0][2 * r + ps] + 256.f * (float)accv[x][1][2 * r + ps];
+        v = fmaf(2.f * vc.plane_coef[2 * x + ps], D, v);
+      }
+    part[pbase + 2 + j0 + r] = fmaf(v, inv, -csum);
+  }
+  if (threadIdx.x < kG) {
+    const int64_t pb = (((int64_t)b * a.hq + (int64_t)h * kG + threadIdx.x) * a.splits + s) * (kD + 2);
+    part[pb] = hstat[0][threadIdx.x];
+    part[pb + 1] = hstat[1][threadIdx.x];
+  }
+}
+
+template <int BK, int BV, bool QJL>
+cudaError_t launch_fast(const TqConsts &kc, const TqConsts &vc, const MmaArgs &a, int batch, const float *qr,
+                        const float *p, uint32_t *kfrag, float *kconst, float *part, cudaStream_t st) {
+  const unsigned groups = (unsigned)(batch * a.hkv);
+  tq_prof_begin(TQK_ATTEND_FRAG, st);
+  kfrag_kernel<BK, QJL><<<groups, kThreads, 0, st>>>(kc, qr, p, kfrag, kconst);
+  tq_prof_end(TQK_ATTEND_FRAG, st);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)a.splits, (unsigned)a.hkv, (unsigned)batch);
+  tq_prof_begin(TQK_ATTEND_SPLIT, st);
+  if (a.chunk == 512)
+    attend_mma_kernel<BK, BV, QJL, 512><<<grid, kThreads, 0, st>>>(kc, vc, a, kfrag, kconst, part);
+  else
+    attend_mma_kernel<BK, BV, QJL, 256><<<grid, kThreads, 0, st>>>(kc, vc, a, kfrag, kconst, part);
+  tq_prof_end(TQK_ATTEND_SPLIT, st);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool attn_fast_eligible(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc) {
+  if (desc.n_kv_heads <= 0 || desc.n_q_heads != kG * desc.n_kv_heads) return false;
+  if (kc.d != kD || vc.d != kD) return false;
+  if (kc.layout != TQ_LAYOUT_ROWS || vc.layout != TQ_LAYOUT_BLOCK16) return false;
+  if (kc.bits < 1 || kc.bits > 3 || (vc.bits != 2 && vc.bits != 3)) return false;
+  if (kc.m != 0 && kc.m != kD) return false;
+  if (!kc.fast_ok || !vc.fast_ok) return false;
+  if (desc.block_table ? (desc.block_size % 16) != 0 : (desc.ctx_stride % 16) != 0) return false;
+  return true;
+}
+
+int attn_fast_chunk(const tq_attn_desc &desc) {
+  const int64_t rows = (int64_t)desc.batch * desc.n_kv_heads;
+  const int maxlen = desc.max_seq_len > 0 ? desc.max_seq_len : 1;
+  const int64_t ctas512 = rows * ((maxlen + 511) / 512);
+  return ctas512 >= 8 * 148 ? 512 : 256;
+}
+
+size_t attn_fast_extra_bytes(const TqConsts &kc, const tq_attn_desc &desc) {
+  const int planes = (kc.bits + (kc.bits == 3 ? 1 : 0)) + (kc.m > 0 ? 1 : 0);
+  const int64_t groups = (int64_t)desc.batch * desc.n_kv_heads;
+  return (size_t)tq_align_up(groups * planes * 16 * 32 * 4, 256) + (size_t)tq_align_up(groups * 16 * 4, 256);
+}
+
+cudaError_t launch_attend_fast(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc,
+                               const AttnPlan &plan, const float *qr, const float *p, void *extra,
+                               float *partials, cudaStream_t st) {
+  MmaArgs a;
+  a.hq = desc.n_q_heads;
+  a.hkv = desc.n_kv_heads;
+  a.max_len = desc.max_seq_len;
+  a.chunk = plan.chunk;
+  a.splits = plan.splits;
+  a.block_size = desc.block_size;
+  a.max_blocks = desc.max_blocks;
+  a.ctx_stride = desc.ctx_stride;
+  a.scale = desc.scale != 0.f ? desc.scale : kc.inv_sqrt_d;
+  a.seq_lens = desc.seq_lens;
+  a.block_table = desc.block_table;
+  a.k = desc.k;
+  a.v = desc.v;
+  const int planes = (kc.bits + (kc.bits == 3 ? 1 : 0)) + (kc.m > 0 ? 1 : 0);
+  const int64_t groups = (int64_t)desc.batch * desc.n_kv_heads;
+  uint32_t *kfrag = static_cast<uint32_t *>(extra);
+  float *kconst = reinterpret_cast<float *>(static_cast<char *>(extra) +
+                                            tq_align_up(groups * planes * 16 * 32 * 4, 256));
+  const bool qjl = kc.m > 0;
+#define TQ_FAST(BKV, BVV, Q)                                                                           \
+  if (kc.bits == BKV && vc.bits == BVV && qjl == Q)                                                    \
+    return launch_fast<BKV, BVV, Q>(kc, vc, a, desc.batch, qr, p, kfrag, kconst, partials, st);
+  TQ_FAST(1, 2, true) TQ_FAST(2, 2, true) TQ_FAST(3, 2, true)
+  TQ_FAST(1, 3, true) TQ_FAST(2, 3, true) TQ_FAST(3, 3, true)
+  TQ_FAST(1, 2, false) TQ_FAST(2, 2, false) TQ_FAST(3, 2, false)
+  TQ_FAST(1, 3, false) TQ_FAST(2, 3, false) TQ_FAST(3, 3, false)
+#undef TQ_FAST
+  return cudaErrorInvalidValue;
+}

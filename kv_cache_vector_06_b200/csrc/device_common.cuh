@@ -16,6 +16,28 @@ __device__ __forceinline__ int code_bit(const uint32_t *row, int t, int j, int d
   return (int)((row[pos >> 5] >> (pos & 31)) & 1u);
 }
 
+// Full code of coordinate j of `slot` in either packed layout (see tq_layout in tq.h).
+__device__ __forceinline__ int slot_code(const uint32_t *codes, int64_t slot, int j, const TqConsts &c) {
+  int code = 0;
+  if (c.layout == TQ_LAYOUT_ROWS) {
+    const uint32_t *row = codes + slot * c.code_words;
+    for (int t = 0; t < c.bits; ++t) code |= code_bit(row, t, j, c.d) << t;
+  } else {
+    const uint32_t *blk = codes + (slot >> 4) * (int64_t)(16 * c.code_words);
+    const int tok = (int)(slot & 15);
+    for (int q = 0; q < c.bits / 2; ++q) {
+      const uint32_t w = blk[q * c.d + j];
+      code |= (int)((w >> tok) & 1u) << (2 * q);
+      code |= (int)((w >> (16 + tok)) & 1u) << (2 * q + 1);
+    }
+    if (c.bits & 1) {
+      const uint32_t w = blk[(c.bits / 2) * c.d + (j >> 1)];
+      code |= (int)((w >> (16 * (j & 1) + tok)) & 1u) << (c.bits - 1);
+    }
+  }
+  return code;
+}
+
 // 32 consecutive coordinates [32w, 32w+32) of bit-plane t as one word (d >= 32), or the whole
 // d-bit plane t in the low d bits (d < 32; then w must be 0).
 __device__ __forceinline__ uint32_t plane_word(const uint32_t *row, int t, int w, int d) {

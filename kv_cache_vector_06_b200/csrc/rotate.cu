@@ -151,6 +151,39 @@ rotate_kernel(TqConsts c, int mode, const void *__restrict__ x, int dtype, int64
       rr = fmaf(v[k][e], v[k][e], rr);
     }
 
+  const int64_t slot = valid ? (slots ? slots[row] : row) : -1;
+  const bool store = valid && slot >= 0 && slot < capacity;
+
+  if (c.layout == TQ_LAYOUT_BLOCK16) {
+    // token-transposed blocks: set this slot's bit in the shared words of its 16-slot block
+    if (store) {
+      uint32_t *blk = codes + (slot >> 4) * (int64_t)(16 * c.code_words);
+      const int tok = (int)(slot & 15);
+#pragma unroll
+      for (int k = 0; k < KCH; ++k)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = 4 * (l + LPV * k) + e;
+          const int cd = code[k][e];
+          for (int q = 0; q < c.bits / 2; ++q) {
+            const uint32_t mask = (1u << tok) | (1u << (16 + tok));
+            const uint32_t val = ((uint32_t)((cd >> (2 * q)) & 1) << tok) |
+                                 ((uint32_t)((cd >> (2 * q + 1)) & 1) << (16 + tok));
+            atomicAnd(&blk[q * D + j], ~mask);
+            atomicOr(&blk[q * D + j], val);
+          }
+          if (c.bits & 1) {
+            const int sh = 16 * (j & 1) + tok;
+            uint32_t *w = &blk[(c.bits / 2) * D + (j >> 1)];
+            atomicAnd(w, ~(1u << sh));
+            atomicOr(w, (uint32_t)((cd >> (c.bits - 1)) & 1) << sh);
+          }
+        }
+      if (l == 0) norm[slot] = nu;
+    }
+    return;  // MSE-only: no residual
+  }
+
   // pack the bit-planes
   uint32_t *st = stage[wib][g];
   for (int i = l; i < c.code_words; i += LPV) st[i] = 0u;
@@ -166,8 +199,6 @@ rotate_kernel(TqConsts c, int mode, const void *__restrict__ x, int dtype, int64
     }
   __syncwarp();
 
-  const int64_t slot = valid ? (slots ? slots[row] : row) : -1;
-  const bool store = valid && slot >= 0 && slot < capacity;
   if (store) {
     uint4 *dst = reinterpret_cast<uint4 *>(codes + slot * c.code_words);
     for (int i = l; i < c.code_words / 4; i += LPV)

@@ -18,6 +18,10 @@ struct TqConsts {
   int m;          // QJL rows (0 or multiple of 32)
   int code_words; // 32-bit words per packed code row
   int sign_words; // 32-bit words per packed sign row
+  int layout;     // tq_layout of the packed codes
+  int fast_ok;    // codebook is an exact odd bit-plane expansion (tensor-core attention path)
+  float plane_coef[4];   // e_P of c(code) = sum e_P s_P (+ e_3 s_0 s_1 s_2), s_P = 2 bit_P - 1
+  float plane_coef_sum;  // sum of plane_coef
   float inv_sqrt_d;
   float qjl_scale;  // sqrt(pi/2)/m, 0 when m == 0
   float centroids[TQ_MAX_LEVELS];
@@ -46,7 +50,7 @@ tq_status tq_cuda_check(cudaError_t e, const char *what);
 // ---------------------------------------------------------------- profile.cu
 enum TqKernelKind {
   TQK_ROTATE_ENCODE = 0, TQK_QJL_PROJECT, TQK_ROTATE_QUERY, TQK_QUERY_PROJECT, TQK_SCORES,
-  TQK_ATTEND_SPLIT, TQK_ATTEND_COMBINE, TQK_SEARCH_SCAN, TQK_SEARCH_MERGE, TQK_COUNT
+  TQK_ATTEND_SPLIT, TQK_ATTEND_COMBINE, TQK_SEARCH_SCAN, TQK_SEARCH_MERGE, TQK_ATTEND_FRAG, TQK_COUNT
 };
 void tq_prof_begin(int kind, cudaStream_t st);
 void tq_prof_end(int kind, cudaStream_t st);
@@ -80,12 +84,21 @@ struct AttnPlan {
   int group;        // n_q_heads / n_kv_heads
   int chunk;        // tokens per split
   int splits;       // splits per (batch, kv head)
+  bool fast;        // tensor-core path (attend_mma.cu)
+  size_t extra;     // workspace bytes of the tensor-core path's query fragments
 };
-AttnPlan attn_plan(const tq_attn_desc &desc);
+AttnPlan attn_plan(const tq_attn_desc &desc, const TqConsts &kc, const TqConsts &vc);
 size_t attn_partials_bytes(const tq_attn_desc &desc, const AttnPlan &plan, int d);
 cudaError_t launch_attend(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc,
                           const AttnPlan &plan, const float *qr, const float *p, float *partials,
                           float *out, cudaStream_t st);
+// attend_mma.cu
+bool attn_fast_eligible(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc);
+int attn_fast_chunk(const tq_attn_desc &desc);
+size_t attn_fast_extra_bytes(const TqConsts &kc, const tq_attn_desc &desc);
+cudaError_t launch_attend_fast(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc,
+                               const AttnPlan &plan, const float *qr, const float *p, void *extra,
+                               float *partials, cudaStream_t st);
 
 // Search: per-(query tile, shard) top-k candidates, then a per-query merge.
 struct SearchPlan {

@@ -27,7 +27,10 @@ class TqError(RuntimeError):
 
 
 class Spec(ctypes.Structure):
-    _fields_ = [("d", c_int32), ("mse_bits", c_int32), ("qjl_m", c_int32)]
+    _fields_ = [("d", c_int32), ("mse_bits", c_int32), ("qjl_m", c_int32), ("layout", c_int32)]
+
+
+LAYOUT_ROWS, LAYOUT_BLOCK16 = 0, 1
 
 
 class PackedC(ctypes.Structure):
@@ -130,7 +133,8 @@ def make_codebook(d: int, bits: int):
 class Context:
     """Quantizer constants for one tensor role, resident on one device."""
 
-    def __init__(self, d: int, mse_bits: int, qjl_m: int, rot_signs, qjl_matrix=None, device: int = 0):
+    def __init__(self, d: int, mse_bits: int, qjl_m: int, rot_signs, qjl_matrix=None, device: int = 0,
+                 layout: int = LAYOUT_ROWS):
         rs = torch.as_tensor(rot_signs).to(torch.int8).contiguous().cpu()
         if rs.numel() != d:
             raise ValueError("rot_signs must have d entries")
@@ -141,8 +145,8 @@ class Context:
             sptr = c_void_p(S.data_ptr())
         else:
             sptr = c_void_p(None)
-        self.d, self.mse_bits, self.qjl_m, self.device = d, mse_bits, qjl_m, device
-        spec = Spec(d, mse_bits, qjl_m)
+        self.d, self.mse_bits, self.qjl_m, self.device, self.layout = d, mse_bits, qjl_m, device, layout
+        spec = Spec(d, mse_bits, qjl_m, layout)
         h = c_void_p()
         _check(LIB.tq_ctx_create(ctypes.byref(spec), c_void_p(rs.data_ptr()), sptr, device, ctypes.byref(h)))
         self._h = h

@@ -124,3 +124,54 @@ def pack_signs(bits_) -> np.ndarray:
 def unpack_signs(buf, m: int) -> np.ndarray:
     buf = np.asarray(buf, dtype=np.uint8)
     return np.unpackbits(buf, axis=1, bitorder="little")[:, :m].astype(np.uint8)
+
+
+# ---------------------------------------------------------------- token-block layout for values
+# Reading (the pages only say "bit-packing"): for attention values the codes of 16 consecutive
+# slots may be stored token-transposed.  Block k = slots 16k..16k+15 owns 16 * code_bytes bytes,
+# read as little-endian 32-bit words W:
+#   W[q*d + j] (q < b//2):    bit t = bit 2q of code_j of slot 16k+t, bit 16+t = bit 2q+1
+#   W[(b//2)*d + j//2] (b odd): bit 16*(j%2) + t = bit b-1 of code_j of slot 16k+t
+def pack_codes_block16(codes, bits: int) -> np.ndarray:
+    """[n, d] codes (n a multiple of 16) -> [n, code_bytes] uint8 in the token-block layout."""
+    codes = np.asarray(codes, dtype=np.int64)
+    n, d = codes.shape
+    if n % 16:
+        raise ValueError("the token-block layout needs a multiple of 16 slots")
+    cb = code_bytes(d, bits)
+    nb = n // 16
+    words = np.zeros((nb, 16 * cb // 4), dtype=np.uint64)
+    blk = codes.reshape(nb, 16, d)                      # [block, token, j]
+    tok = np.arange(16, dtype=np.uint64)[None, :, None]
+    for q in range(bits // 2):
+        lo = ((blk >> (2 * q)) & 1).astype(np.uint64) << tok
+        hi = ((blk >> (2 * q + 1)) & 1).astype(np.uint64) << (tok + np.uint64(16))
+        words[:, q * d:(q + 1) * d] = np.bitwise_or.reduce(lo | hi, axis=1)
+    if bits % 2:
+        j = np.arange(d)
+        sh = (np.uint64(16) * (j % 2).astype(np.uint64))[None, None, :] + tok
+        v = ((blk >> (bits - 1)) & 1).astype(np.uint64) << sh           # [block, token, j]
+        per_j = np.bitwise_or.reduce(v, axis=1)                         # [block, j]
+        base = (bits // 2) * d
+        words[:, base:base + d // 2] = per_j[:, 0::2] | per_j[:, 1::2]
+    return words.astype(np.uint32).view(np.uint8).reshape(n, cb)
+
+
+def unpack_codes_block16(buf, d: int, bits: int) -> np.ndarray:
+    """[n, code_bytes] uint8 in the token-block layout -> [n, d] codes."""
+    buf = np.ascontiguousarray(np.asarray(buf, dtype=np.uint8))
+    n, cb = buf.shape
+    nb = n // 16
+    words = buf.reshape(nb, 16 * cb).view(np.uint32).astype(np.int64)   # [block, words]
+    tok = np.arange(16)[None, :, None]
+    codes = np.zeros((nb, 16, d), dtype=np.int64)
+    for q in range(bits // 2):
+        w = words[:, None, q * d:(q + 1) * d]
+        codes |= ((w >> tok) & 1) << (2 * q)
+        codes |= ((w >> (tok + 16)) & 1) << (2 * q + 1)
+    if bits % 2:
+        j = np.arange(d)
+        base = (bits // 2) * d
+        w = words[:, None, base + j // 2]                                 # [block, 1, j]
+        codes |= ((w >> (16 * (j % 2)[None, None, :] + tok)) & 1) << (bits - 1)
+    return codes.reshape(n, d)

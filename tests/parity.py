@@ -27,13 +27,13 @@ MAX_FLIP_FRACTION = 1e-4
 class Quantizer:
     """One tensor role: the seeded draws (D, S), the oracle codebook and the library context."""
 
-    def __init__(self, d, bits, m, seed, device=0):
+    def __init__(self, d, bits, m, seed, device=0, layout=0):
         from kv_cache_vector_06_b200 import tq
-        self.d, self.bits, self.m = d, bits, m
+        self.d, self.bits, self.m, self.layout = d, bits, m, layout
         self.D = synth.rotation_signs(d, seed)
         self.S = synth.qjl_matrix(m, d, seed + 1000)
         self.c, self.t = ocb.codebook(d, bits)
-        self.ctx = tq.Context(d, bits, m, self.D, self.S if m > 0 else None, device=device)
+        self.ctx = tq.Context(d, bits, m, self.D, self.S if m > 0 else None, device=device, layout=layout)
 
     @property
     def D64(self):
@@ -50,7 +50,11 @@ class Quantizer:
 def unpack(q: Quantizer, packed, rows=None):
     """Library packed arrays (torch, device) -> unpacked numpy (codes, bits, norm, rnorm)."""
     sel = slice(None) if rows is None else torch.as_tensor(rows, device=packed.codes.device)
-    codes = oenc.unpack_codes(packed.codes[sel].cpu().numpy(), q.d, q.bits)
+    if q.layout == 1:   # token-block layout: decode the whole array, then select the rows
+        allc = oenc.unpack_codes_block16(packed.codes.cpu().numpy(), q.d, q.bits)
+        codes = allc if rows is None else allc[np.asarray(torch.as_tensor(rows).cpu())]
+    else:
+        codes = oenc.unpack_codes(packed.codes[sel].cpu().numpy(), q.d, q.bits)
     norm = packed.norm[sel].double().cpu().numpy()
     if q.m > 0:
         bits = oenc.unpack_signs(packed.signs[sel].cpu().numpy(), q.m)

@@ -126,9 +126,9 @@ def test_scores_bf16_queries_and_small_d(tq):
         assert_scores_close(got, ref)
 
 
-def _attention_case(tq, d, kbits, km, vbits, batch, hkv, group, lens, paged, qdtype, seed):
+def _attention_case(tq, d, kbits, km, vbits, batch, hkv, group, lens, paged, qdtype, seed, vlayout=0):
     kq = Quantizer(d, kbits, km, seed=seed)
-    vq = Quantizer(d, vbits, 0, seed=seed + 50)
+    vq = Quantizer(d, vbits, 0, seed=seed + 50, layout=vlayout)
     hq = hkv * group
     maxlen = int(max(lens))
     blk = synth.BLOCK_TOKENS
@@ -138,6 +138,7 @@ def _attention_case(tq, d, kbits, km, vbits, batch, hkv, group, lens, paged, qdt
         cap = nblocks * hkv * blk
     else:
         table = None
+        maxlen = (maxlen + 15) // 16 * 16 if vlayout == 1 else maxlen
         cap = batch * hkv * maxlen
     K = synth.channel_scaled(batch, hkv, maxlen, d, seed=seed + 1)
     V = synth.channel_scaled(batch, hkv, maxlen, d, seed=seed + 2)
@@ -157,7 +158,7 @@ def _attention_case(tq, d, kbits, km, vbits, batch, hkv, group, lens, paged, qdt
     tq.encode_kv(kq.ctx, kx.cuda(), kp, slots=sl.cuda())
     tq.encode_kv(vq.ctx, vx.cuda(), vp, slots=sl.cuda())
     qx = synth.decode_queries(batch, hq, d, seed=seed + 3, dtype=qdtype)
-    out = tq.attend_decode(kq.ctx, vq.ctx, qx.cuda(), kp, vp, lens_t.cuda(), maxlen, n_kv_heads=hkv,
+    out = tq.attend_decode(kq.ctx, vq.ctx, qx.cuda(), kp, vp, lens_t.cuda(), int(max(lens)), n_kv_heads=hkv,
                            ctx_stride=maxlen, block_table=None if table is None else table.cuda(),
                            block_size=blk)
     torch.cuda.synchronize()
@@ -237,3 +238,69 @@ def test_search_k_edge_cases(tq):
             assert ss[r, a] >= ss[r, a + 1]
             if ss[r, a] == ss[r, a + 1]:
                 assert ii[r, a] < ii[r, a + 1]
+
+
+@pytest.mark.parametrize("d,bits", [(8, 1), (64, 2), (128, 3), (128, 4), (256, 2)])
+def test_encode_block16_layout(tq, d, bits):
+    """Values in the token-transposed 16-slot block layout, written at scattered slots (several
+    vectors share each block word, so concurrent writers must not clobber each other)."""
+    n, cap = 300, 512
+    q = Quantizer(d, bits, 0, seed=d + 7 * bits, layout=1)
+    x = torch.randn(n, d, generator=torch.Generator().manual_seed(d)) * 3
+    slots = torch.randperm(cap, generator=torch.Generator().manual_seed(bits))[:n].to(torch.int64)
+    packed = tq.Packed.allocate(q.ctx, cap)
+    packed.codes.fill_(0xA5)                        # stale bits must be cleared for written slots
+    tq.encode_kv(q.ctx, x.cuda(), packed, slots=slots.cuda())
+    torch.cuda.synchronize()
+    codes, sbits, norm, rnorm = unpack(q, packed, rows=slots)
+    compare_encode(q, q.oracle_encode(x.double().numpy()), codes, sbits, norm, rnorm)
+
+
+@pytest.mark.parametrize("vbits", [2, 3])
+def test_attention_block16_values_contiguous(tq, vbits):
+    _attention_case(tq, 128, 2, 128, vbits, batch=2, hkv=2, group=4, lens=[1500, 333], paged=False,
+                    qdtype=torch.bfloat16, seed=81 + vbits, vlayout=1)
+
+
+def test_attention_block16_values_paged(tq):
+    _attention_case(tq, 128, 3, 128, 3, batch=3, hkv=2, group=4, lens=[700, 16, 1031], paged=True,
+                    qdtype=torch.bfloat16, seed=91, vlayout=1)
+
+
+@pytest.mark.parametrize("kbits,km,vbits", [(1, 128, 2), (2, 128, 3), (3, 128, 3), (2, 0, 2), (3, 0, 3)])
+def test_attention_tensor_core_path_variants(tq, kbits, km, vbits):
+    """d = 128, 4 query heads per KV head, token-block values: the tensor-core path
+    (attend_mma.cu); ragged lengths, several 256-token chunks, a sequence shorter than one
+    block."""
+    _attention_case(tq, 128, kbits, km, vbits, batch=3, hkv=2, group=4, lens=[2600, 5, 777], paged=False,
+                    qdtype=torch.bfloat16, seed=101 + 10 * kbits + vbits, vlayout=1)
+
+
+def test_attention_tensor_core_path_paged_and_empty(tq):
+    out = _attention_case(tq, 128, 2, 128, 3, batch=4, hkv=3, group=4, lens=[0, 1, 1500, 33], paged=True,
+                          qdtype=torch.float32, seed=131, vlayout=1)
+    assert torch.all(out[0] == 0)
+
+
+def test_attention_tensor_core_path_matches_general_kernel(tq):
+    """Same packed K and V (bits identical), read once by the general CUDA-core kernel (row-major
+    values) and once by the tensor-core kernel (token-block values)."""
+    d, hkv, group, lens = 128, 2, 4, [3000, 1200]
+    kq = Quantizer(d, 2, d, seed=141)
+    v_rows = Quantizer(d, 3, 0, seed=142, layout=0)
+    v_blk = Quantizer(d, 3, 0, seed=142, layout=1)
+    maxlen = 3008
+    K = synth.channel_scaled(2, hkv, maxlen, d, seed=143).reshape(-1, d)
+    V = synth.channel_scaled(2, hkv, maxlen, d, seed=144).reshape(-1, d)
+    kp = tq.Packed.allocate(kq.ctx, K.shape[0])
+    vr = tq.Packed.allocate(v_rows.ctx, V.shape[0])
+    vb = tq.Packed.allocate(v_blk.ctx, V.shape[0])
+    tq.encode_kv(kq.ctx, K.cuda(), kp)
+    tq.encode_kv(v_rows.ctx, V.cuda(), vr)
+    tq.encode_kv(v_blk.ctx, V.cuda(), vb)
+    q = synth.decode_queries(2, hkv * group, d, seed=145).cuda()
+    lens_t = torch.tensor(lens, dtype=torch.int32).cuda()
+    o_gen = tq.attend_decode(kq.ctx, v_rows.ctx, q, kp, vr, lens_t, maxlen, n_kv_heads=hkv, ctx_stride=maxlen)
+    o_tc = tq.attend_decode(kq.ctx, v_blk.ctx, q, kp, vb, lens_t, maxlen, n_kv_heads=hkv, ctx_stride=maxlen)
+    torch.cuda.synchronize()
+    assert_attention_close(o_tc.cpu().numpy(), o_gen.cpu().numpy())

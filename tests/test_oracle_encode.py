@@ -140,3 +140,34 @@ def test_rotation_removes_outliers_before_quantization():
     assert np.max(np.abs(enc.y)) < 0.6
     u = x / np.linalg.norm(x, axis=1, keepdims=True)
     assert np.max(np.abs(u)) > 0.9
+
+
+def test_block16_layout_hand_example():
+    # d=8, b=3: 16 slots; slot 5 has code_2 = 6 (binary 110) and code_3 = 1, all others 0.
+    #   W[0*8 + 2]: plane 0 of j=2 is 0, plane 1 is 1 -> bit 16+5
+    #   W[0*8 + 3]: plane 0 of j=3 is 1 -> bit 5
+    #   plane 2 (odd last plane) of j=2 is 1 -> W[1*8 + 1], bit 16*0 + 5
+    codes = np.zeros((16, 8), dtype=np.int64)
+    codes[5, 2] = 6
+    codes[5, 3] = 1
+    buf = encode.pack_codes_block16(codes, 3)
+    assert buf.shape == (16, 16)
+    words = buf.reshape(-1).view(np.uint32)
+    expect = np.zeros(64, dtype=np.uint32)
+    expect[2] = 1 << 21
+    expect[3] = 1 << 5
+    expect[8 + 1] = 1 << 5
+    np.testing.assert_array_equal(words, expect)
+    np.testing.assert_array_equal(encode.unpack_codes_block16(buf, 8, 3), codes)
+
+
+@pytest.mark.parametrize("d,bits", [(8, 1), (8, 2), (16, 3), (128, 2), (128, 3), (128, 4), (64, 1)])
+def test_block16_round_trip_and_size(d, bits):
+    rng = np.random.default_rng(d + bits)
+    codes = rng.integers(0, 1 << bits, size=(48, d))
+    buf = encode.pack_codes_block16(codes, bits)
+    assert buf.shape == (48, encode.code_bytes(d, bits))
+    np.testing.assert_array_equal(encode.unpack_codes_block16(buf, d, bits), codes)
+    # same information as the row layout: 16 * (b*d/8) meaningful bytes per block
+    used = 16 * bits * d // 8
+    assert np.all(buf.reshape(3, -1)[:, used:] == 0)
