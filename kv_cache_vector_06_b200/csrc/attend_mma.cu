@@ -17,7 +17,10 @@
 //  * Values are stored token-transposed (TQ_LAYOUT_BLOCK16): one 32-bit word = one coordinate of
 //    16 tokens in two planes, so (w >> t) & 0x01010101 gives four tokens of one coordinate, the
 //    A operand of an MMA that contracts over tokens.  B = the softmax weights times the value
-//    norms in 16-bit fixed point (two byte limbs), columns = 4 heads x 2 planes x 2 limbs.
+//    norms in unsigned 16-bit fixed point (two byte limbs) relative to the chunk's largest one,
+//    rounded with a deterministic dither so that the many sub-unit weights of a long tail are
+//    unbiased rather than all rounded down; columns = 4 heads x 2 planes x 2 limbs.  The
+//    codebook's constant term uses the same integer weights as the MMA.
 //  * Softmax is two-pass per chunk (all logits of the chunk, then one max per head), so every
 //    value product of the chunk shares one fixed-point scale and the int32 accumulators need no
 //    rescaling; splits are merged by attend_combine_kernel as for the general kernel.
@@ -49,6 +52,24 @@ __device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, 
       "{%0,%1,%2,%3};\n"
       : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_u8u8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Uniform value in [0, 1) from a 32-bit key (integer hash; deterministic dither for rounding).
+__device__ __forceinline__ float dither(uint32_t x) {
+  x ^= x >> 16;
+  x *= 0x7feb352du;
+  x ^= x >> 15;
+  x *= 0x846ca68bu;
+  x ^= x >> 16;
+  return (float)(x >> 8) * (1.0f / 16777216.0f);
 }
 
 __device__ __forceinline__ int64_t token_slot(const MmaArgs &a, int b, int h, int t) {
@@ -183,6 +204,7 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
   __shared__ uint4 vfrag[NBLK][32];    // value-side B fragments per 16-token block
   __shared__ float red[kWarps][3 * kG];
   __shared__ float hstat[5][kG];       // max logit, sum w, sum w*nu, fixed-point multiplier, its inverse
+  __shared__ int wsum16[kG];           // sum of the integer value weights of each head
 
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -317,8 +339,9 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
       a2 = fmaxf(a2, red[w][2 * kG + g]);
     }
     int e = 0;
-    frexpf(a2, &e);  // a2 < 2^e
-    const int F = a2 > 0.f ? 14 - e : 0;
+    frexpf(a2, &e);  // a2 < 2^e, so a2 * 2^(15 - e) + 1 < 2^16
+    const int F = a2 > 0.f ? 15 - e : 0;
+    wsum16[g] = 0;
     hstat[1][g] = a0;
     hstat[2][g] = a1;
     hstat[3][g] = ldexpf(1.f, F);
@@ -330,20 +353,25 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
     // tokens t, t+8 (register 0) and t+4, t+12 (register 1); n-tile = limb.
     const int g = gid >> 1, ps = gid & 1;
     const float mul = hstat[3][g];
+    const uint32_t key0 = (uint32_t)((grp * a.splits + s) * CH) * 4u + (uint32_t)g;
+    int mine = 0;
     for (int kb = warp; kb < NBLK; kb += kWarps) {
       const float *wr = &lg[g][kb * 16];
-      int v[4] = {__float2int_rn(wr[t] * mul), __float2int_rn(wr[t + 8] * mul),
-                  __float2int_rn(wr[t + 4] * mul), __float2int_rn(wr[t + 12] * mul)};
-      uint32_t lo[4], hi[4];
+      const int toks[4] = {t, t + 8, t + 4, t + 12};
+      uint32_t v[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        lo[i] = (uint32_t)(next_limb(v[i]) & 255);
-        hi[i] = (uint32_t)(next_limb(v[i]) & 255);
+        const uint32_t key = key0 + 4u * (uint32_t)(kb * 16 + toks[i]);
+        v[i] = (uint32_t)__float2int_rd(fmaf(wr[toks[i]], mul, dither(key)));
       }
+      if (ps == 0) mine += (int)(v[0] + v[1] + v[2] + v[3]);
       const int sh = 16 * ps;
-      vfrag[kb][lane] = make_uint4((lo[0] | (lo[1] << 8)) << sh, (lo[2] | (lo[3] << 8)) << sh,
-                                   (hi[0] | (hi[1] << 8)) << sh, (hi[2] | (hi[3] << 8)) << sh);
+      vfrag[kb][lane] = make_uint4(((v[0] & 255u) | ((v[1] & 255u) << 8)) << sh,
+                                   ((v[2] & 255u) | ((v[3] & 255u) << 8)) << sh,
+                                   ((v[0] >> 8) | ((v[1] >> 8) << 8)) << sh,
+                                   ((v[2] >> 8) | ((v[3] >> 8) << 8)) << sh);
     }
+    atomicAdd(&wsum16[g], mine);
   }
   __syncthreads();
 
@@ -381,13 +409,13 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
     for (int x = 0; x < VT; ++x) {
       const uint32_t a0 = (X[x][0] >> t) & 0x01010101u, a1 = (X[x][1] >> t) & 0x01010101u;
       const uint32_t a2 = (X[x][0] >> (t + 4)) & 0x01010101u, a3 = (X[x][1] >> (t + 4)) & 0x01010101u;
-      mma_u8s8(accv[x][0], a0, a1, a2, a3, fb.x, fb.y);
-      mma_u8s8(accv[x][1], a0, a1, a2, a3, fb.z, fb.w);
+      mma_u8u8(accv[x][0], a0, a1, a2, a3, fb.x, fb.y);
+      mma_u8u8(accv[x][1], a0, a1, a2, a3, fb.z, fb.w);
     }
   }
   // accv[x][limb][c]: c0/c1 = (coordinate j0, head t, plane lo/hi), c2/c3 = (j0 + 1, ...)
   const float inv = hstat[4][t];
-  const float csum = vc.plane_coef_sum * hstat[2][t];
+  const float csum = vc.plane_coef_sum * (float)wsum16[t];
   const int64_t pbase = (((int64_t)b * a.hq + (int64_t)h * kG + t) * a.splits + s) * (kD + 2);
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
@@ -399,7 +427,7 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
         const float D = (float)accv[x][0][2 * r + ps] + 256.f * (float)accv[x][1][2 * r + ps];
         v = fmaf(2.f * vc.plane_coef[2 * x + ps], D, v);
       }
-    part[pbase + 2 + j0 + r] = fmaf(v, inv, -csum);
+    part[pbase + 2 + j0 + r] = (v - csum) * inv;
   }
   if (threadIdx.x < kG) {
     const int64_t pb = (((int64_t)b * a.hq + (int64_t)h * kG + threadIdx.x) * a.splits + s) * (kD + 2);
