@@ -73,7 +73,7 @@ size_t query_prep_bytes(const tq_ctx *c, int64_t nq) {
 tq_status prep_queries(const tq_ctx *c, const void *q, tq_dtype dt, int64_t nq, float *qr, float *p,
                        cudaStream_t st) {
   cudaError_t e = launch_rotate(c->k, ROT_QUERY, q, dt, nq, c->spec.d, nullptr, 0, nullptr,
-                                nullptr, nullptr, qr, st);
+                                nullptr, nullptr, qr, st, nullptr);
   if (e != cudaSuccess) return tq_cuda_check(e, "query rotation launch");
   if (c->spec.qjl_m > 0) {
     e = launch_project(c->k, PROJ_DENSE, qr, nq, nullptr, 0, nullptr, p, st);
@@ -239,7 +239,8 @@ tq_status tq_encode_workspace_size(const tq_ctx *ctx, int64_t n, size_t *bytes) 
   if (!bytes) return tq_fail(TQ_EINVAL, "bytes is NULL");
   if (n < 0) return tq_fail(TQ_EINVAL, "n < 0");
   const int64_t rows = n < kEncodeChunk ? n : kEncodeChunk;
-  *bytes = ctx->spec.qjl_m > 0 ? (size_t)(rows * ctx->spec.d * 4) : 0;
+  const bool fused = n <= kFusedEncodeMaxRows && ctx->spec.d >= 128;
+  *bytes = (ctx->spec.qjl_m > 0 && !fused) ? (size_t)(rows * ctx->spec.d * 4) : 0;
   return TQ_OK;
 }
 
@@ -269,6 +270,13 @@ tq_status tq_encode_kv(const tq_ctx *ctx, const void *x, tq_dtype dtype, int64_t
   if (st != TQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool qjl = ctx->spec.qjl_m > 0;
+  if (qjl && n <= kFusedEncodeMaxRows && ctx->spec.d >= 128) {
+    // one launch: rotate, quantize, pack, project and pack the signs
+    cudaError_t e = launch_rotate(ctx->k, ROT_ENCODE, x, dtype, n, ld, slots, out.capacity,
+                                  static_cast<uint32_t *>(out.codes), out.norm, out.rnorm, nullptr, s,
+                                  static_cast<uint32_t *>(out.signs));
+    return tq_cuda_check(e, "fused encode launch");
+  }
   for (int64_t r0 = 0; r0 < n; r0 += kEncodeChunk) {
     const int64_t rows = (n - r0) < kEncodeChunk ? (n - r0) : kEncodeChunk;
     const char *xr = static_cast<const char *>(x) + r0 * ld * esz;
@@ -405,10 +413,12 @@ tq_status tq_attend_decode(const tq_ctx *kctx, const tq_ctx *vctx, const tq_attn
   float *qr = static_cast<float *>(ws);
   float *p = reinterpret_cast<float *>(static_cast<char *>(ws) + tq_align_up(nq * kctx->spec.d * 4, 256));
   float *part = reinterpret_cast<float *>(static_cast<char *>(ws) + query_prep_bytes(kctx, nq));
-  st = prep_queries(kctx, q, dtype, nq, qr, p, s);
-  if (st != TQ_OK) return st;
   const AttnPlan plan = attn_plan(*desc, kctx->k, vctx->k);
-  return tq_cuda_check(launch_attend(kctx->k, vctx->k, *desc, plan, qr, p, part, out, s),
+  if (!plan.fast) {  // the tensor-core path rotates and projects the queries itself
+    st = prep_queries(kctx, q, dtype, nq, qr, p, s);
+    if (st != TQ_OK) return st;
+  }
+  return tq_cuda_check(launch_attend(kctx->k, vctx->k, *desc, plan, q, (int)dtype, qr, p, part, out, s),
                        "attention launch");
 }
 

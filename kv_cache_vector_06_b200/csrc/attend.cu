@@ -178,28 +178,61 @@ attend_split_kernel(TqConsts kc, TqConsts vc, AttnArgs a, const float *__restric
   }
 }
 
-__global__ void __launch_bounds__(kAtThreads)
+constexpr int kCbThreads = 512;
+
+__device__ __forceinline__ float block_reduce(float v, float *red, bool is_max) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) {
+    const float o = __shfl_xor_sync(TQ_FULL_MASK, v, s);
+    v = is_max ? fmaxf(v, o) : v + o;
+  }
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float r = red[0];
+  for (int w = 1; w < nw; ++w) r = is_max ? fmaxf(r, red[w]) : r + red[w];
+  return r;
+}
+
+// Merge the split partials of one (sequence, query head) with their log-sum-exp weights, then
+// undo the rotation once: o = D_V (1/sqrt d) H (sum_s e^{m_s - M} o~_s) / (sum_s e^{m_s - M} l_s).
+// 512 threads: the splits are summed in parallel by (coordinate, split group) pairs.
+__global__ void __launch_bounds__(kCbThreads)
 attend_combine_kernel(TqConsts vc, int splits, const float *__restrict__ part, float *__restrict__ out) {
   extern __shared__ float sm[];
   const int d = vc.d;
-  float *y = sm;            // [d]
-  float *f = sm + d;        // [splits] merge factors
+  const int ngroups = kCbThreads >= d ? kCbThreads / d : 1;
+  float *f = sm;                       // [splits]
+  float *y = f + splits;               // [d]
+  float *acc = y + d;                  // [ngroups][d]
+  float *red = acc + ngroups * d;      // [32]
   const int64_t bh = blockIdx.x;
   const float *pb = part + bh * splits * (d + 2);
-  float M = -INFINITY;
-  for (int s = 0; s < splits; ++s) M = fmaxf(M, pb[(int64_t)s * (d + 2)]);
+  float m = -INFINITY;
+  for (int s = threadIdx.x; s < splits; s += blockDim.x) m = fmaxf(m, pb[(int64_t)s * (d + 2)]);
+  const float M = block_reduce(m, red, true);
+  float l = 0.f;
   for (int s = threadIdx.x; s < splits; s += blockDim.x) {
     const float ms = pb[(int64_t)s * (d + 2)];
-    f[s] = (ms == -INFINITY) ? 0.f : __expf(ms - M);
+    const float fs = (ms == -INFINITY) ? 0.f : __expf(ms - M);
+    f[s] = fs;
+    l += pb[(int64_t)s * (d + 2) + 1] * fs;
+  }
+  const float L = block_reduce(l, red, false);  // its barriers also publish f[]
+  for (int idx = threadIdx.x; idx < ngroups * d; idx += blockDim.x) {
+    const int j = idx % d, g = idx / d;
+    float a = 0.f;
+#pragma unroll 4
+    for (int s = g; s < splits; s += ngroups) a = fmaf(pb[(int64_t)s * (d + 2) + 2 + j], f[s], a);
+    acc[g * d + j] = a;
   }
   __syncthreads();
-  float Lsum = 0.f;
-  for (int s = 0; s < splits; ++s) Lsum += pb[(int64_t)s * (d + 2) + 1] * f[s];
-  const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+  const float inv = L > 0.f ? 1.f / L : 0.f;
   for (int j = threadIdx.x; j < d; j += blockDim.x) {
-    float o = 0.f;
-    for (int s = 0; s < splits; ++s) o = fmaf(pb[(int64_t)s * (d + 2) + 2 + j], f[s], o);
-    y[j] = o * inv;
+    float a = 0.f;
+    for (int g = 0; g < ngroups; ++g) a += acc[g * d + j];
+    y[j] = a * inv;
   }
   __syncthreads();
   for (int hh = 1; hh < d; hh <<= 1) {
@@ -260,8 +293,8 @@ size_t attn_partials_bytes(const tq_attn_desc &desc, const AttnPlan &plan, int d
 }
 
 cudaError_t launch_attend(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc,
-                          const AttnPlan &plan, const float *qr, const float *p, float *partials,
-                          float *out, cudaStream_t st) {
+                          const AttnPlan &plan, const void *q, int dtype, const float *qr, const float *p,
+                          float *partials, float *out, cudaStream_t st) {
   if (desc.batch <= 0) return cudaSuccess;
   AttnArgs a;
   a.batch = desc.batch;
@@ -283,7 +316,7 @@ cudaError_t launch_attend(const TqConsts &kc, const TqConsts &vc, const tq_attn_
   if (plan.fast) {
     void *extra = reinterpret_cast<char *>(partials) +
                   tq_align_up((int64_t)sizeof(float) * desc.batch * desc.n_q_heads * plan.splits * (kc.d + 2), 256);
-    e = launch_attend_fast(kc, vc, desc, plan, qr, p, extra, partials, st);
+    e = launch_attend_fast(kc, vc, desc, plan, q, dtype, extra, partials, st);
     if (e != cudaSuccess) return e;
   } else switch (plan.group) {
     case 1: e = launch_split<1>(kc, vc, a, grid, qr, p, partials, st); break;
@@ -293,12 +326,13 @@ cudaError_t launch_attend(const TqConsts &kc, const TqConsts &vc, const tq_attn_
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
-  const size_t smem = sizeof(float) * ((size_t)vc.d + plan.splits);
+  const int ngroups = kCbThreads >= vc.d ? kCbThreads / vc.d : 1;
+  const size_t smem = sizeof(float) * ((size_t)plan.splits + vc.d + (size_t)ngroups * vc.d + 32);
   cudaError_t e2 = cudaFuncSetAttribute(attend_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)smem);
   if (e2 != cudaSuccess) return e2;
   tq_prof_begin(TQK_ATTEND_COMBINE, st);
-  attend_combine_kernel<<<(unsigned)((int64_t)desc.batch * desc.n_q_heads), kAtThreads, smem, st>>>(
+  attend_combine_kernel<<<(unsigned)((int64_t)desc.batch * desc.n_q_heads), kCbThreads, smem, st>>>(
       vc, plan.splits, partials, out);
   tq_prof_end(TQK_ATTEND_COMBINE, st);
   return cudaGetLastError();

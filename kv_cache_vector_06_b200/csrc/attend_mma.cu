@@ -62,14 +62,10 @@ __device__ __forceinline__ void mma_u8u8(int (&c)[4], uint32_t a0, uint32_t a1, 
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Uniform value in [0, 1) from a 32-bit key (integer hash; deterministic dither for rounding).
+// Uniform value in [0, 1) from a 32-bit key: the fractional part of key * (golden ratio), a
+// low-discrepancy sequence over consecutive keys (deterministic dither for rounding).
 __device__ __forceinline__ float dither(uint32_t x) {
-  x ^= x >> 16;
-  x *= 0x7feb352du;
-  x ^= x >> 15;
-  x *= 0x846ca68bu;
-  x ^= x >> 16;
-  return (float)(x >> 8) * (1.0f / 16777216.0f);
+  return (float)((x * 2654435769u) >> 8) * (1.0f / 16777216.0f);
 }
 
 __device__ __forceinline__ int64_t token_slot(const MmaArgs &a, int b, int h, int t) {
@@ -112,21 +108,61 @@ struct KPlanes {
 // |X| 2^F <= 2^30.  kconst: 2^-F_code, 2^-F_sign, (sum e_P) sum q', sum p per head.
 template <int BK, bool QJL>
 __global__ void __launch_bounds__(kThreads)
-kfrag_kernel(TqConsts kc, const float *__restrict__ qr, const float *__restrict__ p,
-             uint32_t *__restrict__ kfrag, float *__restrict__ kconst) {
+kfrag_kernel(TqConsts kc, const void *__restrict__ q, int dtype, uint32_t *__restrict__ kfrag,
+             float *__restrict__ kconst) {
   using KP = KPlanes<BK, QJL>;
+  __shared__ float qs[kG][kD];           // q', the rotated queries
   __shared__ float X[KP::all][kG][kD];
   __shared__ float red[kG][4];
   __shared__ int fexp[kG][2];
   const int grp = blockIdx.x;  // b * hkv + h; its query heads are rows grp * 4 + g
   const int tid = threadIdx.x;
+  // q' = (1/sqrt d) H (D q): load with the signs applied, then the butterflies in shared memory
   for (int i = tid; i < kG * kD; i += kThreads) {
     const int g = i / kD, j = i % kD;
-    const float q = qr[((int64_t)grp * kG + g) * kD + j];
+    const int64_t o = ((int64_t)grp * kG + g) * kD + j;
+    const float x = dtype == TQ_F32 ? static_cast<const float *>(q)[o]
+                                    : bf16_to_f32(static_cast<const uint16_t *>(q)[o]);
+    qs[g][j] = x * kc.signs[j];
+  }
+  __syncthreads();
+  for (int hh = 1; hh < kD; hh <<= 1) {
+    const int g = tid >> 6, i = tid & 63;  // 4 heads x 64 butterflies = 256 threads
+    const int lo = (i / hh) * 2 * hh + (i % hh);
+    const float a0 = qs[g][lo], b0 = qs[g][lo + hh];
+    __syncthreads();
+    qs[g][lo] = a0 + b0;
+    qs[g][lo + hh] = a0 - b0;
+    __syncthreads();
+  }
+  for (int i = tid; i < kG * kD; i += kThreads) {
+    const int g = i / kD, j = i % kD;
+    const float qv = qs[g][j] * kc.inv_sqrt_d;
+    qs[g][j] = qv;
 #pragma unroll
-    for (int P = 0; P < BK; ++P) X[P][g][j] = 2.f * kc.plane_coef[P] * q;
-    if constexpr (BK == 3) X[3][g][j] = 2.f * kc.plane_coef[3] * q;
-    if constexpr (QJL) X[KP::code][g][j] = 2.f * p[((int64_t)grp * kG + g) * kD + j];
+    for (int P = 0; P < BK; ++P) X[P][g][j] = 2.f * kc.plane_coef[P] * qv;
+    if constexpr (BK == 3) X[3][g][j] = 2.f * kc.plane_coef[3] * qv;
+  }
+  __syncthreads();
+  if constexpr (QJL) {
+    // p = S q' for the 4 heads: thread (row i, head pair) dots row i of S with two q'
+    const int i = tid & (kD - 1), gp = tid >> 7;
+    const float4 *Srow = reinterpret_cast<const float4 *>(kc.S + (int64_t)i * kD);
+    float p0 = 0.f, p1 = 0.f;
+#pragma unroll 8
+    for (int j4 = 0; j4 < kD / 4; ++j4) {
+      const float4 sv = Srow[j4];
+      p0 = fmaf(sv.x, qs[2 * gp][4 * j4], p0);
+      p0 = fmaf(sv.y, qs[2 * gp][4 * j4 + 1], p0);
+      p0 = fmaf(sv.z, qs[2 * gp][4 * j4 + 2], p0);
+      p0 = fmaf(sv.w, qs[2 * gp][4 * j4 + 3], p0);
+      p1 = fmaf(sv.x, qs[2 * gp + 1][4 * j4], p1);
+      p1 = fmaf(sv.y, qs[2 * gp + 1][4 * j4 + 1], p1);
+      p1 = fmaf(sv.z, qs[2 * gp + 1][4 * j4 + 2], p1);
+      p1 = fmaf(sv.w, qs[2 * gp + 1][4 * j4 + 3], p1);
+    }
+    X[KP::code][2 * gp][i] = 2.f * p0;
+    X[KP::code][2 * gp + 1][i] = 2.f * p1;
   }
   __syncthreads();
   const int warp = tid >> 5, lane = tid & 31;
@@ -140,7 +176,7 @@ kfrag_kernel(TqConsts kc, const float *__restrict__ qr, const float *__restrict_
         ms = fmaxf(ms, fabsf(X[KP::code][g][j]));
         sp += 0.5f * X[KP::code][g][j];
       }
-      sq += qr[((int64_t)grp * kG + g) * kD + j];
+      sq += qs[g][j];
     }
     mc = warp_max_f(mc);
     ms = warp_max_f(ms);
@@ -205,6 +241,8 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
   __shared__ float red[kWarps][3 * kG];
   __shared__ float hstat[5][kG];       // max logit, sum w, sum w*nu, fixed-point multiplier, its inverse
   __shared__ int wsum16[kG];           // sum of the integer value weights of each head
+  __shared__ int64_t vbase[NBLK];      // first value slot of each 16-token block, -1 if none
+  __shared__ float obuf[4][kG][kD];    // value sums of the 4 block groups
 
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -285,6 +323,10 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
         const int i = blk * 16 + gid + 8 * r;
         lg[t][i] = ok[r] ? a.scale * nu[r] * sc : -INFINITY;
         if (t == 0) sslot[i] = ok[r] ? slot[r] : -1;
+      }
+      if (lane == 0) {
+        int64_t base = tb < t1 ? token_slot(a, b, h, tb) : -1;  // a 16-slot block start
+        vbase[blk] = (base >= 0 && base < a.v.capacity) ? base : -1;
       }
     }
   }
@@ -376,58 +418,75 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
   __syncthreads();
 
   // ---------------------------------------------------------------- phase 3: value sum
-  // warp w owns coordinates 16 w .. 16 w + 15; row gid <-> coordinate 16 w + 2 gid, row gid + 8
-  // <-> 16 w + 2 gid + 1, so a thread's two rows are adjacent words.
-  const int j0 = warp * 16 + 2 * gid;
-  int accv[VT][2][4];
+  // warp w: coordinate half ch = w & 1 (64 coordinates = 4 m-tiles) and block group w >> 1
+  // (blocks kb = group, group + 4, ...).  In m-tile mt, row gid <-> coordinate
+  // 64 ch + 8 gid + 2 mt and row gid + 8 <-> the next one, so a thread's coordinates are the
+  // 8 consecutive words [64 ch + 8 gid, +8): two 16-byte loads per block (+ one for plane 2).
+  const int ch = warp & 1, bgrp = warp >> 1;
+  const int jb = 64 * ch + 8 * gid;
+  int accv[4][VT][2][4];
 #pragma unroll
-  for (int x = 0; x < VT; ++x)
-#pragma unroll
-    for (int y = 0; y < 2; ++y)
-#pragma unroll
-      for (int z = 0; z < 4; ++z) accv[x][y][z] = 0;
-#pragma unroll 2
-  for (int kb = 0; kb < NBLK; ++kb) {
-    const int tb = t0 + kb * 16;
-    if (tb >= t1) break;
-    const int64_t base = token_slot(a, b, h, tb);  // first slot of a 16-slot block
-    if (base < 0 || base >= a.v.capacity) continue;
-    const uint32_t *vb = vcodes + (base >> 4) * (int64_t)(16 * vc.code_words);
-    const uint2 A = *reinterpret_cast<const uint2 *>(vb + j0);
-    uint32_t X[VT][2];
-    X[0][0] = A.x;
-    X[0][1] = A.y;
-    if constexpr (BV == 3) {
-      const uint32_t hw = vb[kD + (j0 >> 1)];
-      const uint32_t p0 = (A.x ^ (A.x >> 16) ^ hw) & 0xffffu;
-      const uint32_t p1 = (A.y ^ (A.y >> 16) ^ (hw >> 16)) & 0xffffu;
-      X[VT - 1][0] = (hw & 0xffffu) | (p0 << 16);
-      X[VT - 1][1] = (hw >> 16) | (p1 << 16);
-    }
-    const uint4 fb = vfrag[kb][lane];
-#pragma unroll
-    for (int x = 0; x < VT; ++x) {
-      const uint32_t a0 = (X[x][0] >> t) & 0x01010101u, a1 = (X[x][1] >> t) & 0x01010101u;
-      const uint32_t a2 = (X[x][0] >> (t + 4)) & 0x01010101u, a3 = (X[x][1] >> (t + 4)) & 0x01010101u;
-      mma_u8u8(accv[x][0], a0, a1, a2, a3, fb.x, fb.y);
-      mma_u8u8(accv[x][1], a0, a1, a2, a3, fb.z, fb.w);
-    }
-  }
-  // accv[x][limb][c]: c0/c1 = (coordinate j0, head t, plane lo/hi), c2/c3 = (j0 + 1, ...)
-  const float inv = hstat[4][t];
-  const float csum = vc.plane_coef_sum * (float)wsum16[t];
-  const int64_t pbase = (((int64_t)b * a.hq + (int64_t)h * kG + t) * a.splits + s) * (kD + 2);
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    float v = 0.f;
+  for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
     for (int x = 0; x < VT; ++x)
 #pragma unroll
-      for (int ps = 0; ps < 2; ++ps) {
-        const float D = (float)accv[x][0][2 * r + ps] + 256.f * (float)accv[x][1][2 * r + ps];
-        v = fmaf(2.f * vc.plane_coef[2 * x + ps], D, v);
+      for (int y = 0; y < 2; ++y)
+#pragma unroll
+        for (int z = 0; z < 4; ++z) accv[mt][x][y][z] = 0;
+  for (int kb = bgrp; kb < NBLK; kb += 4) {
+    const int64_t base = vbase[kb];
+    if (base < 0) continue;
+    const uint32_t *vb = vcodes + (base >> 4) * (int64_t)(16 * vc.code_words);
+    const uint4 w0 = *reinterpret_cast<const uint4 *>(vb + jb);
+    const uint4 w1 = *reinterpret_cast<const uint4 *>(vb + jb + 4);
+    uint32_t X[VT][8];
+    X[0][0] = w0.x; X[0][1] = w0.y; X[0][2] = w0.z; X[0][3] = w0.w;
+    X[0][4] = w1.x; X[0][5] = w1.y; X[0][6] = w1.z; X[0][7] = w1.w;
+    if constexpr (BV == 3) {
+      const uint4 hw4 = *reinterpret_cast<const uint4 *>(vb + kD + (jb >> 1));
+      const uint32_t hw[4] = {hw4.x, hw4.y, hw4.z, hw4.w};
+#pragma unroll
+      for (int c2 = 0; c2 < 4; ++c2) {
+        const uint32_t a_lo = X[0][2 * c2], a_hi = X[0][2 * c2 + 1];
+        const uint32_t p0 = (a_lo ^ (a_lo >> 16) ^ hw[c2]) & 0xffffu;
+        const uint32_t p1 = (a_hi ^ (a_hi >> 16) ^ (hw[c2] >> 16)) & 0xffffu;
+        X[1][2 * c2] = (hw[c2] & 0xffffu) | (p0 << 16);
+        X[1][2 * c2 + 1] = (hw[c2] >> 16) | (p1 << 16);
       }
-    part[pbase + 2 + j0 + r] = (v - csum) * inv;
+    }
+    const uint4 fb = vfrag[kb][lane];
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+      for (int x = 0; x < VT; ++x) {
+        const uint32_t r0 = X[x][2 * mt], r1 = X[x][2 * mt + 1];
+        const uint32_t a0 = (r0 >> t) & 0x01010101u, a1 = (r1 >> t) & 0x01010101u;
+        const uint32_t a2 = (r0 >> (t + 4)) & 0x01010101u, a3 = (r1 >> (t + 4)) & 0x01010101u;
+        mma_u8u8(accv[mt][x][0], a0, a1, a2, a3, fb.x, fb.y);
+        mma_u8u8(accv[mt][x][1], a0, a1, a2, a3, fb.z, fb.w);
+      }
+  }
+  // accv[mt][x][limb][c]: c0/c1 = (coordinate jb + 2 mt, head t, plane lo/hi), c2/c3 = (+1, ...)
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      float v = 0.f;
+#pragma unroll
+      for (int x = 0; x < VT; ++x)
+#pragma unroll
+        for (int ps = 0; ps < 2; ++ps) {
+          const float D = (float)accv[mt][x][0][2 * r + ps] + 256.f * (float)accv[mt][x][1][2 * r + ps];
+          v = fmaf(2.f * vc.plane_coef[2 * x + ps], D, v);
+        }
+      obuf[bgrp][t][jb + 2 * mt + r] = v;
+    }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kG * kD; i += kThreads) {
+    const int g = i / kD, j = i % kD;
+    const float v = obuf[0][g][j] + obuf[1][g][j] + obuf[2][g][j] + obuf[3][g][j];
+    const int64_t pb = (((int64_t)b * a.hq + (int64_t)h * kG + g) * a.splits + s) * (kD + 2);
+    part[pb + 2 + j] = (v - vc.plane_coef_sum * (float)wsum16[g]) * hstat[4][g];
   }
   if (threadIdx.x < kG) {
     const int64_t pb = (((int64_t)b * a.hq + (int64_t)h * kG + threadIdx.x) * a.splits + s) * (kD + 2);
@@ -437,11 +496,11 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
 }
 
 template <int BK, int BV, bool QJL>
-cudaError_t launch_fast(const TqConsts &kc, const TqConsts &vc, const MmaArgs &a, int batch, const float *qr,
-                        const float *p, uint32_t *kfrag, float *kconst, float *part, cudaStream_t st) {
+cudaError_t launch_fast(const TqConsts &kc, const TqConsts &vc, const MmaArgs &a, int batch, const void *q,
+                        int dtype, uint32_t *kfrag, float *kconst, float *part, cudaStream_t st) {
   const unsigned groups = (unsigned)(batch * a.hkv);
   tq_prof_begin(TQK_ATTEND_FRAG, st);
-  kfrag_kernel<BK, QJL><<<groups, kThreads, 0, st>>>(kc, qr, p, kfrag, kconst);
+  kfrag_kernel<BK, QJL><<<groups, kThreads, 0, st>>>(kc, q, dtype, kfrag, kconst);
   tq_prof_end(TQK_ATTEND_FRAG, st);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -482,7 +541,7 @@ size_t attn_fast_extra_bytes(const TqConsts &kc, const tq_attn_desc &desc) {
 }
 
 cudaError_t launch_attend_fast(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc,
-                               const AttnPlan &plan, const float *qr, const float *p, void *extra,
+                               const AttnPlan &plan, const void *q, int dtype, void *extra,
                                float *partials, cudaStream_t st) {
   MmaArgs a;
   a.hq = desc.n_q_heads;
@@ -506,7 +565,7 @@ cudaError_t launch_attend_fast(const TqConsts &kc, const TqConsts &vc, const tq_
   const bool qjl = kc.m > 0;
 #define TQ_FAST(BKV, BVV, Q)                                                                           \
   if (kc.bits == BKV && vc.bits == BVV && qjl == Q)                                                    \
-    return launch_fast<BKV, BVV, Q>(kc, vc, a, desc.batch, qr, p, kfrag, kconst, partials, st);
+    return launch_fast<BKV, BVV, Q>(kc, vc, a, desc.batch, q, dtype, kfrag, kconst, partials, st);
   TQ_FAST(1, 2, true) TQ_FAST(2, 2, true) TQ_FAST(3, 2, true)
   TQ_FAST(1, 3, true) TQ_FAST(2, 3, true) TQ_FAST(3, 3, true)
   TQ_FAST(1, 2, false) TQ_FAST(2, 2, false) TQ_FAST(3, 2, false)

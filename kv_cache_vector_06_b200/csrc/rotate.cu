@@ -36,10 +36,12 @@ template <int D>
 __global__ void __launch_bounds__(kRotThreads)
 rotate_kernel(TqConsts c, int mode, const void *__restrict__ x, int dtype, int64_t n, int64_t ld,
               const int64_t *__restrict__ slots, int64_t capacity, uint32_t *__restrict__ codes,
-              float *__restrict__ norm, float *__restrict__ rnorm, float *__restrict__ resid) {
+              float *__restrict__ norm, float *__restrict__ rnorm, float *__restrict__ resid,
+              uint32_t *__restrict__ fsigns) {
   using Lay = RotLayout<D>;
   constexpr int LPV = Lay::LPV, VPW = Lay::VPW, KCH = Lay::KCH;
   __shared__ uint32_t stage[kRotThreads / 32][VPW][Lay::CW];
+  __shared__ float rbuf[kRotThreads / 32][D >= 128 ? D : 1];  // residual, fused projection
 
   const int lane = threadIdx.x & 31;
   const int wib = threadIdx.x >> 5;
@@ -205,6 +207,35 @@ rotate_kernel(TqConsts c, int mode, const void *__restrict__ x, int dtype, int64
       dst[i] = make_uint4(st[4 * i], st[4 * i + 1], st[4 * i + 2], st[4 * i + 3]);
     if (l == 0) norm[slot] = nu;
   }
+  if constexpr (D >= 128) {
+    if (fsigns != nullptr) {
+      // fused QJL projection for small batches: one vector per warp, z_i = <S_i, r> with the
+      // residual broadcast from shared memory, lane = output row within each group of 32
+      const float gamma = sqrtf(group_sum<LPV>(rr));
+      if (store && l == 0) rnorm[slot] = gamma;
+      float *rb = rbuf[wib];
+#pragma unroll
+      for (int k = 0; k < KCH; ++k)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) rb[4 * (l + LPV * k) + e] = v[k][e];
+      __syncwarp();
+      for (int w = 0; w < c.m / 32; ++w) {
+        const float4 *Srow = reinterpret_cast<const float4 *>(c.S + (int64_t)(32 * w + lane) * D);
+        float z = 0.f;
+#pragma unroll 8
+        for (int j4 = 0; j4 < D / 4; ++j4) {
+          const float4 sv = Srow[j4];
+          z = fmaf(sv.x, rb[4 * j4], z);
+          z = fmaf(sv.y, rb[4 * j4 + 1], z);
+          z = fmaf(sv.z, rb[4 * j4 + 2], z);
+          z = fmaf(sv.w, rb[4 * j4 + 3], z);
+        }
+        const unsigned bal = __ballot_sync(TQ_FULL_MASK, z >= 0.f);
+        if (store && lane == 0) fsigns[slot * c.sign_words + w] = bal;
+      }
+      return;
+    }
+  }
   if (resid != nullptr) {
     const float gamma = sqrtf(group_sum<LPV>(rr));
     if (store && l == 0) rnorm[slot] = gamma;
@@ -220,13 +251,13 @@ template <int D>
 cudaError_t launch_rotate_d(const TqConsts &c, RotateMode mode, const void *x, tq_dtype dtype,
                             int64_t n, int64_t ld, const int64_t *slots, int64_t capacity,
                             uint32_t *codes, float *norm, float *rnorm, float *resid,
-                            cudaStream_t st) {
+                            uint32_t *fsigns, cudaStream_t st) {
   constexpr int VPB = (kRotThreads / 32) * RotLayout<D>::VPW;  // vectors per block
   const int64_t blocks = (n + VPB - 1) / VPB;
   const int kind = mode == ROT_ENCODE ? TQK_ROTATE_ENCODE : TQK_ROTATE_QUERY;
   tq_prof_begin(kind, st);
   rotate_kernel<D><<<(unsigned)blocks, kRotThreads, 0, st>>>(c, (int)mode, x, (int)dtype, n, ld, slots,
-                                                             capacity, codes, norm, rnorm, resid);
+                                                             capacity, codes, norm, rnorm, resid, fsigns);
   tq_prof_end(kind, st);
   return cudaGetLastError();
 }
@@ -236,11 +267,11 @@ cudaError_t launch_rotate_d(const TqConsts &c, RotateMode mode, const void *x, t
 cudaError_t launch_rotate(const TqConsts &c, RotateMode mode, const void *x, tq_dtype dtype,
                           int64_t n, int64_t ld, const int64_t *slots, int64_t capacity,
                           uint32_t *codes, float *norm, float *rnorm, float *resid,
-                          cudaStream_t st) {
+                          cudaStream_t st, uint32_t *fsigns) {
   if (n <= 0) return cudaSuccess;
   switch (c.d) {
 #define TQ_ROT_CASE(DD) \
-  case DD: return launch_rotate_d<DD>(c, mode, x, dtype, n, ld, slots, capacity, codes, norm, rnorm, resid, st);
+  case DD: return launch_rotate_d<DD>(c, mode, x, dtype, n, ld, slots, capacity, codes, norm, rnorm, resid, fsigns, st);
     TQ_ROT_CASE(8) TQ_ROT_CASE(16) TQ_ROT_CASE(32) TQ_ROT_CASE(64)
     TQ_ROT_CASE(128) TQ_ROT_CASE(256) TQ_ROT_CASE(512) TQ_ROT_CASE(1024)
 #undef TQ_ROT_CASE

@@ -63,10 +63,14 @@ tq_status tq_codebook_fp64(int d, int bits, double *centroids, double *threshold
 // context has a QJL stage, the residual rows to `resid` and rnorm).  QUERY mode writes
 // q' = (1/sqrt d) H D q (no normalisation) to `resid` as fp32 [n][d].
 enum RotateMode { ROT_ENCODE = 0, ROT_QUERY = 1 };
+// With `fsigns` set (d >= 128, QJL context), the projection and sign packing run in the same
+// kernel (one vector per warp, S read from global memory): used for small batches such as the
+// per-step append; large batches use the tiled projection kernel.
 cudaError_t launch_rotate(const TqConsts &c, RotateMode mode, const void *x, tq_dtype dtype,
                           int64_t n, int64_t ld, const int64_t *slots, int64_t capacity,
                           uint32_t *codes, float *norm, float *rnorm, float *resid,
-                          cudaStream_t st);
+                          cudaStream_t st, uint32_t *fsigns = nullptr);
+constexpr int64_t kFusedEncodeMaxRows = 4096;
 
 // Z = R S^T for rows of R ([n][d] fp32).  SIGNS: pack bit = [z >= 0] into `signs` at the rows'
 // slots.  DENSE: write Z as fp32 [n][m] to `zout`.
@@ -90,14 +94,14 @@ struct AttnPlan {
 AttnPlan attn_plan(const tq_attn_desc &desc, const TqConsts &kc, const TqConsts &vc);
 size_t attn_partials_bytes(const tq_attn_desc &desc, const AttnPlan &plan, int d);
 cudaError_t launch_attend(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc,
-                          const AttnPlan &plan, const float *qr, const float *p, float *partials,
-                          float *out, cudaStream_t st);
+                          const AttnPlan &plan, const void *q, int dtype, const float *qr, const float *p,
+                          float *partials, float *out, cudaStream_t st);
 // attend_mma.cu
 bool attn_fast_eligible(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc);
 int attn_fast_chunk(const tq_attn_desc &desc);
 size_t attn_fast_extra_bytes(const TqConsts &kc, const tq_attn_desc &desc);
 cudaError_t launch_attend_fast(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc,
-                               const AttnPlan &plan, const float *qr, const float *p, void *extra,
+                               const AttnPlan &plan, const void *q, int dtype, void *extra,
                                float *partials, cudaStream_t st);
 
 // Search: per-(query tile, shard) top-k candidates, then a per-query merge.
