@@ -145,9 +145,13 @@ kfrag_kernel(TqConsts kc, const void *__restrict__ q, int dtype, uint32_t *__res
   }
   __syncthreads();
   if constexpr (QJL) {
-    // p = S q' for the 4 heads: thread (row i, head pair) dots row i of S with two q'
+    // p = S q' for the 4 heads: S staged in shared memory (row stride kD + 4), thread (row i,
+    // head pair) dots row i with two q'
+    extern __shared__ __align__(16) float sS[];
+    stage_rows_padded(sS, kc.S, kD, kD);
+    __syncthreads();
     const int i = tid & (kD - 1), gp = tid >> 7;
-    const float4 *Srow = reinterpret_cast<const float4 *>(kc.S + (int64_t)i * kD);
+    const float4 *Srow = reinterpret_cast<const float4 *>(sS + i * (kD + 4));
     float p0 = 0.f, p1 = 0.f;
 #pragma unroll 8
     for (int j4 = 0; j4 < kD / 4; ++j4) {
@@ -227,25 +231,65 @@ kfrag_kernel(TqConsts kc, const void *__restrict__ q, int dtype, uint32_t *__res
   }
 }
 
+// 16-byte asynchronous global -> shared copy (zero-fill when `ok` is false).
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool ok) {
+  const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
+  const int n = ok ? 16 : 0;
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(sa), "l"(gmem), "r"(n));
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
+}
+
+// Shared-memory carve-up of attend_mma_kernel (bytes).
+template <int BK, int BV, bool QJL, int CH>
+struct MmaSmem {
+  static constexpr int NBLK = CH / 16;
+  static constexpr int KCW = BK * 4;                // K code words per key
+  static constexpr int KSW = QJL ? 4 : 0;           // K sign words per key
+  static constexpr int VBW = BV * kD / 2;           // V words per 16-token block
+  static constexpr int X1W = BV == 3 ? kD : 0;      // (plane 2, parity) words per block
+  static constexpr size_t kc = 0;
+  static constexpr size_t ks = kc + (size_t)CH * KCW * 4;
+  static constexpr size_t kn = ks + (size_t)CH * KSW * 4;
+  static constexpr size_t kr = kn + (size_t)CH * 4;
+  static constexpr size_t vc = kr + (size_t)CH * 4;
+  static constexpr size_t vn = vc + (size_t)NBLK * VBW * 4;
+  static constexpr size_t x1 = vn + (size_t)CH * 4;
+  static constexpr size_t lg = x1 + (size_t)NBLK * X1W * 4;
+  static constexpr size_t vf = lg + (size_t)kG * CH * 4;
+  static constexpr size_t vb = vf + (size_t)NBLK * 32 * 16;
+  static constexpr size_t st = vb + (size_t)NBLK * 8;
+  static constexpr size_t total = st + 256;
+  static_assert((size_t)4 * kG * kD * 4 <= st, "the value-sum buffer reuses the staging area");
+};
+
 template <int BK, int BV, bool QJL, int CH>
 __global__ void __launch_bounds__(kThreads, 1)
 attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restrict__ kfrag,
                   const float *__restrict__ kconst, float *__restrict__ part) {
   using KP = KPlanes<BK, QJL>;
-  constexpr int NBLK = CH / 16;
+  using SM = MmaSmem<BK, BV, QJL, CH>;
+  constexpr int NBLK = SM::NBLK;
   constexpr int KB_PER_WARP = NBLK / kWarps;
   constexpr int VT = BV == 3 ? 2 : 1;  // value word types: (p0,p1) and (p2, parity)
-  __shared__ float lg[kG][CH];         // logits, then weights * value norms
-  __shared__ int64_t sslot[CH];        // slot of each chunk token, -1 if masked
-  __shared__ uint4 vfrag[NBLK][32];    // value-side B fragments per 16-token block
-  __shared__ float red[kWarps][3 * kG];
-  __shared__ float hstat[5][kG];       // max logit, sum w, sum w*nu, fixed-point multiplier, its inverse
-  __shared__ int wsum16[kG];           // sum of the integer value weights of each head
-  __shared__ int64_t vbase[NBLK];      // first value slot of each 16-token block, -1 if none
-  __shared__ float obuf[4][kG][kD];    // value sums of the 4 block groups
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint32_t *skc = reinterpret_cast<uint32_t *>(smem + SM::kc);
+  uint32_t *sks = reinterpret_cast<uint32_t *>(smem + SM::ks);
+  float *skn = reinterpret_cast<float *>(smem + SM::kn);
+  float *skr = reinterpret_cast<float *>(smem + SM::kr);
+  uint32_t *svc = reinterpret_cast<uint32_t *>(smem + SM::vc);
+  float *svn = reinterpret_cast<float *>(smem + SM::vn);
+  uint32_t *sx1 = reinterpret_cast<uint32_t *>(smem + SM::x1);
+  float *lg = reinterpret_cast<float *>(smem + SM::lg);          // [kG][CH] logits, then weights
+  uint4 *vfrag = reinterpret_cast<uint4 *>(smem + SM::vf);       // [NBLK][32]
+  int64_t *vbase = reinterpret_cast<int64_t *>(smem + SM::vb);   // [NBLK]
+  float *hstat = reinterpret_cast<float *>(smem + SM::st);       // [4][kG]
+  int *wsum16 = reinterpret_cast<int *>(smem + SM::st) + 4 * kG; // [kG]
+  float *obuf = reinterpret_cast<float *>(smem + SM::kc);        // [4][kG][kD], after phase 3's loop
 
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gid = lane >> 2, t = lane & 3;
   int L = a.seq_lens[b];
   L = L < 0 ? 0 : (L > a.max_len ? a.max_len : L);
@@ -253,9 +297,56 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
   const int t1 = min(L, t0 + CH);
   const int64_t grp = (int64_t)b * a.hkv + h;
   const int64_t cap = min(a.k.capacity, a.v.capacity);
-  const uint32_t *kcodes = static_cast<const uint32_t *>(a.k.codes);
-  const uint32_t *ksigns = static_cast<const uint32_t *>(a.k.signs);
-  const uint32_t *vcodes = static_cast<const uint32_t *>(a.v.codes);
+
+  // ---------------------------------------------------------------- stage 0: the chunk into smem
+  if (tid < NBLK) {
+    const int tb = t0 + 16 * tid;
+    const int64_t base = tb < t1 ? token_slot(a, b, h, tb) : -1;  // a 16-slot block start
+    vbase[tid] = (base >= 0 && base + 16 <= cap) ? base : -1;
+  }
+  __syncthreads();
+  {
+    constexpr int GK = BK * 16, GS = QJL ? 16 : 0, GN = 4, GR = QJL ? 4 : 0, GV = BV * 16, GVN = 4;
+    constexpr int GB = GK + GS + GN + GR + GV + GVN;  // 16-byte granules per block
+    const char *kcodes = static_cast<const char *>(a.k.codes);
+    const char *ksigns = static_cast<const char *>(a.k.signs);
+    const char *knorm = reinterpret_cast<const char *>(a.k.norm);
+    const char *krnorm = reinterpret_cast<const char *>(a.k.rnorm);
+    const char *vcodes = static_cast<const char *>(a.v.codes);
+    const char *vnorm = reinterpret_cast<const char *>(a.v.norm);
+    for (int idx = tid; idx < NBLK * GB; idx += kThreads) {
+      const int kb = idx / GB;
+      int g = idx % GB;
+      const int64_t base = vbase[kb];
+      const bool ok = base >= 0;
+      const int64_t bs = ok ? base : 0;
+      char *dst;
+      const char *src;
+      if (g < GK) {
+        dst = reinterpret_cast<char *>(skc) + (size_t)kb * 16 * SM::KCW * 4 + 16 * g;
+        src = kcodes + bs * kc.code_words * 4 + 16 * g;
+      } else if ((g -= GK) < GS) {
+        dst = reinterpret_cast<char *>(sks) + (size_t)kb * 16 * SM::KSW * 4 + 16 * g;
+        src = ksigns + bs * kc.sign_words * 4 + 16 * g;
+      } else if ((g -= GS) < GN) {
+        dst = reinterpret_cast<char *>(skn) + (size_t)kb * 64 + 16 * g;
+        src = knorm + bs * 4 + 16 * g;
+      } else if ((g -= GN) < GR) {
+        dst = reinterpret_cast<char *>(skr) + (size_t)kb * 64 + 16 * g;
+        src = krnorm + bs * 4 + 16 * g;
+      } else if ((g -= GR) < GV) {
+        dst = reinterpret_cast<char *>(svc) + (size_t)kb * SM::VBW * 4 + 16 * g;
+        src = vcodes + (bs >> 4) * 16 * vc.code_words * 4 + 16 * g;
+      } else {
+        g -= GV;
+        dst = reinterpret_cast<char *>(svn) + (size_t)kb * 64 + 16 * g;
+        src = vnorm + bs * 4 + 16 * g;
+      }
+      cp_async16(dst, src, ok);
+    }
+    cp_async_wait_all();
+  }
+  __syncthreads();
 
   // ---------------------------------------------------------------- phase 1: logits (keys x heads)
   {
@@ -274,23 +365,16 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
 #pragma unroll 1
     for (int mb = 0; mb < KB_PER_WARP; ++mb) {
       const int blk = warp * KB_PER_WARP + mb;
-      const int tb = t0 + blk * 16;
       uint32_t w[2][KP::all];
-      float nu[2], gam[2];
       bool ok[2];
-      int64_t slot[2];
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
-        const int tok = tb + gid + 8 * r;
-        ok[r] = tok < t1;
-        slot[r] = ok[r] ? token_slot(a, b, h, tok) : -1;
-        ok[r] = ok[r] && slot[r] >= 0 && slot[r] < cap;
+        const int i = blk * 16 + gid + 8 * r;
+        ok[r] = vbase[blk] >= 0 && t0 + i < t1;
 #pragma unroll
-        for (int P = 0; P < BK; ++P) w[r][P] = ok[r] ? kcodes[slot[r] * kc.code_words + P * 4 + t] : 0u;
+        for (int P = 0; P < BK; ++P) w[r][P] = skc[i * SM::KCW + P * 4 + t];
         if constexpr (BK == 3) w[r][3] = w[r][0] ^ w[r][1] ^ w[r][2];
-        if constexpr (QJL) w[r][KP::code] = ok[r] ? ksigns[slot[r] * kc.sign_words + t] : 0u;
-        nu[r] = ok[r] ? a.k.norm[slot[r]] : 0.f;
-        gam[r] = (QJL && ok[r]) ? a.k.rnorm[slot[r]] : 0.f;
+        if constexpr (QJL) w[r][KP::code] = sks[i * SM::KSW + t];
       }
       int acc[2][2][4];
 #pragma unroll
@@ -312,21 +396,16 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
       }
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
+        const int i = blk * 16 + gid + 8 * r;
         const float dc = (float)acc[0][0][2 * r] + 256.f * (float)acc[0][0][2 * r + 1] +
                          65536.f * (float)acc[0][1][2 * r] + 16777216.f * (float)acc[0][1][2 * r + 1];
         float sc = fmaf(dc, cfc, -cq);
         if constexpr (QJL) {
           const float ds = (float)acc[1][0][2 * r] + 256.f * (float)acc[1][0][2 * r + 1] +
                            65536.f * (float)acc[1][1][2 * r] + 16777216.f * (float)acc[1][1][2 * r + 1];
-          sc = fmaf(kc.qjl_scale * gam[r], fmaf(ds, cfs, -cp), sc);
+          sc = fmaf(kc.qjl_scale * skr[i], fmaf(ds, cfs, -cp), sc);
         }
-        const int i = blk * 16 + gid + 8 * r;
-        lg[t][i] = ok[r] ? a.scale * nu[r] * sc : -INFINITY;
-        if (t == 0) sslot[i] = ok[r] ? slot[r] : -1;
-      }
-      if (lane == 0) {
-        int64_t base = tb < t1 ? token_slot(a, b, h, tb) : -1;  // a 16-slot block start
-        vbase[blk] = (base >= 0 && base < a.v.capacity) ? base : -1;
+        lg[t * CH + i] = ok[r] ? a.scale * skn[i] * sc : -INFINITY;
       }
     }
   }
@@ -334,71 +413,52 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
 
   // ---------------------------------------------------------------- phase 2: softmax weights
   if (warp < kG) {
+    // warp g: max logit, weights w = e^{l - max}, W = w * ||v||, sum w, max W for head g
+    const int g = warp;
     float mx = -INFINITY;
-    for (int i = lane; i < CH; i += 32) mx = fmaxf(mx, lg[warp][i]);
+    for (int i = lane; i < CH; i += 32) mx = fmaxf(mx, lg[g * CH + i]);
     mx = warp_max_f(mx);
-    if (lane == 0) hstat[0][warp] = mx;
-  }
-  __syncthreads();
-  {
-    float sw[kG], sW[kG], mW[kG];
-#pragma unroll
-    for (int g = 0; g < kG; ++g) sw[g] = sW[g] = mW[g] = 0.f;
-    for (int i = threadIdx.x; i < CH; i += kThreads) {
-      const int64_t sl = sslot[i];
-      const float nv = sl >= 0 ? a.v.norm[sl] : 0.f;
-#pragma unroll
-      for (int g = 0; g < kG; ++g) {
-        const float wgt = sl >= 0 ? __expf(lg[g][i] - hstat[0][g]) : 0.f;
-        const float W = wgt * nv;
-        lg[g][i] = W;
-        sw[g] += wgt;
-        sW[g] += W;
-        mW[g] = fmaxf(mW[g], fabsf(W));
-      }
+    float sw = 0.f, mW = 0.f;
+    for (int i = lane; i < CH; i += 32) {
+      const float l = lg[g * CH + i];
+      const float wgt = l == -INFINITY ? 0.f : __expf(l - mx);
+      const float W = wgt * svn[i];
+      lg[g * CH + i] = W;
+      sw += wgt;
+      mW = fmaxf(mW, W);
     }
-#pragma unroll
-    for (int g = 0; g < kG; ++g) {
-      sw[g] = warp_sum_f(sw[g]);
-      sW[g] = warp_sum_f(sW[g]);
-      mW[g] = warp_max_f(mW[g]);
+    sw = warp_sum_f(sw);
+    mW = warp_max_f(mW);
+    if (lane == 0) {
+      int e = 0;
+      frexpf(mW, &e);  // mW < 2^e, so mW * 2^(15 - e) + 1 < 2^16
+      const int F = mW > 0.f ? 15 - e : 0;
+      hstat[0 * kG + g] = mx;
+      hstat[1 * kG + g] = sw;
+      hstat[2 * kG + g] = ldexpf(1.f, F);
+      hstat[3 * kG + g] = ldexpf(1.f, -F);
+      wsum16[g] = 0;
     }
-    if (lane == 0)
-#pragma unroll
-      for (int g = 0; g < kG; ++g) {
-        red[warp][g] = sw[g];
-        red[warp][kG + g] = sW[g];
-        red[warp][2 * kG + g] = mW[g];
-      }
-  }
-  __syncthreads();
-  if (threadIdx.x < kG) {
-    const int g = threadIdx.x;
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f;
-    for (int w = 0; w < kWarps; ++w) {
-      a0 += red[w][g];
-      a1 += red[w][kG + g];
-      a2 = fmaxf(a2, red[w][2 * kG + g]);
+  } else if constexpr (BV == 3) {
+    // warps 4-7: (plane 2, parity) words, parity = p0 ^ p1 ^ p2, once per block and coordinate
+    for (int idx = tid - kG * 32; idx < NBLK * kD; idx += kThreads - kG * 32) {
+      const int kb = idx / kD, j = idx % kD;
+      const uint32_t A = svc[kb * SM::VBW + j];
+      const uint32_t hw = svc[kb * SM::VBW + kD + (j >> 1)] >> (16 * (j & 1));
+      const uint32_t par = (A ^ (A >> 16) ^ hw) & 0xffffu;
+      sx1[kb * SM::X1W + j] = (hw & 0xffffu) | (par << 16);
     }
-    int e = 0;
-    frexpf(a2, &e);  // a2 < 2^e, so a2 * 2^(15 - e) + 1 < 2^16
-    const int F = a2 > 0.f ? 15 - e : 0;
-    wsum16[g] = 0;
-    hstat[1][g] = a0;
-    hstat[2][g] = a1;
-    hstat[3][g] = ldexpf(1.f, F);
-    hstat[4][g] = ldexpf(1.f, -F);
   }
   __syncthreads();
   {
     // B fragments of the value MMAs: lane (gid, t) = column (head gid/2, plane gid&1) and
     // tokens t, t+8 (register 0) and t+4, t+12 (register 1); n-tile = limb.
     const int g = gid >> 1, ps = gid & 1;
-    const float mul = hstat[3][g];
+    const float mul = hstat[2 * kG + g];
     const uint32_t key0 = (uint32_t)((grp * a.splits + s) * CH) * 4u + (uint32_t)g;
     int mine = 0;
     for (int kb = warp; kb < NBLK; kb += kWarps) {
-      const float *wr = &lg[g][kb * 16];
+      const float *wr = &lg[g * CH + kb * 16];
       const int toks[4] = {t, t + 8, t + 4, t + 12};
       uint32_t v[4];
 #pragma unroll
@@ -408,20 +468,20 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
       }
       if (ps == 0) mine += (int)(v[0] + v[1] + v[2] + v[3]);
       const int sh = 16 * ps;
-      vfrag[kb][lane] = make_uint4(((v[0] & 255u) | ((v[1] & 255u) << 8)) << sh,
-                                   ((v[2] & 255u) | ((v[3] & 255u) << 8)) << sh,
-                                   ((v[0] >> 8) | ((v[1] >> 8) << 8)) << sh,
-                                   ((v[2] >> 8) | ((v[3] >> 8) << 8)) << sh);
+      vfrag[kb * 32 + lane] = make_uint4(((v[0] & 255u) | ((v[1] & 255u) << 8)) << sh,
+                                         ((v[2] & 255u) | ((v[3] & 255u) << 8)) << sh,
+                                         ((v[0] >> 8) | ((v[1] >> 8) << 8)) << sh,
+                                         ((v[2] >> 8) | ((v[3] >> 8) << 8)) << sh);
     }
-    atomicAdd(&wsum16[g], mine);
+    mine += __shfl_xor_sync(TQ_FULL_MASK, mine, 1);  // lanes t and t^1 share a head and plane
+    mine += __shfl_xor_sync(TQ_FULL_MASK, mine, 2);
+    if (t == 0 && ps == 0) atomicAdd(&wsum16[g], mine);
   }
   __syncthreads();
 
   // ---------------------------------------------------------------- phase 3: value sum
-  // warp w: coordinate half ch = w & 1 (64 coordinates = 4 m-tiles) and block group w >> 1
-  // (blocks kb = group, group + 4, ...).  In m-tile mt, row gid <-> coordinate
-  // 64 ch + 8 gid + 2 mt and row gid + 8 <-> the next one, so a thread's coordinates are the
-  // 8 consecutive words [64 ch + 8 gid, +8): two 16-byte loads per block (+ one for plane 2).
+  // warp w: coordinate half ch = w & 1 (64 coordinates = 4 m-tiles) and block group w >> 1.
+  // In m-tile mt, row gid <-> coordinate 64 ch + 8 gid + 2 mt and row gid + 8 <-> the next one.
   const int ch = warp & 1, bgrp = warp >> 1;
   const int jb = 64 * ch + 8 * gid;
   int accv[4][VT][2][4];
@@ -434,27 +494,21 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
 #pragma unroll
         for (int z = 0; z < 4; ++z) accv[mt][x][y][z] = 0;
   for (int kb = bgrp; kb < NBLK; kb += 4) {
-    const int64_t base = vbase[kb];
-    if (base < 0) continue;
-    const uint32_t *vb = vcodes + (base >> 4) * (int64_t)(16 * vc.code_words);
-    const uint4 w0 = *reinterpret_cast<const uint4 *>(vb + jb);
-    const uint4 w1 = *reinterpret_cast<const uint4 *>(vb + jb + 4);
+    if (vbase[kb] < 0) continue;
     uint32_t X[VT][8];
-    X[0][0] = w0.x; X[0][1] = w0.y; X[0][2] = w0.z; X[0][3] = w0.w;
-    X[0][4] = w1.x; X[0][5] = w1.y; X[0][6] = w1.z; X[0][7] = w1.w;
-    if constexpr (BV == 3) {
-      const uint4 hw4 = *reinterpret_cast<const uint4 *>(vb + kD + (jb >> 1));
-      const uint32_t hw[4] = {hw4.x, hw4.y, hw4.z, hw4.w};
-#pragma unroll
-      for (int c2 = 0; c2 < 4; ++c2) {
-        const uint32_t a_lo = X[0][2 * c2], a_hi = X[0][2 * c2 + 1];
-        const uint32_t p0 = (a_lo ^ (a_lo >> 16) ^ hw[c2]) & 0xffffu;
-        const uint32_t p1 = (a_hi ^ (a_hi >> 16) ^ (hw[c2] >> 16)) & 0xffffu;
-        X[1][2 * c2] = (hw[c2] & 0xffffu) | (p0 << 16);
-        X[1][2 * c2 + 1] = (hw[c2] >> 16) | (p1 << 16);
-      }
+    {
+      const uint4 u0 = *reinterpret_cast<const uint4 *>(svc + kb * SM::VBW + jb);
+      const uint4 u1 = *reinterpret_cast<const uint4 *>(svc + kb * SM::VBW + jb + 4);
+      X[0][0] = u0.x; X[0][1] = u0.y; X[0][2] = u0.z; X[0][3] = u0.w;
+      X[0][4] = u1.x; X[0][5] = u1.y; X[0][6] = u1.z; X[0][7] = u1.w;
     }
-    const uint4 fb = vfrag[kb][lane];
+    if constexpr (BV == 3) {
+      const uint4 u0 = *reinterpret_cast<const uint4 *>(sx1 + kb * SM::X1W + jb);
+      const uint4 u1 = *reinterpret_cast<const uint4 *>(sx1 + kb * SM::X1W + jb + 4);
+      X[VT - 1][0] = u0.x; X[VT - 1][1] = u0.y; X[VT - 1][2] = u0.z; X[VT - 1][3] = u0.w;
+      X[VT - 1][4] = u1.x; X[VT - 1][5] = u1.y; X[VT - 1][6] = u1.z; X[VT - 1][7] = u1.w;
+    }
+    const uint4 fb = vfrag[kb * 32 + lane];
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
@@ -467,6 +521,7 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
       }
   }
   // accv[mt][x][limb][c]: c0/c1 = (coordinate jb + 2 mt, head t, plane lo/hi), c2/c3 = (+1, ...)
+  __syncthreads();  // every warp is done with the staged data that obuf overwrites
 #pragma unroll
   for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
@@ -479,39 +534,54 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
           const float D = (float)accv[mt][x][0][2 * r + ps] + 256.f * (float)accv[mt][x][1][2 * r + ps];
           v = fmaf(2.f * vc.plane_coef[2 * x + ps], D, v);
         }
-      obuf[bgrp][t][jb + 2 * mt + r] = v;
+      obuf[(bgrp * kG + t) * kD + jb + 2 * mt + r] = v;
     }
   __syncthreads();
-  for (int i = threadIdx.x; i < kG * kD; i += kThreads) {
+  for (int i = tid; i < kG * kD; i += kThreads) {
     const int g = i / kD, j = i % kD;
-    const float v = obuf[0][g][j] + obuf[1][g][j] + obuf[2][g][j] + obuf[3][g][j];
+    const float v = obuf[(0 * kG + g) * kD + j] + obuf[(1 * kG + g) * kD + j] + obuf[(2 * kG + g) * kD + j] +
+                    obuf[(3 * kG + g) * kD + j];
     const int64_t pb = (((int64_t)b * a.hq + (int64_t)h * kG + g) * a.splits + s) * (kD + 2);
-    part[pb + 2 + j] = (v - vc.plane_coef_sum * (float)wsum16[g]) * hstat[4][g];
+    part[pb + 2 + j] = (v - vc.plane_coef_sum * (float)wsum16[g]) * hstat[3 * kG + g];
   }
-  if (threadIdx.x < kG) {
-    const int64_t pb = (((int64_t)b * a.hq + (int64_t)h * kG + threadIdx.x) * a.splits + s) * (kD + 2);
-    part[pb] = hstat[0][threadIdx.x];
-    part[pb + 1] = hstat[1][threadIdx.x];
+  if (tid < kG) {
+    const int64_t pb = (((int64_t)b * a.hq + (int64_t)h * kG + tid) * a.splits + s) * (kD + 2);
+    part[pb] = hstat[0 * kG + tid];
+    part[pb + 1] = hstat[1 * kG + tid];
   }
+}
+
+template <int BK, int BV, bool QJL, int CH>
+cudaError_t launch_mma(const TqConsts &kc, const TqConsts &vc, const MmaArgs &a, dim3 grid,
+                       const uint32_t *kfrag, const float *kconst, float *part, cudaStream_t st) {
+  const size_t smem = MmaSmem<BK, BV, QJL, CH>::total;
+  cudaError_t e = cudaFuncSetAttribute(attend_mma_kernel<BK, BV, QJL, CH>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  attend_mma_kernel<BK, BV, QJL, CH><<<grid, kThreads, smem, st>>>(kc, vc, a, kfrag, kconst, part);
+  return cudaGetLastError();
 }
 
 template <int BK, int BV, bool QJL>
 cudaError_t launch_fast(const TqConsts &kc, const TqConsts &vc, const MmaArgs &a, int batch, const void *q,
                         int dtype, uint32_t *kfrag, float *kconst, float *part, cudaStream_t st) {
   const unsigned groups = (unsigned)(batch * a.hkv);
+  const size_t fsm = QJL ? sizeof(float) * kD * (kD + 4) : 0;
+  if (fsm) {
+    cudaError_t e0 = cudaFuncSetAttribute(kfrag_kernel<BK, QJL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsm);
+    if (e0 != cudaSuccess) return e0;
+  }
   tq_prof_begin(TQK_ATTEND_FRAG, st);
-  kfrag_kernel<BK, QJL><<<groups, kThreads, 0, st>>>(kc, q, dtype, kfrag, kconst);
+  kfrag_kernel<BK, QJL><<<groups, kThreads, fsm, st>>>(kc, q, dtype, kfrag, kconst);
   tq_prof_end(TQK_ATTEND_FRAG, st);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)a.splits, (unsigned)a.hkv, (unsigned)batch);
   tq_prof_begin(TQK_ATTEND_SPLIT, st);
-  if (a.chunk == 512)
-    attend_mma_kernel<BK, BV, QJL, 512><<<grid, kThreads, 0, st>>>(kc, vc, a, kfrag, kconst, part);
-  else
-    attend_mma_kernel<BK, BV, QJL, 256><<<grid, kThreads, 0, st>>>(kc, vc, a, kfrag, kconst, part);
+  e = a.chunk == 512 ? launch_mma<BK, BV, QJL, 512>(kc, vc, a, grid, kfrag, kconst, part, st)
+                     : launch_mma<BK, BV, QJL, 256>(kc, vc, a, grid, kfrag, kconst, part, st);
   tq_prof_end(TQK_ATTEND_SPLIT, st);
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace

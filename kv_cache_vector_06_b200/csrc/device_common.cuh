@@ -132,6 +132,18 @@ __device__ __forceinline__ void warp_topk_insert(float &bs, int64_t &bi, int k, 
   }
 }
 
+// Copy a rows x cols fp32 row-major matrix (cols a multiple of 4) into shared memory with a row
+// stride of cols + 4 floats, so that 16-byte loads of one column chunk by 8 lanes on 8
+// consecutive rows fall in distinct banks.  Every thread of the block must call it.
+__device__ __forceinline__ void stage_rows_padded(float *dst, const float *__restrict__ src, int rows, int cols) {
+  const int c4 = cols >> 2;
+  for (int idx = threadIdx.x; idx < rows * c4; idx += blockDim.x) {
+    const int r = idx / c4, c = idx - r * c4;
+    *reinterpret_cast<float4 *>(dst + (size_t)r * (cols + 4) + 4 * c) =
+        *reinterpret_cast<const float4 *>(src + (size_t)r * cols + 4 * c);
+  }
+}
+
 __device__ __forceinline__ float bf16_to_f32(uint16_t h) {
   return __uint_as_float(((uint32_t)h) << 16);
 }

@@ -45,6 +45,13 @@ rotate_kernel(TqConsts c, int mode, const void *__restrict__ x, int dtype, int64
 
   const int lane = threadIdx.x & 31;
   const int wib = threadIdx.x >> 5;
+  // fused projection with S staged in shared memory (d = m = 128; row stride 132 floats)
+  extern __shared__ __align__(16) float sS[];
+  const bool staged = D == 128 && fsigns != nullptr && c.m == 128;
+  if (staged) {
+    stage_rows_padded(sS, c.S, 128, 128);
+    __syncthreads();
+  }
   const int g = lane / LPV;
   const int l = lane % LPV;
   const int64_t row = ((int64_t)blockIdx.x * (kRotThreads / 32) + wib) * VPW + g;
@@ -220,7 +227,8 @@ rotate_kernel(TqConsts c, int mode, const void *__restrict__ x, int dtype, int64
         for (int e = 0; e < 4; ++e) rb[4 * (l + LPV * k) + e] = v[k][e];
       __syncwarp();
       for (int w = 0; w < c.m / 32; ++w) {
-        const float4 *Srow = reinterpret_cast<const float4 *>(c.S + (int64_t)(32 * w + lane) * D);
+        const float4 *Srow = staged ? reinterpret_cast<const float4 *>(sS + (32 * w + lane) * (D + 4))
+                                    : reinterpret_cast<const float4 *>(c.S + (int64_t)(32 * w + lane) * D);
         float z = 0.f;
 #pragma unroll 8
         for (int j4 = 0; j4 < D / 4; ++j4) {
@@ -255,9 +263,14 @@ cudaError_t launch_rotate_d(const TqConsts &c, RotateMode mode, const void *x, t
   constexpr int VPB = (kRotThreads / 32) * RotLayout<D>::VPW;  // vectors per block
   const int64_t blocks = (n + VPB - 1) / VPB;
   const int kind = mode == ROT_ENCODE ? TQK_ROTATE_ENCODE : TQK_ROTATE_QUERY;
+  const size_t smem = (D == 128 && fsigns != nullptr && c.m == 128) ? sizeof(float) * 128 * 132 : 0;
+  if (smem) {
+    cudaError_t e0 = cudaFuncSetAttribute(rotate_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e0 != cudaSuccess) return e0;
+  }
   tq_prof_begin(kind, st);
-  rotate_kernel<D><<<(unsigned)blocks, kRotThreads, 0, st>>>(c, (int)mode, x, (int)dtype, n, ld, slots,
-                                                             capacity, codes, norm, rnorm, resid, fsigns);
+  rotate_kernel<D><<<(unsigned)blocks, kRotThreads, smem, st>>>(c, (int)mode, x, (int)dtype, n, ld, slots,
+                                                                capacity, codes, norm, rnorm, resid, fsigns);
   tq_prof_end(kind, st);
   return cudaGetLastError();
 }
