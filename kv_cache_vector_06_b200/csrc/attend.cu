@@ -222,10 +222,20 @@ attend_combine_kernel(TqConsts vc, int splits, const float *__restrict__ part, f
   const float L = block_reduce(l, red, false);  // its barriers also publish f[]
   for (int idx = threadIdx.x; idx < ngroups * d; idx += blockDim.x) {
     const int j = idx % d, g = idx / d;
-    float a = 0.f;
-#pragma unroll 4
-    for (int s = g; s < splits; s += ngroups) a = fmaf(pb[(int64_t)s * (d + 2) + 2 + j], f[s], a);
-    acc[g * d + j] = a;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    int s = g;
+    for (; s + 3 * ngroups < splits; s += 4 * ngroups) {  // four independent loads in flight
+      const float v0 = pb[(int64_t)s * (d + 2) + 2 + j];
+      const float v1 = pb[(int64_t)(s + ngroups) * (d + 2) + 2 + j];
+      const float v2 = pb[(int64_t)(s + 2 * ngroups) * (d + 2) + 2 + j];
+      const float v3 = pb[(int64_t)(s + 3 * ngroups) * (d + 2) + 2 + j];
+      a0 = fmaf(v0, f[s], a0);
+      a1 = fmaf(v1, f[s + ngroups], a1);
+      a2 = fmaf(v2, f[s + 2 * ngroups], a2);
+      a3 = fmaf(v3, f[s + 3 * ngroups], a3);
+    }
+    for (; s < splits; s += ngroups) a0 = fmaf(pb[(int64_t)s * (d + 2) + 2 + j], f[s], a0);
+    acc[g * d + j] = (a0 + a1) + (a2 + a3);
   }
   __syncthreads();
   const float inv = L > 0.f ? 1.f / L : 0.f;

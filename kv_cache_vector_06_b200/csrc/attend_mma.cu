@@ -306,43 +306,42 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
   }
   __syncthreads();
   {
-    constexpr int GK = BK * 16, GS = QJL ? 16 : 0, GN = 4, GR = QJL ? 4 : 0, GV = BV * 16, GVN = 4;
-    constexpr int GB = GK + GS + GN + GR + GV + GVN;  // 16-byte granules per block
+    // one loop per array; granules are 16 bytes, blocks are 16 consecutive slots
     const char *kcodes = static_cast<const char *>(a.k.codes);
-    const char *ksigns = static_cast<const char *>(a.k.signs);
-    const char *knorm = reinterpret_cast<const char *>(a.k.norm);
-    const char *krnorm = reinterpret_cast<const char *>(a.k.rnorm);
     const char *vcodes = static_cast<const char *>(a.v.codes);
-    const char *vnorm = reinterpret_cast<const char *>(a.v.norm);
-    for (int idx = tid; idx < NBLK * GB; idx += kThreads) {
-      const int kb = idx / GB;
-      int g = idx % GB;
+    constexpr int GK = BK * 16, GV = BV * 16;
+    for (int idx = tid; idx < NBLK * GK; idx += kThreads) {
+      const int kb = idx / GK, g = idx - kb * GK;
       const int64_t base = vbase[kb];
-      const bool ok = base >= 0;
-      const int64_t bs = ok ? base : 0;
-      char *dst;
-      const char *src;
-      if (g < GK) {
-        dst = reinterpret_cast<char *>(skc) + (size_t)kb * 16 * SM::KCW * 4 + 16 * g;
-        src = kcodes + bs * kc.code_words * 4 + 16 * g;
-      } else if ((g -= GK) < GS) {
-        dst = reinterpret_cast<char *>(sks) + (size_t)kb * 16 * SM::KSW * 4 + 16 * g;
-        src = ksigns + bs * kc.sign_words * 4 + 16 * g;
-      } else if ((g -= GS) < GN) {
-        dst = reinterpret_cast<char *>(skn) + (size_t)kb * 64 + 16 * g;
-        src = knorm + bs * 4 + 16 * g;
-      } else if ((g -= GN) < GR) {
-        dst = reinterpret_cast<char *>(skr) + (size_t)kb * 64 + 16 * g;
-        src = krnorm + bs * 4 + 16 * g;
-      } else if ((g -= GR) < GV) {
-        dst = reinterpret_cast<char *>(svc) + (size_t)kb * SM::VBW * 4 + 16 * g;
-        src = vcodes + (bs >> 4) * 16 * vc.code_words * 4 + 16 * g;
-      } else {
-        g -= GV;
-        dst = reinterpret_cast<char *>(svn) + (size_t)kb * 64 + 16 * g;
-        src = vnorm + bs * 4 + 16 * g;
+      cp_async16(reinterpret_cast<char *>(skc) + (size_t)idx * 16,
+                 kcodes + (base >= 0 ? base : 0) * (SM::KCW * 4) + 16 * g, base >= 0);
+    }
+    for (int idx = tid; idx < NBLK * GV; idx += kThreads) {
+      const int kb = idx / GV, g = idx - kb * GV;
+      const int64_t base = vbase[kb];
+      cp_async16(reinterpret_cast<char *>(svc) + (size_t)idx * 16,
+                 vcodes + ((base >= 0 ? base : 0) >> 4) * (SM::VBW * 4) + 16 * g, base >= 0);
+    }
+    if constexpr (QJL) {
+      const char *ksigns = static_cast<const char *>(a.k.signs);
+      for (int idx = tid; idx < NBLK * 16; idx += kThreads) {
+        const int kb = idx >> 4, g = idx & 15;
+        const int64_t base = vbase[kb];
+        cp_async16(reinterpret_cast<char *>(sks) + (size_t)idx * 16,
+                   ksigns + (base >= 0 ? base : 0) * 16 + 16 * g, base >= 0);
       }
-      cp_async16(dst, src, ok);
+    }
+    {
+      // norms: 4 granules per block for ||k||, ||v|| (and gamma with QJL)
+      constexpr int NA = QJL ? 3 : 2;
+      for (int idx = tid; idx < NBLK * 4 * NA; idx += kThreads) {
+        const int arr = idx / (NBLK * 4), rem = idx - arr * (NBLK * 4);
+        const int kb = rem >> 2, g = rem & 3;
+        const int64_t base = vbase[kb];
+        const float *src = arr == 0 ? a.k.norm : (arr == 1 ? a.v.norm : a.k.rnorm);
+        float *dst = arr == 0 ? skn : (arr == 1 ? svn : skr);
+        cp_async16(dst + rem * 4, src + (base >= 0 ? base : 0) + 4 * g, base >= 0);
+      }
     }
     cp_async_wait_all();
   }
@@ -598,10 +597,12 @@ bool attn_fast_eligible(const TqConsts &kc, const TqConsts &vc, const tq_attn_de
 }
 
 int attn_fast_chunk(const tq_attn_desc &desc) {
+  // 512-token chunks halve the per-CTA fixed work and the partials to merge; 256 only when
+  // 512 would leave fewer than two CTAs per SM
   const int64_t rows = (int64_t)desc.batch * desc.n_kv_heads;
   const int maxlen = desc.max_seq_len > 0 ? desc.max_seq_len : 1;
   const int64_t ctas512 = rows * ((maxlen + 511) / 512);
-  return ctas512 >= 8 * 148 ? 512 : 256;
+  return ctas512 >= 2 * 148 ? 512 : 256;
 }
 
 size_t attn_fast_extra_bytes(const TqConsts &kc, const tq_attn_desc &desc) {

@@ -137,10 +137,26 @@ __device__ __forceinline__ void warp_topk_insert(float &bs, int64_t &bi, int k, 
 // consecutive rows fall in distinct banks.  Every thread of the block must call it.
 __device__ __forceinline__ void stage_rows_padded(float *dst, const float *__restrict__ src, int rows, int cols) {
   const int c4 = cols >> 2;
-  for (int idx = threadIdx.x; idx < rows * c4; idx += blockDim.x) {
-    const int r = idx / c4, c = idx - r * c4;
-    *reinterpret_cast<float4 *>(dst + (size_t)r * (cols + 4) + 4 * c) =
-        *reinterpret_cast<const float4 *>(src + (size_t)r * cols + 4 * c);
+  const int total = rows * c4;
+  // eight independent 16-byte loads in flight per thread before any store
+  for (int base = threadIdx.x; base < total; base += 8 * blockDim.x) {
+    float4 v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int idx = base + k * blockDim.x;
+      if (idx < total) {
+        const int r = idx / c4, c = idx - r * c4;
+        v[k] = *reinterpret_cast<const float4 *>(src + (size_t)r * cols + 4 * c);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int idx = base + k * blockDim.x;
+      if (idx < total) {
+        const int r = idx / c4, c = idx - r * c4;
+        *reinterpret_cast<float4 *>(dst + (size_t)r * (cols + 4) + 4 * c) = v[k];
+      }
+    }
   }
 }
 

@@ -50,9 +50,16 @@ class Quantizer:
 def unpack(q: Quantizer, packed, rows=None):
     """Library packed arrays (torch, device) -> unpacked numpy (codes, bits, norm, rnorm)."""
     sel = slice(None) if rows is None else torch.as_tensor(rows, device=packed.codes.device)
-    if q.layout == 1:   # token-block layout: decode the whole array, then select the rows
-        allc = oenc.unpack_codes_block16(packed.codes.cpu().numpy(), q.d, q.bits)
-        codes = allc if rows is None else allc[np.asarray(torch.as_tensor(rows).cpu())]
+    if q.layout == 1:   # token-block layout: decode the 16-slot blocks that hold the rows
+        cb = packed.codes.shape[1]
+        if rows is None:
+            codes = oenc.unpack_codes_block16(packed.codes.cpu().numpy(), q.d, q.bits)
+        else:
+            r = np.asarray(torch.as_tensor(rows).cpu()).astype(np.int64)
+            blocks = np.unique(r // 16)
+            blk = packed.codes.view(-1, 16, cb)[torch.as_tensor(blocks, device=packed.codes.device)]
+            dec = oenc.unpack_codes_block16(blk.reshape(-1, cb).cpu().numpy(), q.d, q.bits)
+            codes = dec[np.searchsorted(blocks, r // 16) * 16 + r % 16]
     else:
         codes = oenc.unpack_codes(packed.codes[sel].cpu().numpy(), q.d, q.bits)
     norm = packed.norm[sel].double().cpu().numpy()
@@ -127,3 +134,19 @@ def oracle_cache(q: Quantizer, codes, bits, norm, rnorm):
 def oracle_scores_from_packed(q: Quantizer, queries64, codes, bits, norm, rnorm):
     qr, p = oest.prepare_query(queries64, q.D64, q.S64)
     return oest.scores(qr, p, norm, codes, rnorm, bits, q.c)
+
+
+def oracle_heads(kq, vq, kp, vp, q, pairs, lens, slots_fn, group):
+    """Oracle attention output for sampled (sequence, query head) pairs, decoding only the slots of
+    each pair's KV head from the library's packed arrays.  q: torch [B, Hq, d]."""
+    out = {}
+    for b, hq in pairs:
+        h = hq // group
+        L = int(lens[b])
+        sl = np.asarray(slots_fn(b, h, L), dtype=np.int64)
+        kc = oracle_cache(kq, *unpack(kq, kp, rows=sl))
+        vc = oracle_cache(vq, *unpack(vq, vp, rows=sl))
+        r = oattn.attend_decode(q[b, hq][None, None].double().cpu().numpy(), kc, vc, [L], 1, kq.D64, kq.S64, kq.c,
+                                vq.D64, vq.c, ctx_stride=L)
+        out[(b, hq)] = r[0, 0]
+    return out
