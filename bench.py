@@ -206,22 +206,17 @@ class DecodeLayerBench:
         self.descs = [tq.make_attn_desc(self.kctx, self.vctx, (self.batch, self.hq, self.d), kp, vp, self.seq_lens,
                                         self.ctx, ctx_stride=self.ctx, n_kv_heads=self.hkv)
                       for kp, vp in self.layers]
-        self.ws_att = torch.empty(tq.attend_workspace_size(self.kctx, self.vctx, self.descs[0]), dtype=torch.uint8,
-                                  device=dev)
-        self.ws_new = torch.empty(max(1, tq.encode_workspace_size(self.kctx, self.hkv * self.batch)),
-                                  dtype=torch.uint8, device=dev)
+        self.ws_step = torch.empty(tq.decode_step_workspace_size(self.kctx, self.vctx, self.descs[0],
+                                                                 self.batch * self.hkv), dtype=torch.uint8, device=dev)
         self.keys_per_step = self.batch * self.hkv * self.ctx
         self.bytes_per_step = self.keys_per_step * (packed_bytes_per_key(self.d, self.kmse, self.m)
                                                     + packed_bytes_per_key(self.d, w["v_bits"], 0))
 
     def step(self, layer: int, q=None, out=None, k_new=None, v_new=None):
-        tq = self.tq
-        kp, vp = self.layers[layer]
-        tq.encode_kv(self.kctx, self.k_new if k_new is None else k_new, kp, slots=self.slots, ws=self.ws_new)
-        tq.encode_kv(self.vctx, self.v_new if v_new is None else v_new, vp, slots=self.slots, ws=self.ws_new)
-        tq.attend_decode(self.kctx, self.vctx, self.q if q is None else q, kp, vp, self.seq_lens, self.ctx,
-                         n_kv_heads=self.hkv, out=self.out if out is None else out, ws=self.ws_att,
-                         desc=self.descs[layer])
+        # one decode step of one layer: append the new K and V token of every KV head, attend
+        self.tq.decode_step(self.kctx, self.vctx, self.q if q is None else q, self.k_new if k_new is None else k_new,
+                            self.v_new if v_new is None else v_new, self.slots, self.descs[layer],
+                            out=self.out if out is None else out, ws=self.ws_step)
 
     def capture_graphs(self):
         import torch

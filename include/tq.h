@@ -188,6 +188,23 @@ tq_status tq_attend_decode(const tq_ctx *kctx, const tq_ctx *vctx, const tq_attn
                            const void *q, tq_dtype dtype, float *out, void *ws, size_t ws_bytes,
                            void *stream);
 
+/* One serving decode step: append the new token's key and value of every (sequence, KV head)
+ * to the compressed cache, then attend with the new queries (tq_encode_kv for K and for V, then
+ * tq_attend_decode, as one call).  With the tensor-core attention path the appends and the
+ * query preparation run in a single launch.
+ *   k_new, v_new  device [n_new][d] of kv_dtype, contiguous rows
+ *   new_slots     device int64 [n_new]: slot of each new row in desc->k and desc->v
+ *   desc          as for tq_attend_decode; desc->seq_lens must already count the new tokens
+ *   q, out        as for tq_attend_decode
+ *   ws            device workspace of tq_decode_step_workspace_size() bytes
+ * Errors: as tq_encode_kv and tq_attend_decode; TQ_EINVAL if n_new > 4096. */
+tq_status tq_decode_step_workspace_size(const tq_ctx *kctx, const tq_ctx *vctx, const tq_attn_desc *desc,
+                                        int64_t n_new, size_t *bytes);
+tq_status tq_decode_step(const tq_ctx *kctx, const tq_ctx *vctx, const tq_attn_desc *desc,
+                         const void *k_new, const void *v_new, tq_dtype kv_dtype, int64_t n_new,
+                         const int64_t *new_slots, const void *q, tq_dtype q_dtype, float *out,
+                         void *ws, size_t ws_bytes, void *stream);
+
 /* Allocation-free decode attention.  The pages have no counterpart: this entry point exists for
  * callers that cannot allocate device memory when they run attention, such as an inference
  * engine that gives all device memory to its own pool at start-up and forbids extensions from

@@ -422,6 +422,67 @@ tq_status tq_attend_decode(const tq_ctx *kctx, const tq_ctx *vctx, const tq_attn
                        "attention launch");
 }
 
+tq_status tq_decode_step_workspace_size(const tq_ctx *kctx, const tq_ctx *vctx, const tq_attn_desc *desc,
+                                        int64_t n_new, size_t *bytes) {
+  g_err[0] = 0;
+  if (!bytes) return tq_fail(TQ_EINVAL, "bytes is NULL");
+  if (n_new < 0 || n_new > kFusedEncodeMaxRows) return tq_fail(TQ_EINVAL, "n_new must be in [0, %lld]",
+                                                               (long long)kFusedEncodeMaxRows);
+  size_t att = 0, ek = 0, ev = 0;
+  tq_status st = tq_attend_workspace_size(kctx, vctx, desc, &att);
+  if (st != TQ_OK) return st;
+  tq_encode_workspace_size(kctx, n_new, &ek);
+  tq_encode_workspace_size(vctx, n_new, &ev);
+  *bytes = att + (size_t)tq_align_up((int64_t)(ek > ev ? ek : ev), 256);
+  return TQ_OK;
+}
+
+tq_status tq_decode_step(const tq_ctx *kctx, const tq_ctx *vctx, const tq_attn_desc *desc, const void *k_new,
+                         const void *v_new, tq_dtype kv_dtype, int64_t n_new, const int64_t *new_slots,
+                         const void *q, tq_dtype q_dtype, float *out, void *ws, size_t ws_bytes, void *stream) {
+  g_err[0] = 0;
+  size_t need = 0;
+  tq_status st = tq_decode_step_workspace_size(kctx, vctx, desc, n_new, &need);
+  if (st != TQ_OK) return st;
+  if (desc->batch == 0) return TQ_OK;
+  if (n_new > 0 && (!k_new || !v_new || !new_slots)) return tq_fail(TQ_EINVAL, "k_new/v_new/new_slots is NULL");
+  if (!q || !out) return tq_fail(TQ_EINVAL, "q/out is NULL");
+  if ((kv_dtype != TQ_F32 && kv_dtype != TQ_BF16) || (q_dtype != TQ_F32 && q_dtype != TQ_BF16))
+    return tq_fail(TQ_EINVAL, "unknown dtype");
+  if ((k_new && !aligned16(k_new)) || (v_new && !aligned16(v_new)) || !aligned16(q) || !aligned16(out))
+    return tq_fail(TQ_EINVAL, "k_new/v_new/q/out not 16-byte aligned");
+  if (new_slots && (reinterpret_cast<uintptr_t>(new_slots) & 7u)) return tq_fail(TQ_EINVAL, "new_slots not 8-byte aligned");
+  if (!ws || ws_bytes < need || !aligned16(ws))
+    return tq_fail(TQ_EINVAL, "workspace: %zu bytes (16-byte aligned) needed, %zu given", need, ws_bytes);
+  const AttnPlan plan = attn_plan(*desc, kctx->k, vctx->k);
+  const int esz = kv_dtype == TQ_F32 ? 4 : 2;
+  if (!plan.fast || (kctx->spec.d * esz) % 16 != 0) {
+    // general path: the three calls in order; the encode workspace follows the attention's
+    size_t att = 0;
+    tq_attend_workspace_size(kctx, vctx, desc, &att);
+    void *ews = static_cast<char *>(ws) + att;
+    const size_t eb = ws_bytes - att;
+    if (n_new > 0) {
+      st = tq_encode_kv(kctx, k_new, kv_dtype, n_new, kctx->spec.d, new_slots, desc->k, ews, eb, stream);
+      if (st != TQ_OK) return st;
+      st = tq_encode_kv(vctx, v_new, kv_dtype, n_new, vctx->spec.d, new_slots, desc->v, ews, eb, stream);
+      if (st != TQ_OK) return st;
+    }
+    return tq_attend_decode(kctx, vctx, desc, q, q_dtype, out, ws, att, stream);
+  }
+  st = set_device(kctx);
+  if (st != TQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t nq = (int64_t)desc->batch * desc->n_q_heads;
+  float *part = reinterpret_cast<float *>(static_cast<char *>(ws) + query_prep_bytes(kctx, nq));
+  void *extra = reinterpret_cast<char *>(part) +
+                tq_align_up((int64_t)sizeof(float) * desc->batch * desc->n_q_heads * plan.splits * (kctx->spec.d + 2), 256);
+  cudaError_t e = launch_decode_step_fast(kctx->k, vctx->k, *desc, plan, k_new, v_new, (int)kv_dtype, n_new, new_slots,
+                                          q, (int)q_dtype, extra, part, s);
+  if (e != cudaSuccess) return tq_cuda_check(e, "decode step launch");
+  return tq_cuda_check(launch_attend_combine(vctx->k, *desc, plan, part, out, s), "combine launch");
+}
+
 tq_status tq_search_workspace_size(const tq_ctx *ctx, int32_t nq, int64_t n, int32_t k, size_t *bytes) {
   g_err[0] = 0;
   tq_status st = check_ctx(ctx, "ctx");

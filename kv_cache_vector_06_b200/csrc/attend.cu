@@ -336,6 +336,11 @@ cudaError_t launch_attend(const TqConsts &kc, const TqConsts &vc, const tq_attn_
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
+  return launch_attend_combine(vc, desc, plan, partials, out, st);
+}
+
+cudaError_t launch_attend_combine(const TqConsts &vc, const tq_attn_desc &desc, const AttnPlan &plan,
+                                  const float *partials, float *out, cudaStream_t st) {
   const int ngroups = kCbThreads >= vc.d ? kCbThreads / vc.d : 1;
   const size_t smem = sizeof(float) * ((size_t)plan.splits + vc.d + (size_t)ngroups * vc.d + 32);
   cudaError_t e2 = cudaFuncSetAttribute(attend_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -28,6 +28,7 @@
 #include <cmath>
 
 #include "device_common.cuh"
+#include "rotate_device.cuh"
 
 namespace {
 
@@ -107,15 +108,15 @@ struct KPlanes {
 // X_P = 2 e_P q' (code planes, parity), 2 p (sign plane); F per head and part so that
 // |X| 2^F <= 2^30.  kconst: 2^-F_code, 2^-F_sign, (sum e_P) sum q', sum p per head.
 template <int BK, bool QJL>
-__global__ void __launch_bounds__(kThreads)
-kfrag_kernel(TqConsts kc, const void *__restrict__ q, int dtype, uint32_t *__restrict__ kfrag,
-             float *__restrict__ kconst) {
+__device__ __forceinline__ void kfrag_group(const TqConsts &kc, const void *__restrict__ q, int dtype,
+                                            uint32_t *__restrict__ kfrag, float *__restrict__ kconst, int grp,
+                                            float *sS) {
   using KP = KPlanes<BK, QJL>;
   __shared__ float qs[kG][kD];           // q', the rotated queries
   __shared__ float X[KP::all][kG][kD];
   __shared__ float red[kG][4];
   __shared__ int fexp[kG][2];
-  const int grp = blockIdx.x;  // b * hkv + h; its query heads are rows grp * 4 + g
+  // grp = b * hkv + h; its query heads are rows grp * 4 + g
   const int tid = threadIdx.x;
   // q' = (1/sqrt d) H (D q): load with the signs applied, then the butterflies in shared memory
   for (int i = tid; i < kG * kD; i += kThreads) {
@@ -147,7 +148,6 @@ kfrag_kernel(TqConsts kc, const void *__restrict__ q, int dtype, uint32_t *__res
   if constexpr (QJL) {
     // p = S q' for the 4 heads: S staged in shared memory (row stride kD + 4), thread (row i,
     // head pair) dots row i with two q'
-    extern __shared__ __align__(16) float sS[];
     stage_rows_padded(sS, kc.S, kD, kD);
     __syncthreads();
     const int i = tid & (kD - 1), gp = tid >> 7;
@@ -228,6 +228,37 @@ kfrag_kernel(TqConsts kc, const void *__restrict__ q, int dtype, uint32_t *__res
       word |= (uint32_t)(l & 255) << (8 * i);
     }
     out[idx] = word;
+  }
+}
+
+template <int BK, bool QJL>
+__global__ void __launch_bounds__(kThreads)
+kfrag_kernel(TqConsts kc, const void *__restrict__ q, int dtype, uint32_t *__restrict__ kfrag,
+             float *__restrict__ kconst) {
+  extern __shared__ __align__(16) float sS[];
+  kfrag_group<BK, QJL>(kc, q, dtype, kfrag, kconst, blockIdx.x, sS);
+}
+
+// One launch for the work that precedes the split kernel in a decode step: blocks
+// [0, nkb) append-encode the new keys (8 per block, fused QJL projection), blocks [nkb, nkb + nvb)
+// the new values, and the remaining blocks build one (sequence, KV head)'s query fragments.  The
+// three jobs are independent, so their latencies overlap instead of adding up.
+template <int BK, bool QJL>
+__global__ void __launch_bounds__(kThreads)
+decode_prep_kernel(TqConsts kc, TqConsts vc, const void *__restrict__ knew, const void *__restrict__ vnew,
+                   int kvdtype, int64_t nnew, const int64_t *__restrict__ slots, tq_packed kp, tq_packed vp,
+                   const void *__restrict__ q, int qdtype, uint32_t *__restrict__ kfrag,
+                   float *__restrict__ kconst, int nkb, int nvb) {
+  extern __shared__ __align__(16) float sS[];
+  const int bid = blockIdx.x;
+  if (bid < nkb) {
+    rotate_rows<kD>(kc, ROT_ENCODE, knew, kvdtype, nnew, kD, slots, kp.capacity, static_cast<uint32_t *>(kp.codes),
+                    kp.norm, kp.rnorm, nullptr, QJL ? static_cast<uint32_t *>(kp.signs) : nullptr, bid, sS);
+  } else if (bid < nkb + nvb) {
+    rotate_rows<kD>(vc, ROT_ENCODE, vnew, kvdtype, nnew, kD, slots, vp.capacity, static_cast<uint32_t *>(vp.codes),
+                    vp.norm, nullptr, nullptr, nullptr, bid - nkb, sS);
+  } else {
+    kfrag_group<BK, QJL>(kc, q, qdtype, kfrag, kconst, bid - nkb - nvb, sS);
   }
 }
 
@@ -642,5 +673,69 @@ cudaError_t launch_attend_fast(const TqConsts &kc, const TqConsts &vc, const tq_
   TQ_FAST(1, 2, false) TQ_FAST(2, 2, false) TQ_FAST(3, 2, false)
   TQ_FAST(1, 3, false) TQ_FAST(2, 3, false) TQ_FAST(3, 3, false)
 #undef TQ_FAST
+  return cudaErrorInvalidValue;
+}
+
+namespace {
+template <int BK, int BV, bool QJL>
+cudaError_t launch_step(const TqConsts &kc, const TqConsts &vc, const MmaArgs &a, int batch, const void *knew,
+                        const void *vnew, int kvdtype, int64_t nnew, const int64_t *slots, const void *q, int qdtype,
+                        uint32_t *kfrag, float *kconst, float *part, cudaStream_t st) {
+  const int nb = (int)((nnew + (kThreads / 32) - 1) / (kThreads / 32));  // one vector per warp (d = 128)
+  const unsigned grid0 = (unsigned)(2 * nb + batch * a.hkv);
+  const size_t fsm = QJL ? sizeof(float) * kD * (kD + 4) : 0;
+  if (fsm) {
+    cudaError_t e0 = cudaFuncSetAttribute(decode_prep_kernel<BK, QJL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)fsm);
+    if (e0 != cudaSuccess) return e0;
+  }
+  tq_prof_begin(TQK_DECODE_PREP, st);
+  decode_prep_kernel<BK, QJL><<<grid0, kThreads, fsm, st>>>(kc, vc, knew, vnew, kvdtype, nnew, slots, a.k, a.v, q,
+                                                            qdtype, kfrag, kconst, nb, nb);
+  tq_prof_end(TQK_DECODE_PREP, st);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)a.splits, (unsigned)a.hkv, (unsigned)batch);
+  tq_prof_begin(TQK_ATTEND_SPLIT, st);
+  e = a.chunk == 512 ? launch_mma<BK, BV, QJL, 512>(kc, vc, a, grid, kfrag, kconst, part, st)
+                     : launch_mma<BK, BV, QJL, 256>(kc, vc, a, grid, kfrag, kconst, part, st);
+  tq_prof_end(TQK_ATTEND_SPLIT, st);
+  return e;
+}
+}  // namespace
+
+cudaError_t launch_decode_step_fast(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc,
+                                    const AttnPlan &plan, const void *knew, const void *vnew, int kvdtype,
+                                    int64_t nnew, const int64_t *slots, const void *q, int qdtype, void *extra,
+                                    float *partials, cudaStream_t st) {
+  MmaArgs a;
+  a.hq = desc.n_q_heads;
+  a.hkv = desc.n_kv_heads;
+  a.max_len = desc.max_seq_len;
+  a.chunk = plan.chunk;
+  a.splits = plan.splits;
+  a.block_size = desc.block_size;
+  a.max_blocks = desc.max_blocks;
+  a.ctx_stride = desc.ctx_stride;
+  a.scale = desc.scale != 0.f ? desc.scale : kc.inv_sqrt_d;
+  a.seq_lens = desc.seq_lens;
+  a.block_table = desc.block_table;
+  a.k = desc.k;
+  a.v = desc.v;
+  const int planes = (kc.bits + (kc.bits == 3 ? 1 : 0)) + (kc.m > 0 ? 1 : 0);
+  const int64_t groups = (int64_t)desc.batch * desc.n_kv_heads;
+  uint32_t *kfrag = static_cast<uint32_t *>(extra);
+  float *kconst = reinterpret_cast<float *>(static_cast<char *>(extra) +
+                                            tq_align_up(groups * planes * 16 * 32 * 4, 256));
+  const bool qjl = kc.m > 0;
+#define TQ_STEP(BKV, BVV, Q)                                                                                   \
+  if (kc.bits == BKV && vc.bits == BVV && qjl == Q)                                                            \
+    return launch_step<BKV, BVV, Q>(kc, vc, a, desc.batch, knew, vnew, kvdtype, nnew, slots, q, qdtype, kfrag, \
+                                    kconst, partials, st);
+  TQ_STEP(1, 2, true) TQ_STEP(2, 2, true) TQ_STEP(3, 2, true)
+  TQ_STEP(1, 3, true) TQ_STEP(2, 3, true) TQ_STEP(3, 3, true)
+  TQ_STEP(1, 2, false) TQ_STEP(2, 2, false) TQ_STEP(3, 2, false)
+  TQ_STEP(1, 3, false) TQ_STEP(2, 3, false) TQ_STEP(3, 3, false)
+#undef TQ_STEP
   return cudaErrorInvalidValue;
 }

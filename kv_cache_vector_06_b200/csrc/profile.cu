@@ -10,7 +10,7 @@ namespace {
 
 const char *kNames[TQK_COUNT] = {"rotate_encode", "qjl_project", "rotate_query", "query_project", "scores",
                                  "attend_split", "attend_combine", "search_scan", "search_merge",
-                                 "attend_frag"};
+                                 "attend_frag", "decode_prep"};
 
 struct Pending {
   int kind;

@@ -50,7 +50,7 @@ tq_status tq_cuda_check(cudaError_t e, const char *what);
 // ---------------------------------------------------------------- profile.cu
 enum TqKernelKind {
   TQK_ROTATE_ENCODE = 0, TQK_QJL_PROJECT, TQK_ROTATE_QUERY, TQK_QUERY_PROJECT, TQK_SCORES,
-  TQK_ATTEND_SPLIT, TQK_ATTEND_COMBINE, TQK_SEARCH_SCAN, TQK_SEARCH_MERGE, TQK_ATTEND_FRAG, TQK_COUNT
+  TQK_ATTEND_SPLIT, TQK_ATTEND_COMBINE, TQK_SEARCH_SCAN, TQK_SEARCH_MERGE, TQK_ATTEND_FRAG, TQK_DECODE_PREP, TQK_COUNT
 };
 void tq_prof_begin(int kind, cudaStream_t st);
 void tq_prof_end(int kind, cudaStream_t st);
@@ -103,6 +103,14 @@ size_t attn_fast_extra_bytes(const TqConsts &kc, const tq_attn_desc &desc);
 cudaError_t launch_attend_fast(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc,
                                const AttnPlan &plan, const void *q, int dtype, void *extra,
                                float *partials, cudaStream_t st);
+// Fused decode step (tensor-core path): append-encode nnew K and V rows at `slots`, build the
+// query fragments, run the split kernel (the caller then launches the combine).
+cudaError_t launch_decode_step_fast(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc,
+                                    const AttnPlan &plan, const void *knew, const void *vnew, int kvdtype,
+                                    int64_t nnew, const int64_t *slots, const void *q, int qdtype, void *extra,
+                                    float *partials, cudaStream_t st);
+cudaError_t launch_attend_combine(const TqConsts &vc, const tq_attn_desc &desc, const AttnPlan &plan,
+                                  const float *partials, float *out, cudaStream_t st);
 
 // Search: per-(query tile, shard) top-k candidates, then a per-query merge.
 struct SearchPlan {

@@ -66,6 +66,9 @@ def _load():
                                   c_void_p, c_size_t, c_void_p]),
         "tq_attend_decode_noalloc": (st, [c_void_p, c_void_p, POINTER(AttnDesc), c_void_p, c_int, c_void_p,
                                           c_void_p]),
+        "tq_decode_step_workspace_size": (st, [c_void_p, c_void_p, POINTER(AttnDesc), c_int64, POINTER(c_size_t)]),
+        "tq_decode_step": (st, [c_void_p, c_void_p, POINTER(AttnDesc), c_void_p, c_void_p, c_int, c_int64, c_void_p,
+                                c_void_p, c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
         "tq_search_workspace_size": (st, [c_void_p, c_int32, c_int64, c_int32, POINTER(c_size_t)]),
         "tq_search_topk": (st, [c_void_p, c_void_p, c_int, c_int32, PackedC, c_int64, c_int32, c_void_p,
                                 c_void_p, c_void_p, c_size_t, c_void_p]),
@@ -313,6 +316,31 @@ def attend_decode(kctx: Context, vctx: Context, q: torch.Tensor, kcache: Packed,
     _check(LIB.tq_attend_decode(kctx.handle, vctx.handle, ctypes.byref(desc), _dev(q, kctx.device, "q"),
                                 _dtype_code(q), _dev(out, kctx.device, "out", torch.float32), w, wb,
                                 _stream_ptr(stream)))
+    return out
+
+
+def decode_step_workspace_size(kctx: Context, vctx: Context, desc: AttnDesc, n_new: int) -> int:
+    b = c_size_t()
+    _check(LIB.tq_decode_step_workspace_size(kctx.handle, vctx.handle, ctypes.byref(desc), n_new, ctypes.byref(b)))
+    return b.value
+
+
+def decode_step(kctx: Context, vctx: Context, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                new_slots: torch.Tensor, desc: AttnDesc, out=None, ws=None, stream=None):
+    """tq_decode_step: append k_new / v_new ([n_new, d]) at new_slots, then attend with q
+    ([batch, n_q_heads, d]); desc from make_attn_desc with seq_lens already counting the new tokens."""
+    if k_new.shape != v_new.shape or k_new.dim() != 2 or k_new.shape[1] != kctx.d or k_new.dtype != v_new.dtype:
+        raise ValueError(f"k_new and v_new must both be [n_new, {kctx.d}] with one dtype")
+    n_new = k_new.shape[0]
+    if new_slots.numel() != n_new:
+        raise ValueError("new_slots must have n_new entries")
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    w, wb = _workspace(decode_step_workspace_size(kctx, vctx, desc, n_new), kctx.device, ws)
+    _check(LIB.tq_decode_step(kctx.handle, vctx.handle, ctypes.byref(desc), _dev(k_new, kctx.device, "k_new"),
+                              _dev(v_new, kctx.device, "v_new"), _dtype_code(k_new), n_new,
+                              _dev(new_slots, kctx.device, "new_slots", torch.int64), _dev(q, kctx.device, "q"),
+                              _dtype_code(q), _dev(out, kctx.device, "out", torch.float32), w, wb, _stream_ptr(stream)))
     return out
 
 
