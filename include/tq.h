@@ -254,6 +254,15 @@ tq_status tq_profile_reset(void);
 tq_status tq_profile_read(int32_t index, char *name, int32_t name_len, int64_t *launches,
                           double *total_ms);
 
+/* Device-side status of the library on `device`: the TQ_DEVFLAG_* bits raised by kernels since
+ * the last clear.  Synchronizes the device first; clear != 0 resets the bits.  A kernel that
+ * gives up waiting for its own asynchronous copies (after about a second) raises
+ * TQ_DEVFLAG_STAGING_TIMEOUT and leaves its outputs unwritten.
+ *   flags  host out
+ * Errors: TQ_EINVAL (null flags), TQ_ECUDA. */
+#define TQ_DEVFLAG_STAGING_TIMEOUT 1
+tq_status tq_device_status(int32_t device, int32_t *flags, int32_t clear);
+
 /* Thread-local description of the last error on this thread ("" if none). */
 const char *tq_last_error(void);
 

@@ -180,6 +180,7 @@ tq_status tq_ctx_create(const tq_spec *spec, const int8_t *rot_signs, const floa
   k.fast_ok = 0;
   for (int i = 0; i < 4; ++i) k.plane_coef[i] = 0.f;
   k.plane_coef_sum = 0.f;
+  k.plane_coef_max = 0.f;
   if (spec->mse_bits <= 3) {
     const int b = spec->mse_bits;
     const int nsets = b == 3 ? 4 : b;
@@ -202,6 +203,7 @@ tq_status tq_ctx_create(const tq_spec *spec, const int8_t *rot_signs, const floa
     double sum = 0.0;
     for (int S = 0; S < nsets; ++S) {
       k.plane_coef[S] = (float)coef[S];
+      k.plane_coef_max = std::fmax(k.plane_coef_max, (float)coef[S]);
       sum += coef[S];
     }
     k.plane_coef_sum = (float)sum;

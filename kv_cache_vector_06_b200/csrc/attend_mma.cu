@@ -99,7 +99,7 @@ template <int BK, bool QJL>
 struct KPlanes {
   static constexpr int code = BK + (BK == 3 ? 1 : 0);  // code planes (+ parity plane for 3 bits)
   static constexpr int all = code + (QJL ? 1 : 0);     // + the QJL sign plane
-  static constexpr int regs = all * 4 * 2 * 2;          // planes x k-steps x n-tiles x regs
+  static constexpr int regs = all * 4 * 2 * 2;          // planes x k-steps x n-tiles x registers
 };
 
 // Query-side B fragments of the logit MMAs for one (sequence, KV head): for plane P, k-step s,
@@ -190,6 +190,7 @@ __device__ __forceinline__ void kfrag_group(const TqConsts &kc, const void *__re
       int ec = 0, es = 0;
       frexpf(mc, &ec);  // mc < 2^ec
       frexpf(ms, &es);
+      // |X| 2^F <= 2^30: four signed byte limbs
       fexp[g][0] = mc > 0.f ? 30 - ec : 0;
       fexp[g][1] = ms > 0.f ? 30 - es : 0;
       red[g][0] = ldexpf(1.f, -fexp[g][0]);
@@ -201,15 +202,13 @@ __device__ __forceinline__ void kfrag_group(const TqConsts &kc, const void *__re
   __syncthreads();
   if (tid < 16) kconst[(int64_t)grp * 16 + tid] = red[tid % 4][tid / 4];
   uint32_t *out = kfrag + (int64_t)grp * KP::regs * 32;
+  // layout [plane][k-step][lane][n-tile, register]: one 16-byte load per lane and k-step
   for (int idx = tid; idx < KP::regs * 32; idx += kThreads) {
-    const int ln = idx & 31;
-    int rest = idx >> 5;
-    const int r = rest & 1;
-    rest >>= 1;
-    const int nt = rest & 1;
-    rest >>= 1;
-    const int s = rest & 3;
-    const int P = rest >> 2;
+    const int r = idx & 1;
+    const int nt = (idx >> 1) & 1;
+    const int ln = (idx >> 2) & 31;
+    const int s = (idx >> 7) & 3;
+    const int P = idx >> 9;
     const int gid = ln >> 2, t = ln & 3;
     const int g = gid >> 1, limb = (gid & 1) + 2 * nt;
     const int shift = s + 4 * r;
@@ -262,333 +261,489 @@ decode_prep_kernel(TqConsts kc, TqConsts vc, const void *__restrict__ knew, cons
   }
 }
 
-// 16-byte asynchronous global -> shared copy (zero-fill when `ok` is false).
-__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool ok) {
-  const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
-  const int n = ok ? 16 : 0;
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(sa), "l"(gmem), "r"(n));
+// Device-side status word of the library (bits of tq_device_status): set by a kernel that gave up
+// waiting, read and cleared from the host by tq_device_status.
+__device__ int g_tq_device_flags;
+constexpr int kFlagStagingTimeout = 1;
+
+// Bulk asynchronous copies (global -> this CTA's shared memory) completing on an mbarrier, and
+// the bounded wait for them.  Addresses 16-byte aligned, sizes multiples of 16 bytes.
+// 32-bit multiply kept as such (an opaque multiplier: a power of two here, which would otherwise
+// become a shift on the integer ALU pipe).
+__device__ __forceinline__ uint32_t mul_lo(uint32_t x, uint32_t m) {
+  uint32_t r;
+  asm("mul.lo.u32 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(m));
+  return r;
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
+__device__ __forceinline__ unsigned smem_addr(const void *p) { return (unsigned)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void mbar_init(uint64_t *bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_arrive(uint64_t *bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, unsigned bytes, uint64_t *bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                   smem_addr(dst)),
+               "l"(src), "r"(bytes), "r"(smem_addr(bar))
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Wait for phase `parity` of `bar` to complete, giving up after about a second (each try_wait
+// suspends for a bounded, hardware-defined time).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, unsigned parity) {
+  for (int i = 0; i < (1 << 22); ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
 }
 
-// Shared-memory carve-up of attend_mma_kernel (bytes).
-template <int BK, int BV, bool QJL, int CH>
+constexpr int kSub = 256;          // tokens per sub-chunk (one staging buffer)
+constexpr int kSubBlk = kSub / 16;  // 16-token blocks per sub-chunk
+
+// Shared-memory carve-up of attend_mma_kernel (bytes): two staging buffers (the sub-chunk being
+// computed and the one being loaded), then the per-sub-chunk work arrays.
+template <int BK, int BV, bool QJL>
 struct MmaSmem {
-  static constexpr int NBLK = CH / 16;
-  static constexpr int KCW = BK * 4;                // K code words per key
-  static constexpr int KSW = QJL ? 4 : 0;           // K sign words per key
-  static constexpr int VBW = BV * kD / 2;           // V words per 16-token block
-  static constexpr int X1W = BV == 3 ? kD : 0;      // (plane 2, parity) words per block
+  static constexpr int NB = kSubBlk;
+  static constexpr int KCW = BK * 4;            // K code words per key
+  static constexpr int KSW = QJL ? 4 : 0;       // K sign words per key
+  static constexpr int VBW = BV * kD / 2;       // V words per 16-token block
+  static constexpr int X1W = BV == 3 ? kD : 0;  // (plane 2, parity) words per block
+  // offsets inside one staging buffer
   static constexpr size_t kc = 0;
-  static constexpr size_t ks = kc + (size_t)CH * KCW * 4;
-  static constexpr size_t kn = ks + (size_t)CH * KSW * 4;
-  static constexpr size_t kr = kn + (size_t)CH * 4;
-  static constexpr size_t vc = kr + (size_t)CH * 4;
-  static constexpr size_t vn = vc + (size_t)NBLK * VBW * 4;
-  static constexpr size_t x1 = vn + (size_t)CH * 4;
-  static constexpr size_t lg = x1 + (size_t)NBLK * X1W * 4;
-  static constexpr size_t vf = lg + (size_t)kG * CH * 4;
-  static constexpr size_t vb = vf + (size_t)NBLK * 32 * 16;
-  static constexpr size_t st = vb + (size_t)NBLK * 8;
-  static constexpr size_t total = st + 256;
-  static_assert((size_t)4 * kG * kD * 4 <= st, "the value-sum buffer reuses the staging area");
+  static constexpr size_t ks = kc + (size_t)kSub * KCW * 4;
+  static constexpr size_t kn = ks + (size_t)kSub * KSW * 4;
+  static constexpr size_t kr = kn + (size_t)kSub * 4;
+  static constexpr size_t vc = kr + (size_t)kSub * 4;
+  static constexpr size_t vn = vc + (size_t)NB * VBW * 4;
+  static constexpr size_t buf = vn + (size_t)kSub * 4;
+  // work arrays
+  static constexpr size_t x1 = 2 * buf;
+  static constexpr size_t lg = x1 + (size_t)NB * X1W * 4;
+  static constexpr size_t vf = lg + (size_t)kG * kSub * 4;
+  static constexpr size_t kf = vf + (size_t)NB * 32 * 16;
+  static constexpr size_t vb = kf + (size_t)KPlanes<BK, QJL>::regs * 32 * 4;
+  static constexpr size_t st = vb + (size_t)2 * NB * 8;
+  static constexpr size_t br = st + 16 * kG * 4;  // two mbarriers, one per staging buffer
+  static constexpr size_t total = br + 2 * 8 + 16;
+  static_assert((size_t)4 * kG * kD * 4 <= 2 * buf, "the value-sum buffer reuses the staging buffers");
+  static_assert(buf % 16 == 0 && x1 % 16 == 0 && kf % 16 == 0, "16-byte aligned regions");
 };
 
-template <int BK, int BV, bool QJL, int CH>
-__global__ void __launch_bounds__(kThreads, 1)
+// Issue the bulk copies of one sub-chunk (tokens [tk0, tk0 + kSub) of the CTA's (sequence, KV
+// head), blocks of 16 slots) into staging buffer `sb`, completing on `bar`.  Warp 0 runs it:
+// lane kb < 16 resolves block kb; the valid blocks (inside the sequence and the arrays) are one
+// contiguous run of slots in the contiguous layout (one copy per array) and one copy per array
+// and block when paged.  vb[kb] = first slot of block kb, or -1 (not copied; masked later).
+template <int BK, int BV, bool QJL>
+__device__ __forceinline__ void stage_sub(const MmaArgs &a, int b, int h, int tk0, int tend, int64_t cap,
+                                          unsigned char *sb, int64_t *vb, uint64_t *bar, unsigned extra_bytes) {
+  using SM = MmaSmem<BK, BV, QJL>;
+  constexpr unsigned KB = 16 * SM::KCW * 4, SB = QJL ? 16 * 16 : 0, VB = SM::VBW * 4, NBY = 16 * 4;
+  constexpr unsigned PER_BLOCK = KB + SB + VB + NBY * (QJL ? 3 : 2);
+  const int lane = threadIdx.x & 31;
+  int64_t base = -1;
+  if (lane < SM::NB) {
+    const int tb = tk0 + 16 * lane;
+    if (tb < tend) {
+      base = token_slot(a, b, h, tb);
+      if (base < 0 || base + 16 > cap) base = -1;
+      vb[lane] = base;
+    } else {
+      vb[lane] = -1;
+    }
+  }
+  const unsigned valid = __ballot_sync(TQ_FULL_MASK, base >= 0);
+  int nvalid = __popc(valid);
+  if (!a.block_table) {
+    // a block past the arrays ends the run: keep the leading valid blocks only
+    nvalid = __ffs(~valid) - 1;
+    if (lane < SM::NB && lane >= nvalid) vb[lane] = -1;
+  }
+  const char *kcodes = static_cast<const char *>(a.k.codes);
+  const char *vcodes = static_cast<const char *>(a.v.codes);
+  const char *ksigns = static_cast<const char *>(a.k.signs);
+  if (!a.block_table) {
+    // contiguous: the valid blocks are the first nvalid ones, consecutive in slot space
+    if (lane == 0) {
+      mbar_expect_arrive(bar, PER_BLOCK * (unsigned)nvalid + extra_bytes);
+      if (nvalid > 0) {
+        const int64_t s0 = base;
+        const unsigned n = (unsigned)nvalid;
+        bulk_g2s(sb + SM::kc, kcodes + s0 * (SM::KCW * 4), KB * n, bar);
+        bulk_g2s(sb + SM::vc, vcodes + (s0 >> 4) * (SM::VBW * 4), VB * n, bar);
+        if constexpr (QJL) bulk_g2s(sb + SM::ks, ksigns + s0 * 16, SB * n, bar);
+        bulk_g2s(sb + SM::kn, a.k.norm + s0, NBY * n, bar);
+        bulk_g2s(sb + SM::vn, a.v.norm + s0, NBY * n, bar);
+        if constexpr (QJL) bulk_g2s(sb + SM::kr, a.k.rnorm + s0, NBY * n, bar);
+      }
+    }
+  } else {
+    if (lane == 0) mbar_expect_arrive(bar, PER_BLOCK * (unsigned)nvalid + extra_bytes);
+    __syncwarp();
+    if (base >= 0) {
+      const int kb = lane;
+      bulk_g2s(sb + SM::kc + (size_t)kb * KB, kcodes + base * (SM::KCW * 4), KB, bar);
+      bulk_g2s(sb + SM::vc + (size_t)kb * VB, vcodes + (base >> 4) * (SM::VBW * 4), VB, bar);
+      if constexpr (QJL) bulk_g2s(sb + SM::ks + (size_t)kb * SB, ksigns + base * 16, SB, bar);
+      bulk_g2s(sb + SM::kn + (size_t)kb * NBY, a.k.norm + base, NBY, bar);
+      bulk_g2s(sb + SM::vn + (size_t)kb * NBY, a.v.norm + base, NBY, bar);
+      if constexpr (QJL) bulk_g2s(sb + SM::kr + (size_t)kb * NBY, a.k.rnorm + base, NBY, bar);
+    }
+  }
+}
+
+// One CTA = one (sequence, KV head) and a contiguous range of a.chunk tokens (a multiple of 16),
+// streamed in sub-chunks of kSub tokens: the next sub-chunk's bulk copies are in flight while
+// the current one is computed.  Softmax runs across sub-chunks with a running maximum: the value
+// sums of each sub-chunk use that sub-chunk's own fixed-point scale and are folded into fp32
+// accumulators rescaled by e^{M_old - M_new}.
+template <int BK, int BV, bool QJL>
+__global__ void __launch_bounds__(kThreads, 2)
 attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restrict__ kfrag,
                   const float *__restrict__ kconst, float *__restrict__ part) {
   using KP = KPlanes<BK, QJL>;
-  using SM = MmaSmem<BK, BV, QJL, CH>;
-  constexpr int NBLK = SM::NBLK;
-  constexpr int KB_PER_WARP = NBLK / kWarps;
+  using SM = MmaSmem<BK, BV, QJL>;
+  constexpr int NB = SM::NB;
   constexpr int VT = BV == 3 ? 2 : 1;  // value word types: (p0,p1) and (p2, parity)
   extern __shared__ __align__(16) unsigned char smem[];
-  uint32_t *skc = reinterpret_cast<uint32_t *>(smem + SM::kc);
-  uint32_t *sks = reinterpret_cast<uint32_t *>(smem + SM::ks);
-  float *skn = reinterpret_cast<float *>(smem + SM::kn);
-  float *skr = reinterpret_cast<float *>(smem + SM::kr);
-  uint32_t *svc = reinterpret_cast<uint32_t *>(smem + SM::vc);
-  float *svn = reinterpret_cast<float *>(smem + SM::vn);
   uint32_t *sx1 = reinterpret_cast<uint32_t *>(smem + SM::x1);
-  float *lg = reinterpret_cast<float *>(smem + SM::lg);          // [kG][CH] logits, then weights
-  uint4 *vfrag = reinterpret_cast<uint4 *>(smem + SM::vf);       // [NBLK][32]
-  int64_t *vbase = reinterpret_cast<int64_t *>(smem + SM::vb);   // [NBLK]
-  float *hstat = reinterpret_cast<float *>(smem + SM::st);       // [4][kG]
-  int *wsum16 = reinterpret_cast<int *>(smem + SM::st) + 4 * kG; // [kG]
-  float *obuf = reinterpret_cast<float *>(smem + SM::kc);        // [4][kG][kD], after phase 3's loop
+  float *lg = reinterpret_cast<float *>(smem + SM::lg);          // [kG][kSub] logits, then weights
+  uint4 *vfrag = reinterpret_cast<uint4 *>(smem + SM::vf);       // [NB][32]
+  const uint4 *kf4 = reinterpret_cast<const uint4 *>(smem + SM::kf);  // [plane][k-step][32]
+  int64_t *vbase = reinterpret_cast<int64_t *>(smem + SM::vb);   // [2][NB]
+  float *hM = reinterpret_cast<float *>(smem + SM::st);          // running max per head
+  float *hL = hM + kG;                                           // running sum of e^{l - M}
+  float *hScale = hL + kG;                                       // fixed-point scale of the weights
+  float *hInv = hScale + kG;                                     // 1 / (128 hScale)
+  float *hAlpha = hInv + kG;                                     // e^{M_old - M_new}
+  int *csum = reinterpret_cast<int *>(hAlpha + kG);              // sum of the integer weights X
+  float *obuf = reinterpret_cast<float *>(smem);                 // [4][kG][kD], after the loop
 
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gid = lane >> 2, t = lane & 3;
   int L = a.seq_lens[b];
   L = L < 0 ? 0 : (L > a.max_len ? a.max_len : L);
-  const int t0 = s * CH;
-  const int t1 = min(L, t0 + CH);
+  const int t0 = s * a.chunk;
+  const int t1 = min(L, t0 + a.chunk);
+  const int nsub = t1 > t0 ? (t1 - t0 + kSub - 1) / kSub : 0;
   const int64_t grp = (int64_t)b * a.hkv + h;
   const int64_t cap = min(a.k.capacity, a.v.capacity);
 
-  // ---------------------------------------------------------------- stage 0: the chunk into smem
-  if (tid < NBLK) {
-    const int tb = t0 + 16 * tid;
-    const int64_t base = tb < t1 ? token_slot(a, b, h, tb) : -1;  // a 16-slot block start
-    vbase[tid] = (base >= 0 && base + 16 <= cap) ? base : -1;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::br);
+  int *fail = reinterpret_cast<int *>(smem + SM::br + 16);
+  if (tid == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    *fail = 0;
+  }
+  if (tid < kG) {
+    hM[tid] = -INFINITY;
+    hL[tid] = 0.f;
   }
   __syncthreads();
-  {
-    // one loop per array; granules are 16 bytes, blocks are 16 consecutive slots
-    const char *kcodes = static_cast<const char *>(a.k.codes);
-    const char *vcodes = static_cast<const char *>(a.v.codes);
-    constexpr int GK = BK * 16, GV = BV * 16;
-    for (int idx = tid; idx < NBLK * GK; idx += kThreads) {
-      const int kb = idx / GK, g = idx - kb * GK;
-      const int64_t base = vbase[kb];
-      cp_async16(reinterpret_cast<char *>(skc) + (size_t)idx * 16,
-                 kcodes + (base >= 0 ? base : 0) * (SM::KCW * 4) + 16 * g, base >= 0);
-    }
-    for (int idx = tid; idx < NBLK * GV; idx += kThreads) {
-      const int kb = idx / GV, g = idx - kb * GV;
-      const int64_t base = vbase[kb];
-      cp_async16(reinterpret_cast<char *>(svc) + (size_t)idx * 16,
-                 vcodes + ((base >= 0 ? base : 0) >> 4) * (SM::VBW * 4) + 16 * g, base >= 0);
-    }
-    if constexpr (QJL) {
-      const char *ksigns = static_cast<const char *>(a.k.signs);
-      for (int idx = tid; idx < NBLK * 16; idx += kThreads) {
-        const int kb = idx >> 4, g = idx & 15;
-        const int64_t base = vbase[kb];
-        cp_async16(reinterpret_cast<char *>(sks) + (size_t)idx * 16,
-                   ksigns + (base >= 0 ? base : 0) * 16 + 16 * g, base >= 0);
-      }
-    }
-    {
-      // norms: 4 granules per block for ||k||, ||v|| (and gamma with QJL)
-      constexpr int NA = QJL ? 3 : 2;
-      for (int idx = tid; idx < NBLK * 4 * NA; idx += kThreads) {
-        const int arr = idx / (NBLK * 4), rem = idx - arr * (NBLK * 4);
-        const int kb = rem >> 2, g = rem & 3;
-        const int64_t base = vbase[kb];
-        const float *src = arr == 0 ? a.k.norm : (arr == 1 ? a.v.norm : a.k.rnorm);
-        float *dst = arr == 0 ? skn : (arr == 1 ? svn : skr);
-        cp_async16(dst + rem * 4, src + (base >= 0 ? base : 0) + 4 * g, base >= 0);
-      }
-    }
-    cp_async_wait_all();
+  if (warp == 0 && nsub > 0) {
+    // the first sub-chunk, and the query fragments (one copy per CTA) on the same barrier
+    constexpr unsigned FB = KP::regs * 32 * 4;
+    stage_sub<BK, BV, QJL>(a, b, h, t0, t1, cap, smem, vbase, &bars[0], FB);
+    if (lane == 0) bulk_g2s(smem + SM::kf, kfrag + grp * KP::regs * 32, FB, &bars[0]);
   }
-  __syncthreads();
+  const float cfc = kconst[grp * 16 + t], cfs = kconst[grp * 16 + 4 + t];
+  const float cq = kconst[grp * 16 + 8 + t], cp = kconst[grp * 16 + 12 + t];
 
-  // ---------------------------------------------------------------- phase 1: logits (keys x heads)
-  {
-    uint32_t kb[KP::all][4][2][2];
-    const uint32_t *fr = kfrag + grp * KP::regs * 32 + lane;
+  // value accumulators of this thread: head t, coordinates jb + 2 mt + r
+  const int ch = warp & 1, bgrp = warp >> 1;
+  const int jb = 64 * ch + 8 * gid;
+  float o[4][2];
 #pragma unroll
-    for (int P = 0; P < KP::all; ++P)
-#pragma unroll
-      for (int st = 0; st < 4; ++st)
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int r = 0; r < 2; ++r) kb[P][st][nt][r] = fr[((((P * 4 + st) * 2 + nt) * 2) + r) * 32];
-    const float cfc = kconst[grp * 16 + t], cfs = kconst[grp * 16 + 4 + t];
-    const float cq = kconst[grp * 16 + 8 + t], cp = kconst[grp * 16 + 12 + t];
-#pragma unroll 1
-    for (int mb = 0; mb < KB_PER_WARP; ++mb) {
-      const int blk = warp * KB_PER_WARP + mb;
-      uint32_t w[2][KP::all];
-      bool ok[2];
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int i = blk * 16 + gid + 8 * r;
-        ok[r] = vbase[blk] >= 0 && t0 + i < t1;
-#pragma unroll
-        for (int P = 0; P < BK; ++P) w[r][P] = skc[i * SM::KCW + P * 4 + t];
-        if constexpr (BK == 3) w[r][3] = w[r][0] ^ w[r][1] ^ w[r][2];
-        if constexpr (QJL) w[r][KP::code] = sks[i * SM::KSW + t];
+  for (int mt = 0; mt < 4; ++mt) o[mt][0] = o[mt][1] = 0.f;
+
+  for (int sc = 0; sc < nsub; ++sc) {
+    const int cur = sc & 1;
+    const int tk0 = t0 + sc * kSub;
+    if (warp == 0 && sc + 1 < nsub)
+      stage_sub<BK, BV, QJL>(a, b, h, tk0 + kSub, t1, cap, smem + (cur ^ 1) * SM::buf, vbase + (cur ^ 1) * NB,
+                             &bars[cur ^ 1], 0u);
+    if (!mbar_wait_bounded(&bars[cur], (unsigned)(sc >> 1) & 1u)) *fail = 1;
+    __syncthreads();
+    if (*fail) {
+      // the copies did not land in time: report, give the ones in flight a bounded time to
+      // finish (they write this CTA's shared memory), and leave without writing partials
+      if (tid == 0) {
+        atomicOr(&g_tq_device_flags, kFlagStagingTimeout);
+        mbar_wait_bounded(&bars[cur], (unsigned)(sc >> 1) & 1u);
+        if (sc + 1 < nsub) mbar_wait_bounded(&bars[cur ^ 1], (unsigned)((sc + 1) >> 1) & 1u);
       }
-      int acc[2][2][4];
+      __syncthreads();
+      return;
+    }
+    const unsigned char *sb = smem + cur * SM::buf;
+    const uint32_t *skc = reinterpret_cast<const uint32_t *>(sb + SM::kc);
+    const uint32_t *sks = reinterpret_cast<const uint32_t *>(sb + SM::ks);
+    const float *skn = reinterpret_cast<const float *>(sb + SM::kn);
+    const float *skr = reinterpret_cast<const float *>(sb + SM::kr);
+    const uint32_t *svc = reinterpret_cast<const uint32_t *>(sb + SM::vc);
+    const float *svn = reinterpret_cast<const float *>(sb + SM::vn);
+    const int64_t *vb = vbase + cur * NB;
+
+    // ------------------------------------------------------------ phase 1: logits (keys x heads)
+    {
+      // warp w: blocks 2w and 2w + 1; the query fragments of one (plane, k-step) serve both.
+      // A = the key words masked in place (bytes 0 or 2^shift; B carries 2^-shift).
+      int acc[2][2][2][4];  // [block][plane type][n-tile][c]
 #pragma unroll
-      for (int x = 0; x < 2; ++x)
+      for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
-        for (int y = 0; y < 2; ++y)
+        for (int x = 0; x < 2; ++x)
 #pragma unroll
-          for (int z = 0; z < 4; ++z) acc[x][y][z] = 0;
+          for (int y = 0; y < 2; ++y)
+#pragma unroll
+            for (int z = 0; z < 4; ++z) acc[kb][x][y][z] = 0;
+      uint32_t w[2][2][KP::all];
+#pragma unroll
+      for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int i = (2 * warp + kb) * 16 + gid + 8 * r;
+#pragma unroll
+          for (int P = 0; P < BK; ++P) w[kb][r][P] = skc[i * SM::KCW + P * 4 + t];
+          if constexpr (BK == 3) w[kb][r][3] = w[kb][r][0] ^ w[kb][r][1] ^ w[kb][r][2];
+          if constexpr (QJL) w[kb][r][KP::code] = sks[i * SM::KSW + t];
+        }
 #pragma unroll
       for (int P = 0; P < KP::all; ++P) {
         const int pt = (QJL && P == KP::code) ? 1 : 0;
 #pragma unroll
         for (int st = 0; st < 4; ++st) {
+          const uint4 f = kf4[(P * 4 + st) * 32 + lane];
           const uint32_t mlo = 0x01010101u << st, mhi = 0x01010101u << (st + 4);
-          const uint32_t a0 = w[0][P] & mlo, a1 = w[1][P] & mlo, a2 = w[0][P] & mhi, a3 = w[1][P] & mhi;
 #pragma unroll
-          for (int nt = 0; nt < 2; ++nt) mma_u8s8(acc[pt][nt], a0, a1, a2, a3, kb[P][st][nt][0], kb[P][st][nt][1]);
+          for (int kb = 0; kb < 2; ++kb) {
+            const uint32_t a0 = w[kb][0][P] & mlo, a1 = w[kb][1][P] & mlo;
+            const uint32_t a2 = w[kb][0][P] & mhi, a3 = w[kb][1][P] & mhi;
+            mma_u8s8(acc[kb][pt][0], a0, a1, a2, a3, f.x, f.y);
+            mma_u8s8(acc[kb][pt][1], a0, a1, a2, a3, f.z, f.w);
+          }
         }
       }
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int i = blk * 16 + gid + 8 * r;
-        const float dc = (float)acc[0][0][2 * r] + 256.f * (float)acc[0][0][2 * r + 1] +
-                         65536.f * (float)acc[0][1][2 * r] + 16777216.f * (float)acc[0][1][2 * r + 1];
-        float sc = fmaf(dc, cfc, -cq);
-        if constexpr (QJL) {
-          const float ds = (float)acc[1][0][2 * r] + 256.f * (float)acc[1][0][2 * r + 1] +
-                           65536.f * (float)acc[1][1][2 * r] + 16777216.f * (float)acc[1][1][2 * r + 1];
-          sc = fmaf(kc.qjl_scale * skr[i], fmaf(ds, cfs, -cp), sc);
+      for (int kb = 0; kb < 2; ++kb) {
+        const int blk = 2 * warp + kb;
+        const bool bok = vb[blk] >= 0;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int i = blk * 16 + gid + 8 * r;
+          const float dc = (float)acc[kb][0][0][2 * r] + 256.f * (float)acc[kb][0][0][2 * r + 1] +
+                           65536.f * (float)acc[kb][0][1][2 * r] + 16777216.f * (float)acc[kb][0][1][2 * r + 1];
+          float sc2 = fmaf(dc, cfc, -cq);
+          if constexpr (QJL) {
+            const float ds = (float)acc[kb][1][0][2 * r] + 256.f * (float)acc[kb][1][0][2 * r + 1] +
+                             65536.f * (float)acc[kb][1][1][2 * r] + 16777216.f * (float)acc[kb][1][1][2 * r + 1];
+            sc2 = fmaf(kc.qjl_scale * skr[i], fmaf(ds, cfs, -cp), sc2);
+          }
+          lg[t * kSub + i] = (bok && tk0 + i < t1) ? a.scale * skn[i] * sc2 : -INFINITY;
         }
-        lg[t * CH + i] = ok[r] ? a.scale * skn[i] * sc : -INFINITY;
       }
     }
-  }
-  __syncthreads();
+    __syncthreads();
 
-  // ---------------------------------------------------------------- phase 2: softmax weights
-  if (warp < kG) {
-    // warp g: max logit, weights w = e^{l - max}, W = w * ||v||, sum w, max W for head g
-    const int g = warp;
-    float mx = -INFINITY;
-    for (int i = lane; i < CH; i += 32) mx = fmaxf(mx, lg[g * CH + i]);
-    mx = warp_max_f(mx);
-    float sw = 0.f, mW = 0.f;
-    for (int i = lane; i < CH; i += 32) {
-      const float l = lg[g * CH + i];
-      const float wgt = l == -INFINITY ? 0.f : __expf(l - mx);
-      const float W = wgt * svn[i];
-      lg[g * CH + i] = W;
-      sw += wgt;
-      mW = fmaxf(mW, W);
-    }
-    sw = warp_sum_f(sw);
-    mW = warp_max_f(mW);
-    if (lane == 0) {
-      int e = 0;
-      frexpf(mW, &e);  // mW < 2^e, so mW * 2^(15 - e) + 1 < 2^16
-      const int F = mW > 0.f ? 15 - e : 0;
-      hstat[0 * kG + g] = mx;
-      hstat[1 * kG + g] = sw;
-      hstat[2 * kG + g] = ldexpf(1.f, F);
-      hstat[3 * kG + g] = ldexpf(1.f, -F);
-      wsum16[g] = 0;
-    }
-  } else if constexpr (BV == 3) {
-    // warps 4-7: (plane 2, parity) words, parity = p0 ^ p1 ^ p2, once per block and coordinate
-    for (int idx = tid - kG * 32; idx < NBLK * kD; idx += kThreads - kG * 32) {
-      const int kb = idx / kD, j = idx % kD;
-      const uint32_t A = svc[kb * SM::VBW + j];
-      const uint32_t hw = svc[kb * SM::VBW + kD + (j >> 1)] >> (16 * (j & 1));
-      const uint32_t par = (A ^ (A >> 16) ^ hw) & 0xffffu;
-      sx1[kb * SM::X1W + j] = (hw & 0xffffu) | (par << 16);
-    }
-  }
-  __syncthreads();
-  {
-    // B fragments of the value MMAs: lane (gid, t) = column (head gid/2, plane gid&1) and
-    // tokens t, t+8 (register 0) and t+4, t+12 (register 1); n-tile = limb.
-    const int g = gid >> 1, ps = gid & 1;
-    const float mul = hstat[2 * kG + g];
-    const uint32_t key0 = (uint32_t)((grp * a.splits + s) * CH) * 4u + (uint32_t)g;
-    int mine = 0;
-    for (int kb = warp; kb < NBLK; kb += kWarps) {
-      const float *wr = &lg[g * CH + kb * 16];
-      const int toks[4] = {t, t + 8, t + 4, t + 12};
-      uint32_t v[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t key = key0 + 4u * (uint32_t)(kb * 16 + toks[i]);
-        v[i] = (uint32_t)__float2int_rd(fmaf(wr[toks[i]], mul, dither(key)));
+    // ------------------------------------------------------------ phase 2: softmax weights
+    if (warp < kG) {
+      // warp g: running max, weights w = e^{l - M}, W = w ||v||, running sum, max and sum of W
+      const int g = warp;
+      float mx = -INFINITY;
+      for (int i = lane; i < kSub; i += 32) mx = fmaxf(mx, lg[g * kSub + i]);
+      mx = warp_max_f(mx);
+      const float Mold = hM[g];
+      const float Mnew = fmaxf(Mold, mx);
+      float sw = 0.f, mW = 0.f;
+      for (int i = lane; i < kSub; i += 32) {
+        const float l = lg[g * kSub + i];
+        const float wgt = l == -INFINITY ? 0.f : __expf(l - Mnew);
+        const float W = l == -INFINITY ? 0.f : wgt * svn[i];  // masked slots may hold stale bytes
+        lg[g * kSub + i] = W;
+        sw += wgt;
+        mW = fmaxf(mW, W);
       }
-      if (ps == 0) mine += (int)(v[0] + v[1] + v[2] + v[3]);
-      const int sh = 16 * ps;
-      vfrag[kb * 32 + lane] = make_uint4(((v[0] & 255u) | ((v[1] & 255u) << 8)) << sh,
-                                         ((v[2] & 255u) | ((v[3] & 255u) << 8)) << sh,
-                                         ((v[0] >> 8) | ((v[1] >> 8) << 8)) << sh,
-                                         ((v[2] >> 8) | ((v[3] >> 8) << 8)) << sh);
+      sw = warp_sum_f(sw);
+      mW = warp_max_f(mW);
+      if (lane == 0) {
+        const float alpha = Mnew == -INFINITY ? 1.f : __expf(Mold - Mnew);
+        // integer weights X = floor(W 2 e_P scale + dither) < 2^16 for every plane P
+        const float top = mW * 2.f * vc.plane_coef_max;
+        int e = 0;
+        frexpf(top, &e);  // top < 2^e
+        const float sc = top > 0.f ? ldexpf(1.f - 1.f / 512.f, 16 - e) : 1.f;
+        hM[g] = Mnew;
+        hL[g] = hL[g] * alpha + sw;
+        hAlpha[g] = alpha;
+        hScale[g] = sc;
+        hInv[g] = 1.f / (128.f * sc);
+        csum[g] = 0;
+      }
+    } else if constexpr (BV == 3) {
+      // warps 4-7: (plane 2, parity) words, parity = p0 ^ p1 ^ p2, one coordinate per thread
+      const int j = tid - kG * 32;
+      const int sh = 16 * (j & 1);
+#pragma unroll 4
+      for (int kb = 0; kb < NB; ++kb) {
+        const uint32_t A = svc[kb * SM::VBW + j];
+        const uint32_t hw = svc[kb * SM::VBW + kD + (j >> 1)] >> sh;
+        const uint32_t par = A ^ (A >> 16) ^ hw;
+        sx1[kb * SM::X1W + j] = __byte_perm(hw, par, 0x5410);
+      }
     }
-    mine += __shfl_xor_sync(TQ_FULL_MASK, mine, 1);  // lanes t and t^1 share a head and plane
-    mine += __shfl_xor_sync(TQ_FULL_MASK, mine, 2);
-    if (t == 0 && ps == 0) atomicAdd(&wsum16[g], mine);
-  }
-  __syncthreads();
-
-  // ---------------------------------------------------------------- phase 3: value sum
-  // warp w: coordinate half ch = w & 1 (64 coordinates = 4 m-tiles) and block group w >> 1.
-  // In m-tile mt, row gid <-> coordinate 64 ch + 8 gid + 2 mt and row gid + 8 <-> the next one.
-  const int ch = warp & 1, bgrp = warp >> 1;
-  const int jb = 64 * ch + 8 * gid;
-  int accv[4][VT][2][4];
-#pragma unroll
-  for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-    for (int x = 0; x < VT; ++x)
-#pragma unroll
-      for (int y = 0; y < 2; ++y)
-#pragma unroll
-        for (int z = 0; z < 4; ++z) accv[mt][x][y][z] = 0;
-  for (int kb = bgrp; kb < NBLK; kb += 4) {
-    if (vbase[kb] < 0) continue;
-    uint32_t X[VT][8];
+    __syncthreads();
     {
-      const uint4 u0 = *reinterpret_cast<const uint4 *>(svc + kb * SM::VBW + jb);
-      const uint4 u1 = *reinterpret_cast<const uint4 *>(svc + kb * SM::VBW + jb + 4);
-      X[0][0] = u0.x; X[0][1] = u0.y; X[0][2] = u0.z; X[0][3] = u0.w;
-      X[0][4] = u1.x; X[0][5] = u1.y; X[0][6] = u1.z; X[0][7] = u1.w;
-    }
-    if constexpr (BV == 3) {
-      const uint4 u0 = *reinterpret_cast<const uint4 *>(sx1 + kb * SM::X1W + jb);
-      const uint4 u1 = *reinterpret_cast<const uint4 *>(sx1 + kb * SM::X1W + jb + 4);
-      X[VT - 1][0] = u0.x; X[VT - 1][1] = u0.y; X[VT - 1][2] = u0.z; X[VT - 1][3] = u0.w;
-      X[VT - 1][4] = u1.x; X[VT - 1][5] = u1.y; X[VT - 1][6] = u1.z; X[VT - 1][7] = u1.w;
-    }
-    const uint4 fb = vfrag[kb * 32 + lane];
+      // B fragments of the value MMAs.  Lane (gid, t): column = (head gid/2, limb gid&1).  The
+      // k index runs over (token, plane) pairs in the order the value words give them:
+      // register 0 = tokens t, t+8 of the low plane, then of the high plane; register 1 = the
+      // same for tokens t+4, t+12.  Byte = limb of X = floor(W 2 e_P 2^F + dither), dithered so
+      // that the many sub-unit tail weights are unbiased rather than all rounded down.
+      const int g = gid >> 1, l = gid & 1;
+      const float S2 = 2.f * hScale[g];
+      float C[2 * VT];
 #pragma unroll
-    for (int mt = 0; mt < 4; ++mt)
+      for (int P = 0; P < 2 * VT; ++P) C[P] = S2 * vc.plane_coef[P];
+      const uint32_t sel = (uint32_t)l | ((uint32_t)(4 + l) << 4);  // byte l of two words
+      const uint32_t key0 = ((uint32_t)grp * (uint32_t)a.max_len + (uint32_t)tk0) * 4u + (uint32_t)g;
+      uint32_t xs = 0;  // sum of this lane's X values
 #pragma unroll
-      for (int x = 0; x < VT; ++x) {
-        const uint32_t r0 = X[x][2 * mt], r1 = X[x][2 * mt + 1];
-        const uint32_t a0 = (r0 >> t) & 0x01010101u, a1 = (r1 >> t) & 0x01010101u;
-        const uint32_t a2 = (r0 >> (t + 4)) & 0x01010101u, a3 = (r1 >> (t + 4)) & 0x01010101u;
-        mma_u8u8(accv[mt][x][0], a0, a1, a2, a3, fb.x, fb.y);
-        mma_u8u8(accv[mt][x][1], a0, a1, a2, a3, fb.z, fb.w);
+      for (int kk = 0; kk < NB / kWarps; ++kk) {
+        const int kb = warp + kWarps * kk;
+        const float *wr = &lg[g * kSub + kb * 16];
+        const int toks[4] = {t, t + 8, t + 4, t + 12};
+        float W[4], dz[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          W[i] = wr[toks[i]];
+          dz[i] = dither(key0 + 4u * (uint32_t)(kb * 16 + toks[i]));
+        }
+        uint32_t reg[2 * VT];
+#pragma unroll
+        for (int x = 0; x < VT; ++x)
+#pragma unroll
+          for (int rr = 0; rr < 2; ++rr) {
+            const int i0 = 2 * rr, i1 = 2 * rr + 1;  // the two tokens of this register
+            const uint32_t x0 = __float2uint_rd(fmaf(W[i0], C[2 * x], dz[i0]));
+            const uint32_t x1 = __float2uint_rd(fmaf(W[i1], C[2 * x], dz[i1]));
+            const uint32_t x2 = __float2uint_rd(fmaf(W[i0], C[2 * x + 1], dz[i0]));
+            const uint32_t x3 = __float2uint_rd(fmaf(W[i1], C[2 * x + 1], dz[i1]));
+            reg[2 * x + rr] = __byte_perm(__byte_perm(x0, x1, sel), __byte_perm(x2, x3, sel), 0x5410);
+            xs += (x0 + x1) + (x2 + x3);
+          }
+        vfrag[kb * 32 + lane] = VT == 2 ? make_uint4(reg[0], reg[1], reg[2 * VT - 2], reg[2 * VT - 1])
+                                        : make_uint4(reg[0], reg[1], 0u, 0u);
       }
+      // the codebook's constant term uses the same integers: sum X per head (limb-0 lanes)
+      uint32_t mine = l == 0 ? xs : 0u;
+      mine += __shfl_xor_sync(TQ_FULL_MASK, mine, 1);
+      mine += __shfl_xor_sync(TQ_FULL_MASK, mine, 2);
+      mine += __shfl_xor_sync(TQ_FULL_MASK, mine, 4);
+      if (t == 0 && l == 0) atomicAdd(&csum[g], (int)mine);
+    }
+    __syncthreads();
+
+    // ------------------------------------------------------------ phase 3: value sum
+    // warp w: coordinate half ch = w & 1 (64 coordinates = 4 m-tiles) and blocks bgrp + 4 k.
+    // In m-tile mt, row gid <-> coordinate 64 ch + 8 gid + 2 mt and row gid + 8 <-> the next one.
+    {
+      const uint32_t mlo = 1u << (7 - t), mhi = 1u << (3 - t);
+      int accv[4][VT][4];
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int x = 0; x < VT; ++x)
+#pragma unroll
+          for (int z = 0; z < 4; ++z) accv[mt][x][z] = 0;
+#pragma unroll
+      for (int kk = 0; kk < NB / 4; ++kk) {
+        const int kb = bgrp + 4 * kk;
+        if (vb[kb] < 0) continue;
+        uint32_t X[VT][8];
+        {
+          const uint4 u0 = *reinterpret_cast<const uint4 *>(svc + kb * SM::VBW + jb);
+          const uint4 u1 = *reinterpret_cast<const uint4 *>(svc + kb * SM::VBW + jb + 4);
+          X[0][0] = u0.x; X[0][1] = u0.y; X[0][2] = u0.z; X[0][3] = u0.w;
+          X[0][4] = u1.x; X[0][5] = u1.y; X[0][6] = u1.z; X[0][7] = u1.w;
+        }
+        if constexpr (BV == 3) {
+          const uint4 u0 = *reinterpret_cast<const uint4 *>(sx1 + kb * SM::X1W + jb);
+          const uint4 u1 = *reinterpret_cast<const uint4 *>(sx1 + kb * SM::X1W + jb + 4);
+          X[VT - 1][0] = u0.x; X[VT - 1][1] = u0.y; X[VT - 1][2] = u0.z; X[VT - 1][3] = u0.w;
+          X[VT - 1][4] = u1.x; X[VT - 1][5] = u1.y; X[VT - 1][6] = u1.z; X[VT - 1][7] = u1.w;
+        }
+        const uint4 fb = vfrag[kb * 32 + lane];
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+          for (int x = 0; x < VT; ++x) {
+            // token bits t, t+8 (and t+4, t+12) of both planes moved to bit 7 of each byte by a
+            // multiply (the FMA pipe) and kept by one AND: bytes 0 or 128
+            const uint32_t r0 = X[x][2 * mt], r1 = X[x][2 * mt + 1];
+            const uint32_t a0 = mul_lo(r0, mlo) & 0x80808080u, a1 = mul_lo(r1, mlo) & 0x80808080u;
+            const uint32_t a2 = mul_lo(r0, mhi) & 0x80808080u, a3 = mul_lo(r1, mhi) & 0x80808080u;
+            mma_u8u8(accv[mt][x], a0, a1, a2, a3, x == 0 ? fb.x : fb.z, x == 0 ? fb.y : fb.w);
+          }
+      }
+      // accv[mt][x][c]: c0/c1 = (coordinate jb + 2 mt, head t, limb 0/1), c2/c3 = (+1, ...):
+      // 128 sum_tok X b over the word type's two planes.  With s = 2b - 1 the codebook's
+      // constant term is -(1/2) sum X, added once per sub-chunk by the bgrp 0 warps.
+      const float al = hAlpha[t], inv = hInv[t];
+      const float cterm = bgrp == 0 ? 64.f * (float)csum[t] : 0.f;
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          float v = 0.f;
+#pragma unroll
+          for (int x = 0; x < VT; ++x) v += (float)accv[mt][x][2 * r] + 256.f * (float)accv[mt][x][2 * r + 1];
+          o[mt][r] = fmaf(o[mt][r], al, (v - cterm) * inv);
+        }
+    }
+    __syncthreads();  // the buffers, lg, vfrag and the head statistics are reused next
   }
-  // accv[mt][x][limb][c]: c0/c1 = (coordinate jb + 2 mt, head t, plane lo/hi), c2/c3 = (+1, ...)
-  __syncthreads();  // every warp is done with the staged data that obuf overwrites
+
+  // ---------------------------------------------------------------- partials of the 4 heads
+  __syncthreads();
 #pragma unroll
   for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      float v = 0.f;
-#pragma unroll
-      for (int x = 0; x < VT; ++x)
-#pragma unroll
-        for (int ps = 0; ps < 2; ++ps) {
-          const float D = (float)accv[mt][x][0][2 * r + ps] + 256.f * (float)accv[mt][x][1][2 * r + ps];
-          v = fmaf(2.f * vc.plane_coef[2 * x + ps], D, v);
-        }
-      obuf[(bgrp * kG + t) * kD + jb + 2 * mt + r] = v;
-    }
+    for (int r = 0; r < 2; ++r) obuf[(bgrp * kG + t) * kD + jb + 2 * mt + r] = o[mt][r];
   __syncthreads();
   for (int i = tid; i < kG * kD; i += kThreads) {
     const int g = i / kD, j = i % kD;
     const float v = obuf[(0 * kG + g) * kD + j] + obuf[(1 * kG + g) * kD + j] + obuf[(2 * kG + g) * kD + j] +
                     obuf[(3 * kG + g) * kD + j];
     const int64_t pb = (((int64_t)b * a.hq + (int64_t)h * kG + g) * a.splits + s) * (kD + 2);
-    part[pb + 2 + j] = (v - vc.plane_coef_sum * (float)wsum16[g]) * hstat[3 * kG + g];
+    part[pb + 2 + j] = v;
   }
   if (tid < kG) {
     const int64_t pb = (((int64_t)b * a.hq + (int64_t)h * kG + tid) * a.splits + s) * (kD + 2);
-    part[pb] = hstat[0 * kG + tid];
-    part[pb + 1] = hstat[1 * kG + tid];
+    part[pb] = hM[tid];
+    part[pb + 1] = hL[tid];
   }
 }
 
-template <int BK, int BV, bool QJL, int CH>
+template <int BK, int BV, bool QJL>
 cudaError_t launch_mma(const TqConsts &kc, const TqConsts &vc, const MmaArgs &a, dim3 grid,
                        const uint32_t *kfrag, const float *kconst, float *part, cudaStream_t st) {
-  const size_t smem = MmaSmem<BK, BV, QJL, CH>::total;
-  cudaError_t e = cudaFuncSetAttribute(attend_mma_kernel<BK, BV, QJL, CH>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const size_t smem = MmaSmem<BK, BV, QJL>::total;
+  cudaError_t e = cudaFuncSetAttribute(attend_mma_kernel<BK, BV, QJL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
   if (e != cudaSuccess) return e;
-  attend_mma_kernel<BK, BV, QJL, CH><<<grid, kThreads, smem, st>>>(kc, vc, a, kfrag, kconst, part);
+  attend_mma_kernel<BK, BV, QJL><<<grid, kThreads, smem, st>>>(kc, vc, a, kfrag, kconst, part);
   return cudaGetLastError();
 }
 
@@ -608,8 +763,7 @@ cudaError_t launch_fast(const TqConsts &kc, const TqConsts &vc, const MmaArgs &a
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)a.splits, (unsigned)a.hkv, (unsigned)batch);
   tq_prof_begin(TQK_ATTEND_SPLIT, st);
-  e = a.chunk == 512 ? launch_mma<BK, BV, QJL, 512>(kc, vc, a, grid, kfrag, kconst, part, st)
-                     : launch_mma<BK, BV, QJL, 256>(kc, vc, a, grid, kfrag, kconst, part, st);
+  e = launch_mma<BK, BV, QJL>(kc, vc, a, grid, kfrag, kconst, part, st);
   tq_prof_end(TQK_ATTEND_SPLIT, st);
   return e;
 }
@@ -623,17 +777,30 @@ bool attn_fast_eligible(const TqConsts &kc, const TqConsts &vc, const tq_attn_de
   if (kc.bits < 1 || kc.bits > 3 || (vc.bits != 2 && vc.bits != 3)) return false;
   if (kc.m != 0 && kc.m != kD) return false;
   if (!kc.fast_ok || !vc.fast_ok) return false;
+  // the value weights are unsigned fixed point: every plane coefficient must be >= 0
+  for (int P = 0; P < (vc.bits == 3 ? 4 : vc.bits); ++P)
+    if (!(vc.plane_coef[P] >= 0.f)) return false;
   if (desc.block_table ? (desc.block_size % 16) != 0 : (desc.ctx_stride % 16) != 0) return false;
   return true;
 }
 
 int attn_fast_chunk(const tq_attn_desc &desc) {
-  // 512-token chunks halve the per-CTA fixed work and the partials to merge; 256 only when
-  // 512 would leave fewer than two CTAs per SM
+  // Tokens per CTA (a multiple of 16): the 16-token blocks of all (sequence, KV head) rows split
+  // evenly over two resident CTAs per SM, so that a uniform batch runs as one full wave; at least
+  // 128 tokens (the fixed per-CTA work) and at most 1024 (long or ragged batches then run as
+  // many short waves that the block scheduler balances).
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) sms = n;
+  }
   const int64_t rows = (int64_t)desc.batch * desc.n_kv_heads;
   const int maxlen = desc.max_seq_len > 0 ? desc.max_seq_len : 1;
-  const int64_t ctas512 = rows * ((maxlen + 511) / 512);
-  return ctas512 >= 2 * 148 ? 512 : 256;
+  const int64_t blocks = rows * ((maxlen + 15) / 16);
+  const int64_t slots = 2 * (int64_t)sms;
+  int64_t per = (blocks + slots - 1) / slots;
+  per = per < 8 ? 8 : (per > 64 ? 64 : per);
+  return (int)(16 * per);
 }
 
 size_t attn_fast_extra_bytes(const TqConsts &kc, const tq_attn_desc &desc) {
@@ -697,8 +864,7 @@ cudaError_t launch_step(const TqConsts &kc, const TqConsts &vc, const MmaArgs &a
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)a.splits, (unsigned)a.hkv, (unsigned)batch);
   tq_prof_begin(TQK_ATTEND_SPLIT, st);
-  e = a.chunk == 512 ? launch_mma<BK, BV, QJL, 512>(kc, vc, a, grid, kfrag, kconst, part, st)
-                     : launch_mma<BK, BV, QJL, 256>(kc, vc, a, grid, kfrag, kconst, part, st);
+  e = launch_mma<BK, BV, QJL>(kc, vc, a, grid, kfrag, kconst, part, st);
   tq_prof_end(TQK_ATTEND_SPLIT, st);
   return e;
 }
@@ -738,4 +904,19 @@ cudaError_t launch_decode_step_fast(const TqConsts &kc, const TqConsts &vc, cons
   TQ_STEP(1, 3, false) TQ_STEP(2, 3, false) TQ_STEP(3, 3, false)
 #undef TQ_STEP
   return cudaErrorInvalidValue;
+}
+
+extern "C" tq_status tq_device_status(int32_t device, int32_t *flags, int32_t clear) {
+  if (!flags) return tq_fail(TQ_EINVAL, "flags is NULL");
+  cudaError_t e = cudaSetDevice(device);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  int v = 0;
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&v, g_tq_device_flags, sizeof(int));
+  if (e == cudaSuccess && clear) {
+    const int z = 0;
+    e = cudaMemcpyToSymbol(g_tq_device_flags, &z, sizeof(int));
+  }
+  if (e != cudaSuccess) return tq_fail(TQ_ECUDA, "device status: %s", cudaGetErrorString(e));
+  *flags = v;
+  return TQ_OK;
 }

@@ -22,6 +22,7 @@ struct TqConsts {
   int fast_ok;    // codebook is an exact odd bit-plane expansion (tensor-core attention path)
   float plane_coef[4];   // e_P of c(code) = sum e_P s_P (+ e_3 s_0 s_1 s_2), s_P = 2 bit_P - 1
   float plane_coef_sum;  // sum of plane_coef
+  float plane_coef_max;  // largest plane_coef
   float inv_sqrt_d;
   float qjl_scale;  // sqrt(pi/2)/m, 0 when m == 0
   float centroids[TQ_MAX_LEVELS];

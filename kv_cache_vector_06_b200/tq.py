@@ -69,6 +69,7 @@ def _load():
         "tq_decode_step_workspace_size": (st, [c_void_p, c_void_p, POINTER(AttnDesc), c_int64, POINTER(c_size_t)]),
         "tq_decode_step": (st, [c_void_p, c_void_p, POINTER(AttnDesc), c_void_p, c_void_p, c_int, c_int64, c_void_p,
                                 c_void_p, c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
+        "tq_device_status": (st, [c_int32, POINTER(c_int32), c_int32]),
         "tq_search_workspace_size": (st, [c_void_p, c_int32, c_int64, c_int32, POINTER(c_size_t)]),
         "tq_search_topk": (st, [c_void_p, c_void_p, c_int, c_int32, PackedC, c_int64, c_int32, c_void_p,
                                 c_void_p, c_void_p, c_size_t, c_void_p]),
@@ -342,6 +343,16 @@ def decode_step(kctx: Context, vctx: Context, q: torch.Tensor, k_new: torch.Tens
                               _dev(new_slots, kctx.device, "new_slots", torch.int64), _dev(q, kctx.device, "q"),
                               _dtype_code(q), _dev(out, kctx.device, "out", torch.float32), w, wb, _stream_ptr(stream)))
     return out
+
+
+DEVFLAG_STAGING_TIMEOUT = 1
+
+
+def device_status(device: int = 0, clear: bool = False) -> int:
+    """TQ_DEVFLAG_* bits raised by the library's kernels on `device` (synchronizes it)."""
+    f = c_int32()
+    _check(LIB.tq_device_status(device, ctypes.byref(f), 1 if clear else 0))
+    return f.value
 
 
 NOALLOC_SCRATCH_BYTES = 8 << 20

@@ -87,6 +87,7 @@ def _step_case(tq, d, kbits, km, vbits, vlayout, batch, hkv, group, lens, paged,
     _packed_equal(kp, kp2)
     _packed_equal(vp, vp2)
     assert torch.equal(out, out2)
+    assert tq.device_status() == 0
     pairs = [(b, h) for b in range(batch) for h in range(hq)]
     ref = oracle_heads(kq, vq, kp, vp, q.cpu(), pairs, new_lens, slots_of, group)
     got = out.cpu().numpy()

@@ -167,6 +167,7 @@ def _attention_case(tq, d, kbits, km, vbits, batch, hkv, group, lens, paged, qdt
     ref = oattn.attend_decode(qx.double().numpy(), kc, vc, lens, hkv, kq.D64, kq.S64, kq.c, vq.D64, vq.c,
                               ctx_stride=maxlen, block_table=None if table is None else table.numpy())
     assert_attention_close(out.cpu().numpy(), ref)
+    assert tq.device_status() == 0
     # encode parity on these rows too
     compare_encode(kq, kq.oracle_encode(kx.double().numpy()), *unpack(kq, kp, rows=sl))
     return out
