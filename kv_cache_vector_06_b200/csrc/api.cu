@@ -478,10 +478,11 @@ tq_status tq_decode_step(const tq_ctx *kctx, const tq_ctx *vctx, const tq_attn_d
   const int64_t nq = (int64_t)desc->batch * desc->n_q_heads;
   float *part = reinterpret_cast<float *>(static_cast<char *>(ws) + query_prep_bytes(kctx, nq));
   void *extra = reinterpret_cast<char *>(part) +
-                tq_align_up((int64_t)sizeof(float) * desc->batch * desc->n_q_heads * plan.splits * (kctx->spec.d + 2), 256);
+                tq_align_up((int64_t)sizeof(float) * desc->batch * desc->n_q_heads * plan.splits * (kctx->spec.d + 4), 256);
   cudaError_t e = launch_decode_step_fast(kctx->k, vctx->k, *desc, plan, k_new, v_new, (int)kv_dtype, n_new, new_slots,
-                                          q, (int)q_dtype, extra, part, s);
+                                          q, (int)q_dtype, extra, part, plan.fused ? out : nullptr, s);
   if (e != cudaSuccess) return tq_cuda_check(e, "decode step launch");
+  if (plan.fused) return TQ_OK;
   return tq_cuda_check(launch_attend_combine(vctx->k, *desc, plan, part, out, s), "combine launch");
 }
 

@@ -165,7 +165,7 @@ attend_split_kernel(TqConsts kc, TqConsts vc, AttnArgs a, const float *__restric
 
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    const int64_t base = (((int64_t)b * a.hq + (int64_t)h * G + g) * a.splits + s) * (d + 2);
+    const int64_t base = (((int64_t)b * a.hq + (int64_t)h * G + g) * a.splits + s) * (d + 4);
     if (tid == 0) {
       part[base] = mrun[g];
       part[base + 1] = lrun[g];
@@ -208,16 +208,16 @@ attend_combine_kernel(TqConsts vc, int splits, const float *__restrict__ part, f
   float *acc = y + d;                  // [ngroups][d]
   float *red = acc + ngroups * d;      // [32]
   const int64_t bh = blockIdx.x;
-  const float *pb = part + bh * splits * (d + 2);
+  const float *pb = part + bh * splits * (d + 4);
   float m = -INFINITY;
-  for (int s = threadIdx.x; s < splits; s += blockDim.x) m = fmaxf(m, pb[(int64_t)s * (d + 2)]);
+  for (int s = threadIdx.x; s < splits; s += blockDim.x) m = fmaxf(m, pb[(int64_t)s * (d + 4)]);
   const float M = block_reduce(m, red, true);
   float l = 0.f;
   for (int s = threadIdx.x; s < splits; s += blockDim.x) {
-    const float ms = pb[(int64_t)s * (d + 2)];
+    const float ms = pb[(int64_t)s * (d + 4)];
     const float fs = (ms == -INFINITY) ? 0.f : __expf(ms - M);
     f[s] = fs;
-    l += pb[(int64_t)s * (d + 2) + 1] * fs;
+    l += pb[(int64_t)s * (d + 4) + 1] * fs;
   }
   const float L = block_reduce(l, red, false);  // its barriers also publish f[]
   for (int idx = threadIdx.x; idx < ngroups * d; idx += blockDim.x) {
@@ -225,16 +225,16 @@ attend_combine_kernel(TqConsts vc, int splits, const float *__restrict__ part, f
     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
     int s = g;
     for (; s + 3 * ngroups < splits; s += 4 * ngroups) {  // four independent loads in flight
-      const float v0 = pb[(int64_t)s * (d + 2) + 2 + j];
-      const float v1 = pb[(int64_t)(s + ngroups) * (d + 2) + 2 + j];
-      const float v2 = pb[(int64_t)(s + 2 * ngroups) * (d + 2) + 2 + j];
-      const float v3 = pb[(int64_t)(s + 3 * ngroups) * (d + 2) + 2 + j];
+      const float v0 = pb[(int64_t)s * (d + 4) + 2 + j];
+      const float v1 = pb[(int64_t)(s + ngroups) * (d + 4) + 2 + j];
+      const float v2 = pb[(int64_t)(s + 2 * ngroups) * (d + 4) + 2 + j];
+      const float v3 = pb[(int64_t)(s + 3 * ngroups) * (d + 4) + 2 + j];
       a0 = fmaf(v0, f[s], a0);
       a1 = fmaf(v1, f[s + ngroups], a1);
       a2 = fmaf(v2, f[s + 2 * ngroups], a2);
       a3 = fmaf(v3, f[s + 3 * ngroups], a3);
     }
-    for (; s < splits; s += ngroups) a0 = fmaf(pb[(int64_t)s * (d + 2) + 2 + j], f[s], a0);
+    for (; s < splits; s += ngroups) a0 = fmaf(pb[(int64_t)s * (d + 4) + 2 + j], f[s], a0);
     acc[g * d + j] = (a0 + a1) + (a2 + a3);
   }
   __syncthreads();
@@ -278,11 +278,13 @@ AttnPlan attn_plan(const tq_attn_desc &desc, const TqConsts &kc, const TqConsts 
   AttnPlan p;
   p.group = desc.n_q_heads / desc.n_kv_heads;
   p.fast = attn_fast_eligible(kc, vc, desc);
+  p.fused = false;
   p.extra = 0;
   if (p.fast) {
     const int maxlen = desc.max_seq_len > 0 ? desc.max_seq_len : 1;
     p.chunk = attn_fast_chunk(desc);
     p.splits = (maxlen + p.chunk - 1) / p.chunk;
+    p.fused = p.splits <= kFusedMaxSplits;
     p.extra = attn_fast_extra_bytes(kc, desc);
     return p;
   }
@@ -298,7 +300,7 @@ AttnPlan attn_plan(const tq_attn_desc &desc, const TqConsts &kc, const TqConsts 
 }
 
 size_t attn_partials_bytes(const tq_attn_desc &desc, const AttnPlan &plan, int d) {
-  return (size_t)tq_align_up((int64_t)sizeof(float) * desc.batch * desc.n_q_heads * plan.splits * (d + 2), 256) +
+  return (size_t)tq_align_up((int64_t)sizeof(float) * desc.batch * desc.n_q_heads * plan.splits * (d + 4), 256) +
          plan.extra;
 }
 
@@ -325,9 +327,9 @@ cudaError_t launch_attend(const TqConsts &kc, const TqConsts &vc, const tq_attn_
   cudaError_t e;
   if (plan.fast) {
     void *extra = reinterpret_cast<char *>(partials) +
-                  tq_align_up((int64_t)sizeof(float) * desc.batch * desc.n_q_heads * plan.splits * (kc.d + 2), 256);
-    e = launch_attend_fast(kc, vc, desc, plan, q, dtype, extra, partials, st);
-    if (e != cudaSuccess) return e;
+                  tq_align_up((int64_t)sizeof(float) * desc.batch * desc.n_q_heads * plan.splits * (kc.d + 4), 256);
+    e = launch_attend_fast(kc, vc, desc, plan, q, dtype, extra, partials, plan.fused ? out : nullptr, st);
+    if (e != cudaSuccess || plan.fused) return e;
   } else switch (plan.group) {
     case 1: e = launch_split<1>(kc, vc, a, grid, qr, p, partials, st); break;
     case 2: e = launch_split<2>(kc, vc, a, grid, qr, p, partials, st); break;

@@ -44,6 +44,8 @@ struct MmaArgs {
   const int32_t *seq_lens;
   const int32_t *block_table;
   tq_packed k, v;
+  int *counter;  // per (sequence, KV head): CTAs done (zeroed by the query-fragment kernel)
+  float *out;    // final output when the kernel merges its splits itself, else null
 };
 
 __device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -109,8 +111,8 @@ struct KPlanes {
 // |X| 2^F <= 2^30.  kconst: 2^-F_code, 2^-F_sign, (sum e_P) sum q', sum p per head.
 template <int BK, bool QJL>
 __device__ __forceinline__ void kfrag_group(const TqConsts &kc, const void *__restrict__ q, int dtype,
-                                            uint32_t *__restrict__ kfrag, float *__restrict__ kconst, int grp,
-                                            float *sS) {
+                                            uint32_t *__restrict__ kfrag, float *__restrict__ kconst,
+                                            int *__restrict__ counter, int grp, float *sS) {
   using KP = KPlanes<BK, QJL>;
   __shared__ float qs[kG][kD];           // q', the rotated queries
   __shared__ float X[KP::all][kG][kD];
@@ -201,6 +203,7 @@ __device__ __forceinline__ void kfrag_group(const TqConsts &kc, const void *__re
   }
   __syncthreads();
   if (tid < 16) kconst[(int64_t)grp * 16 + tid] = red[tid % 4][tid / 4];
+  if (tid == 0) counter[grp] = 0;  // the split kernel that follows counts its finished CTAs here
   uint32_t *out = kfrag + (int64_t)grp * KP::regs * 32;
   // layout [plane][k-step][lane][n-tile, register]: one 16-byte load per lane and k-step
   for (int idx = tid; idx < KP::regs * 32; idx += kThreads) {
@@ -233,9 +236,9 @@ __device__ __forceinline__ void kfrag_group(const TqConsts &kc, const void *__re
 template <int BK, bool QJL>
 __global__ void __launch_bounds__(kThreads)
 kfrag_kernel(TqConsts kc, const void *__restrict__ q, int dtype, uint32_t *__restrict__ kfrag,
-             float *__restrict__ kconst) {
+             float *__restrict__ kconst, int *__restrict__ counter) {
   extern __shared__ __align__(16) float sS[];
-  kfrag_group<BK, QJL>(kc, q, dtype, kfrag, kconst, blockIdx.x, sS);
+  kfrag_group<BK, QJL>(kc, q, dtype, kfrag, kconst, counter, blockIdx.x, sS);
 }
 
 // One launch for the work that precedes the split kernel in a decode step: blocks
@@ -247,7 +250,7 @@ __global__ void __launch_bounds__(kThreads)
 decode_prep_kernel(TqConsts kc, TqConsts vc, const void *__restrict__ knew, const void *__restrict__ vnew,
                    int kvdtype, int64_t nnew, const int64_t *__restrict__ slots, tq_packed kp, tq_packed vp,
                    const void *__restrict__ q, int qdtype, uint32_t *__restrict__ kfrag,
-                   float *__restrict__ kconst, int nkb, int nvb) {
+                   float *__restrict__ kconst, int *__restrict__ counter, int nkb, int nvb) {
   extern __shared__ __align__(16) float sS[];
   const int bid = blockIdx.x;
   if (bid < nkb) {
@@ -257,7 +260,7 @@ decode_prep_kernel(TqConsts kc, TqConsts vc, const void *__restrict__ knew, cons
     rotate_rows<kD>(vc, ROT_ENCODE, vnew, kvdtype, nnew, kD, slots, vp.capacity, static_cast<uint32_t *>(vp.codes),
                     vp.norm, nullptr, nullptr, nullptr, bid - nkb, sS);
   } else {
-    kfrag_group<BK, QJL>(kc, q, qdtype, kfrag, kconst, bid - nkb - nvb, sS);
+    kfrag_group<BK, QJL>(kc, q, qdtype, kfrag, kconst, counter, bid - nkb - nvb, sS);
   }
 }
 
@@ -268,6 +271,27 @@ constexpr int kFlagStagingTimeout = 1;
 
 // Bulk asynchronous copies (global -> this CTA's shared memory) completing on an mbarrier, and
 // the bounded wait for them.  Addresses 16-byte aligned, sizes multiples of 16 bytes.
+// 2^e as a float for e in [-126, 127].
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
+// Fixed-point scale of a sub-chunk's value weights: with top = max W * 2 max_P e_P, the integer
+// weights floor(W 2 e_P sc + dither) stay below 2^16.  Returns sc and 1 / (128 sc).
+__device__ __forceinline__ void weight_scale(float top, float &sc, float &inv128) {
+  if (!(top > 0.f)) {
+    sc = 1.f;
+    inv128 = 1.f / 128.f;
+    return;
+  }
+  int e = ((__float_as_int(top) >> 23) & 0xff) - 126;  // top < 2^e
+  e = e < -110 ? -110 : (e > 126 ? 126 : e);
+  sc = pow2i(16 - e) * (1.f - 1.f / 512.f);
+  inv128 = pow2i(e - 23) * (512.f / 511.f);
+}
+// Largest of the 8 per-warp partials of one head.
+__device__ __forceinline__ float max8(const float *p) {
+  const float4 u = *reinterpret_cast<const float4 *>(p), v = *reinterpret_cast<const float4 *>(p + 4);
+  return fmaxf(fmaxf(fmaxf(u.x, u.y), fmaxf(u.z, u.w)), fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+}
+
 // 32-bit multiply kept as such (an opaque multiplier: a power of two here, which would otherwise
 // become a shift on the integer ALU pipe).
 __device__ __forceinline__ uint32_t mul_lo(uint32_t x, uint32_t m) {
@@ -276,6 +300,11 @@ __device__ __forceinline__ uint32_t mul_lo(uint32_t x, uint32_t m) {
   return r;
 }
 __device__ __forceinline__ unsigned smem_addr(const void *p) { return (unsigned)__cvta_generic_to_shared(p); }
+// 16-byte asynchronous global -> shared copy through L2 (the partial rows other CTAs wrote).
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_addr(smem_dst)), "l"(gmem) : "memory");
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t *bar, unsigned count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(count) : "memory");
 }
@@ -308,6 +337,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, unsigned parity
 
 constexpr int kSub = 256;          // tokens per sub-chunk (one staging buffer)
 constexpr int kSubBlk = kSub / 16;  // 16-token blocks per sub-chunk
+constexpr int kLgS = kSub + 8;      // row stride of the logit/weight array (bank-conflict padding)
 
 // Shared-memory carve-up of attend_mma_kernel (bytes): two staging buffers (the sub-chunk being
 // computed and the one being loaded), then the per-sub-chunk work arrays.
@@ -329,76 +359,63 @@ struct MmaSmem {
   // work arrays
   static constexpr size_t x1 = 2 * buf;
   static constexpr size_t lg = x1 + (size_t)NB * X1W * 4;
-  static constexpr size_t vf = lg + (size_t)kG * kSub * 4;
+  static constexpr size_t vf = lg + (size_t)kG * kLgS * 4;
   static constexpr size_t kf = vf + (size_t)NB * 32 * 16;
   static constexpr size_t vb = kf + (size_t)KPlanes<BK, QJL>::regs * 32 * 4;
-  static constexpr size_t st = vb + (size_t)2 * NB * 8;
-  static constexpr size_t br = st + 16 * kG * 4;  // two mbarriers, one per staging buffer
+  static constexpr int MAXBLK = 64;  // blocks per CTA at most (a.chunk <= 1024 tokens)
+  static constexpr size_t st = vb + (size_t)MAXBLK * 8;
+  static constexpr size_t pw = st + 16 * kG * 4;  // per-warp partials (max logit, sum w, sum X, max ||v||)
+  static constexpr size_t br = pw + 4 * kG * kWarps * 4;  // two mbarriers, one per staging buffer
   static constexpr size_t total = br + 2 * 8 + 16;
   static_assert((size_t)4 * kG * kD * 4 <= 2 * buf, "the value-sum buffer reuses the staging buffers");
   static_assert(buf % 16 == 0 && x1 % 16 == 0 && kf % 16 == 0, "16-byte aligned regions");
 };
 
-// Issue the bulk copies of one sub-chunk (tokens [tk0, tk0 + kSub) of the CTA's (sequence, KV
-// head), blocks of 16 slots) into staging buffer `sb`, completing on `bar`.  Warp 0 runs it:
-// lane kb < 16 resolves block kb; the valid blocks (inside the sequence and the arrays) are one
-// contiguous run of slots in the contiguous layout (one copy per array) and one copy per array
-// and block when paged.  vb[kb] = first slot of block kb, or -1 (not copied; masked later).
+// The arrays a sub-chunk is copied from, one bulk copy (or one per block when paged) each.
+template <bool QJL>
+struct StageArrays {
+  static constexpr int n = QJL ? 6 : 4;  // K codes, V codes, ||k||, ||v|| (+ K signs, gamma)
+};
+
+// Issue the bulk copies of sub-chunk `sc` of the CTA (blocks [16 sc, 16 sc + 16) of its range)
+// into staging buffer `sb`, completing on `bar` (initialised with one arrival per array).  Warp
+// `arr` (< StageArrays::n) copies array `arr`.  vb[k] = first slot of the CTA's block k, or -1
+// (resolved once per CTA); nlead = number of leading valid blocks of the CTA (contiguous layout,
+// where they are one run of consecutive slots: one copy per array); paged: one copy per block.
+// `extra` bytes (landing on the same barrier, issued by the caller after this returns) are
+// expected by warp 0.
 template <int BK, int BV, bool QJL>
-__device__ __forceinline__ void stage_sub(const MmaArgs &a, int b, int h, int tk0, int tend, int64_t cap,
-                                          unsigned char *sb, int64_t *vb, uint64_t *bar, unsigned extra_bytes) {
+__device__ __forceinline__ void stage_sub(const MmaArgs &a, int sc, const int64_t *vb, int nlead,
+                                          unsigned char *sb, uint64_t *bar, unsigned extra) {
   using SM = MmaSmem<BK, BV, QJL>;
-  constexpr unsigned KB = 16 * SM::KCW * 4, SB = QJL ? 16 * 16 : 0, VB = SM::VBW * 4, NBY = 16 * 4;
-  constexpr unsigned PER_BLOCK = KB + SB + VB + NBY * (QJL ? 3 : 2);
-  const int lane = threadIdx.x & 31;
-  int64_t base = -1;
-  if (lane < SM::NB) {
-    const int tb = tk0 + 16 * lane;
-    if (tb < tend) {
-      base = token_slot(a, b, h, tb);
-      if (base < 0 || base + 16 > cap) base = -1;
-      vb[lane] = base;
-    } else {
-      vb[lane] = -1;
-    }
+  const int arr = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const char *src;
+  size_t doff;
+  unsigned per;     // bytes per block
+  int64_t sstride;  // source bytes per slot
+  switch (arr) {
+    case 0: src = static_cast<const char *>(a.k.codes); doff = SM::kc; per = 16 * SM::KCW * 4; sstride = SM::KCW * 4; break;
+    case 1: src = static_cast<const char *>(a.v.codes); doff = SM::vc; per = SM::VBW * 4; sstride = SM::VBW * 4 / 16; break;
+    case 2: src = reinterpret_cast<const char *>(a.k.norm); doff = SM::kn; per = 64; sstride = 4; break;
+    case 3: src = reinterpret_cast<const char *>(a.v.norm); doff = SM::vn; per = 64; sstride = 4; break;
+    case 4: src = static_cast<const char *>(a.k.signs); doff = SM::ks; per = 256; sstride = 16; break;
+    default: src = reinterpret_cast<const char *>(a.k.rnorm); doff = SM::kr; per = 64; sstride = 4; break;
   }
-  const unsigned valid = __ballot_sync(TQ_FULL_MASK, base >= 0);
-  int nvalid = __popc(valid);
+  // (V codes are addressed by block: slot / 16 * block bytes == slot * (block bytes / 16))
+  const int k0 = SM::NB * sc;
   if (!a.block_table) {
-    // a block past the arrays ends the run: keep the leading valid blocks only
-    nvalid = __ffs(~valid) - 1;
-    if (lane < SM::NB && lane >= nvalid) vb[lane] = -1;
-  }
-  const char *kcodes = static_cast<const char *>(a.k.codes);
-  const char *vcodes = static_cast<const char *>(a.v.codes);
-  const char *ksigns = static_cast<const char *>(a.k.signs);
-  if (!a.block_table) {
-    // contiguous: the valid blocks are the first nvalid ones, consecutive in slot space
     if (lane == 0) {
-      mbar_expect_arrive(bar, PER_BLOCK * (unsigned)nvalid + extra_bytes);
-      if (nvalid > 0) {
-        const int64_t s0 = base;
-        const unsigned n = (unsigned)nvalid;
-        bulk_g2s(sb + SM::kc, kcodes + s0 * (SM::KCW * 4), KB * n, bar);
-        bulk_g2s(sb + SM::vc, vcodes + (s0 >> 4) * (SM::VBW * 4), VB * n, bar);
-        if constexpr (QJL) bulk_g2s(sb + SM::ks, ksigns + s0 * 16, SB * n, bar);
-        bulk_g2s(sb + SM::kn, a.k.norm + s0, NBY * n, bar);
-        bulk_g2s(sb + SM::vn, a.v.norm + s0, NBY * n, bar);
-        if constexpr (QJL) bulk_g2s(sb + SM::kr, a.k.rnorm + s0, NBY * n, bar);
-      }
+      int n = nlead - k0;
+      n = n < 0 ? 0 : (n > SM::NB ? SM::NB : n);
+      mbar_expect_arrive(bar, per * (unsigned)n + (arr == 0 ? extra : 0u));
+      if (n > 0) bulk_g2s(sb + doff, src + vb[k0] * sstride, per * (unsigned)n, bar);
     }
   } else {
-    if (lane == 0) mbar_expect_arrive(bar, PER_BLOCK * (unsigned)nvalid + extra_bytes);
+    const int64_t base = lane < SM::NB ? vb[k0 + lane] : -1;
+    const unsigned valid = __ballot_sync(TQ_FULL_MASK, base >= 0);
+    if (lane == 0) mbar_expect_arrive(bar, per * (unsigned)__popc(valid) + (arr == 0 ? extra : 0u));
     __syncwarp();
-    if (base >= 0) {
-      const int kb = lane;
-      bulk_g2s(sb + SM::kc + (size_t)kb * KB, kcodes + base * (SM::KCW * 4), KB, bar);
-      bulk_g2s(sb + SM::vc + (size_t)kb * VB, vcodes + (base >> 4) * (SM::VBW * 4), VB, bar);
-      if constexpr (QJL) bulk_g2s(sb + SM::ks + (size_t)kb * SB, ksigns + base * 16, SB, bar);
-      bulk_g2s(sb + SM::kn + (size_t)kb * NBY, a.k.norm + base, NBY, bar);
-      bulk_g2s(sb + SM::vn + (size_t)kb * NBY, a.v.norm + base, NBY, bar);
-      if constexpr (QJL) bulk_g2s(sb + SM::kr + (size_t)kb * NBY, a.k.rnorm + base, NBY, bar);
-    }
+    if (base >= 0) bulk_g2s(sb + doff + (size_t)lane * per, src + base * sstride, per, bar);
   }
 }
 
@@ -417,16 +434,16 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
   constexpr int VT = BV == 3 ? 2 : 1;  // value word types: (p0,p1) and (p2, parity)
   extern __shared__ __align__(16) unsigned char smem[];
   uint32_t *sx1 = reinterpret_cast<uint32_t *>(smem + SM::x1);
-  float *lg = reinterpret_cast<float *>(smem + SM::lg);          // [kG][kSub] logits, then weights
+  float *lg = reinterpret_cast<float *>(smem + SM::lg);          // [kG][kLgS] logits, then weights
   uint4 *vfrag = reinterpret_cast<uint4 *>(smem + SM::vf);       // [NB][32]
   const uint4 *kf4 = reinterpret_cast<const uint4 *>(smem + SM::kf);  // [plane][k-step][32]
-  int64_t *vbase = reinterpret_cast<int64_t *>(smem + SM::vb);   // [2][NB]
+  int64_t *vball = reinterpret_cast<int64_t *>(smem + SM::vb);   // [MAXBLK] first slot of each block
   float *hM = reinterpret_cast<float *>(smem + SM::st);          // running max per head
   float *hL = hM + kG;                                           // running sum of e^{l - M}
-  float *hScale = hL + kG;                                       // fixed-point scale of the weights
-  float *hInv = hScale + kG;                                     // 1 / (128 hScale)
-  float *hAlpha = hInv + kG;                                     // e^{M_old - M_new}
-  int *csum = reinterpret_cast<int *>(hAlpha + kG);              // sum of the integer weights X
+  float *pmax = reinterpret_cast<float *>(smem + SM::pw);        // [kG][kWarps] max logit
+  float *psw = pmax + kG * kWarps;                               // [kG][kWarps] sum of w
+  int *pcs = reinterpret_cast<int *>(psw + kG * kWarps);         // [kG][kWarps] sum of integer weights
+  float *pnv = reinterpret_cast<float *>(pcs + kG * kWarps);     // [kWarps] max ||v|| of valid tokens
   float *obuf = reinterpret_cast<float *>(smem);                 // [4][kG][kD], after the loop
 
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -442,9 +459,23 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
 
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::br);
   int *fail = reinterpret_cast<int *>(smem + SM::br + 16);
+  int *nlead_s = fail + 1;
+  // the CTA's blocks: first slot, or -1 past the sequence or the arrays
+  const int nblk = (t1 - t0 + 15) / 16;
+  if (tid < SM::MAXBLK) {
+    int64_t base = -1;
+    if (tid < nblk) {
+      base = token_slot(a, b, h, t0 + 16 * tid);
+      if (base < 0 || base + 16 > cap) base = -1;
+    }
+    vball[tid] = base;
+    // contiguous layout: the leading run of valid blocks (consecutive slots)
+    const unsigned inval = __ballot_sync(TQ_FULL_MASK, base < 0);
+    if ((tid & 31) == 0) nlead_s[tid >> 5] = inval ? __ffs(inval) - 1 : 32;
+  }
   if (tid == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
+    mbar_init(&bars[0], StageArrays<QJL>::n);
+    mbar_init(&bars[1], StageArrays<QJL>::n);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     *fail = 0;
   }
@@ -453,14 +484,17 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
     hL[tid] = 0.f;
   }
   __syncthreads();
-  if (warp == 0 && nsub > 0) {
+  const int nlead = nlead_s[0] < 32 ? nlead_s[0] : 32 + nlead_s[1];
+  if (warp < StageArrays<QJL>::n && nsub > 0) {
     // the first sub-chunk, and the query fragments (one copy per CTA) on the same barrier
     constexpr unsigned FB = KP::regs * 32 * 4;
-    stage_sub<BK, BV, QJL>(a, b, h, t0, t1, cap, smem, vbase, &bars[0], FB);
-    if (lane == 0) bulk_g2s(smem + SM::kf, kfrag + grp * KP::regs * 32, FB, &bars[0]);
+    stage_sub<BK, BV, QJL>(a, 0, vball, nlead, smem, &bars[0], FB);
+    if (warp == 0 && lane == 0) bulk_g2s(smem + SM::kf, kfrag + grp * KP::regs * 32, FB, &bars[0]);
   }
-  const float cfc = kconst[grp * 16 + t], cfs = kconst[grp * 16 + 4 + t];
-  const float cq = kconst[grp * 16 + 8 + t], cp = kconst[grp * 16 + 12 + t];
+  // the query constants (2^-F_code, 2^-F_sign, Cq, Cp per head), read from shared memory where
+  // used (published by the first sub-chunk's barrier)
+  float *kcs = hL + kG;  // [16]
+  if (tid < 16) kcs[tid] = kconst[grp * 16 + tid];
 
   // value accumulators of this thread: head t, coordinates jb + 2 mt + r
   const int ch = warp & 1, bgrp = warp >> 1;
@@ -472,9 +506,8 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
   for (int sc = 0; sc < nsub; ++sc) {
     const int cur = sc & 1;
     const int tk0 = t0 + sc * kSub;
-    if (warp == 0 && sc + 1 < nsub)
-      stage_sub<BK, BV, QJL>(a, b, h, tk0 + kSub, t1, cap, smem + (cur ^ 1) * SM::buf, vbase + (cur ^ 1) * NB,
-                             &bars[cur ^ 1], 0u);
+    if (warp < StageArrays<QJL>::n && sc + 1 < nsub)
+      stage_sub<BK, BV, QJL>(a, sc + 1, vball, nlead, smem + (cur ^ 1) * SM::buf, &bars[cur ^ 1], 0u);
     if (!mbar_wait_bounded(&bars[cur], (unsigned)(sc >> 1) & 1u)) *fail = 1;
     __syncthreads();
     if (*fail) {
@@ -495,7 +528,7 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
     const float *skr = reinterpret_cast<const float *>(sb + SM::kr);
     const uint32_t *svc = reinterpret_cast<const uint32_t *>(sb + SM::vc);
     const float *svn = reinterpret_cast<const float *>(sb + SM::vn);
-    const int64_t *vb = vbase + cur * NB;
+    const int64_t *vb = vball + NB * sc;  // validity of this sub-chunk's blocks
 
     // ------------------------------------------------------------ phase 1: logits (keys x heads)
     {
@@ -537,6 +570,7 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
           }
         }
       }
+      float lmax = -INFINITY, nvmax = 0.f;
 #pragma unroll
       for (int kb = 0; kb < 2; ++kb) {
         const int blk = 2 * warp + kb;
@@ -546,83 +580,80 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
           const int i = blk * 16 + gid + 8 * r;
           const float dc = (float)acc[kb][0][0][2 * r] + 256.f * (float)acc[kb][0][0][2 * r + 1] +
                            65536.f * (float)acc[kb][0][1][2 * r] + 16777216.f * (float)acc[kb][0][1][2 * r + 1];
-          float sc2 = fmaf(dc, cfc, -cq);
+          float sc2 = fmaf(dc, kcs[t], -kcs[8 + t]);
           if constexpr (QJL) {
             const float ds = (float)acc[kb][1][0][2 * r] + 256.f * (float)acc[kb][1][0][2 * r + 1] +
                              65536.f * (float)acc[kb][1][1][2 * r] + 16777216.f * (float)acc[kb][1][1][2 * r + 1];
-            sc2 = fmaf(kc.qjl_scale * skr[i], fmaf(ds, cfs, -cp), sc2);
+            sc2 = fmaf(kc.qjl_scale * skr[i], fmaf(ds, kcs[4 + t], -kcs[12 + t]), sc2);
           }
-          lg[t * kSub + i] = (bok && tk0 + i < t1) ? a.scale * skn[i] * sc2 : -INFINITY;
+          const bool ok = bok && tk0 + i < t1;
+          const float lgt = ok ? a.scale * skn[i] * sc2 : -INFINITY;
+          lg[t * kLgS + i] = lgt;
+          lmax = fmaxf(lmax, lgt);
+          if (ok) nvmax = fmaxf(nvmax, svn[i]);
         }
       }
+      // this warp's largest logit per head (lanes sharing t hold the same head)
+#pragma unroll
+      for (int m = 4; m <= 16; m <<= 1) {
+        lmax = fmaxf(lmax, __shfl_xor_sync(TQ_FULL_MASK, lmax, m));
+        nvmax = fmaxf(nvmax, __shfl_xor_sync(TQ_FULL_MASK, nvmax, m));
+      }
+      if (gid == 0) pmax[t * kWarps + warp] = lmax;
+      if (lane == 0) pnv[warp] = nvmax;
     }
     __syncthreads();
 
-    // ------------------------------------------------------------ phase 2: softmax weights
-    if (warp < kG) {
-      // warp g: running max, weights w = e^{l - M}, W = w ||v||, running sum, max and sum of W
-      const int g = warp;
-      float mx = -INFINITY;
-      for (int i = lane; i < kSub; i += 32) mx = fmaxf(mx, lg[g * kSub + i]);
-      mx = warp_max_f(mx);
-      const float Mold = hM[g];
-      const float Mnew = fmaxf(Mold, mx);
-      float sw = 0.f, mW = 0.f;
-      for (int i = lane; i < kSub; i += 32) {
-        const float l = lg[g * kSub + i];
-        const float wgt = l == -INFINITY ? 0.f : __expf(l - Mnew);
-        const float W = l == -INFINITY ? 0.f : wgt * svn[i];  // masked slots may hold stale bytes
-        lg[g * kSub + i] = W;
-        sw += wgt;
-        mW = fmaxf(mW, W);
-      }
-      sw = warp_sum_f(sw);
-      mW = warp_max_f(mW);
-      if (lane == 0) {
-        const float alpha = Mnew == -INFINITY ? 1.f : __expf(Mold - Mnew);
-        // integer weights X = floor(W 2 e_P scale + dither) < 2^16 for every plane P
-        const float top = mW * 2.f * vc.plane_coef_max;
-        int e = 0;
-        frexpf(top, &e);  // top < 2^e
-        const float sc = top > 0.f ? ldexpf(1.f - 1.f / 512.f, 16 - e) : 1.f;
-        hM[g] = Mnew;
-        hL[g] = hL[g] * alpha + sw;
-        hAlpha[g] = alpha;
-        hScale[g] = sc;
-        hInv[g] = 1.f / (128.f * sc);
-        csum[g] = 0;
-      }
-    } else if constexpr (BV == 3) {
-      // warps 4-7: (plane 2, parity) words, parity = p0 ^ p1 ^ p2, one coordinate per thread
-      const int j = tid - kG * 32;
-      const int sh = 16 * (j & 1);
-#pragma unroll 4
-      for (int kb = 0; kb < NB; ++kb) {
-        const uint32_t A = svc[kb * SM::VBW + j];
-        const uint32_t hw = svc[kb * SM::VBW + kD + (j >> 1)] >> sh;
-        const uint32_t par = A ^ (A >> 16) ^ hw;
-        sx1[kb * SM::X1W + j] = __byte_perm(hw, par, 0x5410);
-      }
-    }
-    __syncthreads();
+    // ------------------------------------------------------------ phase 2: weights, value fragments
+    // Each warp weights its own two blocks (tokens 32 w ..) and builds their value-MMA B
+    // fragments; the fixed-point scale comes from the sub-chunk's largest ||v|| (W <= ||v||
+    // since w <= 1), so no cross-warp step is needed in between.
     {
+      const int g = lane & 3;  // lane = (head lane & 3, tokens lane / 4 + 8 k)
+      const float Mnew = fmaxf(hM[g], max8(pmax + g * kWarps));
+      float sw = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int i = 32 * warp + (lane >> 2) + 8 * k;
+        const float l = lg[g * kLgS + i];
+        const float wgt = l == -INFINITY ? 0.f : __expf(l - Mnew);
+        lg[g * kLgS + i] = l == -INFINITY ? 0.f : wgt * svn[i];  // masked slots may hold stale bytes
+        sw += wgt;
+      }
+#pragma unroll
+      for (int m = 4; m <= 16; m <<= 1) sw += __shfl_xor_sync(TQ_FULL_MASK, sw, m);
+      if (lane < kG) psw[g * kWarps + warp] = sw;
+      if constexpr (BV == 3) {
+        // (plane 2, parity) words of this warp's two blocks, parity = p0 ^ p1 ^ p2
+#pragma unroll
+        for (int k = 0; k < 2 * kD / 32; ++k) {
+          const int idx = lane + 32 * k;
+          const int kb = 2 * warp + (idx >> 7), j = idx & (kD - 1);
+          const uint32_t A = svc[kb * SM::VBW + j];
+          const uint32_t hw = svc[kb * SM::VBW + kD + (j >> 1)] >> (16 * (j & 1));
+          const uint32_t par = A ^ (A >> 16) ^ hw;
+          sx1[kb * SM::X1W + j] = __byte_perm(hw, par, 0x5410);
+        }
+      }
+      __syncwarp();
       // B fragments of the value MMAs.  Lane (gid, t): column = (head gid/2, limb gid&1).  The
       // k index runs over (token, plane) pairs in the order the value words give them:
       // register 0 = tokens t, t+8 of the low plane, then of the high plane; register 1 = the
-      // same for tokens t+4, t+12.  Byte = limb of X = floor(W 2 e_P 2^F + dither), dithered so
+      // same for tokens t+4, t+12.  Byte = limb of X = floor(W 2 e_P sc + dither), dithered so
       // that the many sub-unit tail weights are unbiased rather than all rounded down.
-      const int g = gid >> 1, l = gid & 1;
-      const float S2 = 2.f * hScale[g];
+      const int gh = gid >> 1, l = gid & 1;
+      float sc, inv;
+      weight_scale(max8(pnv) * 2.f * vc.plane_coef_max, sc, inv);
       float C[2 * VT];
 #pragma unroll
-      for (int P = 0; P < 2 * VT; ++P) C[P] = S2 * vc.plane_coef[P];
+      for (int P = 0; P < 2 * VT; ++P) C[P] = 2.f * sc * vc.plane_coef[P];
       const uint32_t sel = (uint32_t)l | ((uint32_t)(4 + l) << 4);  // byte l of two words
-      const uint32_t key0 = ((uint32_t)grp * (uint32_t)a.max_len + (uint32_t)tk0) * 4u + (uint32_t)g;
+      const uint32_t key0 = ((uint32_t)grp * (uint32_t)a.max_len + (uint32_t)tk0) * 4u + (uint32_t)gh;
       uint32_t xs = 0;  // sum of this lane's X values
 #pragma unroll
-      for (int kk = 0; kk < NB / kWarps; ++kk) {
-        const int kb = warp + kWarps * kk;
-        const float *wr = &lg[g * kSub + kb * 16];
+      for (int kk = 0; kk < 2; ++kk) {
+        const int kb = 2 * warp + kk;
+        const float *wr = &lg[gh * kLgS + kb * 16];
         const int toks[4] = {t, t + 8, t + 4, t + 12};
         float W[4], dz[4];
 #pragma unroll
@@ -651,7 +682,7 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
       mine += __shfl_xor_sync(TQ_FULL_MASK, mine, 1);
       mine += __shfl_xor_sync(TQ_FULL_MASK, mine, 2);
       mine += __shfl_xor_sync(TQ_FULL_MASK, mine, 4);
-      if (t == 0 && l == 0) atomicAdd(&csum[g], (int)mine);
+      if (t == 0 && l == 0) pcs[gh * kWarps + warp] = (int)mine;
     }
     __syncthreads();
 
@@ -700,8 +731,14 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
       // accv[mt][x][c]: c0/c1 = (coordinate jb + 2 mt, head t, limb 0/1), c2/c3 = (+1, ...):
       // 128 sum_tok X b over the word type's two planes.  With s = 2b - 1 the codebook's
       // constant term is -(1/2) sum X, added once per sub-chunk by the bgrp 0 warps.
-      const float al = hAlpha[t], inv = hInv[t];
-      const float cterm = bgrp == 0 ? 64.f * (float)csum[t] : 0.f;
+      const float Mold = hM[t], Mnew = fmaxf(Mold, max8(pmax + t * kWarps));
+      const float al = Mnew == -INFINITY ? 1.f : __expf(Mold - Mnew);
+      float sct, inv;
+      weight_scale(max8(pnv) * 2.f * vc.plane_coef_max, sct, inv);
+      int cs = 0;
+#pragma unroll
+      for (int w2 = 0; w2 < kWarps; ++w2) cs += pcs[t * kWarps + w2];
+      const float cterm = bgrp == 0 ? 64.f * (float)cs : 0.f;
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
@@ -712,7 +749,19 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
           o[mt][r] = fmaf(o[mt][r], al, (v - cterm) * inv);
         }
     }
-    __syncthreads();  // the buffers, lg, vfrag and the head statistics are reused next
+    __syncthreads();  // the buffers, lg, vfrag and the per-warp partials are reused next
+    if (warp == kWarps - 1 && lane < kG) {
+      // head `lane`'s running maximum and sum, from this sub-chunk's per-warp partials (read
+      // before the next sub-chunk's phase 1 rewrites them, published by its first barrier);
+      // the last warp does it, as it issues no copies
+      const float Mold = hM[lane], Mnew = fmaxf(Mold, max8(pmax + lane * kWarps));
+      const float al = Mnew == -INFINITY ? 1.f : __expf(Mold - Mnew);
+      float swh = 0.f;
+#pragma unroll
+      for (int w2 = 0; w2 < kWarps; ++w2) swh += psw[lane * kWarps + w2];
+      hM[lane] = Mnew;
+      hL[lane] = hL[lane] * al + swh;
+    }
   }
 
   // ---------------------------------------------------------------- partials of the 4 heads
@@ -726,13 +775,84 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
     const int g = i / kD, j = i % kD;
     const float v = obuf[(0 * kG + g) * kD + j] + obuf[(1 * kG + g) * kD + j] + obuf[(2 * kG + g) * kD + j] +
                     obuf[(3 * kG + g) * kD + j];
-    const int64_t pb = (((int64_t)b * a.hq + (int64_t)h * kG + g) * a.splits + s) * (kD + 2);
+    const int64_t pb = (((int64_t)b * a.hq + (int64_t)h * kG + g) * a.splits + s) * (kD + 4);
     part[pb + 2 + j] = v;
   }
   if (tid < kG) {
-    const int64_t pb = (((int64_t)b * a.hq + (int64_t)h * kG + tid) * a.splits + s) * (kD + 2);
+    const int64_t pb = (((int64_t)b * a.hq + (int64_t)h * kG + tid) * a.splits + s) * (kD + 4);
     part[pb] = hM[tid];
     part[pb + 1] = hL[tid];
+  }
+  if (a.out == nullptr) return;
+
+  // ---------------------------------------------------------------- merge (last CTA of the group)
+  // The last CTA of this (sequence, KV head) to finish merges the splits of its 4 heads with
+  // their log-sum-exp weights and undoes the rotation once:
+  //   o = D_V (1/sqrt d) H (sum_s e^{m_s - M} o~_s) / (sum_s e^{m_s - M} l_s).
+  __threadfence();
+  __syncthreads();
+  int *last = nlead_s + 2;
+  if (tid == 0) *last = atomicAdd(&a.counter[grp], 1) == a.splits - 1;
+  __syncthreads();
+  if (!*last) return;
+  __threadfence();
+  // The group's partial rows (kD + 4 floats: m, l, o~, pad) pass through shared memory in
+  // batches of up to `nb` splits (cp.async, one round trip per batch), merged online per head.
+  constexpr int PR = kD + 4;
+  float *y = reinterpret_cast<float *>(smem);  // [kG][kD]
+  float *stg = y + kG * kD;                     // [kG][nb][PR]
+  const int nb = (int)((SM::vb - (size_t)kG * kD * 4) / ((size_t)kG * PR * 4));
+  const int64_t pg = ((int64_t)b * a.hq + (int64_t)h * kG) * a.splits * PR;
+  const int g = tid >> 6, jj = tid & 63;  // head, coordinates jj and jj + 64
+  float M = -INFINITY, Lsum = 0.f, acc0 = 0.f, acc1 = 0.f;
+  for (int s0 = 0; s0 < a.splits; s0 += nb) {
+    const int n = min(nb, a.splits - s0);
+    constexpr int GR = PR * 4 / 16;  // 16-byte granules per row
+    for (int idx = tid; idx < kG * n * GR; idx += kThreads) {
+      const int row = idx / GR, gr = idx - row * GR;  // row = head * n + split
+      const int hg = row / n, sp = row - hg * n;
+      cp_async16(stg + (size_t)row * PR + 4 * gr, part + pg + ((int64_t)hg * a.splits + s0 + sp) * PR + 4 * gr);
+    }
+    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
+    __syncthreads();
+    const float *rows = stg + (size_t)g * n * PR;
+    float Mb = M;
+    for (int sp = 0; sp < n; ++sp) Mb = fmaxf(Mb, rows[sp * PR]);
+    if (Mb != -INFINITY) {
+      const float r = __expf(M - Mb);  // 0 while M is -inf
+      acc0 *= r;
+      acc1 *= r;
+      Lsum *= r;
+      M = Mb;
+#pragma unroll 4
+      for (int sp = 0; sp < n; ++sp) {
+        const float ms = rows[sp * PR];
+        const float f = ms == -INFINITY ? 0.f : __expf(ms - M);
+        Lsum = fmaf(f, rows[sp * PR + 1], Lsum);
+        acc0 = fmaf(f, rows[sp * PR + 2 + jj], acc0);
+        acc1 = fmaf(f, rows[sp * PR + 2 + jj + 64], acc1);
+      }
+    }
+    __syncthreads();  // the batch buffer is refilled next
+  }
+  {
+    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+    y[g * kD + jj] = acc0 * inv;
+    y[g * kD + jj + 64] = acc1 * inv;
+  }
+  __syncthreads();
+  for (int hh = 1; hh < kD; hh <<= 1) {
+    const int g = tid >> 6, i = tid & 63;  // 4 heads x 64 butterflies
+    const int lo = (i / hh) * 2 * hh + (i % hh);
+    const float u = y[g * kD + lo], v = y[g * kD + lo + hh];
+    __syncthreads();
+    y[g * kD + lo] = u + v;
+    y[g * kD + lo + hh] = u - v;
+    __syncthreads();
+  }
+  for (int i = tid; i < kG * kD; i += kThreads) {
+    const int g = i / kD, j = i % kD;
+    a.out[((int64_t)b * a.hq + (int64_t)h * kG + g) * kD + j] = vc.signs[j] * y[i] * vc.inv_sqrt_d;
   }
 }
 
@@ -757,7 +877,7 @@ cudaError_t launch_fast(const TqConsts &kc, const TqConsts &vc, const MmaArgs &a
     if (e0 != cudaSuccess) return e0;
   }
   tq_prof_begin(TQK_ATTEND_FRAG, st);
-  kfrag_kernel<BK, QJL><<<groups, kThreads, fsm, st>>>(kc, q, dtype, kfrag, kconst);
+  kfrag_kernel<BK, QJL><<<groups, kThreads, fsm, st>>>(kc, q, dtype, kfrag, kconst, a.counter);
   tq_prof_end(TQK_ATTEND_FRAG, st);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -806,12 +926,13 @@ int attn_fast_chunk(const tq_attn_desc &desc) {
 size_t attn_fast_extra_bytes(const TqConsts &kc, const tq_attn_desc &desc) {
   const int planes = (kc.bits + (kc.bits == 3 ? 1 : 0)) + (kc.m > 0 ? 1 : 0);
   const int64_t groups = (int64_t)desc.batch * desc.n_kv_heads;
-  return (size_t)tq_align_up(groups * planes * 16 * 32 * 4, 256) + (size_t)tq_align_up(groups * 16 * 4, 256);
+  return (size_t)tq_align_up(groups * planes * 16 * 32 * 4, 256) + (size_t)tq_align_up(groups * 16 * 4, 256) +
+         (size_t)tq_align_up(groups * 4, 256);
 }
 
 cudaError_t launch_attend_fast(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc,
                                const AttnPlan &plan, const void *q, int dtype, void *extra,
-                               float *partials, cudaStream_t st) {
+                               float *partials, float *out, cudaStream_t st) {
   MmaArgs a;
   a.hq = desc.n_q_heads;
   a.hkv = desc.n_kv_heads;
@@ -831,6 +952,8 @@ cudaError_t launch_attend_fast(const TqConsts &kc, const TqConsts &vc, const tq_
   uint32_t *kfrag = static_cast<uint32_t *>(extra);
   float *kconst = reinterpret_cast<float *>(static_cast<char *>(extra) +
                                             tq_align_up(groups * planes * 16 * 32 * 4, 256));
+  a.counter = reinterpret_cast<int *>(reinterpret_cast<char *>(kconst) + tq_align_up(groups * 16 * 4, 256));
+  a.out = out;
   const bool qjl = kc.m > 0;
 #define TQ_FAST(BKV, BVV, Q)                                                                           \
   if (kc.bits == BKV && vc.bits == BVV && qjl == Q)                                                    \
@@ -858,7 +981,7 @@ cudaError_t launch_step(const TqConsts &kc, const TqConsts &vc, const MmaArgs &a
   }
   tq_prof_begin(TQK_DECODE_PREP, st);
   decode_prep_kernel<BK, QJL><<<grid0, kThreads, fsm, st>>>(kc, vc, knew, vnew, kvdtype, nnew, slots, a.k, a.v, q,
-                                                            qdtype, kfrag, kconst, nb, nb);
+                                                            qdtype, kfrag, kconst, a.counter, nb, nb);
   tq_prof_end(TQK_DECODE_PREP, st);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -873,7 +996,7 @@ cudaError_t launch_step(const TqConsts &kc, const TqConsts &vc, const MmaArgs &a
 cudaError_t launch_decode_step_fast(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc,
                                     const AttnPlan &plan, const void *knew, const void *vnew, int kvdtype,
                                     int64_t nnew, const int64_t *slots, const void *q, int qdtype, void *extra,
-                                    float *partials, cudaStream_t st) {
+                                    float *partials, float *out, cudaStream_t st) {
   MmaArgs a;
   a.hq = desc.n_q_heads;
   a.hkv = desc.n_kv_heads;
@@ -893,6 +1016,8 @@ cudaError_t launch_decode_step_fast(const TqConsts &kc, const TqConsts &vc, cons
   uint32_t *kfrag = static_cast<uint32_t *>(extra);
   float *kconst = reinterpret_cast<float *>(static_cast<char *>(extra) +
                                             tq_align_up(groups * planes * 16 * 32 * 4, 256));
+  a.counter = reinterpret_cast<int *>(reinterpret_cast<char *>(kconst) + tq_align_up(groups * 16 * 4, 256));
+  a.out = out;
   const bool qjl = kc.m > 0;
 #define TQ_STEP(BKV, BVV, Q)                                                                                   \
   if (kc.bits == BKV && vc.bits == BVV && qjl == Q)                                                            \

@@ -90,7 +90,8 @@ struct AttnPlan {
   int chunk;        // tokens per split
   int splits;       // splits per (batch, kv head)
   bool fast;        // tensor-core path (attend_mma.cu)
-  size_t extra;     // workspace bytes of the tensor-core path's query fragments
+  bool fused;       // tensor-core path merges the splits itself (no combine launch)
+  size_t extra;     // workspace bytes of the tensor-core path's query fragments and counters
 };
 AttnPlan attn_plan(const tq_attn_desc &desc, const TqConsts &kc, const TqConsts &vc);
 size_t attn_partials_bytes(const tq_attn_desc &desc, const AttnPlan &plan, int d);
@@ -100,16 +101,18 @@ cudaError_t launch_attend(const TqConsts &kc, const TqConsts &vc, const tq_attn_
 // attend_mma.cu
 bool attn_fast_eligible(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc);
 int attn_fast_chunk(const tq_attn_desc &desc);
+constexpr int kFusedMaxSplits = 1024;  // splits merged inside the tensor-core kernel at most
 size_t attn_fast_extra_bytes(const TqConsts &kc, const tq_attn_desc &desc);
 cudaError_t launch_attend_fast(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc,
                                const AttnPlan &plan, const void *q, int dtype, void *extra,
-                               float *partials, cudaStream_t st);
+                               float *partials, float *out, cudaStream_t st);
 // Fused decode step (tensor-core path): append-encode nnew K and V rows at `slots`, build the
-// query fragments, run the split kernel (the caller then launches the combine).
+// query fragments, run the split kernel (which merges the splits when plan.fused; otherwise the
+// caller then launches the combine).
 cudaError_t launch_decode_step_fast(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc,
                                     const AttnPlan &plan, const void *knew, const void *vnew, int kvdtype,
                                     int64_t nnew, const int64_t *slots, const void *q, int qdtype, void *extra,
-                                    float *partials, cudaStream_t st);
+                                    float *partials, float *out, cudaStream_t st);
 cudaError_t launch_attend_combine(const TqConsts &vc, const tq_attn_desc &desc, const AttnPlan &plan,
                                   const float *partials, float *out, cudaStream_t st);
 
