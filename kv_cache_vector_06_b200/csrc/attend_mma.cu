@@ -79,13 +79,6 @@ __device__ __forceinline__ int64_t token_slot(const MmaArgs &a, int b, int h, in
   return ((int64_t)b * a.hkv + h) * a.ctx_stride + t;
 }
 
-// Signed byte limbs of v = l0 + 2^8 l1 + 2^16 l2 + 2^24 l3, each l in [-128, 127].
-__device__ __forceinline__ int next_limb(int &v) {
-  const int l = ((v + 128) & 255) - 128;
-  v = (v - l) >> 8;
-  return l;
-}
-
 __device__ __forceinline__ float warp_max_f(float x) {
 #pragma unroll
   for (int s = 16; s >= 1; s >>= 1) x = fmaxf(x, __shfl_xor_sync(TQ_FULL_MASK, x, s));
@@ -120,6 +113,8 @@ __device__ __forceinline__ void kfrag_group(const TqConsts &kc, const void *__re
   __shared__ int fexp[kG][2];
   // grp = b * hkv + h; its query heads are rows grp * 4 + g
   const int tid = threadIdx.x;
+  // S (for p = S q') is copied asynchronously while q' is formed
+  if constexpr (QJL) stage_rows_padded_async(sS, kc.S, kD, kD);
   // q' = (1/sqrt d) H (D q): load with the signs applied, then the butterflies in shared memory
   for (int i = tid; i < kG * kD; i += kThreads) {
     const int g = i / kD, j = i % kD;
@@ -150,7 +145,7 @@ __device__ __forceinline__ void kfrag_group(const TqConsts &kc, const void *__re
   if constexpr (QJL) {
     // p = S q' for the 4 heads: S staged in shared memory (row stride kD + 4), thread (row i,
     // head pair) dots row i with two q'
-    stage_rows_padded(sS, kc.S, kD, kD);
+    stage_async_wait();
     __syncthreads();
     const int i = tid & (kD - 1), gp = tid >> 7;
     const float4 *Srow = reinterpret_cast<const float4 *>(sS + i * (kD + 4));
@@ -195,8 +190,8 @@ __device__ __forceinline__ void kfrag_group(const TqConsts &kc, const void *__re
       // |X| 2^F <= 2^30: four signed byte limbs
       fexp[g][0] = mc > 0.f ? 30 - ec : 0;
       fexp[g][1] = ms > 0.f ? 30 - es : 0;
-      red[g][0] = ldexpf(1.f, -fexp[g][0]);
-      red[g][1] = ldexpf(1.f, -fexp[g][1]);
+      red[g][0] = pow2i(-fexp[g][0]);
+      red[g][1] = pow2i(-fexp[g][1]);
       red[g][2] = kc.plane_coef_sum * sq;
       red[g][3] = sp;
     }
@@ -205,7 +200,9 @@ __device__ __forceinline__ void kfrag_group(const TqConsts &kc, const void *__re
   if (tid < 16) kconst[(int64_t)grp * 16 + tid] = red[tid % 4][tid / 4];
   if (tid == 0) counter[grp] = 0;  // the split kernel that follows counts its finished CTAs here
   uint32_t *out = kfrag + (int64_t)grp * KP::regs * 32;
-  // layout [plane][k-step][lane][n-tile, register]: one 16-byte load per lane and k-step
+  // layout [plane][k-step][lane][n-tile, register]: one 16-byte load per lane and k-step.
+  // Balanced byte limbs: with w = v + 0x80808080 (mod 2^32), limb k of v = byte k of w - 128,
+  // stored as its two's-complement byte, byte k of w ^ 0x80.
   for (int idx = tid; idx < KP::regs * 32; idx += kThreads) {
     const int r = idx & 1;
     const int nt = (idx >> 1) & 1;
@@ -214,22 +211,12 @@ __device__ __forceinline__ void kfrag_group(const TqConsts &kc, const void *__re
     const int P = idx >> 9;
     const int gid = ln >> 2, t = ln & 3;
     const int g = gid >> 1, limb = (gid & 1) + 2 * nt;
-    const int shift = s + 4 * r;
-    const int F = fexp[g][(QJL && P == KP::code) ? 1 : 0];
-    uint32_t word = 0u;
+    const float sc = pow2i(fexp[g][(QJL && P == KP::code) ? 1 : 0] - s - 4 * r);
+    const uint32_t sel = (uint32_t)limb | ((uint32_t)(4 + limb) << 4);  // byte `limb` of two words
+    uint32_t w[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int j = 32 * t + s + 4 * r + 8 * i;
-      int v = __float2int_rn(ldexpf(X[P][g][j], F - shift));
-      int l = 0;
-#pragma unroll
-      for (int k = 0; k <= 3; ++k) {
-        const int li = next_limb(v);
-        if (k == limb) l = li;
-      }
-      word |= (uint32_t)(l & 255) << (8 * i);
-    }
-    out[idx] = word;
+    for (int i = 0; i < 4; ++i) w[i] = (uint32_t)__float2int_rn(X[P][g][32 * t + s + 4 * r + 8 * i] * sc) + 0x80808080u;
+    out[idx] = __byte_perm(__byte_perm(w[0], w[1], sel), __byte_perm(w[2], w[3], sel), 0x5410) ^ 0x80808080u;
   }
 }
 
@@ -264,15 +251,6 @@ decode_prep_kernel(TqConsts kc, TqConsts vc, const void *__restrict__ knew, cons
   }
 }
 
-// Device-side status word of the library (bits of tq_device_status): set by a kernel that gave up
-// waiting, read and cleared from the host by tq_device_status.
-__device__ int g_tq_device_flags;
-constexpr int kFlagStagingTimeout = 1;
-
-// Bulk asynchronous copies (global -> this CTA's shared memory) completing on an mbarrier, and
-// the bounded wait for them.  Addresses 16-byte aligned, sizes multiples of 16 bytes.
-// 2^e as a float for e in [-126, 127].
-__device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
 // Fixed-point scale of a sub-chunk's value weights: with top = max W * 2 max_P e_P, the integer
 // weights floor(W 2 e_P sc + dither) stay below 2^16.  Returns sc and 1 / (128 sc).
 __device__ __forceinline__ void weight_scale(float top, float &sc, float &inv128) {
@@ -299,40 +277,9 @@ __device__ __forceinline__ uint32_t mul_lo(uint32_t x, uint32_t m) {
   asm("mul.lo.u32 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(m));
   return r;
 }
-__device__ __forceinline__ unsigned smem_addr(const void *p) { return (unsigned)__cvta_generic_to_shared(p); }
 // 16-byte asynchronous global -> shared copy through L2 (the partial rows other CTAs wrote).
 __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_addr(smem_dst)), "l"(gmem) : "memory");
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t *bar, unsigned count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_arrive(uint64_t *bar, unsigned bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, unsigned bytes, uint64_t *bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
-                   smem_addr(dst)),
-               "l"(src), "r"(bytes), "r"(smem_addr(bar))
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned parity) {
-  unsigned ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Wait for phase `parity` of `bar` to complete, giving up after about a second (each try_wait
-// suspends for a bounded, hardware-defined time).
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, unsigned parity) {
-  for (int i = 0; i < (1 << 22); ++i)
-    if (mbar_try_wait(bar, parity)) return true;
-  return false;
 }
 
 constexpr int kSub = 256;          // tokens per sub-chunk (one staging buffer)
@@ -366,7 +313,7 @@ struct MmaSmem {
   static constexpr size_t st = vb + (size_t)MAXBLK * 8;
   static constexpr size_t pw = st + 16 * kG * 4;  // per-warp partials (max logit, sum w, sum X, max ||v||)
   static constexpr size_t br = pw + 4 * kG * kWarps * 4;  // two mbarriers, one per staging buffer
-  static constexpr size_t total = br + 2 * 8 + 16;
+  static constexpr size_t total = br + 48;  // + flags at br + 16, merge barrier at br + 32
   static_assert((size_t)4 * kG * kD * 4 <= 2 * buf, "the value-sum buffer reuses the staging buffers");
   static_assert(buf % 16 == 0 && x1 % 16 == 0 && kf % 16 == 0, "16-byte aligned regions");
 };
@@ -476,6 +423,7 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
   if (tid == 0) {
     mbar_init(&bars[0], StageArrays<QJL>::n);
     mbar_init(&bars[1], StageArrays<QJL>::n);
+    mbar_init(&bars[4], 1);  // the merge's copies (br + 32)
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     *fail = 0;
   }
@@ -789,70 +737,114 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
   // The last CTA of this (sequence, KV head) to finish merges the splits of its 4 heads with
   // their log-sum-exp weights and undoes the rotation once:
   //   o = D_V (1/sqrt d) H (sum_s e^{m_s - M} o~_s) / (sum_s e^{m_s - M} l_s).
-  __threadfence();
+  // release: the barrier orders every thread's partial stores before thread 0's fence, which
+  // (cumulatively) orders them before the count at device scope
   __syncthreads();
   int *last = nlead_s + 2;
-  if (tid == 0) *last = atomicAdd(&a.counter[grp], 1) == a.splits - 1;
+  if (tid == 0) {
+    __threadfence();
+    *last = atomicAdd(&a.counter[grp], 1) == a.splits - 1;
+    if (*last) {
+      __threadfence();  // acquire: the other CTAs' partials are read after this ...
+      asm volatile("fence.proxy.async.global;\n" ::: "memory");  // ... by the bulk copies too
+    }
+  }
   __syncthreads();
   if (!*last) return;
-  __threadfence();
   // The group's partial rows (kD + 4 floats: m, l, o~, pad) pass through shared memory in
-  // batches of up to `nb` splits (cp.async, one round trip per batch), merged online per head.
+  // batches of up to `nb` splits (cp.async through L2, one round trip per batch).  Warps g and
+  // g + 4 merge head g online over the even and the odd splits, lane holding coordinates
+  // lane + 32 k; warp g then folds in warp g + 4's share.
   constexpr int PR = kD + 4;
-  float *y = reinterpret_cast<float *>(smem);  // [kG][kD]
-  float *stg = y + kG * kD;                     // [kG][nb][PR]
-  const int nb = (int)((SM::vb - (size_t)kG * kD * 4) / ((size_t)kG * PR * 4));
+  float *stg = reinterpret_cast<float *>(smem);  // [kG][nb][PR]
+  const int nb = (int)(SM::vb / ((size_t)kG * PR * 4));
   const int64_t pg = ((int64_t)b * a.hq + (int64_t)h * kG) * a.splits * PR;
-  const int g = tid >> 6, jj = tid & 63;  // head, coordinates jj and jj + 64
-  float M = -INFINITY, Lsum = 0.f, acc0 = 0.f, acc1 = 0.f;
+  const int hg = warp & (kG - 1), par = warp >> 2;
+  float sgn[4];  // the rotation signs of this lane's output coordinates, loaded early
+#pragma unroll
+  for (int k = 0; k < 4; ++k) sgn[k] = vc.signs[lane + 32 * k] * vc.inv_sqrt_d;
+  float M = -INFINITY, Lsum = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
   for (int s0 = 0; s0 < a.splits; s0 += nb) {
     const int n = min(nb, a.splits - s0);
-    constexpr int GR = PR * 4 / 16;  // 16-byte granules per row
-    for (int idx = tid; idx < kG * n * GR; idx += kThreads) {
-      const int row = idx / GR, gr = idx - row * GR;  // row = head * n + split
-      const int hg = row / n, sp = row - hg * n;
-      cp_async16(stg + (size_t)row * PR + 4 * gr, part + pg + ((int64_t)hg * a.splits + s0 + sp) * PR + 4 * gr);
-    }
-    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
+    // each head's n rows are contiguous in the partials: one bulk copy per head
+    if (tid == 0) mbar_expect_arrive(&bars[4], (unsigned)(kG * n * PR * 4));
     __syncthreads();
-    const float *rows = stg + (size_t)g * n * PR;
+    if (tid < kG)
+      bulk_g2s(stg + (size_t)tid * n * PR, part + pg + ((int64_t)tid * a.splits + s0) * PR, (unsigned)(n * PR * 4),
+               &bars[4]);
+    if (!__syncthreads_and(mbar_wait_bounded(&bars[4], (unsigned)(s0 / nb) & 1u))) {
+      if (tid == 0) {
+        atomicOr(&g_tq_device_flags, kFlagStagingTimeout);
+        mbar_wait_bounded(&bars[4], (unsigned)(s0 / nb) & 1u);
+      }
+      __syncthreads();
+      return;
+    }
+    const float *rows = stg + (size_t)hg * n * PR;
     float Mb = M;
-    for (int sp = 0; sp < n; ++sp) Mb = fmaxf(Mb, rows[sp * PR]);
+    for (int sp = par; sp < n; sp += 2) Mb = fmaxf(Mb, rows[sp * PR]);
     if (Mb != -INFINITY) {
       const float r = __expf(M - Mb);  // 0 while M is -inf
-      acc0 *= r;
-      acc1 *= r;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[k] *= r;
       Lsum *= r;
       M = Mb;
-#pragma unroll 4
-      for (int sp = 0; sp < n; ++sp) {
-        const float ms = rows[sp * PR];
+#pragma unroll 2
+      for (int sp = par; sp < n; sp += 2) {
+        const float *row = rows + sp * PR;
+        const float ms = row[0];
         const float f = ms == -INFINITY ? 0.f : __expf(ms - M);
-        Lsum = fmaf(f, rows[sp * PR + 1], Lsum);
-        acc0 = fmaf(f, rows[sp * PR + 2 + jj], acc0);
-        acc1 = fmaf(f, rows[sp * PR + 2 + jj + 64], acc1);
+        Lsum = fmaf(f, row[1], Lsum);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[k] = fmaf(f, row[2 + lane + 32 * k], acc[k]);
       }
     }
-    __syncthreads();  // the batch buffer is refilled next
+    __syncthreads();  // the batch buffer is refilled next (or the exchange area is used)
   }
-  {
-    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-    y[g * kD + jj] = acc0 * inv;
-    y[g * kD + jj + 64] = acc1 * inv;
+  // warp g + 4 hands its (M, L, acc) to warp g through shared memory
+  float *xw = stg + (size_t)hg * (6 * 32);
+  if (par == 1) {
+    xw[lane] = M;
+    xw[32 + lane] = Lsum;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) xw[64 + 32 * k + lane] = acc[k];
   }
   __syncthreads();
-  for (int hh = 1; hh < kD; hh <<= 1) {
-    const int g = tid >> 6, i = tid & 63;  // 4 heads x 64 butterflies
-    const int lo = (i / hh) * 2 * hh + (i % hh);
-    const float u = y[g * kD + lo], v = y[g * kD + lo + hh];
-    __syncthreads();
-    y[g * kD + lo] = u + v;
-    y[g * kD + lo + hh] = u - v;
-    __syncthreads();
+  if (warp >= kG) return;
+  {
+    const float M2 = xw[lane], L2 = xw[32 + lane];
+    const float Mt = fmaxf(M, M2);
+    const float r1 = Mt == -INFINITY ? 0.f : __expf(M - Mt), r2 = Mt == -INFINITY ? 0.f : __expf(M2 - Mt);
+    Lsum = Lsum * r1 + L2 * r2;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc[k] = acc[k] * r1 + xw[64 + 32 * k + lane] * r2;
   }
-  for (int i = tid; i < kG * kD; i += kThreads) {
-    const int g = i / kD, j = i % kD;
-    a.out[((int64_t)b * a.hq + (int64_t)h * kG + g) * kD + j] = vc.signs[j] * y[i] * vc.inv_sqrt_d;
+  // o = D_V (1/sqrt d) H (acc / L): butterflies of span 32 and 64 within the lane, 1..16 across
+  // lanes (value k of lane i is coordinate i + 32 k)
+  const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) acc[k] *= inv;
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const bool upper = (lane & m) != 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float o = __shfl_xor_sync(TQ_FULL_MASK, acc[k], m);
+      acc[k] = upper ? o - acc[k] : acc[k] + o;
+    }
+  }
+  {
+    const float u0 = acc[0] + acc[1], u1 = acc[0] - acc[1], u2 = acc[2] + acc[3], u3 = acc[2] - acc[3];
+    acc[0] = u0 + u2;
+    acc[1] = u1 + u3;
+    acc[2] = u0 - u2;
+    acc[3] = u1 - u3;
+  }
+  float *dst = a.out + ((int64_t)b * a.hq + (int64_t)h * kG + warp) * kD;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int j = lane + 32 * k;
+    dst[j] = sgn[k] * acc[k];
   }
 }
 
@@ -1035,12 +1027,14 @@ extern "C" tq_status tq_device_status(int32_t device, int32_t *flags, int32_t cl
   if (!flags) return tq_fail(TQ_EINVAL, "flags is NULL");
   cudaError_t e = cudaSetDevice(device);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
-  int v = 0;
+  int v = 0, vr = 0;
   if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&v, g_tq_device_flags, sizeof(int));
+  if (e == cudaSuccess) e = rotate_device_flags(&vr, clear != 0);
   if (e == cudaSuccess && clear) {
     const int z = 0;
     e = cudaMemcpyToSymbol(g_tq_device_flags, &z, sizeof(int));
   }
+  v |= vr;
   if (e != cudaSuccess) return tq_fail(TQ_ECUDA, "device status: %s", cudaGetErrorString(e));
   *flags = v;
   return TQ_OK;

@@ -160,6 +160,61 @@ __device__ __forceinline__ void stage_rows_padded(float *dst, const float *__res
   }
 }
 
+// The same copy issued as asynchronous 16-byte copies (cp.async, no registers held), so that the
+// caller can overlap it with other work; complete it with stage_async_wait() and a block barrier.
+__device__ __forceinline__ void stage_rows_padded_async(float *dst, const float *__restrict__ src, int rows, int cols) {
+  const int c4 = cols >> 2;
+  const int total = rows * c4;
+  for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
+    const int r = idx / c4, c = idx - r * c4;
+    const unsigned sa = (unsigned)__cvta_generic_to_shared(dst + (size_t)r * (cols + 4) + 4 * c);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(sa), "l"(src + (size_t)r * cols + 4 * c) : "memory");
+  }
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+__device__ __forceinline__ void stage_async_wait() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+
+// Device-side status word of the library (bits of tq_device_status), one per translation unit:
+// set by a kernel that gave up waiting, read and cleared from the host by tq_device_status.
+static __device__ int g_tq_device_flags;
+constexpr int kFlagStagingTimeout = 1;
+
+// Bulk asynchronous copies (global -> this CTA's shared memory) completing on an mbarrier, and
+// the bounded wait for them.  Addresses 16-byte aligned, sizes multiples of 16 bytes.
+__device__ __forceinline__ unsigned smem_addr(const void *p) { return (unsigned)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void mbar_init(uint64_t *bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_arrive(uint64_t *bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, unsigned bytes, uint64_t *bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                   smem_addr(dst)),
+               "l"(src), "r"(bytes), "r"(smem_addr(bar))
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Wait for phase `parity` of `bar` to complete, giving up after about a second (each try_wait
+// suspends for a bounded, hardware-defined time).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, unsigned parity) {
+  for (int i = 0; i < (1 << 22); ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+// 2^e as a float for e in [-126, 127].
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
+
 __device__ __forceinline__ float bf16_to_f32(uint16_t h) {
   return __uint_as_float(((uint32_t)h) << 16);
 }

@@ -53,10 +53,7 @@ __device__ __forceinline__ void rotate_rows(const TqConsts &c, int mode, const v
   const int wib = threadIdx.x >> 5;
   // fused projection with S staged in shared memory (d = m = 128; row stride 132 floats)
   const bool staged = D == 128 && fsigns != nullptr && c.m == 128;
-  if (staged) {
-    stage_rows_padded(sS, c.S, 128, 128);
-    __syncthreads();
-  }
+  if (staged) stage_rows_padded_async(sS, c.S, 128, 128);  // completed before the projection
   const int g = lane / LPV;
   const int l = lane % LPV;
   const int64_t row = (vblock * (kRotThreads / 32) + wib) * VPW + g;
@@ -195,6 +192,7 @@ __device__ __forceinline__ void rotate_rows(const TqConsts &c, int mode, const v
         }
       if (l == 0) norm[slot] = nu;
     }
+    if (staged) stage_async_wait();  // no copy may be left in flight
     return;  // MSE-only: no residual
   }
 
@@ -223,6 +221,10 @@ __device__ __forceinline__ void rotate_rows(const TqConsts &c, int mode, const v
     if (fsigns != nullptr) {
       // fused QJL projection for small batches: one vector per warp, z_i = <S_i, r> with the
       // residual broadcast from shared memory, lane = output row within each group of 32
+      if (staged) {
+        stage_async_wait();
+        __syncthreads();
+      }
       const float gamma = sqrtf(group_sum<LPV>(rr));
       if (store && l == 0) rnorm[slot] = gamma;
       float *rb = rbuf[wib];

@@ -101,7 +101,8 @@ cudaError_t launch_attend(const TqConsts &kc, const TqConsts &vc, const tq_attn_
 // attend_mma.cu
 bool attn_fast_eligible(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc);
 int attn_fast_chunk(const tq_attn_desc &desc);
-constexpr int kFusedMaxSplits = 1024;  // splits merged inside the tensor-core kernel at most
+constexpr int kFusedMaxSplits = 1024;
+cudaError_t rotate_device_flags(int *v, bool clear);  // rotate.cu's share of tq_device_status  // splits merged inside the tensor-core kernel at most
 size_t attn_fast_extra_bytes(const TqConsts &kc, const tq_attn_desc &desc);
 cudaError_t launch_attend_fast(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc,
                                const AttnPlan &plan, const void *q, int dtype, void *extra,
