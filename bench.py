@@ -21,6 +21,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import re
 import math
 import os
 import statistics
@@ -66,6 +67,22 @@ def measured_peaks():
                 "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"]))}, "measured"
     except Exception:
         return dict(PEAKS_FALLBACK), "fallback"
+
+
+def recorded_traffic():
+    """DRAM bytes per launch of the tensor-core attention kernel from the committed ncu summary,
+    if it was taken on the kernel revision this library reports (else None)."""
+    from kv_cache_vector_06_b200 import tq
+    path = os.path.join(ROOT, "profiles", "attend_mma_llama8b_decode.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    rev = re.search(r"kernel revision: (\S+)", text)
+    val = re.search(r"traffic_bytes_per_launch: (\d+)", text)
+    if not rev or not val or f"attend_mma {rev.group(1)}" not in tq.version():
+        return None
+    return int(val.group(1))
 
 
 # ------------------------------------------------------------------------------ clocks (NVML)
@@ -478,8 +495,9 @@ def ours_arm(args, world, rank):
     if split_n:
         per_launch_s = split_ms / split_n / 1e3
         achieved = bench.bytes_per_step / per_launch_s / 1e9
-        roof = {"kernel": "attend_mma_kernel (split-context, tensor cores)", "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+        roof = {"kernel": "attend_mma_kernel (tensor cores, streamed sub-chunks, fused split merge)", "bound": "hbm",
+                "achieved": achieved, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": recorded_traffic(),
                 "peak_source": src + " (burst copy)", "us_per_launch": per_launch_s * 1e6,
                 "algorithmic_bytes_per_launch": bench.bytes_per_step}
     kernel_share = {k: {"launches_per_step": n / min(args.steps, 10 * N_LAYERS), "us_per_launch": 1e3 * t / n}

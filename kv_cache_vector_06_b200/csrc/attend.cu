@@ -263,8 +263,7 @@ cudaError_t launch_split(const TqConsts &kc, const TqConsts &vc, const AttnArgs 
   const size_t smem = sizeof(float) * ((size_t)(kc.d + kc.m) * G + (size_t)G * kAtTile +
                                        2 * G * kAtWarps + 32) +
                       sizeof(int64_t) * kAtTile;
-  cudaError_t e = cudaFuncSetAttribute(attend_split_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = tq_smem_limit(reinterpret_cast<const void *>(attend_split_kernel<G>), (int)smem);
   if (e != cudaSuccess) return e;
   tq_prof_begin(TQK_ATTEND_SPLIT, st);
   attend_split_kernel<G><<<grid, kAtThreads, smem, st>>>(kc, vc, a, qr, p, part);
@@ -345,8 +344,7 @@ cudaError_t launch_attend_combine(const TqConsts &vc, const tq_attn_desc &desc, 
                                   const float *partials, float *out, cudaStream_t st) {
   const int ngroups = kCbThreads >= vc.d ? kCbThreads / vc.d : 1;
   const size_t smem = sizeof(float) * ((size_t)plan.splits + vc.d + (size_t)ngroups * vc.d + 32);
-  cudaError_t e2 = cudaFuncSetAttribute(attend_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)smem);
+  cudaError_t e2 = tq_smem_limit(reinterpret_cast<const void *>(attend_combine_kernel), (int)smem);
   if (e2 != cudaSuccess) return e2;
   tq_prof_begin(TQK_ATTEND_COMBINE, st);
   attend_combine_kernel<<<(unsigned)((int64_t)desc.batch * desc.n_q_heads), kCbThreads, smem, st>>>(

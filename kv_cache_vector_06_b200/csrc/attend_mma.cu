@@ -852,7 +852,7 @@ template <int BK, int BV, bool QJL>
 cudaError_t launch_mma(const TqConsts &kc, const TqConsts &vc, const MmaArgs &a, dim3 grid,
                        const uint32_t *kfrag, const float *kconst, float *part, cudaStream_t st) {
   const size_t smem = MmaSmem<BK, BV, QJL>::total;
-  cudaError_t e = cudaFuncSetAttribute(attend_mma_kernel<BK, BV, QJL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = tq_smem_limit(reinterpret_cast<const void *>(attend_mma_kernel<BK, BV, QJL>),
                                        (int)smem);
   if (e != cudaSuccess) return e;
   attend_mma_kernel<BK, BV, QJL><<<grid, kThreads, smem, st>>>(kc, vc, a, kfrag, kconst, part);
@@ -865,7 +865,7 @@ cudaError_t launch_fast(const TqConsts &kc, const TqConsts &vc, const MmaArgs &a
   const unsigned groups = (unsigned)(batch * a.hkv);
   const size_t fsm = QJL ? sizeof(float) * kD * (kD + 4) : 0;
   if (fsm) {
-    cudaError_t e0 = cudaFuncSetAttribute(kfrag_kernel<BK, QJL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsm);
+    cudaError_t e0 = tq_smem_limit(reinterpret_cast<const void *>(kfrag_kernel<BK, QJL>), (int)fsm);
     if (e0 != cudaSuccess) return e0;
   }
   tq_prof_begin(TQK_ATTEND_FRAG, st);
@@ -967,7 +967,7 @@ cudaError_t launch_step(const TqConsts &kc, const TqConsts &vc, const MmaArgs &a
   const unsigned grid0 = (unsigned)(2 * nb + batch * a.hkv);
   const size_t fsm = QJL ? sizeof(float) * kD * (kD + 4) : 0;
   if (fsm) {
-    cudaError_t e0 = cudaFuncSetAttribute(decode_prep_kernel<BK, QJL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e0 = tq_smem_limit(reinterpret_cast<const void *>(decode_prep_kernel<BK, QJL>),
                                           (int)fsm);
     if (e0 != cudaSuccess) return e0;
   }

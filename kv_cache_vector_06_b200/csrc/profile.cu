@@ -4,6 +4,9 @@
 #include <mutex>
 #include <vector>
 
+#include <map>
+#include <utility>
+
 #include "tq_internal.h"
 
 namespace {
@@ -74,6 +77,20 @@ void tq_prof_end(int kind, cudaStream_t st) {
     if (e) g_free.push_back(e);
   }
   t_open[kind] = nullptr;
+}
+
+cudaError_t tq_smem_limit(const void *func, int bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<const void *, int>, int> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  int &have = done[std::make_pair(func, dev)];
+  if (have >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) have = bytes;
+  return e;
 }
 
 extern "C" {

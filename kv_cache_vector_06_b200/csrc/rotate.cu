@@ -36,7 +36,7 @@ cudaError_t launch_rotate_d(const TqConsts &c, RotateMode mode, const void *x, t
   const int kind = mode == ROT_ENCODE ? TQK_ROTATE_ENCODE : TQK_ROTATE_QUERY;
   const size_t smem = (D == 128 && fsigns != nullptr && c.m == 128) ? sizeof(float) * 128 * 132 : 0;
   if (smem) {
-    cudaError_t e0 = cudaFuncSetAttribute(rotate_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e0 = tq_smem_limit(reinterpret_cast<const void *>(rotate_kernel<D>), (int)smem);
     if (e0 != cudaSuccess) return e0;
   }
   tq_prof_begin(kind, st);

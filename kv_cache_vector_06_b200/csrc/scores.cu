@@ -46,7 +46,7 @@ cudaError_t launch_scores(const TqConsts &c, const float *qr, const float *p, in
                           const tq_packed &keys, int64_t n, float *out, cudaStream_t st) {
   if (n <= 0 || nq <= 0) return cudaSuccess;
   const size_t smem = sizeof(float) * ((size_t)(c.d + c.m) * kScQ + TQ_MAX_LEVELS);
-  cudaError_t e = cudaFuncSetAttribute(scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = tq_smem_limit(reinterpret_cast<const void *>(scores_kernel), (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((n + kScThreads - 1) / kScThreads), (unsigned)((nq + kScQ - 1) / kScQ));
   tq_prof_begin(TQK_SCORES, st);

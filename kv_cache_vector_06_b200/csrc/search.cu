@@ -119,7 +119,7 @@ cudaError_t launch_search(const TqConsts &c, const SearchPlan &plan, const float
   if (nq <= 0) return cudaSuccess;
   const int64_t rows_per_shard = (n + plan.shards - 1) / plan.shards;
   const size_t smem = sizeof(float) * ((size_t)(c.d + c.m) * kSrQ + TQ_MAX_LEVELS + kSrQ * kSrThreads);
-  cudaError_t e = cudaFuncSetAttribute(search_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = tq_smem_limit(reinterpret_cast<const void *>(search_scan_kernel), (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)plan.shards, (unsigned)((nq + kSrQ - 1) / kSrQ));
   tq_prof_begin(TQK_SEARCH_SCAN, st);

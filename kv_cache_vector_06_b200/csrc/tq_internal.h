@@ -102,7 +102,11 @@ cudaError_t launch_attend(const TqConsts &kc, const TqConsts &vc, const tq_attn_
 bool attn_fast_eligible(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc);
 int attn_fast_chunk(const tq_attn_desc &desc);
 constexpr int kFusedMaxSplits = 1024;
-cudaError_t rotate_device_flags(int *v, bool clear);  // rotate.cu's share of tq_device_status  // splits merged inside the tensor-core kernel at most
+cudaError_t rotate_device_flags(int *v, bool clear);  // rotate.cu's share of tq_device_status
+// Raise `func`'s dynamic shared-memory limit to at least `bytes` on the current device.  The
+// attribute call is made once per (kernel, device) and larger size (it costs host time that would
+// otherwise land between a kernel's launch and the work queued before it).
+cudaError_t tq_smem_limit(const void *func, int bytes);  // splits merged inside the tensor-core kernel at most
 size_t attn_fast_extra_bytes(const TqConsts &kc, const tq_attn_desc &desc);
 cudaError_t launch_attend_fast(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc,
                                const AttnPlan &plan, const void *q, int dtype, void *extra,
