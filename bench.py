@@ -49,6 +49,11 @@ def parse_args(argv=None):
                     help="K bits per coordinate: (kbits-1) MSE bits + 1 QJL bit")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-seconds", type=float, default=20.0)
+    ap.add_argument("--workload", choices=["decode", "search"], default="decode",
+                    help="decode: the Llama-3.1-8B decode layer (default); search: 10^6 x 1024 unit "
+                         "vectors, 1000 queries, top-10 (encode and scan), one GPU")
+    ap.add_argument("--search-bits", type=int, choices=[2, 4], default=2,
+                    help="search: bits per coordinate, (bits-1) MSE bits + 1 QJL bit with m = d")
     return ap.parse_args(argv)
 
 
@@ -533,12 +538,82 @@ def ours_arm(args, world, rank):
     return 0
 
 
+def search_arm(args):
+    """Vector search at 10^6 rows x d 1024: encode the database (unit vectors, fp32), then top-10
+    for 1000 queries.  Inputs are drawn on the device with a seeded generator (same recipe as the
+    parity tests: N(0, I) rows L2-normalised)."""
+    import torch
+    from kv_cache_vector_06_b200 import tq
+    import synth
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py --workload search needs a CUDA device (there is no CPU fallback)")
+    d, n, nq, k = 1024, 1_000_000, 1000, 10
+    mse, m = args.search_bits - 1, d
+    dev = torch.device("cuda", torch.cuda.current_device())
+    ctx = tq.Context(d, mse, m, synth.rotation_signs(d, 11), synth.qjl_matrix(m, d, 12), device=dev.index)
+    g = torch.Generator(device=dev)
+    g.manual_seed(13)
+    X = torch.randn(n, d, generator=g, device=dev)
+    X /= X.norm(dim=1, keepdim=True)
+    Q = torch.randn(nq, d, generator=g, device=dev)
+    Q /= Q.norm(dim=1, keepdim=True)
+    db = tq.Packed.allocate(ctx, n)
+    ws_e = torch.empty(tq.encode_workspace_size(ctx, n), dtype=torch.uint8, device=dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    tq.encode_kv(ctx, X, db, ws=ws_e)  # warm-up
+    torch.cuda.synchronize()
+    reps = max(1, min(args.steps, 5))
+    start.record()
+    for _ in range(reps):
+        tq.encode_kv(ctx, X, db, ws=ws_e)
+    end.record()
+    torch.cuda.synchronize()
+    enc_ms = start.elapsed_time(end) / reps
+    del X, ws_e
+    row_bytes = packed_bytes_per_key(d, mse, m)
+    ws_s = torch.empty(tq.search_workspace_size(ctx, nq, n, k), dtype=torch.uint8, device=dev)
+    sc = torch.empty(nq, k, dtype=torch.float32, device=dev)
+    ix = torch.empty(nq, k, dtype=torch.int64, device=dev)
+    for _ in range(max(1, min(args.warmup, 3))):
+        tq.search_topk(ctx, Q, db, k, out_scores=sc, out_idx=ix, ws=ws_s)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev.index)
+    with sampler:
+        start.record()
+        for _ in range(reps):
+            tq.search_topk(ctx, Q, db, k, out_scores=sc, out_idx=ix, ws=ws_s)
+        end.record()
+        torch.cuda.synchronize()
+    ms = start.elapsed_time(end) / reps
+    peaks, src = measured_peaks()
+    db_bytes = n * row_bytes
+    line = {
+        "metric": "search queries/s", "value": nq / (ms / 1e3), "unit": "queries/s", "n_gpus": 1,
+        "steps": reps, "warmup": max(1, min(args.warmup, 3)), "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"vector search: 10^6 unit vectors d 1024, {args.search_bits} bits/coord "
+                               f"({mse} MSE + QJL m 1024), 1000 queries, top-10", "rows": n, "d": d, "queries": nq,
+                   "k": k, "l2": "database (%.0f MB packed) larger than L2" % (db_bytes / 1e6)},
+        "scores_per_s": nq * n / (ms / 1e3),
+        "database_passes_per_s": 1e3 / ms,
+        "hbm": {"database_bytes": db_bytes, "gbs_one_read_per_query": nq * db_bytes / (ms / 1e3) / 1e9,
+                "peak": peaks["hbm_gbs"], "peak_source": src},
+        "encode": {"vectors_per_s": n / (enc_ms / 1e3), "ms": enc_ms,
+                   "gbs": n * (4 * d + row_bytes) / (enc_ms / 1e3) / 1e9},
+        "clocks": sampler.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     world, rank, _ = dist_setup(args)
     try:
         if args.impl == "reference":
             return reference_arm(args, world, rank)
+        if args.workload == "search":
+            return search_arm(args)
         return ours_arm(args, world, rank)
     finally:
         if world > 1:

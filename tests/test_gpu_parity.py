@@ -48,6 +48,19 @@ def test_encode_all_dims_and_bits(tq, d, bits):
     compare_encode(q, q.oracle_encode(x.double().numpy()), codes, sbits, norm, rnorm)
 
 
+@pytest.mark.parametrize("d,m,bits", [(128, 128, 2), (256, 128, 3), (1024, 1024, 1)])
+def test_encode_large_batch_projection(tq, d, m, bits):
+    """More rows than the fused small-batch encode takes: the separate QJL projection kernel
+    (tensor cores, 3 x TF32) with a ragged last row tile."""
+    n = 4096 + 300
+    q = Quantizer(d, bits, m, seed=3 * d + bits)
+    g = torch.Generator().manual_seed(d + m)
+    x = torch.randn(n, d, generator=g) * torch.exp(torch.randn(d, generator=g))
+    packed = _enc(tq, q, x)
+    codes, sbits, norm, rnorm = unpack(q, packed)
+    compare_encode(q, q.oracle_encode(x.double().numpy()), codes, sbits, norm, rnorm)
+
+
 @pytest.mark.parametrize("m", [0, 32, 96])
 def test_encode_mse_only_and_odd_m(tq, m):
     d, bits, n = 128, 3, 777
