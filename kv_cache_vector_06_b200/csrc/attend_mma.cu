@@ -324,6 +324,23 @@ struct StageArrays {
   static constexpr int n = QJL ? 6 : 4;  // K codes, V codes, ||k||, ||v|| (+ K signs, gamma)
 };
 
+// Array `arr` of a sub-chunk copy: source base, offset in the staging buffer, bytes per 16-slot
+// block and source bytes per slot.  (V codes are addressed by block: slot / 16 * block bytes ==
+// slot * (block bytes / 16).)
+template <int BK, int BV, bool QJL>
+__device__ __forceinline__ void stage_array(const MmaArgs &a, int arr, const char *&src, size_t &doff, unsigned &per,
+                                            int64_t &sstride) {
+  using SM = MmaSmem<BK, BV, QJL>;
+  switch (arr) {
+    case 0: src = static_cast<const char *>(a.k.codes); doff = SM::kc; per = 16 * SM::KCW * 4; sstride = SM::KCW * 4; break;
+    case 1: src = static_cast<const char *>(a.v.codes); doff = SM::vc; per = SM::VBW * 4; sstride = SM::VBW * 4 / 16; break;
+    case 2: src = reinterpret_cast<const char *>(a.k.norm); doff = SM::kn; per = 64; sstride = 4; break;
+    case 3: src = reinterpret_cast<const char *>(a.v.norm); doff = SM::vn; per = 64; sstride = 4; break;
+    case 4: src = static_cast<const char *>(a.k.signs); doff = SM::ks; per = 256; sstride = 16; break;
+    default: src = reinterpret_cast<const char *>(a.k.rnorm); doff = SM::kr; per = 64; sstride = 4; break;
+  }
+}
+
 // Issue the bulk copies of sub-chunk `sc` of the CTA (blocks [16 sc, 16 sc + 16) of its range)
 // into staging buffer `sb`, completing on `bar` (initialised with one arrival per array).  Warp
 // `arr` (< StageArrays::n) copies array `arr`.  vb[k] = first slot of the CTA's block k, or -1
@@ -338,17 +355,9 @@ __device__ __forceinline__ void stage_sub(const MmaArgs &a, int sc, const int64_
   const int arr = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const char *src;
   size_t doff;
-  unsigned per;     // bytes per block
-  int64_t sstride;  // source bytes per slot
-  switch (arr) {
-    case 0: src = static_cast<const char *>(a.k.codes); doff = SM::kc; per = 16 * SM::KCW * 4; sstride = SM::KCW * 4; break;
-    case 1: src = static_cast<const char *>(a.v.codes); doff = SM::vc; per = SM::VBW * 4; sstride = SM::VBW * 4 / 16; break;
-    case 2: src = reinterpret_cast<const char *>(a.k.norm); doff = SM::kn; per = 64; sstride = 4; break;
-    case 3: src = reinterpret_cast<const char *>(a.v.norm); doff = SM::vn; per = 64; sstride = 4; break;
-    case 4: src = static_cast<const char *>(a.k.signs); doff = SM::ks; per = 256; sstride = 16; break;
-    default: src = reinterpret_cast<const char *>(a.k.rnorm); doff = SM::kr; per = 64; sstride = 4; break;
-  }
-  // (V codes are addressed by block: slot / 16 * block bytes == slot * (block bytes / 16))
+  unsigned per;
+  int64_t sstride;
+  stage_array<BK, BV, QJL>(a, arr, src, doff, per, sstride);
   const int k0 = SM::NB * sc;
   if (!a.block_table) {
     if (lane == 0) {
@@ -396,17 +405,47 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gid = lane >> 2, t = lane & 3;
-  int L = a.seq_lens[b];
-  L = L < 0 ? 0 : (L > a.max_len ? a.max_len : L);
   const int t0 = s * a.chunk;
-  const int t1 = min(L, t0 + a.chunk);
-  const int nsub = t1 > t0 ? (t1 - t0 + kSub - 1) / kSub : 0;
   const int64_t grp = (int64_t)b * a.hkv + h;
   const int64_t cap = min(a.k.capacity, a.v.capacity);
+  constexpr unsigned FB = KP::regs * 32 * 4;  // the query fragments' bytes
 
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::br);
   int *fail = reinterpret_cast<int *>(smem + SM::br + 16);
   int *nlead_s = fail + 1;
+  // Contiguous layout: the first sub-chunk's blocks are consecutive slots known before the
+  // sequence length (bounded by the arrays only), so their copies start at once; blocks past the
+  // sequence are masked later like any other.
+  int early = 0;
+  int64_t base0 = 0;
+  if (!a.block_table) {
+    base0 = ((int64_t)b * a.hkv + h) * a.ctx_stride + t0;
+    int64_t nb = base0 < cap ? (cap - base0) / 16 : 0;
+    const int lim = min(SM::NB, a.chunk / 16);
+    early = (int)(nb < lim ? nb : lim);
+  }
+  if (tid == 0) {
+    mbar_init(&bars[0], StageArrays<QJL>::n);
+    mbar_init(&bars[1], StageArrays<QJL>::n);
+    mbar_init(&bars[4], 1);  // the merge's copies (br + 32)
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    *fail = 0;
+  }
+  __syncthreads();
+  if (early > 0 && warp < StageArrays<QJL>::n && lane == 0) {
+    const char *src;
+    size_t doff;
+    unsigned per;
+    int64_t sstride;
+    stage_array<BK, BV, QJL>(a, warp, src, doff, per, sstride);
+    mbar_expect_arrive(&bars[0], per * (unsigned)early + (warp == 0 ? FB : 0u));
+    bulk_g2s(smem + doff, src + base0 * sstride, per * (unsigned)early, &bars[0]);
+    if (warp == 0) bulk_g2s(smem + SM::kf, kfrag + grp * KP::regs * 32, FB, &bars[0]);
+  }
+  int L = a.seq_lens[b];
+  L = L < 0 ? 0 : (L > a.max_len ? a.max_len : L);
+  const int t1 = min(L, t0 + a.chunk);
+  const int nsub = t1 > t0 ? (t1 - t0 + kSub - 1) / kSub : 0;
   // the CTA's blocks: first slot, or -1 past the sequence or the arrays
   const int nblk = (t1 - t0 + 15) / 16;
   if (tid < SM::MAXBLK) {
@@ -420,24 +459,28 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
     const unsigned inval = __ballot_sync(TQ_FULL_MASK, base < 0);
     if ((tid & 31) == 0) nlead_s[tid >> 5] = inval ? __ffs(inval) - 1 : 32;
   }
-  if (tid == 0) {
-    mbar_init(&bars[0], StageArrays<QJL>::n);
-    mbar_init(&bars[1], StageArrays<QJL>::n);
-    mbar_init(&bars[4], 1);  // the merge's copies (br + 32)
-    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-    *fail = 0;
-  }
   if (tid < kG) {
     hM[tid] = -INFINITY;
     hL[tid] = 0.f;
   }
   __syncthreads();
   const int nlead = nlead_s[0] < 32 ? nlead_s[0] : 32 + nlead_s[1];
-  if (warp < StageArrays<QJL>::n && nsub > 0) {
-    // the first sub-chunk, and the query fragments (one copy per CTA) on the same barrier
-    constexpr unsigned FB = KP::regs * 32 * 4;
+  if (early == 0 && warp < StageArrays<QJL>::n && nsub > 0) {
+    // the first sub-chunk (paged layout), and the query fragments (one copy per CTA) on the same
+    // barrier
     stage_sub<BK, BV, QJL>(a, 0, vball, nlead, smem, &bars[0], FB);
     if (warp == 0 && lane == 0) bulk_g2s(smem + SM::kf, kfrag + grp * KP::regs * 32, FB, &bars[0]);
+  }
+  if (early > 0 && nsub == 0) {
+    // an empty range still owns the early copies in flight: they land before the buffers are
+    // reused for the partials
+    if (!__syncthreads_and(mbar_wait_bounded(&bars[0], 0u))) {
+      if (tid == 0) {
+        atomicOr(&g_tq_device_flags, kFlagStagingTimeout);
+        mbar_wait_bounded(&bars[0], 0u);
+      }
+      __syncthreads();
+    }
   }
   // the query constants (2^-F_code, 2^-F_sign, Cq, Cp per head), read from shared memory where
   // used (published by the first sub-chunk's barrier)
@@ -752,12 +795,15 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
   __syncthreads();
   if (!*last) return;
   // The group's partial rows (kD + 4 floats: m, l, o~, pad) pass through shared memory in
-  // batches of up to `nb` splits (cp.async through L2, one round trip per batch).  Warps g and
-  // g + 4 merge head g online over the even and the odd splits, lane holding coordinates
-  // lane + 32 k; warp g then folds in warp g + 4's share.
+  // batches of up to `nb` splits (one bulk copy per head and batch).  While a batch's copies are
+  // in flight, warp g < 4 reads head g's (m, l) straight from L2 and forms the merge factors
+  // e^{m_s - M}; then warps g and g + 4 accumulate head g's even and odd splits (lane holding
+  // coordinates lane + 32 k), and warp g adds warp g + 4's share.
   constexpr int PR = kD + 4;
-  float *stg = reinterpret_cast<float *>(smem);  // [kG][nb][PR]
-  const int nb = (int)(SM::vb / ((size_t)kG * PR * 4));
+  float *stg = reinterpret_cast<float *>(smem);  // [kG][nb][PR], then fs [kG][nb]
+  const int nb = (int)(SM::vb / ((size_t)kG * (PR + 1) * 4));
+  float *fs = stg + (size_t)kG * nb * PR;
+  float *rfac = hM;  // [kG] rescale of the running sums for the batch
   const int64_t pg = ((int64_t)b * a.hq + (int64_t)h * kG) * a.splits * PR;
   const int hg = warp & (kG - 1), par = warp >> 2;
   float sgn[4];  // the rotation signs of this lane's output coordinates, loaded early
@@ -772,6 +818,43 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
     if (tid < kG)
       bulk_g2s(stg + (size_t)tid * n * PR, part + pg + ((int64_t)tid * a.splits + s0) * PR, (unsigned)(n * PR * 4),
                &bars[4]);
+    if (warp < kG) {
+      const float *pb = part + pg + ((int64_t)warp * a.splits + s0) * PR;
+      float Mb = M, Lb = 0.f;
+      if (n <= 64) {
+        // one round trip: up to two (m, l) pairs per lane held in registers
+        float m2[2], l2[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int sp = lane + 32 * j;
+          m2[j] = sp < n ? __ldcg(pb + (int64_t)sp * PR) : -INFINITY;
+          l2[j] = sp < n ? __ldcg(pb + (int64_t)sp * PR + 1) : 0.f;
+          Mb = fmaxf(Mb, m2[j]);
+        }
+        Mb = warp_max_f(Mb);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int sp = lane + 32 * j;
+          const float f = m2[j] == -INFINITY ? 0.f : __expf(m2[j] - Mb);
+          if (sp < n) fs[warp * nb + sp] = f;
+          Lb = fmaf(f, l2[j], Lb);
+        }
+      } else {
+        for (int sp = lane; sp < n; sp += 32) Mb = fmaxf(Mb, __ldcg(pb + (int64_t)sp * PR));
+        Mb = warp_max_f(Mb);
+        for (int sp = lane; sp < n; sp += 32) {
+          const float ms = __ldcg(pb + (int64_t)sp * PR);
+          const float f = ms == -INFINITY ? 0.f : __expf(ms - Mb);
+          fs[warp * nb + sp] = f;
+          Lb = fmaf(f, __ldcg(pb + (int64_t)sp * PR + 1), Lb);
+        }
+      }
+      Lb = warp_sum_f(Lb);
+      const float r = Mb == -INFINITY ? 1.f : __expf(M - Mb);  // 0 while M is -inf
+      Lsum = fmaf(Lsum, r, Lb);
+      M = Mb;
+      if (lane == 0) rfac[warp] = r;
+    }
     if (!__syncthreads_and(mbar_wait_bounded(&bars[4], (unsigned)(s0 / nb) & 1u))) {
       if (tid == 0) {
         atomicOr(&g_tq_device_flags, kFlagStagingTimeout);
@@ -780,45 +863,32 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
       __syncthreads();
       return;
     }
-    const float *rows = stg + (size_t)hg * n * PR;
-    float Mb = M;
-    for (int sp = par; sp < n; sp += 2) Mb = fmaxf(Mb, rows[sp * PR]);
-    if (Mb != -INFINITY) {
-      const float r = __expf(M - Mb);  // 0 while M is -inf
+    {
+      const float r = rfac[hg];
 #pragma unroll
       for (int k = 0; k < 4; ++k) acc[k] *= r;
-      Lsum *= r;
-      M = Mb;
+      const float *rows = stg + (size_t)hg * n * PR;
+      const float *fg = fs + hg * nb;
 #pragma unroll 2
       for (int sp = par; sp < n; sp += 2) {
-        const float *row = rows + sp * PR;
-        const float ms = row[0];
-        const float f = ms == -INFINITY ? 0.f : __expf(ms - M);
-        Lsum = fmaf(f, row[1], Lsum);
+        const float f = fg[sp];
+        const float *row = rows + sp * PR + 2 + lane;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) acc[k] = fmaf(f, row[2 + lane + 32 * k], acc[k]);
+        for (int k = 0; k < 4; ++k) acc[k] = fmaf(f, row[32 * k], acc[k]);
       }
     }
     __syncthreads();  // the batch buffer is refilled next (or the exchange area is used)
   }
-  // warp g + 4 hands its (M, L, acc) to warp g through shared memory
-  float *xw = stg + (size_t)hg * (6 * 32);
+  // warp g + 4 hands its share of acc to warp g through shared memory (same scale M)
+  float *xw = stg + (size_t)hg * (4 * 32);
   if (par == 1) {
-    xw[lane] = M;
-    xw[32 + lane] = Lsum;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) xw[64 + 32 * k + lane] = acc[k];
+    for (int k = 0; k < 4; ++k) xw[32 * k + lane] = acc[k];
   }
   __syncthreads();
   if (warp >= kG) return;
-  {
-    const float M2 = xw[lane], L2 = xw[32 + lane];
-    const float Mt = fmaxf(M, M2);
-    const float r1 = Mt == -INFINITY ? 0.f : __expf(M - Mt), r2 = Mt == -INFINITY ? 0.f : __expf(M2 - Mt);
-    Lsum = Lsum * r1 + L2 * r2;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) acc[k] = acc[k] * r1 + xw[64 + 32 * k + lane] * r2;
-  }
+  for (int k = 0; k < 4; ++k) acc[k] += xw[32 * k + lane];
   // o = D_V (1/sqrt d) H (acc / L): butterflies of span 32 and 64 within the lane, 1..16 across
   // lanes (value k of lane i is coordinate i + 32 k)
   const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
