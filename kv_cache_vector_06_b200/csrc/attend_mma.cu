@@ -225,6 +225,7 @@ __global__ void __launch_bounds__(kThreads)
 kfrag_kernel(TqConsts kc, const void *__restrict__ q, int dtype, uint32_t *__restrict__ kfrag,
              float *__restrict__ kconst, int *__restrict__ counter) {
   extern __shared__ __align__(16) float sS[];
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");  // the attention grid may start
   kfrag_group<BK, QJL>(kc, q, dtype, kfrag, kconst, counter, blockIdx.x, sS);
 }
 
@@ -239,6 +240,7 @@ decode_prep_kernel(TqConsts kc, TqConsts vc, const void *__restrict__ knew, cons
                    const void *__restrict__ q, int qdtype, uint32_t *__restrict__ kfrag,
                    float *__restrict__ kconst, int *__restrict__ counter, int nkb, int nvb) {
   extern __shared__ __align__(16) float sS[];
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");  // the attention grid may start
   const int bid = blockIdx.x;
   if (bid < nkb) {
     rotate_rows<kD>(kc, ROT_ENCODE, knew, kvdtype, nnew, kD, slots, kp.capacity, static_cast<uint32_t *>(kp.codes),
@@ -431,6 +433,9 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     *fail = 0;
   }
+  // Launched as a programmatic dependent of the query-fragment kernel: everything above overlaps
+  // its tail; the caches (appended rows), fragments and counters are read only after this.
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
   __syncthreads();
   if (early > 0 && warp < StageArrays<QJL>::n && lane == 0) {
     const char *src;
@@ -925,8 +930,19 @@ cudaError_t launch_mma(const TqConsts &kc, const TqConsts &vc, const MmaArgs &a,
   cudaError_t e = tq_smem_limit(reinterpret_cast<const void *>(attend_mma_kernel<BK, BV, QJL>),
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  attend_mma_kernel<BK, BV, QJL><<<grid, kThreads, smem, st>>>(kc, vc, a, kfrag, kconst, part);
-  return cudaGetLastError();
+  // programmatic dependent launch: the grid may start while the preceding kernel on the stream
+  // (the query-fragment or decode-prep kernel) finishes; the kernel waits for it before use
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attend_mma_kernel<BK, BV, QJL>, kc, vc, a, kfrag, kconst, part);
 }
 
 template <int BK, int BV, bool QJL>
