@@ -220,6 +220,110 @@ __device__ __forceinline__ void kfrag_group(const TqConsts &kc, const void *__re
   }
 }
 
+// kfrag_group's work for one query head g of the group: the same arithmetic in the same order
+// (so the fragments are bit-identical), a quarter of the work per block.
+template <int BK, bool QJL>
+__device__ __forceinline__ void kfrag_head(const TqConsts &kc, const void *__restrict__ q, int dtype,
+                                           uint32_t *__restrict__ kfrag, float *__restrict__ kconst,
+                                           int *__restrict__ counter, int grp, int g, float *sS) {
+  using KP = KPlanes<BK, QJL>;
+  __shared__ float qs[kD];
+  __shared__ float X[KP::all][kD];
+  __shared__ float red[4];
+  __shared__ int fexp[2];
+  const int tid = threadIdx.x;
+  if constexpr (QJL) stage_rows_padded_async(sS, kc.S, kD, kD);
+  for (int j = tid; j < kD; j += kThreads) {
+    const int64_t o = ((int64_t)grp * kG + g) * kD + j;
+    const float x = dtype == TQ_F32 ? static_cast<const float *>(q)[o]
+                                    : bf16_to_f32(static_cast<const uint16_t *>(q)[o]);
+    qs[j] = x * kc.signs[j];
+  }
+  __syncthreads();
+  for (int hh = 1; hh < kD; hh <<= 1) {
+    const int i = tid & 63;  // 64 butterflies (threads 64.. repeat them harmlessly: same values)
+    const int lo = (i / hh) * 2 * hh + (i % hh);
+    const float a0 = qs[lo], b0 = qs[lo + hh];
+    __syncthreads();
+    if (tid < 64) {
+      qs[lo] = a0 + b0;
+      qs[lo + hh] = a0 - b0;
+    }
+    __syncthreads();
+  }
+  for (int j = tid; j < kD; j += kThreads) {
+    const float qv = qs[j] * kc.inv_sqrt_d;
+    qs[j] = qv;
+#pragma unroll
+    for (int P = 0; P < BK; ++P) X[P][j] = 2.f * kc.plane_coef[P] * qv;
+    if constexpr (BK == 3) X[3][j] = 2.f * kc.plane_coef[3] * qv;
+  }
+  __syncthreads();
+  if constexpr (QJL) {
+    stage_async_wait();
+    __syncthreads();
+    if (tid < kD) {
+      const float4 *Srow = reinterpret_cast<const float4 *>(sS + tid * (kD + 4));
+      float p0 = 0.f;
+#pragma unroll 8
+      for (int j4 = 0; j4 < kD / 4; ++j4) {
+        const float4 sv = Srow[j4];
+        p0 = fmaf(sv.x, qs[4 * j4], p0);
+        p0 = fmaf(sv.y, qs[4 * j4 + 1], p0);
+        p0 = fmaf(sv.z, qs[4 * j4 + 2], p0);
+        p0 = fmaf(sv.w, qs[4 * j4 + 3], p0);
+      }
+      X[KP::code][tid] = 2.f * p0;
+    }
+  }
+  __syncthreads();
+  const int warp = tid >> 5, lane = tid & 31;
+  if (warp == 0) {
+    float mc = 0.f, ms = 0.f, sq = 0.f, sp = 0.f;
+    for (int j = lane; j < kD; j += 32) {
+#pragma unroll
+      for (int P = 0; P < KP::code; ++P) mc = fmaxf(mc, fabsf(X[P][j]));
+      if constexpr (QJL) {
+        ms = fmaxf(ms, fabsf(X[KP::code][j]));
+        sp += 0.5f * X[KP::code][j];
+      }
+      sq += qs[j];
+    }
+    mc = warp_max_f(mc);
+    ms = warp_max_f(ms);
+    sq = warp_sum_f(sq);
+    sp = warp_sum_f(sp);
+    if (lane == 0) {
+      int ec = 0, es = 0;
+      frexpf(mc, &ec);
+      frexpf(ms, &es);
+      fexp[0] = mc > 0.f ? 30 - ec : 0;
+      fexp[1] = ms > 0.f ? 30 - es : 0;
+      red[0] = pow2i(-fexp[0]);
+      red[1] = pow2i(-fexp[1]);
+      red[2] = kc.plane_coef_sum * sq;
+      red[3] = sp;
+    }
+  }
+  __syncthreads();
+  if (tid < 4) kconst[(int64_t)grp * 16 + 4 * tid + g] = red[tid];
+  if (g == 0 && tid == 0) counter[grp] = 0;  // the split kernel that follows counts its CTAs here
+  // this head's fragment words: lanes 8 g .. 8 g + 7 of every (plane, k-step, n-tile, register)
+  uint32_t *out = kfrag + (int64_t)grp * KP::regs * 32;
+  for (int w = tid; w < KP::regs * 8; w += kThreads) {
+    const int r = w & 1, nt = (w >> 1) & 1, ls = (w >> 2) & 7, st = (w >> 5) & 3, P = w >> 7;
+    const int ln = 8 * g + ls;
+    const int t = ln & 3, limb = ((ln >> 2) & 1) + 2 * nt;
+    const float sc = pow2i(fexp[(QJL && P == KP::code) ? 1 : 0] - st - 4 * r);
+    const uint32_t sel = (uint32_t)limb | ((uint32_t)(4 + limb) << 4);
+    uint32_t wv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) wv[i] = (uint32_t)__float2int_rn(X[P][32 * t + st + 4 * r + 8 * i] * sc) + 0x80808080u;
+    out[(((P * 4 + st) * 32 + ln) * 2 + nt) * 2 + r] =
+        __byte_perm(__byte_perm(wv[0], wv[1], sel), __byte_perm(wv[2], wv[3], sel), 0x5410) ^ 0x80808080u;
+  }
+}
+
 template <int BK, bool QJL>
 __global__ void __launch_bounds__(kThreads)
 kfrag_kernel(TqConsts kc, const void *__restrict__ q, int dtype, uint32_t *__restrict__ kfrag,
@@ -230,9 +334,10 @@ kfrag_kernel(TqConsts kc, const void *__restrict__ q, int dtype, uint32_t *__res
 }
 
 // One launch for the work that precedes the split kernel in a decode step: blocks
-// [0, nkb) append-encode the new keys (8 per block, fused QJL projection), blocks [nkb, nkb + nvb)
-// the new values, and the remaining blocks build one (sequence, KV head)'s query fragments.  The
-// three jobs are independent, so their latencies overlap instead of adding up.
+// [0, nkb) append-encode the new keys (one per block with QJL, whose projection four warps share;
+// else 8 per block), blocks [nkb, nkb + nvb) the new values (8 per block), and the remaining
+// blocks build one query head's fragments each.  The jobs are independent, so their latencies
+// overlap instead of adding up.
 template <int BK, bool QJL>
 __global__ void __launch_bounds__(kThreads)
 decode_prep_kernel(TqConsts kc, TqConsts vc, const void *__restrict__ knew, const void *__restrict__ vnew,
@@ -243,13 +348,15 @@ decode_prep_kernel(TqConsts kc, TqConsts vc, const void *__restrict__ knew, cons
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");  // the attention grid may start
   const int bid = blockIdx.x;
   if (bid < nkb) {
+    // keys: with QJL one row per block (warps 0-3 share its projection), else 8 rows per block
     rotate_rows<kD>(kc, ROT_ENCODE, knew, kvdtype, nnew, kD, slots, kp.capacity, static_cast<uint32_t *>(kp.codes),
-                    kp.norm, kp.rnorm, nullptr, QJL ? static_cast<uint32_t *>(kp.signs) : nullptr, bid, sS);
+                    kp.norm, kp.rnorm, nullptr, QJL ? static_cast<uint32_t *>(kp.signs) : nullptr, bid, sS, QJL);
   } else if (bid < nkb + nvb) {
     rotate_rows<kD>(vc, ROT_ENCODE, vnew, kvdtype, nnew, kD, slots, vp.capacity, static_cast<uint32_t *>(vp.codes),
                     vp.norm, nullptr, nullptr, nullptr, bid - nkb, sS);
   } else {
-    kfrag_group<BK, QJL>(kc, q, qdtype, kfrag, kconst, counter, bid - nkb - nvb, sS);
+    const int qh = bid - nkb - nvb;  // query head: group qh / 4, head qh % 4
+    kfrag_head<BK, QJL>(kc, q, qdtype, kfrag, kconst, counter, qh / kG, qh % kG, sS);
   }
 }
 
@@ -1049,8 +1156,9 @@ template <int BK, int BV, bool QJL>
 cudaError_t launch_step(const TqConsts &kc, const TqConsts &vc, const MmaArgs &a, int batch, const void *knew,
                         const void *vnew, int kvdtype, int64_t nnew, const int64_t *slots, const void *q, int qdtype,
                         uint32_t *kfrag, float *kconst, float *part, cudaStream_t st) {
-  const int nb = (int)((nnew + (kThreads / 32) - 1) / (kThreads / 32));  // one vector per warp (d = 128)
-  const unsigned grid0 = (unsigned)(2 * nb + batch * a.hkv);
+  const int nvb = (int)((nnew + (kThreads / 32) - 1) / (kThreads / 32));  // one value row per warp
+  const int nkb = QJL ? (int)nnew : nvb;                                       // keys: see decode_prep_kernel
+  const unsigned grid0 = (unsigned)(nkb + nvb + batch * a.hq);
   const size_t fsm = QJL ? sizeof(float) * kD * (kD + 4) : 0;
   if (fsm) {
     cudaError_t e0 = tq_smem_limit(reinterpret_cast<const void *>(decode_prep_kernel<BK, QJL>),
@@ -1059,7 +1167,7 @@ cudaError_t launch_step(const TqConsts &kc, const TqConsts &vc, const MmaArgs &a
   }
   tq_prof_begin(TQK_DECODE_PREP, st);
   decode_prep_kernel<BK, QJL><<<grid0, kThreads, fsm, st>>>(kc, vc, knew, vnew, kvdtype, nnew, slots, a.k, a.v, q,
-                                                            qdtype, kfrag, kconst, a.counter, nb, nb);
+                                                            qdtype, kfrag, kconst, a.counter, nkb, nvb);
   tq_prof_end(TQK_DECODE_PREP, st);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -36,14 +36,16 @@ __device__ __forceinline__ float group_sum(float x) {
 // The encode / query-rotation work of one block of kRotThreads threads: rows of block `vblock`.
 // `sS` is dynamic shared memory of at least 128 x 132 floats when d = m = 128 and `fsigns` is set
 // (the fused projection stages S there); every thread of the block must call it with the same
-// arguments.
+// arguments.  With `one_vec` (d = m = 128, fused projection) the block encodes the single row
+// `vblock`: warp 0 rotates and quantizes it and warps 0-3 share its projection, 32 rows each (the
+// same arithmetic as one warp doing all 128).
 template <int D>
 __device__ __forceinline__ void rotate_rows(const TqConsts &c, int mode, const void *__restrict__ x, int dtype,
                                             int64_t n, int64_t ld, const int64_t *__restrict__ slots,
                                             int64_t capacity, uint32_t *__restrict__ codes,
                                             float *__restrict__ norm, float *__restrict__ rnorm,
                                             float *__restrict__ resid, uint32_t *__restrict__ fsigns,
-                                            int64_t vblock, float *sS) {
+                                            int64_t vblock, float *sS, bool one_vec = false) {
   using Lay = RotLayout<D>;
   constexpr int LPV = Lay::LPV, VPW = Lay::VPW, KCH = Lay::KCH;
   __shared__ uint32_t stage[kRotThreads / 32][VPW][Lay::CW];
@@ -56,7 +58,7 @@ __device__ __forceinline__ void rotate_rows(const TqConsts &c, int mode, const v
   if (staged) stage_rows_padded_async(sS, c.S, 128, 128);  // completed before the projection
   const int g = lane / LPV;
   const int l = lane % LPV;
-  const int64_t row = (vblock * (kRotThreads / 32) + wib) * VPW + g;
+  const int64_t row = one_vec ? (wib == 0 && g == 0 ? vblock : n) : (vblock * (kRotThreads / 32) + wib) * VPW + g;
   const bool valid = row < n;
 
   float v[KCH][4];
@@ -227,11 +229,38 @@ __device__ __forceinline__ void rotate_rows(const TqConsts &c, int mode, const v
       }
       const float gamma = sqrtf(group_sum<LPV>(rr));
       if (store && l == 0) rnorm[slot] = gamma;
-      float *rb = rbuf[wib];
+      float *rb = rbuf[one_vec ? 0 : wib];
+      if (!one_vec || wib == 0)
 #pragma unroll
-      for (int k = 0; k < KCH; ++k)
+        for (int k = 0; k < KCH; ++k)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) rb[4 * (l + LPV * k) + e] = v[k][e];
+          for (int e = 0; e < 4; ++e) rb[4 * (l + LPV * k) + e] = v[k][e];
+      if (one_vec) {
+        __shared__ int64_t oslot;
+        __shared__ int ostore;
+        if (threadIdx.x == 0) {
+          oslot = slot;
+          ostore = store ? 1 : 0;
+        }
+        __syncthreads();
+        if (wib < c.m / 32) {
+          const int w = wib;
+          const float4 *Srow = staged ? reinterpret_cast<const float4 *>(sS + (32 * w + lane) * (D + 4))
+                                      : reinterpret_cast<const float4 *>(c.S + (int64_t)(32 * w + lane) * D);
+          float z = 0.f;
+#pragma unroll 8
+          for (int j4 = 0; j4 < D / 4; ++j4) {
+            const float4 sv = Srow[j4];
+            z = fmaf(sv.x, rb[4 * j4], z);
+            z = fmaf(sv.y, rb[4 * j4 + 1], z);
+            z = fmaf(sv.z, rb[4 * j4 + 2], z);
+            z = fmaf(sv.w, rb[4 * j4 + 3], z);
+          }
+          const unsigned bal = __ballot_sync(TQ_FULL_MASK, z >= 0.f);
+          if (ostore && lane == 0) fsigns[oslot * c.sign_words + w] = bal;
+        }
+        return;
+      }
       __syncwarp();
       for (int w = 0; w < c.m / 32; ++w) {
         const float4 *Srow = staged ? reinterpret_cast<const float4 *>(sS + (32 * w + lane) * (D + 4))
