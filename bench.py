@@ -587,6 +587,12 @@ def search_arm(args):
     ms = start.elapsed_time(end) / reps
     peaks, src = measured_peaks()
     db_bytes = n * row_bytes
+    # ALU roofline of the CUDA-core scan: one fp32 FMA per code term and per sign term of every
+    # (query, row) score, against 148 SMs x 128 fp32 lanes x the SM clock
+    props = torch.cuda.get_device_properties(dev)
+    clk_ghz = (sampler.summary().get("sm_mhz") or 1965.0) / 1e3
+    lane_peak = props.multi_processor_count * 128 * clk_ghz * 1e9
+    terms = nq * n * (d + m) / (ms / 1e3)
     line = {
         "metric": "search queries/s", "value": nq / (ms / 1e3), "unit": "queries/s", "n_gpus": 1,
         "steps": reps, "warmup": max(1, min(args.warmup, 3)), "ms_per_step": ms, "higher_is_better": True,
@@ -599,11 +605,48 @@ def search_arm(args):
         "hbm": {"database_bytes": db_bytes, "gbs_one_read_per_query": nq * db_bytes / (ms / 1e3) / 1e9,
                 "peak": peaks["hbm_gbs"], "peak_source": src},
         "encode": {"vectors_per_s": n / (enc_ms / 1e3), "ms": enc_ms,
-                   "gbs": n * (4 * d + row_bytes) / (enc_ms / 1e3) / 1e9},
+                   "gbs": n * (4 * d + row_bytes) / (enc_ms / 1e3) / 1e9,
+                   "roofline": {"bound": "tensor", "achieved": 3 * 2 * m * d * n / (enc_ms / 1e3) / 1e12,
+                                "peak": peaks["bf16_tflops"] / 2, "unit": "TFLOP/s",
+                                "frac": 3 * 2 * m * d * n / (enc_ms / 1e3) / 1e12 / (peaks["bf16_tflops"] / 2),
+                                "traffic": None,
+                                "note": "QJL projection as 3 x TF32 MMA passes; peak = measured bf16 x 1/2 "
+                                        "(the dense tf32:bf16 ratio)"}},
+        "roofline": {"bound": "alu", "achieved": terms / 1e12, "peak": lane_peak / 1e12, "unit": "Tterm/s",
+                     "frac": terms / lane_peak, "traffic": None,
+                     "note": "CUDA-core scan: one fp32 FMA per code and sign term per (query, row); peak = SMs x "
+                             "128 lanes x SM clock"},
         "clocks": sampler.summary(),
     }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = search_cpu_baseline(ctx_d=d, mse=mse, m=m, row_count=n)
     print(json.dumps(line), flush=True)
     return 0
+
+
+def search_cpu_baseline(ctx_d: int, mse: int, m: int, row_count: int):
+    """The oracle on a bounded sample of the search workload: encode 4096 unit rows, score one
+    query against them (timed separately), scaled to queries/s over the full database."""
+    import numpy as np
+    import synth
+    from oracle import codebook as ocb, encode as oenc, estimate as oest
+    rows = 4096
+    D = synth.rotation_signs(ctx_d, 11).double().numpy()
+    S = synth.qjl_matrix(m, ctx_d, 12).double().numpy()
+    c, t = ocb.codebook(ctx_d, mse)
+    X = synth.unit_rows(rows, ctx_d, seed=0).double().numpy()
+    q = synth.unit_rows(1, ctx_d, seed=1).double().numpy()
+    t0 = time.perf_counter()
+    enc = oenc.encode(X, D, S, c, t)
+    t_enc = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    qr, p = oest.prepare_query(q, D, S)
+    oest.scores(qr, p, enc.norm, enc.codes, enc.rnorm, enc.bits, c)
+    t_sc = time.perf_counter() - t0
+    return {"value": 1.0 / (t_sc * row_count / rows), "unit": "queries/s", "cores": cpu_cores_used(),
+            "kind": "oracle", "encode_vectors_per_s": rows / t_enc,
+            "sample": f"encode {rows} rows ({t_enc:.1f} s), score one query against them ({t_sc:.2f} s), "
+                      f"scaled to {row_count} rows; fp64 numpy oracle"}
 
 
 def main(argv=None):

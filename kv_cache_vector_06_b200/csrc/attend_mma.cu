@@ -68,8 +68,13 @@ __device__ __forceinline__ void mma_u8u8(int (&c)[4], uint32_t a0, uint32_t a1, 
 // Uniform value in [0, 1) from a 32-bit key: the fractional part of key * (golden ratio), a
 // low-discrepancy sequence over consecutive keys (deterministic dither for rounding).
 __device__ __forceinline__ float dither(uint32_t x) {
-  return (float)((x * 2654435769u) >> 8) * (1.0f / 16777216.0f);
+  // top 23 bits of the product as the mantissa of a float in [1, 2), minus 1 (no conversion unit)
+  return __uint_as_float(0x3F800000u | ((x * 2654435769u) >> 9)) - 1.0f;
 }
+
+// floor(v) for 0 <= v < 2^23, as the low mantissa bits of 2^23 + floor(v): a round-down add on the
+// FMA pipe instead of a float-to-integer conversion.  The result's bytes 0 and 1 are floor(v)'s.
+__device__ __forceinline__ uint32_t floor_bits(float v) { return __float_as_uint(__fadd_rd(v, 8388608.f)); }
 
 __device__ __forceinline__ int64_t token_slot(const MmaArgs &a, int b, int h, int t) {
   if (a.block_table) {
@@ -770,12 +775,12 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
 #pragma unroll
           for (int rr = 0; rr < 2; ++rr) {
             const int i0 = 2 * rr, i1 = 2 * rr + 1;  // the two tokens of this register
-            const uint32_t x0 = __float2uint_rd(fmaf(W[i0], C[2 * x], dz[i0]));
-            const uint32_t x1 = __float2uint_rd(fmaf(W[i1], C[2 * x], dz[i1]));
-            const uint32_t x2 = __float2uint_rd(fmaf(W[i0], C[2 * x + 1], dz[i0]));
-            const uint32_t x3 = __float2uint_rd(fmaf(W[i1], C[2 * x + 1], dz[i1]));
+            const uint32_t x0 = floor_bits(fmaf(W[i0], C[2 * x], dz[i0]));
+            const uint32_t x1 = floor_bits(fmaf(W[i1], C[2 * x], dz[i1]));
+            const uint32_t x2 = floor_bits(fmaf(W[i0], C[2 * x + 1], dz[i0]));
+            const uint32_t x3 = floor_bits(fmaf(W[i1], C[2 * x + 1], dz[i1]));
             reg[2 * x + rr] = __byte_perm(__byte_perm(x0, x1, sel), __byte_perm(x2, x3, sel), 0x5410);
-            xs += (x0 + x1) + (x2 + x3);
+            xs += (x0 + x1) + (x2 + x3) - 4u * 0x4B000000u;  // the integers themselves
           }
         vfrag[kb * 32 + lane] = VT == 2 ? make_uint4(reg[0], reg[1], reg[2 * VT - 2], reg[2 * VT - 1])
                                         : make_uint4(reg[0], reg[1], 0u, 0u);
