@@ -247,7 +247,8 @@ tq_status tq_search_topk(const tq_ctx *ctx, const void *q, tq_dtype dtype, int32
  * kernel on the stream it runs on).  tq_profile_read waits for the recorded events and reports,
  * for kernel kind `index` (0, 1, ... until it returns TQ_EINVAL), its name, the number of
  * launches and their summed device time in milliseconds since the last reset.  Do not enable
- * while capturing a CUDA graph.
+ * while capturing a CUDA graph.  While enabled, the attention kernel is launched without
+ * programmatic dependence on the kernel before it (an event sits between them).
  *   name  host out buffer of name_len bytes (nullable); launches, total_ms host outs (nullable) */
 tq_status tq_profile_enable(int32_t on);
 tq_status tq_profile_reset(void);

@@ -103,7 +103,7 @@ extern "C" {
 const char *tq_last_error(void) { return g_err; }
 // The revision tag of the tensor-core attention kernel names the device code that a recorded
 // profile (DRAM traffic per launch) was taken on; it changes whenever that code changes.
-const char *tq_version(void) { return "libtq 0.2 (sm_100a; attend_mma r7)"; }
+const char *tq_version(void) { return "libtq 0.2 (sm_100a; attend_mma r8)"; }
 
 tq_status tq_make_codebook(int32_t d, int32_t bits, double *centroids, double *thresholds,
                            double *mse_per_coord) {

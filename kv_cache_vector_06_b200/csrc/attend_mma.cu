@@ -1043,7 +1043,12 @@ cudaError_t launch_mma(const TqConsts &kc, const TqConsts &vc, const MmaArgs &a,
                                        (int)smem);
   if (e != cudaSuccess) return e;
   // programmatic dependent launch: the grid may start while the preceding kernel on the stream
-  // (the query-fragment or decode-prep kernel) finishes; the kernel waits for it before use
+  // (the query-fragment or decode-prep kernel) finishes; the kernel waits for it before use.  With
+  // per-kernel profiling on, an event sits between the two kernels and a plain launch is used.
+  if (tq_prof_on()) {
+    attend_mma_kernel<BK, BV, QJL><<<grid, kThreads, smem, st>>>(kc, vc, a, kfrag, kconst, part);
+    return cudaGetLastError();
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(kThreads);

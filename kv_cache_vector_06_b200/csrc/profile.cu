@@ -54,6 +54,11 @@ void drain_locked() {
 
 }  // namespace
 
+bool tq_prof_on() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  return g_on;
+}
+
 void tq_prof_begin(int kind, cudaStream_t st) {
   std::lock_guard<std::mutex> lk(g_mu);
   if (!g_on) return;

@@ -53,6 +53,7 @@ enum TqKernelKind {
   TQK_ROTATE_ENCODE = 0, TQK_QJL_PROJECT, TQK_ROTATE_QUERY, TQK_QUERY_PROJECT, TQK_SCORES,
   TQK_ATTEND_SPLIT, TQK_ATTEND_COMBINE, TQK_SEARCH_SCAN, TQK_SEARCH_MERGE, TQK_ATTEND_FRAG, TQK_DECODE_PREP, TQK_COUNT
 };
+bool tq_prof_on();  // per-kernel event profiling is enabled
 void tq_prof_begin(int kind, cudaStream_t st);
 void tq_prof_end(int kind, cudaStream_t st);
 
