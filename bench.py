@@ -54,6 +54,8 @@ def parse_args(argv=None):
                          "vectors, 1000 queries, top-10 (encode and scan), one GPU")
     ap.add_argument("--search-bits", type=int, choices=[2, 4], default=2,
                     help="search: bits per coordinate, (bits-1) MSE bits + 1 QJL bit with m = d")
+    ap.add_argument("--search-rows", type=int, default=1_000_000,
+                    help="search: database rows (the workload is 10^6; smaller only for profiler captures)")
     return ap.parse_args(argv)
 
 
@@ -554,7 +556,7 @@ def search_arm(args):
     import synth
     if not torch.cuda.is_available():
         raise RuntimeError("bench.py --workload search needs a CUDA device (there is no CPU fallback)")
-    d, n, nq, k = 1024, 1_000_000, 1000, 10
+    d, n, nq, k = 1024, args.search_rows, 1000, 10
     mse, m = args.search_bits - 1, d
     dev = torch.device("cuda", torch.cuda.current_device())
     ctx = tq.Context(d, mse, m, synth.rotation_signs(d, 11), synth.qjl_matrix(m, d, 12), device=dev.index)
@@ -594,11 +596,13 @@ def search_arm(args):
     ms = start.elapsed_time(end) / reps
     peaks, src = measured_peaks()
     db_bytes = n * row_bytes
-    # ALU roofline of the CUDA-core scan: one fp32 FMA per code term and per sign term of every
-    # (query, row) score, against 148 SMs x 128 fp32 lanes x the SM clock
-    props = torch.cuda.get_device_properties(dev)
-    clk_ghz = (sampler.summary().get("sm_mhz") or 1965.0) / 1e3
-    lane_peak = props.multi_processor_count * 128 * clk_ghz * 1e9
+    # Tensor roofline of the scan: the estimate is a contraction of the rows' bit planes (mse code
+    # planes, a parity plane at 3 MSE bits, the sign plane) with the queries' 24-bit fixed-point
+    # values as three int8 limbs: 2 x planes x d x 3 int8 ops per (query, row), against the measured
+    # bf16 peak x 2 (the dense int8:bf16 ratio)
+    planes = mse + (1 if mse == 3 else 0) + 1
+    int8_ops = 2.0 * planes * d * 3 * nq * n
+    int8_peak = peaks["bf16_tflops"] * 2
     terms = nq * n * (d + m) / (ms / 1e3)
     line = {
         "metric": "search queries/s", "value": nq / (ms / 1e3), "unit": "queries/s", "n_gpus": 1,
@@ -619,10 +623,12 @@ def search_arm(args):
                                 "traffic": None,
                                 "note": "QJL projection as 3 x TF32 MMA passes; peak = measured bf16 x 1/2 "
                                         "(the dense tf32:bf16 ratio)"}},
-        "roofline": {"bound": "alu", "achieved": terms / 1e12, "peak": lane_peak / 1e12, "unit": "Tterm/s",
-                     "frac": terms / lane_peak, "traffic": None,
-                     "note": "CUDA-core scan: one fp32 FMA per code and sign term per (query, row); peak = SMs x "
-                             "128 lanes x SM clock"},
+        "terms_per_s": terms,
+        "roofline": {"kernel": "search_mma_kernel (bit-plane int8 MMAs)", "bound": "tensor",
+                     "achieved": int8_ops / (ms / 1e3) / 1e12, "peak": int8_peak, "unit": "TOP/s",
+                     "frac": int8_ops / (ms / 1e3) / 1e12 / int8_peak, "traffic": None,
+                     "note": "int8 ops of the bit-plane contraction (2 x %d planes x d x 3 limbs per query and row) "
+                             "per search call; peak = measured bf16 x 2 (dense int8:bf16 ratio), %s" % (planes, src)},
         "clocks": sampler.summary(),
     }
     if not args.no_cpu_baseline:

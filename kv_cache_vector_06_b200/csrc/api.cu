@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <algorithm>
 #include <cstring>
 #include <new>
 
@@ -495,9 +496,12 @@ tq_status tq_search_workspace_size(const tq_ctx *ctx, int32_t nq, int64_t n, int
   if (!bytes) return tq_fail(TQ_EINVAL, "bytes is NULL");
   if (nq < 0 || n < 0 || k < 1) return tq_fail(TQ_EINVAL, "nq/n/k");
   if (k > 32) return tq_fail(TQ_EUNSUPPORTED, "k=%d: at most 32", k);
-  const SearchPlan plan = search_plan(nq, n, k);
-  const int64_t cands = (int64_t)nq * plan.shards * k;
-  *bytes = query_prep_bytes(ctx, nq) + (size_t)tq_align_up(cands * 4, 256) + (size_t)tq_align_up(cands * 8, 256);
+  // room for either scan: the tensor-core one also needs 16-byte aligned norms, known only at the call
+  const bool mma = search_mma_eligible(ctx->k) && nq <= kSearchMmaMaxQ;
+  const int shards = std::max(search_plan(nq, n, k).shards, mma ? search_mma_shards(ctx->k, nq, n, k) : 1);
+  const int64_t cands = (int64_t)nq * shards * k;
+  *bytes = query_prep_bytes(ctx, nq) + (size_t)tq_align_up(cands * 4, 256) + (size_t)tq_align_up(cands * 8, 256) +
+           (mma ? search_mma_frag_bytes(ctx->k, nq) : 0);
   return TQ_OK;
 }
 
@@ -525,16 +529,25 @@ tq_status tq_search_topk(const tq_ctx *ctx, const void *q, tq_dtype dtype, int32
   st = set_device(ctx);
   if (st != TQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool mma = search_mma_eligible(ctx->k) && nq <= kSearchMmaMaxQ && aligned16(db.norm) && aligned16(db.rnorm);
   const SearchPlan plan = search_plan(nq, n, k);
-  const int64_t cands = (int64_t)nq * plan.shards * k;
+  const int shards = mma ? search_mma_shards(ctx->k, nq, n, k) : plan.shards;
+  const int64_t cands = (int64_t)nq * shards * k;
   char *w = static_cast<char *>(ws);
   float *qr = reinterpret_cast<float *>(w);
   float *p = reinterpret_cast<float *>(w + tq_align_up((int64_t)nq * ctx->spec.d * 4, 256));
   w += query_prep_bytes(ctx, nq);
   float *cs = reinterpret_cast<float *>(w);
   int64_t *ci = reinterpret_cast<int64_t *>(w + tq_align_up(cands * 4, 256));
+  void *fragws = w + tq_align_up(cands * 4, 256) + tq_align_up(cands * 8, 256);
   st = prep_queries(ctx, q, dtype, nq, qr, p, s);
   if (st != TQ_OK) return st;
+  if (mma) {
+    // tensor-core scan (bit-plane MMAs), then the same merge of the shards' candidates
+    cudaError_t e = launch_search_mma(ctx->k, shards, qr, p, nq, db, n, k, fragws, cs, ci, s);
+    if (e == cudaSuccess) e = launch_search_merge(nq, shards, k, cs, ci, out_scores, out_idx, s);
+    return tq_cuda_check(e, "search launch");
+  }
   return tq_cuda_check(launch_search(ctx->k, plan, qr, p, nq, db, n, k, cs, ci, out_scores, out_idx, s),
                        "search launch");
 }

@@ -128,10 +128,15 @@ cudaError_t launch_search(const TqConsts &c, const SearchPlan &plan, const float
   tq_prof_end(TQK_SEARCH_SCAN, st);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  return launch_search_merge(nq, plan.shards, k, cand_s, cand_i, out_s, out_i, st);
+}
+
+cudaError_t launch_search_merge(int nq, int shards, int k, const float *cand_s, const int64_t *cand_i, float *out_s,
+                                int64_t *out_i, cudaStream_t st) {
   const int wpb = 4;
   tq_prof_begin(TQK_SEARCH_MERGE, st);
-  search_merge_kernel<<<(unsigned)((nq + wpb - 1) / wpb), 32 * wpb, 0, st>>>(nq, plan.shards, k, cand_s,
-                                                                             cand_i, out_s, out_i);
+  search_merge_kernel<<<(unsigned)((nq + wpb - 1) / wpb), 32 * wpb, 0, st>>>(nq, shards, k, cand_s, cand_i, out_s,
+                                                                             out_i);
   tq_prof_end(TQK_SEARCH_MERGE, st);
   return cudaGetLastError();
 }

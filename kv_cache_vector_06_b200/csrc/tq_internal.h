@@ -128,6 +128,19 @@ struct SearchPlan {
   int shards;  // row shards
 };
 SearchPlan search_plan(int nq, int64_t n, int k);
+// Tensor-core scan (search_mma.cu): eligibility, workspace for the query fragments, shard count,
+// and the scan (the existing merge then reduces the candidates).
+// (the scan also needs norm and rnorm 16-byte aligned, and at most kSearchMmaMaxQ queries: 8 per
+// grid row, 65535 rows)
+constexpr int kSearchMmaMaxQ = 8 * 65535;
+bool search_mma_eligible(const TqConsts &c);
+size_t search_mma_frag_bytes(const TqConsts &c, int nq);
+int search_mma_shards(const TqConsts &c, int nq, int64_t n, int k);
+cudaError_t launch_search_mma(const TqConsts &c, int shards, const float *qr, const float *p, int nq,
+                              const tq_packed &db, int64_t n, int k, void *fragws, float *cand_s, int64_t *cand_i,
+                              cudaStream_t st);
+cudaError_t launch_search_merge(int nq, int shards, int k, const float *cand_s, const int64_t *cand_i, float *out_s,
+                                int64_t *out_i, cudaStream_t st);
 cudaError_t launch_search(const TqConsts &c, const SearchPlan &plan, const float *qr,
                           const float *p, int nq, const tq_packed &db, int64_t n, int k,
                           float *cand_s, int64_t *cand_i, float *out_s, int64_t *out_i,

@@ -254,6 +254,54 @@ def test_search_k_edge_cases(tq):
                 assert ii[r, a] < ii[r, a + 1]
 
 
+@pytest.mark.parametrize("d,bits", [(128, 1), (128, 3), (512, 2)])
+def test_search_tensor_core_scan_edges(tq, d, bits):
+    """Bit-plane tensor-core scan (d in 128..1024, m = d, 1..3 bits): databases shorter than one
+    128-row block, ragged tails that are not a multiple of 4 rows, k = n, k = 32, query counts
+    that leave a partial tile of 8, duplicate rows (equal scores in index order), and a norm array
+    at a 4-byte offset (which takes the CUDA-core scan)."""
+    q = Quantizer(d, bits, d, seed=70 + bits)
+    Q = synth.unit_rows(11, d, seed=71)
+    for n, k in ((1, 1), (3, 3), (40, 32), (129, 10), (1030, 32)):
+        X = synth.unit_rows(n, d, seed=72 + n)
+        packed = _enc(tq, q, X)
+        codes, sbits, norm, rnorm = unpack(q, packed)
+        ref_full = oracle_scores_from_packed(q, Q.double().numpy(), codes, sbits, norm, rnorm)
+        ref_s, _ = osearch.topk(ref_full, k)
+        s, i = tq.search_topk(q.ctx, Q.cuda(), packed, k)
+        torch.cuda.synchronize()
+        assert_topk_equivalent(s.cpu().numpy(), i.cpu().numpy(), lambda r, idx: ref_full[r, idx], ref_s)
+    X = synth.unit_rows(300, d, seed=73)
+    Xd = torch.cat([X, X])
+    pd = _enc(tq, q, Xd)
+    s, i = tq.search_topk(q.ctx, Q.cuda(), pd, 32)
+    ii, ss = i.cpu().numpy(), s.cpu().numpy()
+    for r in range(Q.shape[0]):
+        for a in range(31):
+            assert ss[r, a] >= ss[r, a + 1]
+            if ss[r, a] == ss[r, a + 1]:
+                assert ii[r, a] < ii[r, a + 1]
+        # row j and its copy j + 300 score the same, so the list holds the pairs (j, j + 300)
+        assert np.array_equal(ii[r, 0::2] + 300, ii[r, 1::2])
+        assert np.array_equal(ss[r, 0::2], ss[r, 1::2])
+    # a norm array one float off a 16-byte boundary: same results through the CUDA-core scan
+    X = synth.unit_rows(1000, d, seed=74)
+    packed = _enc(tq, q, X)
+    base_s, base_i = tq.search_topk(q.ctx, Q.cuda(), packed, 10)
+    nbuf = torch.empty(1001, dtype=torch.float32, device="cuda")
+    rbuf = torch.empty(1001, dtype=torch.float32, device="cuda")
+    nbuf[1:].copy_(packed.norm)
+    rbuf[1:].copy_(packed.rnorm)
+    shifted = tq.Packed(packed.codes, nbuf[1:], packed.signs, rbuf[1:])
+    s2, i2 = tq.search_topk(q.ctx, Q.cuda(), shifted, 10)
+    torch.cuda.synchronize()
+    codes, sbits, norm, rnorm = unpack(q, packed)
+    ref_full = oracle_scores_from_packed(q, Q.double().numpy(), codes, sbits, norm, rnorm)
+    ref_s, _ = osearch.topk(ref_full, 10)
+    for got_s, got_i in ((base_s, base_i), (s2, i2)):
+        assert_topk_equivalent(got_s.cpu().numpy(), got_i.cpu().numpy(), lambda r, idx: ref_full[r, idx], ref_s)
+
+
 @pytest.mark.parametrize("d,bits", [(8, 1), (64, 2), (128, 3), (128, 4), (256, 2)])
 def test_encode_block16_layout(tq, d, bits):
     """Values in the token-transposed 16-slot block layout, written at scattered slots (several
