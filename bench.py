@@ -624,7 +624,7 @@ def search_arm(args):
                                 "note": "QJL projection as 3 x TF32 MMA passes; peak = measured bf16 x 1/2 "
                                         "(the dense tf32:bf16 ratio)"}},
         "terms_per_s": terms,
-        "roofline": {"kernel": "search_mma_kernel (bit-plane int8 MMAs)", "bound": "tensor",
+        "roofline": {"kernel": "search_tc_kernel (bit-plane tcgen05 kind::i8 MMAs)", "bound": "tensor",
                      "achieved": int8_ops / (ms / 1e3) / 1e12, "peak": int8_peak, "unit": "TOP/s",
                      "frac": int8_ops / (ms / 1e3) / 1e12 / int8_peak, "traffic": None,
                      "note": "int8 ops of the bit-plane contraction (2 x %d planes x d x 3 limbs per query and row) "

@@ -497,11 +497,13 @@ tq_status tq_search_workspace_size(const tq_ctx *ctx, int32_t nq, int64_t n, int
   if (nq < 0 || n < 0 || k < 1) return tq_fail(TQ_EINVAL, "nq/n/k");
   if (k > 32) return tq_fail(TQ_EUNSUPPORTED, "k=%d: at most 32", k);
   // room for either scan: the tensor-core one also needs 16-byte aligned norms, known only at the call
+  const bool tc = search_tc_eligible(ctx->k, nq, k);
   const bool mma = search_mma_eligible(ctx->k) && nq <= kSearchMmaMaxQ;
-  const int shards = std::max(search_plan(nq, n, k).shards, mma ? search_mma_shards(ctx->k, nq, n, k) : 1);
+  const int shards = std::max({search_plan(nq, n, k).shards, mma ? search_mma_shards(ctx->k, nq, n, k) : 1,
+                               tc ? search_tc_shards(nq, n) : 1});
   const int64_t cands = (int64_t)nq * shards * k;
   *bytes = query_prep_bytes(ctx, nq) + (size_t)tq_align_up(cands * 4, 256) + (size_t)tq_align_up(cands * 8, 256) +
-           (mma ? search_mma_frag_bytes(ctx->k, nq) : 0);
+           std::max(mma ? search_mma_frag_bytes(ctx->k, nq) : 0, tc ? search_tc_ws_bytes(ctx->k, nq) : 0);
   return TQ_OK;
 }
 
@@ -529,9 +531,12 @@ tq_status tq_search_topk(const tq_ctx *ctx, const void *q, tq_dtype dtype, int32
   st = set_device(ctx);
   if (st != TQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const bool mma = search_mma_eligible(ctx->k) && nq <= kSearchMmaMaxQ && aligned16(db.norm) && aligned16(db.rnorm);
+  // scan: tcgen05 (many queries), else the bit-plane mma.sync scan, else CUDA cores
+  const bool tc = search_tc_eligible(ctx->k, nq, k);
+  const bool mma = !tc && search_mma_eligible(ctx->k) && nq <= kSearchMmaMaxQ && aligned16(db.norm) &&
+                   aligned16(db.rnorm);
   const SearchPlan plan = search_plan(nq, n, k);
-  const int shards = mma ? search_mma_shards(ctx->k, nq, n, k) : plan.shards;
+  const int shards = tc ? search_tc_shards(nq, n) : mma ? search_mma_shards(ctx->k, nq, n, k) : plan.shards;
   const int64_t cands = (int64_t)nq * shards * k;
   char *w = static_cast<char *>(ws);
   float *qr = reinterpret_cast<float *>(w);
@@ -542,9 +547,10 @@ tq_status tq_search_topk(const tq_ctx *ctx, const void *q, tq_dtype dtype, int32
   void *fragws = w + tq_align_up(cands * 4, 256) + tq_align_up(cands * 8, 256);
   st = prep_queries(ctx, q, dtype, nq, qr, p, s);
   if (st != TQ_OK) return st;
-  if (mma) {
+  if (tc || mma) {
     // tensor-core scan (bit-plane MMAs), then the same merge of the shards' candidates
-    cudaError_t e = launch_search_mma(ctx->k, shards, qr, p, nq, db, n, k, fragws, cs, ci, s);
+    cudaError_t e = tc ? launch_search_tc(ctx->k, shards, qr, p, nq, db, n, k, fragws, cs, ci, s)
+                       : launch_search_mma(ctx->k, shards, qr, p, nq, db, n, k, fragws, cs, ci, s);
     if (e == cudaSuccess) e = launch_search_merge(nq, shards, k, cs, ci, out_scores, out_idx, s);
     return tq_cuda_check(e, "search launch");
   }

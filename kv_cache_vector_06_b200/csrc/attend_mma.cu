@@ -391,10 +391,6 @@ __device__ __forceinline__ uint32_t mul_lo(uint32_t x, uint32_t m) {
   asm("mul.lo.u32 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(m));
   return r;
 }
-// 16-byte asynchronous global -> shared copy through L2 (the partial rows other CTAs wrote).
-__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_addr(smem_dst)), "l"(gmem) : "memory");
-}
 
 constexpr int kSub = 256;          // tokens per sub-chunk (one staging buffer)
 constexpr int kSubBlk = kSub / 16;  // 16-token blocks per sub-chunk
@@ -1231,14 +1227,16 @@ extern "C" tq_status tq_device_status(int32_t device, int32_t *flags, int32_t cl
   if (!flags) return tq_fail(TQ_EINVAL, "flags is NULL");
   cudaError_t e = cudaSetDevice(device);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
-  int v = 0, vr = 0;
+  int v = 0, vr = 0, vm = 0, vt = 0;
   if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&v, g_tq_device_flags, sizeof(int));
   if (e == cudaSuccess) e = rotate_device_flags(&vr, clear != 0);
+  if (e == cudaSuccess) e = search_mma_device_flags(&vm, clear != 0);
+  if (e == cudaSuccess) e = search_tc_device_flags(&vt, clear != 0);
   if (e == cudaSuccess && clear) {
     const int z = 0;
     e = cudaMemcpyToSymbol(g_tq_device_flags, &z, sizeof(int));
   }
-  v |= vr;
+  v |= vr | vm | vt;
   if (e != cudaSuccess) return tq_fail(TQ_ECUDA, "device status: %s", cudaGetErrorString(e));
   *flags = v;
   return TQ_OK;

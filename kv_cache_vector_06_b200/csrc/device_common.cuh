@@ -179,9 +179,25 @@ __device__ __forceinline__ void stage_async_wait() { asm volatile("cp.async.wait
 static __device__ int g_tq_device_flags;
 constexpr int kFlagStagingTimeout = 1;
 
+// Host accessor for this translation unit's status word (read, optionally clear); each unit whose
+// kernels set flags defines one and tq_device_status ORs them.
+#define TQ_DEVICE_FLAGS_ACCESSOR(name)                                   \
+  cudaError_t name(int *v, bool clear) {                                 \
+    cudaError_t e = cudaMemcpyFromSymbol(v, g_tq_device_flags, sizeof(int)); \
+    if (e == cudaSuccess && clear) {                                     \
+      const int z = 0;                                                   \
+      e = cudaMemcpyToSymbol(g_tq_device_flags, &z, sizeof(int));       \
+    }                                                                    \
+    return e;                                                            \
+  }
+
 // Bulk asynchronous copies (global -> this CTA's shared memory) completing on an mbarrier, and
 // the bounded wait for them.  Addresses 16-byte aligned, sizes multiples of 16 bytes.
 __device__ __forceinline__ unsigned smem_addr(const void *p) { return (unsigned)__cvta_generic_to_shared(p); }
+// 16-byte asynchronous global -> shared copy through L2 (both addresses 16-byte aligned).
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_addr(smem_dst)), "l"(gmem) : "memory");
+}
 __device__ __forceinline__ void mbar_init(uint64_t *bar, unsigned count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(count) : "memory");
 }

@@ -64,11 +64,4 @@ cudaError_t launch_rotate(const TqConsts &c, RotateMode mode, const void *x, tq_
 }
 
 // The device flags of this translation unit's kernels (see tq_device_status).
-cudaError_t rotate_device_flags(int *v, bool clear) {
-  cudaError_t e = cudaMemcpyFromSymbol(v, g_tq_device_flags, sizeof(int));
-  if (e == cudaSuccess && clear) {
-    const int z = 0;
-    e = cudaMemcpyToSymbol(g_tq_device_flags, &z, sizeof(int));
-  }
-  return e;
-}
+TQ_DEVICE_FLAGS_ACCESSOR(rotate_device_flags)

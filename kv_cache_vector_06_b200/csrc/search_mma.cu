@@ -531,3 +531,6 @@ cudaError_t launch_search_mma(const TqConsts &c, int shards, const float *qr, co
 #undef TQ_SM
   return cudaErrorInvalidValue;
 }
+
+// The device flags of this translation unit's kernels (see tq_device_status).
+TQ_DEVICE_FLAGS_ACCESSOR(search_mma_device_flags)

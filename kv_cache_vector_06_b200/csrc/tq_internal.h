@@ -103,7 +103,10 @@ cudaError_t launch_attend(const TqConsts &kc, const TqConsts &vc, const tq_attn_
 bool attn_fast_eligible(const TqConsts &kc, const TqConsts &vc, const tq_attn_desc &desc);
 int attn_fast_chunk(const tq_attn_desc &desc);
 constexpr int kFusedMaxSplits = 1024;
-cudaError_t rotate_device_flags(int *v, bool clear);  // rotate.cu's share of tq_device_status
+// the other translation units' shares of tq_device_status
+cudaError_t rotate_device_flags(int *v, bool clear);
+cudaError_t search_mma_device_flags(int *v, bool clear);
+cudaError_t search_tc_device_flags(int *v, bool clear);
 // Raise `func`'s dynamic shared-memory limit to at least `bytes` on the current device.  The
 // attribute call is made once per (kernel, device) and larger size (it costs host time that would
 // otherwise land between a kernel's launch and the work queued before it).
@@ -134,6 +137,13 @@ SearchPlan search_plan(int nq, int64_t n, int k);
 // grid row, 65535 rows)
 constexpr int kSearchMmaMaxQ = 8 * 65535;
 bool search_mma_eligible(const TqConsts &c);
+// tcgen05 scan (search_tc.cu): 64 queries per CTA, k <= 16, at least 32 queries
+bool search_tc_eligible(const TqConsts &c, int nq, int k);
+size_t search_tc_ws_bytes(const TqConsts &c, int nq);
+int search_tc_shards(int nq, int64_t n);
+cudaError_t launch_search_tc(const TqConsts &c, int shards, const float *qr, const float *p, int nq,
+                             const tq_packed &db, int64_t n, int k, void *ws, float *cand_s, int64_t *cand_i,
+                             cudaStream_t st);
 size_t search_mma_frag_bytes(const TqConsts &c, int nq);
 int search_mma_shards(const TqConsts &c, int nq, int64_t n, int k);
 cudaError_t launch_search_mma(const TqConsts &c, int shards, const float *qr, const float *p, int nq,

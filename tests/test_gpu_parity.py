@@ -302,6 +302,34 @@ def test_search_tensor_core_scan_edges(tq, d, bits):
         assert_topk_equivalent(got_s.cpu().numpy(), got_i.cpu().numpy(), lambda r, idx: ref_full[r, idx], ref_s)
 
 
+@pytest.mark.parametrize("d,bits", [(128, 2), (256, 1), (512, 3), (1024, 1), (1024, 3)])
+def test_search_tcgen05_scan(tq, d, bits):
+    """tcgen05 scan (at least 32 queries, k <= 16, d in 128..1024, m = d): a ragged second tile of
+    64 queries, databases shorter than one 128-row block and with ragged tails, k = 1, 10, 16,
+    and duplicate rows (equal scores in index order)."""
+    q = Quantizer(d, bits, d, seed=80 + bits)
+    Q = synth.unit_rows(70, d, seed=81)
+    for n, k in ((1, 1), (3, 3), (129, 10), (1030, 16), (5003, 10)):
+        X = synth.unit_rows(n, d, seed=82 + n)
+        packed = _enc(tq, q, X)
+        codes, sbits, norm, rnorm = unpack(q, packed)
+        ref_full = oracle_scores_from_packed(q, Q.double().numpy(), codes, sbits, norm, rnorm)
+        ref_s, _ = osearch.topk(ref_full, k)
+        s, i = tq.search_topk(q.ctx, Q.cuda(), packed, k)
+        torch.cuda.synchronize()
+        assert tq.device_status() == 0
+        assert_topk_equivalent(s.cpu().numpy(), i.cpu().numpy(), lambda r, idx: ref_full[r, idx], ref_s)
+    X = synth.unit_rows(300, d, seed=83)
+    pd = _enc(tq, q, torch.cat([X, X]))
+    s, i = tq.search_topk(q.ctx, Q.cuda(), pd, 16)
+    ii, ss = i.cpu().numpy(), s.cpu().numpy()
+    for r in range(Q.shape[0]):
+        assert np.all(ss[r, :-1] >= ss[r, 1:])
+        # row j and its copy j + 300 score the same, so the list holds the pairs (j, j + 300)
+        assert np.array_equal(ii[r, 0::2] + 300, ii[r, 1::2])
+        assert np.array_equal(ss[r, 0::2], ss[r, 1::2])
+
+
 @pytest.mark.parametrize("d,bits", [(8, 1), (64, 2), (128, 3), (128, 4), (256, 2)])
 def test_encode_block16_layout(tq, d, bits):
     """Values in the token-transposed 16-slot block layout, written at scattered slots (several
