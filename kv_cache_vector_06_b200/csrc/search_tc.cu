@@ -17,14 +17,15 @@
 // of the limb sums.
 //
 // A CTA takes 64 queries and one shard of rows, in 128-row blocks.  Warp roles:
-//   warps 0-7   expand the rows' packed bits to bytes in shared memory (two threads per row), one
-//               stage = (128 coordinates, plane), in the canonical K-major no-swizzle layout;
+//   warps 0-7   expand the rows' packed bits to bytes in shared memory (two groups of four warps,
+//               one row per thread, alternate planes), one stage = (128 coordinates, plane), in
+//               the canonical K-major no-swizzle layout;
 //   warp 8      allocates tensor memory and issues the MMAs (one thread), committing each stage
 //               back to its producers and each block to the epilogue;
 //   warp 9      streams the query stages (prepared once per call in the same layout) by bulk copy;
-//   warps 10-13 read the accumulators (one row per thread), form the 64 scores, release the
-//               accumulators, then keep a sorted top-k per (warp, query) in shared memory, filtered
-//               by a per-query score floor shared by the four lists;
+//   warps 10-13 read the accumulators (one row per thread), write the 64 scores to a shared
+//               [query][row] tile, release the accumulators, then keep each query's sorted top-k
+//               (one warp per query, the tile's rows filtered by the list's k-th entry);
 //   warps 14-15 copy the rows' packed words (16 B per row, plane and chunk) into a staging ring
 //               with cp.async, so that the expanding threads issue no global loads.
 // Every wait is bounded; on a timeout the CTA sets the device flag, drains its own copies and
@@ -49,7 +50,7 @@ constexpr int kTcThreads = 512;
 constexpr int kTcWMma = 8, kTcWB = 9, kTcWEpi = 10, kTcWLoad = 14;
 
 // row-word staging ring depth (chunks) for lp stored planes per row
-__host__ __device__ constexpr int tc_ring(int lp) { return lp <= 2 ? 8 : 4; }
+__host__ __device__ constexpr int tc_ring(int lp) { return lp <= 2 ? 4 : 2; }
 constexpr int kTcMaxK = 16;
 constexpr uint32_t kTcCols = 512;         // tensor-memory columns: code sums at 0, sign sums at 256
 
@@ -63,7 +64,7 @@ struct TcShape {
 };
 
 struct TcLayout {
-  size_t stg, kq, thr, ls, li, bars, slot, total;
+  size_t stg, kq, sct, ls, li, bars, slot, total;
   int ns;
 };
 
@@ -74,10 +75,10 @@ __host__ __device__ inline TcLayout tc_layout(int k, int ns, int lp) {
   L.ns = ns;
   L.stg = (size_t)ns * kTcStage;                      // [ring][lp][128 rows][16 B]
   L.kq = L.stg + (size_t)tc_ring(lp) * lp * kTcM * 16;
-  L.thr = L.kq + kTcQ * 16;                           // [64] f32
-  L.ls = L.thr + kTcQ * 4;
-  L.li = L.ls + up16((size_t)4 * kTcQ * k * 4);
-  L.bars = L.li + up16((size_t)4 * kTcQ * k * 8);
+  L.sct = L.kq + kTcQ * 16;                           // block scores [64 q][128 rows] f32
+  L.ls = L.sct + (size_t)kTcQ * kTcM * 4;             // per query sorted top-k [64 q][k]
+  L.li = L.ls + up16((size_t)kTcQ * k * 4);
+  L.bars = L.li + up16((size_t)kTcQ * k * 8);
   L.slot = L.bars + (size_t)(3 * ns + 3 + 2 * tc_ring(lp)) * 8;
   L.total = L.slot + 16;
   return L;
@@ -118,6 +119,18 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
+
+// Named barrier 1 over the 128 epilogue threads, returning whether `p` held on all of them.
+__device__ __forceinline__ bool epi_all(bool p) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred pi, po;\n setp.ne.u32 pi, %1, 0;\n bar.red.and.pred po, 1, 128, pi;\n"
+      " selp.u32 %0, 1, 0, po;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)p)
+      : "memory");
+  return r != 0;
+}
 
 // 4 bits -> 4 bytes of 0/1 (bit i to byte i)
 __device__ __forceinline__ uint32_t nib_bytes(uint32_t n) { return (n * 0x00204081u) & 0x01010101u; }
@@ -214,9 +227,9 @@ search_tc_kernel(TqConsts c, const uint8_t *__restrict__ bst, const float *__res
   constexpr int LP = BK + 1;  // stored planes: code planes + sign plane
   constexpr int kR = tc_ring(LP);
   const TcLayout L = tc_layout(k, ns, LP);
-  float *sthr = reinterpret_cast<float *>(smem + L.thr);  // per query: some warp list's k-th score
+  float *sct = reinterpret_cast<float *>(smem + L.sct);
   float *skq = reinterpret_cast<float *>(smem + L.kq);
-  float *ls = reinterpret_cast<float *>(smem + L.ls);        // [4 epilogue warps][64 q][k]
+  float *ls = reinterpret_cast<float *>(smem + L.ls);        // [64 q][k]
   int64_t *li = reinterpret_cast<int64_t *>(smem + L.li);
   uint64_t *afull = reinterpret_cast<uint64_t *>(smem + L.bars);
   uint64_t *bfull = afull + ns, *empty = bfull + ns, *accfull = empty + ns, *accempty = accfull + 1,
@@ -233,16 +246,16 @@ search_tc_kernel(TqConsts c, const uint8_t *__restrict__ bst, const float *__res
 
   if (tid == 0) {
     for (int i = 0; i < ns; ++i) {
-      mbar_init(&afull[i], 256);
+      mbar_init(&afull[i], 4);  // one arrival per warp of the expander group
       mbar_init(&bfull[i], 1);
       mbar_init(&empty[i], 1);
     }
     mbar_init(accfull, 1);
-    mbar_init(accempty, 128);
+    mbar_init(accempty, 4);  // one arrival per epilogue warp
     mbar_init(done, 1);
     for (int i = 0; i < kR; ++i) {
       mbar_init(&rfull[i], 64);
-      mbar_init(&rempty[i], 256);
+      mbar_init(&rempty[i], 8);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -254,8 +267,7 @@ search_tc_kernel(TqConsts c, const uint8_t *__restrict__ bst, const float *__res
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
   }
   for (int i = tid; i < kTcQ * 4; i += kTcThreads) skq[i] = kq[(int64_t)tile * kTcQ * 4 + i];
-  for (int i = tid; i < kTcQ; i += kTcThreads) sthr[i] = -INFINITY;
-  for (int i = tid; i < 4 * kTcQ * k; i += kTcThreads) {
+  for (int i = tid; i < kTcQ * k; i += kTcThreads) {
     ls[i] = -INFINITY;
     li[i] = INT64_MAX;
   }
@@ -269,15 +281,15 @@ search_tc_kernel(TqConsts c, const uint8_t *__restrict__ bst, const float *__res
     // Stages run chunk-major (for each 128 coordinates: the code planes, the parity plane at
     // 3 bits, the sign plane).  A row's words for one chunk (16 B per stored plane) arrive in the
     // staging ring from the loader warps; this thread issues no global loads, so its proxy fences
-    // only wait for its own shared-memory stores.  Two threads per row, each expanding half of
-    // the chunk's 128 coordinates.
+    // only wait for its own shared-memory stores.  Two groups of four warps (one row per thread)
+    // expand alternate planes of a chunk at the same time.
     const int r = tid & (kTcM - 1), hh = tid >> 7;
-    int64_t s = 0;
     bool ok = true;
     const int64_t nchunks = (int64_t)nblk * NC;
     for (int64_t g = 0; g < nchunks && ok; ++g) {
       const int rs = (int)(g % kR);
-      if (!mbar_wait_bounded(&rfull[rs], (unsigned)(g / kR) & 1u)) {
+      // warp-uniform outcome of the bounded waits (each warp arrives once per barrier phase)
+      if (!__all_sync(TQ_FULL_MASK, mbar_wait_bounded(&rfull[rs], (unsigned)(g / kR) & 1u))) {
         ok = false;
         break;
       }
@@ -286,31 +298,35 @@ search_tc_kernel(TqConsts c, const uint8_t *__restrict__ bst, const float *__res
       const uint4 *st = reinterpret_cast<const uint4 *>(smem + L.stg) + (size_t)rs * LP * kTcM + r;
 #pragma unroll
       for (int P = 0; P < LP; ++P) cur[P] = gr < r_end ? st[P * kTcM] : make_uint4(0u, 0u, 0u, 0u);
-      mbar_arrive1(&rempty[rs]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive1(&rempty[rs]);
       uint4 par = make_uint4(0u, 0u, 0u, 0u);
       if (BK == 3)
         par = make_uint4(cur[0].x ^ cur[1].x ^ cur[2].x, cur[0].y ^ cur[1].y ^ cur[2].y,
                          cur[0].z ^ cur[1].z ^ cur[2].z, cur[0].w ^ cur[1].w ^ cur[2].w);
 #pragma unroll
-      for (int P = 0; P < PL; ++P, ++s) {
+      for (int P = 0; P < PL; ++P) {
+        if ((P & 1) != hh) continue;
+        const int64_t s = g * PL + P;
         const uint4 wv = P < BK ? cur[P] : (P == PL - 1 ? cur[BK] : par);
         const int slot = (int)(s % ns);
-        if (s >= ns && !mbar_wait_bounded(&empty[slot], (unsigned)((s / ns) - 1) & 1u)) {
+        if (!__all_sync(TQ_FULL_MASK, s < ns || mbar_wait_bounded(&empty[slot], (unsigned)((s / ns) - 1) & 1u))) {
           ok = false;
           break;
         }
         unsigned char *a = smem + (size_t)slot * kTcStage + (r >> 3) * 1024 + (r & 7) * 16;
         const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-        for (int kh = 0; kh < 4; ++kh) {
-          const int kg = 4 * hh + kh;
+        for (int kg = 0; kg < 8; ++kg) {
           const uint32_t h = (wd[kg >> 1] >> (16 * (kg & 1))) & 0xFFFFu;
           *reinterpret_cast<uint4 *>(a + kg * 128) =
               make_uint4(nib_bytes(h & 0xFu), nib_bytes((h >> 4) & 0xFu), nib_bytes((h >> 8) & 0xFu),
                          nib_bytes(h >> 12));
         }
+        // each thread makes its stores visible to the tensor core; one arrival per warp
         asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-        mbar_arrive1(&afull[slot]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive1(&afull[slot]);
       }
     }
     if (!ok) *abort_flag = 1;
@@ -415,11 +431,14 @@ search_tc_kernel(TqConsts c, const uint8_t *__restrict__ bst, const float *__res
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue: scores and top-k
+    // Thread = row for the scores (its tensor-memory lane), written to a [query][row] tile; then
+    // warp ew keeps the sorted top-k of queries ew, ew + 4, ..., scanning the tile's 128 rows per
+    // query against the list's k-th entry.  Named barrier 1 (the 128 epilogue threads) orders the
+    // tile between the two phases.
     const int quarter = warp & 3, ew = warp - kTcWEpi;
     const int row = 32 * quarter + lane;
-    float *wls = ls + (size_t)ew * kTcQ * k;
-    int64_t *wli = li + (size_t)ew * kTcQ * k;
     const uint32_t tl = tmem + ((uint32_t)(32 * quarter) << 16);
+    const int qn = min(kTcQ, nq - tile * kTcQ);
     bool ok = true;
     // this block's norms are loaded before the wait for its accumulators
     int64_t gr = r_begin + row;
@@ -429,13 +448,13 @@ search_tc_kernel(TqConsts c, const uint8_t *__restrict__ bst, const float *__res
       qg = c.qjl_scale * db.rnorm[gr];
     }
     for (int b = 0; b < nblk; ++b) {
-      const bool rvalid = gr < r_end;
-      if (!mbar_wait_bounded(accfull, (unsigned)b & 1u) || *abort_flag) {
+      // all four warps go on (the previous block's top-k has finished reading the tile) or all stop
+      const bool got = mbar_wait_bounded(accfull, (unsigned)b & 1u) && !*abort_flag;
+      if (!epi_all(got)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float sc[kTcQ];
 #pragma unroll 1
       for (int qb = 0; qb < kTcQ / 16; ++qb) {
         uint32_t v[3][16];
@@ -457,38 +476,45 @@ search_tc_kernel(TqConsts c, const uint8_t *__restrict__ bst, const float *__res
         for (int i = 0; i < 16; ++i) {
           const int q = 16 * qb + i;
           const float ds = (float)(int)v[0][i] + 256.f * (float)(int)v[1][i] + 65536.f * (float)(int)v[2][i];
-          sc[q] = nrm * fmaf(qg, fmaf(ds, skq[4 * q + 1], -skq[4 * q + 3]), a[i]);
+          sct[q * kTcM + row] = nrm * fmaf(qg, fmaf(ds, skq[4 * q + 1], -skq[4 * q + 3]), a[i]);
         }
       }
       // the accumulators may be overwritten by the next block now
       tc_fence_before();
-      mbar_arrive1(accempty);
-      const int64_t g_this = gr;
+      __syncwarp();
+      if (lane == 0) mbar_arrive1(accempty);
+      const int64_t r0 = r_begin + (int64_t)b * kTcM;
+      const int nr = (int)min((int64_t)kTcM, r_end - r0);
       gr += kTcM;
       if (b + 1 < nblk && gr < r_end) {
         nrm = db.norm[gr];
         qg = c.qjl_scale * db.rnorm[gr];
       }
-      const int qn = min(kTcQ, nq - tile * kTcQ);
-      volatile float *vthr = sthr;
+      asm volatile("bar.sync 1, 128;\n" ::: "memory");
 #pragma unroll 1
-      for (int q = 0; q < qn; ++q) {
-        // a row below any warp list's k-th score cannot reach the shard's top-k
-        const float sq = sc[q];
-        const bool cand = rvalid && !(sq < vthr[q]);
-        const unsigned m = __ballot_sync(TQ_FULL_MASK, cand);
-        if (m == 0u) continue;
-        float *Ls = wls + q * k;
-        int64_t *Li = wli + q * k;
+      for (int q = ew; q < qn; q += 4) {
+        float *Ls = ls + q * k;
+        int64_t *Li = li + q * k;
+        const float ts = Ls[k - 1];
+        const int64_t ti = Li[k - 1];
+        // lane l holds rows 4 l .. 4 l + 3
+        const float4 v4 = *reinterpret_cast<const float4 *>(sct + q * kTcM + 4 * lane);
+        const float sv[4] = {v4.x, v4.y, v4.z, v4.w};
+        bool cj[4], any = false;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          cj[j] = 4 * lane + j < nr && tq_better(sv[j], r0 + 4 * lane + j, ts, ti);
+          any |= cj[j];
+        }
+        if (__ballot_sync(TQ_FULL_MASK, any) == 0u) continue;
         float bs = lane < k ? Ls[lane] : -INFINITY;
         int64_t bi = lane < k ? Li[lane] : INT64_MAX;
-        warp_topk_insert(bs, bi, k, sq, g_this, cand);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) warp_topk_insert(bs, bi, k, sv[j], r0 + 4 * lane + j, cj[j]);
         if (lane < k) {
           Ls[lane] = bs;
           Li[lane] = bi;
         }
-        const float kth = __shfl_sync(TQ_FULL_MASK, bs, k - 1);
-        if (lane == 0 && kth > vthr[q]) vthr[q] = kth;  // a racing lower write only weakens the filter
         __syncwarp();
       }
     }
@@ -510,17 +536,10 @@ search_tc_kernel(TqConsts c, const uint8_t *__restrict__ bst, const float *__res
     for (int qi = ew; qi < kTcQ; qi += 4) {
       const int q = tile * kTcQ + qi;
       if (q >= nq) break;
-      float bs = -INFINITY;
-      int64_t bi = INT64_MAX;
-      for (int w2 = 0; w2 < 4; ++w2) {
-        const float s = lane < k ? ls[((size_t)w2 * kTcQ + qi) * k + lane] : -INFINITY;
-        const int64_t i = lane < k ? li[((size_t)w2 * kTcQ + qi) * k + lane] : INT64_MAX;
-        warp_topk_insert(bs, bi, k, s, i, lane < k && i != INT64_MAX);
-      }
       if (lane < k) {
         const int64_t o = ((int64_t)q * shards + shard) * k + lane;
-        cand_s[o] = bs;
-        cand_i[o] = bi;
+        cand_s[o] = ls[qi * k + lane];
+        cand_i[o] = li[qi * k + lane];
       }
     }
   }
