@@ -10,16 +10,16 @@
 //
 // With many queries this is GEMM-shaped, so it runs on the 5th-generation tensor cores: one
 // `tcgen05.mma.kind::i8` per (128 rows, 192 columns, 32 coordinates), A = the rows' plane bits as
-// 0/1 bytes (u8), B = the query values in 24-bit fixed point per query, three signed byte limbs
-// (column = limb · 64 + query), int32 accumulators in tensor memory (code planes and sign plane
-// apart, 192 columns each).  The int32 sums are exact; the only roundings are the fixed-point
+// 0/1 bytes (u8) in tensor memory, B = the query values in 24-bit fixed point per query, three
+// signed byte limbs (column = limb · 64 + query) in shared memory, int32 accumulators in tensor
+// memory (code planes and sign plane apart, 192 columns each).  The int32 sums are exact; the only roundings are the fixed-point
 // quantisation of the query values (2^-23 of each query's largest term) and the float combination
 // of the limb sums.
 //
 // A CTA takes 64 queries and one shard of rows, in 128-row blocks.  Warp roles:
-//   warps 0-7   expand the rows' packed bits to bytes in shared memory (two groups of four warps,
-//               one row per thread, alternate planes), one stage = (128 coordinates, plane), in
-//               the canonical K-major no-swizzle layout;
+//   warps 0-7   expand the rows' packed bits to bytes in tensor memory (two groups of four warps,
+//               one row per thread = its lane, alternate planes), one stage = (128 coordinates,
+//               plane) = 32 columns, in one of four free 32-column slots;
 //   warp 8      allocates tensor memory and issues the MMAs (one thread), committing each stage
 //               back to its producers and each block to the epilogue;
 //   warp 9      streams the query stages (prepared once per call in the same layout) by bulk copy;
@@ -42,17 +42,18 @@ constexpr int kTcQ = 64;                  // queries per CTA
 constexpr int kTcN = 3 * kTcQ;            // MMA N: three limbs per query
 constexpr int kTcM = 128;                 // rows per block (MMA M)
 constexpr int kTcKC = 128;                // coordinates per stage
-constexpr int kTcABytes = kTcM * kTcKC;   // 16 KB
-constexpr int kTcBBytes = kTcN * kTcKC;   // 24 KB
-constexpr int kTcStage = kTcABytes + kTcBBytes;
+constexpr int kTcBBytes = kTcN * kTcKC;   // 24 KB of query operand per stage (shared memory)
+constexpr int kTcStages = 4;              // A stages live in the four free 32-column tensor-memory slots
 constexpr int kTcThreads = 512;
 // warp roles
 constexpr int kTcWMma = 8, kTcWB = 9, kTcWEpi = 10, kTcWLoad = 14;
 
 // row-word staging ring depth (chunks) for lp stored planes per row
-__host__ __device__ constexpr int tc_ring(int lp) { return lp <= 2 ? 4 : 2; }
+__host__ __device__ constexpr int tc_ring(int lp) { return lp <= 2 ? 8 : 4; }
 constexpr int kTcMaxK = 16;
-constexpr uint32_t kTcCols = 512;         // tensor-memory columns: code sums at 0, sign sums at 256
+// tensor-memory columns: code sums [0, 192), sign sums [256, 448), A stages at 192, 224, 448, 480
+constexpr uint32_t kTcCols = 512;
+__host__ __device__ constexpr uint32_t tc_acol(int slot) { return slot < 2 ? 192u + 32u * slot : 448u + 32u * (slot - 2); }
 
 template <int BK, int D>
 struct TcShape {
@@ -73,7 +74,7 @@ __host__ __device__ inline TcLayout tc_layout(int k, int ns, int lp) {
   auto up16 = [](size_t x) { return (x + 15) & ~(size_t)15; };
   TcLayout L;
   L.ns = ns;
-  L.stg = (size_t)ns * kTcStage;                      // [ring][lp][128 rows][16 B]
+  L.stg = (size_t)ns * kTcBBytes;                     // [ring][lp][128 rows][16 B]
   L.kq = L.stg + (size_t)tc_ring(lp) * lp * kTcM * 16;
   L.sct = L.kq + kTcQ * 16;                           // block scores [64 q][128 rows] f32
   L.ls = L.sct + (size_t)kTcQ * kTcM * 4;             // per query sorted top-k [64 q][k]
@@ -100,6 +101,27 @@ __device__ __forceinline__ void umma_i8(uint32_t dtmem, uint64_t da, uint64_t db
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n}\n" ::"r"(dtmem),
       "l"(da), "l"(db), "r"(idesc), "r"(accum), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+      : "memory");
+}
+
+// A (M x K bytes) from tensor memory: lane = row, four K-bytes per 32-bit column, 8 columns per MMA
+__device__ __forceinline__ void umma_i8_ta(uint32_t dtmem, uint32_t atmem, uint64_t db, uint32_t idesc,
+                                           uint32_t accum) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n}\n" ::"r"(dtmem),
+      "r"(atmem), "l"(db), "r"(idesc), "r"(accum), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+      "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+      "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
       : "memory");
 }
 
@@ -280,9 +302,8 @@ search_tc_kernel(TqConsts c, const uint8_t *__restrict__ bst, const float *__res
     // ------------------------------------------------------------ producers: bits -> bytes
     // Stages run chunk-major (for each 128 coordinates: the code planes, the parity plane at
     // 3 bits, the sign plane).  A row's words for one chunk (16 B per stored plane) arrive in the
-    // staging ring from the loader warps; this thread issues no global loads, so its proxy fences
-    // only wait for its own shared-memory stores.  Two groups of four warps (one row per thread)
-    // expand alternate planes of a chunk at the same time.
+    // staging ring from the loader warps.  Two groups of four warps (one row per thread, the row
+    // being the thread's tensor-memory lane) expand alternate planes of a chunk at the same time.
     const int r = tid & (kTcM - 1), hh = tid >> 7;
     bool ok = true;
     const int64_t nchunks = (int64_t)nblk * NC;
@@ -314,17 +335,20 @@ search_tc_kernel(TqConsts c, const uint8_t *__restrict__ bst, const float *__res
           ok = false;
           break;
         }
-        unsigned char *a = smem + (size_t)slot * kTcStage + (r >> 3) * 1024 + (r & 7) * 16;
+        // the row's 128 coordinates as 0/1 bytes, 4 per tensor-memory column of its lane
         const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
+        uint32_t o[32];
 #pragma unroll
         for (int kg = 0; kg < 8; ++kg) {
           const uint32_t h = (wd[kg >> 1] >> (16 * (kg & 1))) & 0xFFFFu;
-          *reinterpret_cast<uint4 *>(a + kg * 128) =
-              make_uint4(nib_bytes(h & 0xFu), nib_bytes((h >> 4) & 0xFu), nib_bytes((h >> 8) & 0xFu),
-                         nib_bytes(h >> 12));
+          o[4 * kg] = nib_bytes(h & 0xFu);
+          o[4 * kg + 1] = nib_bytes((h >> 4) & 0xFu);
+          o[4 * kg + 2] = nib_bytes((h >> 8) & 0xFu);
+          o[4 * kg + 3] = nib_bytes(h >> 12);
         }
-        // each thread makes its stores visible to the tensor core; one arrival per warp
-        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+        tmem_st32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + tc_acol(slot), o);
+        asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive1(&afull[slot]);
       }
@@ -391,11 +415,10 @@ search_tc_kernel(TqConsts c, const uint8_t *__restrict__ bst, const float *__res
           const int P = j % PL;  // chunk-major stages
           const uint32_t acc = tmem + (P == PL - 1 ? 256u : 0u);
           const bool first = j == 0 || j == PL - 1;
-          const uint32_t a0 = sbase + (uint32_t)slot * kTcStage, b0 = a0 + kTcABytes;
+          const uint32_t a0 = tmem + tc_acol(slot), b0 = sbase + (uint32_t)slot * kTcBBytes;
 #pragma unroll
           for (int t = 0; t < kTcKC / 32; ++t)
-            umma_i8(acc, umma_desc(a0 + 256u * t, 128u, 1024u), umma_desc(b0 + 256u * t, 128u, 1024u), idesc,
-                    (first && t == 0) ? 0u : 1u);
+            umma_i8_ta(acc, a0 + 8u * t, umma_desc(b0 + 256u * t, 128u, 1024u), idesc, (first && t == 0) ? 0u : 1u);
           umma_commit(&empty[slot]);
         }
         if (ok) umma_commit(accfull);
@@ -419,7 +442,7 @@ search_tc_kernel(TqConsts c, const uint8_t *__restrict__ bst, const float *__res
           break;
         }
         mbar_expect_arrive(&bfull[slot], kTcBBytes);
-        bulk_g2s(smem + (size_t)slot * kTcStage + kTcABytes, src + (s % SPB) * kTcBBytes, kTcBBytes, &bfull[slot]);
+        bulk_g2s(smem + (size_t)slot * kTcBBytes, src + (s % SPB) * kTcBBytes, kTcBBytes, &bfull[slot]);
       }
       if (!ok) {
         *abort_flag = 1;
@@ -545,10 +568,10 @@ search_tc_kernel(TqConsts c, const uint8_t *__restrict__ bst, const float *__res
   }
 }
 
-constexpr size_t kTcSmemPerCta = 232448;
+constexpr size_t kTcSmemPerCta = 232448, kTcSmemOneCta = 120 * 1024;
 
 inline int tc_stages(int k, int lp) {
-  int ns = 6;
+  int ns = kTcStages;
   while (ns > 2 && tc_layout(k, ns, lp).total > kTcSmemPerCta) --ns;
   return ns;
 }
@@ -574,6 +597,9 @@ cudaError_t launch_tc(const TqConsts &c, int shards, const float *qr, const floa
   float *kq = reinterpret_cast<float *>(bst + tq_align_up((int64_t)tiles * TS::SPB * kTcBBytes, 256));
   const int ns = tc_stages(k, BK + 1);
   const TcLayout L = tc_layout(k, ns, BK + 1);
+  // more than half an SM's shared memory, so that one CTA (and one 512-column tensor-memory
+  // allocation) is resident per SM
+  const size_t smem = std::max(L.total, kTcSmemOneCta);
   tq_prof_begin(TQK_SEARCH_SCAN, st);
   search_tc_scale_kernel<D><<<(tiles * kTcQ + 7) / 8, 256, 0, st>>>(c, qr, p, nq, tiles * kTcQ, kq);
   cudaError_t e = cudaGetLastError();
@@ -581,10 +607,10 @@ cudaError_t launch_tc(const TqConsts &c, int shards, const float *qr, const floa
     search_tc_bfrag_kernel<BK, D><<<dim3((unsigned)tiles, (unsigned)TS::SPB), 256, 0, st>>>(c, qr, p, nq, kq, bst);
     e = cudaGetLastError();
   }
-  if (e == cudaSuccess) e = tq_smem_limit(reinterpret_cast<const void *>(search_tc_kernel<BK, D>), (int)L.total);
+  if (e == cudaSuccess) e = tq_smem_limit(reinterpret_cast<const void *>(search_tc_kernel<BK, D>), (int)smem);
   if (e == cudaSuccess) {
     const int64_t rows_per_shard = ((n + shards - 1) / shards + kTcM - 1) / kTcM * kTcM;
-    search_tc_kernel<BK, D><<<dim3((unsigned)shards, (unsigned)tiles), kTcThreads, L.total, st>>>(
+    search_tc_kernel<BK, D><<<dim3((unsigned)shards, (unsigned)tiles), kTcThreads, smem, st>>>(
         c, bst, kq, nq, db, n, k, rows_per_shard, shards, ns, cand_s, cand_i);
     e = cudaGetLastError();
   }
