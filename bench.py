@@ -176,6 +176,12 @@ def max_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
+def aggregate_rate(world: int, units_per_step: float, steps: int, ms: float) -> float:
+    """Whole-job throughput under weak scaling: every rank processes units_per_step per step, and
+    ms is the slowest rank's time for `steps` steps."""
+    return world * units_per_step * steps / (ms / 1e3)
+
+
 def barrier(world: int):
     if world > 1:
         import torch.distributed as dist
@@ -497,8 +503,8 @@ def ours_arm(args, world, rank):
     ms = time_graph_steps(graphs, args.steps, args.warmup, world, sampler)
     ms = max_over_ranks(ms, world)
     ms_step = ms / args.steps
-    value = world * bench.keys_per_step * args.steps / (ms / 1e3)
-    hbm_gbs = world * bench.bytes_per_step * args.steps / (ms / 1e3) / 1e9
+    value = aggregate_rate(world, bench.keys_per_step, args.steps, ms)
+    hbm_gbs = aggregate_rate(world, bench.bytes_per_step, args.steps, ms) / 1e9
 
     prof_steps = min(args.steps, N_LAYERS)
     prof = profile_kernels(bench, prof_steps)
@@ -520,7 +526,7 @@ def ours_arm(args, world, rank):
     e2e_steps = min(args.steps, 500)
     e_ms, h2d, d2h = time_e2e(bench, e2e_steps, min(args.warmup, 20))
     e_ms = max_over_ranks(e_ms, world)
-    e2e_value = world * bench.keys_per_step * e2e_steps / (e_ms / 1e3)
+    e2e_value = aggregate_rate(world, bench.keys_per_step, e2e_steps, e_ms)
 
     enc_vps, enc_ms = time_encode(bench)
     enc_ms = max_over_ranks(enc_ms, world)
@@ -547,10 +553,11 @@ def ours_arm(args, world, rank):
     return 0
 
 
-def search_arm(args):
+def search_arm(args, world=1, rank=0):
     """Vector search at 10^6 rows x d 1024: encode the database (unit vectors, fp32), then top-10
     for 1000 queries.  Inputs are drawn on the device with a seeded generator (same recipe as the
-    parity tests: N(0, I) rows L2-normalised)."""
+    parity tests: N(0, I) rows L2-normalised).  Under torchrun every rank searches its own
+    database (weak scaling); times are the slowest rank's and rank 0 prints the line."""
     import torch
     from kv_cache_vector_06_b200 import tq
     import synth
@@ -561,7 +568,7 @@ def search_arm(args):
     dev = torch.device("cuda", torch.cuda.current_device())
     ctx = tq.Context(d, mse, m, synth.rotation_signs(d, 11), synth.qjl_matrix(m, d, 12), device=dev.index)
     g = torch.Generator(device=dev)
-    g.manual_seed(13)
+    g.manual_seed(13 + rank)
     X = torch.randn(n, d, generator=g, device=dev)
     X /= X.norm(dim=1, keepdim=True)
     Q = torch.randn(nq, d, generator=g, device=dev)
@@ -572,12 +579,13 @@ def search_arm(args):
     tq.encode_kv(ctx, X, db, ws=ws_e)  # warm-up
     torch.cuda.synchronize()
     reps = max(1, min(args.steps, 5))
+    barrier(world)
     start.record()
     for _ in range(reps):
         tq.encode_kv(ctx, X, db, ws=ws_e)
     end.record()
     torch.cuda.synchronize()
-    enc_ms = start.elapsed_time(end) / reps
+    enc_ms = max_over_ranks(start.elapsed_time(end), world) / reps
     del X, ws_e
     row_bytes = packed_bytes_per_key(d, mse, m)
     ws_s = torch.empty(tq.search_workspace_size(ctx, nq, n, k), dtype=torch.uint8, device=dev)
@@ -586,6 +594,7 @@ def search_arm(args):
     for _ in range(max(1, min(args.warmup, 3))):
         tq.search_topk(ctx, Q, db, k, out_scores=sc, out_idx=ix, ws=ws_s)
     torch.cuda.synchronize()
+    barrier(world)
     sampler = ClockSampler(dev.index)
     with sampler:
         start.record()
@@ -593,7 +602,24 @@ def search_arm(args):
             tq.search_topk(ctx, Q, db, k, out_scores=sc, out_idx=ix, ws=ws_s)
         end.record()
         torch.cuda.synchronize()
-    ms = start.elapsed_time(end) / reps
+    ms = max_over_ranks(start.elapsed_time(end), world) / reps
+    # end to end through the API: each call's queries from pinned host memory, its top-k back to
+    # pinned host memory
+    h_q = Q.cpu().pin_memory()
+    h_s = torch.empty(nq, k, dtype=torch.float32).pin_memory()
+    h_i = torch.empty(nq, k, dtype=torch.int64).pin_memory()
+    d_q = torch.empty_like(Q)
+    torch.cuda.synchronize()
+    barrier(world)
+    start.record()
+    for _ in range(reps):
+        d_q.copy_(h_q, non_blocking=True)
+        tq.search_topk(ctx, d_q, db, k, out_scores=sc, out_idx=ix, ws=ws_s)
+        h_s.copy_(sc, non_blocking=True)
+        h_i.copy_(ix, non_blocking=True)
+    end.record()
+    torch.cuda.synchronize()
+    e_ms = max_over_ranks(start.elapsed_time(end), world) / reps
     peaks, src = measured_peaks()
     db_bytes = n * row_bytes
     # Tensor roofline of the scan: the estimate is a contraction of the rows' bit planes (mse code
@@ -605,7 +631,8 @@ def search_arm(args):
     int8_peak = peaks["bf16_tflops"] * 2
     terms = nq * n * (d + m) / (ms / 1e3)
     line = {
-        "metric": "search queries/s", "value": nq / (ms / 1e3), "unit": "queries/s", "n_gpus": 1,
+        "metric": "search queries/s", "value": aggregate_rate(world, nq, 1, ms), "unit": "queries/s",
+        "n_gpus": world,
         "steps": reps, "warmup": max(1, min(args.warmup, 3)), "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": f"vector search: 10^6 unit vectors d 1024, {args.search_bits} bits/coord "
@@ -629,11 +656,17 @@ def search_arm(args):
                      "frac": int8_ops / (ms / 1e3) / 1e12 / int8_peak, "traffic": None,
                      "note": "int8 ops of the bit-plane contraction (2 x %d planes x d x 3 limbs per query and row) "
                              "per search call; peak = measured bf16 x 2 (dense int8:bf16 ratio), %s" % (planes, src)},
+        "e2e": {"value": aggregate_rate(world, nq, 1, e_ms), "unit": "queries/s",
+                "h2d_bytes_per_step": h_q.numel() * h_q.element_size(),
+                "d2h_bytes_per_step": h_s.numel() * 4 + h_i.numel() * 8},
+        # per call: query rotation, query projection, per-query scales, query operand, scan, merge
+        "gpu_launches": 6 * reps,
         "clocks": sampler.summary(),
     }
-    if not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = search_cpu_baseline(ctx_d=d, mse=mse, m=m, row_count=n)
-    print(json.dumps(line), flush=True)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
     return 0
 
 
@@ -669,7 +702,7 @@ def main(argv=None):
         if args.impl == "reference":
             return reference_arm(args, world, rank)
         if args.workload == "search":
-            return search_arm(args)
+            return search_arm(args, world, rank)
         return ours_arm(args, world, rank)
     finally:
         if world > 1:
