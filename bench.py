@@ -635,7 +635,8 @@ def search_arm(args, world=1, rank=0):
         "n_gpus": world,
         "steps": reps, "warmup": max(1, min(args.warmup, 3)), "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": f"vector search: 10^6 unit vectors d 1024, {args.search_bits} bits/coord "
+        "config": {"workload": f"vector search: {'10^6' if n == 1_000_000 else n} unit vectors d 1024, "
+                               f"{args.search_bits} bits/coord "
                                f"({mse} MSE + QJL m 1024), 1000 queries, top-10", "rows": n, "d": d, "queries": nq,
                    "k": k, "l2": "database (%.0f MB packed) larger than L2" % (db_bytes / 1e6)},
         "scores_per_s": nq * n / (ms / 1e3),
