@@ -96,14 +96,6 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46);
 }
 
-__device__ __forceinline__ void umma_i8(uint32_t dtmem, uint64_t da, uint64_t db, uint32_t idesc, uint32_t accum) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n}\n" ::"r"(dtmem),
-      "l"(da), "l"(db), "r"(idesc), "r"(accum), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
-      : "memory");
-}
-
 // A (M x K bytes) from tensor memory: lane = row, four K-bytes per 32-bit column, 8 columns per MMA
 __device__ __forceinline__ void umma_i8_ta(uint32_t dtmem, uint32_t atmem, uint64_t db, uint32_t idesc,
                                            uint32_t accum) {
