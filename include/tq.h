@@ -233,9 +233,18 @@ tq_status tq_attend_decode_noalloc(const tq_ctx *kctx, const tq_ctx *vctx, const
  *   q           device [nq][d] of dtype
  *   out_scores  device fp32 [nq][k]
  *   out_idx     device int64 [nq][k]
- *   ws          device workspace of tq_search_workspace_size() bytes
+ *   ws          device workspace of tq_search_workspace_size() bytes (16-byte aligned; covers
+ *               every scan the call may choose)
+ * The scan depends on the shape. d in {128, 256, 512, 1024} with qjl_m = d, 1-3 MSE bits and a
+ * symmetric codebook runs on tensor cores:
+ *   - nq >= 32 and k <= 16: tcgen05 MMAs, 64 queries per CTA;
+ *   - otherwise mma.sync, 8 queries per CTA (norm and rnorm 16-byte aligned);
+ *   - any other shape, or unaligned norms for the second case: CUDA cores.
+ * All give the same top-k within the documented tolerances (the tensor-core scans round each
+ * query term to 2^-23 of the query's largest term).
  * Errors: TQ_EINVAL (nulls, k > n, alignment, ws too small), TQ_EUNSUPPORTED (k > 32),
- * TQ_ECUDA. */
+ * TQ_ECUDA.  A scan that gave up waiting for its copies sets TQ_DEVFLAG_STAGING_TIMEOUT (see
+ * tq_device_status) and leaves its outputs unspecified. */
 tq_status tq_search_workspace_size(const tq_ctx *ctx, int32_t nq, int64_t n, int32_t k,
                                    size_t *bytes);
 tq_status tq_search_topk(const tq_ctx *ctx, const void *q, tq_dtype dtype, int32_t nq,
