@@ -635,11 +635,7 @@ def search_arm(args, world=1, rank=0):
         "n_gpus": world,
         "steps": reps, "warmup": max(1, min(args.warmup, 3)), "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": f"vector search: {'10^6' if n == 1_000_000 else n} unit vectors d 1024, "
-                               f"{args.search_bits} bits/coord "
-                               f"({mse} MSE + QJL m 1024), 1000 queries, top-10", "rows": n, "d": d, "queries": nq,
-                   "k": k, "l2": "database (%.0f MB packed) %s than the 126 MB L2" % (
-                       db_bytes / 1e6, "larger" if db_bytes > 126e6 else "smaller")},
+        "config": search_config(args, n, db_bytes),
         "scores_per_s": nq * n / (ms / 1e3),
         "database_passes_per_s": 1e3 / ms,
         "hbm": {"database_bytes": db_bytes, "gbs_one_read_per_query": nq * db_bytes / (ms / 1e3) / 1e9,
@@ -669,6 +665,56 @@ def search_arm(args, world=1, rank=0):
         line["cpu_baseline"] = search_cpu_baseline(ctx_d=d, mse=mse, m=m, row_count=n)
     if rank == 0:
         print(json.dumps(line), flush=True)
+    return 0
+
+
+def search_config(args, n: int, db_bytes: int) -> dict:
+    mse = args.search_bits - 1
+    return {"workload": f"vector search: {'10^6' if n == 1_000_000 else n} unit vectors d 1024, "
+                        f"{args.search_bits} bits/coord ({mse} MSE + QJL m 1024), 1000 queries, top-10",
+            "rows": n, "d": 1024, "queries": 1000, "k": 10,
+            "l2": "database (%.0f MB packed) %s than the 126 MB L2" % (
+                db_bytes / 1e6, "larger" if db_bytes > 126e6 else "smaller")}
+
+
+def reference_search_arm(args, world, rank):
+    """The oracle on the search workload, on the host cores: each step scores one query against a
+    4096-row sample of the database (encoded by the oracle beforehand, untimed) and takes its
+    top-10; queries/s is scaled to the full database."""
+    if rank != 0:
+        return 0
+    import synth
+    from oracle import codebook as ocb, encode as oenc, estimate as oest, search as osearch
+    d, n, rows, k = 1024, args.search_rows, 4096, 10
+    mse, m = args.search_bits - 1, 1024
+    D = synth.rotation_signs(d, 11).double().numpy()
+    S = synth.qjl_matrix(m, d, 12).double().numpy()
+    c, t = ocb.codebook(d, mse)
+    enc = oenc.encode(synth.unit_rows(rows, d, seed=0).double().numpy(), D, S, c, t)
+    Q = synth.unit_rows(max(1, args.steps + args.warmup), d, seed=1).double().numpy()
+
+    def one(i):
+        qr, p = oest.prepare_query(Q[i:i + 1], D, S)
+        osearch.topk(oest.scores(qr, p, enc.norm, enc.codes, enc.rnorm, enc.bits, c), k)
+
+    for i in range(args.warmup):
+        one(args.steps + i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        one(i)
+    dt = (time.perf_counter() - t0) / args.steps * (n / rows)  # seconds per query over n rows
+    value = 1.0 / dt
+    line = {
+        "impl": "reference", "metric": "search queries/s", "value": value, "unit": "queries/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": search_config(args, n, n * packed_bytes_per_key(d, mse, m)),
+        "cpu_baseline": {"value": value, "unit": "queries/s", "cores": cpu_cores_used(), "kind": "oracle",
+                         "sample": f"each step: one query scored against {rows} oracle-encoded rows and its "
+                                   f"top-{k}, scaled to {n} rows; fp64 numpy oracle"},
+        "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
     return 0
 
 
@@ -702,6 +748,8 @@ def main(argv=None):
     world, rank, _ = dist_setup(args)
     try:
         if args.impl == "reference":
+            if args.workload == "search":
+                return reference_search_arm(args, world, rank)
             return reference_arm(args, world, rank)
         if args.workload == "search":
             return search_arm(args, world, rank)

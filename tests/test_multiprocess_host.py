@@ -74,3 +74,21 @@ def test_reference_arm_runs_on_rank_zero_only():
     args = bench.parse_args(["--impl", "reference", "--gpus", "2", "--steps", "3", "--warmup", "3"])
     # a non-zero rank returns at once, without touching the oracle
     assert bench.reference_arm(args, 2, 1) == 0
+
+
+def test_search_reference_arm_prints_one_contract_line(capsys):
+    """The oracle arm of the search workload: one JSON line with the search metric, its own
+    cpu_baseline and e2e (no host-device copies), timed on a bounded sample."""
+    import json
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.main(["--impl", "reference", "--workload", "search", "--steps", "1", "--warmup", "1"]) == 0
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["metric"] == "search queries/s" and rec["unit"] == "queries/s"
+    assert rec["value"] > 0 and rec["higher_is_better"] is True and rec["dtype"] == "f64"
+    assert rec["cpu_baseline"]["kind"] == "oracle" and rec["cpu_baseline"]["value"] == rec["value"]
+    assert rec["e2e"] == {"value": rec["value"], "unit": "queries/s", "h2d_bytes_per_step": 0,
+                          "d2h_bytes_per_step": 0}
+    assert rec["config"]["rows"] == 1_000_000 and rec["config"]["k"] == 10
