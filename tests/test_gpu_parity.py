@@ -330,6 +330,23 @@ def test_search_tcgen05_scan(tq, d, bits):
         assert np.array_equal(ss[r, 0::2], ss[r, 1::2])
 
 
+def test_search_tcgen05_bf16_queries_many_shards(tq):
+    """bf16 queries through the tcgen05 scan, with a database long enough for one shard per SM
+    (two 64-query tiles x 67 shards of 7 row blocks) and k = 16."""
+    d, bits, n, nq, k = 256, 2, 60000, 100, 16
+    q = Quantizer(d, bits, d, seed=95)
+    X = synth.unit_rows(n, d, seed=96)
+    Q = synth.unit_rows(nq, d, seed=97).to(torch.bfloat16)
+    packed = _enc(tq, q, X)
+    codes, sbits, norm, rnorm = unpack(q, packed)
+    ref_full = oracle_scores_from_packed(q, Q.double().numpy(), codes, sbits, norm, rnorm)
+    ref_s, _ = osearch.topk(ref_full, k)
+    s, i = tq.search_topk(q.ctx, Q.cuda(), packed, k)
+    torch.cuda.synchronize()
+    assert tq.device_status() == 0
+    assert_topk_equivalent(s.cpu().numpy(), i.cpu().numpy(), lambda r, idx: ref_full[r, idx], ref_s)
+
+
 @pytest.mark.parametrize("d,bits", [(8, 1), (64, 2), (128, 3), (128, 4), (256, 2)])
 def test_encode_block16_layout(tq, d, bits):
     """Values in the token-transposed 16-slot block layout, written at scattered slots (several
