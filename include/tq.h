@@ -29,7 +29,7 @@
  *
  * Supported sizes: d (vector length) a power of two in [8, 1024]; mse_bits in [1, 4];
  * qjl_m = 0 (MSE stage only) or a multiple of 32 in [32, 1024]; attention group size
- * n_q_heads / n_kv_heads in {1, 2, 4, 8}; search k in [1, 32].
+ * n_q_heads / n_kv_heads in {1, 2, 4, 8}; search k in [1, 1024].
  */
 #ifndef TQ_H
 #define TQ_H
@@ -47,7 +47,8 @@ typedef enum {
   TQ_EUNSUPPORTED = 2,  /* well-formed but outside the supported sizes listed above */
   TQ_ENOMEM = 3,        /* context creation could not allocate its constants */
   TQ_ECUDA = 4,         /* a CUDA call or kernel launch failed */
-  TQ_ETIMEOUT = 5       /* reserved for bounded device waits (no call waits on the device today) */
+  TQ_ETIMEOUT = 5       /* a kernel gave up a bounded wait for its own asynchronous copies; returned
+                           by tq_device_status, which reports it (see TQ_DEVFLAG_STAGING_TIMEOUT) */
 } tq_status;
 
 typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
@@ -235,14 +236,18 @@ tq_status tq_attend_decode_noalloc(const tq_ctx *kctx, const tq_ctx *vctx, const
  *   out_idx     device int64 [nq][k]
  *   ws          device workspace of tq_search_workspace_size() bytes (16-byte aligned; covers
  *               every scan the call may choose)
- * The scan depends on the shape. d in {128, 256, 512, 1024} with qjl_m = d, 1-3 MSE bits and a
- * symmetric codebook runs on tensor cores:
+ * The scan depends on the shape. With k <= 32, d in {128, 256, 512, 1024} with qjl_m = d, 1-3
+ * MSE bits and a symmetric codebook runs on tensor cores:
  *   - nq >= 32 and k <= 16: tcgen05 MMAs, 64 queries per CTA;
  *   - otherwise mma.sync, 8 queries per CTA (norm and rnorm 16-byte aligned);
- *   - any other shape, or unaligned norms for the second case: CUDA cores.
+ *   - any other shape with k <= 32, or unaligned norms for the second case: CUDA cores, 8 queries
+ *     per CTA, one running top-k list per warp;
+ *   - 32 < k <= 1024: CUDA cores, 4 queries per CTA, each query's running top-k kept in shared
+ *     memory with the candidates that beat its current k-th entry, sorted (bitonic) when the
+ *     buffer fills; the shards' lists are merged the same way.
  * All give the same top-k within the documented tolerances (the tensor-core scans round each
  * query term to 2^-23 of the query's largest term).
- * Errors: TQ_EINVAL (nulls, k > n, alignment, ws too small), TQ_EUNSUPPORTED (k > 32),
+ * Errors: TQ_EINVAL (nulls, k < 1, k > n, alignment, ws too small), TQ_EUNSUPPORTED (k > 1024),
  * TQ_ECUDA.  A scan that gave up waiting for its copies sets TQ_DEVFLAG_STAGING_TIMEOUT (see
  * tq_device_status) and leaves its outputs unspecified. */
 tq_status tq_search_workspace_size(const tq_ctx *ctx, int32_t nq, int64_t n, int32_t k,
@@ -265,13 +270,26 @@ tq_status tq_profile_read(int32_t index, char *name, int32_t name_len, int64_t *
                           double *total_ms);
 
 /* Device-side status of the library on `device`: the TQ_DEVFLAG_* bits raised by kernels since
- * the last clear.  Synchronizes the device first; clear != 0 resets the bits.  A kernel that
- * gives up waiting for its own asynchronous copies (after about a second) raises
- * TQ_DEVFLAG_STAGING_TIMEOUT and leaves its outputs unwritten.
- *   flags  host out
+ * the last clear.  Synchronizes the device first; clear != 0 resets the bits.  Every wait of a
+ * kernel for its own asynchronous copies (bulk copies on an mbarrier) is bounded: a kernel that
+ * gives up (after about a second) raises TQ_DEVFLAG_STAGING_TIMEOUT, waits once more (bounded)
+ * for the copies it issued, and returns without writing its outputs; the CUDA context stays
+ * usable.  The caller's current device is restored on return.
+ *   flags  host out (written whenever the device could be read, also with TQ_ETIMEOUT)
+ * Returns TQ_ETIMEOUT when TQ_DEVFLAG_STAGING_TIMEOUT is among the flags read (the outputs of the
+ * work since the last clear are then unspecified), else TQ_OK.
  * Errors: TQ_EINVAL (null flags), TQ_ECUDA. */
 #define TQ_DEVFLAG_STAGING_TIMEOUT 1
 tq_status tq_device_status(int32_t device, int32_t *flags, int32_t clear);
+
+/* Test hook for the bounded waits, off by default; the pages have no counterpart.  With
+ * polls > 0, every CTA of the tensor-core attention kernel on `device` first makes one bounded
+ * wait of `polls` polls on a shared-memory barrier that is armed for bytes no copy sends, so the
+ * wait runs out (no fault, no unbounded wait): the CTA raises TQ_DEVFLAG_STAGING_TIMEOUT, drains
+ * the copies it had already issued, and returns.  polls = 0 switches the hook off.  Synchronous
+ * with respect to the host; not for use while other work runs on the device.
+ * Errors: TQ_EINVAL (polls < 0), TQ_ECUDA. */
+tq_status tq_debug_wait_probe(int32_t device, int32_t polls);
 
 /* Thread-local description of the last error on this thread ("" if none). */
 const char *tq_last_error(void);

@@ -37,13 +37,6 @@ tq_status check_ctx(const tq_ctx *c, const char *name) {
   return TQ_OK;
 }
 
-tq_status set_device(const tq_ctx *c) {
-  int cur = -1;
-  cudaError_t e = cudaGetDevice(&cur);
-  if (e != cudaSuccess) return tq_cuda_check(e, "cudaGetDevice");
-  if (cur != c->device) return tq_cuda_check(cudaSetDevice(c->device), "cudaSetDevice");
-  return TQ_OK;
-}
 
 tq_status check_packed(const tq_ctx *c, const tq_packed &p, int64_t need, const char *name,
                        bool need_signs) {
@@ -138,11 +131,13 @@ tq_status tq_ctx_create(const tq_spec *spec, const int8_t *rot_signs, const floa
   c->sign_bytes = m > 0 ? tq_align_up((m + 7) / 8, 16) : 0;
   tq_codebook_fp64(d, spec->mse_bits, c->centroids, c->thresholds, &c->mse_per_coord);
 
-  cudaError_t e = cudaSetDevice(device);
-  if (e != cudaSuccess) {
+  DeviceScope dev_scope;
+  st = dev_scope.enter(device);
+  if (st != TQ_OK) {
     delete c;
-    return tq_cuda_check(e, "cudaSetDevice");
+    return st;
   }
+  cudaError_t e = cudaSuccess;
   float hs[1024];
   for (int j = 0; j < d; ++j) hs[j] = (float)rot_signs[j];
   e = cudaMalloc(&c->dev_signs, sizeof(float) * d);
@@ -271,7 +266,8 @@ tq_status tq_encode_kv(const tq_ctx *ctx, const void *x, tq_dtype dtype, int64_t
   tq_encode_workspace_size(ctx, n, &need);
   if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws)))
     return tq_fail(TQ_EINVAL, "workspace: %zu bytes (16-byte aligned) needed, %zu given", need, ws_bytes);
-  st = set_device(ctx);
+  DeviceScope dev_scope;
+  st = dev_scope.enter(ctx->device);
   if (st != TQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool qjl = ctx->spec.qjl_m > 0;
@@ -336,7 +332,8 @@ tq_status tq_scores(const tq_ctx *ctx, const void *q, tq_dtype dtype, int32_t nq
   const size_t need = query_prep_bytes(ctx, nq);
   if (!ws || ws_bytes < need || !aligned16(ws))
     return tq_fail(TQ_EINVAL, "workspace: %zu bytes (16-byte aligned) needed, %zu given", need, ws_bytes);
-  st = set_device(ctx);
+  DeviceScope dev_scope;
+  st = dev_scope.enter(ctx->device);
   if (st != TQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   float *qr = static_cast<float *>(ws);
@@ -411,7 +408,8 @@ tq_status tq_attend_decode(const tq_ctx *kctx, const tq_ctx *vctx, const tq_attn
   tq_attend_workspace_size(kctx, vctx, desc, &need);
   if (!ws || ws_bytes < need || !aligned16(ws))
     return tq_fail(TQ_EINVAL, "workspace: %zu bytes (16-byte aligned) needed, %zu given", need, ws_bytes);
-  st = set_device(kctx);
+  DeviceScope dev_scope;
+  st = dev_scope.enter(kctx->device);
   if (st != TQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t nq = (int64_t)desc->batch * desc->n_q_heads;
@@ -475,7 +473,8 @@ tq_status tq_decode_step(const tq_ctx *kctx, const tq_ctx *vctx, const tq_attn_d
     }
     return tq_attend_decode(kctx, vctx, desc, q, q_dtype, out, ws, att, stream);
   }
-  st = set_device(kctx);
+  DeviceScope dev_scope;
+  st = dev_scope.enter(kctx->device);
   if (st != TQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t nq = (int64_t)desc->batch * desc->n_q_heads;
@@ -491,11 +490,18 @@ tq_status tq_decode_step(const tq_ctx *kctx, const tq_ctx *vctx, const tq_attn_d
 
 tq_status tq_search_workspace_size(const tq_ctx *ctx, int32_t nq, int64_t n, int32_t k, size_t *bytes) {
   g_err[0] = 0;
+  // the supported range of k is checked first (it does not depend on the context)
+  if (k < 1) return tq_fail(TQ_EINVAL, "k=%d: must be >= 1", k);
+  if (k > kSearchMaxK) return tq_fail(TQ_EUNSUPPORTED, "k=%d: at most %d", k, kSearchMaxK);
   tq_status st = check_ctx(ctx, "ctx");
   if (st != TQ_OK) return st;
   if (!bytes) return tq_fail(TQ_EINVAL, "bytes is NULL");
-  if (nq < 0 || n < 0 || k < 1) return tq_fail(TQ_EINVAL, "nq/n/k");
-  if (k > 32) return tq_fail(TQ_EUNSUPPORTED, "k=%d: at most 32", k);
+  if (nq < 0 || n < 0) return tq_fail(TQ_EINVAL, "nq/n");
+  if (k > kSearchWarpMaxK) {  // the large-k scan only
+    const int64_t cands = (int64_t)nq * search_bigk_shards(nq, n) * k;
+    *bytes = query_prep_bytes(ctx, nq) + (size_t)tq_align_up(cands * 4, 256) + (size_t)tq_align_up(cands * 8, 256);
+    return TQ_OK;
+  }
   // room for either scan: the tensor-core one also needs 16-byte aligned norms, known only at the call
   const bool tc = search_tc_eligible(ctx->k, nq, k);
   const bool mma = search_mma_eligible(ctx->k) && nq <= kSearchMmaMaxQ;
@@ -511,11 +517,12 @@ tq_status tq_search_topk(const tq_ctx *ctx, const void *q, tq_dtype dtype, int32
                          int64_t n, int32_t k, float *out_scores, int64_t *out_idx, void *ws,
                          size_t ws_bytes, void *stream) {
   g_err[0] = 0;
+  if (k < 1) return tq_fail(TQ_EINVAL, "k=%d: must be >= 1", k);
+  if (k > kSearchMaxK) return tq_fail(TQ_EUNSUPPORTED, "k=%d: at most %d", k, kSearchMaxK);
   tq_status st = check_ctx(ctx, "ctx");
   if (st != TQ_OK) return st;
   if (nq < 0 || n < 0) return tq_fail(TQ_EINVAL, "nq < 0 or n < 0");
-  if (k < 1 || k > n) return tq_fail(TQ_EINVAL, "k=%d must be in [1, n=%lld]", k, (long long)n);
-  if (k > 32) return tq_fail(TQ_EUNSUPPORTED, "k=%d: at most 32", k);
+  if (k > n) return tq_fail(TQ_EINVAL, "k=%d must be in [1, n=%lld]", k, (long long)n);
   if (nq == 0) return TQ_OK;
   if (!q || !out_scores || !out_idx) return tq_fail(TQ_EINVAL, "q/out is NULL");
   if (dtype != TQ_F32 && dtype != TQ_BF16) return tq_fail(TQ_EINVAL, "unknown dtype %d", (int)dtype);
@@ -528,9 +535,25 @@ tq_status tq_search_topk(const tq_ctx *ctx, const void *q, tq_dtype dtype, int32
   tq_search_workspace_size(ctx, nq, n, k, &need);
   if (!ws || ws_bytes < need || !aligned16(ws))
     return tq_fail(TQ_EINVAL, "workspace: %zu bytes (16-byte aligned) needed, %zu given", need, ws_bytes);
-  st = set_device(ctx);
+  DeviceScope dev_scope;
+  st = dev_scope.enter(ctx->device);
   if (st != TQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (k > kSearchWarpMaxK) {
+    // large k: CUDA-core scan with shared-memory top-k buffers, then their merge
+    const int shards = search_bigk_shards(nq, n);
+    const int64_t cands = (int64_t)nq * shards * k;
+    char *w = static_cast<char *>(ws);
+    float *qr = reinterpret_cast<float *>(w);
+    float *p = reinterpret_cast<float *>(w + tq_align_up((int64_t)nq * ctx->spec.d * 4, 256));
+    w += query_prep_bytes(ctx, nq);
+    float *cs = reinterpret_cast<float *>(w);
+    int64_t *ci = reinterpret_cast<int64_t *>(w + tq_align_up(cands * 4, 256));
+    st = prep_queries(ctx, q, dtype, nq, qr, p, s);
+    if (st != TQ_OK) return st;
+    return tq_cuda_check(launch_search_bigk(ctx->k, shards, qr, p, nq, db, n, k, cs, ci, out_scores, out_idx, s),
+                         "search launch");
+  }
   // scan: tcgen05 (many queries), else the bit-plane mma.sync scan, else CUDA cores
   const bool tc = search_tc_eligible(ctx->k, nq, k);
   const bool mma = !tc && search_mma_eligible(ctx->k) && nq <= kSearchMmaMaxQ && aligned16(db.norm) &&

@@ -34,6 +34,9 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kG = 4;
+
+// Poll count of the test hook's bounded wait (0 = off); see tq_debug_wait_probe.
+__device__ int g_tq_wait_probe;
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 
@@ -593,6 +596,27 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
         mbar_wait_bounded(&bars[0], 0u);
       }
       __syncthreads();
+    }
+  }
+  // Test hook (tq_debug_wait_probe): one bounded wait on the merge barrier, armed for bytes that
+  // no copy sends, so that it runs out while the first sub-chunk's copies are in flight; the CTA
+  // then takes the same abort path as a staging timeout (flag, drain its copies, return).
+  const int probe = g_tq_wait_probe;
+  if (probe > 0) {
+    if (tid == 0) {
+      mbar_expect_arrive(&bars[4], 16u);
+      bool ok = false;
+      for (int i = 0; i < probe && !ok; ++i) ok = mbar_try_wait(&bars[4], 0u);
+      if (!ok) *fail = 1;
+    }
+    __syncthreads();
+    if (*fail) {
+      if (tid == 0) {
+        atomicOr(&g_tq_device_flags, kFlagStagingTimeout);
+        if (nsub > 0 || early > 0) mbar_wait_bounded(&bars[0], 0u);
+      }
+      __syncthreads();
+      return;
     }
   }
   // the query constants (2^-F_code, 2^-F_sign, Cq, Cp per head), read from shared memory where
@@ -1225,8 +1249,10 @@ cudaError_t launch_decode_step_fast(const TqConsts &kc, const TqConsts &vc, cons
 
 extern "C" tq_status tq_device_status(int32_t device, int32_t *flags, int32_t clear) {
   if (!flags) return tq_fail(TQ_EINVAL, "flags is NULL");
-  cudaError_t e = cudaSetDevice(device);
-  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  DeviceScope dev_scope;
+  tq_status st = dev_scope.enter(device);
+  if (st != TQ_OK) return st;
+  cudaError_t e = cudaDeviceSynchronize();
   int v = 0, vr = 0, vm = 0, vt = 0;
   if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&v, g_tq_device_flags, sizeof(int));
   if (e == cudaSuccess) e = rotate_device_flags(&vr, clear != 0);
@@ -1239,5 +1265,16 @@ extern "C" tq_status tq_device_status(int32_t device, int32_t *flags, int32_t cl
   v |= vr | vm | vt;
   if (e != cudaSuccess) return tq_fail(TQ_ECUDA, "device status: %s", cudaGetErrorString(e));
   *flags = v;
+  if (v & TQ_DEVFLAG_STAGING_TIMEOUT)
+    return tq_fail(TQ_ETIMEOUT, "a kernel on device %d gave up waiting for its asynchronous copies and left "
+                                "its outputs unwritten%s", device, clear ? " (flag now cleared)" : "");
   return TQ_OK;
+}
+
+extern "C" tq_status tq_debug_wait_probe(int32_t device, int32_t polls) {
+  if (polls < 0) return tq_fail(TQ_EINVAL, "polls < 0");
+  DeviceScope dev_scope;
+  tq_status st = dev_scope.enter(device);
+  if (st != TQ_OK) return st;
+  return tq_cuda_check(cudaMemcpyToSymbol(g_tq_wait_probe, &polls, sizeof(int)), "wait probe");
 }

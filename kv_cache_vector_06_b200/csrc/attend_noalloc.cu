@@ -58,13 +58,9 @@ extern "C" tq_status tq_attend_decode_noalloc(const tq_ctx *kctx, const tq_ctx *
                    "tq_attend_decode_noalloc: this request needs %zu bytes of scratch, more than the "
                    "%zu-byte static array; call tq_attend_decode with a workspace instead",
                    need, (size_t)TQ_NOALLOC_SCRATCH_BYTES);
-  int cur = -1;
-  cudaError_t e = cudaGetDevice(&cur);
-  if (e != cudaSuccess) return tq_cuda_check(e, "cudaGetDevice");
-  if (cur != kctx->device) {
-    e = cudaSetDevice(kctx->device);
-    if (e != cudaSuccess) return tq_cuda_check(e, "cudaSetDevice");
-  }
+  DeviceScope dev_scope;  // the caller's current device is restored on return
+  st = dev_scope.enter(kctx->device);
+  if (st != TQ_OK) return st;
   void *ws = nullptr;
   st = scratch_address(kctx->device, &ws);
   if (st != TQ_OK) return st;

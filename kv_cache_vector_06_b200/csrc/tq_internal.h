@@ -47,6 +47,30 @@ struct tq_ctx {
 // ---------------------------------------------------------------- host helpers (api.cu)
 tq_status tq_fail(tq_status st, const char *fmt, ...);
 tq_status tq_cuda_check(cudaError_t e, const char *what);
+// Makes a device current for the duration of one C-ABI call and restores the caller's
+// current device when the call returns (the work itself is only enqueued).
+class DeviceScope {
+ public:
+  DeviceScope() = default;
+  DeviceScope(const DeviceScope &) = delete;
+  DeviceScope &operator=(const DeviceScope &) = delete;
+  ~DeviceScope() {
+    if (prev_ >= 0) cudaSetDevice(prev_);
+  }
+  tq_status enter(int device) {
+    int cur = -1;
+    cudaError_t e = cudaGetDevice(&cur);
+    if (e != cudaSuccess) return tq_cuda_check(e, "cudaGetDevice");
+    if (cur == device) return TQ_OK;
+    e = cudaSetDevice(device);
+    if (e != cudaSuccess) return tq_cuda_check(e, "cudaSetDevice");
+    prev_ = cur;
+    return TQ_OK;
+  }
+
+ private:
+  int prev_ = -1;
+};
 
 // ---------------------------------------------------------------- profile.cu
 enum TqKernelKind {
@@ -151,6 +175,14 @@ cudaError_t launch_search_mma(const TqConsts &c, int shards, const float *qr, co
                               cudaStream_t st);
 cudaError_t launch_search_merge(int nq, int shards, int k, const float *cand_s, const int64_t *cand_i, float *out_s,
                                 int64_t *out_i, cudaStream_t st);
+// Large k (32 < k <= 1024): CUDA-core scan with per-query shared-memory top-k buffers, then a
+// merge of the shards' lists in the same way (search.cu).
+constexpr int kSearchMaxK = 1024;
+constexpr int kSearchWarpMaxK = 32;  // above this, the large-k scan
+int search_bigk_shards(int nq, int64_t n);
+cudaError_t launch_search_bigk(const TqConsts &c, int shards, const float *qr, const float *p, int nq,
+                               const tq_packed &db, int64_t n, int k, float *cand_s, int64_t *cand_i,
+                               float *out_s, int64_t *out_i, cudaStream_t st);
 cudaError_t launch_search(const TqConsts &c, const SearchPlan &plan, const float *qr,
                           const float *p, int nq, const tq_packed &db, int64_t n, int k,
                           float *cand_s, int64_t *cand_i, float *out_s, int64_t *out_i,

@@ -70,6 +70,7 @@ def _load():
         "tq_decode_step": (st, [c_void_p, c_void_p, POINTER(AttnDesc), c_void_p, c_void_p, c_int, c_int64, c_void_p,
                                 c_void_p, c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
         "tq_device_status": (st, [c_int32, POINTER(c_int32), c_int32]),
+        "tq_debug_wait_probe": (st, [c_int32, c_int32]),
         "tq_search_workspace_size": (st, [c_void_p, c_int32, c_int64, c_int32, POINTER(c_size_t)]),
         "tq_search_topk": (st, [c_void_p, c_void_p, c_int, c_int32, PackedC, c_int64, c_int32, c_void_p,
                                 c_void_p, c_void_p, c_size_t, c_void_p]),
@@ -293,6 +294,8 @@ def make_attn_desc(kctx: Context, vctx: Context, q_shape, kcache: Packed, vcache
     desc.max_seq_len = max_seq_len
     desc.k = kcache.c(kctx)
     desc.v = vcache.c(vctx)
+    # the descriptor holds raw device pointers: it keeps the tensors they point into alive
+    desc._keep = (seq_lens, block_table, kcache, vcache)
     return desc
 
 
@@ -348,11 +351,30 @@ def decode_step(kctx: Context, vctx: Context, q: torch.Tensor, k_new: torch.Tens
 DEVFLAG_STAGING_TIMEOUT = 1
 
 
+TQ_ETIMEOUT = 5
+
+
 def device_status(device: int = 0, clear: bool = False) -> int:
-    """TQ_DEVFLAG_* bits raised by the library's kernels on `device` (synchronizes it)."""
+    """TQ_DEVFLAG_* bits raised by the library's kernels on `device` (synchronizes it).  The C call
+    returns TQ_ETIMEOUT when a kernel gave up a bounded wait; the flags say so here, and
+    check_device() raises for it."""
+    f = c_int32()
+    st = LIB.tq_device_status(device, ctypes.byref(f), 1 if clear else 0)
+    if st not in (0, TQ_ETIMEOUT):
+        _check(st)
+    return f.value
+
+
+def check_device(device: int = 0, clear: bool = False):
+    """Raise TqError(TQ_ETIMEOUT) if a kernel on `device` gave up waiting since the last clear."""
     f = c_int32()
     _check(LIB.tq_device_status(device, ctypes.byref(f), 1 if clear else 0))
-    return f.value
+
+
+def debug_wait_probe(device: int, polls: int):
+    """Test hook: make one bounded wait of every tensor-core attention CTA run out after `polls`
+    polls (0 switches it off); see tq_debug_wait_probe."""
+    _check(LIB.tq_debug_wait_probe(device, polls))
 
 
 NOALLOC_SCRATCH_BYTES = 8 << 20

@@ -37,11 +37,35 @@ def test_exports_every_declared_symbol(lib):
         assert hasattr(raw, n), n
 
 
-def test_library_is_built_for_sm100a(lib):
-    import subprocess
-    out = subprocess.run(["/usr/local/cuda/bin/cuobjdump", "--list-elf", lib.LIB_PATH], capture_output=True,
-                         text=True).stdout
-    assert "sm_100a" in out
+def test_library_is_built_for_sm100a_only(lib):
+    # the build compiles every translation unit and links with exactly one target: sm_100a
+    from kv_cache_vector_06_b200 import build
+    assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+    assert not any("compute_" in f or "sm_" in f for f in build.FLAGS)
+    assert "sm_100a" in lib.version()
+
+
+def test_search_k_range_checked_before_anything_else(lib):
+    """k in [1, 1024] is supported (k > 32 takes the large-k scan); larger k is refused with
+    TQ_EUNSUPPORTED and k < 1 with TQ_EINVAL, before the context is looked at."""
+    from ctypes import byref, c_size_t
+    L, b = lib.LIB, c_size_t()
+    assert L.tq_search_workspace_size(None, 10, 5000, 1025, byref(b)) == 2
+    assert b"at most 1024" in L.tq_last_error()
+    assert L.tq_search_workspace_size(None, 10, 5000, 0, byref(b)) == 1
+    for k in (1, 32, 33, 1024):  # accepted: the next check (the NULL context) answers
+        assert L.tq_search_workspace_size(None, 10, 5000, k, byref(b)) == 1
+        assert b"ctx is NULL" in L.tq_last_error()
+    assert L.tq_search_topk(None, None, 0, 1, lib.PackedC(), 5000, 4096, None, None, None, 0, None) == 2
+    assert L.tq_search_topk(None, None, 0, 1, lib.PackedC(), 5000, 1024, None, None, None, 0, None) == 1
+
+
+def test_status_codes_match_the_header(lib):
+    # the binding's status names follow tq.h's enum, TQ_ETIMEOUT included
+    hdr = open(os.path.join(ROOT, "include", "tq.h")).read()
+    for code, name in lib.STATUS.items():
+        assert re.search(rf"\b{name}\s*=\s*{code}\b", hdr), name
+    assert lib.TQ_ETIMEOUT == 5 and lib.STATUS[5] == "TQ_ETIMEOUT"
 
 
 @pytest.mark.parametrize("d", [8, 16, 32, 64, 128, 256, 512, 1024])

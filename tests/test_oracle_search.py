@@ -70,3 +70,15 @@ def test_turboquant_recall_on_unit_vectors(bits, expect):
     _, i = search.search_topk(Q, e.norm, e.codes, e.rnorm, e.bits, D, S, c, 10)
     _, ie = search.exact_topk(Q, X, 10)
     assert search.recall_at_k(i, ie) > expect
+
+
+def test_recall_hand_counted():
+    # two queries, k = 4: 3 of 4 exact neighbours found, then 1 of 4 (order inside a list and the
+    # extra wrong entries do not matter): recall = (3/4 + 1/4) / 2 = 0.5
+    exact = [[7, 1, 5, 2], [10, 11, 12, 13]]
+    found = [[1, 2, 9, 7], [13, 3, 4, 8]]
+    assert search.recall_at_k(found, exact) == 0.5
+    assert search.recall_at_k([[1, 2, 9, 7]], [[7, 1, 5, 2]]) == 0.75
+    # a found list longer than k (k is the exact list's length): hits / k, not hits / len(found)
+    assert search.recall_at_k([[7, 1, 5, 2, 99, 98]], [[7, 1, 5, 2]]) == 1.0
+    assert search.recall_at_k([[0, 0, 0, 0]], [[7, 1, 5, 2]]) == 0.0

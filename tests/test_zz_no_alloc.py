@@ -18,9 +18,9 @@ from parity import Quantizer, assert_attention_close
 pytestmark = pytest.mark.gpu
 
 
-def _cache(tq, d, hkv, lens, paged, seed):
+def _cache(tq, d, hkv, lens, paged, seed, vlayout=0):
     kq = Quantizer(d, 2, d, seed=seed)
-    vq = Quantizer(d, 3, 0, seed=seed + 1)
+    vq = Quantizer(d, 3, 0, seed=seed + 1, layout=vlayout)
     batch, maxlen = len(lens), int(max(lens))
     lens_t = torch.tensor(lens, dtype=torch.int32)
     table = None
@@ -46,11 +46,15 @@ def _cache(tq, d, hkv, lens, paged, seed):
 
 
 @pytest.mark.parametrize("paged", [False, True])
-def test_noalloc_matches_workspace_entry_point_twice(paged):
+@pytest.mark.parametrize("vlayout", [0, 1])
+def test_noalloc_matches_workspace_entry_point_twice(paged, vlayout):
+    """vlayout 0: values in rows (the general CUDA-core attention); 1: values in 16-token blocks
+    (the tensor-core attention, whose per-call counters live in the scratch array too)."""
     from kv_cache_vector_06_b200 import tq
     d, hkv, group = 128, 4, 4
-    lens = [2500, 700, 1] if paged else [3000, 1234]
-    kq, vq, kp, vp, lens_t, maxlen, table = _cache(tq, d, hkv, lens, paged, seed=71 + int(paged))
+    lens = [2500, 700, 1] if paged else [3008, 1234]
+    kq, vq, kp, vp, lens_t, maxlen, table = _cache(tq, d, hkv, lens, paged, seed=71 + int(paged),
+                                                   vlayout=vlayout)
     desc = tq.make_attn_desc(kq.ctx, vq.ctx, (len(lens), hkv * group, d), kp, vp, lens_t, maxlen,
                              ctx_stride=maxlen, block_table=table, block_size=synth.BLOCK_TOKENS,
                              n_kv_heads=hkv)
