@@ -140,6 +140,24 @@ tq_status tq_make_codebook(int32_t d, int32_t bits, double *centroids, double *t
 tq_status tq_ctx_create(const tq_spec *spec, const int8_t *rot_signs, const float *qjl_matrix,
                         int32_t device, tq_ctx **out);
 
+/* Create a context whose QJL stage uses a structured JL matrix instead of a caller-drawn dense
+ * Gaussian one ([LP] 二.2 "Johnson-Lindenstrauss 实现技术": the fast JL transform y = P H D x):
+ *   S = P H D2,  S[i][j] = H[i][j] D2[j] for i < qjl_m,
+ * H the d x d Sylvester Hadamard matrix left unnormalised (entries +-1), D2 a diagonal of random
+ * signs drawn independently of the rotation's, P keeping the first qjl_m rows.  The entries are
+ * +-1 with unit variance like N(0,1) draws, the rows are orthogonal, and the estimator keeps the
+ * sqrt(pi/2)/m scale; over D2 it is unbiased to within Monte-Carlo resolution (exactly so only for
+ * Gaussian rows).  Encode computes S r as a Walsh-Hadamard transform of D2 r in registers: no
+ * projection matrix is read and tq_encode_workspace_size is 0.  Every other call is unchanged.
+ *   spec        host; qjl_m a multiple of 32 in [32, d]
+ *   rot_signs   host int8 [d], entries +1 or -1 (D)
+ *   qjl_signs   host int8 [d], entries +1 or -1 (D2)
+ *   out         host out: the new context
+ * Errors: TQ_EINVAL (nulls, a sign not +-1), TQ_EUNSUPPORTED (sizes, qjl_m = 0 or > d),
+ * TQ_ENOMEM, TQ_ECUDA. */
+tq_status tq_ctx_create_srht(const tq_spec *spec, const int8_t *rot_signs, const int8_t *qjl_signs,
+                             int32_t device, tq_ctx **out);
+
 /* Free a context (NULL is accepted).  The caller must ensure no queued work still uses it. */
 tq_status tq_ctx_destroy(tq_ctx *ctx);
 

@@ -109,9 +109,9 @@ tq_status tq_make_codebook(int32_t d, int32_t bits, double *centroids, double *t
   return tq_codebook_fp64(d, bits, centroids, thresholds, mse_per_coord);
 }
 
-tq_status tq_ctx_create(const tq_spec *spec, const int8_t *rot_signs, const float *qjl_matrix,
-                        int32_t device, tq_ctx **out) {
-  g_err[0] = 0;
+// Shared by tq_ctx_create (caller-drawn S) and tq_ctx_create_srht (S = P H D2 built here).
+static tq_status ctx_create(const tq_spec *spec, const int8_t *rot_signs, const float *qjl_matrix,
+                            const int8_t *qjl_signs, int32_t device, tq_ctx **out) {
   if (!out) return tq_fail(TQ_EINVAL, "out is NULL");
   *out = nullptr;
   tq_status st = check_spec(spec);
@@ -140,10 +140,15 @@ tq_status tq_ctx_create(const tq_spec *spec, const int8_t *rot_signs, const floa
   cudaError_t e = cudaSuccess;
   float hs[1024];
   for (int j = 0; j < d; ++j) hs[j] = (float)rot_signs[j];
+  float hs2[1024];
+  if (qjl_signs)
+    for (int j = 0; j < d; ++j) hs2[j] = (float)qjl_signs[j];
   e = cudaMalloc(&c->dev_signs, sizeof(float) * d);
   if (e == cudaSuccess && m > 0) e = cudaMalloc(&c->dev_S, sizeof(float) * (size_t)m * d);
+  if (e == cudaSuccess && qjl_signs) e = cudaMalloc(&c->dev_qjl_signs, sizeof(float) * d);
   if (e != cudaSuccess) {
     cudaFree(c->dev_signs);
+    cudaFree(c->dev_S);
     delete c;
     cudaGetLastError();
     return tq_fail(TQ_ENOMEM, "cudaMalloc of context constants failed");
@@ -151,9 +156,12 @@ tq_status tq_ctx_create(const tq_spec *spec, const int8_t *rot_signs, const floa
   e = cudaMemcpy(c->dev_signs, hs, sizeof(float) * d, cudaMemcpyHostToDevice);
   if (e == cudaSuccess && m > 0)
     e = cudaMemcpy(c->dev_S, qjl_matrix, sizeof(float) * (size_t)m * d, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && qjl_signs)
+    e = cudaMemcpy(c->dev_qjl_signs, hs2, sizeof(float) * d, cudaMemcpyHostToDevice);
   if (e != cudaSuccess) {
     cudaFree(c->dev_signs);
     cudaFree(c->dev_S);
+    cudaFree(c->dev_qjl_signs);
     delete c;
     return tq_cuda_check(e, "upload of context constants");
   }
@@ -173,6 +181,8 @@ tq_status tq_ctx_create(const tq_spec *spec, const int8_t *rot_signs, const floa
   }
   k.signs = c->dev_signs;
   k.S = c->dev_S;
+  k.srht = qjl_signs ? 1 : 0;
+  k.qjl_signs = c->dev_qjl_signs;
   // odd bit-plane expansion of the codebook for the tensor-core attention path:
   // e_S = 2^-b sum_code c[code] prod_{P in S} s_P(code), S in {0}, {1}, {2}, {0,1,2}
   k.fast_ok = 0;
@@ -211,6 +221,37 @@ tq_status tq_ctx_create(const tq_spec *spec, const int8_t *rot_signs, const floa
   return TQ_OK;
 }
 
+
+tq_status tq_ctx_create(const tq_spec *spec, const int8_t *rot_signs, const float *qjl_matrix,
+                        int32_t device, tq_ctx **out) {
+  g_err[0] = 0;
+  return ctx_create(spec, rot_signs, qjl_matrix, nullptr, device, out);
+}
+
+tq_status tq_ctx_create_srht(const tq_spec *spec, const int8_t *rot_signs, const int8_t *qjl_signs,
+                             int32_t device, tq_ctx **out) {
+  g_err[0] = 0;
+  if (!out) return tq_fail(TQ_EINVAL, "out is NULL");
+  *out = nullptr;
+  tq_status st = check_spec(spec);
+  if (st != TQ_OK) return st;
+  if (!qjl_signs) return tq_fail(TQ_EINVAL, "qjl_signs is NULL");
+  const int d = spec->d, m = spec->qjl_m;
+  if (m <= 0 || m > d)
+    return tq_fail(TQ_EUNSUPPORTED, "structured QJL: qjl_m=%d must be in [32, d=%d]", m, d);
+  for (int j = 0; j < d; ++j)
+    if (qjl_signs[j] != 1 && qjl_signs[j] != -1)
+      return tq_fail(TQ_EINVAL, "qjl_signs[%d] = %d: must be +1 or -1", j, (int)qjl_signs[j]);
+  // S[i][j] = H[i][j] D2[j], H the unnormalised Sylvester Hadamard matrix: (-1)^popcount(i & j)
+  float *S = new (std::nothrow) float[(size_t)m * d];
+  if (!S) return tq_fail(TQ_ENOMEM, "host allocation failed");
+  for (int i = 0; i < m; ++i)
+    for (int j = 0; j < d; ++j) S[(size_t)i * d + j] = (__builtin_popcount((unsigned)(i & j)) & 1) ? -qjl_signs[j] : qjl_signs[j];
+  st = ctx_create(spec, rot_signs, S, qjl_signs, device, out);
+  delete[] S;
+  return st;
+}
+
 tq_status tq_ctx_destroy(tq_ctx *ctx) {
   if (!ctx) return TQ_OK;
   int cur = -1;
@@ -218,6 +259,7 @@ tq_status tq_ctx_destroy(tq_ctx *ctx) {
   cudaSetDevice(ctx->device);
   cudaFree(ctx->dev_signs);
   cudaFree(ctx->dev_S);
+  cudaFree(ctx->dev_qjl_signs);
   if (cur >= 0) cudaSetDevice(cur);
   delete ctx;
   return TQ_OK;
@@ -239,7 +281,7 @@ tq_status tq_encode_workspace_size(const tq_ctx *ctx, int64_t n, size_t *bytes) 
   if (!bytes) return tq_fail(TQ_EINVAL, "bytes is NULL");
   if (n < 0) return tq_fail(TQ_EINVAL, "n < 0");
   const int64_t rows = n < kEncodeChunk ? n : kEncodeChunk;
-  const bool fused = n <= kFusedEncodeMaxRows && ctx->spec.d >= 128;
+  const bool fused = (n <= kFusedEncodeMaxRows && ctx->spec.d >= 128) || ctx->k.srht;
   *bytes = (ctx->spec.qjl_m > 0 && !fused) ? (size_t)(rows * ctx->spec.d * 4) : 0;
   return TQ_OK;
 }
@@ -271,6 +313,13 @@ tq_status tq_encode_kv(const tq_ctx *ctx, const void *x, tq_dtype dtype, int64_t
   if (st != TQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool qjl = ctx->spec.qjl_m > 0;
+  if (qjl && ctx->k.srht) {
+    // structured QJL: the kernel transforms the residual itself (Walsh-Hadamard), any batch size
+    cudaError_t e = launch_rotate(ctx->k, ROT_ENCODE, x, dtype, n, ld, slots, out.capacity,
+                                  static_cast<uint32_t *>(out.codes), out.norm, out.rnorm, nullptr, s,
+                                  static_cast<uint32_t *>(out.signs));
+    return tq_cuda_check(e, "encode launch");
+  }
   if (qjl && n <= kFusedEncodeMaxRows && ctx->spec.d >= 128) {
     // one launch: rotate, quantize, pack, project and pack the signs
     cudaError_t e = launch_rotate(ctx->k, ROT_ENCODE, x, dtype, n, ld, slots, out.capacity,

@@ -34,7 +34,7 @@ cudaError_t launch_rotate_d(const TqConsts &c, RotateMode mode, const void *x, t
   constexpr int VPB = (kRotThreads / 32) * RotLayout<D>::VPW;  // vectors per block
   const int64_t blocks = (n + VPB - 1) / VPB;
   const int kind = mode == ROT_ENCODE ? TQK_ROTATE_ENCODE : TQK_ROTATE_QUERY;
-  const size_t smem = (D == 128 && fsigns != nullptr && c.m == 128) ? sizeof(float) * 128 * 132 : 0;
+  const size_t smem = (D == 128 && fsigns != nullptr && c.m == 128 && !c.srht) ? sizeof(float) * 128 * 132 : 0;
   if (smem) {
     cudaError_t e0 = tq_smem_limit(reinterpret_cast<const void *>(rotate_kernel<D>), (int)smem);
     if (e0 != cudaSuccess) return e0;

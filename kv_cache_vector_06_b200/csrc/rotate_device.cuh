@@ -33,6 +33,42 @@ __device__ __forceinline__ float group_sum(float x) {
   return x;
 }
 
+// Unnormalised Walsh-Hadamard transform v <- H v of one vector held in the lane layout above
+// (lane l of the group owns coordinates 4 (l + LPV k) + e): distances 1 and 2 inside a lane's
+// 4-chunk, 4 .. 2 LPV across lanes, >= 4 LPV across the lane's chunks.
+template <int D>
+__device__ __forceinline__ void fwht_lanes(float (&v)[RotLayout<D>::KCH][4], int l) {
+  constexpr int LPV = RotLayout<D>::LPV, KCH = RotLayout<D>::KCH;
+#pragma unroll
+  for (int k = 0; k < KCH; ++k) {
+    const float a = v[k][0] + v[k][1], b = v[k][0] - v[k][1];
+    const float p = v[k][2] + v[k][3], q = v[k][2] - v[k][3];
+    v[k][0] = a + p; v[k][1] = b + q; v[k][2] = a - p; v[k][3] = b - q;
+  }
+#pragma unroll
+  for (int s = 1; s < LPV; s <<= 1) {
+    const bool hi = (l & s) != 0;
+#pragma unroll
+    for (int k = 0; k < KCH; ++k)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float o = __shfl_xor_sync(TQ_FULL_MASK, v[k][e], s);
+        v[k][e] = hi ? (o - v[k][e]) : (v[k][e] + o);
+      }
+  }
+#pragma unroll
+  for (int h = 1; h < KCH; h <<= 1)
+#pragma unroll
+    for (int k = 0; k < KCH; ++k)
+      if ((k & h) == 0)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a = v[k][e], b = v[k + h][e];
+          v[k][e] = a + b;
+          v[k + h][e] = a - b;
+        }
+}
+
 // The encode / query-rotation work of one block of kRotThreads threads: rows of block `vblock`.
 // `sS` is dynamic shared memory of at least 128 x 132 floats when d = m = 128 and `fsigns` is set
 // (the fused projection stages S there); every thread of the block must call it with the same
@@ -54,7 +90,7 @@ __device__ __forceinline__ void rotate_rows(const TqConsts &c, int mode, const v
   const int lane = threadIdx.x & 31;
   const int wib = threadIdx.x >> 5;
   // fused projection with S staged in shared memory (d = m = 128; row stride 132 floats)
-  const bool staged = D == 128 && fsigns != nullptr && c.m == 128;
+  const bool staged = D == 128 && fsigns != nullptr && c.m == 128 && !c.srht;
   if (staged) stage_rows_padded_async(sS, c.S, 128, 128);  // completed before the projection
   const int g = lane / LPV;
   const int l = lane % LPV;
@@ -99,37 +135,8 @@ __device__ __forceinline__ void rotate_rows(const TqConsts &c, int mode, const v
     const float4 sg = *reinterpret_cast<const float4 *>(c.signs + 4 * (l + LPV * k));
     v[k][0] *= inv * sg.x; v[k][1] *= inv * sg.y; v[k][2] *= inv * sg.z; v[k][3] *= inv * sg.w;
   }
-  // Walsh-Hadamard butterflies: distances 1 and 2 inside the 4-chunk
-#pragma unroll
-  for (int k = 0; k < KCH; ++k) {
-    const float a = v[k][0] + v[k][1], b = v[k][0] - v[k][1];
-    const float p = v[k][2] + v[k][3], q = v[k][2] - v[k][3];
-    v[k][0] = a + p; v[k][1] = b + q; v[k][2] = a - p; v[k][3] = b - q;
-  }
-  // distances 4 .. 2 LPV across lanes
-#pragma unroll
-  for (int s = 1; s < LPV; s <<= 1) {
-    const bool hi = (l & s) != 0;
-#pragma unroll
-    for (int k = 0; k < KCH; ++k)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float o = __shfl_xor_sync(TQ_FULL_MASK, v[k][e], s);
-        v[k][e] = hi ? (o - v[k][e]) : (v[k][e] + o);
-      }
-  }
-  // distances >= 4 LPV across the lane's chunks
-#pragma unroll
-  for (int h = 1; h < KCH; h <<= 1)
-#pragma unroll
-    for (int k = 0; k < KCH; ++k)
-      if ((k & h) == 0)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float a = v[k][e], b = v[k + h][e];
-          v[k][e] = a + b;
-          v[k + h][e] = a - b;
-        }
+  // Walsh-Hadamard butterflies
+  fwht_lanes<D>(v, l);
 #pragma unroll
   for (int k = 0; k < KCH; ++k)
 #pragma unroll
@@ -218,6 +225,38 @@ __device__ __forceinline__ void rotate_rows(const TqConsts &c, int mode, const v
     for (int i = l; i < c.code_words / 4; i += LPV)
       dst[i] = make_uint4(st[4 * i], st[4 * i + 1], st[4 * i + 2], st[4 * i + 3]);
     if (l == 0) norm[slot] = nu;
+  }
+  if (c.srht && fsigns != nullptr) {
+    // structured QJL ("TurboQuant 学习路径" 二.2, fast JL y = P H D x): z = H (D2 r), the first m
+    // coordinates' signs, by the same butterflies as the rotation (no projection matrix)
+    const float gamma = sqrtf(group_sum<LPV>(rr));
+    if (store && l == 0) rnorm[slot] = gamma;
+#pragma unroll
+    for (int k = 0; k < KCH; ++k) {
+      const float4 sg = *reinterpret_cast<const float4 *>(c.qjl_signs + 4 * (l + LPV * k));
+      v[k][0] *= sg.x; v[k][1] *= sg.y; v[k][2] *= sg.z; v[k][3] *= sg.w;
+    }
+    fwht_lanes<D>(v, l);
+    __syncwarp();  // the staging words were read by the code store above
+    for (int i = l; i < c.sign_words; i += LPV) st[i] = 0u;
+    __syncwarp();
+#pragma unroll
+    for (int k = 0; k < KCH; ++k) {
+      const int j0 = 4 * (l + LPV * k);
+      if (j0 < c.m) {
+        uint32_t nib = 0u;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) nib |= (v[k][e] >= 0.f ? 1u : 0u) << e;
+        atomicOr(&st[j0 >> 5], nib << (j0 & 31));
+      }
+    }
+    __syncwarp();
+    if (store) {
+      uint4 *dst = reinterpret_cast<uint4 *>(fsigns + slot * c.sign_words);
+      for (int i = l; i < c.sign_words / 4; i += LPV)
+        dst[i] = make_uint4(st[4 * i], st[4 * i + 1], st[4 * i + 2], st[4 * i + 3]);
+    }
+    return;
   }
   if constexpr (D >= 128) {
     if (fsigns != nullptr) {

@@ -29,6 +29,8 @@ struct TqConsts {
   float thresholds[TQ_MAX_LEVELS];  // [levels-1] used
   const float *signs;  // device [d], +-1.0f (rotation D)
   const float *S;      // device [m][d] row-major (JL matrix)
+  int srht;               // S = P H D2 (structured QJL): encode transforms the residual instead
+  const float *qjl_signs; // device [d], +-1.0f (D2), srht only
 };
 
 struct tq_ctx {
@@ -41,6 +43,7 @@ struct tq_ctx {
   double mse_per_coord;
   float *dev_signs;  // [d]
   float *dev_S;      // [m][d]
+  float *dev_qjl_signs;  // [d] (structured QJL only)
   TqConsts k;        // kernel view
 };
 

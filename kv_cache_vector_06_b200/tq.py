@@ -53,6 +53,7 @@ def _load():
     sig = {
         "tq_make_codebook": (st, [c_int32, c_int32, POINTER(c_double), POINTER(c_double), POINTER(c_double)]),
         "tq_ctx_create": (st, [POINTER(Spec), c_void_p, c_void_p, c_int32, POINTER(c_void_p)]),
+        "tq_ctx_create_srht": (st, [POINTER(Spec), c_void_p, c_void_p, c_int32, POINTER(c_void_p)]),
         "tq_ctx_destroy": (st, [c_void_p]),
         "tq_ctx_layout": (st, [c_void_p, POINTER(c_int64), POINTER(c_int64)]),
         "tq_encode_workspace_size": (st, [c_void_p, c_int64, POINTER(c_size_t)]),
@@ -139,21 +140,31 @@ class Context:
     """Quantizer constants for one tensor role, resident on one device."""
 
     def __init__(self, d: int, mse_bits: int, qjl_m: int, rot_signs, qjl_matrix=None, device: int = 0,
-                 layout: int = LAYOUT_ROWS):
+                 layout: int = LAYOUT_ROWS, qjl_signs=None):
+        """qjl_matrix: the dense JL matrix [qjl_m, d] (tq_ctx_create); or qjl_signs: the sign
+        vector D2 [d] of the structured matrix S = P H D2 (tq_ctx_create_srht)."""
         rs = torch.as_tensor(rot_signs).to(torch.int8).contiguous().cpu()
         if rs.numel() != d:
             raise ValueError("rot_signs must have d entries")
-        if qjl_m > 0:
-            S = torch.as_tensor(qjl_matrix).to(torch.float32).contiguous().cpu()
-            if tuple(S.shape) != (qjl_m, d):
-                raise ValueError(f"qjl_matrix must be [{qjl_m}, {d}]")
-            sptr = c_void_p(S.data_ptr())
-        else:
-            sptr = c_void_p(None)
         self.d, self.mse_bits, self.qjl_m, self.device, self.layout = d, mse_bits, qjl_m, device, layout
+        self.srht = qjl_signs is not None
         spec = Spec(d, mse_bits, qjl_m, layout)
         h = c_void_p()
-        _check(LIB.tq_ctx_create(ctypes.byref(spec), c_void_p(rs.data_ptr()), sptr, device, ctypes.byref(h)))
+        if self.srht:
+            d2 = torch.as_tensor(qjl_signs).to(torch.int8).contiguous().cpu()
+            if d2.numel() != d:
+                raise ValueError("qjl_signs must have d entries")
+            _check(LIB.tq_ctx_create_srht(ctypes.byref(spec), c_void_p(rs.data_ptr()), c_void_p(d2.data_ptr()),
+                                          device, ctypes.byref(h)))
+        else:
+            if qjl_m > 0:
+                S = torch.as_tensor(qjl_matrix).to(torch.float32).contiguous().cpu()
+                if tuple(S.shape) != (qjl_m, d):
+                    raise ValueError(f"qjl_matrix must be [{qjl_m}, {d}]")
+                sptr = c_void_p(S.data_ptr())
+            else:
+                sptr = c_void_p(None)
+            _check(LIB.tq_ctx_create(ctypes.byref(spec), c_void_p(rs.data_ptr()), sptr, device, ctypes.byref(h)))
         self._h = h
         cb, sb = c_int64(), c_int64()
         _check(LIB.tq_ctx_layout(h, ctypes.byref(cb), ctypes.byref(sb)))

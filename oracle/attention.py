@@ -16,6 +16,13 @@ Definitions (R = reading where the pages are silent):
   grouped-query attention: query head hq reads KV head hq // (Hq / Hkv)  (R)
   an empty context gives o = 0 (R)
 
+Sparse V ([ZC] 第六部分 "Sparse V Dequant"): the attention weights act as a gate, and value rows
+whose weight is below a threshold tau (the pages use 1e-6) are not dequantized, i.e. they are left
+out of the weighted sum; the softmax normalisation itself still covers every token (R: the pages
+skip only the value decompression step):
+  o = sum_{t : w_t >= tau} w_t v^_t
+tau = 0 (the default) keeps every row.
+
 Cache addressing: every packed array is indexed by a slot.
   contiguous: slot(b, h, t) = (b * Hkv + h) * ctx_stride + t
   paged:      slot(b, h, t) = (block_table[b, t // B] * Hkv + h) * B + t % B,  B = 16 tokens
@@ -59,9 +66,10 @@ def token_slots(b: int, h: int, length: int, n_kv: int, ctx_stride=None, block_t
 def attend_decode(q, kcache: Cache, vcache: Cache, ctx_lens, n_kv: int,
                   k_signs, k_S, k_centroids, v_signs, v_centroids,
                   scale=None, ctx_stride=None, block_table=None, block_tokens: int = 16,
-                  heads=None):
+                  heads=None, sparse_v: float = 0.0):
     """q [B, Hq, d] -> o [B, Hq, d].  `heads` optionally restricts the (b, hq) pairs computed
-    (others are left as NaN), for sampled checks at large sizes."""
+    (others are left as NaN), for sampled checks at large sizes.  `sparse_v` is the Sparse V
+    threshold tau on the softmax weights (0 = every value row is used)."""
     q = np.asarray(q, dtype=np.float64)
     B, Hq, d = q.shape
     G = Hq // n_kv
@@ -84,7 +92,8 @@ def attend_decode(q, kcache: Cache, vcache: Cache, ctx_lens, n_kv: int,
         logits = scale * s
         w = np.exp(logits - np.max(logits))
         w /= np.sum(w)
-        cv = np.asarray(v_centroids, dtype=np.float64)[vcache.codes[sl]]
-        vhat = vcache.norm[sl][:, None] * unrotate(cv, v_signs)
-        out[b, hq] = w @ vhat
+        keep = w >= sparse_v if sparse_v > 0 else np.ones(L, dtype=bool)
+        cv = np.asarray(v_centroids, dtype=np.float64)[vcache.codes[sl][keep]]
+        vhat = vcache.norm[sl][keep][:, None] * unrotate(cv, v_signs)
+        out[b, hq] = w[keep] @ vhat
     return out

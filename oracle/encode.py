@@ -9,7 +9,9 @@ Source.
   [JJ] 第二部分 第二步 (QJL) and [VC] 第二階段: the residual of the first stage is projected
        with a Johnson-Lindenstrauss matrix and only the sign of each projected coordinate is
        kept (1 bit each).
-  [LP] 二.2: the standard JL matrix has iid N(0,1) entries.
+  [LP] 二.2: the standard JL matrix has iid N(0,1) entries; the same section gives the fast
+       (FJLT, y = P H D x) and sparse (Achlioptas) alternatives.  `srht_matrix` builds the
+       structured one used as an option here: S = P H D2.
   [LP] 二.4 "CUDA/GPU 优化": codes are bit-packed into machine words.
 
 Definitions (readings where the pages are silent are marked R):
@@ -35,7 +37,7 @@ from dataclasses import dataclass
 
 import numpy as np
 
-from .rotation import rotate
+from .rotation import rotate, sylvester
 
 
 def code_bytes(d: int, bits: int) -> int:
@@ -175,3 +177,18 @@ def unpack_codes_block16(buf, d: int, bits: int) -> np.ndarray:
         w = words[:, None, base + j // 2]                                 # [block, 1, j]
         codes |= ((w >> (16 * (j % 2)[None, None, :] + tok)) & 1) << (bits - 1)
     return codes.reshape(n, d)
+
+
+def srht_matrix(qjl_signs, m: int) -> np.ndarray:
+    """Structured QJL matrix ([LP] 二.2, the fast JL transform y = P H D x): S = P H D2, with
+    H the d x d Sylvester Hadamard matrix left unnormalised (entries +-1), D2 a diagonal of random
+    signs (drawn independently of the rotation's D) and P keeping the first m rows (R: the random
+    signs supply the randomness, so the kept rows are fixed).  S[i, j] = H[i, j] * D2[j]: entries
+    +-1, unit variance like N(0,1) draws, and the rows are orthogonal.  The estimator keeps the
+    Gaussian scale sqrt(pi/2)/m; it is unbiased over D2 to within Monte-Carlo resolution (exactly
+    unbiased only for Gaussian rows)."""
+    D2 = np.asarray(qjl_signs, dtype=np.float64)
+    d = D2.shape[0]
+    if not 0 < m <= d:
+        raise ValueError("m must be in [1, d]")
+    return sylvester(d)[:m] * D2[None, :]

@@ -27,13 +27,20 @@ MAX_FLIP_FRACTION = 1e-4
 class Quantizer:
     """One tensor role: the seeded draws (D, S), the oracle codebook and the library context."""
 
-    def __init__(self, d, bits, m, seed, device=0, layout=0):
+    def __init__(self, d, bits, m, seed, device=0, layout=0, srht=False):
+        """srht: structured QJL, S = P H D2 with D2 drawn like D (the oracle builds S, the library
+        receives only D2)."""
         from kv_cache_vector_06_b200 import tq
         self.d, self.bits, self.m, self.layout = d, bits, m, layout
         self.D = synth.rotation_signs(d, seed)
-        self.S = synth.qjl_matrix(m, d, seed + 1000)
         self.c, self.t = ocb.codebook(d, bits)
-        self.ctx = tq.Context(d, bits, m, self.D, self.S if m > 0 else None, device=device, layout=layout)
+        if srht:
+            self.D2 = synth.rotation_signs(d, seed + 2000)
+            self.S = torch.from_numpy(oenc.srht_matrix(self.D2.double().numpy(), m))
+            self.ctx = tq.Context(d, bits, m, self.D, device=device, layout=layout, qjl_signs=self.D2)
+        else:
+            self.S = synth.qjl_matrix(m, d, seed + 1000)
+            self.ctx = tq.Context(d, bits, m, self.D, self.S if m > 0 else None, device=device, layout=layout)
 
     @property
     def D64(self):

@@ -38,8 +38,8 @@ def _packed_equal(a, b):
 
 
 def _step_case(tq, d, kbits, km, vbits, vlayout, batch, hkv, group, lens, paged, seed, kvdtype=torch.float32,
-               qdtype=torch.bfloat16):
-    kq = Quantizer(d, kbits, km, seed=seed)
+               qdtype=torch.bfloat16, srht=False):
+    kq = Quantizer(d, kbits, km, seed=seed, srht=srht)
     vq = Quantizer(d, vbits, 0, seed=seed + 50, layout=vlayout)
     hq = hkv * group
     blk = synth.BLOCK_TOKENS
@@ -116,3 +116,11 @@ def test_decode_step_general_path(tq, d, group, vlayout):
     """Shapes the tensor-core kernel does not take: the step runs the separate calls."""
     _step_case(tq, d, 2, d, 3, vlayout, batch=2, hkv=2, group=group, lens=[300, 47], paged=False,
                seed=351 + d + group)
+
+
+@pytest.mark.parametrize("vlayout", [1, 0])
+def test_decode_step_structured_qjl(tq, vlayout):
+    """Keys with the structured QJL matrix S = P H D2: the appended key's signs come from the
+    in-register Walsh-Hadamard transform, the queries are projected with the same S."""
+    _step_case(tq, 128, 2, 128, 3, vlayout, batch=2, hkv=2, group=4, lens=[1500, 33], paged=vlayout == 1,
+               seed=371 + vlayout, srht=True)

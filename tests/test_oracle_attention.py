@@ -147,3 +147,55 @@ def test_four_bit_attention_is_close_to_exact():
     ref = plain_attention(q[0, 0], K, V, 1 / math.sqrt(d))
     # a sanity bound only: the QJL term is unbiased but noisy, so sharp softmaxes amplify it
     assert np.linalg.norm(out - ref) < 0.25 * np.linalg.norm(ref)
+
+
+def _small_case(seed, d=16, ctx=60, kb=2, vb=3, spread=8.0):
+    rng = np.random.default_rng(seed)
+    K = rng.standard_normal((ctx, d)) * spread
+    V = rng.standard_normal((ctx, d))
+    Dk = rng.choice([-1.0, 1.0], size=d)
+    Dv = rng.choice([-1.0, 1.0], size=d)
+    ck, tk = codebook.codebook(d, kb)
+    cv, tv = codebook.codebook(d, vb)
+    kc, ke = _cache(K, Dk, np.zeros((0, d)), ck, tk)
+    vc, ve = _cache(V, Dv, np.zeros((0, d)), cv, tv)
+    q = rng.standard_normal((1, 1, d)) * spread
+    return q, kc, ke, vc, ve, Dk, Dv, ck, cv
+
+
+def test_sparse_v_threshold_zero_is_plain_attention():
+    q, kc, ke, vc, ve, Dk, Dv, ck, cv = _small_case(5)
+    a = attention.attend_decode(q, kc, vc, [60], 1, Dk, np.zeros((0, 16)), ck, Dv, cv, ctx_stride=60)
+    b = attention.attend_decode(q, kc, vc, [60], 1, Dk, np.zeros((0, 16)), ck, Dv, cv, ctx_stride=60,
+                                sparse_v=0.0)
+    np.testing.assert_array_equal(a, b)
+
+
+def test_sparse_v_drops_exactly_the_rows_below_the_threshold():
+    """Hand-built gate: the rows whose softmax weight (over all tokens, normalisation unchanged)
+    is below tau are left out of the sum, every other row is kept with its full weight."""
+    d, ctx = 16, 60
+    q, kc, ke, vc, ve, Dk, Dv, ck, cv = _small_case(6)
+    Kh = _recon(ke.norm, ke.codes, Dk, ck)
+    Vh = _recon(ve.norm, ve.codes, Dv, cv)
+    logits = (Kh @ q[0, 0]) / math.sqrt(d)
+    w = np.exp(logits - logits.max())
+    w /= w.sum()
+    order = np.sort(w)
+    tau = 0.5 * (order[20] + order[21])  # a threshold between the 21st and 22nd smallest weights
+    dropped = w < tau
+    assert dropped.sum() == 21
+    expect = (w * ~dropped) @ Vh
+    got = attention.attend_decode(q, kc, vc, [ctx], 1, Dk, np.zeros((0, d)), ck, Dv, cv, ctx_stride=ctx,
+                                  sparse_v=tau)[0, 0]
+    np.testing.assert_allclose(got, expect, rtol=1e-11, atol=1e-12)
+    # the dropped mass is what changes: |o - o_sparse| <= sum of dropped weights x max |v^|
+    full = attention.attend_decode(q, kc, vc, [ctx], 1, Dk, np.zeros((0, d)), ck, Dv, cv, ctx_stride=ctx)[0, 0]
+    assert np.max(np.abs(full - got)) <= w[dropped].sum() * np.max(np.abs(Vh)) + 1e-15
+    # a threshold above every weight leaves nothing; one at or below the smallest keeps all
+    none = attention.attend_decode(q, kc, vc, [ctx], 1, Dk, np.zeros((0, d)), ck, Dv, cv, ctx_stride=ctx,
+                                   sparse_v=1.01)[0, 0]
+    np.testing.assert_array_equal(none, np.zeros(d))
+    allk = attention.attend_decode(q, kc, vc, [ctx], 1, Dk, np.zeros((0, d)), ck, Dv, cv, ctx_stride=ctx,
+                                   sparse_v=order[0])[0, 0]
+    np.testing.assert_allclose(allk, full, rtol=1e-12, atol=1e-14)

@@ -108,3 +108,58 @@ def test_zero_norm_key_scores_zero():
     c, t = codebook.codebook(d, 2)
     enc = encode.encode(np.zeros((1, d)), D, S, c, t)
     assert estimate.score_encoded(rng.standard_normal((3, d)), enc, D, S, c).tolist() == [[0.0]] * 3
+
+
+# ---------------------------------------------------------------- structured QJL (SRHT)
+@pytest.mark.parametrize("d,m", [(8, 8), (128, 128), (128, 32), (1024, 256)])
+def test_srht_matrix_is_signed_hadamard_rows(d, m):
+    rng = np.random.default_rng(d + m)
+    D2 = rng.choice([-1.0, 1.0], size=d)
+    S = encode.srht_matrix(D2, m)
+    # scipy's Hadamard matrix (an independent construction), first m rows, columns times D2
+    np.testing.assert_array_equal(S, hadamard(d)[:m] * D2[None, :])
+    assert set(np.unique(S)) == {-1.0, 1.0}
+    np.testing.assert_array_equal(S @ S.T, d * np.eye(m))  # orthogonal rows
+
+
+def test_srht_estimator_unbiased_monte_carlo():
+    """Over 10^5 independent sign vectors D2 the SRHT sign estimator of <q', r> averages to the
+    truth within 3 standard errors, at m = d and with m < d rows kept (the transform of D2 * r is
+    computed with scipy's Hadamard matrix)."""
+    d = 128
+    rng = np.random.default_rng(11)
+    r = rng.standard_normal(d) * 0.03
+    q = rng.standard_normal(d)
+    H = hadamard(d).astype(np.float64)
+    for m in (128, 32):
+        vals = []
+        for _ in range(20):
+            D2 = rng.choice([-1.0, 1.0], size=(5000, d))
+            z = (D2 * r) @ H[:m].T
+            p = (D2 * q) @ H[:m].T
+            vals.append(math.sqrt(math.pi / 2) / m * np.linalg.norm(r) * np.sum(np.where(z >= 0, 1.0, -1.0) * p, axis=1))
+        vals = np.concatenate(vals)
+        se = vals.std() / math.sqrt(vals.size)
+        assert abs(vals.mean() - r @ q) < 3 * se, (m, vals.mean(), r @ q, se)
+
+
+def test_srht_oracle_estimator_unbiased_and_variance_falls_with_m():
+    """The oracle's encode + estimator with S = srht_matrix(D2, m), averaged over independent D2
+    (and rotations D): mean within 4 standard errors of <q, x>; the spread falls as m grows."""
+    d, bits, trials = 32, 2, 3000
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal(d) * 3
+    q = rng.standard_normal(d)
+    c, t = codebook.codebook(d, bits)
+    spread = {}
+    for m in (8, 32):
+        vals = []
+        for _ in range(trials):
+            D = rng.choice([-1.0, 1.0], size=d)
+            S = encode.srht_matrix(rng.choice([-1.0, 1.0], size=d), m)
+            enc = encode.encode(x[None], D, S, c, t)
+            vals.append(estimate.score_encoded(q[None], enc, D, S, c)[0, 0])
+        vals = np.array(vals)
+        assert abs(vals.mean() - q @ x) < 4 * vals.std() / math.sqrt(trials), m
+        spread[m] = vals.std()
+    assert spread[32] < 0.75 * spread[8]
