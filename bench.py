@@ -376,6 +376,11 @@ class DecodeBench:
         return {"n_vectors": 2 * n, "ms": ms, "bytes": n * (2 * 2 * self.d + kb + vb),
                 "flop": 2.0 * self.m * self.d * n, "kernels": prof}
 
+    def set_sparse_v(self, tau: float):
+        """Sparse V threshold of every step's descriptor (0 = off)."""
+        for desc, _, _, _ in self.steps:
+            desc.sparse_v = tau
+
     def step(self, i: int, q=None, out=None, k_new=None, v_new=None):
         desc, _, slots, _ = self.steps[i % len(self.steps)]
         self.tq.decode_step(self.kctx, self.vctx, self.q if q is None else q,
@@ -553,6 +558,19 @@ def ours_decode(args, world, rank):
     e_ms, h2d, d2h = time_e2e(bench, e2e_steps, min(args.warmup, 10))
     e_ms = max_over_ranks(e_ms, world)
     e2e_value = aggregate_rate(world, bench.keys_per_step, e2e_steps, e_ms)
+    # Sparse V ("TurboQuant+ 深度解析" 第六部分) on the same steps: value rows whose softmax weight is
+    # below 1e-6 are skipped; reported beside the plain step (the headline keeps every row)
+    sparse = None
+    if args.sparse_v == 0:
+        tau = 1e-6
+        bench.set_sparse_v(tau)
+        sgraphs = bench.capture_graphs()
+        s_ms = max_over_ranks(time_graph_steps(sgraphs, args.steps, args.warmup, world), world)
+        bench.set_sparse_v(0.0)
+        del sgraphs
+        sparse = {"threshold": tau, "ms_per_step": s_ms / args.steps,
+                  "value": aggregate_rate(world, bench.keys_per_step, args.steps, s_ms), "unit": "keys/s",
+                  "speedup_vs_all_rows": ms / s_ms}
     enc = encode_summary(bench.encode_timing, peaks, src, bench.d)
     enc_ms = max_over_ranks(enc["ms"], world)
     enc["value"] = world * bench.encode_timing["n_vectors"] / (enc_ms / 1e3)
@@ -569,6 +587,7 @@ def ours_decode(args, world, rank):
         "gpu_launches": int(round(launches_per_step * args.steps)),
         "clocks": sampler.summary(),
         "encode": enc,
+        "sparse_v": sparse,
     }
     del graphs
     cpu = None

@@ -115,6 +115,11 @@ typedef struct {
   int32_t max_seq_len;         /* host-known upper bound of seq_lens; sizes the split grid */
   tq_packed k;                 /* keys, encoded with the K context */
   tq_packed v;                 /* values, encoded with the V context (MSE stage only) */
+  float sparse_v;              /* Sparse V threshold tau ("TurboQuant+ 深度解析" 第六部分): value rows
+                                  whose softmax weight is below tau are not dequantized; 0 = off.
+                                  Tensor-core path (TQ_LAYOUT_BLOCK16 values): a row is dropped
+                                  when a running bound on its weight is below tau, so every dropped
+                                  row has final weight < tau; the general path ignores it. */
 } tq_attn_desc;
 
 /* Lloyd-Max codebook for one coordinate of a randomly rotated unit vector in R^d.

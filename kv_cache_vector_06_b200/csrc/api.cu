@@ -97,7 +97,7 @@ extern "C" {
 const char *tq_last_error(void) { return g_err; }
 // The revision tags of the tensor-core kernels name the device code that a recorded profile (DRAM
 // traffic per launch) was taken on; each changes whenever its kernel's code changes.
-const char *tq_version(void) { return "libtq 0.3 (sm_100a; attend_mma r8; search_tc r2)"; }
+const char *tq_version(void) { return "libtq 0.3 (sm_100a; attend_mma r9; search_tc r2)"; }
 
 tq_status tq_make_codebook(int32_t d, int32_t bits, double *centroids, double *thresholds,
                            double *mse_per_coord) {
@@ -313,6 +313,18 @@ tq_status tq_encode_kv(const tq_ctx *ctx, const void *x, tq_dtype dtype, int64_t
   if (st != TQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool qjl = ctx->spec.qjl_m > 0;
+  if (n > kFusedEncodeMaxRows && encode_tpr_eligible(ctx->k, slots, dtype)) {
+    // bulk rows at d = 128: one row per thread
+    const int64_t nt = encode_tpr_rows(ctx->k, n);
+    cudaError_t e = launch_encode_tpr(ctx->k, x, dtype, nt, ld, slots, out.capacity, static_cast<uint32_t *>(out.codes),
+                                      out.norm, out.rnorm, static_cast<uint32_t *>(out.signs), s);
+    if (e != cudaSuccess || nt == n) return tq_cuda_check(e, "encode launch");
+    // the ragged tail of a token-block layout (rows nt.. go to slots nt..; nt is a whole block)
+    e = launch_rotate(ctx->k, ROT_ENCODE, static_cast<const char *>(x) + nt * ld * esz, dtype, n - nt, ld, nullptr,
+                      out.capacity - nt, static_cast<uint32_t *>(out.codes) + nt * (ctx->code_bytes / 4), out.norm + nt,
+                      nullptr, nullptr, s);
+    return tq_cuda_check(e, "encode launch");
+  }
   if (qjl && ctx->k.srht) {
     // structured QJL: the kernel transforms the residual itself (Walsh-Hadamard), any batch size
     cudaError_t e = launch_rotate(ctx->k, ROT_ENCODE, x, dtype, n, ld, slots, out.capacity,

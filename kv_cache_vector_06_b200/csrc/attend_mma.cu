@@ -49,6 +49,7 @@ struct MmaArgs {
   tq_packed k, v;
   int *counter;  // per (sequence, KV head): CTAs done (zeroed by the query-fragment kernel)
   float *out;    // final output when the kernel merges its splits itself, else null
+  float sparse_v;  // Sparse V threshold on the softmax weights (0 = off)
 };
 
 __device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -395,12 +396,26 @@ __device__ __forceinline__ uint32_t mul_lo(uint32_t x, uint32_t m) {
   return r;
 }
 
-constexpr int kSub = 256;          // tokens per sub-chunk (one staging buffer)
-constexpr int kSubBlk = kSub / 16;  // 16-token blocks per sub-chunk
-constexpr int kLgS = kSub + 8;      // row stride of the logit/weight array (bank-conflict padding)
+constexpr int kSub = 256;            // tokens per sub-chunk: kCWarps consumer warps x 32 tokens
+constexpr int kSubBlk = kSub / 16;   // 16-token blocks per sub-chunk
+#ifndef TQ_ATTN_STAGES
+#define TQ_ATTN_STAGES 3
+#endif
+#ifndef TQ_ATTN_MAX_CHUNK
+#define TQ_ATTN_MAX_CHUNK 4096
+#endif
+constexpr int kStagesMax = TQ_ATTN_STAGES;  // staging ring depth (sub-chunks in flight), when it fits
+#ifndef TQ_ATTN_PRODUCERS
+#define TQ_ATTN_PRODUCERS 3
+#endif
+constexpr int kCWarps = 8;           // consumer warps
+constexpr int kProd = TQ_ATTN_PRODUCERS;  // warps that issue the bulk copies (arrays split among them)
+constexpr int kMmaThreads = (kCWarps + kProd) * 32;
+constexpr int kMaxChunk = TQ_ATTN_MAX_CHUNK;  // tokens per CTA at most
+constexpr int kLgS = 40;             // row stride of a warp's weight array (bank-conflict free)
 
-// Shared-memory carve-up of attend_mma_kernel (bytes): two staging buffers (the sub-chunk being
-// computed and the one being loaded), then the per-sub-chunk work arrays.
+// Shared-memory carve-up of attend_mma_kernel (bytes): the staging ring, each consumer warp's
+// private scratch, the query fragments, the CTA's block slots, the barriers.
 template <int BK, int BV, bool QJL>
 struct MmaSmem {
   static constexpr int NB = kSubBlk;
@@ -416,19 +431,24 @@ struct MmaSmem {
   static constexpr size_t vc = kr + (size_t)kSub * 4;
   static constexpr size_t vn = vc + (size_t)NB * VBW * 4;
   static constexpr size_t buf = vn + (size_t)kSub * 4;
-  // work arrays
-  static constexpr size_t x1 = 2 * buf;
-  static constexpr size_t lg = x1 + (size_t)NB * X1W * 4;
-  static constexpr size_t vf = lg + (size_t)kG * kLgS * 4;
-  static constexpr size_t kf = vf + (size_t)NB * 32 * 16;
+  // ring depth: three buffers where two CTAs per SM still fit, else two
+  static constexpr int NS = kStagesMax * buf <= 90 * 1024 ? kStagesMax : 2;
+  // per consumer warp: its 32 tokens' value weights [kG][32] and its two blocks' (plane 2,
+  // parity) words [2][kD]
+  static constexpr size_t WLG = (size_t)kG * kLgS * 4;
+  static constexpr size_t WPER = WLG + (size_t)2 * X1W * 4;
+  static constexpr size_t ws = NS * buf;
+  static constexpr size_t kf = ws + (size_t)kCWarps * WPER;
   static constexpr size_t vb = kf + (size_t)KPlanes<BK, QJL>::regs * 32 * 4;
-  static constexpr int MAXBLK = 64;  // blocks per CTA at most (a.chunk <= 1024 tokens)
-  static constexpr size_t st = vb + (size_t)MAXBLK * 8;
-  static constexpr size_t pw = st + 16 * kG * 4;  // per-warp partials (max logit, sum w, sum X, max ||v||)
-  static constexpr size_t br = pw + 4 * kG * kWarps * 4;  // two mbarriers, one per staging buffer
-  static constexpr size_t total = br + 48;  // + flags at br + 16, merge barrier at br + 32
-  static_assert((size_t)4 * kG * kD * 4 <= 2 * buf, "the value-sum buffer reuses the staging buffers");
-  static_assert(buf % 16 == 0 && x1 % 16 == 0 && kf % 16 == 0, "16-byte aligned regions");
+  static constexpr int MAXBLK = kMaxChunk / 16;
+  static constexpr size_t br = vb + (size_t)MAXBLK * 8;
+  // full[NS], empty[NS], the merge barrier, then flags, query constants, merge factors
+  static constexpr size_t fl = br + (size_t)(2 * NS + 1) * 8;
+  static constexpr size_t total = fl + 8 * 4 + 16 * 4 + kG * 4;
+  static_assert(2 + kProd <= 8, "flag words");
+  // the warps' partial states at the end of the range reuse the staging ring
+  static_assert((size_t)kCWarps * kG * (kD + 2) * 4 <= NS * buf, "warp partials fit the ring");
+  static_assert(buf % 16 == 0 && ws % 16 == 0 && kf % 16 == 0 && vb % 16 == 0, "16-byte aligned regions");
 };
 
 // The arrays a sub-chunk is copied from, one bulk copy (or one per block when paged) each.
@@ -454,47 +474,72 @@ __device__ __forceinline__ void stage_array(const MmaArgs &a, int arr, const cha
   }
 }
 
-// Issue the bulk copies of sub-chunk `sc` of the CTA (blocks [16 sc, 16 sc + 16) of its range)
-// into staging buffer `sb`, completing on `bar` (initialised with one arrival per array).  Warp
-// `arr` (< StageArrays::n) copies array `arr`.  vb[k] = first slot of the CTA's block k, or -1
-// (resolved once per CTA); nlead = number of leading valid blocks of the CTA (contiguous layout,
-// where they are one run of consecutive slots: one copy per array); paged: one copy per block.
-// `extra` bytes (landing on the same barrier, issued by the caller after this returns) are
-// expected by warp 0.
+// Producer warp p's copies of sub-chunk `sc` (blocks [NB sc, NB sc + NB) of the CTA's range) into
+// staging buffer `sb`, completing on `bar`: one arrival with the expected bytes of its arrays (plus
+// `extra` bytes the caller copies on the same barrier), then the copies.  vb[k] = first slot of the
+// CTA's block k or -1; contiguous caches copy the nlead leading valid blocks (consecutive slots)
+// with one copy per array, paged caches one copy per valid block.
 template <int BK, int BV, bool QJL>
 __device__ __forceinline__ void stage_sub(const MmaArgs &a, int sc, const int64_t *vb, int nlead,
-                                          unsigned char *sb, uint64_t *bar, unsigned extra) {
+                                          unsigned char *sb, uint64_t *bar, unsigned extra, int p) {
   using SM = MmaSmem<BK, BV, QJL>;
-  const int arr = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const char *src;
-  size_t doff;
-  unsigned per;
-  int64_t sstride;
-  stage_array<BK, BV, QJL>(a, arr, src, doff, per, sstride);
+  constexpr int NA = StageArrays<QJL>::n;  // producer p copies arrays p, p + kProd, ...
+  const int lane = threadIdx.x & 31;
   const int k0 = SM::NB * sc;
+  unsigned nvalid;
   if (!a.block_table) {
-    if (lane == 0) {
-      int n = nlead - k0;
-      n = n < 0 ? 0 : (n > SM::NB ? SM::NB : n);
-      mbar_expect_arrive(bar, per * (unsigned)n + (arr == 0 ? extra : 0u));
-      if (n > 0) bulk_g2s(sb + doff, src + vb[k0] * sstride, per * (unsigned)n, bar);
-    }
+    int n = nlead - k0;
+    nvalid = (unsigned)(n < 0 ? 0 : (n > SM::NB ? SM::NB : n));
   } else {
-    const int64_t base = lane < SM::NB ? vb[k0 + lane] : -1;
-    const unsigned valid = __ballot_sync(TQ_FULL_MASK, base >= 0);
-    if (lane == 0) mbar_expect_arrive(bar, per * (unsigned)__popc(valid) + (arr == 0 ? extra : 0u));
-    __syncwarp();
-    if (base >= 0) bulk_g2s(sb + doff + (size_t)lane * per, src + base * sstride, per, bar);
+    nvalid = (unsigned)__popc(__ballot_sync(TQ_FULL_MASK, lane < SM::NB && vb[k0 + lane] >= 0));
+  }
+  unsigned bytes = extra;
+#pragma unroll
+  for (int arr = p; arr < NA; arr += kProd) {
+    const char *src;
+    size_t doff;
+    unsigned per;
+    int64_t sstride;
+    stage_array<BK, BV, QJL>(a, arr, src, doff, per, sstride);
+    bytes += per * nvalid;
+  }
+  if (lane == 0) mbar_expect_arrive(bar, bytes);
+  __syncwarp();
+#pragma unroll
+  for (int arr = p; arr < NA; arr += kProd) {
+    const char *src;
+    size_t doff;
+    unsigned per;
+    int64_t sstride;
+    stage_array<BK, BV, QJL>(a, arr, src, doff, per, sstride);
+    if (!a.block_table) {
+      if (lane == 0 && nvalid > 0) bulk_g2s(sb + doff, src + vb[k0] * sstride, per * nvalid, bar);
+    } else {
+      const int64_t base = lane < SM::NB ? vb[k0 + lane] : -1;
+      if (base >= 0) bulk_g2s(sb + doff + (size_t)lane * per, src + base * sstride, per, bar);
+    }
   }
 }
 
-// One CTA = one (sequence, KV head) and a contiguous range of a.chunk tokens (a multiple of 16),
-// streamed in sub-chunks of kSub tokens: the next sub-chunk's bulk copies are in flight while
-// the current one is computed.  Softmax runs across sub-chunks with a running maximum: the value
-// sums of each sub-chunk use that sub-chunk's own fixed-point scale and are folded into fp32
-// accumulators rescaled by e^{M_old - M_new}.
+// One CTA = one (sequence, KV head) and a contiguous range of a.chunk tokens (a multiple of 16).
+// Warps kCWarps.. (kProd of them) stream the range into a ring of NS sub-chunk buffers with bulk
+// copies (each its share of the arrays);
+// every other warp owns 32 tokens (two 16-token blocks) of each sub-chunk and runs the whole
+// decode on them with its own running softmax state, so no CTA-wide barrier falls inside the
+// loop:
+//   1. logits of the 4 query heads (bit-plane u8 x s8 MMAs against the query fragments);
+//   2. running maximum and sum of the warp's tokens, value weights W = e^{l - M} ||v|| (Sparse V:
+//      W = 0 where the weight is below the threshold, see below), their 16-bit fixed-point
+//      fragments with the warp's own scale;
+//   3. the value MMAs of both blocks over all 128 coordinates into one set of int32
+//      accumulators, folded into fp32 sums rescaled by e^{M_old - M_new}.
+// At the end the warps' (m, l, o~) are merged in shared memory into the CTA's partial.
+// Sparse V ("TurboQuant+ 深度解析" 第六部分): with a threshold tau > 0 a token's value row is left
+// out when e^{l - M} < tau max(1, l_old e^{M_old - M}), a bound that is at least its final softmax
+// weight (the running sum only grows and the running maximum's token counts 1), so every row it
+// drops has a final weight below tau; blocks whose rows are all dropped skip their value MMAs.
 template <int BK, int BV, bool QJL>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kMmaThreads, 2)
 attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restrict__ kfrag,
                   const float *__restrict__ kconst, float *__restrict__ part) {
   using KP = KPlanes<BK, QJL>;
@@ -502,18 +547,14 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
   constexpr int NB = SM::NB;
   constexpr int VT = BV == 3 ? 2 : 1;  // value word types: (p0,p1) and (p2, parity)
   extern __shared__ __align__(16) unsigned char smem[];
-  uint32_t *sx1 = reinterpret_cast<uint32_t *>(smem + SM::x1);
-  float *lg = reinterpret_cast<float *>(smem + SM::lg);          // [kG][kLgS] logits, then weights
-  uint4 *vfrag = reinterpret_cast<uint4 *>(smem + SM::vf);       // [NB][32]
   const uint4 *kf4 = reinterpret_cast<const uint4 *>(smem + SM::kf);  // [plane][k-step][32]
-  int64_t *vball = reinterpret_cast<int64_t *>(smem + SM::vb);   // [MAXBLK] first slot of each block
-  float *hM = reinterpret_cast<float *>(smem + SM::st);          // running max per head
-  float *hL = hM + kG;                                           // running sum of e^{l - M}
-  float *pmax = reinterpret_cast<float *>(smem + SM::pw);        // [kG][kWarps] max logit
-  float *psw = pmax + kG * kWarps;                               // [kG][kWarps] sum of w
-  int *pcs = reinterpret_cast<int *>(psw + kG * kWarps);         // [kG][kWarps] sum of integer weights
-  float *pnv = reinterpret_cast<float *>(pcs + kG * kWarps);     // [kWarps] max ||v|| of valid tokens
-  float *obuf = reinterpret_cast<float *>(smem);                 // [4][kG][kD], after the loop
+  int64_t *vball = reinterpret_cast<int64_t *>(smem + SM::vb);       // [MAXBLK] first slot of each block
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + SM::br);      // [SM::NS] copies landed
+  uint64_t *empty = full + SM::NS;                                  // [SM::NS] consumers done
+  uint64_t *mbar = empty + SM::NS;                                  // the merge's copies
+  volatile int *flags = reinterpret_cast<volatile int *>(smem + SM::fl);  // [0] abort, [1] last, [2] issued
+  float *kcs = reinterpret_cast<float *>(smem + SM::fl + 32);        // [16] query constants
+  float *hM = kcs + 16;                                              // [kG] merge rescale factors
 
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -523,265 +564,228 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
   const int64_t cap = min(a.k.capacity, a.v.capacity);
   constexpr unsigned FB = KP::regs * 32 * 4;  // the query fragments' bytes
 
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::br);
-  int *fail = reinterpret_cast<int *>(smem + SM::br + 16);
-  int *nlead_s = fail + 1;
-  // Contiguous layout: the first sub-chunk's blocks are consecutive slots known before the
-  // sequence length (bounded by the arrays only), so their copies start at once; blocks past the
-  // sequence are masked later like any other.
-  int early = 0;
-  int64_t base0 = 0;
-  if (!a.block_table) {
-    base0 = ((int64_t)b * a.hkv + h) * a.ctx_stride + t0;
-    int64_t nb = base0 < cap ? (cap - base0) / 16 : 0;
-    const int lim = min(SM::NB, a.chunk / 16);
-    early = (int)(nb < lim ? nb : lim);
-  }
   if (tid == 0) {
-    mbar_init(&bars[0], StageArrays<QJL>::n);
-    mbar_init(&bars[1], StageArrays<QJL>::n);
-    mbar_init(&bars[4], 1);  // the merge's copies (br + 32)
+    for (int i = 0; i < SM::NS; ++i) {
+      mbar_init(&full[i], kProd);
+      mbar_init(&empty[i], kCWarps);
+    }
+    mbar_init(mbar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-    *fail = 0;
+    flags[0] = 0;
+    for (int i = 0; i < kProd; ++i) flags[2 + i] = 0;
   }
   // Launched as a programmatic dependent of the query-fragment kernel: everything above overlaps
   // its tail; the caches (appended rows), fragments and counters are read only after this.
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
-  __syncthreads();
-  if (early > 0 && warp < StageArrays<QJL>::n && lane == 0) {
-    const char *src;
-    size_t doff;
-    unsigned per;
-    int64_t sstride;
-    stage_array<BK, BV, QJL>(a, warp, src, doff, per, sstride);
-    mbar_expect_arrive(&bars[0], per * (unsigned)early + (warp == 0 ? FB : 0u));
-    bulk_g2s(smem + doff, src + base0 * sstride, per * (unsigned)early, &bars[0]);
-    if (warp == 0) bulk_g2s(smem + SM::kf, kfrag + grp * KP::regs * 32, FB, &bars[0]);
-  }
   int L = a.seq_lens[b];
   L = L < 0 ? 0 : (L > a.max_len ? a.max_len : L);
   const int t1 = min(L, t0 + a.chunk);
   const int nsub = t1 > t0 ? (t1 - t0 + kSub - 1) / kSub : 0;
-  // the CTA's blocks: first slot, or -1 past the sequence or the arrays
+  // the CTA's blocks: first slot, or -1 past the sequence or the arrays (contiguous caches: the
+  // valid blocks are a prefix, the slots consecutive)
   const int nblk = (t1 - t0 + 15) / 16;
-  if (tid < SM::MAXBLK) {
+  int nlead = 0;
+  if (!a.block_table) {
+    const int64_t base0 = grp * a.ctx_stride + t0;
+    const int64_t fit = base0 < cap ? (cap - base0) / 16 : 0;
+    nlead = (int)(fit < nblk ? fit : nblk);
+  }
+  for (int i = tid; i < SM::MAXBLK; i += kMmaThreads) {
     int64_t base = -1;
-    if (tid < nblk) {
-      base = token_slot(a, b, h, t0 + 16 * tid);
+    if (i < nblk) {
+      base = token_slot(a, b, h, t0 + 16 * i);
       if (base < 0 || base + 16 > cap) base = -1;
     }
-    vball[tid] = base;
-    // contiguous layout: the leading run of valid blocks (consecutive slots)
-    const unsigned inval = __ballot_sync(TQ_FULL_MASK, base < 0);
-    if ((tid & 31) == 0) nlead_s[tid >> 5] = inval ? __ffs(inval) - 1 : 32;
+    vball[i] = base;
   }
-  if (tid < kG) {
-    hM[tid] = -INFINITY;
-    hL[tid] = 0.f;
-  }
+  if (tid < 16) kcs[tid] = kconst[grp * 16 + tid];
   __syncthreads();
-  const int nlead = nlead_s[0] < 32 ? nlead_s[0] : 32 + nlead_s[1];
-  if (early == 0 && warp < StageArrays<QJL>::n && nsub > 0) {
-    // the first sub-chunk (paged layout), and the query fragments (one copy per CTA) on the same
-    // barrier
-    stage_sub<BK, BV, QJL>(a, 0, vball, nlead, smem, &bars[0], FB);
-    if (warp == 0 && lane == 0) bulk_g2s(smem + SM::kf, kfrag + grp * KP::regs * 32, FB, &bars[0]);
-  }
-  if (early > 0 && nsub == 0) {
-    // an empty range still owns the early copies in flight: they land before the buffers are
-    // reused for the partials
-    if (!__syncthreads_and(mbar_wait_bounded(&bars[0], 0u))) {
-      if (tid == 0) {
-        atomicOr(&g_tq_device_flags, kFlagStagingTimeout);
-        mbar_wait_bounded(&bars[0], 0u);
-      }
-      __syncthreads();
-    }
-  }
+
+  // consumer state: running maximum and sum of head t (same on every gid of a warp) and the value
+  // sums of head t at coordinates 16 gid + i (rotated domain)
+  float Mrun = -INFINITY, Lw = 0.f;
+  float o[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) o[i] = 0.f;
   // Test hook (tq_debug_wait_probe): one bounded wait on the merge barrier, armed for bytes that
-  // no copy sends, so that it runs out while the first sub-chunk's copies are in flight; the CTA
+  // no copy sends, so that it runs out while the first sub-chunks' copies are in flight; the CTA
   // then takes the same abort path as a staging timeout (flag, drain its copies, return).
   const int probe = g_tq_wait_probe;
-  if (probe > 0) {
-    if (tid == 0) {
-      mbar_expect_arrive(&bars[4], 16u);
-      bool ok = false;
-      for (int i = 0; i < probe && !ok; ++i) ok = mbar_try_wait(&bars[4], 0u);
-      if (!ok) *fail = 1;
-    }
-    __syncthreads();
-    if (*fail) {
-      if (tid == 0) {
-        atomicOr(&g_tq_device_flags, kFlagStagingTimeout);
-        if (nsub > 0 || early > 0) mbar_wait_bounded(&bars[0], 0u);
-      }
-      __syncthreads();
-      return;
-    }
+  if (probe > 0 && tid == 0) {
+    mbar_expect_arrive(mbar, 16u);
+    bool ok = false;
+    for (int i = 0; i < probe && !ok; ++i) ok = mbar_try_wait(mbar, 0u);
+    if (!ok) flags[0] = 1;
   }
-  // the query constants (2^-F_code, 2^-F_sign, Cq, Cp per head), read from shared memory where
-  // used (published by the first sub-chunk's barrier)
-  float *kcs = hL + kG;  // [16]
-  if (tid < 16) kcs[tid] = kconst[grp * 16 + tid];
 
-  // value accumulators of this thread: head t, coordinates jb + 2 mt + r
-  const int ch = warp & 1, bgrp = warp >> 1;
-  const int jb = 64 * ch + 8 * gid;
-  float o[4][2];
-#pragma unroll
-  for (int mt = 0; mt < 4; ++mt) o[mt][0] = o[mt][1] = 0.f;
-
-  for (int sc = 0; sc < nsub; ++sc) {
-    const int cur = sc & 1;
-    const int tk0 = t0 + sc * kSub;
-    if (warp < StageArrays<QJL>::n && sc + 1 < nsub)
-      stage_sub<BK, BV, QJL>(a, sc + 1, vball, nlead, smem + (cur ^ 1) * SM::buf, &bars[cur ^ 1], 0u);
-    if (!mbar_wait_bounded(&bars[cur], (unsigned)(sc >> 1) & 1u)) *fail = 1;
-    __syncthreads();
-    if (*fail) {
-      // the copies did not land in time: report, give the ones in flight a bounded time to
-      // finish (they write this CTA's shared memory), and leave without writing partials
-      if (tid == 0) {
-        atomicOr(&g_tq_device_flags, kFlagStagingTimeout);
-        mbar_wait_bounded(&bars[cur], (unsigned)(sc >> 1) & 1u);
-        if (sc + 1 < nsub) mbar_wait_bounded(&bars[cur ^ 1], (unsigned)((sc + 1) >> 1) & 1u);
+  if (warp >= kCWarps) {
+    // ------------------------------------------------------------ producers: the staging ring
+    const int pw = warp - kCWarps;
+    int sc = 0;
+    for (; sc < nsub; ++sc) {
+      const int st = sc % SM::NS;
+      if (sc >= SM::NS) {
+        const bool ok = mbar_wait_bounded(&empty[st], (unsigned)((sc / SM::NS) - 1) & 1u);
+        if (!__all_sync(TQ_FULL_MASK, ok) || flags[0]) {
+          if (lane == 0) flags[0] = 1;
+          break;
+        }
       }
-      __syncthreads();
-      return;
+      stage_sub<BK, BV, QJL>(a, sc, vball, nlead, smem + (size_t)st * SM::buf, &full[st],
+                             (sc == 0 && pw == 0) ? FB : 0u, pw);
+      if (sc == 0 && pw == 0 && lane == 0) bulk_g2s(smem + SM::kf, kfrag + grp * KP::regs * 32, FB, &full[0]);
     }
-    const unsigned char *sb = smem + cur * SM::buf;
-    const uint32_t *skc = reinterpret_cast<const uint32_t *>(sb + SM::kc);
-    const uint32_t *sks = reinterpret_cast<const uint32_t *>(sb + SM::ks);
-    const float *skn = reinterpret_cast<const float *>(sb + SM::kn);
-    const float *skr = reinterpret_cast<const float *>(sb + SM::kr);
-    const uint32_t *svc = reinterpret_cast<const uint32_t *>(sb + SM::vc);
-    const float *svn = reinterpret_cast<const float *>(sb + SM::vn);
-    const int64_t *vb = vball + NB * sc;  // validity of this sub-chunk's blocks
+    if (lane == 0) flags[2 + pw] = sc;  // sub-chunks issued
+  } else {
+    // ------------------------------------------------------------ consumers: 32 tokens each
+    unsigned char *wsp = smem + SM::ws + (size_t)warp * SM::WPER;
+    float *lgw = reinterpret_cast<float *>(wsp);                       // [kG][kLgS] value weights
+    uint32_t *x1w = reinterpret_cast<uint32_t *>(wsp + SM::WLG);       // [2][kD] (plane 2, parity)
+    const float tau = a.sparse_v;
+    for (int sc = 0; sc < nsub; ++sc) {
+      const int st = sc % SM::NS;
+      const bool ok = mbar_wait_bounded(&full[st], (unsigned)(sc / SM::NS) & 1u);
+      if (!__all_sync(TQ_FULL_MASK, ok) || flags[0]) {
+        if (lane == 0) flags[0] = 1;
+        break;
+      }
+      const unsigned char *sb = smem + (size_t)st * SM::buf;
+      const uint32_t *skc = reinterpret_cast<const uint32_t *>(sb + SM::kc);
+      const uint32_t *sks = reinterpret_cast<const uint32_t *>(sb + SM::ks);
+      const float *skn = reinterpret_cast<const float *>(sb + SM::kn);
+      const float *skr = reinterpret_cast<const float *>(sb + SM::kr);
+      const uint32_t *svc = reinterpret_cast<const uint32_t *>(sb + SM::vc);
+      const float *svn = reinterpret_cast<const float *>(sb + SM::vn);
+      const int64_t *vb = vball + NB * sc;  // validity of this sub-chunk's blocks
+      const int tk0 = t0 + sc * kSub;
 
-    // ------------------------------------------------------------ phase 1: logits (keys x heads)
-    {
-      // warp w: blocks 2w and 2w + 1; the query fragments of one (plane, k-step) serve both.
-      // A = the key words masked in place (bytes 0 or 2^shift; B carries 2^-shift).
-      int acc[2][2][2][4];  // [block][plane type][n-tile][c]
+      // ---------------------------------------------------------- 1. logits (tokens x heads)
+      // blocks 2w and 2w + 1; the query fragments of one (plane, k-step) serve both.  A = the key
+      // words masked in place (bytes 0 or 2^shift; B carries 2^-shift).
+      float lgt[2][2], nvk[2][2];
+      {
+        int acc[2][2][2][4];  // [block][plane type][n-tile][c]
 #pragma unroll
-      for (int kb = 0; kb < 2; ++kb)
+        for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
-        for (int x = 0; x < 2; ++x)
+          for (int x = 0; x < 2; ++x)
 #pragma unroll
-          for (int y = 0; y < 2; ++y)
+            for (int y = 0; y < 2; ++y)
 #pragma unroll
-            for (int z = 0; z < 4; ++z) acc[kb][x][y][z] = 0;
-      uint32_t w[2][2][KP::all];
+              for (int z = 0; z < 4; ++z) acc[kb][x][y][z] = 0;
+        uint32_t w[2][2][KP::all];
 #pragma unroll
-      for (int kb = 0; kb < 2; ++kb)
+        for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const int i = (2 * warp + kb) * 16 + gid + 8 * r;
+          for (int r = 0; r < 2; ++r) {
+            const int i = (2 * warp + kb) * 16 + gid + 8 * r;
 #pragma unroll
-          for (int P = 0; P < BK; ++P) w[kb][r][P] = skc[i * SM::KCW + P * 4 + t];
-          if constexpr (BK == 3) w[kb][r][3] = w[kb][r][0] ^ w[kb][r][1] ^ w[kb][r][2];
-          if constexpr (QJL) w[kb][r][KP::code] = sks[i * SM::KSW + t];
+            for (int P = 0; P < BK; ++P) w[kb][r][P] = skc[i * SM::KCW + P * 4 + t];
+            if constexpr (BK == 3) w[kb][r][3] = w[kb][r][0] ^ w[kb][r][1] ^ w[kb][r][2];
+            if constexpr (QJL) w[kb][r][KP::code] = sks[i * SM::KSW + t];
+          }
+#pragma unroll
+        for (int P = 0; P < KP::all; ++P) {
+          const int pt = (QJL && P == KP::code) ? 1 : 0;
+#pragma unroll
+          for (int stp = 0; stp < 4; ++stp) {
+            const uint4 f = kf4[(P * 4 + stp) * 32 + lane];
+            const uint32_t mlo = 0x01010101u << stp, mhi = 0x01010101u << (stp + 4);
+#pragma unroll
+            for (int kb = 0; kb < 2; ++kb) {
+              const uint32_t a0 = w[kb][0][P] & mlo, a1 = w[kb][1][P] & mlo;
+              const uint32_t a2 = w[kb][0][P] & mhi, a3 = w[kb][1][P] & mhi;
+              mma_u8s8(acc[kb][pt][0], a0, a1, a2, a3, f.x, f.y);
+              mma_u8s8(acc[kb][pt][1], a0, a1, a2, a3, f.z, f.w);
+            }
+          }
         }
 #pragma unroll
-      for (int P = 0; P < KP::all; ++P) {
-        const int pt = (QJL && P == KP::code) ? 1 : 0;
+        for (int kb = 0; kb < 2; ++kb) {
+          const int blk = 2 * warp + kb;
+          const bool bok = vb[blk] >= 0;
 #pragma unroll
-        for (int st = 0; st < 4; ++st) {
-          const uint4 f = kf4[(P * 4 + st) * 32 + lane];
-          const uint32_t mlo = 0x01010101u << st, mhi = 0x01010101u << (st + 4);
-#pragma unroll
-          for (int kb = 0; kb < 2; ++kb) {
-            const uint32_t a0 = w[kb][0][P] & mlo, a1 = w[kb][1][P] & mlo;
-            const uint32_t a2 = w[kb][0][P] & mhi, a3 = w[kb][1][P] & mhi;
-            mma_u8s8(acc[kb][pt][0], a0, a1, a2, a3, f.x, f.y);
-            mma_u8s8(acc[kb][pt][1], a0, a1, a2, a3, f.z, f.w);
+          for (int r = 0; r < 2; ++r) {
+            const int i = blk * 16 + gid + 8 * r;
+            const float dc = (float)acc[kb][0][0][2 * r] + 256.f * (float)acc[kb][0][0][2 * r + 1] +
+                             65536.f * (float)acc[kb][0][1][2 * r] + 16777216.f * (float)acc[kb][0][1][2 * r + 1];
+            float sc2 = fmaf(dc, kcs[t], -kcs[8 + t]);
+            if constexpr (QJL) {
+              const float ds = (float)acc[kb][1][0][2 * r] + 256.f * (float)acc[kb][1][0][2 * r + 1] +
+                               65536.f * (float)acc[kb][1][1][2 * r] + 16777216.f * (float)acc[kb][1][1][2 * r + 1];
+              sc2 = fmaf(kc.qjl_scale * skr[i], fmaf(ds, kcs[4 + t], -kcs[12 + t]), sc2);
+            }
+            const bool okt = bok && tk0 + i < t1;
+            lgt[kb][r] = okt ? a.scale * skn[i] * sc2 : -INFINITY;
+            nvk[kb][r] = okt ? svn[i] : 0.f;  // masked slots may hold stale bytes
           }
         }
       }
-      float lmax = -INFINITY, nvmax = 0.f;
-#pragma unroll
-      for (int kb = 0; kb < 2; ++kb) {
-        const int blk = 2 * warp + kb;
-        const bool bok = vb[blk] >= 0;
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const int i = blk * 16 + gid + 8 * r;
-          const float dc = (float)acc[kb][0][0][2 * r] + 256.f * (float)acc[kb][0][0][2 * r + 1] +
-                           65536.f * (float)acc[kb][0][1][2 * r] + 16777216.f * (float)acc[kb][0][1][2 * r + 1];
-          float sc2 = fmaf(dc, kcs[t], -kcs[8 + t]);
-          if constexpr (QJL) {
-            const float ds = (float)acc[kb][1][0][2 * r] + 256.f * (float)acc[kb][1][0][2 * r + 1] +
-                             65536.f * (float)acc[kb][1][1][2 * r] + 16777216.f * (float)acc[kb][1][1][2 * r + 1];
-            sc2 = fmaf(kc.qjl_scale * skr[i], fmaf(ds, kcs[4 + t], -kcs[12 + t]), sc2);
-          }
-          const bool ok = bok && tk0 + i < t1;
-          const float lgt = ok ? a.scale * skn[i] * sc2 : -INFINITY;
-          lg[t * kLgS + i] = lgt;
-          lmax = fmaxf(lmax, lgt);
-          if (ok) nvmax = fmaxf(nvmax, svn[i]);
-        }
-      }
-      // this warp's largest logit per head (lanes sharing t hold the same head)
+
+      // ---------------------------------------------------------- 2. softmax state, weights
+      // lane (gid, t) holds head t of tokens gid, gid + 8 of both blocks; lanes sharing t see
+      // the same head, so reductions run over gid (xor 4, 8, 16)
+      float lmax = fmaxf(fmaxf(lgt[0][0], lgt[0][1]), fmaxf(lgt[1][0], lgt[1][1]));
+      float nvmax = fmaxf(fmaxf(nvk[0][0], nvk[0][1]), fmaxf(nvk[1][0], nvk[1][1]));
 #pragma unroll
       for (int m = 4; m <= 16; m <<= 1) {
         lmax = fmaxf(lmax, __shfl_xor_sync(TQ_FULL_MASK, lmax, m));
         nvmax = fmaxf(nvmax, __shfl_xor_sync(TQ_FULL_MASK, nvmax, m));
       }
-      if (gid == 0) pmax[t * kWarps + warp] = lmax;
-      if (lane == 0) pnv[warp] = nvmax;
-    }
-    __syncthreads();
-
-    // ------------------------------------------------------------ phase 2: weights, value fragments
-    // Each warp weights its own two blocks (tokens 32 w ..) and builds their value-MMA B
-    // fragments; the fixed-point scale comes from the sub-chunk's largest ||v|| (W <= ||v||
-    // since w <= 1), so no cross-warp step is needed in between.
-    {
-      const int g = lane & 3;  // lane = (head lane & 3, tokens lane / 4 + 8 k)
-      const float Mnew = fmaxf(hM[g], max8(pmax + g * kWarps));
+      const float Mnew = fmaxf(Mrun, lmax);
+      const float al = Mnew == -INFINITY ? 1.f : __expf(Mrun - Mnew);
+      const float gate = tau * fmaxf(1.f, Lw * al);  // Sparse V: drop rows with e^{l - M} < gate
       float sw = 0.f;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int i = 32 * warp + (lane >> 2) + 8 * k;
-        const float l = lg[g * kLgS + i];
-        const float wgt = l == -INFINITY ? 0.f : __expf(l - Mnew);
-        lg[g * kLgS + i] = l == -INFINITY ? 0.f : wgt * svn[i];  // masked slots may hold stale bytes
-        sw += wgt;
-      }
+      for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const float l = lgt[kb][r];
+          const float wgt = l == -INFINITY ? 0.f : __expf(l - Mnew);
+          sw += wgt;
+          lgw[t * kLgS + kb * 16 + gid + 8 * r] = (wgt < gate) ? 0.f : wgt * nvk[kb][r];
+        }
 #pragma unroll
       for (int m = 4; m <= 16; m <<= 1) sw += __shfl_xor_sync(TQ_FULL_MASK, sw, m);
-      if (lane < kG) psw[g * kWarps + warp] = sw;
+      Lw = fmaf(Lw, al, sw);
+      Mrun = Mnew;
       if constexpr (BV == 3) {
-        // (plane 2, parity) words of this warp's two blocks, parity = p0 ^ p1 ^ p2
+        // (plane 2, parity) words of the two blocks, parity = p0 ^ p1 ^ p2: lane computes
+        // coordinates 4 lane .. 4 lane + 3 of each block
 #pragma unroll
-        for (int k = 0; k < 2 * kD / 32; ++k) {
-          const int idx = lane + 32 * k;
-          const int kb = 2 * warp + (idx >> 7), j = idx & (kD - 1);
-          const uint32_t A = svc[kb * SM::VBW + j];
-          const uint32_t hw = svc[kb * SM::VBW + kD + (j >> 1)] >> (16 * (j & 1));
-          const uint32_t par = A ^ (A >> 16) ^ hw;
-          sx1[kb * SM::X1W + j] = __byte_perm(hw, par, 0x5410);
+        for (int kk = 0; kk < 2; ++kk) {
+          const uint32_t *bw = svc + (2 * warp + kk) * SM::VBW;
+          const uint4 A = *reinterpret_cast<const uint4 *>(bw + 4 * lane);
+          const uint2 hw2 = *reinterpret_cast<const uint2 *>(bw + kD + 2 * lane);
+          const uint32_t A4[4] = {A.x, A.y, A.z, A.w};
+          const uint32_t H4[4] = {hw2.x, hw2.x >> 16, hw2.y, hw2.y >> 16};
+          uint32_t X4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) X4[e] = __byte_perm(H4[e], A4[e] ^ (A4[e] >> 16) ^ H4[e], 0x5410);
+          *reinterpret_cast<uint4 *>(x1w + kk * kD + 4 * lane) = make_uint4(X4[0], X4[1], X4[2], X4[3]);
         }
       }
       __syncwarp();
-      // B fragments of the value MMAs.  Lane (gid, t): column = (head gid/2, limb gid&1).  The
-      // k index runs over (token, plane) pairs in the order the value words give them:
-      // register 0 = tokens t, t+8 of the low plane, then of the high plane; register 1 = the
-      // same for tokens t+4, t+12.  Byte = limb of X = floor(W 2 e_P sc + dither), dithered so
-      // that the many sub-unit tail weights are unbiased rather than all rounded down.
+      // B fragments of the value MMAs.  Lane (gid, t): column = (head gid/2, limb gid&1).  The k
+      // index runs over (token, plane) pairs in the order the value words give them: register 0
+      // = tokens t, t+8 of the low plane, then of the high plane; register 1 = the same for
+      // tokens t+4, t+12.  Byte = limb of X = floor(W 2 e_P sc + dither), dithered so that the
+      // many sub-unit tail weights are unbiased rather than all rounded down.
       const int gh = gid >> 1, l = gid & 1;
-      float sc, inv;
-      weight_scale(max8(pnv) * 2.f * vc.plane_coef_max, sc, inv);
+      float scl, inv;
+      weight_scale(nvmax * 2.f * vc.plane_coef_max, scl, inv);
       float C[2 * VT];
 #pragma unroll
-      for (int P = 0; P < 2 * VT; ++P) C[P] = 2.f * sc * vc.plane_coef[P];
+      for (int P = 0; P < 2 * VT; ++P) C[P] = 2.f * scl * vc.plane_coef[P];
       const uint32_t sel = (uint32_t)l | ((uint32_t)(4 + l) << 4);  // byte l of two words
       const uint32_t key0 = ((uint32_t)grp * (uint32_t)a.max_len + (uint32_t)tk0) * 4u + (uint32_t)gh;
       uint32_t xs = 0;  // sum of this lane's X values
+      uint32_t bfr[2][2 * VT];
+      bool live[2];
 #pragma unroll
       for (int kk = 0; kk < 2; ++kk) {
         const int kb = 2 * warp + kk;
-        const float *wr = &lg[gh * kLgS + kb * 16];
+        const float *wr = &lgw[gh * kLgS + kk * 16];
         const int toks[4] = {t, t + 8, t + 4, t + 12};
         float W[4], dz[4];
 #pragma unroll
@@ -789,7 +793,7 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
           W[i] = wr[toks[i]];
           dz[i] = dither(key0 + 4u * (uint32_t)(kb * 16 + toks[i]));
         }
-        uint32_t reg[2 * VT];
+        live[kk] = __any_sync(TQ_FULL_MASK, (W[0] > 0.f) | (W[1] > 0.f) | (W[2] > 0.f) | (W[3] > 0.f));
 #pragma unroll
         for (int x = 0; x < VT; ++x)
 #pragma unroll
@@ -799,117 +803,112 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
             const uint32_t x1 = floor_bits(fmaf(W[i1], C[2 * x], dz[i1]));
             const uint32_t x2 = floor_bits(fmaf(W[i0], C[2 * x + 1], dz[i0]));
             const uint32_t x3 = floor_bits(fmaf(W[i1], C[2 * x + 1], dz[i1]));
-            reg[2 * x + rr] = __byte_perm(__byte_perm(x0, x1, sel), __byte_perm(x2, x3, sel), 0x5410);
+            bfr[kk][2 * x + rr] = __byte_perm(__byte_perm(x0, x1, sel), __byte_perm(x2, x3, sel), 0x5410);
             xs += (x0 + x1) + (x2 + x3) - 4u * 0x4B000000u;  // the integers themselves
           }
-        vfrag[kb * 32 + lane] = VT == 2 ? make_uint4(reg[0], reg[1], reg[2 * VT - 2], reg[2 * VT - 1])
-                                        : make_uint4(reg[0], reg[1], 0u, 0u);
       }
-      // the codebook's constant term uses the same integers: sum X per head (limb-0 lanes)
+      // the codebook's constant term uses the same integers: sum X per head (limb-0 lanes), then
+      // head t's sum for the accumulator lanes (lane 8 t holds head t)
       uint32_t mine = l == 0 ? xs : 0u;
       mine += __shfl_xor_sync(TQ_FULL_MASK, mine, 1);
       mine += __shfl_xor_sync(TQ_FULL_MASK, mine, 2);
       mine += __shfl_xor_sync(TQ_FULL_MASK, mine, 4);
-      if (t == 0 && l == 0) pcs[gh * kWarps + warp] = (int)mine;
-    }
-    __syncthreads();
+      const float cterm = 64.f * (float)(int)__shfl_sync(TQ_FULL_MASK, mine, 8 * t);
 
-    // ------------------------------------------------------------ phase 3: value sum
-    // warp w: coordinate half ch = w & 1 (64 coordinates = 4 m-tiles) and blocks bgrp + 4 k.
-    // In m-tile mt, row gid <-> coordinate 64 ch + 8 gid + 2 mt and row gid + 8 <-> the next one.
-    {
+      // ---------------------------------------------------------- 3. value sum, all coordinates
+      // m-tile mt: row gid <-> coordinate 16 gid + 2 mt, row gid + 8 <-> 16 gid + 2 mt + 1.
+      // Token bits t, t+8 (and t+4, t+12) of both planes of a word are moved to bit 7 of each byte
+      // by a multiply (the FMA pipe) and kept by one AND: bytes 0 or 128.
+      int accv[8][4];
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+        for (int z = 0; z < 4; ++z) accv[mt][z] = 0;
       const uint32_t mlo = 1u << (7 - t), mhi = 1u << (3 - t);
-      int accv[4][VT][4];
 #pragma unroll
-      for (int mt = 0; mt < 4; ++mt)
+      for (int kk = 0; kk < 2; ++kk) {
+        const int kb = 2 * warp + kk;
+        if (!live[kk] || vb[kb] < 0) continue;
 #pragma unroll
-        for (int x = 0; x < VT; ++x)
+        for (int x = 0; x < VT; ++x) {
+          const uint32_t *src = (x == 0) ? svc + kb * SM::VBW + 16 * gid : x1w + kk * kD + 16 * gid;
+          uint32_t X[16];
 #pragma unroll
-          for (int z = 0; z < 4; ++z) accv[mt][x][z] = 0;
+          for (int q = 0; q < 4; ++q) {
+            const uint4 u = *reinterpret_cast<const uint4 *>(src + 4 * q);
+            X[4 * q] = u.x; X[4 * q + 1] = u.y; X[4 * q + 2] = u.z; X[4 * q + 3] = u.w;
+          }
 #pragma unroll
-      for (int kk = 0; kk < NB / 4; ++kk) {
-        const int kb = bgrp + 4 * kk;
-        if (vb[kb] < 0) continue;
-        uint32_t X[VT][8];
-        {
-          const uint4 u0 = *reinterpret_cast<const uint4 *>(svc + kb * SM::VBW + jb);
-          const uint4 u1 = *reinterpret_cast<const uint4 *>(svc + kb * SM::VBW + jb + 4);
-          X[0][0] = u0.x; X[0][1] = u0.y; X[0][2] = u0.z; X[0][3] = u0.w;
-          X[0][4] = u1.x; X[0][5] = u1.y; X[0][6] = u1.z; X[0][7] = u1.w;
-        }
-        if constexpr (BV == 3) {
-          const uint4 u0 = *reinterpret_cast<const uint4 *>(sx1 + kb * SM::X1W + jb);
-          const uint4 u1 = *reinterpret_cast<const uint4 *>(sx1 + kb * SM::X1W + jb + 4);
-          X[VT - 1][0] = u0.x; X[VT - 1][1] = u0.y; X[VT - 1][2] = u0.z; X[VT - 1][3] = u0.w;
-          X[VT - 1][4] = u1.x; X[VT - 1][5] = u1.y; X[VT - 1][6] = u1.z; X[VT - 1][7] = u1.w;
-        }
-        const uint4 fb = vfrag[kb * 32 + lane];
-#pragma unroll
-        for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-          for (int x = 0; x < VT; ++x) {
-            // token bits t, t+8 (and t+4, t+12) of both planes moved to bit 7 of each byte by a
-            // multiply (the FMA pipe) and kept by one AND: bytes 0 or 128
-            const uint32_t r0 = X[x][2 * mt], r1 = X[x][2 * mt + 1];
+          for (int mt = 0; mt < 8; ++mt) {
+            const uint32_t r0 = X[2 * mt], r1 = X[2 * mt + 1];
             const uint32_t a0 = mul_lo(r0, mlo) & 0x80808080u, a1 = mul_lo(r1, mlo) & 0x80808080u;
             const uint32_t a2 = mul_lo(r0, mhi) & 0x80808080u, a3 = mul_lo(r1, mhi) & 0x80808080u;
-            mma_u8u8(accv[mt][x], a0, a1, a2, a3, x == 0 ? fb.x : fb.z, x == 0 ? fb.y : fb.w);
+            mma_u8u8(accv[mt], a0, a1, a2, a3, bfr[kk][2 * x], bfr[kk][2 * x + 1]);
           }
+        }
       }
-      // accv[mt][x][c]: c0/c1 = (coordinate jb + 2 mt, head t, limb 0/1), c2/c3 = (+1, ...):
-      // 128 sum_tok X b over the word type's two planes.  With s = 2b - 1 the codebook's
-      // constant term is -(1/2) sum X, added once per sub-chunk by the bgrp 0 warps.
-      const float Mold = hM[t], Mnew = fmaxf(Mold, max8(pmax + t * kWarps));
-      const float al = Mnew == -INFINITY ? 1.f : __expf(Mold - Mnew);
-      float sct, inv;
-      weight_scale(max8(pnv) * 2.f * vc.plane_coef_max, sct, inv);
-      int cs = 0;
+      // accv[mt]: c0/c1 = (coordinate 16 gid + 2 mt, head t, limb 0/1), c2/c3 = (+1, ...):
+      // 128 sum_tok X b; with s = 2b - 1 the codebook's constant term is -(1/2) sum X
 #pragma unroll
-      for (int w2 = 0; w2 < kWarps; ++w2) cs += pcs[t * kWarps + w2];
-      const float cterm = bgrp == 0 ? 64.f * (float)cs : 0.f;
-#pragma unroll
-      for (int mt = 0; mt < 4; ++mt)
+      for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-          float v = 0.f;
-#pragma unroll
-          for (int x = 0; x < VT; ++x) v += (float)accv[mt][x][2 * r] + 256.f * (float)accv[mt][x][2 * r + 1];
-          o[mt][r] = fmaf(o[mt][r], al, (v - cterm) * inv);
+          const float v = (float)accv[mt][2 * r] + 256.f * (float)accv[mt][2 * r + 1];
+          o[2 * mt + r] = fmaf(o[2 * mt + r], al, (v - cterm) * inv);
         }
+      __syncwarp();
+      if (lane == 0) mbar_arrive1(&empty[st]);
     }
-    __syncthreads();  // the buffers, lg, vfrag and the per-warp partials are reused next
-    if (warp == kWarps - 1 && lane < kG) {
-      // head `lane`'s running maximum and sum, from this sub-chunk's per-warp partials (read
-      // before the next sub-chunk's phase 1 rewrites them, published by its first barrier);
-      // the last warp does it, as it issues no copies
-      const float Mold = hM[lane], Mnew = fmaxf(Mold, max8(pmax + lane * kWarps));
-      const float al = Mnew == -INFINITY ? 1.f : __expf(Mold - Mnew);
-      float swh = 0.f;
-#pragma unroll
-      for (int w2 = 0; w2 < kWarps; ++w2) swh += psw[lane * kWarps + w2];
-      hM[lane] = Mnew;
-      hL[lane] = hL[lane] * al + swh;
+  }
+  __syncthreads();
+  if (flags[0]) {
+    // a wait gave up: report, give the copies still in flight a bounded time to land (they write
+    // this CTA's shared memory), and leave without writing partials
+    if (tid == 0) {
+      atomicOr(&g_tq_device_flags, kFlagStagingTimeout);
+      int issued = 0;
+      for (int i = 0; i < kProd; ++i) issued = max(issued, flags[2 + i]);
+      for (int sc = issued > SM::NS ? issued - SM::NS : 0; sc < issued; ++sc)
+        mbar_wait_bounded(&full[sc % SM::NS], (unsigned)(sc / SM::NS) & 1u);
     }
+    __syncthreads();
+    return;
   }
 
-  // ---------------------------------------------------------------- partials of the 4 heads
-  __syncthreads();
+  // ---------------------------------------------------------------- the CTA's partials
+  // every copy has been consumed: the warps' states go through the ring, then one (m, l, o~) per
+  // head is formed from them with their log-sum-exp weights
+  constexpr int WR = kD + 2;
+  float *wst = reinterpret_cast<float *>(smem);  // [kCWarps][kG][WR]: m, l, o~
+  if (warp < kCWarps) {
+    float *row = wst + (warp * kG + t) * WR;
 #pragma unroll
-  for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-    for (int r = 0; r < 2; ++r) obuf[(bgrp * kG + t) * kD + jb + 2 * mt + r] = o[mt][r];
+    for (int i = 0; i < 16; ++i) row[2 + 16 * gid + i] = o[i];
+    if (gid == 0) {
+      row[0] = Mrun;
+      row[1] = Lw;
+    }
+  }
   __syncthreads();
-  for (int i = tid; i < kG * kD; i += kThreads) {
+  for (int i = tid; i < kG * kD; i += kMmaThreads) {
     const int g = i / kD, j = i % kD;
-    const float v = obuf[(0 * kG + g) * kD + j] + obuf[(1 * kG + g) * kD + j] + obuf[(2 * kG + g) * kD + j] +
-                    obuf[(3 * kG + g) * kD + j];
+    float Mx = -INFINITY;
+#pragma unroll
+    for (int w2 = 0; w2 < kCWarps; ++w2) Mx = fmaxf(Mx, wst[(w2 * kG + g) * WR]);
+    float v = 0.f, lsum = 0.f;
+#pragma unroll
+    for (int w2 = 0; w2 < kCWarps; ++w2) {
+      const float *row = wst + (w2 * kG + g) * WR;
+      const float f = row[0] == -INFINITY ? 0.f : __expf(row[0] - Mx);
+      v = fmaf(f, row[2 + j], v);
+      lsum = fmaf(f, row[1], lsum);
+    }
     const int64_t pb = (((int64_t)b * a.hq + (int64_t)h * kG + g) * a.splits + s) * (kD + 4);
     part[pb + 2 + j] = v;
-  }
-  if (tid < kG) {
-    const int64_t pb = (((int64_t)b * a.hq + (int64_t)h * kG + tid) * a.splits + s) * (kD + 4);
-    part[pb] = hM[tid];
-    part[pb + 1] = hL[tid];
+    if (j == 0) {
+      part[pb] = Mx;
+      part[pb + 1] = lsum;
+    }
   }
   if (a.out == nullptr) return;
 
@@ -920,7 +919,7 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
   // release: the barrier orders every thread's partial stores before thread 0's fence, which
   // (cumulatively) orders them before the count at device scope
   __syncthreads();
-  int *last = nlead_s + 2;
+  volatile int *last = flags + 1;
   if (tid == 0) {
     __threadfence();
     *last = atomicAdd(&a.counter[grp], 1) == a.splits - 1;
@@ -950,11 +949,11 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
   for (int s0 = 0; s0 < a.splits; s0 += nb) {
     const int n = min(nb, a.splits - s0);
     // each head's n rows are contiguous in the partials: one bulk copy per head
-    if (tid == 0) mbar_expect_arrive(&bars[4], (unsigned)(kG * n * PR * 4));
+    if (tid == 0) mbar_expect_arrive(mbar, (unsigned)(kG * n * PR * 4));
     __syncthreads();
     if (tid < kG)
       bulk_g2s(stg + (size_t)tid * n * PR, part + pg + ((int64_t)tid * a.splits + s0) * PR, (unsigned)(n * PR * 4),
-               &bars[4]);
+               mbar);
     if (warp < kG) {
       const float *pb = part + pg + ((int64_t)warp * a.splits + s0) * PR;
       float Mb = M, Lb = 0.f;
@@ -992,10 +991,10 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
       M = Mb;
       if (lane == 0) rfac[warp] = r;
     }
-    if (!__syncthreads_and(mbar_wait_bounded(&bars[4], (unsigned)(s0 / nb) & 1u))) {
+    if (!__syncthreads_and(mbar_wait_bounded(mbar, (unsigned)(s0 / nb) & 1u))) {
       if (tid == 0) {
         atomicOr(&g_tq_device_flags, kFlagStagingTimeout);
-        mbar_wait_bounded(&bars[4], (unsigned)(s0 / nb) & 1u);
+        mbar_wait_bounded(mbar, (unsigned)(s0 / nb) & 1u);
       }
       __syncthreads();
       return;
@@ -1066,12 +1065,12 @@ cudaError_t launch_mma(const TqConsts &kc, const TqConsts &vc, const MmaArgs &a,
   // (the query-fragment or decode-prep kernel) finishes; the kernel waits for it before use.  With
   // per-kernel profiling on, an event sits between the two kernels and a plain launch is used.
   if (tq_prof_on()) {
-    attend_mma_kernel<BK, BV, QJL><<<grid, kThreads, smem, st>>>(kc, vc, a, kfrag, kconst, part);
+    attend_mma_kernel<BK, BV, QJL><<<grid, kMmaThreads, smem, st>>>(kc, vc, a, kfrag, kconst, part);
     return cudaGetLastError();
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(kMmaThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -1122,8 +1121,8 @@ bool attn_fast_eligible(const TqConsts &kc, const TqConsts &vc, const tq_attn_de
 int attn_fast_chunk(const tq_attn_desc &desc) {
   // Tokens per CTA (a multiple of 16): the 16-token blocks of all (sequence, KV head) rows split
   // evenly over two resident CTAs per SM, so that a uniform batch runs as one full wave; at least
-  // 128 tokens (the fixed per-CTA work) and at most 1024 (long or ragged batches then run as
-  // many short waves that the block scheduler balances).
+  // one sub-chunk (256 tokens) and at most kMaxChunk (long or ragged batches then run as several
+  // waves that the block scheduler balances).
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) {
     int n = 0;
@@ -1134,7 +1133,8 @@ int attn_fast_chunk(const tq_attn_desc &desc) {
   const int64_t blocks = rows * ((maxlen + 15) / 16);
   const int64_t slots = 2 * (int64_t)sms;
   int64_t per = (blocks + slots - 1) / slots;
-  per = per < 8 ? 8 : (per > 64 ? 64 : per);
+  const int64_t lo = kSub / 16, hi = kMaxChunk / 16;
+  per = per < lo ? lo : (per > hi ? hi : per);
   return (int)(16 * per);
 }
 
@@ -1162,6 +1162,7 @@ cudaError_t launch_attend_fast(const TqConsts &kc, const TqConsts &vc, const tq_
   a.block_table = desc.block_table;
   a.k = desc.k;
   a.v = desc.v;
+  a.sparse_v = desc.sparse_v > 0.f ? desc.sparse_v : 0.f;
   const int planes = (kc.bits + (kc.bits == 3 ? 1 : 0)) + (kc.m > 0 ? 1 : 0);
   const int64_t groups = (int64_t)desc.batch * desc.n_kv_heads;
   uint32_t *kfrag = static_cast<uint32_t *>(extra);
@@ -1227,6 +1228,7 @@ cudaError_t launch_decode_step_fast(const TqConsts &kc, const TqConsts &vc, cons
   a.block_table = desc.block_table;
   a.k = desc.k;
   a.v = desc.v;
+  a.sparse_v = desc.sparse_v > 0.f ? desc.sparse_v : 0.f;
   const int planes = (kc.bits + (kc.bits == 3 ? 1 : 0)) + (kc.m > 0 ? 1 : 0);
   const int64_t groups = (int64_t)desc.batch * desc.n_kv_heads;
   uint32_t *kfrag = static_cast<uint32_t *>(extra);

@@ -211,6 +211,10 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, unsigned by
                "l"(src), "r"(bytes), "r"(smem_addr(bar))
                : "memory");
 }
+// One plain arrival (no transaction bytes).
+__device__ __forceinline__ void mbar_arrive1(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_addr(bar)) : "memory");
+}
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned parity) {
   unsigned ok;
   asm volatile(

@@ -188,7 +188,9 @@ search_mma_kernel(TqConsts c, const uint2 *__restrict__ frag, const float *__res
   float *ls = reinterpret_cast<float *>(smem + L.ls);  // [warp][q][k]
   int64_t *li = reinterpret_cast<int64_t *>(smem + L.li);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
-  const int shard = blockIdx.x, tile = blockIdx.y;
+  // the query tiles of a shard are adjacent in launch order (x fastest), so they run at the same
+  // time and the shard's rows come from DRAM once, the other tiles reading them from L2
+  const int tile = blockIdx.x, shard = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gid = lane >> 2, t = lane & 3;
   const int rg = warp & 3, kh = warp >> 2;
   const int g0 = WPL >= 2 ? kh * HW : 0, st0 = WPL >= 2 ? 0 : 2 * kh;
@@ -484,7 +486,7 @@ cudaError_t launch_mma_search(const TqConsts &c, int shards, const float *qr, co
     e = tq_smem_limit(reinterpret_cast<const void *>(search_mma_kernel<BK, D>), (int)L.total);
     if (e == cudaSuccess) {
       const int64_t rows_per_shard = ((n + shards - 1) / shards + kSmRB - 1) / kSmRB * kSmRB;
-      search_mma_kernel<BK, D><<<dim3((unsigned)shards, (unsigned)tiles), kSmThreads, L.total, st>>>(
+      search_mma_kernel<BK, D><<<dim3((unsigned)tiles, (unsigned)shards), kSmThreads, L.total, st>>>(
           c, frag, kq, nq, db, n, k, rows_per_shard, shards, L.nbuf, cand_s, cand_i);
       e = cudaGetLastError();
     }

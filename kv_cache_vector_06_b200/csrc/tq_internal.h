@@ -100,6 +100,14 @@ cudaError_t launch_rotate(const TqConsts &c, RotateMode mode, const void *x, tq_
                           uint32_t *codes, float *norm, float *rnorm, float *resid,
                           cudaStream_t st, uint32_t *fsigns = nullptr);
 constexpr int64_t kFusedEncodeMaxRows = 4096;
+// Bulk encode at d = 128, one row per thread (encode_tpr.cu): MSE-only contexts in either layout
+// (token blocks: slots == NULL, whole blocks), structured-QJL contexts, and dense Gaussian QJL
+// with m = d on bf16 rows (the projection on tcgen05).
+bool encode_tpr_eligible(const TqConsts &c, const int64_t *slots, tq_dtype dtype);
+int64_t encode_tpr_rows(const TqConsts &c, int64_t n);  // rows it takes (a block-layout tail is left)
+cudaError_t launch_encode_tpr(const TqConsts &c, const void *x, tq_dtype dtype, int64_t n, int64_t ld,
+                              const int64_t *slots, int64_t capacity, uint32_t *codes, float *norm, float *rnorm,
+                              uint32_t *signs, cudaStream_t st);
 
 // Z = R S^T for rows of R ([n][d] fp32).  SIGNS: pack bit = [z >= 0] into `signs` at the rows'
 // slots.  DENSE: write Z as fp32 [n][m] to `zout`.

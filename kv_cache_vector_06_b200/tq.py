@@ -42,7 +42,7 @@ class AttnDesc(ctypes.Structure):
     _fields_ = [("batch", c_int32), ("n_q_heads", c_int32), ("n_kv_heads", c_int32), ("scale", c_float),
                 ("seq_lens", c_void_p), ("block_table", c_void_p), ("max_blocks", c_int32),
                 ("block_size", c_int32), ("ctx_stride", c_int64), ("max_seq_len", c_int32),
-                ("k", PackedC), ("v", PackedC)]
+                ("k", PackedC), ("v", PackedC), ("sparse_v", c_float)]
 
 
 def _load():
@@ -281,7 +281,7 @@ def scores(ctx: Context, q: torch.Tensor, keys: Packed, n: int = None, out=None,
 
 def make_attn_desc(kctx: Context, vctx: Context, q_shape, kcache: Packed, vcache: Packed, seq_lens,
                    max_seq_len: int, ctx_stride: int = None, block_table=None, block_size: int = 16,
-                   scale: float = 0.0, n_kv_heads: int = None) -> AttnDesc:
+                   scale: float = 0.0, n_kv_heads: int = None, sparse_v: float = 0.0) -> AttnDesc:
     batch, hq, _ = q_shape
     if n_kv_heads is None:
         raise ValueError("n_kv_heads is required")
@@ -305,6 +305,7 @@ def make_attn_desc(kctx: Context, vctx: Context, q_shape, kcache: Packed, vcache
     desc.max_seq_len = max_seq_len
     desc.k = kcache.c(kctx)
     desc.v = vcache.c(vctx)
+    desc.sparse_v = sparse_v
     # the descriptor holds raw device pointers: it keeps the tensors they point into alive
     desc._keep = (seq_lens, block_table, kcache, vcache)
     return desc

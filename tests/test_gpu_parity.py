@@ -14,6 +14,7 @@ import torch
 
 import synth
 from oracle import attention as oattn
+from oracle import encode as oenc
 from oracle import search as osearch
 from parity import (Quantizer, assert_attention_close, assert_scores_close, assert_topk_equivalent,
                     compare_encode, oracle_cache, oracle_scores_from_packed, unpack)
@@ -361,6 +362,34 @@ def test_encode_block16_layout(tq, d, bits):
     torch.cuda.synchronize()
     codes, sbits, norm, rnorm = unpack(q, packed, rows=slots)
     compare_encode(q, q.oracle_encode(x.double().numpy()), codes, sbits, norm, rnorm)
+
+
+@pytest.mark.parametrize("layout,bits", [(0, 1), (0, 2), (0, 3), (0, 4), (1, 2), (1, 3), (1, 4), (1, 1)])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_encode_bulk_rows_d128(tq, layout, bits, dtype):
+    """More rows than the fused small-batch limit at d = 128 (one row per thread): row layout
+    and the token-block layout (whole blocks by ballots, a ragged tail of 13 rows through the
+    general kernel next to it, stale bytes in the untouched slots of the last block)."""
+    n = 5011
+    cap = (n + 15) // 16 * 16 + 32
+    q = Quantizer(128, bits, 0, seed=600 + 10 * bits + layout, layout=layout)
+    x = (torch.randn(n, 128, generator=torch.Generator().manual_seed(bits)) *
+         torch.exp(torch.randn(128, generator=torch.Generator().manual_seed(7)))).to(dtype)
+    x[17] = 0  # a zero vector
+    packed = tq.Packed.allocate(q.ctx, cap)
+    packed.codes.fill_(0x5A)
+    tq.encode_kv(q.ctx, x.cuda(), packed)
+    torch.cuda.synchronize()
+    rows = np.arange(n)
+    codes, sbits, norm, rnorm = unpack(q, packed, rows=rows)
+    compare_encode(q, q.oracle_encode(x.double().numpy()), codes, sbits, norm, rnorm)
+    if layout == 1:
+        # slots past n in the last partial block keep their earlier bytes (the tail kernel only
+        # changes the bits of the slots it writes)
+        tail = np.arange(n, (n + 15) // 16 * 16)
+        stale = unpack(q, packed, rows=tail)[0]
+        full = oenc.unpack_codes_block16(np.full((16, packed.codes.shape[1]), 0x5A, dtype=np.uint8), 128, bits)
+        assert np.array_equal(stale, full[tail % 16])
 
 
 @pytest.mark.parametrize("vbits", [2, 3])
