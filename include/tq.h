@@ -163,6 +163,28 @@ tq_status tq_ctx_create(const tq_spec *spec, const int8_t *rot_signs, const floa
 tq_status tq_ctx_create_srht(const tq_spec *spec, const int8_t *rot_signs, const int8_t *qjl_signs,
                              int32_t device, tq_ctx **out);
 
+/* Create a context whose first stage is PolarQuant instead of the per-coordinate quantizer
+ * ([JJ] 第二部分 第一步 "PolarQuant——换一个坐标系来看数据"; [VC] 第一階段): after the same random
+ * rotation, coordinates are paired into (radius, angle), the radii paired again, recursively, to
+ * one radius (the stored norm) and d - 1 angles, each angle quantized with spec->mse_bits bits by
+ * the Lloyd-Max codebook of its level's known law (tq_polar_codebook); no per-block constants.
+ * The QJL stage, when qjl_m > 0, sketches the residual y/||x|| - y^ with the dense S as usual.
+ * Packed arrays as for tq_ctx_create: code slot p holds angle p (level 1 first: d/2 angles, then
+ * level 2, ..., the last level's single angle at d - 2; slot d - 1 is 0).  Supported calls:
+ * tq_encode_kv and tq_scores; the attention and search calls return TQ_EUNSUPPORTED.
+ *   spec  d = 128, TQ_LAYOUT_ROWS, mse_bits 1..4, qjl_m 0 or a multiple of 32 up to 1024
+ * Errors: as tq_ctx_create; TQ_EUNSUPPORTED for other d or layouts. */
+tq_status tq_ctx_create_polar(const tq_spec *spec, const int8_t *rot_signs, const float *qjl_matrix,
+                              int32_t device, tq_ctx **out);
+
+/* PolarQuant angle codebook of one level (host, fp64).  Level 1 angles of a uniformly random
+ * direction are uniform on (-pi, pi]: 2^bits equal cells from -pi, centroids at the cell middles.
+ * A level-l angle, l >= 2, is atan2 of two independent radii of k = 2^(l-1) coordinates each, with
+ * density 2 (sin a cos a)^(k-1) / B(k/2, k/2) on [0, pi/2]: its Lloyd-Max codebook.
+ *   centroids host out [2^bits], thresholds host out [2^bits - 1]
+ * Errors: TQ_EINVAL (nulls), TQ_EUNSUPPORTED (level outside 1..10, bits outside 1..4). */
+tq_status tq_polar_codebook(int32_t level, int32_t bits, double *centroids, double *thresholds);
+
 /* Free a context (NULL is accepted).  The caller must ensure no queued work still uses it. */
 tq_status tq_ctx_destroy(tq_ctx *ctx);
 

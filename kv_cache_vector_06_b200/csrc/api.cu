@@ -111,7 +111,7 @@ tq_status tq_make_codebook(int32_t d, int32_t bits, double *centroids, double *t
 
 // Shared by tq_ctx_create (caller-drawn S) and tq_ctx_create_srht (S = P H D2 built here).
 static tq_status ctx_create(const tq_spec *spec, const int8_t *rot_signs, const float *qjl_matrix,
-                            const int8_t *qjl_signs, int32_t device, tq_ctx **out) {
+                            const int8_t *qjl_signs, bool polar, int32_t device, tq_ctx **out) {
   if (!out) return tq_fail(TQ_EINVAL, "out is NULL");
   *out = nullptr;
   tq_status st = check_spec(spec);
@@ -158,10 +158,27 @@ static tq_status ctx_create(const tq_spec *spec, const int8_t *rot_signs, const 
     e = cudaMemcpy(c->dev_S, qjl_matrix, sizeof(float) * (size_t)m * d, cudaMemcpyHostToDevice);
   if (e == cudaSuccess && qjl_signs)
     e = cudaMemcpy(c->dev_qjl_signs, hs2, sizeof(float) * d, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && polar) {
+    // PolarQuant angle tables: per level, the thresholds and the cos / sin of the centroids
+    constexpr int kLv = 7;
+    float tab[kLv][3][16] = {};
+    for (int l = 1; l <= kLv; ++l) {
+      double cc[16], tt[16];
+      tq_polar_codebook_fp64(l, spec->mse_bits, cc, tt);
+      for (int i = 0; i < L; ++i) {
+        tab[l - 1][0][i] = i < L - 1 ? (float)tt[i] : INFINITY;
+        tab[l - 1][1][i] = (float)std::cos(cc[i]);
+        tab[l - 1][2][i] = (float)std::sin(cc[i]);
+      }
+    }
+    e = cudaMalloc(&c->dev_polar, sizeof(tab));
+    if (e == cudaSuccess) e = cudaMemcpy(c->dev_polar, tab, sizeof(tab), cudaMemcpyHostToDevice);
+  }
   if (e != cudaSuccess) {
     cudaFree(c->dev_signs);
     cudaFree(c->dev_S);
     cudaFree(c->dev_qjl_signs);
+    cudaFree(c->dev_polar);
     delete c;
     return tq_cuda_check(e, "upload of context constants");
   }
@@ -183,6 +200,8 @@ static tq_status ctx_create(const tq_spec *spec, const int8_t *rot_signs, const 
   k.S = c->dev_S;
   k.srht = qjl_signs ? 1 : 0;
   k.qjl_signs = c->dev_qjl_signs;
+  k.polar = polar ? 1 : 0;
+  k.polar_tab = c->dev_polar;
   // odd bit-plane expansion of the codebook for the tensor-core attention path:
   // e_S = 2^-b sum_code c[code] prod_{P in S} s_P(code), S in {0}, {1}, {2}, {0,1,2}
   k.fast_ok = 0;
@@ -225,7 +244,25 @@ static tq_status ctx_create(const tq_spec *spec, const int8_t *rot_signs, const 
 tq_status tq_ctx_create(const tq_spec *spec, const int8_t *rot_signs, const float *qjl_matrix,
                         int32_t device, tq_ctx **out) {
   g_err[0] = 0;
-  return ctx_create(spec, rot_signs, qjl_matrix, nullptr, device, out);
+  return ctx_create(spec, rot_signs, qjl_matrix, nullptr, false, device, out);
+}
+
+tq_status tq_ctx_create_polar(const tq_spec *spec, const int8_t *rot_signs, const float *qjl_matrix,
+                              int32_t device, tq_ctx **out) {
+  g_err[0] = 0;
+  tq_status st = check_spec(spec);
+  if (st != TQ_OK) return st;
+  if (spec->d != 128 || spec->layout != TQ_LAYOUT_ROWS)
+    return tq_fail(TQ_EUNSUPPORTED, "PolarQuant contexts: d = 128 and TQ_LAYOUT_ROWS");
+  return ctx_create(spec, rot_signs, qjl_matrix, nullptr, true, device, out);
+}
+
+tq_status tq_polar_codebook(int32_t level, int32_t bits, double *centroids, double *thresholds) {
+  g_err[0] = 0;
+  if (!centroids || !thresholds) return tq_fail(TQ_EINVAL, "centroids/thresholds is NULL");
+  if (level < 1 || level > 10 || bits < 1 || bits > 4)
+    return tq_fail(TQ_EUNSUPPORTED, "level %d / bits %d: levels 1..10, bits 1..4", level, bits);
+  return tq_polar_codebook_fp64(level, bits, centroids, thresholds);
 }
 
 tq_status tq_ctx_create_srht(const tq_spec *spec, const int8_t *rot_signs, const int8_t *qjl_signs,
@@ -247,7 +284,7 @@ tq_status tq_ctx_create_srht(const tq_spec *spec, const int8_t *rot_signs, const
   if (!S) return tq_fail(TQ_ENOMEM, "host allocation failed");
   for (int i = 0; i < m; ++i)
     for (int j = 0; j < d; ++j) S[(size_t)i * d + j] = (__builtin_popcount((unsigned)(i & j)) & 1) ? -qjl_signs[j] : qjl_signs[j];
-  st = ctx_create(spec, rot_signs, S, qjl_signs, device, out);
+  st = ctx_create(spec, rot_signs, S, qjl_signs, false, device, out);
   delete[] S;
   return st;
 }
@@ -260,6 +297,7 @@ tq_status tq_ctx_destroy(tq_ctx *ctx) {
   cudaFree(ctx->dev_signs);
   cudaFree(ctx->dev_S);
   cudaFree(ctx->dev_qjl_signs);
+  cudaFree(ctx->dev_polar);
   if (cur >= 0) cudaSetDevice(cur);
   delete ctx;
   return TQ_OK;
@@ -281,7 +319,7 @@ tq_status tq_encode_workspace_size(const tq_ctx *ctx, int64_t n, size_t *bytes) 
   if (!bytes) return tq_fail(TQ_EINVAL, "bytes is NULL");
   if (n < 0) return tq_fail(TQ_EINVAL, "n < 0");
   const int64_t rows = n < kEncodeChunk ? n : kEncodeChunk;
-  const bool fused = (n <= kFusedEncodeMaxRows && ctx->spec.d >= 128) || ctx->k.srht;
+  const bool fused = !ctx->k.polar && ((n <= kFusedEncodeMaxRows && ctx->spec.d >= 128) || ctx->k.srht);
   *bytes = (ctx->spec.qjl_m > 0 && !fused) ? (size_t)(rows * ctx->spec.d * 4) : 0;
   return TQ_OK;
 }
@@ -313,6 +351,31 @@ tq_status tq_encode_kv(const tq_ctx *ctx, const void *x, tq_dtype dtype, int64_t
   if (st != TQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool qjl = ctx->spec.qjl_m > 0;
+  if (ctx->k.polar) {
+    // PolarQuant first stage; with a QJL stage the residual rows pass through the workspace
+    for (int64_t r0 = 0; r0 < n; r0 += kEncodeChunk) {
+      const int64_t rows = (n - r0) < kEncodeChunk ? (n - r0) : kEncodeChunk;
+      const char *xr = static_cast<const char *>(x) + r0 * ld * esz;
+      const int64_t *sl = slots ? slots + r0 : nullptr;
+      tq_packed o = out;
+      if (!slots) {
+        o.codes = static_cast<char *>(out.codes) + r0 * ctx->code_bytes;
+        o.norm = out.norm + r0;
+        if (qjl) {
+          o.signs = static_cast<char *>(out.signs) + r0 * ctx->sign_bytes;
+          o.rnorm = out.rnorm + r0;
+        }
+        o.capacity = out.capacity - r0;
+      }
+      cudaError_t e = launch_encode_polar(ctx->k, xr, dtype, rows, ld, sl, o.capacity, static_cast<uint32_t *>(o.codes),
+                                          o.norm, qjl ? o.rnorm : nullptr, qjl ? static_cast<float *>(ws) : nullptr, s);
+      if (e == cudaSuccess && qjl)
+        e = launch_project(ctx->k, PROJ_SIGNS, static_cast<const float *>(ws), rows, sl, o.capacity,
+                           static_cast<uint32_t *>(o.signs), nullptr, s);
+      if (e != cudaSuccess) return tq_cuda_check(e, "polar encode launch");
+    }
+    return TQ_OK;
+  }
   if (n > kFusedEncodeMaxRows && encode_tpr_eligible(ctx->k, slots, dtype)) {
     // bulk rows at d = 128: one row per thread
     const int64_t nt = encode_tpr_rows(ctx->k, n);
@@ -401,6 +464,7 @@ tq_status tq_scores(const tq_ctx *ctx, const void *q, tq_dtype dtype, int32_t nq
   float *p = reinterpret_cast<float *>(static_cast<char *>(ws) + tq_align_up((int64_t)nq * ctx->spec.d * 4, 256));
   st = prep_queries(ctx, q, dtype, nq, qr, p, s);
   if (st != TQ_OK) return st;
+  if (ctx->k.polar) return tq_cuda_check(launch_scores_polar(ctx->k, qr, p, nq, keys, n, out, s), "scores launch");
   return tq_cuda_check(launch_scores(ctx->k, qr, p, nq, keys, n, out, s), "scores launch");
 }
 
@@ -412,6 +476,8 @@ static tq_status check_attn(const tq_ctx *kctx, const tq_ctx *vctx, const tq_att
   if (!desc) return tq_fail(TQ_EINVAL, "desc is NULL");
   if (kctx->spec.d != vctx->spec.d)
     return tq_fail(TQ_EUNSUPPORTED, "K and V contexts differ in d (%d vs %d)", kctx->spec.d, vctx->spec.d);
+  if (kctx->k.polar || vctx->k.polar)
+    return tq_fail(TQ_EUNSUPPORTED, "PolarQuant contexts: encode and scores only");
   if (vctx->spec.qjl_m != 0)
     return tq_fail(TQ_EUNSUPPORTED, "the V context must be MSE-only (qjl_m == 0)");
   if (kctx->spec.layout != TQ_LAYOUT_ROWS)
@@ -590,6 +656,7 @@ tq_status tq_search_topk(const tq_ctx *ctx, const void *q, tq_dtype dtype, int32
   if (!aligned16(q) || !aligned16(out_scores) || !aligned16(out_idx))
     return tq_fail(TQ_EINVAL, "q/out not 16-byte aligned");
   if (ctx->spec.layout != TQ_LAYOUT_ROWS) return tq_fail(TQ_EUNSUPPORTED, "tq_search_topk needs TQ_LAYOUT_ROWS");
+  if (ctx->k.polar) return tq_fail(TQ_EUNSUPPORTED, "PolarQuant contexts: encode and scores only");
   st = check_packed(ctx, db, n, "db", true);
   if (st != TQ_OK) return st;
   size_t need = 0;

@@ -38,7 +38,6 @@ constexpr int kG = 4;
 // Poll count of the test hook's bounded wait (0 = off); see tq_debug_wait_probe.
 __device__ int g_tq_wait_probe;
 constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
 
 struct MmaArgs {
   int hq, hkv, max_len, chunk, splits, block_size, max_blocks;
@@ -382,12 +381,6 @@ __device__ __forceinline__ void weight_scale(float top, float &sc, float &inv128
   sc = pow2i(16 - e) * (1.f - 1.f / 512.f);
   inv128 = pow2i(e - 23) * (512.f / 511.f);
 }
-// Largest of the 8 per-warp partials of one head.
-__device__ __forceinline__ float max8(const float *p) {
-  const float4 u = *reinterpret_cast<const float4 *>(p), v = *reinterpret_cast<const float4 *>(p + 4);
-  return fmaxf(fmaxf(fmaxf(u.x, u.y), fmaxf(u.z, u.w)), fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
-}
-
 // 32-bit multiply kept as such (an opaque multiplier: a power of two here, which would otherwise
 // become a shift on the integer ALU pipe).
 __device__ __forceinline__ uint32_t mul_lo(uint32_t x, uint32_t m) {

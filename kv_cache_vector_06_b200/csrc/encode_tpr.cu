@@ -254,9 +254,9 @@ cudaError_t launch_tpr_t(const TqConsts &c, const TprArgs &a, cudaStream_t st) {
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t ntiles = (a.n + kTRows - 1) / kTRows;
   const int64_t grid = ntiles < 3 * (int64_t)sms ? ntiles : 3 * (int64_t)sms;
-  tq_prof_begin(TQK_ROTATE_ENCODE, st);
+  tq_prof_begin(TQK_ENCODE_ROWS, st);
   encode_tpr_kernel<DT, BITS, BLK, SRHT><<<(unsigned)grid, kTRows, smem, st>>>(c, a);
-  tq_prof_end(TQK_ROTATE_ENCODE, st);
+  tq_prof_end(TQK_ENCODE_ROWS, st);
   return cudaGetLastError();
 }
 
@@ -296,17 +296,18 @@ __device__ __forceinline__ void pack_signs_from_z(uint32_t zaddr, const TqConsts
   if (slot >= 0) *reinterpret_cast<uint4 *>(a.signs + slot * c.sign_words) = make_uint4(sb[0], sb[1], sb[2], sb[3]);
 }
 
-// tpr_stage with the copies spread over `nthreads` threads.
+// tpr_stage by the 128 threads of one group (gt = thread index within the group).
 template <int DT>
-__device__ __forceinline__ void tpr_stage_n(const char *__restrict__ x, int64_t ld_bytes, int64_t n, int64_t r0,
-                                            unsigned char *dst, int nthreads) {
+__device__ __forceinline__ void tpr_stage_g(const char *__restrict__ x, int64_t ld_bytes, int64_t n, int64_t r0,
+                                            unsigned char *dst, int gt) {
   using R = TprRow<DT>;
-  for (int c = threadIdx.x; c < kTRows * R::chunks; c += nthreads) {
-    const int row = c / R::chunks, col = c % R::chunks;
+  for (int cc = gt; cc < kTRows * R::chunks; cc += kTRows) {
+    const int row = cc / R::chunks, col = cc % R::chunks;
     if (r0 + row < n) cp_async16(dst + row * R::stride + col * 16, x + (r0 + row) * ld_bytes + col * 16);
   }
   asm volatile("cp.async.commit_group;\n" ::: "memory");
 }
+
 
 // ------------------------------------------------------------------ Gaussian QJL on tcgen05
 // Keys with a dense Gaussian JL matrix (m = d = 128): the same front end (one row per thread), then
@@ -314,23 +315,27 @@ __device__ __forceinline__ void tpr_stage_n(const char *__restrict__ x, int64_t 
 // operand split as x = tf32(x) + (x - tf32(x)); the dropped r_lo S_lo term is below 2^-22 of the
 // products), which keeps z within a few fp32 ulps of the fp32 dot product.
 //   A = the tile's residual rows, written by their own threads into tensor memory (lane = row,
-//       one column per coordinate; r_hi at columns 0-127, r_lo at 128-255);
+//       one column per coordinate): r_hi for the first two products, then r_lo in the same
+//       columns for the third;
 //   B = S_hi, S_lo in shared memory (canonical K-major layout, staged once per CTA);
-//   D = z in tensor memory (columns 256-383), read back by the row's thread for its sign bits.
-// Warps 0-3 compute (thread = row = tensor-memory lane), warp 4 issues the MMAs (one thread) and
-// owns the tensor-memory allocation.  While the MMAs of tile i run, the compute warps encode tile
-// i + 1; they read tile i's z (and pack its signs) just before writing tile i + 1's residual.
-constexpr int kQThreads = 160;
+//   D = z in tensor memory, read back by the row's thread for its sign bits.
+// Two groups of four compute warps (thread = row = tensor-memory lane) take alternate tiles, each
+// with its own 256 tensor-memory columns (residual 128, z 128) and staging buffer; warp 8 issues
+// the MMAs (one thread) and owns the allocation.  A group packs its previous tile's signs before
+// encoding its next tile, so while one group waits for its products the other one computes.
+constexpr int kQGroups = 2;
+constexpr int kQThreads = (4 * kQGroups + 1) * 32;
+constexpr int kQMmaWarp = 4 * kQGroups;
 constexpr uint32_t kQLbo = 128, kQSbo = 4096;  // S: 8-row x 16-byte core matrices, K-major
 constexpr int kQSBytes = kTD * kTD * 4;        // one of S_hi / S_lo
 
 template <int DT>
 struct QSmem {
-  static constexpr size_t x = 0;  // two staged tiles of rows
-  static constexpr size_t shi = x + (size_t)2 * kTRows * TprRow<DT>::stride;
+  static constexpr size_t x = 0;  // one staged tile of rows per group
+  static constexpr size_t shi = x + (size_t)kQGroups * kTRows * TprRow<DT>::stride;
   static constexpr size_t slo = shi + kQSBytes;
-  static constexpr size_t bars = slo + kQSBytes;  // rfull, zfull, done
-  static constexpr size_t total = bars + 64;
+  static constexpr size_t bars = slo + kQSBytes;  // per group: rhi, rlo, hidone, zfull; then done
+  static constexpr size_t total = bars + (size_t)(4 * kQGroups + 1) * 8;
   static_assert(shi % 128 == 0, "descriptor base alignment");
 };
 
@@ -340,6 +345,13 @@ __device__ __forceinline__ bool qwait(uint64_t *bar, unsigned parity, volatile i
     if (*abort_flag) return false;
   }
   return false;
+}
+
+__device__ __forceinline__ void group_sync(int g) {
+  if (g == 0)
+    asm volatile("bar.sync 1, 128;\n" ::: "memory");
+  else
+    asm volatile("bar.sync 2, 128;\n" ::: "memory");
 }
 
 template <int DT, int BITS>
@@ -352,8 +364,8 @@ encode_tcq_kernel(TqConsts c, TprArgs a) {
   __shared__ uint32_t tslot;
   __shared__ int abort_flag_s;
   volatile int *abort_flag = &abort_flag_s;
-  uint64_t *rfull = reinterpret_cast<uint64_t *>(smem + SM::bars);
-  uint64_t *zfull = rfull + 1, *done = rfull + 2;
+  uint64_t *gb = reinterpret_cast<uint64_t *>(smem + SM::bars);  // [group][rhi, rlo, hidone, zfull]
+  uint64_t *done = gb + 4 * kQGroups;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   constexpr int L = 1 << BITS;
 
@@ -367,16 +379,20 @@ encode_tcq_kernel(TqConsts c, TprArgs a) {
     *reinterpret_cast<uint32_t *>(smem + SM::shi + off) = hi;
     *reinterpret_cast<uint32_t *>(smem + SM::slo + off) = to_tf32(lo);
   }
-  for (int j = tid; j < kTD; j += kQThreads) sgn[j] = c.signs[j];
+  for (int jj = tid; jj < kTD; jj += kQThreads) sgn[jj] = c.signs[jj];
   if (tid < TQ_MAX_LEVELS) cen[tid] = c.centroids[tid];
   if (tid == 0) {
-    mbar_init(rfull, 4);
-    mbar_init(zfull, 1);
+    for (int g = 0; g < kQGroups; ++g) {
+      mbar_init(&gb[4 * g + 0], 4);
+      mbar_init(&gb[4 * g + 1], 4);
+      mbar_init(&gb[4 * g + 2], 1);
+      mbar_init(&gb[4 * g + 3], 1);
+    }
     mbar_init(done, 1);
     abort_flag_s = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
-  if (warp == 4) {
+  if (warp == kQMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_addr(&tslot)),
                  "r"(512)
                  : "memory");
@@ -390,7 +406,7 @@ encode_tcq_kernel(TqConsts c, TprArgs a) {
   const int64_t ntiles = (a.n + kTRows - 1) / kTRows;
   const int64_t mytiles = ntiles > blockIdx.x ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
-  if (warp == 4) {
+  if (warp == kQMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       // D f32, A and B tf32, both K-major, N = 128, M = 128
@@ -398,22 +414,31 @@ encode_tcq_kernel(TqConsts c, TprArgs a) {
                              ((uint32_t)(kTRows >> 4) << 24);
       const uint32_t shi = smem_addr(smem + SM::shi), slo = smem_addr(smem + SM::slo);
       for (int64_t i = 0; i < mytiles; ++i) {
-        if (!qwait(rfull, (unsigned)(i & 1), abort_flag)) {
+        const int g = (int)(i % kQGroups);
+        const unsigned ph = (unsigned)((i / kQGroups) & 1);
+        uint64_t *b = gb + 4 * g;
+        const uint32_t rcol = tmem + 256u * g, zcol = rcol + 128u;
+        if (!qwait(&b[0], ph, abort_flag)) {
           *abort_flag = 1;
           break;
         }
         tc_fence_after();
-        const uint32_t zcol = tmem + 256u;
 #pragma unroll
-        for (int pass = 0; pass < 3; ++pass) {
-          const uint32_t acol = tmem + (pass == 2 ? 128u : 0u);  // r_hi, r_hi, r_lo
-          const uint32_t bsm = pass == 1 ? slo : shi;           // S_hi, S_lo, S_hi
+        for (int pass = 0; pass < 2; ++pass)  // r_hi S_hi, r_hi S_lo
 #pragma unroll
           for (int ks = 0; ks < kTD / 8; ++ks)
-            umma_tf32_ta(zcol, acol + 8u * ks, umma_desc(bsm + 2u * kQLbo * ks, kQLbo, kQSbo), idesc,
+            umma_tf32_ta(zcol, rcol + 8u * ks, umma_desc((pass ? slo : shi) + 2u * kQLbo * ks, kQLbo, kQSbo), idesc,
                          (pass == 0 && ks == 0) ? 0u : 1u);
+        umma_commit(&b[2]);
+        if (!qwait(&b[1], ph, abort_flag)) {
+          *abort_flag = 1;
+          break;
         }
-        umma_commit(zfull);
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < kTD / 8; ++ks)  // r_lo S_hi
+          umma_tf32_ta(zcol, rcol + 8u * ks, umma_desc(shi + 2u * kQLbo * ks, kQLbo, kQSbo), idesc, 1u);
+        umma_commit(&b[3]);
       }
       umma_commit(done);  // every MMA this thread issued has completed when `done` fires
       qwait(done, 0u, abort_flag);
@@ -421,46 +446,54 @@ encode_tcq_kernel(TqConsts c, TprArgs a) {
     __syncwarp();
   } else {
     // ------------------------------------------------------------ compute: one row per thread
-    float thr[L - 1];
-#pragma unroll
-    for (int i = 0; i < L - 1; ++i) thr[i] = c.thresholds[i];
+    const int g = warp >> 2, gt = tid & 127;  // group, row within the tile
+    uint64_t *b = gb + 4 * g;
+    unsigned char *xbuf = smem + SM::x + (size_t)g * kTRows * R::stride;
     const float sqrtd = 1.f / c.inv_sqrt_d;
-    const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
+    const uint32_t rbase = tmem + 256u * g + ((uint32_t)(32 * (warp & 3)) << 16), zbase = rbase + 128u;
     int64_t prev_slot = -1;
-    int buf = 0;
-    int64_t tile = blockIdx.x;
-    if (tile < ntiles) tpr_stage_n<DT>(a.x, a.ld_bytes, a.n, tile * kTRows, smem + SM::x, 128);
-    for (int64_t i = 0; i < mytiles; ++i, tile += gridDim.x) {
-      const int64_t next = tile + gridDim.x;
-      if (next < ntiles) {
-        tpr_stage_n<DT>(a.x, a.ld_bytes, a.n, next * kTRows, smem + SM::x + (buf ^ 1) * kTRows * R::stride, 128);
-        asm volatile("cp.async.wait_group 1;\n" ::: "memory");
-      } else {
-        asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+    bool ok = true;
+    int64_t j = 0;  // this group's tiles so far
+    int64_t i = g;  // local tile index
+    if (i < mytiles) tpr_stage_g<DT>(a.x, a.ld_bytes, a.n, (blockIdx.x + i * gridDim.x) * kTRows, xbuf, gt);
+    for (; i < mytiles; i += kQGroups, ++j) {
+      const int64_t tile = blockIdx.x + i * gridDim.x;
+      // this group's previous z: its signs first (its columns are then free for this tile)
+      if (j > 0) {
+        ok = qwait(&b[3], (unsigned)((j - 1) & 1), abort_flag);
+        if (!__all_sync(TQ_FULL_MASK, ok)) {
+          if (lane == 0) *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        pack_signs_from_z(zbase, c, a, prev_slot);
       }
-      asm volatile("bar.sync 1, 128;\n" ::: "memory");
-      const int64_t row = tile * kTRows + tid;
+      asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+      group_sync(g);
+      const int64_t row = tile * kTRows + gt;
       const bool valid = row < a.n;
       const int64_t slot = valid ? (a.slots ? a.slots[row] : row) : -1;
       const bool store = valid && slot >= 0 && slot < a.capacity;
       float v[kTD];
-      tpr_load<DT>(smem + SM::x + buf * kTRows * R::stride + tid * R::stride, v);
-      asm volatile("bar.sync 1, 128;\n" ::: "memory");  // this buffer is refilled next iteration
+      tpr_load<DT>(xbuf + gt * R::stride, v);
+      group_sync(g);  // the buffer is free: stage this group's next tile
+      if (i + kQGroups < mytiles)
+        tpr_stage_g<DT>(a.x, a.ld_bytes, a.n, (blockIdx.x + (i + kQGroups) * gridDim.x) * kTRows, xbuf, gt);
       float ss = 0.f;
 #pragma unroll
-      for (int j = 0; j < kTD; ++j) ss = fmaf(v[j], v[j], ss);
+      for (int jj = 0; jj < kTD; ++jj) ss = fmaf(v[jj], v[jj], ss);
       const float nu = sqrtf(ss);
 #pragma unroll
-      for (int j = 0; j < kTD; j += 4) {
-        const float4 s4 = *reinterpret_cast<const float4 *>(sgn + j);
-        v[j] *= s4.x; v[j + 1] *= s4.y; v[j + 2] *= s4.z; v[j + 3] *= s4.w;
+      for (int jj = 0; jj < kTD; jj += 4) {
+        const float4 s4 = *reinterpret_cast<const float4 *>(sgn + jj);
+        v[jj] *= s4.x; v[jj + 1] *= s4.y; v[jj + 2] *= s4.z; v[jj + 3] *= s4.w;
       }
       fwht128(v);
       const float scl = nu > 0.f ? nu * sqrtd : 1.f;
       const float inv = nu > 0.f ? 1.f / scl : 0.f;
       float T[L - 1];
 #pragma unroll
-      for (int k = 0; k < L - 1; ++k) T[k] = thr[k] * scl;
+      for (int k = 0; k < L - 1; ++k) T[k] = c.thresholds[k] * scl;
       uint32_t w[BITS][kTD / 32];
 #pragma unroll
       for (int P = 0; P < BITS; ++P)
@@ -468,14 +501,14 @@ encode_tcq_kernel(TqConsts c, TprArgs a) {
         for (int q = 0; q < kTD / 32; ++q) w[P][q] = 0u;
       float rr = 0.f;
 #pragma unroll
-      for (int j = 0; j < kTD; ++j) {
+      for (int jj = 0; jj < kTD; ++jj) {
         int code = 0;
 #pragma unroll
-        for (int k = 0; k < L - 1; ++k) code += v[j] >= T[k] ? 1 : 0;
+        for (int k = 0; k < L - 1; ++k) code += v[jj] >= T[k] ? 1 : 0;
 #pragma unroll
-        for (int P = 0; P < BITS; ++P) w[P][j >> 5] |= (uint32_t)((code >> P) & 1) << (j & 31);
-        const float r = fmaf(v[j], inv, -cen[code]);
-        v[j] = r;
+        for (int P = 0; P < BITS; ++P) w[P][jj >> 5] |= (uint32_t)((code >> P) & 1) << (jj & 31);
+        const float r = fmaf(v[jj], inv, -cen[code]);
+        v[jj] = r;
         rr = fmaf(r, r, rr);
       }
       if (store) {
@@ -485,41 +518,47 @@ encode_tcq_kernel(TqConsts c, TprArgs a) {
         a.norm[slot] = nu;
         a.rnorm[slot] = sqrtf(rr);
       }
-      // tile i - 1's z is ready (and the residual columns free) once its MMAs completed
-      bool ok = true;
-      if (i > 0) ok = qwait(zfull, (unsigned)((i - 1) & 1), abort_flag);
+      // r_hi -> tensor memory, then the first two products may start
+#pragma unroll
+      for (int cb = 0; cb < kTD / 16; ++cb) {
+        uint32_t hv[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          hv[e] = to_tf32(v[16 * cb + e]);
+          v[16 * cb + e] -= __uint_as_float(hv[e]);  // r_lo from here on (exact in fp32)
+        }
+        tmem_st16(rbase + 16u * cb, hv);
+      }
+      asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive1(&b[0]);
+      // r_lo into the same columns once those products have read r_hi
+      ok = qwait(&b[2], (unsigned)(j & 1), abort_flag);
       if (!__all_sync(TQ_FULL_MASK, ok)) {
         if (lane == 0) *abort_flag = 1;
         break;
       }
       tc_fence_after();
-      // residual -> tensor memory: r_hi (columns 0-127), r_lo (128-255)
 #pragma unroll
-      for (int cb = 0; cb < kTD / 32; ++cb) {
-        uint32_t hv[32], lv[32];
+      for (int cb = 0; cb < kTD / 16; ++cb) {
+        uint32_t lv[16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float r = v[32 * cb + e];
-          hv[e] = to_tf32(r);
-          lv[e] = __float_as_uint(r - __uint_as_float(hv[e]));
-        }
-        tmem_st32(lane_base + 32u * cb, hv);
-        tmem_st32(lane_base + 128u + 32u * cb, lv);
+        for (int e = 0; e < 16; ++e) lv[e] = __float_as_uint(v[16 * cb + e]);
+        tmem_st16(rbase + 16u * cb, lv);
       }
-      if (i > 0) pack_signs_from_z(lane_base + 256u, c, a, prev_slot);
       asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive1(rfull);
+      if (lane == 0) mbar_arrive1(&b[1]);
       prev_slot = store ? slot : -1;
-      buf ^= 1;
     }
-    // the last tile's signs
-    if (mytiles > 0 && !*abort_flag) {
-      const bool ok = qwait(zfull, (unsigned)((mytiles - 1) & 1), abort_flag);
+    // the group's last tile's signs
+    if (j > 0 && !*abort_flag) {
+      ok = qwait(&b[3], (unsigned)((j - 1) & 1), abort_flag);
       if (__all_sync(TQ_FULL_MASK, ok)) {
         tc_fence_after();
-        pack_signs_from_z(lane_base + 256u, c, a, prev_slot);
+        pack_signs_from_z(zbase, c, a, prev_slot);
       } else if (lane == 0) {
         *abort_flag = 1;
       }
@@ -529,7 +568,7 @@ encode_tcq_kernel(TqConsts c, TprArgs a) {
   tc_fence_before();
   __syncthreads();
   if (*abort_flag && tid == 0) atomicOr(&g_tq_device_flags, kFlagStagingTimeout);
-  if (warp == 4) {
+  if (warp == kQMmaWarp) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(512) : "memory");
   }
@@ -544,9 +583,9 @@ cudaError_t launch_tcq_t(const TqConsts &c, const TprArgs &a, cudaStream_t st) {
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t ntiles = (a.n + kTRows - 1) / kTRows;
   const int64_t grid = ntiles < (int64_t)sms ? ntiles : (int64_t)sms;
-  tq_prof_begin(TQK_ROTATE_ENCODE, st);
+  tq_prof_begin(TQK_ENCODE_QJL_TC, st);
   encode_tcq_kernel<DT, BITS><<<(unsigned)grid, kQThreads, smem, st>>>(c, a);
-  tq_prof_end(TQK_ROTATE_ENCODE, st);
+  tq_prof_end(TQK_ENCODE_QJL_TC, st);
   return cudaGetLastError();
 }
 

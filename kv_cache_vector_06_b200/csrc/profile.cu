@@ -13,7 +13,7 @@ namespace {
 
 const char *kNames[TQK_COUNT] = {"rotate_encode", "qjl_project", "rotate_query", "query_project", "scores",
                                  "attend_split", "attend_combine", "search_scan", "search_merge",
-                                 "attend_frag", "decode_prep"};
+                                 "attend_frag", "decode_prep", "encode_rows", "encode_qjl_tc"};
 
 struct Pending {
   int kind;

@@ -31,6 +31,8 @@ struct TqConsts {
   const float *S;      // device [m][d] row-major (JL matrix)
   int srht;               // S = P H D2 (structured QJL): encode transforms the residual instead
   const float *qjl_signs; // device [d], +-1.0f (D2), srht only
+  int polar;              // PolarQuant first stage (angle codes in place of coordinate codes)
+  const float *polar_tab; // device [levels][thresholds | cos c | sin c][16], polar only
 };
 
 struct tq_ctx {
@@ -44,6 +46,7 @@ struct tq_ctx {
   float *dev_signs;  // [d]
   float *dev_S;      // [m][d]
   float *dev_qjl_signs;  // [d] (structured QJL only)
+  float *dev_polar;      // PolarQuant angle tables (polar only)
   TqConsts k;        // kernel view
 };
 
@@ -78,7 +81,8 @@ class DeviceScope {
 // ---------------------------------------------------------------- profile.cu
 enum TqKernelKind {
   TQK_ROTATE_ENCODE = 0, TQK_QJL_PROJECT, TQK_ROTATE_QUERY, TQK_QUERY_PROJECT, TQK_SCORES,
-  TQK_ATTEND_SPLIT, TQK_ATTEND_COMBINE, TQK_SEARCH_SCAN, TQK_SEARCH_MERGE, TQK_ATTEND_FRAG, TQK_DECODE_PREP, TQK_COUNT
+  TQK_ATTEND_SPLIT, TQK_ATTEND_COMBINE, TQK_SEARCH_SCAN, TQK_SEARCH_MERGE, TQK_ATTEND_FRAG, TQK_DECODE_PREP,
+  TQK_ENCODE_ROWS, TQK_ENCODE_QJL_TC, TQK_COUNT
 };
 bool tq_prof_on();  // per-kernel event profiling is enabled
 void tq_prof_begin(int kind, cudaStream_t st);
@@ -86,6 +90,8 @@ void tq_prof_end(int kind, cudaStream_t st);
 
 // ---------------------------------------------------------------- codebook.cpp
 tq_status tq_codebook_fp64(int d, int bits, double *centroids, double *thresholds, double *mse);
+// PolarQuant angle codebook of one level (level 1 uniform on (-pi, pi], levels >= 2 Lloyd-Max).
+tq_status tq_polar_codebook_fp64(int level, int bits, double *centroids, double *thresholds);
 
 // ---------------------------------------------------------------- kernels (launchers)
 // Rotate rows of x: ENCODE mode normalises, quantizes, packs codes, writes norm (and, when the
@@ -115,6 +121,15 @@ enum ProjEpilogue { PROJ_SIGNS = 0, PROJ_DENSE = 1 };
 cudaError_t launch_project(const TqConsts &c, ProjEpilogue ep, const float *R, int64_t n,
                            const int64_t *slots, int64_t capacity, uint32_t *signs, float *zout,
                            cudaStream_t st);
+
+// PolarQuant first stage at d = 128 (polar.cu): encode (codes, norm; with a QJL stage also the
+// residual rows to `resid` and rnorm, for launch_project) and estimated scores.
+bool polar_supported(const TqConsts &c);
+cudaError_t launch_encode_polar(const TqConsts &c, const void *x, tq_dtype dtype, int64_t n, int64_t ld,
+                                const int64_t *slots, int64_t capacity, uint32_t *codes, float *norm, float *rnorm,
+                                float *resid, cudaStream_t st);
+cudaError_t launch_scores_polar(const TqConsts &c, const float *qr, const float *p, int nq, const tq_packed &keys,
+                                int64_t n, float *out, cudaStream_t st);
 
 // out[i][k] = estimated score of prepared query i against slot k.
 cudaError_t launch_scores(const TqConsts &c, const float *qr, const float *p, int nq,

@@ -54,6 +54,8 @@ def _load():
         "tq_make_codebook": (st, [c_int32, c_int32, POINTER(c_double), POINTER(c_double), POINTER(c_double)]),
         "tq_ctx_create": (st, [POINTER(Spec), c_void_p, c_void_p, c_int32, POINTER(c_void_p)]),
         "tq_ctx_create_srht": (st, [POINTER(Spec), c_void_p, c_void_p, c_int32, POINTER(c_void_p)]),
+        "tq_ctx_create_polar": (st, [POINTER(Spec), c_void_p, c_void_p, c_int32, POINTER(c_void_p)]),
+        "tq_polar_codebook": (st, [c_int32, c_int32, POINTER(c_double), POINTER(c_double)]),
         "tq_ctx_destroy": (st, [c_void_p]),
         "tq_ctx_layout": (st, [c_void_p, POINTER(c_int64), POINTER(c_int64)]),
         "tq_encode_workspace_size": (st, [c_void_p, c_int64, POINTER(c_size_t)]),
@@ -126,6 +128,15 @@ def _dev(t: torch.Tensor, device: int, name: str, dtype=None, contiguous=True):
     return c_void_p(t.data_ptr())
 
 
+def make_polar_codebook(level: int, bits: int):
+    """PolarQuant angle codebook of one level, computed by the library on the host (fp64)."""
+    L = 1 << bits
+    c = (c_double * L)()
+    t = (c_double * max(L - 1, 1))()
+    _check(LIB.tq_polar_codebook(level, bits, c, t))
+    return [c[i] for i in range(L)], [t[i] for i in range(L - 1)]
+
+
 def make_codebook(d: int, bits: int):
     """Lloyd-Max codebook computed by the library on the host (fp64)."""
     L = 1 << bits
@@ -140,9 +151,10 @@ class Context:
     """Quantizer constants for one tensor role, resident on one device."""
 
     def __init__(self, d: int, mse_bits: int, qjl_m: int, rot_signs, qjl_matrix=None, device: int = 0,
-                 layout: int = LAYOUT_ROWS, qjl_signs=None):
+                 layout: int = LAYOUT_ROWS, qjl_signs=None, polar: bool = False):
         """qjl_matrix: the dense JL matrix [qjl_m, d] (tq_ctx_create); or qjl_signs: the sign
-        vector D2 [d] of the structured matrix S = P H D2 (tq_ctx_create_srht)."""
+        vector D2 [d] of the structured matrix S = P H D2 (tq_ctx_create_srht).  polar: the
+        PolarQuant first stage (tq_ctx_create_polar)."""
         rs = torch.as_tensor(rot_signs).to(torch.int8).contiguous().cpu()
         if rs.numel() != d:
             raise ValueError("rot_signs must have d entries")
@@ -164,7 +176,9 @@ class Context:
                 sptr = c_void_p(S.data_ptr())
             else:
                 sptr = c_void_p(None)
-            _check(LIB.tq_ctx_create(ctypes.byref(spec), c_void_p(rs.data_ptr()), sptr, device, ctypes.byref(h)))
+            create = LIB.tq_ctx_create_polar if polar else LIB.tq_ctx_create
+            _check(create(ctypes.byref(spec), c_void_p(rs.data_ptr()), sptr, device, ctypes.byref(h)))
+        self.polar = polar
         self._h = h
         cb, sb = c_int64(), c_int64()
         _check(LIB.tq_ctx_layout(h, ctypes.byref(cb), ctypes.byref(sb)))

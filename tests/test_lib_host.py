@@ -113,3 +113,22 @@ def test_null_arguments_rejected(lib):
     assert L.tq_scores(None, None, 0, 1, lib.PackedC(), 1, None, None, 0, None) == 1
     assert L.tq_attend_decode(None, None, None, None, 0, None, None, 0, None) == 1
     assert L.tq_search_topk(None, None, 0, 1, lib.PackedC(), 1, 1, None, None, None, 0, None) == 1
+
+
+@pytest.mark.parametrize("level", [1, 2, 3, 5, 7])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_host_polar_codebook_matches_oracle(lib, level, bits):
+    """The library's PolarQuant angle codebooks (host, fp64, Gauss-Legendre quadrature) against
+    the oracle's (adaptive quadrature)."""
+    from oracle import polar
+    c, t = lib.make_polar_codebook(level, bits)
+    co, to = polar.angle_codebook(level, bits)
+    np.testing.assert_allclose(c, co, rtol=0, atol=1e-9)
+    np.testing.assert_allclose(t, to, rtol=0, atol=1e-9)
+
+
+def test_polar_codebook_rejects_bad_sizes(lib):
+    for lv, b in [(0, 2), (11, 2), (3, 0), (3, 5)]:
+        with pytest.raises(lib.TqError) as e:
+            lib.make_polar_codebook(lv, b)
+        assert e.value.status == 2
