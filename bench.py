@@ -82,6 +82,8 @@ def parse_args(argv=None):
                     help="search: bits per coordinate, (bits-1) MSE bits + 1 QJL bit with m = d")
     ap.add_argument("--search-rows", type=int, default=1_000_000,
                     help="search: database rows (the workload is 10^6; smaller only for profiler captures)")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="ragged: number of sequences (the workload is 64; smaller only for profiler captures)")
     ap.add_argument("--sparse-v", type=float, default=0.0,
                     help="decode: Sparse V threshold on the softmax weight (0 = off)")
     a = ap.parse_args(argv)
@@ -94,6 +96,8 @@ def workload(args) -> dict:
     cfg = dict(CONFIGS[args.config])
     if args.config == "llama8b" and args.kbits is not None:
         cfg["k_bits"] = args.kbits
+    if args.config == "ragged" and args.batch is not None:
+        cfg["batch"] = args.batch
     return cfg
 
 

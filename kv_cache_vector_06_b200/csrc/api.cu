@@ -7,6 +7,7 @@
 #include <algorithm>
 #include <cstring>
 #include <new>
+#include <vector>
 
 #include "tq_internal.h"
 
@@ -145,10 +146,12 @@ static tq_status ctx_create(const tq_spec *spec, const int8_t *rot_signs, const 
     for (int j = 0; j < d; ++j) hs2[j] = (float)qjl_signs[j];
   e = cudaMalloc(&c->dev_signs, sizeof(float) * d);
   if (e == cudaSuccess && m > 0) e = cudaMalloc(&c->dev_S, sizeof(float) * (size_t)m * d);
+  if (e == cudaSuccess && m > 0) e = cudaMalloc(&c->dev_St, sizeof(float) * (size_t)m * d);
   if (e == cudaSuccess && qjl_signs) e = cudaMalloc(&c->dev_qjl_signs, sizeof(float) * d);
   if (e != cudaSuccess) {
     cudaFree(c->dev_signs);
     cudaFree(c->dev_S);
+    cudaFree(c->dev_St);
     delete c;
     cudaGetLastError();
     return tq_fail(TQ_ENOMEM, "cudaMalloc of context constants failed");
@@ -156,6 +159,12 @@ static tq_status ctx_create(const tq_spec *spec, const int8_t *rot_signs, const 
   e = cudaMemcpy(c->dev_signs, hs, sizeof(float) * d, cudaMemcpyHostToDevice);
   if (e == cudaSuccess && m > 0)
     e = cudaMemcpy(c->dev_S, qjl_matrix, sizeof(float) * (size_t)m * d, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && m > 0) {
+    std::vector<float> st((size_t)m * d);
+    for (int i = 0; i < m; ++i)
+      for (int j = 0; j < d; ++j) st[(size_t)j * m + i] = qjl_matrix[(size_t)i * d + j];
+    e = cudaMemcpy(c->dev_St, st.data(), sizeof(float) * (size_t)m * d, cudaMemcpyHostToDevice);
+  }
   if (e == cudaSuccess && qjl_signs)
     e = cudaMemcpy(c->dev_qjl_signs, hs2, sizeof(float) * d, cudaMemcpyHostToDevice);
   if (e == cudaSuccess && polar) {
@@ -177,6 +186,7 @@ static tq_status ctx_create(const tq_spec *spec, const int8_t *rot_signs, const 
   if (e != cudaSuccess) {
     cudaFree(c->dev_signs);
     cudaFree(c->dev_S);
+    cudaFree(c->dev_St);
     cudaFree(c->dev_qjl_signs);
     cudaFree(c->dev_polar);
     delete c;
@@ -198,6 +208,7 @@ static tq_status ctx_create(const tq_spec *spec, const int8_t *rot_signs, const 
   }
   k.signs = c->dev_signs;
   k.S = c->dev_S;
+  k.St = c->dev_St;
   k.srht = qjl_signs ? 1 : 0;
   k.qjl_signs = c->dev_qjl_signs;
   k.polar = polar ? 1 : 0;
@@ -296,6 +307,7 @@ tq_status tq_ctx_destroy(tq_ctx *ctx) {
   cudaSetDevice(ctx->device);
   cudaFree(ctx->dev_signs);
   cudaFree(ctx->dev_S);
+  cudaFree(ctx->dev_St);
   cudaFree(ctx->dev_qjl_signs);
   cudaFree(ctx->dev_polar);
   if (cur >= 0) cudaSetDevice(cur);

@@ -121,8 +121,9 @@ __device__ __forceinline__ void kfrag_group(const TqConsts &kc, const void *__re
   __shared__ int fexp[kG][2];
   // grp = b * hkv + h; its query heads are rows grp * 4 + g
   const int tid = threadIdx.x;
-  // S (for p = S q') is copied asynchronously while q' is formed
-  if constexpr (QJL) stage_rows_padded_async(sS, kc.S, kD, kD);
+  // S (for p = S q') is copied asynchronously while q' is formed (sS null: read from global)
+  if constexpr (QJL)
+    if (sS) stage_rows_padded_async(sS, kc.S, kD, kD);
   // q' = (1/sqrt d) H (D q): load with the signs applied, then the butterflies in shared memory
   for (int i = tid; i < kG * kD; i += kThreads) {
     const int g = i / kD, j = i % kD;
@@ -153,22 +154,32 @@ __device__ __forceinline__ void kfrag_group(const TqConsts &kc, const void *__re
   if constexpr (QJL) {
     // p = S q' for the 4 heads: S staged in shared memory (row stride kD + 4), thread (row i,
     // head pair) dots row i with two q'
-    stage_async_wait();
+    if (sS) stage_async_wait();
     __syncthreads();
     const int i = tid & (kD - 1), gp = tid >> 7;
-    const float4 *Srow = reinterpret_cast<const float4 *>(sS + i * (kD + 4));
     float p0 = 0.f, p1 = 0.f;
+    if (sS) {
+      const float4 *Srow = reinterpret_cast<const float4 *>(sS + i * (kD + 4));
 #pragma unroll 8
-    for (int j4 = 0; j4 < kD / 4; ++j4) {
-      const float4 sv = Srow[j4];
-      p0 = fmaf(sv.x, qs[2 * gp][4 * j4], p0);
-      p0 = fmaf(sv.y, qs[2 * gp][4 * j4 + 1], p0);
-      p0 = fmaf(sv.z, qs[2 * gp][4 * j4 + 2], p0);
-      p0 = fmaf(sv.w, qs[2 * gp][4 * j4 + 3], p0);
-      p1 = fmaf(sv.x, qs[2 * gp + 1][4 * j4], p1);
-      p1 = fmaf(sv.y, qs[2 * gp + 1][4 * j4 + 1], p1);
-      p1 = fmaf(sv.z, qs[2 * gp + 1][4 * j4 + 2], p1);
-      p1 = fmaf(sv.w, qs[2 * gp + 1][4 * j4 + 3], p1);
+      for (int j4 = 0; j4 < kD / 4; ++j4) {
+        const float4 sv = Srow[j4];
+        p0 = fmaf(sv.x, qs[2 * gp][4 * j4], p0);
+        p0 = fmaf(sv.y, qs[2 * gp][4 * j4 + 1], p0);
+        p0 = fmaf(sv.z, qs[2 * gp][4 * j4 + 2], p0);
+        p0 = fmaf(sv.w, qs[2 * gp][4 * j4 + 3], p0);
+        p1 = fmaf(sv.x, qs[2 * gp + 1][4 * j4], p1);
+        p1 = fmaf(sv.y, qs[2 * gp + 1][4 * j4 + 1], p1);
+        p1 = fmaf(sv.z, qs[2 * gp + 1][4 * j4 + 2], p1);
+        p1 = fmaf(sv.w, qs[2 * gp + 1][4 * j4 + 3], p1);
+      }
+    } else {
+      // S transposed in global memory: consecutive rows i per warp, coalesced (same order of sums)
+#pragma unroll 32
+      for (int j = 0; j < kD; ++j) {
+        const float sv = kc.St[j * kc.m + i];
+        p0 = fmaf(sv, qs[2 * gp][j], p0);
+        p1 = fmaf(sv, qs[2 * gp + 1][j], p1);
+      }
     }
     X[KP::code][2 * gp][i] = 2.f * p0;
     X[KP::code][2 * gp + 1][i] = 2.f * p1;
@@ -240,7 +251,8 @@ __device__ __forceinline__ void kfrag_head(const TqConsts &kc, const void *__res
   __shared__ float red[4];
   __shared__ int fexp[2];
   const int tid = threadIdx.x;
-  if constexpr (QJL) stage_rows_padded_async(sS, kc.S, kD, kD);
+  if constexpr (QJL)
+    if (sS) stage_rows_padded_async(sS, kc.S, kD, kD);
   for (int j = tid; j < kD; j += kThreads) {
     const int64_t o = ((int64_t)grp * kG + g) * kD + j;
     const float x = dtype == TQ_F32 ? static_cast<const float *>(q)[o]
@@ -268,18 +280,23 @@ __device__ __forceinline__ void kfrag_head(const TqConsts &kc, const void *__res
   }
   __syncthreads();
   if constexpr (QJL) {
-    stage_async_wait();
+    if (sS) stage_async_wait();
     __syncthreads();
     if (tid < kD) {
-      const float4 *Srow = reinterpret_cast<const float4 *>(sS + tid * (kD + 4));
       float p0 = 0.f;
+      if (sS) {
+        const float4 *Srow = reinterpret_cast<const float4 *>(sS + tid * (kD + 4));
 #pragma unroll 8
-      for (int j4 = 0; j4 < kD / 4; ++j4) {
-        const float4 sv = Srow[j4];
-        p0 = fmaf(sv.x, qs[4 * j4], p0);
-        p0 = fmaf(sv.y, qs[4 * j4 + 1], p0);
-        p0 = fmaf(sv.z, qs[4 * j4 + 2], p0);
-        p0 = fmaf(sv.w, qs[4 * j4 + 3], p0);
+        for (int j4 = 0; j4 < kD / 4; ++j4) {
+          const float4 sv = Srow[j4];
+          p0 = fmaf(sv.x, qs[4 * j4], p0);
+          p0 = fmaf(sv.y, qs[4 * j4 + 1], p0);
+          p0 = fmaf(sv.z, qs[4 * j4 + 2], p0);
+          p0 = fmaf(sv.w, qs[4 * j4 + 3], p0);
+        }
+      } else {
+#pragma unroll 32
+        for (int j = 0; j < kD; ++j) p0 = fmaf(kc.St[j * kc.m + tid], qs[j], p0);
       }
       X[KP::code][tid] = 2.f * p0;
     }
@@ -344,27 +361,33 @@ kfrag_kernel(TqConsts kc, const void *__restrict__ q, int dtype, uint32_t *__res
 // One launch for the work that precedes the split kernel in a decode step: blocks
 // [0, nkb) append-encode the new keys (one per block with QJL, whose projection four warps share;
 // else 8 per block), blocks [nkb, nkb + nvb) the new values (8 per block), and the remaining
-// blocks build one query head's fragments each.  The jobs are independent, so their latencies
-// overlap instead of adding up.
+// blocks build the query fragments: one query head each (`per_head`, for small batches, so that
+// more blocks share the latency) or one (sequence, KV head) group each.  The jobs are
+// independent, so their latencies overlap instead of adding up.  Small launches stage S in each
+// block's shared memory; large ones read its transposed copy from global memory (coalesced; it
+// stays in L1 and L2), so that many blocks fit on an SM.
 template <int BK, bool QJL>
 __global__ void __launch_bounds__(kThreads)
 decode_prep_kernel(TqConsts kc, TqConsts vc, const void *__restrict__ knew, const void *__restrict__ vnew,
                    int kvdtype, int64_t nnew, const int64_t *__restrict__ slots, tq_packed kp, tq_packed vp,
                    const void *__restrict__ q, int qdtype, uint32_t *__restrict__ kfrag,
-                   float *__restrict__ kconst, int *__restrict__ counter, int nkb, int nvb) {
-  extern __shared__ __align__(16) float sS[];
+                   float *__restrict__ kconst, int *__restrict__ counter, int nkb, int nvb, int per_head) {
+  extern __shared__ __align__(16) float sS[];  // S staged per block for small launches (per_head)
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");  // the attention grid may start
+  float *ss = per_head ? sS : nullptr;
   const int bid = blockIdx.x;
   if (bid < nkb) {
     // keys: with QJL one row per block (warps 0-3 share its projection), else 8 rows per block
     rotate_rows<kD>(kc, ROT_ENCODE, knew, kvdtype, nnew, kD, slots, kp.capacity, static_cast<uint32_t *>(kp.codes),
-                    kp.norm, kp.rnorm, nullptr, QJL ? static_cast<uint32_t *>(kp.signs) : nullptr, bid, sS, QJL);
+                    kp.norm, kp.rnorm, nullptr, QJL ? static_cast<uint32_t *>(kp.signs) : nullptr, bid, ss, QJL);
   } else if (bid < nkb + nvb) {
     rotate_rows<kD>(vc, ROT_ENCODE, vnew, kvdtype, nnew, kD, slots, vp.capacity, static_cast<uint32_t *>(vp.codes),
-                    vp.norm, nullptr, nullptr, nullptr, bid - nkb, sS);
-  } else {
+                    vp.norm, nullptr, nullptr, nullptr, bid - nkb, ss);
+  } else if (per_head) {
     const int qh = bid - nkb - nvb;  // query head: group qh / 4, head qh % 4
-    kfrag_head<BK, QJL>(kc, q, qdtype, kfrag, kconst, counter, qh / kG, qh % kG, sS);
+    kfrag_head<BK, QJL>(kc, q, qdtype, kfrag, kconst, counter, qh / kG, qh % kG, ss);
+  } else {
+    kfrag_group<BK, QJL>(kc, q, qdtype, kfrag, kconst, counter, bid - nkb - nvb, nullptr);
   }
 }
 
@@ -1182,16 +1205,20 @@ cudaError_t launch_step(const TqConsts &kc, const TqConsts &vc, const MmaArgs &a
                         uint32_t *kfrag, float *kconst, float *part, cudaStream_t st) {
   const int nvb = (int)((nnew + (kThreads / 32) - 1) / (kThreads / 32));  // one value row per warp
   const int nkb = QJL ? (int)nnew : nvb;                                       // keys: see decode_prep_kernel
-  const unsigned grid0 = (unsigned)(nkb + nvb + batch * a.hq);
-  const size_t fsm = QJL ? sizeof(float) * kD * (kD + 4) : 0;
+  // one block per query head while that keeps the launch under one block per SM, else per group
+  const int groups = batch * a.hkv;
+  const int per_head = batch * a.hq <= tq_sm_count() ? 1 : 0;
+  const unsigned grid0 = (unsigned)(nkb + nvb + (per_head ? batch * a.hq : groups));
+  // small launches stage S in each block's shared memory (all of it requested at once); large
+  // ones read its transposed copy from L1 / L2 so that many blocks fit on an SM
+  const size_t fsm = (QJL && per_head) ? sizeof(float) * kD * (kD + 4) : 0;
   if (fsm) {
-    cudaError_t e0 = tq_smem_limit(reinterpret_cast<const void *>(decode_prep_kernel<BK, QJL>),
-                                          (int)fsm);
+    cudaError_t e0 = tq_smem_limit(reinterpret_cast<const void *>(decode_prep_kernel<BK, QJL>), (int)fsm);
     if (e0 != cudaSuccess) return e0;
   }
   tq_prof_begin(TQK_DECODE_PREP, st);
   decode_prep_kernel<BK, QJL><<<grid0, kThreads, fsm, st>>>(kc, vc, knew, vnew, kvdtype, nnew, slots, a.k, a.v, q,
-                                                            qdtype, kfrag, kconst, a.counter, nkb, nvb);
+                                                            qdtype, kfrag, kconst, a.counter, nkb, nvb, per_head);
   tq_prof_end(TQK_DECODE_PREP, st);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -78,6 +78,83 @@ __device__ __forceinline__ void tpr_load(const unsigned char *rowp, float (&v)[k
   }
 }
 
+// Codes by the codebook's symmetry.  The thresholds are antisymmetric (t_(L-2-k) = -t_k, the middle
+// one 0), so with the H = L/2 - 1 positive ones t+_k:
+//   code = L/2 + #{k : |y| >= t+_k}        for y >= 0,
+//   code = L/2 - 1 - #{k : |y| > t+_k}     for y < 0,
+// the same count as #{i : t_i <= y} (ties go up).  The strict comparison of a negative y is the
+// non-strict one on the float just below |y|.  Each comparison sets bit j of a word of its own (a
+// thermometer code), and the bit planes of the code are XORs of those words: half the
+// comparisons of the plain count and no per-coordinate bit extraction.
+template <int BITS>
+struct Sym {
+  static constexpr int H = (1 << (BITS - 1)) - 1;
+  static constexpr int HW = H > 0 ? H : 1;
+};
+
+// One coordinate j (of the NW 32-bit words a thread packs): sets bit j of the sign word and of the
+// thermometer words; returns the code.
+template <int BITS, int NW>
+__device__ __forceinline__ int sym_quant(float y, const float (&Tp)[Sym<BITS>::HW], uint32_t (&sw)[NW],
+                                         uint32_t (&tw)[Sym<BITS>::HW][NW], int j) {
+  constexpr int L = 1 << BITS;
+  const bool pos = y >= 0.f;
+  const uint32_t bit = 1u << (j & 31);
+  if (pos) sw[j >> 5] |= bit;
+  const float a = __uint_as_float((__float_as_uint(y) & 0x7fffffffu) - (pos ? 0u : 1u));
+  int cnt = 0;
+#pragma unroll
+  for (int k = 0; k < Sym<BITS>::H; ++k) {
+    const bool ge = a >= Tp[k];
+    if (ge) tw[k][j >> 5] |= bit;
+    cnt += ge ? 1 : 0;
+  }
+  return pos ? L / 2 + cnt : L / 2 - 1 - cnt;
+}
+
+// The code's bit planes from the sign word s and the thermometer words: plane BITS - 1 is s; the
+// lower planes are the bits of the count, complemented where y < 0.
+template <int BITS, int NW>
+__device__ __forceinline__ void sym_planes(const uint32_t (&sw)[NW], const uint32_t (&tw)[Sym<BITS>::HW][NW],
+                                           uint32_t (&w)[BITS][NW]) {
+#pragma unroll
+  for (int q = 0; q < NW; ++q) {
+    const uint32_t n = ~sw[q];
+    w[BITS - 1][q] = sw[q];
+    if constexpr (BITS == 2) w[0][q] = tw[0][q] ^ n;
+    if constexpr (BITS == 3) {
+      w[1][q] = tw[1][q] ^ n;
+      w[0][q] = tw[0][q] ^ tw[1][q] ^ tw[2][q] ^ n;
+    }
+    if constexpr (BITS == 4) {
+      w[2][q] = tw[3][q] ^ n;
+      w[1][q] = tw[1][q] ^ tw[3][q] ^ tw[5][q] ^ n;
+      w[0][q] = tw[0][q] ^ tw[1][q] ^ tw[2][q] ^ tw[3][q] ^ tw[4][q] ^ tw[5][q] ^ tw[6][q] ^ n;
+    }
+  }
+}
+
+// 32 x 32 bit transpose across a warp: lane i holds row i (bit j = element (i, j)) and gets back
+// column `lane` (bit i = element (i, lane)).  Five exchange stages with the partner lane at
+// distance 16, 8, 4, 2, 1: the halves and bytes move by byte permutes, the nibbles, pairs and
+// single bits by a rotate of the partner's word and a bit select.
+__device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, int lane) {
+  uint32_t y = __shfl_xor_sync(TQ_FULL_MASK, x, 16);
+  x = __byte_perm(x, y, (lane & 16) ? 0x3276 : 0x5410);
+  y = __shfl_xor_sync(TQ_FULL_MASK, x, 8);
+  x = __byte_perm(x, y, (lane & 8) ? 0x3715 : 0x6240);
+#pragma unroll
+  for (int s = 4; s >= 1; s >>= 1) {
+    const uint32_t m = s == 4 ? 0x0F0F0F0Fu : (s == 2 ? 0x33333333u : 0x55555555u);
+    y = __shfl_xor_sync(TQ_FULL_MASK, x, s);
+    const bool hi = (lane & s) != 0;
+    const uint32_t keep = hi ? ~m : m;
+    const uint32_t r = __funnelshift_r(y, y, hi ? s : 32 - s);
+    x = (x & keep) | (r & ~keep);
+  }
+  return x;
+}
+
 struct TprArgs {
   const char *x;
   int64_t ld_bytes;
@@ -88,6 +165,42 @@ struct TprArgs {
   float *norm, *rnorm;
   uint32_t *signs;       // structured QJL only
 };
+
+// Token-block layout: the 32 rows of a warp, rows [wrow0, wrow0 + 32), are two 16-slot blocks
+// (slot = row).  A bit transpose of each plane word gives lane j coordinate 32 g + j of all 32
+// rows, i.e. its word of both blocks.  Only whole blocks are written (the caller passes a
+// multiple of 16 rows).  Called by all lanes of the warp.
+template <int BITS>
+__device__ __forceinline__ void store_blk16(const TqConsts &c, const TprArgs &a, const uint32_t (&w)[BITS][kTD / 32],
+                                            int64_t wrow0, int lane) {
+  if (wrow0 >= a.n) return;  // uniform over the warp
+  const bool twoblk = wrow0 + 16 < a.n;
+  uint32_t *blkA = a.codes + (wrow0 >> 4) * (int64_t)(16 * c.code_words);
+  uint32_t *blkB = blkA + 16 * c.code_words;
+#pragma unroll
+  for (int q2 = 0; q2 < BITS / 2; ++q2)
+#pragma unroll
+    for (int g = 0; g < kTD / 32; ++g) {
+      const uint32_t lo = warp_transpose32(w[2 * q2][g], lane), hi = warp_transpose32(w[2 * q2 + 1][g], lane);
+      blkA[q2 * kTD + 32 * g + lane] = __byte_perm(lo, hi, 0x5410);
+      if (twoblk) blkB[q2 * kTD + 32 * g + lane] = __byte_perm(lo, hi, 0x7632);
+    }
+  if constexpr (BITS & 1) {
+    // the odd last plane packs coordinates 2 j' (bits 0-15) and 2 j' + 1 (bits 16-31): lane j'
+    // takes them from the transposed words of coordinates 64 g .. 64 g + 63
+#pragma unroll
+    for (int g = 0; g < kTD / 64; ++g) {
+      const uint32_t ta = warp_transpose32(w[BITS - 1][2 * g], lane);
+      const uint32_t tb = warp_transpose32(w[BITS - 1][2 * g + 1], lane);
+      const int se = (2 * lane) & 31;
+      const uint32_t ea = __shfl_sync(TQ_FULL_MASK, ta, se), eb = __shfl_sync(TQ_FULL_MASK, tb, se);
+      const uint32_t oa = __shfl_sync(TQ_FULL_MASK, ta, se + 1), ob = __shfl_sync(TQ_FULL_MASK, tb, se + 1);
+      const uint32_t ev = lane < 16 ? ea : eb, od = lane < 16 ? oa : ob;
+      blkA[(BITS / 2) * kTD + 32 * g + lane] = __byte_perm(ev, od, 0x5410);
+      if (twoblk) blkB[(BITS / 2) * kTD + 32 * g + lane] = __byte_perm(ev, od, 0x7632);
+    }
+  }
+}
 
 // One thread per row.  BITS: MSE bits; BLK: token-block layout (full blocks, slot = row);
 // SRHT: structured QJL signs of the residual.
@@ -104,9 +217,11 @@ encode_tpr_kernel(TqConsts c, TprArgs a) {
   }
   if (tid < TQ_MAX_LEVELS) cen[tid] = c.centroids[tid];
   constexpr int L = 1 << BITS;
-  float thr[L - 1];
+  // the positive thresholds (codes by symmetry), or all of them where the residual is formed
+  constexpr int NT = SRHT ? L - 1 : Sym<BITS>::HW;
+  float thr[NT];
 #pragma unroll
-  for (int i = 0; i < L - 1; ++i) thr[i] = c.thresholds[i];
+  for (int i = 0; i < (SRHT ? L - 1 : Sym<BITS>::H); ++i) thr[i] = c.thresholds[SRHT ? i : L / 2 + i];
   const float sqrtd = 1.f / c.inv_sqrt_d;
   const int64_t ntiles = (a.n + kTRows - 1) / kTRows;
   int64_t tile = blockIdx.x;
@@ -139,76 +254,43 @@ encode_tpr_kernel(TqConsts c, TprArgs a) {
     // codes against the scaled thresholds, bit-planes packed in registers, residual
     const float scl = nu > 0.f ? nu * sqrtd : 1.f;
     const float inv = nu > 0.f ? 1.f / scl : 0.f;
-    float T[L - 1];
+    float T[NT];
 #pragma unroll
-    for (int i = 0; i < L - 1; ++i) T[i] = thr[i] * scl;
+    for (int i = 0; i < (SRHT ? L - 1 : Sym<BITS>::H); ++i) T[i] = thr[i] * scl;
     uint32_t w[BITS][kTD / 32];
-#pragma unroll
-    for (int P = 0; P < BITS; ++P)
-#pragma unroll
-      for (int q = 0; q < kTD / 32; ++q) w[P][q] = 0u;
     float rr = 0.f;
+    if constexpr (SRHT) {
+      // the plain count, whose code feeds the residual (fewer live registers than the
+      // thermometer words here)
 #pragma unroll
-    for (int j = 0; j < kTD; ++j) {
-      int code = 0;
+      for (int P = 0; P < BITS; ++P)
 #pragma unroll
-      for (int i = 0; i < L - 1; ++i) code += v[j] >= T[i] ? 1 : 0;
+        for (int q = 0; q < kTD / 32; ++q) w[P][q] = 0u;
 #pragma unroll
-      for (int P = 0; P < BITS; ++P) w[P][j >> 5] |= (uint32_t)((code >> P) & 1) << (j & 31);
-      if constexpr (SRHT) {
+      for (int j = 0; j < kTD; ++j) {
+        int code = 0;
+#pragma unroll
+        for (int i = 0; i < L - 1; ++i) code += v[j] >= T[i] ? 1 : 0;
+#pragma unroll
+        for (int P = 0; P < BITS; ++P) w[P][j >> 5] |= (uint32_t)((code >> P) & 1) << (j & 31);
         const float r = fmaf(v[j], inv, -cen[code]);  // residual, rotated domain
         v[j] = r;
         rr = fmaf(r, r, rr);
       }
+    } else {
+      uint32_t sw[kTD / 32], tw[Sym<BITS>::HW][kTD / 32];
+#pragma unroll
+      for (int q = 0; q < kTD / 32; ++q) {
+        sw[q] = 0u;
+#pragma unroll
+        for (int k = 0; k < Sym<BITS>::HW; ++k) tw[k][q] = 0u;
+      }
+#pragma unroll
+      for (int j = 0; j < kTD; ++j) sym_quant<BITS, kTD / 32>(v[j], T, sw, tw, j);
+      sym_planes<BITS, kTD / 32>(sw, tw, w);
     }
     if constexpr (BLK) {
-      // two whole blocks per warp (slot = row); block words assembled with ballots, lane q of a
-      // 32-word group keeps word q
-      const int64_t wrow0 = tile * kTRows + 32 * warp;
-      if (wrow0 < a.n) {  // the caller passes a multiple of 32 rows... or of 16: guard each block
-        const bool twoblk = wrow0 + 16 < a.n;
-        uint32_t *blkA = a.codes + (wrow0 >> 4) * (int64_t)(16 * c.code_words);
-        uint32_t *blkB = blkA + 16 * c.code_words;
-#pragma unroll
-        for (int q2 = 0; q2 < BITS / 2; ++q2)
-#pragma unroll
-          for (int g = 0; g < kTD / 32; ++g) {
-            uint32_t kA = 0u, kB = 0u;
-#pragma unroll 4
-            for (int jj = 0; jj < 32; ++jj) {
-              const unsigned lo = __ballot_sync(TQ_FULL_MASK, (w[2 * q2][g] >> jj) & 1u);
-              const unsigned hi = __ballot_sync(TQ_FULL_MASK, (w[2 * q2 + 1][g] >> jj) & 1u);
-              if (lane == jj) {
-                kA = (lo & 0xFFFFu) | (hi << 16);
-                kB = (lo >> 16) | (hi & 0xFFFF0000u);
-              }
-            }
-            blkA[q2 * kTD + 32 * g + lane] = kA;
-            if (twoblk) blkB[q2 * kTD + 32 * g + lane] = kB;
-          }
-        if constexpr (BITS & 1) {
-          // the odd last plane packs coordinates 2 j' (bits 0-15) and 2 j' + 1 (bits 16-31)
-#pragma unroll
-          for (int g = 0; g < kTD / 64; ++g) {
-            uint32_t kA = 0u, kB = 0u;
-            const uint32_t we = w[BITS - 1][2 * g], wo = w[BITS - 1][2 * g + 1];
-#pragma unroll 4
-            for (int jj = 0; jj < 32; ++jj) {
-              // coordinates 64 g + 2 jj and 64 g + 2 jj + 1: bits 2 jj, 2 jj + 1 of word 2 g (jj < 16) or 2 g + 1
-              const uint32_t wd = jj < 16 ? we : wo;
-              const int sh = (2 * jj) & 31;
-              const unsigned ev = __ballot_sync(TQ_FULL_MASK, (wd >> sh) & 1u);
-              const unsigned od = __ballot_sync(TQ_FULL_MASK, (wd >> (sh + 1)) & 1u);
-              if (lane == jj) {
-                kA = (ev & 0xFFFFu) | (od << 16);
-                kB = (ev >> 16) | (od & 0xFFFF0000u);
-              }
-            }
-            blkA[(BITS / 2) * kTD + 32 * g + lane] = kA;
-            if (twoblk) blkB[(BITS / 2) * kTD + 32 * g + lane] = kB;
-          }
-        }
-      }
+      store_blk16<BITS>(c, a, w, tile * kTRows + 32 * warp, lane);
       if (valid) a.norm[row] = nu;
     } else {
       const int64_t slot = valid ? (a.slots ? a.slots[row] : row) : -1;
@@ -276,11 +358,113 @@ cudaError_t launch_tpr_dt(const TqConsts &c, const TprArgs &a, cudaStream_t st) 
 }
 
 
-// A thread's row of z (tensor memory, 128 fp32 columns from `zaddr`): sign bits of its slot.
-__device__ __forceinline__ void pack_signs_from_z(uint32_t zaddr, const TqConsts &c, const TprArgs &a, int64_t slot) {
-  uint32_t sb[kTD / 32];
+// ------------------------------------------------------------------ bf16 rows on tcgen05
+// bf16 rows: the rotation runs on the tensor cores.  With B[n][k] = (-1)^popcount(n & k) D_k
+// (entries +-1, exact in bf16), y = H (D x) = X B^T is one 128 x 128 x 128 bf16 MMA with fp32
+// accumulation per tile of 128 rows: the sums the butterflies form, added in another order.  The
+// norm follows from ||y|| = sqrt(d) ||x||, and the thresholds are scaled by ||y||.
+//
+// Keys with a dense Gaussian JL matrix (m = d = 128) then form z = S r on the tensor cores as three
+// TF32 products (r_hi S_hi + r_hi S_lo + r_lo S_hi, each operand split as x = tf32(x) +
+// (x - tf32(x)); the dropped r_lo S_lo term is below 2^-22 of the products), which keeps z within
+// a few fp32 ulps of the fp32 dot product:
+//   A = the tile's residual rows, written by their own threads into tensor memory (lane = row,
+//       one column per coordinate): r_hi for the first two products, then r_lo in the same
+//       columns for the third;
+//   B = S_hi, S_lo in shared memory (canonical K-major layout, staged once per CTA);
+//   D = z in tensor memory, read back by the row's thread for its sign bits.
+//
+// Two groups of eight compute warps take alternate tiles, each with its own staging buffer and
+// tensor-memory columns (y, later the residual; with QJL also z).  Warps w and w + 4 of a group
+// see the same 32 tensor-memory lanes (rows), so each row is shared by two threads: one per half
+// of the 128 columns (half the registers of a whole row, twice the warps).  The two halves of a
+// row's sums of squares are added through shared memory in a fixed order.  Warp 16 issues the
+// MMAs (one thread) and owns the allocation.  The MMA thread issues a tile's rotation before the
+// other group's products, so that one group's rotation is not queued behind them, and a group
+// packs its previous tile's signs before it encodes its next tile.
+// The staged tile: bf16 (r, k) at (k / 8) 2048 + 16 r + 2 (k % 8), i.e. each K chunk of 8
+// elements holds all 128 rows contiguously (core matrices of 8 rows x 16 bytes).
+constexpr int kQGroups = 2;
+constexpr int kQWarps = 8;                                 // compute warps per group
+constexpr int kQGThreads = kQWarps * 32;
+constexpr int kQThreads = (kQWarps * kQGroups + 1) * 32;
+constexpr int kQMmaWarp = kQWarps * kQGroups;
+constexpr int kHalf = kTD / 2;                             // columns per compute thread
+constexpr int kHW = kHalf / 32;                            // plane words per compute thread
+constexpr uint32_t kXLbo = 2048, kXSbo = 128;   // bf16 tiles (rows and the rotation)
+constexpr uint32_t kQLbo = 128, kQSbo = 4096;   // S: (n, k) at (n / 8) 4096 + (k / 4) 128 + 16 (n % 8) + 4 (k % 4)
+constexpr int kXBytes = kTRows * kTD * 2;      // one staged bf16 tile
+constexpr int kQSBytes = kTD * kTD * 4;        // one of S_hi / S_lo
+
+template <bool QJL>
+struct TcSmem {
+  static constexpr size_t x = 0;                                  // [group] staged tile
+  static constexpr size_t rot = x + (size_t)kQGroups * kXBytes;    // B of the rotation
+  static constexpr size_t shi = rot + kXBytes;
+  static constexpr size_t slo = shi + (QJL ? kQSBytes : 0);
+  static constexpr size_t xch = slo + (QJL ? kQSBytes : 0);       // [group][half][row] partial sums
+  static constexpr size_t bars = xch + (size_t)kQGroups * 2 * kTRows * 4;
+  // per group: xfull, yfull, yfree, rhi, hidone, rlo, zfull; then done
+  static constexpr int NB = 7;
+  static constexpr size_t total = bars + (size_t)(NB * kQGroups + 1) * 8;
+  static_assert(rot % 1024 == 0 && shi % 1024 == 0, "descriptor base alignment");
+};
+enum { kBxFull = 0, kByFull, kByFree, kBrHi, kBhiDone, kBrLo, kBzFull };
+
+// Issue the cp.async copies of tile rows [r0, r0 + 128) into the canonical layout (rows past n are
+// skipped), by the 256 threads of one group: lane = row within 32 consecutive rows, so that each
+// warp's 16-byte writes are contiguous in shared memory.
+__device__ __forceinline__ void tc_stage_x(const char *__restrict__ x, int64_t ld_bytes, int64_t n, int64_t r0,
+                                           unsigned char *dst, int gi) {
+#pragma unroll 4
+  for (int cc = gi; cc < kTRows * 16; cc += kQGThreads) {
+    const int row = cc & (kTRows - 1), col = cc >> 7;
+    if (r0 + row < n) cp_async16(dst + col * kXLbo + row * 16, x + (r0 + row) * ld_bytes + col * 16);
+  }
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+
+__device__ __forceinline__ bool qwait(uint64_t *bar, unsigned parity, volatile int *abort_flag) {
+  for (int i = 0; i < (1 << 22); ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+  }
+  return false;
+}
+
+__device__ __forceinline__ void group_sync(int g) {
+  if (g == 0)
+    asm volatile("bar.sync 1, 256;\n" ::: "memory");
+  else
+    asm volatile("bar.sync 2, 256;\n" ::: "memory");
+}
+
+// True on every thread of group g when `fail` holds on any of its 256 threads (a barrier with an
+// OR reduction), so that the group leaves its loop as one and no warp is left at a group barrier.
+__device__ __forceinline__ bool group_any(int g, bool fail) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, %2, 256, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)fail), "r"(g + 1)
+      : "memory");
+  return r != 0;
+}
+
+// The group's copies have landed: make them visible to the tensor cores and signal the MMA thread.
+__device__ __forceinline__ void tc_x_ready(int g, uint64_t *xfull, int gi) {
+  asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+  group_sync(g);
+  if (gi == 0) mbar_arrive1(xfull);
+}
+
+// A thread's half row of z (tensor memory, 64 fp32 columns from `zaddr`): sign words 2 h, 2 h + 1.
+__device__ __forceinline__ void pack_signs_half(uint32_t zaddr, const TqConsts &c, const TprArgs &a, int64_t slot,
+                                                int h) {
+  uint32_t sb[kHW];
 #pragma unroll
-  for (int q = 0; q < kTD / 32; ++q) {
+  for (int q = 0; q < kHW; ++q) {
     uint32_t z0[16], z1[16];
     tmem_ld16(zaddr + 32u * q, z0);
     tmem_ld16(zaddr + 32u * q + 16u, z1);
@@ -293,100 +477,87 @@ __device__ __forceinline__ void pack_signs_from_z(uint32_t zaddr, const TqConsts
     }
     sb[q] = m;
   }
-  if (slot >= 0) *reinterpret_cast<uint4 *>(a.signs + slot * c.sign_words) = make_uint4(sb[0], sb[1], sb[2], sb[3]);
+  if (slot >= 0) *reinterpret_cast<uint2 *>(a.signs + slot * c.sign_words + kHW * h) = make_uint2(sb[0], sb[1]);
 }
 
-// tpr_stage by the 128 threads of one group (gt = thread index within the group).
-template <int DT>
-__device__ __forceinline__ void tpr_stage_g(const char *__restrict__ x, int64_t ld_bytes, int64_t n, int64_t r0,
-                                            unsigned char *dst, int gt) {
-  using R = TprRow<DT>;
-  for (int cc = gt; cc < kTRows * R::chunks; cc += kTRows) {
-    const int row = cc / R::chunks, col = cc % R::chunks;
-    if (r0 + row < n) cp_async16(dst + row * R::stride + col * 16, x + (r0 + row) * ld_bytes + col * 16);
+// store_blk16 for the half of the coordinates [64 h, 64 h + 64) whose plane words a warp holds.
+template <int BITS>
+__device__ __forceinline__ void store_blk16_half(const TqConsts &c, const TprArgs &a, const uint32_t (&w)[BITS][kHW],
+                                                 int64_t wrow0, int lane, int h) {
+  if (wrow0 >= a.n) return;  // uniform over the warp
+  const bool twoblk = wrow0 + 16 < a.n;
+  uint32_t *blkA = a.codes + (wrow0 >> 4) * (int64_t)(16 * c.code_words);
+  uint32_t *blkB = blkA + 16 * c.code_words;
+#pragma unroll
+  for (int q2 = 0; q2 < BITS / 2; ++q2)
+#pragma unroll
+    for (int gg = 0; gg < kHW; ++gg) {
+      const int g = kHW * h + gg;
+      const uint32_t lo = warp_transpose32(w[2 * q2][gg], lane), hi = warp_transpose32(w[2 * q2 + 1][gg], lane);
+      blkA[q2 * kTD + 32 * g + lane] = __byte_perm(lo, hi, 0x5410);
+      if (twoblk) blkB[q2 * kTD + 32 * g + lane] = __byte_perm(lo, hi, 0x7632);
+    }
+  if constexpr (BITS & 1) {
+    // odd last plane: coordinates 64 h .. 64 h + 63, two per word
+    const uint32_t ta = warp_transpose32(w[BITS - 1][0], lane);
+    const uint32_t tb = warp_transpose32(w[BITS - 1][1], lane);
+    const int se = (2 * lane) & 31;
+    const uint32_t ea = __shfl_sync(TQ_FULL_MASK, ta, se), eb = __shfl_sync(TQ_FULL_MASK, tb, se);
+    const uint32_t oa = __shfl_sync(TQ_FULL_MASK, ta, se + 1), ob = __shfl_sync(TQ_FULL_MASK, tb, se + 1);
+    const uint32_t ev = lane < 16 ? ea : eb, od = lane < 16 ? oa : ob;
+    blkA[(BITS / 2) * kTD + 32 * h + lane] = __byte_perm(ev, od, 0x5410);
+    if (twoblk) blkB[(BITS / 2) * kTD + 32 * h + lane] = __byte_perm(ev, od, 0x7632);
   }
-  asm volatile("cp.async.commit_group;\n" ::: "memory");
 }
 
-
-// ------------------------------------------------------------------ Gaussian QJL on tcgen05
-// Keys with a dense Gaussian JL matrix (m = d = 128): the same front end (one row per thread), then
-// z = S r on the tensor cores as three TF32 products (r_hi S_hi + r_hi S_lo + r_lo S_hi, each
-// operand split as x = tf32(x) + (x - tf32(x)); the dropped r_lo S_lo term is below 2^-22 of the
-// products), which keeps z within a few fp32 ulps of the fp32 dot product.
-//   A = the tile's residual rows, written by their own threads into tensor memory (lane = row,
-//       one column per coordinate): r_hi for the first two products, then r_lo in the same
-//       columns for the third;
-//   B = S_hi, S_lo in shared memory (canonical K-major layout, staged once per CTA);
-//   D = z in tensor memory, read back by the row's thread for its sign bits.
-// Two groups of four compute warps (thread = row = tensor-memory lane) take alternate tiles, each
-// with its own 256 tensor-memory columns (residual 128, z 128) and staging buffer; warp 8 issues
-// the MMAs (one thread) and owns the allocation.  A group packs its previous tile's signs before
-// encoding its next tile, so while one group waits for its products the other one computes.
-constexpr int kQGroups = 2;
-constexpr int kQThreads = (4 * kQGroups + 1) * 32;
-constexpr int kQMmaWarp = 4 * kQGroups;
-constexpr uint32_t kQLbo = 128, kQSbo = 4096;  // S: 8-row x 16-byte core matrices, K-major
-constexpr int kQSBytes = kTD * kTD * 4;        // one of S_hi / S_lo
-
-template <int DT>
-struct QSmem {
-  static constexpr size_t x = 0;  // one staged tile of rows per group
-  static constexpr size_t shi = x + (size_t)kQGroups * kTRows * TprRow<DT>::stride;
-  static constexpr size_t slo = shi + kQSBytes;
-  static constexpr size_t bars = slo + kQSBytes;  // per group: rhi, rlo, hidone, zfull; then done
-  static constexpr size_t total = bars + (size_t)(4 * kQGroups + 1) * 8;
-  static_assert(shi % 128 == 0, "descriptor base alignment");
-};
-
-__device__ __forceinline__ bool qwait(uint64_t *bar, unsigned parity, volatile int *abort_flag) {
-  for (int i = 0; i < (1 << 22); ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-  }
-  return false;
-}
-
-__device__ __forceinline__ void group_sync(int g) {
-  if (g == 0)
-    asm volatile("bar.sync 1, 128;\n" ::: "memory");
-  else
-    asm volatile("bar.sync 2, 128;\n" ::: "memory");
-}
-
-template <int DT, int BITS>
+template <int BITS, bool QJL, bool BLK>
 __global__ void __launch_bounds__(kQThreads, 1)
-encode_tcq_kernel(TqConsts c, TprArgs a) {
-  using R = TprRow<DT>;
-  using SM = QSmem<DT>;
-  extern __shared__ __align__(1024) unsigned char smem[];
-  __shared__ float sgn[kTD], cen[TQ_MAX_LEVELS];
+encode_tc_kernel(TqConsts c, TprArgs a) {
+  using SM = TcSmem<QJL>;
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ float cen[TQ_MAX_LEVELS];
   __shared__ uint32_t tslot;
   __shared__ int abort_flag_s;
   volatile int *abort_flag = &abort_flag_s;
-  uint64_t *gb = reinterpret_cast<uint64_t *>(smem + SM::bars);  // [group][rhi, rlo, hidone, zfull]
-  uint64_t *done = gb + 4 * kQGroups;
+  uint64_t *gb = reinterpret_cast<uint64_t *>(smem + SM::bars);  // [group][SM::NB]
+  uint64_t *done = gb + SM::NB * kQGroups;
+  float *xch = reinterpret_cast<float *>(smem + SM::xch);       // [group][half][row]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   constexpr int L = 1 << BITS;
+  constexpr uint32_t kCols = QJL ? 512u : 256u;  // per group: y / residual (128) [, z (128)]
+  constexpr uint32_t kGCols = kCols / kQGroups;
 
-  // S_hi and S_lo in the canonical K-major layout: (n, k) at (n/8) SBO + (k/4) LBO + (n%8) 16 + (k%4) 4
+  // B of the rotation: (n, k) = (-1)^popcount(n & k) D_k as bf16, at (k / 8) 2048 + 16 n + 2 (k % 8)
   for (int idx = tid; idx < kTD * kTD; idx += kQThreads) {
     const int n = idx / kTD, k = idx % kTD;
-    const float sv = c.S[idx];
-    const uint32_t hi = to_tf32(sv);
-    const float lo = sv - __uint_as_float(hi);
-    const uint32_t off = (uint32_t)(n >> 3) * kQSbo + (uint32_t)(k >> 2) * kQLbo + (uint32_t)(n & 7) * 16 + (uint32_t)(k & 3) * 4;
-    *reinterpret_cast<uint32_t *>(smem + SM::shi + off) = hi;
-    *reinterpret_cast<uint32_t *>(smem + SM::slo + off) = to_tf32(lo);
+    const bool neg = ((__popc(n & k) & 1) != 0) != (c.signs[k] < 0.f);
+    *reinterpret_cast<uint16_t *>(smem + SM::rot + (k >> 3) * kXLbo + n * 16 + (k & 7) * 2) =
+        neg ? (uint16_t)0xBF80u : (uint16_t)0x3F80u;
   }
-  for (int jj = tid; jj < kTD; jj += kQThreads) sgn[jj] = c.signs[jj];
+  if constexpr (QJL) {
+    // S_hi and S_lo in the canonical K-major layout
+    for (int idx = tid; idx < kTD * kTD; idx += kQThreads) {
+      const int n = idx / kTD, k = idx % kTD;
+      const float sv = c.S[idx];
+      const uint32_t hi = to_tf32(sv);
+      const float lo = sv - __uint_as_float(hi);
+      const uint32_t off = (uint32_t)(n >> 3) * kQSbo + (uint32_t)(k >> 2) * kQLbo + (uint32_t)(n & 7) * 16 +
+                           (uint32_t)(k & 3) * 4;
+      *reinterpret_cast<uint32_t *>(smem + SM::shi + off) = hi;
+      *reinterpret_cast<uint32_t *>(smem + SM::slo + off) = to_tf32(lo);
+    }
+  }
   if (tid < TQ_MAX_LEVELS) cen[tid] = c.centroids[tid];
   if (tid == 0) {
     for (int g = 0; g < kQGroups; ++g) {
-      mbar_init(&gb[4 * g + 0], 4);
-      mbar_init(&gb[4 * g + 1], 4);
-      mbar_init(&gb[4 * g + 2], 1);
-      mbar_init(&gb[4 * g + 3], 1);
+      uint64_t *b = gb + SM::NB * g;
+      mbar_init(&b[kBxFull], 1);
+      mbar_init(&b[kByFull], 1);
+      mbar_init(&b[kByFree], kQWarps);
+      mbar_init(&b[kBrHi], kQWarps);
+      mbar_init(&b[kBhiDone], 1);
+      mbar_init(&b[kBrLo], kQWarps);
+      mbar_init(&b[kBzFull], 1);
     }
     mbar_init(done, 1);
     abort_flag_s = 0;
@@ -394,11 +565,11 @@ encode_tcq_kernel(TqConsts c, TprArgs a) {
   }
   if (warp == kQMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_addr(&tslot)),
-                 "r"(512)
+                 "r"(kCols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
   }
-  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // S visible to the tensor cores
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // B operands visible to the tensor cores
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -409,160 +580,244 @@ encode_tcq_kernel(TqConsts c, TprArgs a) {
   if (warp == kQMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      // D f32, A and B tf32, both K-major, N = 128, M = 128
-      const uint32_t idesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(kTD >> 3) << 17) |
-                             ((uint32_t)(kTRows >> 4) << 24);
+      // rotation: D f32, A and B bf16, both K-major, N = M = 128; products: A and B tf32
+      const uint32_t idesc_r = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kTD >> 3) << 17) |
+                               ((uint32_t)(kTRows >> 4) << 24);
+      const uint32_t idesc_q = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(kTD >> 3) << 17) |
+                               ((uint32_t)(kTRows >> 4) << 24);
+      const uint32_t xs = smem_addr(smem + SM::x), rs = smem_addr(smem + SM::rot);
       const uint32_t shi = smem_addr(smem + SM::shi), slo = smem_addr(smem + SM::slo);
-      for (int64_t i = 0; i < mytiles; ++i) {
-        const int g = (int)(i % kQGroups);
-        const unsigned ph = (unsigned)((i / kQGroups) & 1);
-        uint64_t *b = gb + 4 * g;
-        const uint32_t rcol = tmem + 256u * g, zcol = rcol + 128u;
-        if (!qwait(&b[0], ph, abort_flag)) {
-          *abort_flag = 1;
-          break;
-        }
+      bool ok = true;
+      // the products of local tile t (QJL)
+      auto products = [&](int64_t t) -> bool {
+        const int g = (int)(t % kQGroups);
+        const unsigned ph = (unsigned)((t / kQGroups) & 1);
+        uint64_t *b = gb + SM::NB * g;
+        const uint32_t acol = tmem + kGCols * g, zcol = acol + 128u;
+        if (!qwait(&b[kBrHi], ph, abort_flag)) return false;
         tc_fence_after();
 #pragma unroll
         for (int pass = 0; pass < 2; ++pass)  // r_hi S_hi, r_hi S_lo
 #pragma unroll
           for (int ks = 0; ks < kTD / 8; ++ks)
-            umma_tf32_ta(zcol, rcol + 8u * ks, umma_desc((pass ? slo : shi) + 2u * kQLbo * ks, kQLbo, kQSbo), idesc,
-                         (pass == 0 && ks == 0) ? 0u : 1u);
-        umma_commit(&b[2]);
-        if (!qwait(&b[1], ph, abort_flag)) {
-          *abort_flag = 1;
-          break;
-        }
+            umma_tf32_ta(zcol, acol + 8u * ks, umma_desc((pass ? slo : shi) + 2u * kQLbo * ks, kQLbo, kQSbo),
+                         idesc_q, (pass == 0 && ks == 0) ? 0u : 1u);
+        umma_commit(&b[kBhiDone]);
+        if (!qwait(&b[kBrLo], ph, abort_flag)) return false;
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < kTD / 8; ++ks)  // r_lo S_hi
-          umma_tf32_ta(zcol, rcol + 8u * ks, umma_desc(shi + 2u * kQLbo * ks, kQLbo, kQSbo), idesc, 1u);
-        umma_commit(&b[3]);
+          umma_tf32_ta(zcol, acol + 8u * ks, umma_desc(shi + 2u * kQLbo * ks, kQLbo, kQSbo), idesc_q, 1u);
+        umma_commit(&b[kBzFull]);
+        return true;
+      };
+      for (int64_t i = 0; i < mytiles && ok; ++i) {
+        const int g = (int)(i % kQGroups);
+        const unsigned ph = (unsigned)((i / kQGroups) & 1);
+        uint64_t *b = gb + SM::NB * g;
+        const uint32_t acol = tmem + kGCols * g;
+        if (!qwait(&b[kBxFull], ph, abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (i >= kQGroups) {
+          // the group's columns are free: its previous residual has been used (QJL) or its
+          // previous y has been read (values)
+          if (!qwait(&b[QJL ? kBzFull : kByFree], ph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+        }
+        tc_fence_after();
+        const uint32_t xg = xs + (uint32_t)g * kXBytes;
+#pragma unroll
+        for (int ks = 0; ks < kTD / 16; ++ks)
+          umma_f16_ss(acol, umma_desc(xg + 2u * kXLbo * ks, kXLbo, kXSbo), umma_desc(rs + 2u * kXLbo * ks, kXLbo, kXSbo),
+                      idesc_r, ks == 0 ? 0u : 1u);
+        umma_commit(&b[kByFull]);
+        if constexpr (QJL)
+          if (i >= 1 && !products(i - 1)) ok = false;
       }
+      if constexpr (QJL)
+        if (ok && mytiles > 0 && !products(mytiles - 1)) ok = false;
+      if (!ok) *abort_flag = 1;
       umma_commit(done);  // every MMA this thread issued has completed when `done` fires
       qwait(done, 0u, abort_flag);
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ compute: one row per thread
-    const int g = warp >> 2, gt = tid & 127;  // group, row within the tile
-    uint64_t *b = gb + 4 * g;
-    unsigned char *xbuf = smem + SM::x + (size_t)g * kTRows * R::stride;
-    const float sqrtd = 1.f / c.inv_sqrt_d;
-    const uint32_t rbase = tmem + 256u * g + ((uint32_t)(32 * (warp & 3)) << 16), zbase = rbase + 128u;
+    // ------------------------------------------------------------ compute: half a row per thread
+    const int g = warp / kQWarps, gw = warp % kQWarps;  // group, warp within the group
+    const int quad = gw & 3, h = gw >> 2;               // lane quadrant (rows), column half
+    const int gt = 32 * quad + lane;                    // row within the tile
+    const int gi = tid - g * kQGThreads;                // thread within the group
+    uint64_t *b = gb + SM::NB * g;
+    unsigned char *xbuf = smem + SM::x + (size_t)g * kXBytes;
+    float *myx = xch + (g * 2 + h) * kTRows + gt, *otx = xch + g * 2 * kTRows + gt;
+    const uint32_t lanes = (uint32_t)(32 * quad) << 16;
+    const uint32_t abase = tmem + kGCols * g + lanes + (uint32_t)(kHalf * h), zbase = abase + 128u;
+    float thr[Sym<BITS>::HW];  // the positive thresholds (value codes by symmetry)
+#pragma unroll
+    for (int k = 0; k < Sym<BITS>::H; ++k) thr[k] = c.thresholds[L / 2 + k];
     int64_t prev_slot = -1;
-    bool ok = true;
     int64_t j = 0;  // this group's tiles so far
     int64_t i = g;  // local tile index
-    if (i < mytiles) tpr_stage_g<DT>(a.x, a.ld_bytes, a.n, (blockIdx.x + i * gridDim.x) * kTRows, xbuf, gt);
+    if (i < mytiles) {
+      tc_stage_x(a.x, a.ld_bytes, a.n, (blockIdx.x + i * gridDim.x) * kTRows, xbuf, gi);
+      tc_x_ready(g, &b[kBxFull], gi);
+    }
     for (; i < mytiles; i += kQGroups, ++j) {
       const int64_t tile = blockIdx.x + i * gridDim.x;
-      // this group's previous z: its signs first (its columns are then free for this tile)
-      if (j > 0) {
-        ok = qwait(&b[3], (unsigned)((j - 1) & 1), abort_flag);
-        if (!__all_sync(TQ_FULL_MASK, ok)) {
-          if (lane == 0) *abort_flag = 1;
-          break;
+      bool ok = true;
+      if constexpr (QJL) {
+        // this group's previous z: its signs first (its columns are then free for this tile)
+        if (j > 0) {
+          ok = qwait(&b[kBzFull], (unsigned)((j - 1) & 1), abort_flag);
+          if (group_any(g, !ok || *abort_flag)) break;
+          tc_fence_after();
+          pack_signs_half(zbase, c, a, prev_slot, h);
         }
-        tc_fence_after();
-        pack_signs_from_z(zbase, c, a, prev_slot);
       }
-      asm volatile("cp.async.wait_group 0;\n" ::: "memory");
-      group_sync(g);
+      ok = qwait(&b[kByFull], (unsigned)(j & 1), abort_flag);
+      if (group_any(g, !ok || *abort_flag)) break;
+      tc_fence_after();
+      float v[kHalf];
+#pragma unroll
+      for (int cb = 0; cb < kHalf / 16; ++cb) {
+        uint32_t u[16];
+        tmem_ld16(abase + 16u * cb, u);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[16 * cb + e] = __uint_as_float(u[e]);
+      }
+      asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+      if constexpr (!QJL) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive1(&b[kByFree]);
+      }
+      // the rotation has read this group's tile: stage its next one
+      const bool more = i + kQGroups < mytiles;
+      if (more) tc_stage_x(a.x, a.ld_bytes, a.n, (blockIdx.x + (i + kQGroups) * gridDim.x) * kTRows, xbuf, gi);
+
       const int64_t row = tile * kTRows + gt;
       const bool valid = row < a.n;
       const int64_t slot = valid ? (a.slots ? a.slots[row] : row) : -1;
       const bool store = valid && slot >= 0 && slot < a.capacity;
-      float v[kTD];
-      tpr_load<DT>(xbuf + gt * R::stride, v);
-      group_sync(g);  // the buffer is free: stage this group's next tile
-      if (i + kQGroups < mytiles)
-        tpr_stage_g<DT>(a.x, a.ld_bytes, a.n, (blockIdx.x + (i + kQGroups) * gridDim.x) * kTRows, xbuf, gt);
-      float ss = 0.f;
+      // ||y||^2 = d ||x||^2: eight partial sums per half, the halves added in a fixed order
+      float ps[8];
 #pragma unroll
-      for (int jj = 0; jj < kTD; ++jj) ss = fmaf(v[jj], v[jj], ss);
-      const float nu = sqrtf(ss);
+      for (int e = 0; e < 8; ++e) ps[e] = 0.f;
 #pragma unroll
-      for (int jj = 0; jj < kTD; jj += 4) {
-        const float4 s4 = *reinterpret_cast<const float4 *>(sgn + jj);
-        v[jj] *= s4.x; v[jj + 1] *= s4.y; v[jj + 2] *= s4.z; v[jj + 3] *= s4.w;
-      }
-      fwht128(v);
-      const float scl = nu > 0.f ? nu * sqrtd : 1.f;
-      const float inv = nu > 0.f ? 1.f / scl : 0.f;
-      float T[L - 1];
+      for (int jj = 0; jj < kHalf; ++jj) ps[jj & 7] = fmaf(v[jj], v[jj], ps[jj & 7]);
+      *myx = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      group_sync(g);
+      const float ssy = otx[0] + otx[kTRows];
+      const float ny = sqrtf(ssy);
+      const float nu = ny * c.inv_sqrt_d;
+      const float scl = ny > 0.f ? ny : 1.f;
+      uint32_t w[BITS][kHW];
+      if constexpr (QJL) {
+        const float inv = ny > 0.f ? 1.f / scl : 0.f;
+        float T[L - 1];
 #pragma unroll
-      for (int k = 0; k < L - 1; ++k) T[k] = c.thresholds[k] * scl;
-      uint32_t w[BITS][kTD / 32];
+        for (int k = 0; k < L - 1; ++k) T[k] = c.thresholds[k] * scl;
 #pragma unroll
-      for (int P = 0; P < BITS; ++P)
+        for (int P = 0; P < BITS; ++P)
 #pragma unroll
-        for (int q = 0; q < kTD / 32; ++q) w[P][q] = 0u;
-      float rr = 0.f;
+          for (int q = 0; q < kHW; ++q) w[P][q] = 0u;
+        float rr = 0.f;
 #pragma unroll
-      for (int jj = 0; jj < kTD; ++jj) {
-        int code = 0;
+        for (int jj = 0; jj < kHalf; ++jj) {
+          int code = 0;
 #pragma unroll
-        for (int k = 0; k < L - 1; ++k) code += v[jj] >= T[k] ? 1 : 0;
+          for (int k = 0; k < L - 1; ++k) code += v[jj] >= T[k] ? 1 : 0;
 #pragma unroll
-        for (int P = 0; P < BITS; ++P) w[P][jj >> 5] |= (uint32_t)((code >> P) & 1) << (jj & 31);
-        const float r = fmaf(v[jj], inv, -cen[code]);
-        v[jj] = r;
-        rr = fmaf(r, r, rr);
-      }
-      if (store) {
-        uint4 *dst = reinterpret_cast<uint4 *>(a.codes + slot * c.code_words);
-#pragma unroll
-        for (int P = 0; P < BITS; ++P) dst[P] = make_uint4(w[P][0], w[P][1], w[P][2], w[P][3]);
-        a.norm[slot] = nu;
-        a.rnorm[slot] = sqrtf(rr);
-      }
-      // r_hi -> tensor memory, then the first two products may start
-#pragma unroll
-      for (int cb = 0; cb < kTD / 16; ++cb) {
-        uint32_t hv[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          hv[e] = to_tf32(v[16 * cb + e]);
-          v[16 * cb + e] -= __uint_as_float(hv[e]);  // r_lo from here on (exact in fp32)
+          for (int P = 0; P < BITS; ++P) w[P][jj >> 5] |= (uint32_t)((code >> P) & 1) << (jj & 31);
+          const float r = fmaf(v[jj], inv, -cen[code]);
+          v[jj] = r;
+          rr = fmaf(r, r, rr);
         }
-        tmem_st16(rbase + 16u * cb, hv);
-      }
-      asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive1(&b[0]);
-      // r_lo into the same columns once those products have read r_hi
-      ok = qwait(&b[2], (unsigned)(j & 1), abort_flag);
-      if (!__all_sync(TQ_FULL_MASK, ok)) {
-        if (lane == 0) *abort_flag = 1;
-        break;
-      }
-      tc_fence_after();
+        group_sync(g);  // both halves have read the norm partials
+        *myx = rr;
+        group_sync(g);
+        const float rr2 = otx[0] + otx[kTRows];
+        if (store) {
+          uint32_t *dst = a.codes + slot * c.code_words + kHW * h;
 #pragma unroll
-      for (int cb = 0; cb < kTD / 16; ++cb) {
-        uint32_t lv[16];
+          for (int P = 0; P < BITS; ++P) *reinterpret_cast<uint2 *>(dst + 4 * P) = make_uint2(w[P][0], w[P][1]);
+          if (h == 0) {
+            a.norm[slot] = nu;
+            a.rnorm[slot] = sqrtf(rr2);
+          }
+        }
+        // r_hi -> tensor memory (the columns y came from), then the first two products may start
 #pragma unroll
-        for (int e = 0; e < 16; ++e) lv[e] = __float_as_uint(v[16 * cb + e]);
-        tmem_st16(rbase + 16u * cb, lv);
-      }
-      asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive1(&b[1]);
-      prev_slot = store ? slot : -1;
-    }
-    // the group's last tile's signs
-    if (j > 0 && !*abort_flag) {
-      ok = qwait(&b[3], (unsigned)((j - 1) & 1), abort_flag);
-      if (__all_sync(TQ_FULL_MASK, ok)) {
+        for (int cb = 0; cb < kHalf / 16; ++cb) {
+          uint32_t hv[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            hv[e] = to_tf32(v[16 * cb + e]);
+            v[16 * cb + e] -= __uint_as_float(hv[e]);  // r_lo from here on (exact in fp32)
+          }
+          tmem_st16(abase + 16u * cb, hv);
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive1(&b[kBrHi]);
+        // r_lo into the same columns once those products have read r_hi
+        ok = qwait(&b[kBhiDone], (unsigned)(j & 1), abort_flag);
+        if (group_any(g, !ok || *abort_flag)) break;
         tc_fence_after();
-        pack_signs_from_z(zbase, c, a, prev_slot);
-      } else if (lane == 0) {
-        *abort_flag = 1;
+#pragma unroll
+        for (int cb = 0; cb < kHalf / 16; ++cb) {
+          uint32_t lv[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) lv[e] = __float_as_uint(v[16 * cb + e]);
+          tmem_st16(abase + 16u * cb, lv);
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive1(&b[kBrLo]);
+        prev_slot = store ? slot : -1;
+      } else {
+        float T[Sym<BITS>::HW];
+#pragma unroll
+        for (int k = 0; k < Sym<BITS>::H; ++k) T[k] = thr[k] * scl;
+        uint32_t sw[kHW], tw[Sym<BITS>::HW][kHW];
+#pragma unroll
+        for (int q = 0; q < kHW; ++q) {
+          sw[q] = 0u;
+#pragma unroll
+          for (int k = 0; k < Sym<BITS>::HW; ++k) tw[k][q] = 0u;
+        }
+#pragma unroll
+        for (int jj = 0; jj < kHalf; ++jj) sym_quant<BITS, kHW>(v[jj], T, sw, tw, jj);
+        sym_planes<BITS, kHW>(sw, tw, w);
+        if constexpr (BLK) {
+          store_blk16_half<BITS>(c, a, w, tile * kTRows + 32 * quad, lane, h);
+          if (valid && h == 0) a.norm[row] = nu;
+        } else if (store) {
+          uint32_t *dst = a.codes + slot * c.code_words + kHW * h;
+#pragma unroll
+          for (int P = 0; P < BITS; ++P) *reinterpret_cast<uint2 *>(dst + 4 * P) = make_uint2(w[P][0], w[P][1]);
+          if (h == 0) a.norm[slot] = nu;
+        }
+      }
+      if (more) tc_x_ready(g, &b[kBxFull], gi);
+    }
+    if constexpr (QJL) {
+      // the group's last tile's signs
+      if (i >= mytiles && j > 0) {
+        const bool ok = qwait(&b[kBzFull], (unsigned)((j - 1) & 1), abort_flag);
+        if (__all_sync(TQ_FULL_MASK, ok)) {
+          tc_fence_after();
+          pack_signs_half(zbase, c, a, prev_slot, h);
+        }
       }
     }
+    if (i < mytiles && lane == 0) *abort_flag = 1;  // left the loop on a failed wait
     asm volatile("cp.async.wait_group 0;\n" ::: "memory");
   }
   tc_fence_before();
@@ -570,33 +825,32 @@ encode_tcq_kernel(TqConsts c, TprArgs a) {
   if (*abort_flag && tid == 0) atomicOr(&g_tq_device_flags, kFlagStagingTimeout);
   if (warp == kQMmaWarp) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(512) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kCols) : "memory");
   }
 }
 
-template <int DT, int BITS>
-cudaError_t launch_tcq_t(const TqConsts &c, const TprArgs &a, cudaStream_t st) {
-  const size_t smem = QSmem<DT>::total;
-  cudaError_t e = tq_smem_limit(reinterpret_cast<const void *>(encode_tcq_kernel<DT, BITS>), (int)smem);
+template <int BITS, bool QJL, bool BLK>
+cudaError_t launch_tc_t(const TqConsts &c, const TprArgs &a, cudaStream_t st) {
+  static_assert(TcSmem<QJL>::total + 512 <= 227 * 1024, "the tensor-core encode's shared memory (with its static part)");
+  const size_t smem = TcSmem<QJL>::total;
+  cudaError_t e = tq_smem_limit(reinterpret_cast<const void *>(encode_tc_kernel<BITS, QJL, BLK>), (int)smem);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t ntiles = (a.n + kTRows - 1) / kTRows;
-  const int64_t grid = ntiles < (int64_t)sms ? ntiles : (int64_t)sms;
-  tq_prof_begin(TQK_ENCODE_QJL_TC, st);
-  encode_tcq_kernel<DT, BITS><<<(unsigned)grid, kQThreads, smem, st>>>(c, a);
-  tq_prof_end(TQK_ENCODE_QJL_TC, st);
+  const int64_t sms = tq_sm_count();
+  const int64_t grid = ntiles < sms ? ntiles : sms;
+  tq_prof_begin(QJL ? TQK_ENCODE_QJL_TC : TQK_ENCODE_ROWS, st);
+  encode_tc_kernel<BITS, QJL, BLK><<<(unsigned)grid, kQThreads, smem, st>>>(c, a);
+  tq_prof_end(QJL ? TQK_ENCODE_QJL_TC : TQK_ENCODE_ROWS, st);
   return cudaGetLastError();
 }
 
-template <int DT>
-cudaError_t launch_tcq_dt(const TqConsts &c, const TprArgs &a, cudaStream_t st) {
-  static_assert(QSmem<DT>::total <= 227 * 1024, "the tensor-core encode's shared memory");
+template <bool QJL, bool BLK>
+cudaError_t launch_tc_b(const TqConsts &c, const TprArgs &a, cudaStream_t st) {
   switch (c.bits) {
-    case 1: return launch_tcq_t<DT, 1>(c, a, st);
-    case 2: return launch_tcq_t<DT, 2>(c, a, st);
-    case 3: return launch_tcq_t<DT, 3>(c, a, st);
-    case 4: return launch_tcq_t<DT, 4>(c, a, st);
+    case 1: return launch_tc_t<1, QJL, BLK>(c, a, st);
+    case 2: return launch_tc_t<2, QJL, BLK>(c, a, st);
+    case 3: return launch_tc_t<3, QJL, BLK>(c, a, st);
+    case 4: return launch_tc_t<4, QJL, BLK>(c, a, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -630,6 +884,8 @@ cudaError_t launch_encode_tpr(const TqConsts &c, const void *x, tq_dtype dtype, 
   a.norm = norm;
   a.rnorm = rnorm;
   a.signs = signs;
-  if (c.m > 0 && !c.srht) return launch_tcq_dt<TQ_BF16>(c, a, st);  // bf16 rows only (eligibility)
+  if (c.m > 0 && !c.srht) return launch_tc_b<true, false>(c, a, st);  // bf16 rows only (eligibility)
+  if (dtype == TQ_BF16 && !c.srht)
+    return c.layout == TQ_LAYOUT_BLOCK16 ? launch_tc_b<false, true>(c, a, st) : launch_tc_b<false, false>(c, a, st);
   return dtype == TQ_F32 ? launch_tpr_dt<TQ_F32>(c, a, st) : launch_tpr_dt<TQ_BF16>(c, a, st);
 }

@@ -71,7 +71,8 @@ __device__ __forceinline__ void fwht_lanes(float (&v)[RotLayout<D>::KCH][4], int
 
 // The encode / query-rotation work of one block of kRotThreads threads: rows of block `vblock`.
 // `sS` is dynamic shared memory of at least 128 x 132 floats when d = m = 128 and `fsigns` is set
-// (the fused projection stages S there); every thread of the block must call it with the same
+// (the fused projection stages S there), or null to read S rows from global memory (same
+// arithmetic, same results); every thread of the block must call it with the same
 // arguments.  With `one_vec` (d = m = 128, fused projection) the block encodes the single row
 // `vblock`: warp 0 rotates and quantizes it and warps 0-3 share its projection, 32 rows each (the
 // same arithmetic as one warp doing all 128).
@@ -90,7 +91,7 @@ __device__ __forceinline__ void rotate_rows(const TqConsts &c, int mode, const v
   const int lane = threadIdx.x & 31;
   const int wib = threadIdx.x >> 5;
   // fused projection with S staged in shared memory (d = m = 128; row stride 132 floats)
-  const bool staged = D == 128 && fsigns != nullptr && c.m == 128 && !c.srht;
+  const bool staged = D == 128 && fsigns != nullptr && c.m == 128 && !c.srht && sS != nullptr;
   if (staged) stage_rows_padded_async(sS, c.S, 128, 128);  // completed before the projection
   const int g = lane / LPV;
   const int l = lane % LPV;
@@ -284,16 +285,22 @@ __device__ __forceinline__ void rotate_rows(const TqConsts &c, int mode, const v
         __syncthreads();
         if (wib < c.m / 32) {
           const int w = wib;
-          const float4 *Srow = staged ? reinterpret_cast<const float4 *>(sS + (32 * w + lane) * (D + 4))
-                                      : reinterpret_cast<const float4 *>(c.S + (int64_t)(32 * w + lane) * D);
           float z = 0.f;
+          if (staged) {
+            const float4 *Srow = reinterpret_cast<const float4 *>(sS + (32 * w + lane) * (D + 4));
 #pragma unroll 8
-          for (int j4 = 0; j4 < D / 4; ++j4) {
-            const float4 sv = Srow[j4];
-            z = fmaf(sv.x, rb[4 * j4], z);
-            z = fmaf(sv.y, rb[4 * j4 + 1], z);
-            z = fmaf(sv.z, rb[4 * j4 + 2], z);
-            z = fmaf(sv.w, rb[4 * j4 + 3], z);
+            for (int j4 = 0; j4 < D / 4; ++j4) {
+              const float4 sv = Srow[j4];
+              z = fmaf(sv.x, rb[4 * j4], z);
+              z = fmaf(sv.y, rb[4 * j4 + 1], z);
+              z = fmaf(sv.z, rb[4 * j4 + 2], z);
+              z = fmaf(sv.w, rb[4 * j4 + 3], z);
+            }
+          } else {
+            // S transposed: the warp reads 32 consecutive floats per coordinate (same order of sums)
+            const float *Sc = c.St + 32 * w + lane;
+#pragma unroll 32
+            for (int j = 0; j < D; ++j) z = fmaf(Sc[(int64_t)j * c.m], rb[j], z);
           }
           const unsigned bal = __ballot_sync(TQ_FULL_MASK, z >= 0.f);
           if (ostore && lane == 0) fsigns[oslot * c.sign_words + w] = bal;
@@ -302,16 +309,21 @@ __device__ __forceinline__ void rotate_rows(const TqConsts &c, int mode, const v
       }
       __syncwarp();
       for (int w = 0; w < c.m / 32; ++w) {
-        const float4 *Srow = staged ? reinterpret_cast<const float4 *>(sS + (32 * w + lane) * (D + 4))
-                                    : reinterpret_cast<const float4 *>(c.S + (int64_t)(32 * w + lane) * D);
         float z = 0.f;
+        if (staged) {
+          const float4 *Srow = reinterpret_cast<const float4 *>(sS + (32 * w + lane) * (D + 4));
 #pragma unroll 8
-        for (int j4 = 0; j4 < D / 4; ++j4) {
-          const float4 sv = Srow[j4];
-          z = fmaf(sv.x, rb[4 * j4], z);
-          z = fmaf(sv.y, rb[4 * j4 + 1], z);
-          z = fmaf(sv.z, rb[4 * j4 + 2], z);
-          z = fmaf(sv.w, rb[4 * j4 + 3], z);
+          for (int j4 = 0; j4 < D / 4; ++j4) {
+            const float4 sv = Srow[j4];
+            z = fmaf(sv.x, rb[4 * j4], z);
+            z = fmaf(sv.y, rb[4 * j4 + 1], z);
+            z = fmaf(sv.z, rb[4 * j4 + 2], z);
+            z = fmaf(sv.w, rb[4 * j4 + 3], z);
+          }
+        } else {
+          const float *Sc = c.St + 32 * w + lane;
+#pragma unroll 32
+          for (int j = 0; j < D; ++j) z = fmaf(Sc[(int64_t)j * c.m], rb[j], z);
         }
         const unsigned bal = __ballot_sync(TQ_FULL_MASK, z >= 0.f);
         if (store && lane == 0) fsigns[slot * c.sign_words + w] = bal;

@@ -78,3 +78,14 @@ __device__ __forceinline__ uint32_t to_tf32(float x) {
   asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
   return r;
 }
+
+// kind::f16 with both operands in shared memory (descriptors): D (f32, tensor memory) += A x B^T,
+// A and B bf16 per the instruction descriptor, K = 16 elements per MMA; accum = 0 overwrites D
+__device__ __forceinline__ void umma_f16_ss(uint32_t dtmem, uint64_t da, uint64_t db, uint32_t idesc,
+                                            uint32_t accum) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(dtmem), "l"(da), "l"(db),
+      "r"(idesc), "r"(accum)
+      : "memory");
+}

@@ -29,6 +29,7 @@ struct TqConsts {
   float thresholds[TQ_MAX_LEVELS];  // [levels-1] used
   const float *signs;  // device [d], +-1.0f (rotation D)
   const float *S;      // device [m][d] row-major (JL matrix)
+  const float *St;     // device [d][m]: S transposed (coalesced reads with lane = row of S)
   int srht;               // S = P H D2 (structured QJL): encode transforms the residual instead
   const float *qjl_signs; // device [d], +-1.0f (D2), srht only
   int polar;              // PolarQuant first stage (angle codes in place of coordinate codes)
@@ -45,6 +46,7 @@ struct tq_ctx {
   double mse_per_coord;
   float *dev_signs;  // [d]
   float *dev_S;      // [m][d]
+  float *dev_St;     // [d][m]
   float *dev_qjl_signs;  // [d] (structured QJL only)
   float *dev_polar;      // PolarQuant angle tables (polar only)
   TqConsts k;        // kernel view
@@ -215,3 +217,11 @@ cudaError_t launch_search(const TqConsts &c, const SearchPlan &plan, const float
                           cudaStream_t st);
 
 static inline int64_t tq_align_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
+// SMs of the current device (148 on a B200 if the query fails).
+static inline int tq_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+      n > 0)
+    return n;
+  return 148;
+}

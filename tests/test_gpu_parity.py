@@ -392,6 +392,28 @@ def test_encode_bulk_rows_d128(tq, layout, bits, dtype):
         assert np.array_equal(stale, full[tail % 16])
 
 
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_encode_bulk_keys_qjl_bf16(tq, bits):
+    """bf16 keys with a dense JL matrix (d = m = 128) past the fused small-batch limit: the
+    tensor-core encode (rotation as a bf16 MMA, z = S r as three TF32 products), with scattered
+    slots, a zero vector, a ragged last tile and out-of-range slots that must be skipped."""
+    n, d = 5011, 128
+    cap = n + 64
+    q = Quantizer(d, bits, 128, seed=700 + bits)
+    x = (torch.randn(n, d, generator=torch.Generator().manual_seed(40 + bits)) *
+         torch.exp(torch.randn(d, generator=torch.Generator().manual_seed(8)))).to(torch.bfloat16)
+    x[5] = 0
+    slots = torch.randperm(cap, generator=torch.Generator().manual_seed(bits))[:n].to(torch.int64)
+    slots[9] = cap + 3  # out of range: not written
+    packed = tq.Packed.allocate(q.ctx, cap)
+    packed.codes.fill_(0xA5)
+    tq.encode_kv(q.ctx, x.cuda(), packed, slots=slots.cuda())
+    torch.cuda.synchronize()
+    keep = np.array([i for i in range(n) if i != 9])
+    codes, sbits, norm, rnorm = unpack(q, packed, rows=slots.numpy()[keep])
+    compare_encode(q, q.oracle_encode(x.double().numpy()[keep]), codes, sbits, norm, rnorm)
+
+
 @pytest.mark.parametrize("vbits", [2, 3])
 def test_attention_block16_values_contiguous(tq, vbits):
     _attention_case(tq, 128, 2, 128, vbits, batch=2, hkv=2, group=4, lens=[1500, 333], paged=False,
