@@ -58,9 +58,12 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 BLOCK = 16
 DTYPE_DECODE = ("int8 tensor-core limbs: 32-bit fixed-point query terms x 0/1 key bit planes, 16-bit "
                 "fixed-point value weights; fp32 softmax and accumulation")
-# DRAM bytes per launch of the attention kernel, from one ncu capture of the kernel revision named
-# in the library's version string (profiles/attend_mma_<workload>.md); null for any other revision
-NCU_TRAFFIC = {}
+# DRAM bytes (read + write) per launch of the attention kernel, from one ncu capture (one pass,
+# `dram__bytes_read.sum` + `dram__bytes_write.sum`) of the kernel revision named in the library's
+# version string, on the workload named; null for any other revision or workload
+NCU_TRAFFIC = {
+    ("attend_mma", "r10", "ragged"): 949.95e6 + 14.92e6,
+}
 
 
 def parse_args(argv=None):
@@ -240,6 +243,14 @@ def ragged_layout(cfg, seed: int):
     return lens, table, nblocks
 
 
+def cache_block_table(lens, seed: int, ci: int):
+    """Block table of cache `ci` of a paged workload: the same lengths as every other cache (so
+    every step does the same work), another permutation of the physical blocks."""
+    import synth
+    tab, _ = synth.shuffled_block_table(lens, seed=seed + 1 + 17 * ci)
+    return tab
+
+
 class DecodeBench:
     """Device-resident compressed caches of one decode workload plus the per-step inputs.
 
@@ -307,8 +318,7 @@ class DecodeBench:
             del xs
             table = None
             if self.paged:
-                _, tab, _ = ragged_layout(cfg, 1102 + seed + 17 * ci)  # same lengths, another permutation
-                table = tab.to(dev)
+                table = cache_block_table(self.lens, 1102 + seed, ci).to(dev)
             self.caches.append((kp, vp, table))
         torch.cuda.synchronize()
         # per-step inputs: the queries and the new token's K/V of every (sequence, KV head)
@@ -551,7 +561,7 @@ def ours_decode(args, world, rank):
         achieved = bench.bytes_per_step / per_launch_s / 1e9
         roof = {"kernel": "attend_mma_kernel (tensor cores, streamed sub-chunks, fused split merge)", "bound": "hbm",
                 "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": recorded_traffic("attend_mma", args.config),
+                "frac": achieved / peaks["hbm_gbs"], "traffic": recorded_traffic("attend_mma", args.config if args.batch is None else None),
                 "peak_source": src + " (burst copy)", "us_per_launch": per_launch_s * 1e6,
                 "algorithmic_bytes_per_launch": bench.bytes_per_step,
                 "bytes_per_unit": bench.kv_bytes, "units_per_launch": bench.keys_per_step}

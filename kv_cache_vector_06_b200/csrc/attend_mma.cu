@@ -79,6 +79,32 @@ __device__ __forceinline__ float dither(uint32_t x) {
 // FMA pipe instead of a float-to-integer conversion.  The result's bytes 0 and 1 are floor(v)'s.
 __device__ __forceinline__ uint32_t floor_bits(float v) { return __float_as_uint(__fadd_rd(v, 8388608.f)); }
 
+// Two fp32 FMAs in one packed instruction (f32x2): d_i = a_i b + c_i, each rounded as fmaf.
+__device__ __forceinline__ void fma2(float a0, float a1, float b, float c0, float c1, float &d0, float &d1) {
+  uint64_t r;
+  asm("{\n .reg .b64 pa, pb, pc;\n mov.b64 pa, {%1, %2};\n mov.b64 pb, {%3, %3};\n mov.b64 pc, {%4, %5};\n"
+      " fma.rn.f32x2 %0, pa, pb, pc;\n}"
+      : "=l"(r)
+      : "r"(__float_as_uint(a0)), "r"(__float_as_uint(a1)), "r"(__float_as_uint(b)), "r"(__float_as_uint(c0)),
+        "r"(__float_as_uint(c1)));
+  d0 = __uint_as_float((uint32_t)r);
+  d1 = __uint_as_float((uint32_t)(r >> 32));
+}
+
+// floor_bits(fmaf(w_i, c, z_i)) for a pair, in two packed instructions.
+__device__ __forceinline__ void fma_floor2(float w0, float w1, float c, float z0, float z1, uint32_t &x0,
+                                           uint32_t &x1) {
+  uint64_t r;
+  asm("{\n .reg .b64 pa, pb, pc, pm, pt;\n mov.b64 pa, {%1, %2};\n mov.b64 pb, {%3, %3};\n"
+      " mov.b64 pc, {%4, %5};\n fma.rn.f32x2 pt, pa, pb, pc;\n mov.b64 pm, {%6, %6};\n"
+      " add.rm.f32x2 %0, pt, pm;\n}"
+      : "=l"(r)
+      : "r"(__float_as_uint(w0)), "r"(__float_as_uint(w1)), "r"(__float_as_uint(c)), "r"(__float_as_uint(z0)),
+        "r"(__float_as_uint(z1)), "r"(0x4B000000u));
+  x0 = (uint32_t)r;
+  x1 = (uint32_t)(r >> 32);
+}
+
 __device__ __forceinline__ int64_t token_slot(const MmaArgs &a, int b, int h, int t) {
   if (a.block_table) {
     const int blk = a.block_table[(int64_t)b * a.max_blocks + t / a.block_size];
@@ -720,21 +746,33 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
         for (int kb = 0; kb < 2; ++kb) {
           const int blk = 2 * warp + kb;
           const bool bok = vb[blk] >= 0;
-#pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            const int i = blk * 16 + gid + 8 * r;
-            const float dc = (float)acc[kb][0][0][2 * r] + 256.f * (float)acc[kb][0][0][2 * r + 1] +
-                             65536.f * (float)acc[kb][0][1][2 * r] + 16777216.f * (float)acc[kb][0][1][2 * r + 1];
-            float sc2 = fmaf(dc, kcs[t], -kcs[8 + t]);
-            if constexpr (QJL) {
-              const float ds = (float)acc[kb][1][0][2 * r] + 256.f * (float)acc[kb][1][0][2 * r + 1] +
-                               65536.f * (float)acc[kb][1][1][2 * r] + 16777216.f * (float)acc[kb][1][1][2 * r + 1];
-              sc2 = fmaf(kc.qjl_scale * skr[i], fmaf(ds, kcs[4 + t], -kcs[12 + t]), sc2);
-            }
-            const bool okt = bok && tk0 + i < t1;
-            lgt[kb][r] = okt ? a.scale * skn[i] * sc2 : -INFINITY;
-            nvk[kb][r] = okt ? svn[i] : 0.f;  // masked slots may hold stale bytes
+          // the four limbs of each of the two tokens (gid, gid + 8) combined in pairs
+          const int i0 = blk * 16 + gid, i1 = i0 + 8;
+          float dc0, dc1, sc0, sc1;
+          {
+            const int (&A)[4] = acc[kb][0][0];
+            const int (&B)[4] = acc[kb][0][1];
+            fma2((float)A[1], (float)A[3], 256.f, (float)A[0], (float)A[2], dc0, dc1);
+            fma2((float)B[0], (float)B[2], 65536.f, dc0, dc1, dc0, dc1);
+            fma2((float)B[1], (float)B[3], 16777216.f, dc0, dc1, dc0, dc1);
+            fma2(dc0, dc1, kcs[t], -kcs[8 + t], -kcs[8 + t], sc0, sc1);
           }
+          if constexpr (QJL) {
+            const int (&A)[4] = acc[kb][1][0];
+            const int (&B)[4] = acc[kb][1][1];
+            float ds0, ds1;
+            fma2((float)A[1], (float)A[3], 256.f, (float)A[0], (float)A[2], ds0, ds1);
+            fma2((float)B[0], (float)B[2], 65536.f, ds0, ds1, ds0, ds1);
+            fma2((float)B[1], (float)B[3], 16777216.f, ds0, ds1, ds0, ds1);
+            fma2(ds0, ds1, kcs[4 + t], -kcs[12 + t], -kcs[12 + t], ds0, ds1);
+            sc0 = fmaf(kc.qjl_scale * skr[i0], ds0, sc0);
+            sc1 = fmaf(kc.qjl_scale * skr[i1], ds1, sc1);
+          }
+          const bool ok0 = bok && tk0 + i0 < t1, ok1 = bok && tk0 + i1 < t1;
+          lgt[kb][0] = ok0 ? a.scale * skn[i0] * sc0 : -INFINITY;
+          lgt[kb][1] = ok1 ? a.scale * skn[i1] * sc1 : -INFINITY;
+          nvk[kb][0] = ok0 ? svn[i0] : 0.f;  // masked slots may hold stale bytes
+          nvk[kb][1] = ok1 ? svn[i1] : 0.f;
         }
       }
 
@@ -815,10 +853,9 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
 #pragma unroll
           for (int rr = 0; rr < 2; ++rr) {
             const int i0 = 2 * rr, i1 = 2 * rr + 1;  // the two tokens of this register
-            const uint32_t x0 = floor_bits(fmaf(W[i0], C[2 * x], dz[i0]));
-            const uint32_t x1 = floor_bits(fmaf(W[i1], C[2 * x], dz[i1]));
-            const uint32_t x2 = floor_bits(fmaf(W[i0], C[2 * x + 1], dz[i0]));
-            const uint32_t x3 = floor_bits(fmaf(W[i1], C[2 * x + 1], dz[i1]));
+            uint32_t x0, x1, x2, x3;
+            fma_floor2(W[i0], W[i1], C[2 * x], dz[i0], dz[i1], x0, x1);
+            fma_floor2(W[i0], W[i1], C[2 * x + 1], dz[i0], dz[i1], x2, x3);
             bfr[kk][2 * x + rr] = __byte_perm(__byte_perm(x0, x1, sel), __byte_perm(x2, x3, sel), 0x5410);
             xs += (x0 + x1) + (x2 + x3) - 4u * 0x4B000000u;  // the integers themselves
           }
@@ -865,13 +902,14 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
       }
       // accv[mt]: c0/c1 = (coordinate 16 gid + 2 mt, head t, limb 0/1), c2/c3 = (+1, ...):
       // 128 sum_tok X b; with s = 2b - 1 the codebook's constant term is -(1/2) sum X
+      const float ct2 = -cterm * inv;
 #pragma unroll
-      for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const float v = (float)accv[mt][2 * r] + 256.f * (float)accv[mt][2 * r + 1];
-          o[2 * mt + r] = fmaf(o[2 * mt + r], al, (v - cterm) * inv);
-        }
+      for (int mt = 0; mt < 8; ++mt) {
+        float v0, v1, u0, u1;
+        fma2((float)accv[mt][1], (float)accv[mt][3], 256.f, (float)accv[mt][0], (float)accv[mt][2], v0, v1);
+        fma2(v0, v1, inv, ct2, ct2, u0, u1);
+        fma2(o[2 * mt], o[2 * mt + 1], al, u0, u1, o[2 * mt], o[2 * mt + 1]);
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive1(&empty[st]);
     }

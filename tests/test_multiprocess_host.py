@@ -92,3 +92,28 @@ def test_search_reference_arm_prints_one_contract_line(capsys):
     assert rec["e2e"] == {"value": rec["value"], "unit": "queries/s", "h2d_bytes_per_step": 0,
                           "d2h_bytes_per_step": 0}
     assert rec["config"]["rows"] == 1_000_000 and rec["config"]["k"] == 10
+
+
+def test_ragged_caches_share_lengths_and_cover_every_block():
+    """Every cache of the paged workload maps each sequence's positions to its own distinct, valid
+    physical blocks (so no step reads a block twice or outside the cache), and the caches differ
+    only in the permutation."""
+    import torch
+
+    import bench
+    import synth
+    cfg = dict(bench.CONFIGS["ragged"])
+    lens, table0, nblocks = bench.ragged_layout(cfg, 1102)
+    seen_tables = []
+    for ci in range(cfg["caches"]):
+        tab = bench.cache_block_table(lens, 1102, ci)
+        if ci == 0:
+            assert torch.equal(tab, table0)
+        used = []
+        for b, L in enumerate(lens.tolist()):
+            k = (L + synth.BLOCK_TOKENS - 1) // synth.BLOCK_TOKENS
+            used.extend(tab[b, :k].tolist())
+        assert len(used) == nblocks and len(set(used)) == nblocks
+        assert min(used) >= 0 and max(used) < nblocks
+        seen_tables.append(tab)
+    assert not torch.equal(seen_tables[0], seen_tables[1])
