@@ -365,9 +365,9 @@ cudaError_t launch_tpr_dt(const TqConsts &c, const TprArgs &a, cudaStream_t st) 
 // norm follows from ||y|| = sqrt(d) ||x||, and the thresholds are scaled by ||y||.
 //
 // Keys with a dense Gaussian JL matrix (m = d = 128) then form z = S r on the tensor cores as three
-// TF32 products (r_hi S_hi + r_hi S_lo + r_lo S_hi, each operand split as x = tf32(x) +
-// (x - tf32(x)); the dropped r_lo S_lo term is below 2^-22 of the products), which keeps z within
-// a few fp32 ulps of the fp32 dot product:
+// TF32 products (r_hi S_hi + r_hi S_lo + r_lo S_hi, each operand split as x = head + (x - head),
+// the head being x with its low 13 mantissa bits cleared; the dropped r_lo S_lo term is below
+// 2^-20 of the products), which keeps z within about 2^-20 of the fp32 dot product's scale:
 //   A = the tile's residual rows, written by their own threads into tensor memory (lane = row,
 //       one column per coordinate): r_hi for the first two products, then r_lo in the same
 //       columns for the third;
@@ -539,12 +539,12 @@ encode_tc_kernel(TqConsts c, TprArgs a) {
     for (int idx = tid; idx < kTD * kTD; idx += kQThreads) {
       const int n = idx / kTD, k = idx % kTD;
       const float sv = c.S[idx];
-      const uint32_t hi = to_tf32(sv);
+      const uint32_t hi = tf32_head(sv);
       const float lo = sv - __uint_as_float(hi);
       const uint32_t off = (uint32_t)(n >> 3) * kQSbo + (uint32_t)(k >> 2) * kQLbo + (uint32_t)(n & 7) * 16 +
                            (uint32_t)(k & 3) * 4;
       *reinterpret_cast<uint32_t *>(smem + SM::shi + off) = hi;
-      *reinterpret_cast<uint32_t *>(smem + SM::slo + off) = to_tf32(lo);
+      *reinterpret_cast<uint32_t *>(smem + SM::slo + off) = __float_as_uint(lo);
     }
   }
   if (tid < TQ_MAX_LEVELS) cen[tid] = c.centroids[tid];
@@ -721,21 +721,59 @@ encode_tc_kernel(TqConsts c, TprArgs a) {
         float T[L - 1];
 #pragma unroll
         for (int k = 0; k < L - 1; ++k) T[k] = c.thresholds[k] * scl;
-#pragma unroll
-        for (int P = 0; P < BITS; ++P)
-#pragma unroll
-          for (int q = 0; q < kHW; ++q) w[P][q] = 0u;
         float rr = 0.f;
+        if constexpr (BITS <= 2) {
+          // one or two bits: a thermometer word per threshold (code = the number of thresholds
+          // passed) and the centroid selected by the same comparisons; the planes are the count's
+          // bits (bit 1 = the middle threshold, bit 0 = the parity of the three)
+          float cl[L];
 #pragma unroll
-        for (int jj = 0; jj < kHalf; ++jj) {
-          int code = 0;
+          for (int k = 0; k < L; ++k) cl[k] = c.centroids[k];
+          uint32_t tw[L - 1][kHW];
 #pragma unroll
-          for (int k = 0; k < L - 1; ++k) code += v[jj] >= T[k] ? 1 : 0;
+          for (int k = 0; k < L - 1; ++k)
 #pragma unroll
-          for (int P = 0; P < BITS; ++P) w[P][jj >> 5] |= (uint32_t)((code >> P) & 1) << (jj & 31);
-          const float r = fmaf(v[jj], inv, -cen[code]);
-          v[jj] = r;
-          rr = fmaf(r, r, rr);
+            for (int q = 0; q < kHW; ++q) tw[k][q] = 0u;
+#pragma unroll
+          for (int jj = 0; jj < kHalf; ++jj) {
+            const float y = v[jj];
+            const uint32_t bit = 1u << (jj & 31);
+            float cc = cl[0];
+#pragma unroll
+            for (int k = 0; k < L - 1; ++k) {
+              const bool ge = y >= T[k];
+              if (ge) tw[k][jj >> 5] |= bit;
+              cc = ge ? cl[k + 1] : cc;
+            }
+            const float r = fmaf(y, inv, -cc);
+            v[jj] = r;
+            rr = fmaf(r, r, rr);
+          }
+#pragma unroll
+          for (int q = 0; q < kHW; ++q) {
+            if constexpr (BITS == 1) {
+              w[0][q] = tw[0][q];
+            } else {
+              w[1][q] = tw[1][q];
+              w[0][q] = tw[0][q] ^ tw[1][q] ^ tw[2][q];
+            }
+          }
+        } else {
+#pragma unroll
+          for (int P = 0; P < BITS; ++P)
+#pragma unroll
+            for (int q = 0; q < kHW; ++q) w[P][q] = 0u;
+#pragma unroll
+          for (int jj = 0; jj < kHalf; ++jj) {
+            int code = 0;
+#pragma unroll
+            for (int k = 0; k < L - 1; ++k) code += v[jj] >= T[k] ? 1 : 0;
+#pragma unroll
+            for (int P = 0; P < BITS; ++P) w[P][jj >> 5] |= (uint32_t)((code >> P) & 1) << (jj & 31);
+            const float r = fmaf(v[jj], inv, -cen[code]);
+            v[jj] = r;
+            rr = fmaf(r, r, rr);
+          }
         }
         group_sync(g);  // both halves have read the norm partials
         *myx = rr;
@@ -756,7 +794,7 @@ encode_tc_kernel(TqConsts c, TprArgs a) {
           uint32_t hv[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            hv[e] = to_tf32(v[16 * cb + e]);
+            hv[e] = tf32_head(v[16 * cb + e]);
             v[16 * cb + e] -= __uint_as_float(hv[e]);  // r_lo from here on (exact in fp32)
           }
           tmem_st16(abase + 16u * cb, hv);

@@ -71,13 +71,11 @@ __device__ __forceinline__ void umma_tf32_ta(uint32_t dtmem, uint32_t atmem, uin
       : "memory");
 }
 
-// fp32 -> tf32 rounded to nearest (ties away from zero), as a 32-bit pattern with the low 13 bits
-// clear
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return r;
-}
+// The tf32 head of an fp32 value by truncation: its bit pattern with the low 13 mantissa bits clear
+// (one logic op).  x - head is exact in fp32 and below 2^-10 |x|; a TF32 MMA reads an fp32 operand
+// the same way (the low 13 bits ignored), so the two-term split x = head + (x - head) keeps about
+// 21 significant bits through the products.
+__device__ __forceinline__ uint32_t tf32_head(float x) { return __float_as_uint(x) & 0xFFFFE000u; }
 
 // kind::f16 with both operands in shared memory (descriptors): D (f32, tensor memory) += A x B^T,
 // A and B bf16 per the instruction descriptor, K = 16 elements per MMA; accum = 0 overwrites D
