@@ -79,58 +79,59 @@ __device__ __forceinline__ void tpr_load(const unsigned char *rowp, float (&v)[k
 }
 
 // Codes by the codebook's symmetry.  The thresholds are antisymmetric (t_(L-2-k) = -t_k, the middle
-// one 0), so with the H = L/2 - 1 positive ones t+_k:
-//   code = L/2 + #{k : |y| >= t+_k}        for y >= 0,
-//   code = L/2 - 1 - #{k : |y| > t+_k}     for y < 0,
+// one 0), so with the H = L/2 - 1 positive ones t+_k and cnt = #{k : |y| >= t+_k}:
+//   code = L/2 + cnt                       for y >= 0,
+//   code = L/2 - 1 - cnt (= ~cnt mod L/2)    for y < 0 (with > in place of >=),
 // the same count as #{i : t_i <= y} (ties go up).  The strict comparison of a negative y is the
-// non-strict one on the float just below |y|.  Each comparison sets bit j of a word of its own (a
-// thermometer code), and the bit planes of the code are XORs of those words: half the
-// comparisons of the plain count and no per-coordinate bit extraction.
+// non-strict one on the float just below |y|.  cnt's b - 1 bits come from a binary search over
+// the positive thresholds (b - 1 comparisons), each setting bit j of a word of its own; the code's
+// bit planes are then the sign word and the count words complemented where y < 0.
 template <int BITS>
 struct Sym {
-  static constexpr int H = (1 << (BITS - 1)) - 1;
+  static constexpr int H = (1 << (BITS - 1)) - 1;  // positive thresholds
   static constexpr int HW = H > 0 ? H : 1;
+  static constexpr int CW = BITS > 1 ? BITS - 1 : 1;  // count words
 };
 
-// One coordinate j (of the NW 32-bit words a thread packs): sets bit j of the sign word and of the
-// thermometer words; returns the code.
+// One coordinate j (of the NW 32-bit words a thread packs): bit j of the sign word and of the count
+// words.
 template <int BITS, int NW>
-__device__ __forceinline__ int sym_quant(float y, const float (&Tp)[Sym<BITS>::HW], uint32_t (&sw)[NW],
-                                         uint32_t (&tw)[Sym<BITS>::HW][NW], int j) {
-  constexpr int L = 1 << BITS;
+__device__ __forceinline__ void sym_quant(float y, const float (&Tp)[Sym<BITS>::HW], uint32_t (&sw)[NW],
+                                          uint32_t (&cw)[Sym<BITS>::CW][NW], int j) {
   const bool pos = y >= 0.f;
   const uint32_t bit = 1u << (j & 31);
   if (pos) sw[j >> 5] |= bit;
-  const float a = __uint_as_float((__float_as_uint(y) & 0x7fffffffu) - (pos ? 0u : 1u));
-  int cnt = 0;
-#pragma unroll
-  for (int k = 0; k < Sym<BITS>::H; ++k) {
-    const bool ge = a >= Tp[k];
-    if (ge) tw[k][j >> 5] |= bit;
-    cnt += ge ? 1 : 0;
+  if constexpr (BITS >= 2) {
+    const float a = __uint_as_float((__float_as_uint(y) & 0x7fffffffu) - (pos ? 0u : 1u));
+    if constexpr (BITS == 2) {
+      if (a >= Tp[0]) cw[0][j >> 5] |= bit;
+    } else if constexpr (BITS == 3) {
+      const bool b1 = a >= Tp[1];
+      const bool b0 = a >= (b1 ? Tp[2] : Tp[0]);
+      if (b1) cw[1][j >> 5] |= bit;
+      if (b0) cw[0][j >> 5] |= bit;
+    } else {
+      const bool b2 = a >= Tp[3];
+      const bool b1 = a >= (b2 ? Tp[5] : Tp[1]);
+      const bool b0 = a >= (b2 ? (b1 ? Tp[6] : Tp[4]) : (b1 ? Tp[2] : Tp[0]));
+      if (b2) cw[2][j >> 5] |= bit;
+      if (b1) cw[1][j >> 5] |= bit;
+      if (b0) cw[0][j >> 5] |= bit;
+    }
   }
-  return pos ? L / 2 + cnt : L / 2 - 1 - cnt;
 }
 
-// The code's bit planes from the sign word s and the thermometer words: plane BITS - 1 is s; the
-// lower planes are the bits of the count, complemented where y < 0.
+// The code's bit planes: plane BITS - 1 is the sign word; the lower planes are the count's bits,
+// complemented where y < 0.
 template <int BITS, int NW>
-__device__ __forceinline__ void sym_planes(const uint32_t (&sw)[NW], const uint32_t (&tw)[Sym<BITS>::HW][NW],
+__device__ __forceinline__ void sym_planes(const uint32_t (&sw)[NW], const uint32_t (&cw)[Sym<BITS>::CW][NW],
                                            uint32_t (&w)[BITS][NW]) {
 #pragma unroll
   for (int q = 0; q < NW; ++q) {
     const uint32_t n = ~sw[q];
     w[BITS - 1][q] = sw[q];
-    if constexpr (BITS == 2) w[0][q] = tw[0][q] ^ n;
-    if constexpr (BITS == 3) {
-      w[1][q] = tw[1][q] ^ n;
-      w[0][q] = tw[0][q] ^ tw[1][q] ^ tw[2][q] ^ n;
-    }
-    if constexpr (BITS == 4) {
-      w[2][q] = tw[3][q] ^ n;
-      w[1][q] = tw[1][q] ^ tw[3][q] ^ tw[5][q] ^ n;
-      w[0][q] = tw[0][q] ^ tw[1][q] ^ tw[2][q] ^ tw[3][q] ^ tw[4][q] ^ tw[5][q] ^ tw[6][q] ^ n;
-    }
+#pragma unroll
+    for (int k = 0; k < BITS - 1; ++k) w[k][q] = cw[k][q] ^ n;
   }
 }
 
@@ -278,12 +279,12 @@ encode_tpr_kernel(TqConsts c, TprArgs a) {
         rr = fmaf(r, r, rr);
       }
     } else {
-      uint32_t sw[kTD / 32], tw[Sym<BITS>::HW][kTD / 32];
+      uint32_t sw[kTD / 32], tw[Sym<BITS>::CW][kTD / 32];
 #pragma unroll
       for (int q = 0; q < kTD / 32; ++q) {
         sw[q] = 0u;
 #pragma unroll
-        for (int k = 0; k < Sym<BITS>::HW; ++k) tw[k][q] = 0u;
+        for (int k = 0; k < Sym<BITS>::CW; ++k) tw[k][q] = 0u;
       }
 #pragma unroll
       for (int j = 0; j < kTD; ++j) sym_quant<BITS, kTD / 32>(v[j], T, sw, tw, j);
@@ -823,12 +824,12 @@ encode_tc_kernel(TqConsts c, TprArgs a) {
         float T[Sym<BITS>::HW];
 #pragma unroll
         for (int k = 0; k < Sym<BITS>::H; ++k) T[k] = thr[k] * scl;
-        uint32_t sw[kHW], tw[Sym<BITS>::HW][kHW];
+        uint32_t sw[kHW], tw[Sym<BITS>::CW][kHW];
 #pragma unroll
         for (int q = 0; q < kHW; ++q) {
           sw[q] = 0u;
 #pragma unroll
-          for (int k = 0; k < Sym<BITS>::HW; ++k) tw[k][q] = 0u;
+          for (int k = 0; k < Sym<BITS>::CW; ++k) tw[k][q] = 0u;
         }
 #pragma unroll
         for (int jj = 0; jj < kHalf; ++jj) sym_quant<BITS, kHW>(v[jj], T, sw, tw, jj);
