@@ -63,7 +63,12 @@ typedef struct {
   int32_t d;
   int32_t mse_bits;
   int32_t qjl_m;
-  int32_t layout;   /* tq_layout of the packed codes (TQ_LAYOUT_ROWS unless stated) */
+  int32_t layout;     /* tq_layout of the packed codes (TQ_LAYOUT_ROWS unless stated) */
+  int32_t norm_bits;  /* storage of norm and rnorm: 32 (or 0) = fp32, 16 = fp16 (IEEE half, round
+                         to nearest, values above 65504 stored as 65504).  The norms are the only
+                         per-vector constants, and quantizers keep such constants in FP16 or FP32
+                         ([JJ] 第一部分); fp16 saves 4 bytes per vector with a QJL stage, 0.25 bit
+                         per coordinate at d = 128. */
 } tq_spec;
 
 /* Packed-code layouts.
@@ -83,14 +88,16 @@ typedef enum { TQ_LAYOUT_ROWS = 0, TQ_LAYOUT_BLOCK16 = 1 } tq_layout;
  *                                  bit t of code_j is bit (t*d + j) of the vector's
  *                                  little-endian bit stream; padded to a multiple of 16 bytes.
  *   signs  [capacity][sign_bytes]  QJL bits, bit i = [ (S r)_i >= 0 ]; NULL when qjl_m == 0.
- *   norm   [capacity]  fp32 ||x||
- *   rnorm  [capacity]  fp32 ||r||, r the rotated-domain residual; NULL when qjl_m == 0.
- * code_bytes = roundup(b*d/8, 16), sign_bytes = roundup(m/8, 16) (tq_ctx_layout). */
+ *   norm   [capacity]  ||x||, fp32 or fp16 per tq_spec.norm_bits (4- or 2-byte aligned)
+ *   rnorm  [capacity]  ||r||, r the rotated-domain residual, same type; NULL when qjl_m == 0.
+ * code_bytes = roundup(b*d/8, 16), sign_bytes = roundup(m/8, 16) (tq_ctx_layout).  The
+ * tensor-core attention path also wants the norm arrays 16-byte aligned (it copies them in bulk);
+ * other alignments take the general path. */
 typedef struct {
   void *codes;
   void *signs;
-  float *norm;
-  float *rnorm;
+  void *norm;
+  void *rnorm;
   int64_t capacity;
 } tq_packed;
 

@@ -30,8 +30,13 @@ tq_status check_spec(const tq_spec *s) {
     return tq_fail(TQ_EINVAL, "layout=%d: unknown", s->layout);
   if (s->layout == TQ_LAYOUT_BLOCK16 && s->qjl_m != 0)
     return tq_fail(TQ_EUNSUPPORTED, "TQ_LAYOUT_BLOCK16 holds MSE-only codes (qjl_m must be 0)");
+  if (s->norm_bits != 0 && s->norm_bits != 16 && s->norm_bits != 32)
+    return tq_fail(TQ_EINVAL, "norm_bits=%d: must be 32 (or 0) or 16", s->norm_bits);
   return TQ_OK;
 }
+
+// Address of stored norm i (fp16 or fp32 per the context).
+void *norm_at(const tq_ctx *c, void *p, int64_t i) { return static_cast<char *>(p) + i * (c->k.norm16 ? 2 : 4); }
 
 tq_status check_ctx(const tq_ctx *c, const char *name) {
   if (!c) return tq_fail(TQ_EINVAL, "%s is NULL", name);
@@ -43,13 +48,14 @@ tq_status check_packed(const tq_ctx *c, const tq_packed &p, int64_t need, const 
                        bool need_signs) {
   if (!p.codes || !p.norm) return tq_fail(TQ_EINVAL, "%s: codes/norm is NULL", name);
   if (!aligned16(p.codes)) return tq_fail(TQ_EINVAL, "%s: codes not 16-byte aligned", name);
-  if ((reinterpret_cast<uintptr_t>(p.norm) & 3u) != 0)
-    return tq_fail(TQ_EINVAL, "%s: norm not 4-byte aligned", name);
+  const uintptr_t nal = c->k.norm16 ? 1u : 3u;  // fp16 or fp32 norms
+  if ((reinterpret_cast<uintptr_t>(p.norm) & nal) != 0)
+    return tq_fail(TQ_EINVAL, "%s: norm not %d-byte aligned", name, (int)nal + 1);
   if (need_signs && c->spec.qjl_m > 0) {
     if (!p.signs || !p.rnorm) return tq_fail(TQ_EINVAL, "%s: signs/rnorm is NULL", name);
     if (!aligned16(p.signs)) return tq_fail(TQ_EINVAL, "%s: signs not 16-byte aligned", name);
-    if ((reinterpret_cast<uintptr_t>(p.rnorm) & 3u) != 0)
-      return tq_fail(TQ_EINVAL, "%s: rnorm not 4-byte aligned", name);
+    if ((reinterpret_cast<uintptr_t>(p.rnorm) & nal) != 0)
+      return tq_fail(TQ_EINVAL, "%s: rnorm not %d-byte aligned", name, (int)nal + 1);
   }
   if (p.capacity < 0) return tq_fail(TQ_EINVAL, "%s: negative capacity", name);
   if (c->spec.layout == TQ_LAYOUT_BLOCK16 && (p.capacity % 16) != 0)
@@ -200,6 +206,7 @@ static tq_status ctx_create(const tq_spec *spec, const int8_t *rot_signs, const 
   k.code_words = (int)(c->code_bytes / 4);
   k.sign_words = (int)(c->sign_bytes / 4);
   k.layout = spec->layout;
+  k.norm16 = spec->norm_bits == 16 ? 1 : 0;
   k.inv_sqrt_d = (float)(1.0 / std::sqrt((double)d));
   k.qjl_scale = m > 0 ? (float)(std::sqrt(M_PI / 2.0) / m) : 0.0f;
   for (int i = 0; i < TQ_MAX_LEVELS; ++i) {
@@ -372,10 +379,10 @@ tq_status tq_encode_kv(const tq_ctx *ctx, const void *x, tq_dtype dtype, int64_t
       tq_packed o = out;
       if (!slots) {
         o.codes = static_cast<char *>(out.codes) + r0 * ctx->code_bytes;
-        o.norm = out.norm + r0;
+        o.norm = norm_at(ctx, out.norm, r0);
         if (qjl) {
           o.signs = static_cast<char *>(out.signs) + r0 * ctx->sign_bytes;
-          o.rnorm = out.rnorm + r0;
+          o.rnorm = norm_at(ctx, out.rnorm, r0);
         }
         o.capacity = out.capacity - r0;
       }
@@ -396,7 +403,7 @@ tq_status tq_encode_kv(const tq_ctx *ctx, const void *x, tq_dtype dtype, int64_t
     if (e != cudaSuccess || nt == n) return tq_cuda_check(e, "encode launch");
     // the ragged tail of a token-block layout (rows nt.. go to slots nt..; nt is a whole block)
     e = launch_rotate(ctx->k, ROT_ENCODE, static_cast<const char *>(x) + nt * ld * esz, dtype, n - nt, ld, nullptr,
-                      out.capacity - nt, static_cast<uint32_t *>(out.codes) + nt * (ctx->code_bytes / 4), out.norm + nt,
+                      out.capacity - nt, static_cast<uint32_t *>(out.codes) + nt * (ctx->code_bytes / 4), norm_at(ctx, out.norm, nt),
                       nullptr, nullptr, s);
     return tq_cuda_check(e, "encode launch");
   }
@@ -422,10 +429,10 @@ tq_status tq_encode_kv(const tq_ctx *ctx, const void *x, tq_dtype dtype, int64_t
     tq_packed o = out;
     if (!slots) {
       o.codes = static_cast<char *>(out.codes) + r0 * ctx->code_bytes;
-      o.norm = out.norm + r0;
+      o.norm = norm_at(ctx, out.norm, r0);
       if (qjl) {
         o.signs = static_cast<char *>(out.signs) + r0 * ctx->sign_bytes;
-        o.rnorm = out.rnorm + r0;
+        o.rnorm = norm_at(ctx, out.rnorm, r0);
       }
       o.capacity = out.capacity - r0;
     }
@@ -697,7 +704,7 @@ tq_status tq_search_topk(const tq_ctx *ctx, const void *q, tq_dtype dtype, int32
   // scan: tcgen05 (many queries), else the bit-plane mma.sync scan, else CUDA cores
   const bool tc = search_tc_eligible(ctx->k, nq, k);
   const bool mma = !tc && search_mma_eligible(ctx->k) && nq <= kSearchMmaMaxQ && aligned16(db.norm) &&
-                   aligned16(db.rnorm);
+                   aligned16(db.rnorm) && !ctx->k.norm16;  // that scan copies fp32 norms in bulk
   const SearchPlan plan = search_plan(nq, n, k);
   const int shards = tc ? search_tc_shards(nq, n) : mma ? search_mma_shards(ctx->k, nq, n, k) : plan.shards;
   const int64_t cands = (int64_t)nq * shards * k;

@@ -103,11 +103,11 @@ attend_split_kernel(TqConsts kc, TqConsts vc, AttnArgs a, const float *__restric
     float nuv = 0.f;
     if (ok) {
       estimate_scores<G>(kc, kcodes + slot * kc.code_words,
-                         m > 0 ? ksigns + slot * kc.sign_words : nullptr, a.k.norm[slot],
-                         m > 0 ? a.k.rnorm[slot] : 0.f, qs, ps, centK, sc);
+                         m > 0 ? ksigns + slot * kc.sign_words : nullptr, ld_norm(a.k.norm, slot, kc.norm16),
+                         m > 0 ? ld_norm(a.k.rnorm, slot, kc.norm16) : 0.f, qs, ps, centK, sc);
 #pragma unroll
       for (int g = 0; g < G; ++g) sc[g] *= a.scale;
-      nuv = a.v.norm[slot];
+      nuv = ld_norm(a.v.norm, slot, vc.norm16);
     } else {
 #pragma unroll
       for (int g = 0; g < G; ++g) sc[g] = -INFINITY;

@@ -49,7 +49,13 @@ struct MmaArgs {
   int *counter;  // per (sequence, KV head): CTAs done (zeroed by the query-fragment kernel)
   float *out;    // final output when the kernel merges its splits itself, else null
   float sparse_v;  // Sparse V threshold on the softmax weights (0 = off)
+  int kn4, vn4;    // log2 of the bytes of one stored K / V norm: 2 (fp32) or 1 (fp16)
 };
+
+// Norm i of a staged array (fp32 or fp16, `l2` = log2 of its bytes).
+__device__ __forceinline__ float staged_norm(const unsigned char *base, int i, int l2) {
+  return l2 == 1 ? __half2float(reinterpret_cast<const __half *>(base)[i]) : reinterpret_cast<const float *>(base)[i];
+}
 
 __device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
@@ -509,10 +515,10 @@ __device__ __forceinline__ void stage_array(const MmaArgs &a, int arr, const cha
   switch (arr) {
     case 0: src = static_cast<const char *>(a.k.codes); doff = SM::kc; per = 16 * SM::KCW * 4; sstride = SM::KCW * 4; break;
     case 1: src = static_cast<const char *>(a.v.codes); doff = SM::vc; per = SM::VBW * 4; sstride = SM::VBW * 4 / 16; break;
-    case 2: src = reinterpret_cast<const char *>(a.k.norm); doff = SM::kn; per = 64; sstride = 4; break;
-    case 3: src = reinterpret_cast<const char *>(a.v.norm); doff = SM::vn; per = 64; sstride = 4; break;
+    case 2: src = static_cast<const char *>(a.k.norm); doff = SM::kn; per = 16u << a.kn4; sstride = 1 << a.kn4; break;
+    case 3: src = static_cast<const char *>(a.v.norm); doff = SM::vn; per = 16u << a.vn4; sstride = 1 << a.vn4; break;
     case 4: src = static_cast<const char *>(a.k.signs); doff = SM::ks; per = 256; sstride = 16; break;
-    default: src = reinterpret_cast<const char *>(a.k.rnorm); doff = SM::kr; per = 64; sstride = 4; break;
+    default: src = static_cast<const char *>(a.k.rnorm); doff = SM::kr; per = 16u << a.kn4; sstride = 1 << a.kn4; break;
   }
 }
 
@@ -694,10 +700,9 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
       const unsigned char *sb = smem + (size_t)st * SM::buf;
       const uint32_t *skc = reinterpret_cast<const uint32_t *>(sb + SM::kc);
       const uint32_t *sks = reinterpret_cast<const uint32_t *>(sb + SM::ks);
-      const float *skn = reinterpret_cast<const float *>(sb + SM::kn);
-      const float *skr = reinterpret_cast<const float *>(sb + SM::kr);
+      const unsigned char *skn = sb + SM::kn, *skr = sb + SM::kr;
       const uint32_t *svc = reinterpret_cast<const uint32_t *>(sb + SM::vc);
-      const float *svn = reinterpret_cast<const float *>(sb + SM::vn);
+      const unsigned char *svn = sb + SM::vn;
       const int64_t *vb = vball + NB * sc;  // validity of this sub-chunk's blocks
       const int tk0 = t0 + sc * kSub;
 
@@ -765,14 +770,14 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
             fma2((float)B[0], (float)B[2], 65536.f, ds0, ds1, ds0, ds1);
             fma2((float)B[1], (float)B[3], 16777216.f, ds0, ds1, ds0, ds1);
             fma2(ds0, ds1, kcs[4 + t], -kcs[12 + t], -kcs[12 + t], ds0, ds1);
-            sc0 = fmaf(kc.qjl_scale * skr[i0], ds0, sc0);
-            sc1 = fmaf(kc.qjl_scale * skr[i1], ds1, sc1);
+            sc0 = fmaf(kc.qjl_scale * staged_norm(skr, i0, a.kn4), ds0, sc0);
+            sc1 = fmaf(kc.qjl_scale * staged_norm(skr, i1, a.kn4), ds1, sc1);
           }
           const bool ok0 = bok && tk0 + i0 < t1, ok1 = bok && tk0 + i1 < t1;
-          lgt[kb][0] = ok0 ? a.scale * skn[i0] * sc0 : -INFINITY;
-          lgt[kb][1] = ok1 ? a.scale * skn[i1] * sc1 : -INFINITY;
-          nvk[kb][0] = ok0 ? svn[i0] : 0.f;  // masked slots may hold stale bytes
-          nvk[kb][1] = ok1 ? svn[i1] : 0.f;
+          lgt[kb][0] = ok0 ? a.scale * staged_norm(skn, i0, a.kn4) * sc0 : -INFINITY;
+          lgt[kb][1] = ok1 ? a.scale * staged_norm(skn, i1, a.kn4) * sc1 : -INFINITY;
+          nvk[kb][0] = ok0 ? staged_norm(svn, i0, a.vn4) : 0.f;  // masked slots may hold stale bytes
+          nvk[kb][1] = ok1 ? staged_norm(svn, i1, a.vn4) : 0.f;
         }
       }
 
@@ -1169,6 +1174,9 @@ bool attn_fast_eligible(const TqConsts &kc, const TqConsts &vc, const tq_attn_de
   for (int P = 0; P < (vc.bits == 3 ? 4 : vc.bits); ++P)
     if (!(vc.plane_coef[P] >= 0.f)) return false;
   if (desc.block_table ? (desc.block_size % 16) != 0 : (desc.ctx_stride % 16) != 0) return false;
+  // the norm arrays are copied in bulk: 16-byte aligned bases
+  auto a16 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  if (!a16(desc.k.norm) || !a16(desc.v.norm) || (kc.m > 0 && !a16(desc.k.rnorm))) return false;
   return true;
 }
 
@@ -1217,6 +1225,8 @@ cudaError_t launch_attend_fast(const TqConsts &kc, const TqConsts &vc, const tq_
   a.k = desc.k;
   a.v = desc.v;
   a.sparse_v = desc.sparse_v > 0.f ? desc.sparse_v : 0.f;
+  a.kn4 = kc.norm16 ? 1 : 2;
+  a.vn4 = vc.norm16 ? 1 : 2;
   const int planes = (kc.bits + (kc.bits == 3 ? 1 : 0)) + (kc.m > 0 ? 1 : 0);
   const int64_t groups = (int64_t)desc.batch * desc.n_kv_heads;
   uint32_t *kfrag = static_cast<uint32_t *>(extra);
@@ -1287,6 +1297,8 @@ cudaError_t launch_decode_step_fast(const TqConsts &kc, const TqConsts &vc, cons
   a.k = desc.k;
   a.v = desc.v;
   a.sparse_v = desc.sparse_v > 0.f ? desc.sparse_v : 0.f;
+  a.kn4 = kc.norm16 ? 1 : 2;
+  a.vn4 = vc.norm16 ? 1 : 2;
   const int planes = (kc.bits + (kc.bits == 3 ? 1 : 0)) + (kc.m > 0 ? 1 : 0);
   const int64_t groups = (int64_t)desc.batch * desc.n_kv_heads;
   uint32_t *kfrag = static_cast<uint32_t *>(extra);

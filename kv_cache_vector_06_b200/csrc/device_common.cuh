@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -44,6 +45,17 @@ __device__ __forceinline__ uint32_t plane_word(const uint32_t *row, int t, int w
   if (d >= 32) return row[t * (d >> 5) + w];
   const uint64_t v = (uint64_t)row[0] | ((uint64_t)row[1] << 32);
   return (uint32_t)((v >> (t * d)) & ((1ull << d) - 1ull));
+}
+
+// A stored norm (||x|| or ||r||) of slot i: fp16 or fp32 per the context.
+__device__ __forceinline__ float ld_norm(const void *p, int64_t i, int half) {
+  return half ? __half2float(static_cast<const __half *>(p)[i]) : static_cast<const float *>(p)[i];
+}
+__device__ __forceinline__ void st_norm(void *p, int64_t i, float v, int half) {
+  if (half)
+    static_cast<__half *>(p)[i] = __float2half_rn(fminf(v, 65504.f));
+  else
+    static_cast<float *>(p)[i] = v;
 }
 
 // Estimated inner products of NQ prepared queries with one packed key:

@@ -163,7 +163,7 @@ struct TprArgs {
   const int64_t *slots;  // ROWS layout only (NULL: slot = row)
   int64_t capacity;
   uint32_t *codes;
-  float *norm, *rnorm;
+  void *norm, *rnorm;  // fp32 or fp16 (TqConsts::norm16)
   uint32_t *signs;       // structured QJL only
 };
 
@@ -292,7 +292,7 @@ encode_tpr_kernel(TqConsts c, TprArgs a) {
     }
     if constexpr (BLK) {
       store_blk16<BITS>(c, a, w, tile * kTRows + 32 * warp, lane);
-      if (valid) a.norm[row] = nu;
+      if (valid) st_norm(a.norm, row, nu, c.norm16);
     } else {
       const int64_t slot = valid ? (a.slots ? a.slots[row] : row) : -1;
       if (valid && slot >= 0 && slot < a.capacity) {
@@ -300,10 +300,10 @@ encode_tpr_kernel(TqConsts c, TprArgs a) {
         // b planes of 4 words = the row's b * 16 bytes (code_words = 4 b at d = 128)
 #pragma unroll
         for (int P = 0; P < BITS; ++P) dst[P] = make_uint4(w[P][0], w[P][1], w[P][2], w[P][3]);
-        a.norm[slot] = nu;
+        st_norm(a.norm, slot, nu, c.norm16);
         if constexpr (SRHT) {
           // structured QJL: z = H (D2 r), the first m signs
-          a.rnorm[slot] = sqrtf(rr);
+          st_norm(a.rnorm, slot, sqrtf(rr), c.norm16);
 #pragma unroll
           for (int j = 0; j < kTD; j += 4) {
             const float4 s4 = *reinterpret_cast<const float4 *>(sgn2 + j);
@@ -785,8 +785,8 @@ encode_tc_kernel(TqConsts c, TprArgs a) {
 #pragma unroll
           for (int P = 0; P < BITS; ++P) *reinterpret_cast<uint2 *>(dst + 4 * P) = make_uint2(w[P][0], w[P][1]);
           if (h == 0) {
-            a.norm[slot] = nu;
-            a.rnorm[slot] = sqrtf(rr2);
+            st_norm(a.norm, slot, nu, c.norm16);
+            st_norm(a.rnorm, slot, sqrtf(rr2), c.norm16);
           }
         }
         // r_hi -> tensor memory (the columns y came from), then the first two products may start
@@ -836,12 +836,12 @@ encode_tc_kernel(TqConsts c, TprArgs a) {
         sym_planes<BITS, kHW>(sw, tw, w);
         if constexpr (BLK) {
           store_blk16_half<BITS>(c, a, w, tile * kTRows + 32 * quad, lane, h);
-          if (valid && h == 0) a.norm[row] = nu;
+          if (valid && h == 0) st_norm(a.norm, row, nu, c.norm16);
         } else if (store) {
           uint32_t *dst = a.codes + slot * c.code_words + kHW * h;
 #pragma unroll
           for (int P = 0; P < BITS; ++P) *reinterpret_cast<uint2 *>(dst + 4 * P) = make_uint2(w[P][0], w[P][1]);
-          if (h == 0) a.norm[slot] = nu;
+          if (h == 0) st_norm(a.norm, slot, nu, c.norm16);
         }
       }
       if (more) tc_x_ready(g, &b[kBxFull], gi);
@@ -910,7 +910,7 @@ int64_t encode_tpr_rows(const TqConsts &c, int64_t n) {
 }
 
 cudaError_t launch_encode_tpr(const TqConsts &c, const void *x, tq_dtype dtype, int64_t n, int64_t ld,
-                              const int64_t *slots, int64_t capacity, uint32_t *codes, float *norm, float *rnorm,
+                              const int64_t *slots, int64_t capacity, uint32_t *codes, void *norm, void *rnorm,
                               uint32_t *signs, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
   TprArgs a;

@@ -77,7 +77,7 @@ __device__ __forceinline__ void reconstruct(const uint32_t (&w)[4][4], const Pol
 template <int DT, int BITS>
 __global__ void __launch_bounds__(kPRows)
 encode_polar_kernel(TqConsts c, const char *__restrict__ x, int64_t ld_bytes, int64_t n, const int64_t *__restrict__ slots,
-                    int64_t capacity, uint32_t *__restrict__ codes, float *__restrict__ norm, float *__restrict__ rnorm,
+                    int64_t capacity, uint32_t *__restrict__ codes, void *__restrict__ norm, void *__restrict__ rnorm,
                     float *__restrict__ resid) {
   __shared__ PolarTab tab;
   __shared__ float sgn[kPD];
@@ -141,7 +141,7 @@ encode_polar_kernel(TqConsts c, const char *__restrict__ x, int64_t ld_bytes, in
     uint4 *dst = reinterpret_cast<uint4 *>(codes + slot * c.code_words);
 #pragma unroll
     for (int P = 0; P < BITS; ++P) dst[P] = make_uint4(w[P][0], w[P][1], w[P][2], w[P][3]);
-    norm[slot] = nu;
+    st_norm(norm, slot, nu, c.norm16);
   }
   if (resid == nullptr) return;
   // residual r = y / ||x|| - y^ (rotated domain): y^ first, then the row is transformed again
@@ -161,7 +161,7 @@ encode_polar_kernel(TqConsts c, const char *__restrict__ x, int64_t ld_bytes, in
     rr = fmaf(r0, r0, fmaf(r1, r1, fmaf(r2, r2, fmaf(r3, r3, rr))));
     reinterpret_cast<float4 *>(rr_row)[q] = make_float4(r0, r1, r2, r3);
   }
-  if (store) rnorm[slot] = sqrtf(rr);
+  if (store) st_norm(rnorm, slot, sqrtf(rr), c.norm16);
 }
 
 // Estimated inner products with PolarQuant keys: nu ( <q', y^> + sqrt(pi/2)/m gamma <p, 2 b - 1> ).
@@ -205,7 +205,7 @@ scores_polar_kernel(TqConsts c, const float *__restrict__ qr, const float *__res
     for (int q = 0; q < kPQ; ++q) acc[q] = fmaf(qs[j * kPQ + q], t[j], acc[q]);
   float gamma = 0.f;
   if (c.m > 0) {
-    gamma = keys.rnorm[key];
+    gamma = ld_norm(keys.rnorm, key, c.norm16);
     const uint32_t *srow = static_cast<const uint32_t *>(keys.signs) + key * c.sign_words;
     for (int wd = 0; wd < c.m / 32; ++wd) {
       const uint32_t sw = srow[wd];
@@ -217,7 +217,7 @@ scores_polar_kernel(TqConsts c, const float *__restrict__ qr, const float *__res
       }
     }
   }
-  const float nu = keys.norm[key], cg = c.qjl_scale * gamma;
+  const float nu = ld_norm(keys.norm, key, c.norm16), cg = c.qjl_scale * gamma;
 #pragma unroll
   for (int q = 0; q < kPQ; ++q)
     if (q0 + q < nq) out[(int64_t)(q0 + q) * n + key] = nu * fmaf(cg, s2[q], acc[q]);
@@ -228,7 +228,7 @@ scores_polar_kernel(TqConsts c, const float *__restrict__ qr, const float *__res
 bool polar_supported(const TqConsts &c) { return c.d == kPD && c.layout == TQ_LAYOUT_ROWS && c.bits >= 1 && c.bits <= 4; }
 
 cudaError_t launch_encode_polar(const TqConsts &c, const void *x, tq_dtype dtype, int64_t n, int64_t ld,
-                                const int64_t *slots, int64_t capacity, uint32_t *codes, float *norm, float *rnorm,
+                                const int64_t *slots, int64_t capacity, uint32_t *codes, void *norm, void *rnorm,
                                 float *resid, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
   const unsigned grid = (unsigned)((n + kPRows - 1) / kPRows);

@@ -19,7 +19,7 @@ template <int D>
 __global__ void __launch_bounds__(kRotThreads)
 rotate_kernel(TqConsts c, int mode, const void *__restrict__ x, int dtype, int64_t n, int64_t ld,
               const int64_t *__restrict__ slots, int64_t capacity, uint32_t *__restrict__ codes,
-              float *__restrict__ norm, float *__restrict__ rnorm, float *__restrict__ resid,
+              void *__restrict__ norm, void *__restrict__ rnorm, float *__restrict__ resid,
               uint32_t *__restrict__ fsigns) {
   extern __shared__ __align__(16) float sS[];
   rotate_rows<D>(c, mode, x, dtype, n, ld, slots, capacity, codes, norm, rnorm, resid, fsigns,
@@ -29,7 +29,7 @@ rotate_kernel(TqConsts c, int mode, const void *__restrict__ x, int dtype, int64
 template <int D>
 cudaError_t launch_rotate_d(const TqConsts &c, RotateMode mode, const void *x, tq_dtype dtype,
                             int64_t n, int64_t ld, const int64_t *slots, int64_t capacity,
-                            uint32_t *codes, float *norm, float *rnorm, float *resid,
+                            uint32_t *codes, void *norm, void *rnorm, float *resid,
                             uint32_t *fsigns, cudaStream_t st) {
   constexpr int VPB = (kRotThreads / 32) * RotLayout<D>::VPW;  // vectors per block
   const int64_t blocks = (n + VPB - 1) / VPB;
@@ -50,7 +50,7 @@ cudaError_t launch_rotate_d(const TqConsts &c, RotateMode mode, const void *x, t
 
 cudaError_t launch_rotate(const TqConsts &c, RotateMode mode, const void *x, tq_dtype dtype,
                           int64_t n, int64_t ld, const int64_t *slots, int64_t capacity,
-                          uint32_t *codes, float *norm, float *rnorm, float *resid,
+                          uint32_t *codes, void *norm, void *rnorm, float *resid,
                           cudaStream_t st, uint32_t *fsigns) {
   if (n <= 0) return cudaSuccess;
   switch (c.d) {

@@ -80,7 +80,7 @@ template <int D>
 __device__ __forceinline__ void rotate_rows(const TqConsts &c, int mode, const void *__restrict__ x, int dtype,
                                             int64_t n, int64_t ld, const int64_t *__restrict__ slots,
                                             int64_t capacity, uint32_t *__restrict__ codes,
-                                            float *__restrict__ norm, float *__restrict__ rnorm,
+                                            void *__restrict__ norm, void *__restrict__ rnorm,
                                             float *__restrict__ resid, uint32_t *__restrict__ fsigns,
                                             int64_t vblock, float *sS, bool one_vec = false) {
   using Lay = RotLayout<D>;
@@ -200,7 +200,7 @@ __device__ __forceinline__ void rotate_rows(const TqConsts &c, int mode, const v
             atomicOr(w, (uint32_t)((cd >> (c.bits - 1)) & 1) << sh);
           }
         }
-      if (l == 0) norm[slot] = nu;
+      if (l == 0) st_norm(norm, slot, nu, c.norm16);
     }
     if (staged) stage_async_wait();  // no copy may be left in flight
     return;  // MSE-only: no residual
@@ -225,13 +225,13 @@ __device__ __forceinline__ void rotate_rows(const TqConsts &c, int mode, const v
     uint4 *dst = reinterpret_cast<uint4 *>(codes + slot * c.code_words);
     for (int i = l; i < c.code_words / 4; i += LPV)
       dst[i] = make_uint4(st[4 * i], st[4 * i + 1], st[4 * i + 2], st[4 * i + 3]);
-    if (l == 0) norm[slot] = nu;
+    if (l == 0) st_norm(norm, slot, nu, c.norm16);
   }
   if (c.srht && fsigns != nullptr) {
     // structured QJL ("TurboQuant 学习路径" 二.2, fast JL y = P H D x): z = H (D2 r), the first m
     // coordinates' signs, by the same butterflies as the rotation (no projection matrix)
     const float gamma = sqrtf(group_sum<LPV>(rr));
-    if (store && l == 0) rnorm[slot] = gamma;
+    if (store && l == 0) st_norm(rnorm, slot, gamma, c.norm16);
 #pragma unroll
     for (int k = 0; k < KCH; ++k) {
       const float4 sg = *reinterpret_cast<const float4 *>(c.qjl_signs + 4 * (l + LPV * k));
@@ -268,7 +268,7 @@ __device__ __forceinline__ void rotate_rows(const TqConsts &c, int mode, const v
         __syncthreads();
       }
       const float gamma = sqrtf(group_sum<LPV>(rr));
-      if (store && l == 0) rnorm[slot] = gamma;
+      if (store && l == 0) st_norm(rnorm, slot, gamma, c.norm16);
       float *rb = rbuf[one_vec ? 0 : wib];
       if (!one_vec || wib == 0)
 #pragma unroll
@@ -333,7 +333,7 @@ __device__ __forceinline__ void rotate_rows(const TqConsts &c, int mode, const v
   }
   if (resid != nullptr) {
     const float gamma = sqrtf(group_sum<LPV>(rr));
-    if (store && l == 0) rnorm[slot] = gamma;
+    if (store && l == 0) st_norm(rnorm, slot, gamma, c.norm16);
     if (valid)
 #pragma unroll
       for (int k = 0; k < KCH; ++k)

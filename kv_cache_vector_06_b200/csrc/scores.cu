@@ -59,9 +59,9 @@ scores_kernel(TqConsts c, const float *__restrict__ qr, const float *__restrict_
   if (key >= n) return;
   const uint32_t *crow = ct + threadIdx.x * cst;
   const uint32_t *srow = c.m > 0 ? stl + threadIdx.x * sst : nullptr;
-  const float gamma = c.m > 0 ? keys.rnorm[key] : 0.f;
+  const float gamma = c.m > 0 ? ld_norm(keys.rnorm, key, c.norm16) : 0.f;
   float sc[kScQ];
-  estimate_scores<kScQ>(c, crow, srow, keys.norm[key], gamma, qs, ps, cent, sc);
+  estimate_scores<kScQ>(c, crow, srow, ld_norm(keys.norm, key, c.norm16), gamma, qs, ps, cent, sc);
 #pragma unroll
   for (int q = 0; q < kScQ; ++q)
     if (q0 + q < nq) out[(int64_t)(q0 + q) * n + key] = sc[q];

@@ -49,8 +49,8 @@ search_scan_kernel(TqConsts c, const float *__restrict__ qr, const float *__rest
     float sc[kSrQ];
     if (row < r_end) {
       estimate_scores<kSrQ>(c, codes + row * c.code_words,
-                            c.m > 0 ? signs + row * c.sign_words : nullptr, db.norm[row],
-                            c.m > 0 ? db.rnorm[row] : 0.f, qs, ps, cent, sc);
+                            c.m > 0 ? signs + row * c.sign_words : nullptr, ld_norm(db.norm, row, c.norm16),
+                            c.m > 0 ? ld_norm(db.rnorm, row, c.norm16) : 0.f, qs, ps, cent, sc);
     } else {
 #pragma unroll
       for (int q = 0; q < kSrQ; ++q) sc[q] = -INFINITY;
@@ -218,7 +218,7 @@ search_bigk_scan_kernel(TqConsts c, const float *__restrict__ qr, const float *_
     float sc[kBkQ];
     if (row < r_end) {
       estimate_scores<kBkQ>(c, codes + row * c.code_words, c.m > 0 ? signs + row * c.sign_words : nullptr,
-                            db.norm[row], c.m > 0 ? db.rnorm[row] : 0.f, qs, ps, cent, sc);
+                            ld_norm(db.norm, row, c.norm16), c.m > 0 ? ld_norm(db.rnorm, row, c.norm16) : 0.f, qs, ps, cent, sc);
     } else {
 #pragma unroll
       for (int q = 0; q < kBkQ; ++q) sc[q] = -INFINITY;

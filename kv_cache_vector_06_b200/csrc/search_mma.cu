@@ -222,12 +222,12 @@ search_mma_kernel(TqConsts c, const uint2 *__restrict__ frag, const float *__res
     bulk_g2s(buf + L.rs, static_cast<const char *>(db.signs) + r0 * SP::SIGN_BYTES, (unsigned)nr * SP::SIGN_BYTES,
              bar);
     if (nr4 > 0) {
-      bulk_g2s(buf + L.rn, db.norm + r0, (unsigned)nr4 * 4, bar);
-      bulk_g2s(buf + L.rr, db.rnorm + r0, (unsigned)nr4 * 4, bar);
+      bulk_g2s(buf + L.rn, static_cast<const float *>(db.norm) + r0, (unsigned)nr4 * 4, bar);
+      bulk_g2s(buf + L.rr, static_cast<const float *>(db.rnorm) + r0, (unsigned)nr4 * 4, bar);
     }
     for (int r = nr4; r < nr; ++r) {
-      reinterpret_cast<float *>(buf + L.rn)[r] = db.norm[r0 + r];
-      reinterpret_cast<float *>(buf + L.rr)[r] = db.rnorm[r0 + r];
+      reinterpret_cast<float *>(buf + L.rn)[r] = static_cast<const float *>(db.norm)[r0 + r];  // fp32 norms only
+      reinterpret_cast<float *>(buf + L.rr)[r] = static_cast<const float *>(db.rnorm)[r0 + r];
     }
     if (b == 0) {
       bulk_g2s(smem, frag + (int64_t)tile * (SP::FRAG_WORDS / 2), (unsigned)SP::FRAG_WORDS * 4u, bar);

@@ -414,8 +414,8 @@ search_tc_kernel(TqConsts c, const uint8_t *__restrict__ bst, const float *__res
     int64_t gr = r_begin + row;
     float nrm = 0.f, qg = 0.f;
     if (nblk > 0 && gr < r_end) {
-      nrm = db.norm[gr];
-      qg = c.qjl_scale * db.rnorm[gr];
+      nrm = ld_norm(db.norm, gr, c.norm16);
+      qg = c.qjl_scale * ld_norm(db.rnorm, gr, c.norm16);
     }
     for (int b = 0; b < nblk; ++b) {
       // all four warps go on (the previous block's top-k has finished reading the tile) or all stop
@@ -457,8 +457,8 @@ search_tc_kernel(TqConsts c, const uint8_t *__restrict__ bst, const float *__res
       const int nr = (int)min((int64_t)kTcM, r_end - r0);
       gr += kTcM;
       if (b + 1 < nblk && gr < r_end) {
-        nrm = db.norm[gr];
-        qg = c.qjl_scale * db.rnorm[gr];
+        nrm = ld_norm(db.norm, gr, c.norm16);
+        qg = c.qjl_scale * ld_norm(db.rnorm, gr, c.norm16);
       }
       asm volatile("bar.sync 1, 128;\n" ::: "memory");
 #pragma unroll 1

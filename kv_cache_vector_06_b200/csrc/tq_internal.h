@@ -32,6 +32,7 @@ struct TqConsts {
   const float *St;     // device [d][m]: S transposed (coalesced reads with lane = row of S)
   int srht;               // S = P H D2 (structured QJL): encode transforms the residual instead
   const float *qjl_signs; // device [d], +-1.0f (D2), srht only
+  int norm16;             // norm and rnorm stored as fp16 (else fp32)
   int polar;              // PolarQuant first stage (angle codes in place of coordinate codes)
   const float *polar_tab; // device [levels][thresholds | cos c | sin c][16], polar only
 };
@@ -105,7 +106,7 @@ enum RotateMode { ROT_ENCODE = 0, ROT_QUERY = 1 };
 // per-step append; large batches use the tiled projection kernel.
 cudaError_t launch_rotate(const TqConsts &c, RotateMode mode, const void *x, tq_dtype dtype,
                           int64_t n, int64_t ld, const int64_t *slots, int64_t capacity,
-                          uint32_t *codes, float *norm, float *rnorm, float *resid,
+                          uint32_t *codes, void *norm, void *rnorm, float *resid,
                           cudaStream_t st, uint32_t *fsigns = nullptr);
 constexpr int64_t kFusedEncodeMaxRows = 4096;
 // Bulk encode at d = 128, one row per thread (encode_tpr.cu): MSE-only contexts in either layout
@@ -114,7 +115,7 @@ constexpr int64_t kFusedEncodeMaxRows = 4096;
 bool encode_tpr_eligible(const TqConsts &c, const int64_t *slots, tq_dtype dtype);
 int64_t encode_tpr_rows(const TqConsts &c, int64_t n);  // rows it takes (a block-layout tail is left)
 cudaError_t launch_encode_tpr(const TqConsts &c, const void *x, tq_dtype dtype, int64_t n, int64_t ld,
-                              const int64_t *slots, int64_t capacity, uint32_t *codes, float *norm, float *rnorm,
+                              const int64_t *slots, int64_t capacity, uint32_t *codes, void *norm, void *rnorm,
                               uint32_t *signs, cudaStream_t st);
 
 // Z = R S^T for rows of R ([n][d] fp32).  SIGNS: pack bit = [z >= 0] into `signs` at the rows'
@@ -128,7 +129,7 @@ cudaError_t launch_project(const TqConsts &c, ProjEpilogue ep, const float *R, i
 // residual rows to `resid` and rnorm, for launch_project) and estimated scores.
 bool polar_supported(const TqConsts &c);
 cudaError_t launch_encode_polar(const TqConsts &c, const void *x, tq_dtype dtype, int64_t n, int64_t ld,
-                                const int64_t *slots, int64_t capacity, uint32_t *codes, float *norm, float *rnorm,
+                                const int64_t *slots, int64_t capacity, uint32_t *codes, void *norm, void *rnorm,
                                 float *resid, cudaStream_t st);
 cudaError_t launch_scores_polar(const TqConsts &c, const float *qr, const float *p, int nq, const tq_packed &keys,
                                 int64_t n, float *out, cudaStream_t st);

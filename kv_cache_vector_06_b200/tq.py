@@ -27,7 +27,8 @@ class TqError(RuntimeError):
 
 
 class Spec(ctypes.Structure):
-    _fields_ = [("d", c_int32), ("mse_bits", c_int32), ("qjl_m", c_int32), ("layout", c_int32)]
+    _fields_ = [("d", c_int32), ("mse_bits", c_int32), ("qjl_m", c_int32), ("layout", c_int32),
+                ("norm_bits", c_int32)]
 
 
 LAYOUT_ROWS, LAYOUT_BLOCK16 = 0, 1
@@ -151,16 +152,19 @@ class Context:
     """Quantizer constants for one tensor role, resident on one device."""
 
     def __init__(self, d: int, mse_bits: int, qjl_m: int, rot_signs, qjl_matrix=None, device: int = 0,
-                 layout: int = LAYOUT_ROWS, qjl_signs=None, polar: bool = False):
+                 layout: int = LAYOUT_ROWS, qjl_signs=None, polar: bool = False, norm_bits: int = 32):
         """qjl_matrix: the dense JL matrix [qjl_m, d] (tq_ctx_create); or qjl_signs: the sign
         vector D2 [d] of the structured matrix S = P H D2 (tq_ctx_create_srht).  polar: the
-        PolarQuant first stage (tq_ctx_create_polar)."""
+        PolarQuant first stage (tq_ctx_create_polar).  norm_bits: 32 or 16, the storage of the
+        norms (tq_spec.norm_bits)."""
         rs = torch.as_tensor(rot_signs).to(torch.int8).contiguous().cpu()
         if rs.numel() != d:
             raise ValueError("rot_signs must have d entries")
         self.d, self.mse_bits, self.qjl_m, self.device, self.layout = d, mse_bits, qjl_m, device, layout
         self.srht = qjl_signs is not None
-        spec = Spec(d, mse_bits, qjl_m, layout)
+        self.norm_bits = norm_bits
+        self.norm_dtype = torch.float16 if norm_bits == 16 else torch.float32
+        spec = Spec(d, mse_bits, qjl_m, layout, norm_bits)
         h = c_void_p()
         if self.srht:
             d2 = torch.as_tensor(qjl_signs).to(torch.int8).contiguous().cpu()
@@ -212,11 +216,11 @@ class Packed:
     def allocate(ctx: Context, capacity: int) -> "Packed":
         dev = torch.device("cuda", ctx.device)
         codes = torch.zeros(capacity, ctx.code_bytes, dtype=torch.uint8, device=dev)
-        norm = torch.zeros(capacity, dtype=torch.float32, device=dev)
+        norm = torch.zeros(capacity, dtype=ctx.norm_dtype, device=dev)
         signs = rnorm = None
         if ctx.qjl_m > 0:
             signs = torch.zeros(capacity, ctx.sign_bytes, dtype=torch.uint8, device=dev)
-            rnorm = torch.zeros(capacity, dtype=torch.float32, device=dev)
+            rnorm = torch.zeros(capacity, dtype=ctx.norm_dtype, device=dev)
         return Packed(codes, norm, signs, rnorm)
 
     @property
@@ -227,7 +231,7 @@ class Packed:
         if self.codes.dim() != 2 or self.codes.shape[1] != ctx.code_bytes or self.codes.dtype != torch.uint8:
             raise ValueError(f"codes must be uint8 [capacity, {ctx.code_bytes}]")
         p = PackedC(_dev(self.codes, ctx.device, "codes", torch.uint8),
-                    c_void_p(None), _dev(self.norm, ctx.device, "norm", torch.float32),
+                    c_void_p(None), _dev(self.norm, ctx.device, "norm", ctx.norm_dtype),
                     c_void_p(None), self.codes.shape[0])
         if self.norm.numel() < self.capacity:
             raise ValueError("norm is shorter than codes")
@@ -237,7 +241,7 @@ class Packed:
             if self.rnorm is None or self.rnorm.numel() < self.capacity:
                 raise ValueError("rnorm must have capacity entries")
             p.signs = _dev(self.signs, ctx.device, "signs", torch.uint8)
-            p.rnorm = _dev(self.rnorm, ctx.device, "rnorm", torch.float32)
+            p.rnorm = _dev(self.rnorm, ctx.device, "rnorm", ctx.norm_dtype)
         return p
 
 

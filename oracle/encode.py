@@ -94,6 +94,20 @@ def encode(x, signs, S, centroids, thresholds) -> Encoded:
     return Encoded(norm=norm, codes=codes, rnorm=rnorm, bits=bits, y=y, z=z)
 
 
+def store_norms(enc: Encoded, norm_bits: int = 32) -> Encoded:
+    """The encoding as stored: with norm_bits = 16 the norms ||x|| and gamma are kept in IEEE half
+    precision (round to nearest even, values above the largest half 65504 kept as 65504), the only
+    per-vector constants being quantization metadata kept in FP16 or FP32 ([JJ] 第一部分)
+    (reading: the option saves 4 bytes per vector with a QJL stage).  Codes and signs are unchanged
+    (they come from the exact norm)."""
+    if norm_bits == 32:
+        return enc
+    if norm_bits != 16:
+        raise ValueError("norm_bits must be 32 or 16")
+    h = lambda a: np.minimum(np.asarray(a, dtype=np.float64), 65504.0).astype(np.float16).astype(np.float64)
+    return Encoded(**{**enc.__dict__, "norm": h(enc.norm), "rnorm": h(enc.rnorm)})
+
+
 def pack_codes(codes, bits: int) -> np.ndarray:
     """[n, d] codes -> [n, code_bytes] uint8, plane-major LSB-first."""
     codes = np.asarray(codes, dtype=np.int64)

@@ -38,9 +38,9 @@ def _packed_equal(a, b):
 
 
 def _step_case(tq, d, kbits, km, vbits, vlayout, batch, hkv, group, lens, paged, seed, kvdtype=torch.float32,
-               qdtype=torch.bfloat16, srht=False):
-    kq = Quantizer(d, kbits, km, seed=seed, srht=srht)
-    vq = Quantizer(d, vbits, 0, seed=seed + 50, layout=vlayout)
+               qdtype=torch.bfloat16, srht=False, norm_bits=32):
+    kq = Quantizer(d, kbits, km, seed=seed, srht=srht, norm_bits=norm_bits)
+    vq = Quantizer(d, vbits, 0, seed=seed + 50, layout=vlayout, norm_bits=norm_bits)
     hq = hkv * group
     blk = synth.BLOCK_TOKENS
     new_lens = [L + 1 for L in lens]
@@ -124,3 +124,10 @@ def test_decode_step_structured_qjl(tq, vlayout):
     in-register Walsh-Hadamard transform, the queries are projected with the same S."""
     _step_case(tq, 128, 2, 128, 3, vlayout, batch=2, hkv=2, group=4, lens=[1500, 33], paged=vlayout == 1,
                seed=371 + vlayout, srht=True)
+
+
+def test_decode_step_fp16_norms(tq):
+    """tq_decode_step with norms stored in fp16: the appended rows and the attention equal the
+    separate calls' and match the oracle on the library's own bytes."""
+    _step_case(tq, 128, 2, 128, 3, 1, batch=3, hkv=2, group=4, lens=[700, 15, 1031], paged=True, seed=211,
+               kvdtype=torch.bfloat16, norm_bits=16)

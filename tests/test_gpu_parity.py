@@ -140,9 +140,9 @@ def test_scores_bf16_queries_and_small_d(tq):
         assert_scores_close(got, ref)
 
 
-def _attention_case(tq, d, kbits, km, vbits, batch, hkv, group, lens, paged, qdtype, seed, vlayout=0):
-    kq = Quantizer(d, kbits, km, seed=seed)
-    vq = Quantizer(d, vbits, 0, seed=seed + 50, layout=vlayout)
+def _attention_case(tq, d, kbits, km, vbits, batch, hkv, group, lens, paged, qdtype, seed, vlayout=0, norm_bits=32):
+    kq = Quantizer(d, kbits, km, seed=seed, norm_bits=norm_bits)
+    vq = Quantizer(d, vbits, 0, seed=seed + 50, layout=vlayout, norm_bits=norm_bits)
     hq = hkv * group
     maxlen = int(max(lens))
     blk = synth.BLOCK_TOKENS
@@ -462,3 +462,54 @@ def test_attention_tensor_core_path_matches_general_kernel(tq):
     o_tc = tq.attend_decode(kq.ctx, v_blk.ctx, q, kp, vb, lens_t, maxlen, n_kv_heads=hkv, ctx_stride=maxlen)
     torch.cuda.synchronize()
     assert_attention_close(o_tc.cpu().numpy(), o_gen.cpu().numpy())
+
+
+# ------------------------------------------------------------------ fp16 norms (tq_spec.norm_bits = 16)
+@pytest.mark.parametrize("path", ["bulk_keys_bf16", "bulk_values_block_bf16", "bulk_fp32", "small_batch", "srht"])
+def test_norm16_encode_paths(tq, path):
+    """Norms stored in fp16 through every encode path: the stored norm is the oracle's fp16 norm
+    (within one half ulp, the library rounding its fp32 norm), codes and signs as with fp32 norms."""
+    d = 128
+    n = {"small_batch": 333}.get(path, 5011)
+    layout = 1 if path == "bulk_values_block_bf16" else 0
+    m = 0 if path == "bulk_values_block_bf16" else 128
+    q = Quantizer(d, 2, m, seed=800 + len(path), layout=layout, norm_bits=16, srht=(path == "srht"))
+    x = (torch.randn(n, d, generator=torch.Generator().manual_seed(5)) *
+         torch.exp(torch.randn(d, generator=torch.Generator().manual_seed(6))))
+    if path != "bulk_fp32" and path != "small_batch":
+        x = x.to(torch.bfloat16)
+    x[3] = 0
+    cap = (n + 15) // 16 * 16
+    packed = tq.Packed.allocate(q.ctx, cap)
+    assert packed.norm.dtype == torch.float16
+    tq.encode_kv(q.ctx, x.cuda(), packed)
+    torch.cuda.synchronize()
+    rows = np.arange(n)
+    compare_encode(q, q.oracle_encode(x.double().numpy()), *unpack(q, packed, rows=rows))
+
+
+@pytest.mark.parametrize("vlayout", [0, 1])
+def test_norm16_attention(tq, vlayout):
+    """fp16 norms through the general (row values) and the tensor-core (token-block values)
+    attention paths, paged and ragged; the oracle reads the library's own stored norms."""
+    _attention_case(tq, 128, 2, 128, 3, batch=3, hkv=2, group=4, lens=[700, 16, 1031], paged=True,
+                    qdtype=torch.bfloat16, seed=97, vlayout=vlayout, norm_bits=16)
+
+
+def test_norm16_scores_and_search(tq):
+    """fp16 norms in tq_scores and the three search scans (CUDA cores for few queries, tcgen05 for
+    many, the large-k scan)."""
+    d, n = 128, 3001
+    q = Quantizer(d, 2, d, seed=99, norm_bits=16)
+    X = synth.unit_rows(n, d, seed=7) * 3.0
+    packed = _enc(tq, q, X)
+    codes, sbits, norm, rnorm = unpack(q, packed)
+    for nq, k in ((5, 10), (40, 10), (6, 100)):
+        Q = synth.unit_rows(nq, d, seed=8 + nq)
+        ref_full = oracle_scores_from_packed(q, Q.double().numpy(), codes, sbits, norm, rnorm)
+        if nq == 5:
+            assert_scores_close(tq.scores(q.ctx, Q.cuda(), packed).cpu().numpy(), ref_full)
+        s, i = tq.search_topk(q.ctx, Q.cuda(), packed, k)
+        ref_s, _ = osearch.topk(ref_full, k)
+        assert_topk_equivalent(s.cpu().numpy(), i.cpu().numpy(), lambda r, idx: ref_full[r, idx], ref_s)
+    assert tq.device_status() == 0

@@ -104,6 +104,10 @@ def test_ctx_create_validates_before_device(lib):
     with pytest.raises(lib.TqError) as e:
         lib.Context(128, 2, 0, bad)
     assert e.value.status == 1
+    # norm storage: 32 (or 0) or 16 bits only
+    with pytest.raises(lib.TqError) as e:
+        lib.Context(128, 2, 0, torch.ones(128, dtype=torch.int8), norm_bits=8)
+    assert e.value.status == 1 and "norm_bits" in str(e.value)
 
 
 def test_null_arguments_rejected(lib):

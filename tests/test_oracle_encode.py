@@ -171,3 +171,28 @@ def test_block16_round_trip_and_size(d, bits):
     # same information as the row layout: 16 * (b*d/8) meaningful bytes per block
     used = 16 * bits * d // 8
     assert np.all(buf.reshape(3, -1)[:, used:] == 0)
+
+
+def test_store_norms_half_precision():
+    """fp16 norm storage: round to nearest even on the half grid (2^-10 spacing in [1, 2)),
+    saturation at the largest half, codes and signs untouched; 32 bits leaves the encoding as is."""
+    n = 6
+    enc = encode.Encoded(norm=np.array([1.0, 1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11, 3.14159, 1e6, 0.0]),
+                       codes=np.zeros((n, 4), dtype=np.int64),
+                       rnorm=np.array([0.5, 0.25 + 2.0 ** -13, 2.0 ** -14 * 1.5, 70000.0, 1e-3, 0.0]),
+                       bits=np.ones((n, 4), dtype=np.uint8), y=np.zeros((n, 4)), z=np.zeros((n, 4)))
+    assert encode.store_norms(enc, 32) is enc
+    h = encode.store_norms(enc, 16)
+    # halfway cases go to the even neighbour: 1 + 2^-11 -> 1, 1 + 3 2^-11 -> 1 + 2^-9
+    np.testing.assert_array_equal(h.norm[:3], [1.0, 1.0, 1.0 + 2.0 ** -9])
+    # pi on the half grid of [2, 4) (spacing 2^-9): 3.140625 (1608 * 2^-9)
+    assert h.norm[3] == 1608 * 2.0 ** -9
+    assert h.norm[4] == 65504.0 and h.rnorm[3] == 65504.0
+    # 0.25 + 2^-13 is halfway on the [0.25, 0.5) grid (spacing 2^-12): even -> 0.25
+    assert h.rnorm[1] == 0.25
+    # 1.5 * 2^-14 is a normal half exactly
+    assert h.rnorm[2] == 1.5 * 2.0 ** -14
+    np.testing.assert_array_equal(h.codes, enc.codes)
+    np.testing.assert_array_equal(h.bits, enc.bits)
+    with pytest.raises(ValueError):
+        encode.store_norms(enc, 8)
