@@ -52,9 +52,13 @@ struct MmaArgs {
   int kn4, vn4;    // log2 of the bytes of one stored K / V norm: 2 (fp32) or 1 (fp16)
 };
 
-// Norm i of a staged array (fp32 or fp16, `l2` = log2 of its bytes).
-__device__ __forceinline__ float staged_norm(const unsigned char *base, int i, int l2) {
-  return l2 == 1 ? __half2float(reinterpret_cast<const __half *>(base)[i]) : reinterpret_cast<const float *>(base)[i];
+// Norm i of a staged array (fp16 when NH, else fp32).
+template <bool NH>
+__device__ __forceinline__ float staged_norm(const unsigned char *base, int i) {
+  if constexpr (NH)
+    return __half2float(reinterpret_cast<const __half *>(base)[i]);
+  else
+    return reinterpret_cast<const float *>(base)[i];
 }
 
 __device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -586,7 +590,7 @@ __device__ __forceinline__ void stage_sub(const MmaArgs &a, int sc, const int64_
 // out when e^{l - M} < tau max(1, l_old e^{M_old - M}), a bound that is at least its final softmax
 // weight (the running sum only grows and the running maximum's token counts 1), so every row it
 // drops has a final weight below tau; blocks whose rows are all dropped skip their value MMAs.
-template <int BK, int BV, bool QJL>
+template <int BK, int BV, bool QJL, bool NH>
 __global__ void __launch_bounds__(kMmaThreads, 2)
 attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restrict__ kfrag,
                   const float *__restrict__ kconst, float *__restrict__ part) {
@@ -770,14 +774,14 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
             fma2((float)B[0], (float)B[2], 65536.f, ds0, ds1, ds0, ds1);
             fma2((float)B[1], (float)B[3], 16777216.f, ds0, ds1, ds0, ds1);
             fma2(ds0, ds1, kcs[4 + t], -kcs[12 + t], -kcs[12 + t], ds0, ds1);
-            sc0 = fmaf(kc.qjl_scale * staged_norm(skr, i0, a.kn4), ds0, sc0);
-            sc1 = fmaf(kc.qjl_scale * staged_norm(skr, i1, a.kn4), ds1, sc1);
+            sc0 = fmaf(kc.qjl_scale * staged_norm<NH>(skr, i0), ds0, sc0);
+            sc1 = fmaf(kc.qjl_scale * staged_norm<NH>(skr, i1), ds1, sc1);
           }
           const bool ok0 = bok && tk0 + i0 < t1, ok1 = bok && tk0 + i1 < t1;
-          lgt[kb][0] = ok0 ? a.scale * staged_norm(skn, i0, a.kn4) * sc0 : -INFINITY;
-          lgt[kb][1] = ok1 ? a.scale * staged_norm(skn, i1, a.kn4) * sc1 : -INFINITY;
-          nvk[kb][0] = ok0 ? staged_norm(svn, i0, a.vn4) : 0.f;  // masked slots may hold stale bytes
-          nvk[kb][1] = ok1 ? staged_norm(svn, i1, a.vn4) : 0.f;
+          lgt[kb][0] = ok0 ? a.scale * staged_norm<NH>(skn, i0) * sc0 : -INFINITY;
+          lgt[kb][1] = ok1 ? a.scale * staged_norm<NH>(skn, i1) * sc1 : -INFINITY;
+          nvk[kb][0] = ok0 ? staged_norm<NH>(svn, i0) : 0.f;  // masked slots may hold stale bytes
+          nvk[kb][1] = ok1 ? staged_norm<NH>(svn, i1) : 0.f;
         }
       }
 
@@ -1117,14 +1121,15 @@ template <int BK, int BV, bool QJL>
 cudaError_t launch_mma(const TqConsts &kc, const TqConsts &vc, const MmaArgs &a, dim3 grid,
                        const uint32_t *kfrag, const float *kconst, float *part, cudaStream_t st) {
   const size_t smem = MmaSmem<BK, BV, QJL>::total;
-  cudaError_t e = tq_smem_limit(reinterpret_cast<const void *>(attend_mma_kernel<BK, BV, QJL>),
-                                       (int)smem);
+  // norms in fp16 (both roles; mixed storage takes the general path) or fp32
+  auto kern = a.kn4 == 1 ? attend_mma_kernel<BK, BV, QJL, true> : attend_mma_kernel<BK, BV, QJL, false>;
+  cudaError_t e = tq_smem_limit(reinterpret_cast<const void *>(kern), (int)smem);
   if (e != cudaSuccess) return e;
   // programmatic dependent launch: the grid may start while the preceding kernel on the stream
   // (the query-fragment or decode-prep kernel) finishes; the kernel waits for it before use.  With
   // per-kernel profiling on, an event sits between the two kernels and a plain launch is used.
   if (tq_prof_on()) {
-    attend_mma_kernel<BK, BV, QJL><<<grid, kMmaThreads, smem, st>>>(kc, vc, a, kfrag, kconst, part);
+    kern<<<grid, kMmaThreads, smem, st>>>(kc, vc, a, kfrag, kconst, part);
     return cudaGetLastError();
   }
   cudaLaunchConfig_t cfg = {};
@@ -1137,7 +1142,7 @@ cudaError_t launch_mma(const TqConsts &kc, const TqConsts &vc, const MmaArgs &a,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, attend_mma_kernel<BK, BV, QJL>, kc, vc, a, kfrag, kconst, part);
+  return cudaLaunchKernelEx(&cfg, kern, kc, vc, a, kfrag, kconst, part);
 }
 
 template <int BK, int BV, bool QJL>
@@ -1174,6 +1179,7 @@ bool attn_fast_eligible(const TqConsts &kc, const TqConsts &vc, const tq_attn_de
   for (int P = 0; P < (vc.bits == 3 ? 4 : vc.bits); ++P)
     if (!(vc.plane_coef[P] >= 0.f)) return false;
   if (desc.block_table ? (desc.block_size % 16) != 0 : (desc.ctx_stride % 16) != 0) return false;
+  if (kc.norm16 != vc.norm16) return false;  // one norm storage for both roles
   // the norm arrays are copied in bulk: 16-byte aligned bases
   auto a16 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
   if (!a16(desc.k.norm) || !a16(desc.v.norm) || (kc.m > 0 && !a16(desc.k.rnorm))) return false;
