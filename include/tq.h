@@ -177,8 +177,10 @@ tq_status tq_ctx_create_srht(const tq_spec *spec, const int8_t *rot_signs, const
  * the Lloyd-Max codebook of its level's known law (tq_polar_codebook); no per-block constants.
  * The QJL stage, when qjl_m > 0, sketches the residual y/||x|| - y^ with the dense S as usual.
  * Packed arrays as for tq_ctx_create: code slot p holds angle p (level 1 first: d/2 angles, then
- * level 2, ..., the last level's single angle at d - 2; slot d - 1 is 0).  Supported calls:
- * tq_encode_kv and tq_scores; the attention and search calls return TQ_EUNSUPPORTED.
+ * level 2, ..., the last level's single angle at d - 2; slot d - 1 is 0).  Every call accepts such
+ * contexts (for keys, values or a database): scores through the reconstructed direction y^, value
+ * coordinates as products of the cos / sin of the angles along their path.  They take the CUDA-core
+ * attention and search paths (the tensor-core paths rest on the coordinate codebook's bit planes).
  *   spec  d = 128, TQ_LAYOUT_ROWS, mse_bits 1..4, qjl_m 0 or a multiple of 32 up to 1024
  * Errors: as tq_ctx_create; TQ_EUNSUPPORTED for other d or layouts. */
 tq_status tq_ctx_create_polar(const tq_spec *spec, const int8_t *rot_signs, const float *qjl_matrix,

@@ -254,6 +254,7 @@ static tq_status ctx_create(const tq_spec *spec, const int8_t *rot_signs, const 
     k.plane_coef_sum = (float)sum;
     k.fast_ok = worst <= 1e-9 * std::fabs(c->centroids[L - 1]) ? 1 : 0;
   }
+  if (polar) k.fast_ok = 0;  // angle codes: the bit-plane tensor-core paths do not apply
   *out = c;
   return TQ_OK;
 }
@@ -495,8 +496,6 @@ static tq_status check_attn(const tq_ctx *kctx, const tq_ctx *vctx, const tq_att
   if (!desc) return tq_fail(TQ_EINVAL, "desc is NULL");
   if (kctx->spec.d != vctx->spec.d)
     return tq_fail(TQ_EUNSUPPORTED, "K and V contexts differ in d (%d vs %d)", kctx->spec.d, vctx->spec.d);
-  if (kctx->k.polar || vctx->k.polar)
-    return tq_fail(TQ_EUNSUPPORTED, "PolarQuant contexts: encode and scores only");
   if (vctx->spec.qjl_m != 0)
     return tq_fail(TQ_EUNSUPPORTED, "the V context must be MSE-only (qjl_m == 0)");
   if (kctx->spec.layout != TQ_LAYOUT_ROWS)
@@ -675,7 +674,6 @@ tq_status tq_search_topk(const tq_ctx *ctx, const void *q, tq_dtype dtype, int32
   if (!aligned16(q) || !aligned16(out_scores) || !aligned16(out_idx))
     return tq_fail(TQ_EINVAL, "q/out not 16-byte aligned");
   if (ctx->spec.layout != TQ_LAYOUT_ROWS) return tq_fail(TQ_EUNSUPPORTED, "tq_search_topk needs TQ_LAYOUT_ROWS");
-  if (ctx->k.polar) return tq_fail(TQ_EUNSUPPORTED, "PolarQuant contexts: encode and scores only");
   st = check_packed(ctx, db, n, "db", true);
   if (st != TQ_OK) return st;
   size_t need = 0;

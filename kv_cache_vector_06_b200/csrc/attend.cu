@@ -3,6 +3,7 @@
 //
 // Per CTA, for tiles of 128 tokens (one thread per token):
 //   logits  l_t = scale * nu_t (<q', c_K[code_t]> + sqrt(pi/2)/m gamma_t <2 bits_t - 1, p>)
+//           (PolarQuant keys: <q', y^_t>, y^_t the direction rebuilt from the angle codes)
 //           for the G query heads that share the KV head ("谷歌 TurboQuant 深度拆解" 第二部分
 //           第二步 and 第三部分 "推理速度": logits against the compressed keys);
 //   online softmax: running max and sum per head, earlier partial sums rescaled;
@@ -14,6 +15,7 @@
 #include <cmath>
 
 #include "device_common.cuh"
+#include "polar_device.cuh"
 
 namespace {
 
@@ -42,10 +44,13 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
-template <int G>
+// KP / VP: PolarQuant keys / values (d = 128): the key scores through the reconstructed direction,
+// a value coordinate as the product of cos / sin of the angles along its path.
+template <int G, bool KP, bool VP>
 __global__ void __launch_bounds__(kAtThreads)
 attend_split_kernel(TqConsts kc, TqConsts vc, AttnArgs a, const float *__restrict__ qr,
                     const float *__restrict__ p, float *__restrict__ part) {
+  __shared__ PolarTab ktab, vtab;
   extern __shared__ float sm[];
   const int d = kc.d, m = kc.m;
   float *qs = sm;                        // [d][G]
@@ -71,6 +76,8 @@ attend_split_kernel(TqConsts kc, TqConsts vc, AttnArgs a, const float *__restric
     centK[tid] = kc.centroids[tid];
     centV[tid] = vc.centroids[tid];
   }
+  if (KP) polar_tab_stage(ktab, kc.polar_tab, tid, kAtThreads);
+  if (VP) polar_tab_stage(vtab, vc.polar_tab, tid, kAtThreads);
   __syncthreads();
 
   const uint32_t *kcodes = static_cast<const uint32_t *>(a.k.codes);
@@ -102,9 +109,12 @@ attend_split_kernel(TqConsts kc, TqConsts vc, AttnArgs a, const float *__restric
     float sc[G];
     float nuv = 0.f;
     if (ok) {
-      estimate_scores<G>(kc, kcodes + slot * kc.code_words,
-                         m > 0 ? ksigns + slot * kc.sign_words : nullptr, ld_norm(a.k.norm, slot, kc.norm16),
-                         m > 0 ? ld_norm(a.k.rnorm, slot, kc.norm16) : 0.f, qs, ps, centK, sc);
+      const uint32_t *kr = kcodes + slot * kc.code_words, *ks = m > 0 ? ksigns + slot * kc.sign_words : nullptr;
+      const float nuk = ld_norm(a.k.norm, slot, kc.norm16), gk = m > 0 ? ld_norm(a.k.rnorm, slot, kc.norm16) : 0.f;
+      if constexpr (KP)
+        polar_scores<G>(kc, kr, ks, nuk, gk, qs, ps, ktab, sc);
+      else
+        estimate_scores<G>(kc, kr, ks, nuk, gk, qs, ps, centK, sc);
 #pragma unroll
       for (int g = 0; g < G; ++g) sc[g] *= a.scale;
       nuv = ld_norm(a.v.norm, slot, vc.norm16);
@@ -154,7 +164,11 @@ attend_split_kernel(TqConsts kc, TqConsts vc, AttnArgs a, const float *__restric
       for (int dd = 0; dd < kMaxDpt; ++dd) {
         const int j = tid + dd * kAtThreads;
         if (j < d) {
-          const float cv = centV[slot_code(vcodes, si, j, vc)];
+          float cv;
+          if constexpr (VP)
+            cv = polar_coord(vcodes + si * vc.code_words, j, vc.bits, vtab);
+          else
+            cv = centV[slot_code(vcodes, si, j, vc)];
 #pragma unroll
           for (int g = 0; g < G; ++g) acc[g][dd] = fmaf(wv[g], cv, acc[g][dd]);
         }
@@ -263,10 +277,12 @@ cudaError_t launch_split(const TqConsts &kc, const TqConsts &vc, const AttnArgs 
   const size_t smem = sizeof(float) * ((size_t)(kc.d + kc.m) * G + (size_t)G * kAtTile +
                                        2 * G * kAtWarps + 32) +
                       sizeof(int64_t) * kAtTile;
-  cudaError_t e = tq_smem_limit(reinterpret_cast<const void *>(attend_split_kernel<G>), (int)smem);
+  auto kern = kc.polar ? (vc.polar ? attend_split_kernel<G, true, true> : attend_split_kernel<G, true, false>)
+                       : (vc.polar ? attend_split_kernel<G, false, true> : attend_split_kernel<G, false, false>);
+  cudaError_t e = tq_smem_limit(reinterpret_cast<const void *>(kern), (int)smem);
   if (e != cudaSuccess) return e;
   tq_prof_begin(TQK_ATTEND_SPLIT, st);
-  attend_split_kernel<G><<<grid, kAtThreads, smem, st>>>(kc, vc, a, qr, p, part);
+  kern<<<grid, kAtThreads, smem, st>>>(kc, vc, a, qr, p, part);
   tq_prof_end(TQK_ATTEND_SPLIT, st);
   return cudaGetLastError();
 }

@@ -15,11 +15,11 @@
 //
 // One row per thread (registers); the angle tables (thresholds, cos and sin of the centroids per
 // level) sit in shared memory.  The residual rows go to a workspace for the projection kernel.
-#include "device_common.cuh"
+#include "polar_device.cuh"
 
 namespace {
 
-constexpr int kPD = 128, kPLevels = 7, kPRows = 128;
+constexpr int kPD = kPolarD, kPLevels = kPolarLevels, kPRows = 128;
 
 __device__ __forceinline__ void fwht128p(float (&v)[kPD]) {
 #pragma unroll
@@ -33,13 +33,6 @@ __device__ __forceinline__ void fwht128p(float (&v)[kPD]) {
       }
 }
 
-// first code slot of each level (level 1 at 0)
-__host__ __device__ constexpr int level_off(int l) { return kPD - (kPD >> (l - 1)); }
-
-// Tables in shared memory: [level][0: thresholds | 1: cos c | 2: sin c][16]
-struct PolarTab {
-  float v[kPLevels][3][16];
-};
 
 template <int BITS>
 __device__ __forceinline__ int angle_code(float a, const float *thr) {
@@ -66,7 +59,7 @@ __device__ __forceinline__ void reconstruct(const uint32_t (&w)[4][4], const Pol
     const int n = kPD >> l;  // angles of level l
 #pragma unroll
     for (int i = n - 1; i >= 0; --i) {
-      const int c = code_at<BITS>(w, level_off(l) + i);
+      const int c = code_at<BITS>(w, polar_level_off(l) + i);
       const float r = t[i];
       t[2 * i] = r * tab.v[l - 1][1][c];
       t[2 * i + 1] = r * tab.v[l - 1][2][c];
@@ -131,7 +124,7 @@ encode_polar_kernel(TqConsts c, const char *__restrict__ x, int64_t ld_bytes, in
     for (int i = 0; i < nl; ++i) {
       const float a0 = v[2 * i], a1 = v[2 * i + 1];
       const int code = angle_code<BITS>(atan2f(a1, a0), tab.v[l - 1][0]);
-      const int p = level_off(l) + i;
+      const int p = polar_level_off(l) + i;
 #pragma unroll
       for (int P = 0; P < BITS; ++P) w[P][p >> 5] |= (uint32_t)((code >> P) & 1) << (p & 31);
       v[i] = sqrtf(fmaf(a0, a0, a1 * a1));

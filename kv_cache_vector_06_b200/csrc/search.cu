@@ -2,19 +2,21 @@
 // 第三部分 "向量搜索"), ordered by (estimated score descending, index ascending).
 //
 // Scan: a CTA takes a tile of 8 queries and one shard of rows.  For each block of 256 rows every
-// thread scores one row against the 8 prepared queries (shared memory, broadcast reads) into a
-// shared tile; then warp w merges query w's 256 scores into its running top-k, which lives one
+// thread scores one row against the 8 prepared queries (shared memory, broadcast reads; PolarQuant
+// rows through their reconstructed direction) into a shared tile; then warp w merges query w's 256 scores into its running top-k, which lives one
 // entry per lane (k <= 32) and is updated by ballot + shuffle insertion.  Each CTA writes its
 // shard's candidates; a merge kernel (one warp per query) reduces the shards to the final list.
 #include <cmath>
 
 #include "device_common.cuh"
+#include "polar_device.cuh"
 
 namespace {
 
 constexpr int kSrThreads = 256;
 constexpr int kSrQ = 8;  // queries per CTA = warps per CTA
 
+template <bool POLAR>
 __global__ void __launch_bounds__(kSrThreads)
 search_scan_kernel(TqConsts c, const float *__restrict__ qr, const float *__restrict__ p, int nq,
                    tq_packed db, int64_t n, int k, int64_t rows_per_shard, int shards,
@@ -24,9 +26,11 @@ search_scan_kernel(TqConsts c, const float *__restrict__ qr, const float *__rest
   float *ps = qs + c.d * kSrQ;          // [m][8]
   float *cent = ps + c.m * kSrQ;        // [16]
   float *tile = cent + TQ_MAX_LEVELS;   // [8][256]
+  __shared__ PolarTab ptab;              // PolarQuant contexts: the angle tables
   const int shard = blockIdx.x;
   const int q0 = blockIdx.y * kSrQ;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (POLAR) polar_tab_stage(ptab, c.polar_tab, tid, kSrThreads);
   for (int i = tid; i < c.d * kSrQ; i += kSrThreads) {
     const int j = i / kSrQ, q = i % kSrQ;
     qs[i] = (q0 + q < nq) ? qr[(int64_t)(q0 + q) * c.d + j] : 0.f;
@@ -48,9 +52,12 @@ search_scan_kernel(TqConsts c, const float *__restrict__ qr, const float *__rest
     const int64_t row = r0 + tid;
     float sc[kSrQ];
     if (row < r_end) {
-      estimate_scores<kSrQ>(c, codes + row * c.code_words,
-                            c.m > 0 ? signs + row * c.sign_words : nullptr, ld_norm(db.norm, row, c.norm16),
-                            c.m > 0 ? ld_norm(db.rnorm, row, c.norm16) : 0.f, qs, ps, cent, sc);
+      const uint32_t *cr = codes + row * c.code_words, *sr = c.m > 0 ? signs + row * c.sign_words : nullptr;
+      const float nu = ld_norm(db.norm, row, c.norm16), ga = c.m > 0 ? ld_norm(db.rnorm, row, c.norm16) : 0.f;
+      if constexpr (POLAR)
+        polar_scores<kSrQ>(c, cr, sr, nu, ga, qs, ps, ptab, sc);
+      else
+        estimate_scores<kSrQ>(c, cr, sr, nu, ga, qs, ps, cent, sc);
     } else {
 #pragma unroll
       for (int q = 0; q < kSrQ; ++q) sc[q] = -INFINITY;
@@ -181,6 +188,7 @@ struct BigTopK {
   }
 };
 
+template <bool POLAR>
 __global__ void __launch_bounds__(kBkThreads)
 search_bigk_scan_kernel(TqConsts c, const float *__restrict__ qr, const float *__restrict__ p, int nq,
                         tq_packed db, int64_t n, int k, int64_t rows_per_shard, int shards,
@@ -192,9 +200,11 @@ search_bigk_scan_kernel(TqConsts c, const float *__restrict__ qr, const float *_
   float *ps = qs + c.d * kBkQ;                       // [m][kBkQ]
   float *cent = ps + c.m * kBkQ;                     // [16]
   float *tile = cent + TQ_MAX_LEVELS;                // [kBkQ][kBkThreads]
+  __shared__ PolarTab ptab;                          // PolarQuant contexts: the angle tables
   const int shard = blockIdx.x;
   const int q0 = blockIdx.y * kBkQ;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (POLAR) polar_tab_stage(ptab, c.polar_tab, tid, kBkThreads);
   for (int i = tid; i < c.d * kBkQ; i += kBkThreads) {
     const int j = i / kBkQ, q = i % kBkQ;
     qs[i] = (q0 + q < nq) ? qr[(int64_t)(q0 + q) * c.d + j] : 0.f;
@@ -217,8 +227,12 @@ search_bigk_scan_kernel(TqConsts c, const float *__restrict__ qr, const float *_
     const int64_t row = r0 + tid;
     float sc[kBkQ];
     if (row < r_end) {
-      estimate_scores<kBkQ>(c, codes + row * c.code_words, c.m > 0 ? signs + row * c.sign_words : nullptr,
-                            ld_norm(db.norm, row, c.norm16), c.m > 0 ? ld_norm(db.rnorm, row, c.norm16) : 0.f, qs, ps, cent, sc);
+      const uint32_t *cr = codes + row * c.code_words, *sr = c.m > 0 ? signs + row * c.sign_words : nullptr;
+      const float nu = ld_norm(db.norm, row, c.norm16), ga = c.m > 0 ? ld_norm(db.rnorm, row, c.norm16) : 0.f;
+      if constexpr (POLAR)
+        polar_scores<kBkQ>(c, cr, sr, nu, ga, qs, ps, ptab, sc);
+      else
+        estimate_scores<kBkQ>(c, cr, sr, nu, ga, qs, ps, cent, sc);
     } else {
 #pragma unroll
       for (int q = 0; q < kBkQ; ++q) sc[q] = -INFINITY;
@@ -297,15 +311,15 @@ cudaError_t launch_search_bigk(const TqConsts &c, int shards, const float *qr, c
   if (nq <= 0) return cudaSuccess;
   const size_t buf = (size_t)kBkQ * kBkCap * (sizeof(float) + sizeof(int64_t));
   const size_t smem = buf + sizeof(float) * ((size_t)(c.d + c.m) * kBkQ + TQ_MAX_LEVELS + kBkQ * kBkThreads);
-  cudaError_t e = tq_smem_limit(reinterpret_cast<const void *>(search_bigk_scan_kernel), (int)smem);
+  auto scan = c.polar ? search_bigk_scan_kernel<true> : search_bigk_scan_kernel<false>;
+  cudaError_t e = tq_smem_limit(reinterpret_cast<const void *>(scan), (int)smem);
   if (e != cudaSuccess) return e;
   e = tq_smem_limit(reinterpret_cast<const void *>(search_bigk_merge_kernel), (int)buf);
   if (e != cudaSuccess) return e;
   const int64_t rows_per_shard = (n + shards - 1) / shards;
   dim3 grid((unsigned)shards, (unsigned)((nq + kBkQ - 1) / kBkQ));
   tq_prof_begin(TQK_SEARCH_SCAN, st);
-  search_bigk_scan_kernel<<<grid, kBkThreads, smem, st>>>(c, qr, p, nq, db, n, k, rows_per_shard, shards, cand_s,
-                                                          cand_i);
+  scan<<<grid, kBkThreads, smem, st>>>(c, qr, p, nq, db, n, k, rows_per_shard, shards, cand_s, cand_i);
   tq_prof_end(TQK_SEARCH_SCAN, st);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -336,12 +350,12 @@ cudaError_t launch_search(const TqConsts &c, const SearchPlan &plan, const float
   if (nq <= 0) return cudaSuccess;
   const int64_t rows_per_shard = (n + plan.shards - 1) / plan.shards;
   const size_t smem = sizeof(float) * ((size_t)(c.d + c.m) * kSrQ + TQ_MAX_LEVELS + kSrQ * kSrThreads);
-  cudaError_t e = tq_smem_limit(reinterpret_cast<const void *>(search_scan_kernel), (int)smem);
+  auto scan = c.polar ? search_scan_kernel<true> : search_scan_kernel<false>;
+  cudaError_t e = tq_smem_limit(reinterpret_cast<const void *>(scan), (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)plan.shards, (unsigned)((nq + kSrQ - 1) / kSrQ));
   tq_prof_begin(TQK_SEARCH_SCAN, st);
-  search_scan_kernel<<<grid, kSrThreads, smem, st>>>(c, qr, p, nq, db, n, k, rows_per_shard, plan.shards,
-                                                     cand_s, cand_i);
+  scan<<<grid, kSrThreads, smem, st>>>(c, qr, p, nq, db, n, k, rows_per_shard, plan.shards, cand_s, cand_i);
   tq_prof_end(TQK_SEARCH_SCAN, st);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -41,6 +41,7 @@ from dataclasses import dataclass
 
 import numpy as np
 
+from . import polar
 from .estimate import prepare_query, scores
 from .rotation import unrotate
 
@@ -66,10 +67,12 @@ def token_slots(b: int, h: int, length: int, n_kv: int, ctx_stride=None, block_t
 def attend_decode(q, kcache: Cache, vcache: Cache, ctx_lens, n_kv: int,
                   k_signs, k_S, k_centroids, v_signs, v_centroids,
                   scale=None, ctx_stride=None, block_table=None, block_tokens: int = 16,
-                  heads=None, sparse_v: float = 0.0):
+                  heads=None, sparse_v: float = 0.0, k_polar=None, v_polar=None):
     """q [B, Hq, d] -> o [B, Hq, d].  `heads` optionally restricts the (b, hq) pairs computed
     (others are left as NaN), for sampled checks at large sizes.  `sparse_v` is the Sparse V
-    threshold tau on the softmax weights (0 = every value row is used)."""
+    threshold tau on the softmax weights (0 = every value row is used).  `k_polar` / `v_polar`:
+    the bits per angle when the keys / values carry PolarQuant angle codes (oracle.polar), whose
+    scores and reconstructions then replace the coordinate codebook's."""
     q = np.asarray(q, dtype=np.float64)
     B, Hq, d = q.shape
     G = Hq // n_kv
@@ -88,12 +91,18 @@ def attend_decode(q, kcache: Cache, vcache: Cache, ctx_lens, n_kv: int,
         qr, p = prepare_query(q[b, hq][None, :], k_signs, k_S)
         rn = kcache.rnorm[sl] if kcache.rnorm is not None else np.zeros(L)
         bt = kcache.bits[sl] if kcache.bits is not None else np.zeros((L, 0))
-        s = scores(qr, p, kcache.norm[sl], kcache.codes[sl], rn, bt, k_centroids)[0]
+        if k_polar:
+            s = polar.scores(qr, p, kcache.norm[sl], kcache.codes[sl], rn, bt, k_polar)[0]
+        else:
+            s = scores(qr, p, kcache.norm[sl], kcache.codes[sl], rn, bt, k_centroids)[0]
         logits = scale * s
         w = np.exp(logits - np.max(logits))
         w /= np.sum(w)
         keep = w >= sparse_v if sparse_v > 0 else np.ones(L, dtype=bool)
-        cv = np.asarray(v_centroids, dtype=np.float64)[vcache.codes[sl][keep]]
-        vhat = vcache.norm[sl][keep][:, None] * unrotate(cv, v_signs)
+        if v_polar:
+            vhat = polar.reconstruct(vcache.norm[sl][keep], vcache.codes[sl][keep], v_signs, v_polar)
+        else:
+            cv = np.asarray(v_centroids, dtype=np.float64)[vcache.codes[sl][keep]]
+            vhat = vcache.norm[sl][keep][:, None] * unrotate(cv, v_signs)
         out[b, hq] = w[keep] @ vhat
     return out

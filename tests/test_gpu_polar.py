@@ -87,9 +87,64 @@ def test_polar_scores_match_oracle(tq, bits, m):
     assert_scores_close(got, ref)
 
 
-def test_polar_rejects_attention_and_search(tq):
-    ctx, D, S = _ctx(tq, 2, 128, 350)
-    packed = tq.Packed.allocate(ctx, 64)
-    with pytest.raises(tq.TqError) as e:
-        tq.search_topk(ctx, torch.randn(3, 128).cuda(), packed, 4)
-    assert e.value.status == 2
+@pytest.mark.parametrize("bits,m,k", [(2, 128, 10), (3, 0, 40)])
+def test_polar_search_topk(tq, bits, m, k):
+    """PolarQuant database through the CUDA-core scans (k <= 32 and the large-k scan), against the
+    oracle's PolarQuant scores of the library's own bytes."""
+    from oracle import search as osearch
+    from parity import assert_topk_equivalent
+    n, d = 3001, 128
+    ctx, D, S = _ctx(tq, bits, m, 360 + bits)
+    X = synth.unit_rows(n, d, seed=11) * 2.0
+    packed = tq.Packed.allocate(ctx, n)
+    tq.encode_kv(ctx, X.cuda(), packed)
+    for nq in (5, 40):
+        Q = synth.unit_rows(nq, d, seed=12 + nq)
+        s, i = tq.search_topk(ctx, Q.cuda(), packed, k)
+        codes = oenc.unpack_codes(packed.codes.cpu().numpy(), d, bits)
+        sb = oenc.unpack_signs(packed.signs.cpu().numpy(), m) if m else np.zeros((n, 0))
+        rn = packed.rnorm.double().cpu().numpy() if m else np.zeros(n)
+        qr, p = oest.prepare_query(Q.double().numpy(), D, S)
+        ref_full = polar.scores(qr, p, packed.norm.double().cpu().numpy(), codes, rn, sb, bits)
+        ref_s, _ = osearch.topk(ref_full, k)
+        assert_topk_equivalent(s.cpu().numpy(), i.cpu().numpy(), lambda r, idx: ref_full[r, idx], ref_s)
+
+
+@pytest.mark.parametrize("kpolar,vpolar", [(True, True), (True, False), (False, True)])
+def test_polar_attention(tq, kpolar, vpolar):
+    """Decode attention with PolarQuant keys and/or values (the general path), paged and ragged,
+    GQA 4, against the oracle evaluated on the library's own bytes."""
+    from oracle import attention as oattn
+    from oracle import codebook as ocb
+    from parity import assert_attention_close
+    d, hkv, group, lens, bits_k, bits_v = 128, 2, 4, [300, 17, 513], 2, 3
+    batch = len(lens)
+    DK, DV = synth.rotation_signs(d, 401), synth.rotation_signs(d, 402)
+    SK = synth.qjl_matrix(128, d, 403)
+    kctx = tq.Context(d, bits_k, 128, DK, SK, polar=kpolar)
+    vctx = tq.Context(d, bits_v, 0, DV, polar=vpolar)
+    lens_t = torch.tensor(lens, dtype=torch.int32)
+    table, nblocks = synth.shuffled_block_table(lens_t, seed=404)
+    cap = nblocks * hkv * synth.BLOCK_TOKENS
+    K = synth.channel_scaled(batch, hkv, max(lens), d, seed=405)
+    V = synth.channel_scaled(batch, hkv, max(lens), d, seed=406)
+    kp, vp = tq.Packed.allocate(kctx, cap), tq.Packed.allocate(vctx, cap)
+    for b in range(batch):
+        for h in range(hkv):
+            sl = torch.as_tensor(oattn.token_slots(b, h, lens[b], hkv, block_table=table.numpy()), dtype=torch.int64)
+            tq.encode_kv(kctx, K[b, h, :lens[b]].cuda(), kp, slots=sl.cuda())
+            tq.encode_kv(vctx, V[b, h, :lens[b]].cuda(), vp, slots=sl.cuda())
+    q = synth.decode_queries(batch, hkv * group, d, seed=407, dtype=torch.bfloat16)
+    out = tq.attend_decode(kctx, vctx, q.cuda(), kp, vp, lens_t.cuda(), max(lens), n_kv_heads=hkv,
+                           block_table=table.cuda(), block_size=synth.BLOCK_TOKENS)
+    torch.cuda.synchronize()
+    kcache = oattn.Cache(norm=kp.norm.double().cpu().numpy(), codes=oenc.unpack_codes(kp.codes.cpu().numpy(), d, bits_k),
+                         rnorm=kp.rnorm.double().cpu().numpy(), bits=oenc.unpack_signs(kp.signs.cpu().numpy(), 128))
+    vcache = oattn.Cache(norm=vp.norm.double().cpu().numpy(), codes=oenc.unpack_codes(vp.codes.cpu().numpy(), d, bits_v))
+    ck, _ = ocb.codebook(d, bits_k)
+    cv, _ = ocb.codebook(d, bits_v)
+    ref = oattn.attend_decode(q.double().numpy(), kcache, vcache, lens, hkv, DK.double().numpy(), SK.double().numpy(), ck,
+                              DV.double().numpy(), cv, block_table=table.numpy(),
+                              k_polar=bits_k if kpolar else None, v_polar=bits_v if vpolar else None)
+    assert_attention_close(out.cpu().numpy(), ref)
+    assert tq.device_status() == 0

@@ -148,3 +148,33 @@ def test_qjl_corrected_score_unbiased_over_projections():
     qr, p = estimate.prepare_query(q[None], D, np.zeros((0, d)))
     xh = polar.reconstruct(enc.norm, enc.codes, D, b)[0]
     assert polar.scores(qr, p, enc.norm, enc.codes, enc.rnorm, enc.bits, b)[0, 0] == pytest.approx(q @ xh, rel=1e-12)
+
+
+def test_polar_attention_is_softmax_over_reconstructed_keys_and_values():
+    """The oracle's decode attention with PolarQuant keys and values (no QJL stage) equals plain
+    softmax attention over the vectors rebuilt from the angle codes, computed here directly."""
+    from oracle import attention
+    d, b, L, hkv, G = 16, 2, 9, 2, 2
+    rng = np.random.default_rng(23)
+    DK = rng.choice([-1.0, 1.0], size=d)
+    DV = rng.choice([-1.0, 1.0], size=d)
+    K = rng.standard_normal((b * hkv * L, d))
+    V = rng.standard_normal((b * hkv * L, d))
+    ek = polar.encode(K, DK, np.zeros((0, d)), b)
+    ev = polar.encode(V, DV, np.zeros((0, d)), b)
+    kc = attention.Cache(norm=ek.norm, codes=ek.codes)
+    vc = attention.Cache(norm=ev.norm, codes=ev.codes)
+    q = rng.standard_normal((b, hkv * G, d))
+    out = attention.attend_decode(q, kc, vc, [L, L - 4], hkv, DK, np.zeros((0, d)), None, DV, None,
+                                  ctx_stride=L, k_polar=b, v_polar=b)
+    Kh = polar.reconstruct(ek.norm, ek.codes, DK, b)
+    Vh = polar.reconstruct(ev.norm, ev.codes, DV, b)
+    for bb in range(b):
+        n = [L, L - 4][bb]
+        for hq in range(hkv * G):
+            h = hq // G
+            rows = (bb * hkv + h) * L + np.arange(n)
+            lg = Kh[rows] @ q[bb, hq] / math.sqrt(d)
+            w = np.exp(lg - lg.max())
+            w /= w.sum()
+            np.testing.assert_allclose(out[bb, hq], w @ Vh[rows], rtol=1e-12, atol=1e-12)
