@@ -78,16 +78,11 @@ __device__ __forceinline__ void mma_u8u8(int (&c)[4], uint32_t a0, uint32_t a1, 
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Uniform value in [0, 1) from a 32-bit key: the fractional part of key * (golden ratio), a
-// low-discrepancy sequence over consecutive keys (deterministic dither for rounding).
-__device__ __forceinline__ float dither(uint32_t x) {
-  // top 23 bits of the product as the mantissa of a float in [1, 2), minus 1 (no conversion unit)
-  return __uint_as_float(0x3F800000u | ((x * 2654435769u) >> 9)) - 1.0f;
-}
+// 1 + u, u uniform in [0, 1), from a 32-bit key: u = the fractional part of key * (golden ratio)
+// to 23 bits (5184445 / 2^23), a low-discrepancy sequence over consecutive keys (deterministic
+// dither for rounding), as the mantissa of a float in [1, 2): one multiply and one logic op.
+__device__ __forceinline__ float dither1(uint32_t x) { return __uint_as_float(0x3F800000u | ((x * 5184445u) & 0x7FFFFFu)); }
 
-// floor(v) for 0 <= v < 2^23, as the low mantissa bits of 2^23 + floor(v): a round-down add on the
-// FMA pipe instead of a float-to-integer conversion.  The result's bytes 0 and 1 are floor(v)'s.
-__device__ __forceinline__ uint32_t floor_bits(float v) { return __float_as_uint(__fadd_rd(v, 8388608.f)); }
 
 // Two fp32 FMAs in one packed instruction (f32x2): d_i = a_i b + c_i, each rounded as fmaf.
 __device__ __forceinline__ void fma2(float a0, float a1, float b, float c0, float c1, float &d0, float &d1) {
@@ -101,7 +96,10 @@ __device__ __forceinline__ void fma2(float a0, float a1, float b, float c0, floa
   d1 = __uint_as_float((uint32_t)(r >> 32));
 }
 
-// floor_bits(fmaf(w_i, c, z_i)) for a pair, in two packed instructions.
+// floor(w_i c + z_i - 1) for a pair, in two packed instructions, as the low mantissa bits of
+// 2^23 + that integer (a round-down add on the FMA pipe instead of a float-to-integer conversion;
+// the result's bytes 0 and 1 are the integer's): z_i = 1 + dither in [1, 2), so the sum plus
+// 2^23 - 1 lies on the integer grid of [2^23, 2^24).
 __device__ __forceinline__ void fma_floor2(float w0, float w1, float c, float z0, float z1, uint32_t &x0,
                                            uint32_t &x1) {
   uint64_t r;
@@ -110,7 +108,7 @@ __device__ __forceinline__ void fma_floor2(float w0, float w1, float c, float z0
       " add.rm.f32x2 %0, pt, pm;\n}"
       : "=l"(r)
       : "r"(__float_as_uint(w0)), "r"(__float_as_uint(w1)), "r"(__float_as_uint(c)), "r"(__float_as_uint(z0)),
-        "r"(__float_as_uint(z1)), "r"(0x4B000000u));
+        "r"(__float_as_uint(z1)), "r"(0x4AFFFFFEu));
   x0 = (uint32_t)r;
   x1 = (uint32_t)(r >> 32);
 }
@@ -842,7 +840,6 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
       for (int P = 0; P < 2 * VT; ++P) C[P] = 2.f * scl * vc.plane_coef[P];
       const uint32_t sel = (uint32_t)l | ((uint32_t)(4 + l) << 4);  // byte l of two words
       const uint32_t key0 = ((uint32_t)grp * (uint32_t)a.max_len + (uint32_t)tk0) * 4u + (uint32_t)gh;
-      uint32_t xs = 0;  // sum of this lane's X values
       uint32_t bfr[2][2 * VT];
       bool live[2];
 #pragma unroll
@@ -854,7 +851,7 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           W[i] = wr[toks[i]];
-          dz[i] = dither(key0 + 4u * (uint32_t)(kb * 16 + toks[i]));
+          dz[i] = dither1(key0 + 4u * (uint32_t)(kb * 16 + toks[i]));
         }
         live[kk] = __any_sync(TQ_FULL_MASK, (W[0] > 0.f) | (W[1] > 0.f) | (W[2] > 0.f) | (W[3] > 0.f));
 #pragma unroll
@@ -866,16 +863,8 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
             fma_floor2(W[i0], W[i1], C[2 * x], dz[i0], dz[i1], x0, x1);
             fma_floor2(W[i0], W[i1], C[2 * x + 1], dz[i0], dz[i1], x2, x3);
             bfr[kk][2 * x + rr] = __byte_perm(__byte_perm(x0, x1, sel), __byte_perm(x2, x3, sel), 0x5410);
-            xs += (x0 + x1) + (x2 + x3) - 4u * 0x4B000000u;  // the integers themselves
           }
       }
-      // the codebook's constant term uses the same integers: sum X per head (limb-0 lanes), then
-      // head t's sum for the accumulator lanes (lane 8 t holds head t)
-      uint32_t mine = l == 0 ? xs : 0u;
-      mine += __shfl_xor_sync(TQ_FULL_MASK, mine, 1);
-      mine += __shfl_xor_sync(TQ_FULL_MASK, mine, 2);
-      mine += __shfl_xor_sync(TQ_FULL_MASK, mine, 4);
-      const float cterm = 64.f * (float)(int)__shfl_sync(TQ_FULL_MASK, mine, 8 * t);
 
       // ---------------------------------------------------------- 3. value sum, all coordinates
       // m-tile mt: row gid <-> coordinate 16 gid + 2 mt, row gid + 8 <-> 16 gid + 2 mt + 1.
@@ -886,6 +875,9 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
       for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
         for (int z = 0; z < 4; ++z) accv[mt][z] = 0;
+      // the codebook's constant term uses the same integers: one more MMA per fragment pair with
+      // every A byte 128 gives 128 sum X of head t in limbs c0 (low), c1 (high) of lane (gid, t)
+      int accc[4] = {0, 0, 0, 0};
       const uint32_t mlo = 1u << (7 - t), mhi = 1u << (3 - t);
 #pragma unroll
       for (int kk = 0; kk < 2; ++kk) {
@@ -893,6 +885,7 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
         if (!live[kk] || vb[kb] < 0) continue;
 #pragma unroll
         for (int x = 0; x < VT; ++x) {
+          mma_u8u8(accc, 0x80808080u, 0x80808080u, 0x80808080u, 0x80808080u, bfr[kk][2 * x], bfr[kk][2 * x + 1]);
           const uint32_t *src = (x == 0) ? svc + kb * SM::VBW + 16 * gid : x1w + kk * kD + 16 * gid;
           uint32_t X[16];
 #pragma unroll
@@ -911,6 +904,7 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
       }
       // accv[mt]: c0/c1 = (coordinate 16 gid + 2 mt, head t, limb 0/1), c2/c3 = (+1, ...):
       // 128 sum_tok X b; with s = 2b - 1 the codebook's constant term is -(1/2) sum X
+      const float cterm = 0.5f * fmaf(256.f, (float)accc[1], (float)accc[0]);  // 64 sum X
       const float ct2 = -cterm * inv;
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt) {
