@@ -461,6 +461,9 @@ __device__ __forceinline__ void tc_x_ready(int g, uint64_t *xfull, int gi) {
 }
 
 // A thread's half row of z (tensor memory, 64 fp32 columns from `zaddr`): sign words 2 h, 2 h + 1.
+// Bit e of a word is set when z >= 0: the words are built from the sign bits, one funnel shift per
+// element (m = (m << 1) | sign, last element first) and one complement at the end.  A negative zero
+// sum counts as negative here; such a z lies far inside any rounding band around 0.
 __device__ __forceinline__ void pack_signs_half(uint32_t zaddr, const TqConsts &c, const TprArgs &a, int64_t slot,
                                                 int h) {
   uint32_t sb[kHW];
@@ -472,11 +475,10 @@ __device__ __forceinline__ void pack_signs_half(uint32_t zaddr, const TqConsts &
     asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
     uint32_t m = 0u;
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      m |= (__uint_as_float(z0[e]) >= 0.f ? 1u : 0u) << e;
-      m |= (__uint_as_float(z1[e]) >= 0.f ? 1u : 0u) << (16 + e);
-    }
-    sb[q] = m;
+    for (int e = 15; e >= 0; --e) m = __funnelshift_l(z1[e], m, 1);
+#pragma unroll
+    for (int e = 15; e >= 0; --e) m = __funnelshift_l(z0[e], m, 1);
+    sb[q] = ~m;
   }
   if (slot >= 0) *reinterpret_cast<uint2 *>(a.signs + slot * c.sign_words + kHW * h) = make_uint2(sb[0], sb[1]);
 }
@@ -776,20 +778,8 @@ encode_tc_kernel(TqConsts c, TprArgs a) {
             rr = fmaf(r, r, rr);
           }
         }
-        group_sync(g);  // both halves have read the norm partials
-        *myx = rr;
-        group_sync(g);
-        const float rr2 = otx[0] + otx[kTRows];
-        if (store) {
-          uint32_t *dst = a.codes + slot * c.code_words + kHW * h;
-#pragma unroll
-          for (int P = 0; P < BITS; ++P) *reinterpret_cast<uint2 *>(dst + 4 * P) = make_uint2(w[P][0], w[P][1]);
-          if (h == 0) {
-            st_norm(a.norm, slot, nu, c.norm16);
-            st_norm(a.rnorm, slot, sqrtf(rr2), c.norm16);
-          }
-        }
-        // r_hi -> tensor memory (the columns y came from), then the first two products may start
+        // r_hi -> tensor memory (the columns y came from): the first two products start while the
+        // residual norms are exchanged and the codes stored
 #pragma unroll
         for (int cb = 0; cb < kHalf / 16; ++cb) {
           uint32_t hv[16];
@@ -804,6 +794,19 @@ encode_tc_kernel(TqConsts c, TprArgs a) {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive1(&b[kBrHi]);
+        group_sync(g);  // both halves have read the norm partials
+        *myx = rr;
+        group_sync(g);
+        const float rr2 = otx[0] + otx[kTRows];
+        if (store) {
+          uint32_t *dst = a.codes + slot * c.code_words + kHW * h;
+#pragma unroll
+          for (int P = 0; P < BITS; ++P) *reinterpret_cast<uint2 *>(dst + 4 * P) = make_uint2(w[P][0], w[P][1]);
+          if (h == 0) {
+            st_norm(a.norm, slot, nu, c.norm16);
+            st_norm(a.rnorm, slot, sqrtf(rr2), c.norm16);
+          }
+        }
         // r_lo into the same columns once those products have read r_hi
         ok = qwait(&b[kBhiDone], (unsigned)(j & 1), abort_flag);
         if (group_any(g, !ok || *abort_flag)) break;
