@@ -99,9 +99,6 @@ __device__ __forceinline__ bool epi_all(bool p) {
   return r != 0;
 }
 
-// 4 bits -> 4 bytes of 0/1 (bit i to byte i)
-__device__ __forceinline__ uint32_t nib_bytes(uint32_t n) { return (n * 0x00204081u) & 0x01010101u; }
-
 // Per query: kq[q] = {2^-Fc, 2^-Fs, (Σ_P e_P) Σ q', Σ p}, F chosen so that |2 e_P q'| 2^Fc and
 // |2 p| 2^Fs stay below 2^22 (three balanced signed byte limbs); zeros past nq.  One warp per query.
 template <int D>
@@ -165,7 +162,9 @@ search_tc_bfrag_kernel(TqConsts c, const float *__restrict__ qr, const float *__
       uint32_t b[3][4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int jj = kTcKC * cc + 16 * g + 4 * i4 + i;
+        // K index 16 g + 4 i4 + i of the stage = 32 kw + 4 t + i with kw = g / 2, t = 4 (g % 2) + i4:
+        // coordinate 32 kw + 8 i + t (the order the expander writes the row bits in)
+        const int jj = kTcKC * cc + 32 * (g >> 1) + 8 * i + 4 * (g & 1) + i4;
         const float x = q < nq ? coef * (sgn ? p[(int64_t)q * D + jj] : qr[(int64_t)q * D + jj]) : 0.f;
         const uint32_t u = (uint32_t)__float2int_rn(x * sc) + 0x80808080u;  // balanced limbs: byte l ^ 0x80
 #pragma unroll
@@ -282,17 +281,16 @@ search_tc_kernel(TqConsts c, const uint8_t *__restrict__ bst, const float *__res
           ok = false;
           break;
         }
-        // the row's 128 coordinates as 0/1 bytes, 4 per tensor-memory column of its lane
+        // the row's 128 coordinates as 0/1 bytes, 4 per tensor-memory column of its lane: column
+        // 8 k + t holds bits t, t + 8, t + 16, t + 24 of word k (one shift and one mask), so K
+        // index 32 k + 4 t + i of the stage is coordinate 32 k + 8 i + t (the query operand is
+        // built in the same order)
         const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
         uint32_t o[32];
 #pragma unroll
-        for (int kg = 0; kg < 8; ++kg) {
-          const uint32_t h = (wd[kg >> 1] >> (16 * (kg & 1))) & 0xFFFFu;
-          o[4 * kg] = nib_bytes(h & 0xFu);
-          o[4 * kg + 1] = nib_bytes((h >> 4) & 0xFu);
-          o[4 * kg + 2] = nib_bytes((h >> 8) & 0xFu);
-          o[4 * kg + 3] = nib_bytes(h >> 12);
-        }
+        for (int kw = 0; kw < 4; ++kw)
+#pragma unroll
+          for (int t = 0; t < 8; ++t) o[8 * kw + t] = (wd[kw] >> t) & 0x01010101u;
         tmem_st32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + tc_acol(slot), o);
         asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
         tc_fence_before();
