@@ -555,18 +555,33 @@ __device__ __forceinline__ void stage_sub(const MmaArgs &a, int sc, const int64_
   }
   if (lane == 0) mbar_expect_arrive(bar, bytes);
   __syncwarp();
+  if (!a.block_table) {
 #pragma unroll
-  for (int arr = p; arr < NA; arr += kProd) {
-    const char *src;
-    size_t doff;
-    unsigned per;
-    int64_t sstride;
-    stage_array<BK, BV, QJL>(a, arr, src, doff, per, sstride);
-    if (!a.block_table) {
+    for (int arr = p; arr < NA; arr += kProd) {
+      const char *src;
+      size_t doff;
+      unsigned per;
+      int64_t sstride;
+      stage_array<BK, BV, QJL>(a, arr, src, doff, per, sstride);
       if (lane == 0 && nvalid > 0) bulk_g2s(sb + doff, src + vb[k0] * sstride, per * nvalid, bar);
-    } else {
-      const int64_t base = lane < SM::NB ? vb[k0 + lane] : -1;
-      if (base >= 0) bulk_g2s(sb + doff + (size_t)lane * per, src + base * sstride, per, bar);
+    }
+  } else {
+    // one copy per valid block; two arrays per round: lanes 0-15 take the blocks of one array,
+    // lanes 16-31 the same blocks of the producer's next array
+    static_assert(SM::NB == 16, "16 blocks per sub-chunk: half a warp per array");
+    const int bl = lane & 15;
+    const int64_t base = vb[k0 + bl];
+#pragma unroll
+    for (int arr0 = p; arr0 < NA; arr0 += 2 * kProd) {
+      const int arr = arr0 + (lane >> 4) * kProd;
+      if (arr < NA && base >= 0) {
+        const char *src;
+        size_t doff;
+        unsigned per;
+        int64_t sstride;
+        stage_array<BK, BV, QJL>(a, arr, src, doff, per, sstride);
+        bulk_g2s(sb + doff + (size_t)bl * per, src + base * sstride, per, bar);
+      }
     }
   }
 }
