@@ -64,7 +64,7 @@ DTYPE_DECODE = ("int8 tensor-core limbs: 32-bit fixed-point query terms x 0/1 ke
 # `dram__bytes_read.sum` + `dram__bytes_write.sum`) of the kernel revision named in the library's
 # version string, on the workload named; null for any other revision or workload
 NCU_TRAFFIC = {
-    ("attend_mma", "r12", "ragged"): 949.94e6 + 13.31e6,
+    ("attend_mma", "r14", "ragged"): 949.94e6 + 13.79e6,
 }
 
 

@@ -104,7 +104,7 @@ extern "C" {
 const char *tq_last_error(void) { return g_err; }
 // The revision tags of the tensor-core kernels name the device code that a recorded profile (DRAM
 // traffic per launch) was taken on; each changes whenever its kernel's code changes.
-const char *tq_version(void) { return "libtq 0.4 (sm_100a; attend_mma r12; search_tc r3; encode_tc r3)"; }
+const char *tq_version(void) { return "libtq 0.4 (sm_100a; attend_mma r14; search_tc r3; encode_tc r3)"; }
 
 tq_status tq_make_codebook(int32_t d, int32_t bits, double *centroids, double *thresholds,
                            double *mse_per_coord) {

@@ -84,6 +84,13 @@ __device__ __forceinline__ void mma_u8u8(int (&c)[4], uint32_t a0, uint32_t a1, 
 __device__ __forceinline__ float dither1(uint32_t x) { return __uint_as_float(0x3F800000u | ((x * 5184445u) & 0x7FFFFFu)); }
 
 
+// A float's order-preserving int (for an integer atomicMax over floats, -inf included) and back.
+__device__ __forceinline__ int ord_float(float f) {
+  const int i = __float_as_int(f);
+  return i >= 0 ? i : i ^ 0x7FFFFFFF;
+}
+__device__ __forceinline__ float unord_float(int i) { return __int_as_float(i >= 0 ? i : i ^ 0x7FFFFFFF); }
+
 // Two fp32 FMAs in one packed instruction (f32x2): d_i = a_i b + c_i, each rounded as fmaf.
 __device__ __forceinline__ void fma2(float a0, float a1, float b, float c0, float c1, float &d0, float &d1) {
   uint64_t r;
@@ -494,7 +501,7 @@ struct MmaSmem {
   static constexpr size_t br = vb + (size_t)MAXBLK * 8;
   // full[NS], empty[NS], the merge barrier, then flags, query constants, merge factors
   static constexpr size_t fl = br + (size_t)(2 * NS + 1) * 8;
-  static constexpr size_t total = fl + 8 * 4 + 16 * 4 + kG * 4;
+  static constexpr size_t total = fl + 8 * 4 + 16 * 4 + kG * 4 + kG * 4;
   static_assert(2 + kProd <= 8, "flag words");
   // the warps' partial states at the end of the range reuse the staging ring
   static_assert((size_t)kCWarps * kG * (kD + 2) * 4 <= NS * buf, "warp partials fit the ring");
@@ -601,9 +608,12 @@ __device__ __forceinline__ void stage_sub(const MmaArgs &a, int sc, const int64_
 // At the end the warps' (m, l, o~) are merged in shared memory into the CTA's partial.
 // Sparse V ("TurboQuant+ 深度解析" 第六部分): with a threshold tau > 0 a token's value row is left
 // out when e^{l - M} < tau max(1, l_old e^{M_old - M}), a bound that is at least its final softmax
-// weight (the running sum only grows and the running maximum's token counts 1), so every row it
-// drops has a final weight below tau; blocks whose rows are all dropped skip their value MMAs.
-template <int BK, int BV, bool QJL, bool NH>
+// weight (the running sum only grows and the running maximum's token counts 1), or when
+// e^{l - Mc} < tau with Mc the CTA's running maximum of the head over every consumer warp's tokens
+// (a lower bound of the final maximum too, shared through one atomic per warp and sub-chunk), so
+// every row it drops has a final weight below tau; blocks whose rows are all dropped skip their
+// value MMAs.
+template <int BK, int BV, bool QJL, bool NH, bool SPV>
 __global__ void __launch_bounds__(kMmaThreads, 2)
 attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restrict__ kfrag,
                   const float *__restrict__ kconst, float *__restrict__ part) {
@@ -620,6 +630,7 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
   volatile int *flags = reinterpret_cast<volatile int *>(smem + SM::fl);  // [0] abort, [1] last, [2] issued
   float *kcs = reinterpret_cast<float *>(smem + SM::fl + 32);        // [16] query constants
   float *hM = kcs + 16;                                              // [kG] merge rescale factors
+  int *cmax = reinterpret_cast<int *>(hM + kG);  // [kG] CTA running logit maximum (ordered int), Sparse V
 
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -664,6 +675,8 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
     vball[i] = base;
   }
   if (tid < 16) kcs[tid] = kconst[grp * 16 + tid];
+  if constexpr (SPV)
+    if (tid < kG) cmax[tid] = ord_float(-INFINITY);
   __syncthreads();
 
   // consumer state: running maximum and sum of head t (same on every gid of a warp) and the value
@@ -810,7 +823,15 @@ attend_mma_kernel(TqConsts kc, TqConsts vc, MmaArgs a, const uint32_t *__restric
       }
       const float Mnew = fmaxf(Mrun, lmax);
       const float al = Mnew == -INFINITY ? 1.f : __expf(Mrun - Mnew);
-      const float gate = tau * fmaxf(1.f, Lw * al);  // Sparse V: drop rows with e^{l - M} < gate
+      float gate = tau * fmaxf(1.f, Lw * al);  // Sparse V: drop rows with e^{l - M} < gate
+      if (SPV && Mnew != -INFINITY) {
+        // the CTA's running maximum of head t (every consumer warp's tokens so far) is also at most
+        // the final maximum, so a row with e^{l - Mc} < tau has a final weight below tau
+        if (gid == 0) atomicMax(&cmax[t], ord_float(Mnew));
+        __syncwarp();
+        const float Mc = unord_float(cmax[t]);
+        gate = fmaxf(gate, tau * __expf(Mc - Mnew));
+      }
       float sw = 0.f;
 #pragma unroll
       for (int kb = 0; kb < 2; ++kb)
@@ -1130,8 +1151,12 @@ template <int BK, int BV, bool QJL>
 cudaError_t launch_mma(const TqConsts &kc, const TqConsts &vc, const MmaArgs &a, dim3 grid,
                        const uint32_t *kfrag, const float *kconst, float *part, cudaStream_t st) {
   const size_t smem = MmaSmem<BK, BV, QJL>::total;
-  // norms in fp16 (both roles; mixed storage takes the general path) or fp32
-  auto kern = a.kn4 == 1 ? attend_mma_kernel<BK, BV, QJL, true> : attend_mma_kernel<BK, BV, QJL, false>;
+  // norms in fp16 (both roles; mixed storage takes the general path) or fp32; the Sparse V gate
+  // over the CTA's running maximum only in the variant launched with a threshold
+  auto kern = a.sparse_v > 0.f ? (a.kn4 == 1 ? attend_mma_kernel<BK, BV, QJL, true, true>
+                                             : attend_mma_kernel<BK, BV, QJL, false, true>)
+                               : (a.kn4 == 1 ? attend_mma_kernel<BK, BV, QJL, true, false>
+                                             : attend_mma_kernel<BK, BV, QJL, false, false>);
   cudaError_t e = tq_smem_limit(reinterpret_cast<const void *>(kern), (int)smem);
   if (e != cudaSuccess) return e;
   // programmatic dependent launch: the grid may start while the preceding kernel on the stream
